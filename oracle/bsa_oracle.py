@@ -1,0 +1,498 @@
+"""Plain fp64 CPU oracle for query-dependent block-sparse causal attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module: only the tests, the
+smoke check in ``__graft_entry__`` and the ``cpu_baseline`` / ``--impl reference`` legs of the
+benchmark may call it.  It shares no code with the CUDA library.  It is deliberately slow: every
+function is the plain definition, one query (or one block) at a time, in float64, with NumPy only
+for array storage, matrix-vector products and sums.
+
+Sources (cited by page title and the section / equation on it):
+
+* [SAS] the review page "SAS: Simple Attention Sparsification via End-to-End Optimization of
+  Context Ranking" -- sections "Background: the problem they solved" (Eq. 1-3), "The new
+  approach: SAS" (Eq. 4, Eq. 9), "Why the four design choices matter" (Eq. 5 and the softmax gate
+  log g = s - LSE(s)), "How it works: a worked example" (steps 1-6), "Decoding efficiency"
+  (Fig. 7).
+* [FreeSolo] the summary page "FreeSolo가 학습 길이의 64배까지 제로샷 검색을 유지한다" --
+  section "How it works" (cells, the three summaries, the query-block prefix, the erf-biased cell
+  score, top-K cells, the RoPE sliding-window branch, the NoPE long branch, the per-head mix).
+* [Monodratic] the article "Monodratic、学習ルーティングによりスパース因果アテンションの選択性を高め
+  られると主張" -- section on turning sparse attention into a retrieval decision (guaranteed local
+  block, exact causal softmax over the selected tokens, no future block reachable, sparse-vs-dense
+  mask parity).
+
+Readings where the pages are silent or garbled (each listed with its reason in the design doc):
+
+* R1 gate normaliser: log g_m = s_m - LSE over either the selected history blocks
+  ("selected") or every history block ("all"); the worked example of [SAS] uses all blocks.
+* R2 GQA: query head h reads kv head h // (Hq // Hk); selection is per query head.
+* R3 current block of the query at position i is cur = i // b; history blocks are 0 .. cur-1.
+* R4 fewer candidates than K: all candidates are taken.  FreeSolo queries with no candidate cell
+  use the short branch alone.
+* R5 top-K order: larger score first, lower block index first among equal scores, NaN below
+  everything; the result is reported in ascending block order.
+* R6 logits and dot-product scores use the scale 1/sqrt(d).
+* R7 block centre = mean position of the tokens in the block (c*b + (b-1)/2 for a full block).
+* R8 FreeSolo mix o = (1 - alpha_h) * o_short + alpha_h * o_long; RoPE with base 10000,
+  rotate-half pairing, absolute positions; the window holds the ``window`` most recent keys,
+  the query's own key included.
+* R9 erf argument (i - p_c) / (2 sigma_h), as printed, positive for past cells.
+* R10 dg is the derivative with respect to g_m (not log g_m), one value per (query unit, selected
+  history block); with per-query-block selection it sums over the unit's queries.
+* R11 a computed selector score is rounded to float32 before top-K, the precision in which the
+  CUDA kernels take the same decision; supplied scores are float32 already.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+NEG_INF = -math.inf
+
+# ----------------------------------------------------------------------------------------------
+# Block partition and summaries
+# ----------------------------------------------------------------------------------------------
+
+
+def block_range(c: int, n: int, b: int) -> tuple[int, int]:
+    """Token range [lo, hi) of block c when n positions are cut into blocks of b tokens.
+
+    [SAS] "Background", Eq. 3: the n context positions form C = n / b blocks B_1..B_C of b tokens.
+    A final block shorter than b (n not a multiple of b) keeps the remaining tokens.
+    """
+    return c * b, min(n, (c + 1) * b)
+
+
+def num_blocks(n: int, b: int) -> int:
+    return (n + b - 1) // b
+
+
+def block_summaries(k: np.ndarray, b: int):
+    """Per-block key summaries of one (batch, kv head): mean key, max key norm, centre.
+
+    [FreeSolo] "How it works": each cell keeps its mean key (content used for routing), its
+    centre position (for the relative distance) and the largest key norm inside it (a
+    query-independent priority).  [SAS] "Limitations" names its summary a pooled block summary.
+    Returns mean_k [C, d], max_norm [C], centre [C] in float64.
+    """
+    k = np.asarray(k, dtype=np.float64)
+    n, d = k.shape
+    C = num_blocks(n, b)
+    mean_k = np.zeros((C, d))
+    max_norm = np.zeros(C)
+    centre = np.zeros(C)
+    for c in range(C):
+        lo, hi = block_range(c, n, b)
+        blk = k[lo:hi]
+        mean_k[c] = blk.sum(axis=0) / (hi - lo)
+        max_norm[c] = max(math.sqrt(float(np.dot(row, row))) for row in blk)
+        centre[c] = sum(range(lo, hi)) / (hi - lo)  # R7: mean token position
+    return mean_k, max_norm, centre
+
+
+# ----------------------------------------------------------------------------------------------
+# Block scoring
+# ----------------------------------------------------------------------------------------------
+
+
+def dot_scores(q: np.ndarray, mean_k: np.ndarray, n_cand: int) -> np.ndarray:
+    """s_c = q . kbar_c / sqrt(d) for the n_cand candidate blocks (c < n_cand).
+
+    First term of the cell score r_ic of [FreeSolo] "How it works"; the plain query-summary score
+    a learned selector is replaced by when no selector weights exist.  R6.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    return np.array([float(np.dot(q, mean_k[c])) / math.sqrt(d) for c in range(n_cand)])
+
+
+def freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, n_cand) -> np.ndarray:
+    """r_ic = q_i . kbar_c / sqrt(d) + lambda_h * a_c * erf((i - p_c) / (2 sigma_h)).
+
+    [FreeSolo] "How it works", the cell score.  ``erf`` is the library error function.  R9.
+    """
+    base = dot_scores(q, mean_k, n_cand)
+    bias = np.array([lam * max_norm[c] * float(_erf((i - centre[c]) / (2.0 * sigma)))
+                     for c in range(n_cand)])
+    return base + bias
+
+
+def sas_num_candidates(i: int, b: int) -> int:
+    """History blocks available to the query at position i: blocks 0 .. cur-1, cur = i // b.
+
+    [SAS] "The new approach", Eq. 4: the selector scores only history blocks; the current block
+    B_0 is always kept outside the selection.  R3.
+    """
+    return i // b
+
+
+def freesolo_num_candidates(i: int, cell: int, q_block: int) -> int:
+    """Cells whose tokens all lie before the start of the query's block of q_block queries.
+
+    [FreeSolo] "How it works": the prefix is fixed per query block (B = 128), so every query of
+    one block sees the same candidate cells: those ending at or before floor(i / B) * B.
+    """
+    prefix = (i // q_block) * q_block
+    return prefix // cell
+
+
+# ----------------------------------------------------------------------------------------------
+# Top-K selection
+# ----------------------------------------------------------------------------------------------
+
+
+def _rank_key(value: float, idx: int):
+    """Sort key: NaN last, then larger score first, then lower index first (R5)."""
+    if math.isnan(value):
+        return (1, 0.0, idx)
+    return (0, -value, idx)
+
+
+def topk_blocks(s, n_cand: int, K: int) -> list[int]:
+    """Indices of the K highest-scoring candidate blocks c < n_cand, in ascending order.
+
+    [SAS] "Background", Eq. 3 (I = Top-K(s, K)) and "How it works" step 3; fewer than K candidates
+    are all taken (R4).  A full stable sort over the candidates decides the set.
+    """
+    order = sorted(range(n_cand), key=lambda c: _rank_key(float(s[c]), c))
+    return sorted(order[:min(K, n_cand)])
+
+
+def round_f32(x):
+    """R11: the precision in which a computed score decides the selection."""
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------------------------
+# Softmax log-gate
+# ----------------------------------------------------------------------------------------------
+
+
+def logsumexp(x) -> float:
+    x = np.asarray(x, dtype=np.float64)
+    if x.size == 0:
+        return NEG_INF
+    m = float(np.max(x))
+    if m == NEG_INF:
+        return NEG_INF
+    return m + math.log(float(np.sum(np.exp(x - m))))
+
+
+def log_gates(s, n_cand: int, selected, norm: str) -> dict[int, float]:
+    """log g_m = s_m - LSE(s) for each selected history block m.
+
+    [SAS] "Why the four design choices matter": the softmax gate gives log g_m = s_m - LSE(s);
+    "The new approach", Eq. 4: the current block keeps g_0 = 1.  ``norm`` picks the set the LSE
+    runs over (R1): "all" = every history block c < n_cand, "selected" = the selected ones.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    if norm == "all":
+        L = logsumexp(s[:n_cand])
+    elif norm == "selected":
+        L = logsumexp(s[list(selected)]) if len(selected) else 0.0
+    else:
+        raise ValueError(norm)
+    return {int(m): float(s[m]) - L for m in selected}
+
+
+# ----------------------------------------------------------------------------------------------
+# Exact softmax over the gathered tokens
+# ----------------------------------------------------------------------------------------------
+
+
+def token_set(i: int, b: int, selected, n: int, keep_current: bool = True):
+    """Tokens a query at position i attends: every token of the selected history blocks and the
+    tokens j <= i of its current block.
+
+    [SAS] "Background", Eq. 2 (attention restricted to the selected set S) and "How it works"
+    step 3 (S = B_0 united with the selected blocks); [Monodratic] (guaranteed local block plus the
+    selected remote blocks, causal mask applied inside the selected set).  Returns (tokens,
+    owning block of each token).
+    """
+    toks, owner = [], []
+    for m in sorted(selected):
+        lo, hi = block_range(m, n, b)
+        for j in range(lo, hi):
+            if j <= i:  # history blocks lie wholly before i; kept for safety of the definition
+                toks.append(j)
+                owner.append(m)
+    if keep_current:
+        cur = i // b
+        lo, _ = block_range(cur, n, b)
+        for j in range(lo, i + 1):
+            toks.append(j)
+            owner.append(-1)  # -1 marks the current block
+    return np.array(toks, dtype=np.int64), np.array(owner, dtype=np.int64)
+
+
+def attend(q, k, v, toks, bias):
+    """Exact softmax attention of one query over the listed tokens.
+
+    z_j = q . k_j / sqrt(d) + bias_j; p = softmax(z); o = sum_j p_j v_j; lse = log sum_j exp z_j.
+    [SAS] "Background", Eq. 1-2 (standard attention restricted to S), R6.  Returns o, lse, p.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    kk = np.asarray(k[toks], dtype=np.float64)
+    vv = np.asarray(v[toks], dtype=np.float64)
+    z = kk @ q / math.sqrt(d) + bias
+    m = float(np.max(z))
+    e = np.exp(z - m)
+    l = float(np.sum(e))
+    p = e / l
+    o = p @ vv
+    return o, m + math.log(l), p
+
+
+def sparse_attention_row(q, k, v, i, b, selected, gate=None, keep_current=True):
+    """Output and log-sum-exp of one query at position i over its gathered token set.
+
+    Without a gate this is the inference path of [SAS] "How it works" step 6 (plain Top-K, exact
+    softmax over the kept blocks).  With ``gate`` (a dict m -> log g_m) it is the training-mode
+    forward of [SAS] "The new approach", Eq. 9: log g_m is added to the logits of every token of
+    selected history block m, the current block gets log 1 = 0.
+    """
+    n = k.shape[0]
+    toks, owner = token_set(i, b, selected, n, keep_current)
+    bias = np.zeros(len(toks))
+    if gate is not None:
+        for t, m in enumerate(owner):
+            if m >= 0:
+                bias[t] = gate[int(m)]
+    o, lse, _ = attend(q, k, v, toks, bias)
+    return o, lse
+
+
+def masked_attention_row(q, k, v, i, b, selected, gate=None, keep_current=True):
+    """The same quantity written as dense attention over all n keys with a -inf mask.
+
+    Independent restatement used to pin the gather path: [Monodratic] compares its sparse
+    selected-set attention against an independently built dense mask oracle.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    n, d = k.shape
+    z = np.asarray(k, dtype=np.float64) @ q / math.sqrt(d)
+    allowed = np.zeros(n, dtype=bool)
+    bias = np.zeros(n)
+    for m in selected:
+        lo, hi = block_range(m, n, b)
+        allowed[lo:hi] = True
+        if gate is not None:
+            bias[lo:hi] = gate[int(m)]
+    if keep_current:
+        lo, _ = block_range(i // b, n, b)
+        allowed[lo:i + 1] = True
+    allowed[i + 1:] = False
+    z = np.where(allowed, z + bias, NEG_INF)
+    w = np.exp(z - z.max())
+    w /= w.sum()
+    return w @ np.asarray(v, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------------------------
+# Closed-form gate gradient
+# ----------------------------------------------------------------------------------------------
+
+
+def gate_grad_rows(qs, k, v, positions, b, selected, gate, douts):
+    """dg_m for each selected history block m, summed over the given queries.
+
+    [SAS] "Why the four design choices matter", Eq. 5 (inner gate):
+        dg_m = sum_{i in B_m} (ptilde_i / g_m) * do^T (v_i - o),
+    where ptilde is the gated softmax of the query over its token set and o its output.  The
+    queries of one unit share one gate vector, so their contributions add (R10).
+    Returns dict m -> dg_m.
+    """
+    n = k.shape[0]
+    dg = {int(m): 0.0 for m in selected}
+    for q, i, do in zip(qs, positions, douts):
+        toks, owner = token_set(int(i), b, selected, n)
+        bias = np.array([gate[int(m)] if m >= 0 else 0.0 for m in owner])
+        o, _, p = attend(q, k, v, toks, bias)
+        do = np.asarray(do, dtype=np.float64)
+        for t, m in enumerate(owner):
+            if m < 0:
+                continue
+            g_m = math.exp(gate[int(m)])
+            vi = np.asarray(v[toks[t]], dtype=np.float64)
+            dg[int(m)] += p[t] / g_m * float(np.dot(do, vi - o))
+    return dg
+
+
+def gated_loss(qs, k, v, positions, b, selected, g, douts) -> float:
+    """L = sum_i do_i . o_i(g) for gates g (dict m -> g_m > 0); used for finite differences."""
+    gate = {m: math.log(gm) for m, gm in g.items()}
+    total = 0.0
+    for q, i, do in zip(qs, positions, douts):
+        o, _ = sparse_attention_row(q, k, v, int(i), b, selected, gate)
+        total += float(np.dot(np.asarray(do, dtype=np.float64), o))
+    return total
+
+
+# ----------------------------------------------------------------------------------------------
+# Whole-call drivers (decode and prefill), written on top of the row functions
+# ----------------------------------------------------------------------------------------------
+
+
+def decode_reference(q, k, v, seq_lens, b, K, scores=None, gate_norm=None, rows=None,
+                     summaries=None):
+    """One decode step for every (batch, query head) row, or for the listed ``rows``.
+
+    Chain of [SAS] "How it works" step 6 / the inference algorithm: score the history blocks of
+    the query at position seq_len-1 (supplied ``scores`` [B, Hq, C], else q . kbar / sqrt(d)),
+    take Top-K, keep the current block, exact softmax over the gathered tokens.  ``gate_norm``
+    ("selected" / "all") adds the training-mode log-gate of the supplied or computed scores.
+    Returns dict (bi, h) -> {"idx", "scores", "o", "lse"}.
+    """
+    B, Hq, d = q.shape
+    Hk = k.shape[1]
+    G = Hq // Hk
+    out = {}
+    if rows is None:
+        rows = [(bi, h) for bi in range(B) for h in range(Hq)]
+    cache = {} if summaries is None else summaries
+    for bi, h in rows:
+        kh = h // G
+        L = int(seq_lens[bi])
+        i = L - 1
+        kk = k[bi, kh, :L]
+        vv = v[bi, kh, :L]
+        nc = sas_num_candidates(i, b)
+        if scores is not None:
+            s = np.asarray(scores[bi, h, :nc], dtype=np.float64)
+        else:
+            if (bi, kh) not in cache:
+                cache[(bi, kh)] = block_summaries(kk, b)
+            mean_k = cache[(bi, kh)][0]
+            s = round_f32(dot_scores(q[bi, h], mean_k, nc))
+        sel = topk_blocks(s, nc, K)
+        gate = log_gates(s, nc, sel, gate_norm) if gate_norm else None
+        o, lse = sparse_attention_row(q[bi, h], kk, vv, i, b, sel, gate)
+        out[(bi, h)] = {"idx": sel, "scores": s, "o": o, "lse": lse}
+    return out
+
+
+def prefill_unit_reference(q, k, v, scores, b, q_block, K, bi, h, u, gate_norm=None,
+                           dout=None):
+    """Prefill of one query unit (query block u of head h): selection shared by the unit.
+
+    The unit's candidates are the history blocks of its first query (c < (u*q_block) // b), its
+    selection is Top-K of the supplied scores ``scores[bi, h, u]``; each query i of the unit keeps
+    its own current block i // b with the causal mask j <= i ([SAS] "The new approach", Eq. 9 and
+    the training forward it describes).  With ``gate_norm`` the log-gate is added; with ``dout``
+    the gate gradient dg of Eq. 5 is returned too.
+    """
+    Hk = k.shape[1]
+    Hq = q.shape[1]
+    G = Hq // Hk
+    kh = h // G
+    n = k.shape[2]
+    lo = u * q_block
+    hi = min(n, lo + q_block)
+    nc = sas_num_candidates(lo, b)
+    s = np.asarray(scores[bi, h, u, :nc], dtype=np.float64)
+    sel = topk_blocks(s, nc, K)
+    gate = log_gates(s, nc, sel, gate_norm) if gate_norm else None
+    kk, vv = k[bi, kh], v[bi, kh]
+    o = np.zeros((hi - lo, q.shape[3]))
+    lse = np.zeros(hi - lo)
+    for t, i in enumerate(range(lo, hi)):
+        o[t], lse[t] = sparse_attention_row(q[bi, h, i], kk, vv, i, b, sel, gate)
+    res = {"idx": sel, "o": o, "lse": lse}
+    if dout is not None and gate is not None:
+        dg = gate_grad_rows(q[bi, h, lo:hi], kk, vv, range(lo, hi), b, sel, gate,
+                            dout[bi, h, lo:hi])
+        res["dg"] = np.array([dg[m] for m in sel])
+    return res
+
+
+# ----------------------------------------------------------------------------------------------
+# FreeSolo two-branch prefill
+# ----------------------------------------------------------------------------------------------
+
+
+def rope(x, pos: int, theta: float = 10000.0):
+    """Rotary position embedding of one vector at absolute position ``pos`` (R8).
+
+    Rotate-half pairing: dimension t (t < d/2) pairs with t + d/2 and both rotate by the angle
+    pos * theta^(-2t/d).  [FreeSolo] "How it works" applies RoPE inside the local window only.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[0] // 2
+    ang = pos * theta ** (-2.0 * np.arange(half) / x.shape[0])
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[:half], x[half:]
+    return np.concatenate([a * c - b * s, b * c + a * s])
+
+
+def freesolo_row(q, k, v, i, summaries, cell, q_block, K, window, lam, sigma, alpha, theta):
+    """Two-branch output of the query at position i of one head ([FreeSolo] "How it works").
+
+    Short branch: softmax attention of RoPE(q_i) over RoPE(k_j), j in [i-window+1, i].
+    Long branch: candidate cells fixed by the query block, cell score r_ic, Top-K cells, one
+    softmax over the raw (unrotated) tokens of those cells.  Mix (R8):
+    o = (1 - alpha) o_short + alpha o_long; o = o_short when no cell is a candidate (R4).
+    Returns o, and the selected cells.
+    """
+    d = q.shape[0]
+    mean_k, max_norm, centre = summaries
+    lo = max(0, i - window + 1)
+    qr = rope(q, i, theta)
+    kr = np.array([rope(k[j], j, theta) for j in range(lo, i + 1)])
+    z = kr @ qr / math.sqrt(d)
+    w = np.exp(z - z.max())
+    w /= w.sum()
+    o_short = w @ np.asarray(v[lo:i + 1], dtype=np.float64)
+    nc = freesolo_num_candidates(i, cell, q_block)
+    if nc == 0:
+        return o_short, []
+    r = round_f32(freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, nc))
+    sel = topk_blocks(r, nc, K)
+    toks = np.concatenate([np.arange(*block_range(c, k.shape[0], cell)) for c in sel])
+    o_long, _, _ = attend(q, k, v, toks, np.zeros(len(toks)))
+    return (1.0 - alpha) * o_short + alpha * o_long, sel
+
+
+# ----------------------------------------------------------------------------------------------
+# Helpers the tests use to judge near-tie selections
+# ----------------------------------------------------------------------------------------------
+
+
+def selection_gap(s, n_cand: int, K: int):
+    """(s_(K), s_(K+1)) of the descending order of the candidates, or None if n_cand <= K."""
+    if n_cand <= K:
+        return None
+    order = sorted(range(n_cand), key=lambda c: _rank_key(float(s[c]), c))
+    return float(s[order[K - 1]]), float(s[order[K]])
+
+
+def valid_selections(s, n_cand: int, K: int, rel: float = 1e-4, limit: int = 64):
+    """Every block set a selector may return for scores ``s`` (tie tolerance ``rel``).
+
+    When the K-th and (K+1)-th largest scores differ by more than ``rel`` relative, only the exact
+    Top-K set is valid.  Otherwise, with tau = rel * max(|s_(K)|, |s_(K+1)|), a valid set holds
+    every block scoring above s_(K) + tau, K blocks in all, the rest drawn from the blocks within
+    tau of s_(K).  Returns a list of ascending index lists, or None if there are more than
+    ``limit`` of them.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    exact = topk_blocks(s, n_cand, K)
+    gap = selection_gap(s, n_cand, K)
+    if gap is None:
+        return [exact]
+    hi_s, lo_s = gap
+    if math.isnan(hi_s) or math.isnan(lo_s):
+        return [exact]
+    tau = rel * max(abs(hi_s), abs(lo_s))
+    if hi_s - lo_s > tau:
+        return [exact]
+    sure = [c for c in range(n_cand) if s[c] > hi_s + tau]
+    maybe = [c for c in range(n_cand) if hi_s - tau <= s[c] <= hi_s + tau]
+    need = K - len(sure)
+    combos = list(itertools.islice(itertools.combinations(maybe, need), limit + 1))
+    if len(combos) > limit:
+        return None
+    return [sorted(sure + list(cb)) for cb in combos]
