@@ -1,0 +1,401 @@
+"""Benchmark of the block-sparse decode step on B200 (one JSON line on stdout).
+
+Workload (default): SAS-style GQA decode, bf16 -- batch 8, 32 query / 8 kv heads, d = 128,
+context 32,768, blocks of 64, top-15 history blocks + the current block, keys with 16 planted
+needle blocks per (batch, kv head).  One step = one pass of the decode hot path over the batch:
+refresh the summary of the current block, score every history block, Top-K, sparse attention
+(4 kernel launches, replayed as CUDA graphs).  L2 (126 MB) is flushed between steps by writing a
+256 MiB buffer outside the timed events; every step is timed with CUDA events on the launching
+stream and the step times are summed.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload instead (a bounded sample of
+batch rows per step) and prints the same JSON line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode tokens/s and HBM GB/s (% roofline); prefill TFLOP/s (% peak)"
+
+WORKLOADS = {
+    "sas_gqa_decode_32k": dict(B=8, Hq=32, Hk=8, d=128, n=32768, b=64, K=15, needles=16,
+                               needle_layout="random", seed=2000),
+    "long_decode_512k": dict(B=1, Hq=32, Hk=8, d=128, n=524288, b=64, K=31, needles=64,
+                             needle_layout="stride", seed=3000),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int = 0, period_ms: int = 50):
+        self.samples = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.period = period_ms
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.samples:
+            if self.t0 is not None and not (self.t0 - 0.05 <= ts <= (self.t1 or ts) + 0.05):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append(parts)
+        if not rows:  # timed window shorter than the sampling period: use the whole run
+            rows = [[p.strip() for p in line.split(",")] for _, line in self.samples]
+            rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def oracle_decode_sample(case, rows_b, summaries):
+    """Time the oracle's decode of the listed batch rows (all heads) on one host thread;
+    returns seconds."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import bsa_oracle as orc
+    rows = [(bi, h) for bi in rows_b for h in range(case.Hq)]
+    with threadpool_limits(limits=1):
+        t = time.perf_counter()
+        orc.decode_reference(case.q, case.k, case.v, case.seq_lens, case.b, case.K, rows=rows,
+                             summaries=summaries)
+        return time.perf_counter() - t
+
+
+def oracle_summaries(case, rows_b):
+    from oracle import bsa_oracle as orc
+    G = case.Hq // case.Hk
+    out = {}
+    for bi in rows_b:
+        for kh in range(case.Hk):
+            out[(bi, kh)] = orc.block_summaries(case.k[bi, kh, :case.seq_lens[bi]], case.b)
+    del G
+    return out
+
+
+def make_case(wl):
+    from block_sparse_attention_summaries_b200 import inputs
+    w = WORKLOADS[wl]
+    return inputs.decode_case(w["seed"], B=w["B"], Hq=w["Hq"], Hk=w["Hk"], d=w["d"], n=w["n"],
+                              b=w["b"], K=w["K"], needles=w["needles"],
+                              needle_layout=w["needle_layout"])
+
+
+def run_reference(args):
+    """fp64 CPU oracle timed on the host: each step decodes one batch row (all heads)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    case = make_case(args.workload)
+    nb = case.B
+    summ = oracle_summaries(case, range(nb))
+    for i in range(args.warmup):
+        oracle_decode_sample(case, [i % nb], summ)
+    total = 0.0
+    for i in range(args.steps):
+        total += oracle_decode_sample(case, [i % nb], summ)
+    ms = total / args.steps * 1e3
+    value = args.steps / total  # one token (all heads of one sequence) per step
+    w = WORKLOADS[args.workload]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), bf16-rounded, planted needle blocks)",
+        "config": {"workload": args.workload, **{k: w[k] for k in ("B", "Hq", "Hk", "d", "n",
+                                                                   "b", "K")}},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "one batch row (all 32 query heads) per step, summaries "
+                                   "precomputed as on the GPU"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_summaries_b200 as bsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    bsa.lib()
+
+    w = WORKLOADS[args.workload]
+    case = make_case(args.workload)
+    B, Hq, Hk, d, n, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K"))
+    G = Hq // Hk
+    C = (n + b - 1) // b
+
+    q = torch.from_numpy(case.q).to(dev, torch.bfloat16)
+    k = torch.from_numpy(case.k).to(dev, torch.bfloat16)
+    v = torch.from_numpy(case.v).to(dev, torch.bfloat16)
+    # prefill-time state: summaries of every block (not part of the decode step)
+    mean_k, max_norm, centre = bsa.build_block_summaries(k, b)
+    scores = torch.empty(B, Hq, C, device=dev, dtype=torch.float32)
+    n_cand = torch.empty(B * Hq, device=dev, dtype=torch.int32)
+    idx = torch.empty(B, Hq, K, device=dev, dtype=torch.int32)
+    count = torch.empty(B, Hq, device=dev, dtype=torch.int32)
+    o = torch.empty(B, Hq, d, device=dev, dtype=torch.bfloat16)
+    lse = torch.empty(B, Hq, device=dev, dtype=torch.float32)
+    ws = torch.zeros(bsa.sparse_attn_workspace_bytes(B, Hq, Hk, 1, n, d, b, K), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def stage_select():
+        bsa.build_block_summaries(k, b, None, -1, 1, mean_k, max_norm, centre)
+        bsa.score_blocks(q, mean_k, n, b, scores=scores, n_cand=n_cand)
+
+    def stage_topk():
+        bsa.topk_blocks(scores, K, n_cand=n_cand, idx=idx, count=count)
+
+    def stage_attn():
+        bsa.sparse_attn_fwd(q, k, v, idx, b, count=count, o=o, lse=lse, ws=ws)
+
+    stream = torch.cuda.Stream(dev)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for fn in (stage_select, stage_topk, stage_attn):  # eager run before capture
+            fn()
+        torch.cuda.synchronize(dev)
+        for fn in (stage_select, stage_topk, stage_attn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+    torch.cuda.synchronize(dev)
+    launches_per_step = 4  # append + score, top-K, attention
+
+    # algorithmic bytes of the attention launch: union of the selected blocks per kv group
+    idx_h = idx.cpu().numpy()
+    union_blocks = 0
+    per_head_blocks = 0
+    cur = (n - 1) // b
+    for bi in range(B):
+        for kh in range(Hk):
+            sel = set(int(x) for x in idx_h[bi, kh * G:(kh + 1) * G].ravel() if x >= 0)
+            union_blocks += len(sel) + 1  # + current block
+            per_head_blocks += int((idx_h[bi, kh * G:(kh + 1) * G] >= 0).sum()) + G
+    cur_tokens = n - cur * b
+    kv_bytes = (union_blocks - B * Hk) * b * d * 2 * 2 + B * Hk * cur_tokens * d * 2 * 2
+    attn_bytes = kv_bytes + B * Hq * d * 2 * 2 + B * Hq * (K * 4 + 4 + 4)  # + q, o, idx, lse
+    score_bytes = B * Hk * cur * (d * 4) + B * Hq * d * 2 + B * Hq * C * 4
+    step_bytes = kv_bytes + B * Hk * cur * (d * 4)  # selected KV + summaries (spec count)
+
+    # needle recall of the selection
+    hits = tot = 0
+    for (bi, kh), blocks in case.needles.items():
+        sel = set(int(x) for x in idx_h[bi, kh * G:(kh + 1) * G].ravel() if x >= 0)
+        hits += len(sel & set(int(c) for c in blocks))
+        tot += len(blocks)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+
+    def one_step(evs):
+        flush.zero_()  # evict L2 before every step (outside the events)
+        evs[0].record(stream)
+        graphs[0].replay()
+        evs[1].record(stream)
+        graphs[1].replay()
+        evs[2].record(stream)
+        graphs[2].replay()
+        evs[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        sampler.mark("t0")
+        events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                  for _ in range(args.steps)]
+        for i in range(args.steps):
+            one_step(events[i])
+        torch.cuda.synchronize(dev)
+        sampler.mark("t1")
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+    sel_ms = [e[0].elapsed_time(e[1]) for e in events]
+    topk_ms = [e[1].elapsed_time(e[2]) for e in events]
+    attn_ms = [e[2].elapsed_time(e[3]) for e in events]
+    step_ms = [e[0].elapsed_time(e[3]) for e in events]
+    total_ms = sum(step_ms)
+
+    # end to end through the public API: pinned host q in, o out, every step
+    q_host = torch.from_numpy(case.q).to(torch.bfloat16).pin_memory()
+    o_host = torch.empty(B, Hq, d, dtype=torch.bfloat16).pin_memory()
+    e2e_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.copy_(q_host, non_blocking=True)
+            for g in graphs:
+                g.replay()
+            o_host.copy_(o, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= args.warmup:
+                e2e_ms.append(e0.elapsed_time(e1))
+    sampler.stop()
+    clocks = sampler.summary()
+
+    mx_total = total_ms
+    if world > 1:
+        t = torch.tensor([total_ms, sum(e2e_ms)], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mx_total, e2e_total = float(t[0]), float(t[1])
+    else:
+        e2e_total = sum(e2e_ms)
+    ms_per_step = mx_total / args.steps
+    tokens = B * world * args.steps
+    value = tokens / (mx_total / 1e3)
+    e2e_value = tokens / (e2e_total / 1e3)
+
+    peaks = load_peaks()
+    attn_avg = statistics.fmean(attn_ms)
+    achieved = attn_bytes / (attn_avg / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), bf16-rounded, 16 planted needle blocks per kv head)",
+        "config": {"workload": args.workload, **{x: w[x] for x in ("B", "Hq", "Hk", "d", "n", "b",
+                                                                   "K")},
+                   "parallelism": f"replicas{world}",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)",
+                   "graphs": "3 CUDA graphs per step (select, top-K, attention)"},
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "algorithmic_bytes": attn_bytes,
+                     "peak_source": peaks["source"]},
+        "breakdown_us": {"append_summary+score": statistics.fmean(sel_ms) * 1e3,
+                         "topk": statistics.fmean(topk_ms) * 1e3, "attention": attn_avg * 1e3},
+        "step_hbm": {"bytes": step_bytes, "gbs": step_bytes / (ms_per_step / 1e3) / 1e9,
+                     "frac": step_bytes / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+                     "what": "selected K/V union + summaries read, over the whole step time"},
+        "score_kernel_bytes": score_bytes,
+        "union_blocks": union_blocks, "per_head_blocks": per_head_blocks,
+        "needle_recall": hits / max(1, tot),
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": q.numel() * 2,
+                "d2h_bytes_per_step": o.numel() * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "clock_samples": clocks["samples"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        summ = oracle_summaries(case, range(case.B))
+        tsec, done = 0.0, 0
+        while tsec < args.cpu_seconds and done < 64:
+            tsec += oracle_decode_sample(case, [done % case.B], summ)
+            done += 1
+        line["cpu_baseline"] = {"value": done / tsec, "unit": "tokens/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"{done} decode tokens (batch rows, all 32 heads) of "
+                                          "the same workload, summaries precomputed"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="sas_gqa_decode_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

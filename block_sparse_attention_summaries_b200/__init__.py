@@ -1,0 +1,264 @@
+"""Python binding of libbsa.so: block-sparse causal attention with per-block summaries (B200).
+
+Every function here only marshals arguments (tensor pointers, sizes, the current CUDA stream) to
+the C entry point of the same name in ``include/bsa.h`` (``build_block_summaries`` ->
+``bsa_build_block_summaries`` and so on) and allocates output tensors with PyTorch.  All
+arithmetic runs in the library's CUDA kernels; there is no CPU or PyTorch fallback: if the shared
+library is missing, importing the binding's functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+
+BSA_F32, BSA_BF16 = 0, 1
+GATE_NONE, GATE_LOG_SOFTMAX = 0, 1
+NORM_SELECTED, NORM_ALL_HISTORY = 0, 1
+STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_ARG", 2: "BSA_ERR_SHAPE", 3: "BSA_ERR_DTYPE",
+                4: "BSA_ERR_UNSUPPORTED", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_TIMEOUT",
+                7: "BSA_ERR_WORKSPACE"}
+
+# (name, restype, argtypes) of every exported entry point, in header order.
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = [
+    ("bsa_status_string", ctypes.c_char_p, [_I]),
+    ("bsa_version", _I, []),
+    ("bsa_build_block_summaries", _I, [_P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _P, _P, _P, _P]),
+    ("bsa_score_blocks", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                              _P]),
+    ("bsa_topk_blocks", _I, [_P, _I, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]),
+    ("bsa_sparse_attn_fwd", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _I,
+                                 _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
+    ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
+                           _P, _I, _P, _P]),
+    ("bsa_workspace_status", _I, [_P, _P]),
+    ("bsa_selftest_bounded_wait", _I, [_P, _I, _P]),
+]
+
+_lib = None
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libbsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m block_sparse_attention_summaries_b200.build_lib`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise BsaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BSA_BF16
+    if t.dtype == torch.float32:
+        return BSA_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def _i32(t):
+    if t is None:
+        return None
+    if t.dtype != torch.int32:
+        raise ValueError("index tensors must be int32")
+    return t
+
+
+def _norm_code(norm: str) -> int:
+    return {"selected": NORM_SELECTED, "all": NORM_ALL_HISTORY}[norm]
+
+
+# ---------------------------------------------------------------------------------------------
+# Entry points
+# ---------------------------------------------------------------------------------------------
+
+
+def build_block_summaries(k, b, seq_lens=None, first_block=0, num_blocks=-1, mean_k=None,
+                          max_norm=None, centre=None):
+    """Mean key, max key norm and centre of every block of b tokens of K [B, Hk, n, d]."""
+    _cuda(k, seq_lens, mean_k, max_norm, centre)
+    B, Hk, n, d = k.shape
+    C = (n + b - 1) // b
+    if mean_k is None:
+        mean_k = torch.empty(B, Hk, C, d, device=k.device, dtype=torch.float32)
+    if max_norm is None:
+        max_norm = torch.empty(B, Hk, C, device=k.device, dtype=torch.float32)
+    if centre is None:
+        centre = torch.empty(B, Hk, C, device=k.device, dtype=torch.float32)
+    _check(lib().bsa_build_block_summaries(_ptr(k), _dtype_code(k), B, Hk, n, d, b,
+                                           _ptr(_i32(seq_lens)), first_block, num_blocks,
+                                           _ptr(mean_k), _ptr(max_norm), _ptr(centre),
+                                           _stream(k.device)), "bsa_build_block_summaries")
+    return mean_k, max_norm, centre
+
+
+def score_blocks(q, mean_k, n, b, seq_lens=None, max_norm=None, centre=None, lambda_h=None,
+                 sigma_h=None, prefix_block=0, scores=None, n_cand=None, Hk=None):
+    """Decode block scores [B, Hq, C] of q [B, Hq, d] (and candidate counts [B*Hq])."""
+    _cuda(q, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, scores, n_cand)
+    B, Hq, d = q.shape
+    Hk = mean_k.shape[1] if Hk is None else Hk
+    C = (n + b - 1) // b
+    if scores is None:
+        scores = torch.empty(B, Hq, C, device=q.device, dtype=torch.float32)
+    if n_cand is None:
+        n_cand = torch.empty(B * Hq, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_score_blocks(_ptr(q), _dtype_code(q), B, Hq, Hk, n, d, b,
+                                  _ptr(_i32(seq_lens)), _ptr(mean_k), _ptr(max_norm),
+                                  _ptr(centre), _ptr(lambda_h), _ptr(sigma_h), prefix_block,
+                                  _ptr(scores), _ptr(n_cand), _stream(q.device)),
+           "bsa_score_blocks")
+    return scores, n_cand
+
+
+def topk_blocks(scores, K, n_cand=None, units=0, q_block=0, b=0, C=None, idx=None, count=None):
+    """Top-K block indices (ascending, -1 padded) of every row of scores [..., C]."""
+    _cuda(scores, n_cand, idx, count)
+    ld = scores.shape[-1]
+    C = ld if C is None else C
+    rows = scores.numel() // ld
+    lead = scores.shape[:-1]
+    if idx is None:
+        idx = torch.empty(*lead, K, device=scores.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(*lead, device=scores.device, dtype=torch.int32)
+    _check(lib().bsa_topk_blocks(_ptr(scores), rows, C, ld, _ptr(_i32(n_cand)), units, q_block, b,
+                                 K, _ptr(idx), _ptr(count), _stream(scores.device)),
+           "bsa_topk_blocks")
+    return idx, count
+
+
+_workspaces: dict = {}
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A zero-filled device workspace of at least ``nbytes`` cached per device (reused)."""
+    key = torch.device(device)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=key)
+        _workspaces[key] = ws
+    return ws
+
+
+def sparse_attn_workspace_bytes(B, Hq, Hk, nq, n, d, b, K) -> int:
+    return int(lib().bsa_sparse_attn_workspace_bytes(B, Hq, Hk, nq, n, d, b, K))
+
+
+def sparse_attn_fwd(q, k, v, idx, b, count=None, seq_lens=None, q_block=None, gate=False,
+                    norm="selected", scores=None, o=None, lse=None, ws=None):
+    """Exact causal softmax over the gathered tokens.
+
+    Decode: q [B, Hq, d] or [B, Hq, 1, d], idx [B, Hq, K].
+    Prefill: q [B, Hq, n, d], idx [B, Hq, U, K] with U = ceil(n / q_block).
+    Returns (o, lse).
+    """
+    _cuda(q, k, v, idx, count, seq_lens, scores, o, lse)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    decode = q.dim() == 3 or q.shape[2] == 1
+    nq = 1 if decode else q.shape[2]
+    K = idx.shape[-1]
+    if q_block is None:
+        q_block = b
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    need = sparse_attn_workspace_bytes(B, Hq, Hk, nq, n, d, b, K)
+    if ws is None:
+        ws = workspace(need, q.device)
+    scores_ld = scores.shape[-1] if scores is not None else 0
+    _check(lib().bsa_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, nq, n,
+                                     d, b, _ptr(_i32(seq_lens)), q_block, _ptr(_i32(idx)),
+                                     _ptr(_i32(count)), K,
+                                     GATE_LOG_SOFTMAX if gate else GATE_NONE, _norm_code(norm),
+                                     _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _ptr(ws),
+                                     ws.numel(), _stream(q.device)), "bsa_sparse_attn_fwd")
+    return o, lse
+
+
+def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, norm="selected",
+              dg=None):
+    """dg [B, Hq, U, K] of the inner log-gates (closed form, Eq. 5 of the SAS review)."""
+    _cuda(q, k, v, o, lse, dout, idx, scores, count, dg)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    K = idx.shape[-1]
+    if q_block is None:
+        q_block = b
+    U = (n + q_block - 1) // q_block
+    if dg is None:
+        dg = torch.empty(B, Hq, U, K, device=q.device, dtype=torch.float32)
+    _check(lib().bsa_gate_grad(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                               _dtype_code(q), B, Hq, Hk, n, d, b, q_block, _ptr(_i32(idx)),
+                               _ptr(_i32(count)), K, _norm_code(norm), _ptr(scores),
+                               scores.shape[-1], _ptr(dg), _stream(q.device)), "bsa_gate_grad")
+    return dg
+
+
+def workspace_status(ws) -> int:
+    """Status word of a workspace (0 ok, else BSA_ERR_TIMEOUT); clears it."""
+    return int(lib().bsa_workspace_status(_ptr(ws), _stream(ws.device)))
+
+
+def selftest_bounded_wait(ws, polls=1000) -> None:
+    """Launch the bounded-wait self-test kernel on ``ws`` (see bsa_selftest_bounded_wait)."""
+    _check(lib().bsa_selftest_bounded_wait(_ptr(ws), polls, _stream(ws.device)),
+           "bsa_selftest_bounded_wait")
+
+
+def decode_step(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_norm=None, centre=None,
+                out=None):
+    """One SAS decode step (the inference algorithm of the SAS review, step 6):
+    refresh the summary of the current block, score every history block with q . kbar / sqrt(d),
+    take Top-K, attend the selected blocks plus the current block.  Returns (o, lse, idx)."""
+    B, Hk, n, d = k.shape
+    if append:
+        # first_block = -1: the block holding each row's newest token
+        build_block_summaries(k, b, seq_lens, -1, 1, mean_k, max_norm, centre)
+    scores, n_cand = score_blocks(q, mean_k, n, b, seq_lens)
+    idx, count = topk_blocks(scores, K, n_cand=n_cand)
+    o, lse = sparse_attn_fwd(q, k, v, idx, b, count=count, seq_lens=seq_lens, o=out)
+    return o, lse, idx

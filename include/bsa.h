@@ -1,0 +1,195 @@
+/*
+ * bsa.h -- C ABI of libbsa.so: query-dependent block-sparse causal attention with per-block key
+ * summaries, hand-written for NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and the section / equation on it:
+ *   [SAS]        review page "SAS: Simple Attention Sparsification via End-to-End Optimization of
+ *                Context Ranking": "Background" (Eq. 1-3), "The new approach" (Eq. 4, Eq. 9),
+ *                "Why the four design choices matter" (Eq. 5, log g = s - LSE(s)),
+ *                "How it works: a worked example", "Decoding efficiency" (Fig. 7).
+ *   [FreeSolo]   summary page "FreeSolo가 학습 길이의 64배까지 제로샷 검색을 유지한다": "How it works".
+ *   [Monodratic] article "Monodratic、学習ルーティングによりスパース因果アテンションの選択性を高められると
+ *                主張": guaranteed local block + exact causal softmax over the selected tokens.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named q, k, v, o, dout, mean_k, ... are DEVICE pointers; sizes are host ints.
+ *  - Layouts are row-major with the head dimension d fastest:
+ *        Q, O, dO  [B, Hq, nq, d]      K, V  [B, Hk, n, d]
+ *    Query head h reads kv head h / (Hq / Hk) (contiguous GQA groups).
+ *  - Context of n positions is cut into C = ceil(n / b) blocks of b tokens; a short final block
+ *    keeps the remaining tokens ([SAS] "Background", Eq. 3).
+ *  - Block indices are int32, padding is -1; summaries, scores, lse and dg are float32.
+ *  - The caller owns every buffer (allocate with any allocator, e.g. PyTorch).  The library
+ *    never allocates or frees device memory and keeps no state between calls.
+ *  - Every call is asynchronous on the given cudaStream_t (passed as void*; NULL = legacy
+ *    default stream).  Arguments are checked on the host first; a bad argument returns an
+ *    error status and launches nothing.  A failed launch returns BSA_ERR_CUDA.
+ *  - Kernels that wait on the copy engine bound every wait; when a bound runs out they write a
+ *    nonzero word at the start of the workspace and stop.  bsa_workspace_status() reads it
+ *    (BSA_ERR_TIMEOUT) and clears it.
+ *  - Supported: dtype BSA_F32 or BSA_BF16, head dim d in {64, 128}, Hq % Hk == 0 with
+ *    Hq / Hk in {1, 2, 4, 8}, block size b in [1, 128] (decode) / [1, 1024] (summaries).
+ *    Other valid values return BSA_ERR_UNSUPPORTED.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_ARG = 1,          /* null pointer, negative size or unknown enum value */
+  BSA_ERR_SHAPE = 2,        /* sizes inconsistent with each other (Hq % Hk, K < 1, ...) */
+  BSA_ERR_DTYPE = 3,        /* unknown dtype */
+  BSA_ERR_UNSUPPORTED = 4,  /* valid request this build has no kernel for (e.g. d = 96) */
+  BSA_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+  BSA_ERR_TIMEOUT = 6,      /* a bounded device-side wait ran out (reported by status query) */
+  BSA_ERR_WORKSPACE = 7     /* workspace missing or smaller than *_workspace_bytes() */
+} bsa_status;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
+
+/* Training-mode gate of [SAS] "The new approach", Eq. 9. */
+typedef enum { BSA_GATE_NONE = 0, BSA_GATE_LOG_SOFTMAX = 1 } bsa_gate_mode;
+
+/* Set the softmax gate normalises over ([SAS] "Why the four design choices matter"):
+ * SELECTED = LSE over the selected history blocks, ALL_HISTORY = LSE over every history block. */
+typedef enum { BSA_NORM_SELECTED = 0, BSA_NORM_ALL_HISTORY = 1 } bsa_gate_norm;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* bsa_status_string(bsa_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int bsa_version(void);
+
+/*
+ * bsa_build_block_summaries -- per-block key summaries ([FreeSolo] "How it works": mean key of
+ * the cell, its centre position, the largest key norm inside it).
+ *
+ *   k         [B, Hk, n, d] keys (dtype dt).
+ *   seq_lens  optional [B] int32 device array of valid lengths (1..n); NULL = n for every row.
+ *             Tokens at or after seq_lens[b] are ignored; a block with no valid token gets
+ *             mean 0, max norm 0 and the centre of a full block.
+ *   b         block (cell) size in tokens.
+ *   first_block, num_blocks: compute blocks [first_block, first_block + num_blocks) only;
+ *             num_blocks = -1 means "to the end".  first_block = -1 computes, for every batch
+ *             row, the one block holding its newest token (position seq_lens[b] - 1): the
+ *             decode-time append of the block being filled.
+ *   mean_k    [B, Hk, C, d] float32 out:  (1/|c|) * sum_{j in c} k_j
+ *   max_norm  [B, Hk, C]    float32 out:  max_{j in c} ||k_j||_2
+ *   centre    [B, Hk, C]    float32 out:  mean position of the block's valid tokens
+ *   (max_norm and centre may be NULL when not wanted.)
+ */
+bsa_status bsa_build_block_summaries(const void* k, bsa_dtype dt, int B, int Hk, int n, int d,
+                                     int b, const int* seq_lens, int first_block, int num_blocks,
+                                     float* mean_k, float* max_norm, float* centre, void* stream);
+
+/*
+ * bsa_score_blocks -- decode block scores of one query per (batch, query head).
+ * The query of row b sits at position pos = seq_lens[b] - 1 (n - 1 if seq_lens is NULL).
+ *
+ *   s_c = q . kbar_c / sqrt(d)                                   ([SAS] Eq. 3 selector input;
+ *       + lambda_h * a_c * erf((pos - p_c) / (2 sigma_h))        [FreeSolo] cell score r_ic)
+ *
+ *   q         [B, Hq, d] (dtype dt); mean_k/max_norm/centre as written by the summaries call.
+ *   lambda_h, sigma_h: optional [Hq] float32 device arrays; both NULL = plain dot score.
+ *             max_norm and centre may be NULL when lambda_h is NULL.
+ *   prefix_block: 0 = SAS candidates c < pos / b ([SAS] Eq. 4: history blocks only);
+ *             P > 0 = FreeSolo candidates, cells lying before floor(pos / P) * P.
+ *   scores    [B, Hq, C] float32 out; non-candidate entries are written as -inf.
+ *   n_cand    optional [B * Hq] int32 out: number of candidates of each row.
+ */
+bsa_status bsa_score_blocks(const void* q, bsa_dtype dt, int B, int Hq, int Hk, int n, int d,
+                            int b, const int* seq_lens, const float* mean_k,
+                            const float* max_norm, const float* centre, const float* lambda_h,
+                            const float* sigma_h, int prefix_block, float* scores, int* n_cand,
+                            void* stream);
+
+/*
+ * bsa_topk_blocks -- I = Top-K(s, K) per row ([SAS] "Background", Eq. 3; worked example step 3).
+ *
+ *   scores    [rows, ld] float32; only the first C columns take part.
+ *   Candidates of a row are its columns c < n_cand(row), where
+ *       n_cand(row) = n_cand[row]                        if n_cand != NULL,
+ *                   = ((row % units) * q_block) / b      if n_cand == NULL and units > 0
+ *                     (prefill: history blocks of the first query of unit row % units),
+ *                   = C                                  otherwise.
+ *   Order: larger score first; equal scores -> lower index first; NaN ranks below everything
+ *   (and -0.0 equals +0.0).  Exactly min(K, n_cand) blocks are selected.
+ *   idx       [rows, K] int32 out, selected indices in ascending order, padded with -1.
+ *   count     optional [rows] int32 out, min(K, n_cand(row)).
+ *   Requires C <= 16384 and K <= 256.
+ */
+bsa_status bsa_topk_blocks(const float* scores, int rows, int C, int ld, const int* n_cand,
+                           int units, int q_block, int b, int K, int* idx, int* count,
+                           void* stream);
+
+/*
+ * bsa_sparse_attn_fwd -- exact causal softmax over the gathered tokens
+ * ([SAS] Eq. 2 and "How it works" step 6; [Monodratic]), optionally with the log-gate of
+ * [SAS] Eq. 9.
+ *
+ * Query i attends the tokens of the selected history blocks of its unit plus the tokens
+ * j <= i of its current block cur = i / b (always kept, gate 1):
+ *     o_i = sum_j softmax_j(q_i . k_j / sqrt(d) + [gate] log g_m(j)) v_j,  lse_i = log sum exp.
+ *
+ *   Decode (nq == 1): q [B, Hq, 1, d]; the query of row b sits at seq_lens[b] - 1 (n - 1 if
+ *     seq_lens is NULL); idx [B, Hq, K]; scores (gate only) [B, Hq, scores_ld].
+ *   Prefill (nq == n, seq_lens must be NULL): queries 0..n-1 in units of q_block consecutive
+ *     queries sharing one selection; idx [B, Hq, U, K] with U = ceil(n / q_block);
+ *     scores (gate only) [B, Hq, U, scores_ld].  The candidates of unit u are the history
+ *     blocks c < (u * q_block) / b of its first query.
+ *   idx       selected history blocks (ascending, -1 padded), e.g. from bsa_topk_blocks.
+ *   count     optional per-row/per-unit int32 count of valid idx entries; NULL = up to first -1.
+ *   gate      BSA_GATE_LOG_SOFTMAX adds log g_m = s_m - LSE(normaliser set) to the logits of
+ *             selected history block m; the current block gets 0 ([SAS] Eq. 4).
+ *   o         [B, Hq, nq, d] out (dtype dt);  lse  optional [B, Hq, nq] float32 out.
+ *   workspace device scratch of bsa_sparse_attn_workspace_bytes() bytes, zero-filled before its
+ *             first use; each successful call leaves it reusable.  Calls sharing one workspace
+ *             must not run concurrently.
+ */
+bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                               int Hq, int Hk, int nq, int n, int d, int b,
+                               const int* seq_lens, int q_block, const int* idx,
+                               const int* count, int K, bsa_gate_mode gate, bsa_gate_norm norm,
+                               const float* scores, int scores_ld, void* o, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+size_t bsa_sparse_attn_workspace_bytes(int B, int Hq, int Hk, int nq, int n, int d, int b,
+                                       int K);
+
+/*
+ * bsa_gate_grad -- closed-form gradient of the loss with respect to the inner gates
+ * ([SAS] "Why the four design choices matter", Eq. 5):
+ *     dg_m = sum_{i in B_m} (ptilde_i / g_m) * do^T (v_i - o),
+ * summed over the queries of the unit that shares gate g_m.  Same layouts as the prefill form of
+ * bsa_sparse_attn_fwd; o and lse are that call's gated outputs, dout the upstream gradient.
+ *   dg        [B, Hq, U, K] float32 out (0 in padded slots).
+ */
+bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, bsa_dtype dt, int B, int Hq, int Hk,
+                         int n, int d, int b, int q_block, const int* idx, const int* count,
+                         int K, bsa_gate_norm norm, const float* scores, int scores_ld,
+                         float* dg, void* stream);
+
+/* Read and clear the status word a bounded device wait writes into a workspace
+ * (synchronises the stream).  Returns BSA_OK or BSA_ERR_TIMEOUT (or BSA_ERR_CUDA). */
+bsa_status bsa_workspace_status(void* workspace, void* stream);
+
+/* Failure-path self-test (no counterpart in the pages): one thread waits on an mbarrier that is
+ * never completed, gives up after `polls` polls and writes the timeout into the status word of
+ * `workspace` (>= 256 bytes, device).  A following bsa_workspace_status() returns
+ * BSA_ERR_TIMEOUT; the CUDA context stays usable. */
+bsa_status bsa_selftest_bounded_wait(void* workspace, int polls, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -25,3 +25,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def bsa_lib():
+    """libbsa.so, built in-tree from the CUDA sources when missing or stale (nvcc cross-compiles
+    for sm_100a without a GPU)."""
+    from block_sparse_attention_summaries_b200 import build_lib
+    import block_sparse_attention_summaries_b200 as bsa
+    build_lib.build()
+    return bsa.lib()

@@ -1,0 +1,146 @@
+"""The C ABI: the library loads, exports every symbol include/bsa.h declares, and rejects bad
+arguments on the host before touching the GPU (CPU only: no compute call is made)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import block_sparse_attention_summaries_b200 as bsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsa.h")
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails validation first
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for must in ["bsa_build_block_summaries", "bsa_score_blocks", "bsa_topk_blocks",
+                 "bsa_sparse_attn_fwd", "bsa_gate_grad"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(bsa_lib):
+    for name in declared_functions():
+        assert hasattr(bsa_lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", bsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (bsa_\w+)", out))
+    assert set(declared_functions()) <= exported
+    # every binding signature names an exported symbol
+    assert {n for n, _, _ in bsa.SIGNATURES} <= exported
+
+
+def test_binding_covers_header():
+    assert {n for n, _, _ in bsa.SIGNATURES} == set(declared_functions())
+
+
+def test_status_strings(bsa_lib):
+    for code in range(8):
+        s = bsa_lib.bsa_status_string(code)
+        assert s and s != b"unknown status"
+    assert bsa_lib.bsa_status_string(42) == b"unknown status"
+    assert bsa_lib.bsa_version() >= 100
+
+
+def test_summaries_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_build_block_summaries
+    ok = dict(k=FAKE, dt=1, B=1, Hk=1, n=128, d=128, b=64, seq=None, first=0, nb=-1,
+              mean=FAKE, mx=None, ce=None, st=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["k"], a["dt"], a["B"], a["Hk"], a["n"], a["d"], a["b"], a["seq"], a["first"],
+                 a["nb"], a["mean"], a["mx"], a["ce"], a["st"])
+
+    assert call(k=None) == 1
+    assert call(mean=None) == 1
+    assert call(dt=9) == 3
+    assert call(n=0) == 1
+    assert call(b=-1) == 1
+    assert call(d=96) == 4
+    assert call(first=3) == 2  # past the last block
+    assert call(first=1, nb=5) == 2
+    assert call(first=2, nb=0) == 0  # empty range: nothing to do, nothing launched
+
+
+def test_score_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_score_blocks
+    base = [FAKE, 1, 2, 8, 2, 1024, 128, 64, None, FAKE, None, None, None, None, 0, FAKE, None,
+            None]
+    assert f(*base[:0], None, *base[1:]) == 1
+    bad = list(base); bad[4] = 3
+    assert f(*bad) == 2  # Hq % Hk
+    bad = list(base); bad[3] = 24; bad[4] = 2
+    assert f(*bad) == 4  # group of 12
+    bad = list(base); bad[12] = FAKE  # lambda without sigma
+    assert f(*bad) == 1
+    bad = list(base); bad[12] = FAKE; bad[13] = FAKE  # lambda without max_norm / centre
+    assert f(*bad) == 1
+    bad = list(base); bad[6] = 80
+    assert f(*bad) == 4
+
+
+def test_topk_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_topk_blocks
+    assert f(None, 4, 16, 16, None, 0, 0, 0, 4, FAKE, None, None) == 1
+    assert f(FAKE, 4, 16, 8, None, 0, 0, 0, 4, FAKE, None, None) == 1  # ld < C
+    assert f(FAKE, 4, 16, 16, None, 0, 0, 0, 0, FAKE, None, None) == 1  # K = 0
+    assert f(FAKE, 4, 20000, 20000, None, 0, 0, 0, 4, FAKE, None, None) == 4
+    assert f(FAKE, 4, 16, 16, None, 0, 0, 0, 300, FAKE, None, None) == 4
+    assert f(FAKE, 4, 16, 16, None, 3, 0, 0, 4, FAKE, None, None) == 1  # units w/o q_block
+    assert f(FAKE, 0, 16, 16, None, 0, 0, 0, 4, FAKE, None, None) == 0  # no rows: no launch
+
+
+def test_attention_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_sparse_attn_fwd
+    base = [FAKE, FAKE, FAKE, 1, 2, 8, 2, 1, 1024, 128, 64, None, 64, FAKE, None, 4, 0, 0, None,
+            0, FAKE, None, FAKE, 1 << 20, None]
+    bad = list(base); bad[1] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[3] = 5
+    assert f(*bad) == 3
+    bad = list(base); bad[16] = 1  # gate without scores
+    assert f(*bad) == 1
+    bad = list(base); bad[16] = 1; bad[18] = FAKE; bad[19] = 3  # scores_ld < C
+    assert f(*bad) == 2
+    bad = list(base); bad[22] = None  # decode needs a workspace
+    assert f(*bad) == 7
+    bad = list(base); bad[23] = 16  # too small
+    assert f(*bad) == 7
+    bad = list(base); bad[7] = 512  # prefill needs nq == n
+    assert f(*bad) == 2
+    bad = list(base); bad[7] = 1024; bad[11] = FAKE  # prefill takes no seq_lens
+    assert f(*bad) == 1
+    bad = list(base); bad[10] = 256  # decode block too large
+    assert f(*bad) == 4
+
+
+def test_workspace_size_query(bsa_lib):
+    q = bsa_lib.bsa_sparse_attn_workspace_bytes
+    n = q(8, 32, 8, 1, 32768, 128, 64, 15)
+    assert n > 8 * 32 * (128 + 2) * 4
+    assert q(8, 32, 8, 1, 32768, 128, 64, 15) == n  # deterministic, no device query
+    assert q(8, 30, 8, 1, 32768, 128, 64, 15) == 0
+    assert q(2, 32, 8, 16384, 16384, 128, 64, 16) >= 256
+
+
+def test_gate_grad_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_gate_grad
+    base = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 8, 2, 1024, 128, 64, 64, FAKE, None, 4, 0,
+            FAKE, 16, FAKE, None]
+    bad = list(base); bad[5] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[18] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[19] = 8
+    assert f(*bad) == 2
+    bad = list(base); bad[17] = 5
+    assert f(*bad) == 1
