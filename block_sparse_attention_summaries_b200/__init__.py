@@ -35,6 +35,8 @@ SIGNATURES = [
     ("bsa_sparse_attn_fwd", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _I,
                                  _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
     ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    ("bsa_sparse_attn_decode_noalloc", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
+                                            _I, _I, _I, _P, _I, _P, _P, _P]),
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
     ("bsa_workspace_status", _I, [_P, _P]),
@@ -216,6 +218,29 @@ def sparse_attn_fwd(q, k, v, idx, b, count=None, seq_lens=None, q_block=None, ga
                                      GATE_LOG_SOFTMAX if gate else GATE_NONE, _norm_code(norm),
                                      _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _ptr(ws),
                                      ws.numel(), _stream(q.device)), "bsa_sparse_attn_fwd")
+    return o, lse
+
+
+def sparse_attn_decode_noalloc(q, k, v, idx, b, count=None, seq_lens=None, gate=False,
+                               norm="selected", scores=None, o=None, lse=None):
+    """Decode attention like ``sparse_attn_fwd`` but with no workspace: the library's fixed
+    per-device scratch array is used instead (for callers that cannot allocate device memory).
+    Concurrent calls race on that array; the first call on a device must precede stream
+    capture."""
+    _cuda(q, k, v, idx, count, seq_lens, scores, o, lse)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    K = idx.shape[-1]
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    scores_ld = scores.shape[-1] if scores is not None else 0
+    _check(lib().bsa_sparse_attn_decode_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b, _ptr(_i32(seq_lens)),
+        _ptr(_i32(idx)), _ptr(_i32(count)), K, GATE_LOG_SOFTMAX if gate else GATE_NONE,
+        _norm_code(norm), _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _stream(q.device)),
+        "bsa_sparse_attn_decode_noalloc")
     return o, lse
 
 

@@ -19,6 +19,8 @@
 //  * Logits of R = 32/G tokens x G heads are reduced with one 31-shuffle transpose-reduce.
 #include "bsa_common.cuh"
 
+#include <mutex>
+
 namespace bsa {
 namespace {
 
@@ -471,3 +473,86 @@ bsa_status decode_attn(const void* q, const void* k, const void* v, bsa_dtype dt
 }
 
 }  // namespace bsa
+
+// ------------------------------------------------------------------------------------------
+// Decode attention without any caller-provided or library-allocated workspace.
+//
+// Some callers cannot hand the library device memory: an inference engine that plans every
+// device byte up front and forbids any allocation outside that plan, a plugin invoked by a host
+// framework that owns the allocator and exposes none to it, or a driver loop whose latency budget
+// rules out an allocator call.  For them the split-K scratch (status word, arrival counters,
+// per-split partials) lives in one file-scope device array of fixed size that every GPU loading
+// this library holds until the process exits.  Callers still pass inputs and outputs.
+// ------------------------------------------------------------------------------------------
+
+namespace bsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once per device.  In
+// host code `g_noalloc_scratch` names a host-side stand-in, not device memory, so the address
+// must come from cudaGetSymbolAddress with the device current.
+bsa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      (void)cudaGetLastError();
+      return BSA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" bsa_status bsa_sparse_attn_decode_noalloc(
+    const void* q, const void* k, const void* v, bsa_dtype dt, int B, int Hq, int Hk, int n,
+    int d, int b, const int* seq_lens, const int* idx, const int* count, int K,
+    bsa_gate_mode gate, bsa_gate_norm norm, const float* scores, int scores_ld, void* o,
+    float* lse, void* stream) {
+  using namespace bsa;
+  BSA_REQUIRE(dtype_ok(dt), BSA_ERR_DTYPE);
+  BSA_REQUIRE(q && k && v && idx && o, BSA_ERR_ARG);
+  BSA_REQUIRE(B > 0 && Hq > 0 && Hk > 0 && n > 0 && d > 0 && b > 0 && K > 0, BSA_ERR_ARG);
+  BSA_REQUIRE(Hq % Hk == 0, BSA_ERR_SHAPE);
+  BSA_REQUIRE(group_ok(Hq, Hk), BSA_ERR_UNSUPPORTED);
+  BSA_REQUIRE(head_dim_ok(d), BSA_ERR_UNSUPPORTED);
+  BSA_REQUIRE(B <= 65535 && Hk <= 65535 && b <= 128, BSA_ERR_UNSUPPORTED);
+  BSA_REQUIRE(all_aligned16(q, k, v, o), BSA_ERR_ARG);
+  BSA_REQUIRE(gate == BSA_GATE_NONE || gate == BSA_GATE_LOG_SOFTMAX, BSA_ERR_ARG);
+  BSA_REQUIRE(norm == BSA_NORM_SELECTED || norm == BSA_NORM_ALL_HISTORY, BSA_ERR_ARG);
+  if (gate == BSA_GATE_LOG_SOFTMAX) {
+    BSA_REQUIRE(scores != nullptr, BSA_ERR_ARG);
+    BSA_REQUIRE(scores_ld >= ceil_div(n, b), BSA_ERR_SHAPE);
+  }
+  const int S = decode_splits(B, Hk, Hq / Hk, K);
+  const size_t need = decode_workspace_bytes(B, Hq, Hk, d, K, S);
+  if (need > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* ws = nullptr;
+  bsa_status rc = noalloc_scratch(&ws);
+  if (rc != BSA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: zero the status word and arrival counters
+  const size_t zero_bytes = 256 + align_up((size_t)B * Hk * sizeof(int), 256);
+  if (cudaMemsetAsync(ws, 0, zero_bytes, st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  return decode_attn(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, idx, count, K, gate, norm,
+                     scores, scores_ld, o, lse, ws, kNoAllocScratchBytes, st);
+}

@@ -178,6 +178,33 @@ bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void
                          int K, bsa_gate_norm norm, const float* scores, int scores_ld,
                          float* dg, void* stream);
 
+/*
+ * bsa_sparse_attn_decode_noalloc -- the decode form of bsa_sparse_attn_fwd (nq == 1) for callers
+ * that cannot provide device memory: an engine that plans all device memory ahead and forbids
+ * any other allocation, or a plugin whose host framework owns the allocator and gives it none.
+ * The pages have no counterpart to this call; it exists for those callers only.
+ *
+ * Arguments, layouts and results are those of bsa_sparse_attn_fwd with nq = 1, minus the
+ * workspace.  Instead of a workspace it uses one fixed 4 MiB device array inside the library,
+ * which every GPU that loads the library keeps until the process exits.  Nothing is allocated:
+ * no cudaMalloc, cudaFree or allocating library routine is called.
+ *  - Limit: a problem whose split-K scratch (see bsa_sparse_attn_workspace_bytes with nq = 1)
+ *    exceeds 4 MiB is rejected with BSA_ERR_WORKSPACE, before any launch.
+ *  - The first call on a device looks up the array's device address (once per device, with the
+ *    device current); make that first call before any CUDA stream capture.
+ *  - Every call shares the one array, which keeps the previous call's contents; each call zeroes
+ *    the parts that must start at zero.  Calls that overlap on the GPU (other streams, other
+ *    threads, concurrent graph launches) race on the array and give wrong results.
+ *  - A bounded wait that runs out is not reported by this call (the status word is cleared at
+ *    the start of the next one).
+ */
+bsa_status bsa_sparse_attn_decode_noalloc(const void* q, const void* k, const void* v,
+                                          bsa_dtype dt, int B, int Hq, int Hk, int n, int d,
+                                          int b, const int* seq_lens, const int* idx,
+                                          const int* count, int K, bsa_gate_mode gate,
+                                          bsa_gate_norm norm, const float* scores, int scores_ld,
+                                          void* o, float* lse, void* stream);
+
 /* Read and clear the status word a bounded device wait writes into a workspace
  * (synchronises the stream).  Returns BSA_OK or BSA_ERR_TIMEOUT (or BSA_ERR_CUDA). */
 bsa_status bsa_workspace_status(void* workspace, void* stream);
