@@ -39,6 +39,11 @@ SIGNATURES = [
                                             _I, _I, _I, _P, _I, _P, _P, _P]),
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
+    ("bsa_freesolo_select", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P,
+                                 _P]),
+    ("bsa_freesolo_attn", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P,
+                               _P, _I, _P, _P, _Z, _P]),
+    ("bsa_freesolo_workspace_bytes", _Z, [_I, _I, _I, _I, _I]),
     ("bsa_workspace_status", _I, [_P, _P]),
     ("bsa_selftest_bounded_wait", _I, [_P, _I, _P]),
 ]
@@ -261,6 +266,40 @@ def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, n
                                _ptr(_i32(count)), K, _norm_code(norm), _ptr(scores),
                                scores.shape[-1], _ptr(dg), _stream(q.device)), "bsa_gate_grad")
     return dg
+
+
+def freesolo_select(q, mean_k, max_norm, centre, lambda_h, sigma_h, cell, q_block, K,
+                    idx=None, count=None):
+    """Per-query top-K cells of the FreeSolo long branch: idx [B, H, n, K], count [B, H, n]."""
+    _cuda(q, mean_k, max_norm, centre, lambda_h, sigma_h, idx, count)
+    B, H, n, d = q.shape
+    if idx is None:
+        idx = torch.empty(B, H, n, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, H, n, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_freesolo_select(_ptr(q), _dtype_code(q), B, H, n, d, cell, q_block,
+                                     _ptr(mean_k), _ptr(max_norm), _ptr(centre), _ptr(lambda_h),
+                                     _ptr(sigma_h), K, _ptr(idx), _ptr(count), _stream(q.device)),
+           "bsa_freesolo_select")
+    return idx, count
+
+
+def freesolo_attn(q, k, v, alpha_h, idx, count, cell, window, rope_theta=10000.0, o=None,
+                  ws=None):
+    """FreeSolo two-branch output o [B, H, n, d]."""
+    _cuda(q, k, v, alpha_h, idx, count, o)
+    B, H, n, d = q.shape
+    K = idx.shape[-1]
+    if o is None:
+        o = torch.empty_like(q)
+    need = int(lib().bsa_freesolo_workspace_bytes(_dtype_code(q), B, H, n, d))
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check(lib().bsa_freesolo_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, H, n, d, cell,
+                                   window, float(rope_theta), _ptr(alpha_h), _ptr(_i32(idx)),
+                                   _ptr(_i32(count)), K, _ptr(o), _ptr(ws), ws.numel(),
+                                   _stream(q.device)), "bsa_freesolo_attn")
+    return o
 
 
 def workspace_status(ws) -> int:

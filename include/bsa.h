@@ -179,6 +179,42 @@ bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void
                          float* dg, void* stream);
 
 /*
+ * bsa_freesolo_select -- per-query cell selection of the FreeSolo long branch (prefill),
+ * [FreeSolo] "How it works": for the query at position i of head h the candidates are the cells
+ * c lying wholly before the start of its query block, (c + 1) * cell <= floor(i / q_block) *
+ * q_block, scored by
+ *     r_ic = q_i . kbar_c / sqrt(d) + lambda_h * a_c * erf((i - p_c) / (2 sigma_h)),
+ * and the K best cells are kept (ties to the lower index, NaN last).
+ *   q         [B, H, n, d] (MHA: one kv head per query head).
+ *   mean_k, max_norm, centre: cell summaries [B, H, C, d] / [B, H, C] / [B, H, C] with
+ *             C = ceil(n / cell), from bsa_build_block_summaries with b = cell.
+ *   lambda_h, sigma_h: [H] float32 device arrays.
+ *   idx       [B, H, n, K] int32 out, ascending, -1 padded; count optional [B, H, n] out.
+ *   K <= 8.
+ */
+bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, int H, int n, int d,
+                               int cell, int q_block, const float* mean_k, const float* max_norm,
+                               const float* centre, const float* lambda_h, const float* sigma_h,
+                               int K, int* idx, int* count, void* stream);
+
+/*
+ * bsa_freesolo_attn -- FreeSolo two-branch prefill output ([FreeSolo] "How it works"):
+ *     o_i = (1 - alpha_h) o_short_i + alpha_h o_long_i      (o_short_i alone when count = 0)
+ * o_short: softmax attention of RoPE(q_i) over RoPE(k_j), j in [i - window + 1, i] (RoPE base
+ * rope_theta, rotate-half pairing t <-> t + d/2, absolute positions).
+ * o_long: softmax attention of the raw q_i over the raw tokens of its selected cells (NoPE).
+ *   idx/count as written by bsa_freesolo_select (cells not wholly at or before i are ignored).
+ *   alpha_h   [H] float32 device array.   o  [B, H, n, d] out (dtype dt).
+ *   workspace device scratch of bsa_freesolo_workspace_bytes() bytes (holds the rotated keys).
+ */
+bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                             int H, int n, int d, int cell, int window, float rope_theta,
+                             const float* alpha_h, const int* idx, const int* count, int K,
+                             void* o, void* workspace, size_t workspace_bytes, void* stream);
+
+size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d);
+
+/*
  * bsa_sparse_attn_decode_noalloc -- the decode form of bsa_sparse_attn_fwd (nq == 1) for callers
  * that cannot provide device memory: an engine that plans all device memory ahead and forbids
  * any other allocation, or a plugin whose host framework owns the allocator and gives it none.

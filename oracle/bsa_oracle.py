@@ -428,14 +428,16 @@ def rope(x, pos: int, theta: float = 10000.0):
     return np.concatenate([a * c - b * s, b * c + a * s])
 
 
-def freesolo_row(q, k, v, i, summaries, cell, q_block, K, window, lam, sigma, alpha, theta):
+def freesolo_row(q, k, v, i, summaries, cell, q_block, K, window, lam, sigma, alpha, theta,
+                 selection=None):
     """Two-branch output of the query at position i of one head ([FreeSolo] "How it works").
 
     Short branch: softmax attention of RoPE(q_i) over RoPE(k_j), j in [i-window+1, i].
     Long branch: candidate cells fixed by the query block, cell score r_ic, Top-K cells, one
     softmax over the raw (unrotated) tokens of those cells.  Mix (R8):
     o = (1 - alpha) o_short + alpha o_long; o = o_short when no cell is a candidate (R4).
-    Returns o, and the selected cells.
+    ``selection`` replaces the Top-K set by another set of candidate cells (used to evaluate the
+    other valid sets of a near-tie).  Returns o, and the selected cells.
     """
     d = q.shape[0]
     mean_k, max_norm, centre = summaries
@@ -450,7 +452,7 @@ def freesolo_row(q, k, v, i, summaries, cell, q_block, K, window, lam, sigma, al
     if nc == 0:
         return o_short, []
     r = round_f32(freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, nc))
-    sel = topk_blocks(r, nc, K)
+    sel = topk_blocks(r, nc, K) if selection is None else list(selection)
     toks = np.concatenate([np.arange(*block_range(c, k.shape[0], cell)) for c in sel])
     o_long, _, _ = attend(q, k, v, toks, np.zeros(len(toks)))
     return (1.0 - alpha) * o_short + alpha * o_long, sel

@@ -455,3 +455,17 @@ def test_planted_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(orc, "block_range", lambda c, nn, bb: (c * bb, min(nn, (c + 1) * bb - 1)))
     assert worst() > 1e-3  # a block that loses its last token
     monkeypatch.setattr(orc, "block_range", good_range)
+
+
+def test_freesolo_explicit_selection_matches_default():
+    n, d, cell, qb = 96, 8, 8, 32
+    q, k, v = rnd(42, n, d), rnd(43, n, d), rnd(44, n, d)
+    summ = orc.block_summaries(k, cell)
+    args = dict(cell=cell, q_block=qb, K=2, window=16, lam=0.5, sigma=50.0, alpha=0.4,
+                theta=10000.0)
+    for i in [40, 70, 95]:
+        o1, sel = orc.freesolo_row(q[i], k, v, i, summ, **args)
+        o2, sel2 = orc.freesolo_row(q[i], k, v, i, summ, selection=sel, **args)
+        assert sel2 == sel and np.max(np.abs(o1 - o2)) == 0.0
+        o3, _ = orc.freesolo_row(q[i], k, v, i, summ, selection=[0], **args)
+        assert np.max(np.abs(o3 - o1)) > 0  # a different set changes the long branch
