@@ -32,6 +32,8 @@ SIGNATURES = [
     ("bsa_score_blocks", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                               _P]),
     ("bsa_topk_blocks", _I, [_P, _I, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]),
+    ("bsa_decode_step", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P,
+                             _I, _I, _P, _P, _P, _P, _P, _P]),
     ("bsa_sparse_attn_fwd", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _I,
                                  _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
     ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -313,11 +315,35 @@ def selftest_bounded_wait(ws, polls=1000) -> None:
            "bsa_selftest_bounded_wait")
 
 
+def decode_step_fused(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_norm=None,
+                      centre=None, lambda_h=None, sigma_h=None, prefix_block=0, o=None, lse=None,
+                      idx=None, count=None, status=None):
+    """One whole decode step in one launch (bsa_decode_step): returns (o, lse, idx, count)."""
+    _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    if idx is None:
+        idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b,
+                                 _ptr(_i32(seq_lens)), _ptr(mean_k), _ptr(max_norm), _ptr(centre),
+                                 1 if append else 0, _ptr(lambda_h), _ptr(sigma_h), prefix_block,
+                                 K, _ptr(o), _ptr(lse), _ptr(idx), _ptr(count), _ptr(status),
+                                 _stream(q.device)), "bsa_decode_step")
+    return o, lse, idx, count
+
+
 def decode_step(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_norm=None, centre=None,
                 out=None):
-    """One SAS decode step (the inference algorithm of the SAS review, step 6):
-    refresh the summary of the current block, score every history block with q . kbar / sqrt(d),
-    take Top-K, attend the selected blocks plus the current block.  Returns (o, lse, idx)."""
+    """One SAS decode step through the separate calls (the inference algorithm of the SAS review,
+    step 6): refresh the summary of the current block, score every history block with
+    q . kbar / sqrt(d), take Top-K, attend the selected blocks plus the current block.
+    Returns (o, lse, idx)."""
     B, Hk, n, d = k.shape
     if append:
         # first_block = -1: the block holding each row's newest token

@@ -1,17 +1,466 @@
-// Tensor-core (tcgen05) sparse prefill attention -- placeholder until the kernel lands.
-#include "bsa_common.cuh"
+// Sparse prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// [SAS] review: "Background" Eq. 2 (exact softmax over the selected set only), "The new approach"
+// Eq. 4 / Eq. 9 (current block always kept with gate 1; in training mode log g_m added to the
+// logits of selected history block m), "Kernel implementation" paragraph of "How it works" (the
+// gate is fused into a FlashAttention-style tiled qK^T loop: K/V tiles stream in, the log-gate is
+// added to the logits, unselected blocks never enter, the current block is unbiased, an online
+// softmax keeps the attention matrix out of memory).
+//
+// One CTA takes two query units (64 queries each) -- heads h and h+1 of the same kv group at the
+// same unit u -- and runs them in lockstep over their block lists (selected history blocks, then
+// the diagonal current block).  Each unit is an M = 64 tile; the two tiles' accumulators occupy
+// complementary halves of the TMEM lanes (rows of unit 0 in lanes 0-15 of every 32-lane
+// sub-partition, unit 1 in lanes 16-31), so the four softmax warps own one row per thread.
+//
+//   warp 4  (1 thread): TMA producer: Q tiles once, then per step the K and V blocks of both units
+//                       (128-byte swizzled 64x64 boxes) into a 2-stage ring.
+//   warp 5  (1 thread): MMA issuer: S_j = Q K_j^T into a double-buffered TMEM score tile, issued one
+//                       step ahead; O += P_j V_j once the softmax has written P_j.
+//   warps 0-3 (128):    softmax: tcgen05.ld of the score row, gate bias / causal mask, online max
+//                       with lazy rescaling (O in TMEM is rescaled only when the row max grows by
+//                       more than 2^8), P written to shared memory in the MMA's swizzled layout;
+//                       epilogue O / l and lse.
+// Every mbarrier wait is bounded; on timeout the CTA records it, skips the rest of its work and
+// still reaches its final barrier and TMEM release.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tc_common.cuh"
 
 namespace bsa {
+namespace {
 
-bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq, int Hk) {
-  (void)dt; (void)d; (void)b; (void)q_block; (void)K; (void)Hq; (void)Hk;
-  return false;
+constexpr int kTiles = 64;         // queries per unit = keys per block
+constexpr int kMaxKtc = 64;        // selected history blocks per unit
+constexpr int kThreadsTc = 192;    // 4 softmax warps + producer + MMA
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.f;    // lazy rescale threshold (log2 units)
+
+struct TcParams {
+  int B, Hq, Hk, n, U, K;
+  const int* idx;
+  const int* count;
+  int gate, norm;
+  const float* scores;
+  int scores_ld;
+  void* o;
+  float* lse;
+  int* status;
+};
+
+template <int D>
+struct TcSmem {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTiles * D * 2;  // one [64 x D] bf16 tile
+  static constexpr int kQ = 0;                       // 2 query tiles
+  static constexpr int kStage = 2 * kTileBytes;      // stages: K0 V0 K1 V1
+  static constexpr int kStageBytes = 4 * kTileBytes;
+  static constexpr int kP = kStage + 2 * kStageBytes;  // 2 P tiles [64 x 64] bf16
+  static constexpr int kPBytes = kTiles * 64 * 2;
+  static constexpr int kBars = kP + 2 * kPBytes;
+  static constexpr int kTotal = kBars + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                      const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const TcParams p) {
+  using L = TcSmem<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment of the swizzled tiles
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* fin = bars + 11;
+
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_blk[2][kMaxKtc + 1];
+  __shared__ float s_bias[2][kMaxKtc + 1];
+  __shared__ int s_cnt[2];
+  __shared__ int s_steps;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.x, hp = blockIdx.y, bi = blockIdx.z;
+  const int hq[2] = {2 * hp, 2 * hp + 1};
+  const int G = p.Hq / p.Hk;
+  const int kh = hq[0] / G;  // both heads of the pair share the kv head (G is even)
+  const int nc = u;          // history blocks before unit u (q_block == b)
+
+  // ---- prologue: block lists and gate biases of both units (warps 0 and 1) -----------------
+  if (warp < 2) {
+    const int it = warp;
+    const size_t row = ((size_t)bi * p.Hq + hq[it]) * p.U + u;
+    const int cnt_in = p.count ? min(p.count[row], p.K) : p.K;
+    int base = 0;
+    for (int j0 = 0; j0 < cnt_in; j0 += 32) {
+      const int j = j0 + lane;
+      const int m = j < cnt_in ? p.idx[row * p.K + j] : -1;
+      const bool ok = j < cnt_in && m >= 0 && m < nc;
+      const unsigned bal = __ballot_sync(0xffffffffu, ok);
+      if (ok && base + __popc(bal & ((1u << lane) - 1u)) < kMaxKtc)
+        s_blk[it][base + __popc(bal & ((1u << lane) - 1u))] = m;
+      base += __popc(bal);
+    }
+    base = min(base, kMaxKtc);
+    float lnorm = 0.f;
+    if (p.gate == BSA_GATE_LOG_SOFTMAX) {
+      const float* srow = p.scores + row * p.scores_ld;
+      __syncwarp();
+      float mx = -INFINITY, acc = 0.f;
+      if (p.norm == BSA_NORM_ALL_HISTORY) {
+        for (int c = lane; c < nc; c += 32) mx = fmaxf(mx, srow[c]);
+        mx = warp_max(mx);
+        for (int c = lane; c < nc; c += 32) acc += exp2f((srow[c] - mx) * kLog2e);
+      } else {
+        for (int j = lane; j < base; j += 32) mx = fmaxf(mx, srow[s_blk[it][j]]);
+        mx = warp_max(mx);
+        for (int j = lane; j < base; j += 32) acc += exp2f((srow[s_blk[it][j]] - mx) * kLog2e);
+      }
+      acc = warp_sum(acc);
+      lnorm = mx == -INFINITY ? 0.f : mx + logf(acc);
+      for (int j = lane; j < base; j += 32) s_bias[it][j] = (srow[s_blk[it][j]] - lnorm) * kLog2e;
+    } else {
+      for (int j = lane; j < base; j += 32) s_bias[it][j] = 0.f;
+    }
+    if (lane == 0) s_cnt[it] = base;
+  }
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(fin, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(&s_tmem, 256);
+    tc::tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tc::prefetch_tmap(&tmq);
+    tc::prefetch_tmap(&tmk);
+    tc::prefetch_tmap(&tmv);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int steps = max(s_cnt[0], s_cnt[1]) + 1;
+  const uint32_t tmem = s_tmem;
+  // step j of unit it: history block, filler (fully masked) or the current block (last step)
+  auto step_block = [&](int it, int j) { return j < s_cnt[it] ? s_blk[it][j] : u; };
+
+  unsigned char* sq[2] = {smem + L::kQ, smem + L::kQ + L::kTileBytes};
+  auto stage_tile = [&](int st, int which) {  // which: 0 K0, 1 V0, 2 K1, 3 V1
+    return smem + L::kStage + st * L::kStageBytes + which * L::kTileBytes;
+  };
+  unsigned char* sp[2] = {smem + L::kP, smem + L::kP + L::kPBytes};
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+      for (int it = 0; it < 2; ++it) {
+        const int y = ((bi * p.Hq + hq[it]) * p.n) + u * kTiles;
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tc::tma_load_2d(sq[it] + hf * 8192, &tmq, hf * 64, y, q_full);
+      }
+      int issued = 0;
+      for (int j = 0; j < steps; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) - 1) & 1)) {
+          s_abort = 1;
+          break;
+        }
+        issued = j + 1;
+        mbar_arrive_expect_tx(&kv_full[st], 4 * L::kTileBytes);
+        for (int it = 0; it < 2; ++it) {
+          const int y = ((bi * p.Hk + kh) * p.n) + step_block(it, j) * kTiles;
+          for (int hf = 0; hf < L::kHalves; ++hf) {
+            tc::tma_load_2d(stage_tile(st, 2 * it) + hf * 8192, &tmk, hf * 64, y, &kv_full[st]);
+            tc::tma_load_2d(stage_tile(st, 2 * it + 1) + hf * 8192, &tmv, hf * 64, y,
+                            &kv_full[st]);
+          }
+        }
+      }
+      if (s_abort) {  // loads still in flight land before the CTA leaves
+        for (int j = max(0, issued - 2); j < issued; ++j)
+          (void)mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, 1u << 16);
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(64, D, false, true);
+      auto issue_s = [&](int j) {
+        const int st = j & 1;
+        for (int it = 0; it < 2; ++it) {
+          const uint32_t d_s = tmem + (uint32_t)(st * 64) + ((uint32_t)(16 * it) << 16);
+          const unsigned char* kt = stage_tile(st, 2 * it);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int hf = kk >> 2, off = (kk & 3) * 32;
+            const uint64_t a = tc::smem_desc_sw128(sq[it] + hf * 8192 + off, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(kt + hf * 8192 + off, 16, 1024);
+            tc::mma_f16_ss(d_s, a, b, idS, kk > 0);
+          }
+        }
+        tc::mma_commit(&s_full[st]);
+      };
+      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&kv_full[0], 0);
+      if (ok) {
+        tc::fence_after_sync();
+        issue_s(0);
+      }
+      for (int j = 0; ok && j < steps; ++j) {
+        if (j + 1 < steps) {
+          const int st1 = (j + 1) & 1;
+          ok = mbar_wait_bounded(&kv_full[st1], ((j + 1) >> 1) & 1);
+          if (ok && j + 1 >= 2) ok = mbar_wait_bounded(&s_free[st1], (((j + 1) >> 1) - 1) & 1);
+          if (!ok) break;
+          tc::fence_after_sync();
+          issue_s(j + 1);
+        }
+        if (!mbar_wait_bounded(p_full, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const int st = j & 1;
+        for (int it = 0; it < 2; ++it) {
+          const uint32_t d_o = tmem + 128u + ((uint32_t)(16 * it) << 16);
+          const unsigned char* vt = stage_tile(st, 2 * it + 1);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 64 keys in steps of 16
+            const uint64_t a = tc::smem_desc_sw128(sp[it] + kk * 32, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(vt + kk * 2048, 8192, 1024);
+            tc::mma_f16_ss(d_o, a, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(o_done);
+        tc::mma_commit(&kv_empty[st]);
+      }
+      if (!ok) s_abort = 1;
+      // drain: every MMA this thread issued has completed before TMEM is released
+      tc::mma_commit(fin);
+      if (!mbar_wait_bounded(fin, 0)) s_abort = 1;
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps 0-3
+    const int it = lane >> 4;                  // unit of this thread's row
+    const int r = 16 * warp + (lane & 15);     // row within the unit
+    const int i = u * kTiles + r;              // query position
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const float qk_scale = rsqrtf((float)D) * kLog2e;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < steps && ok; ++j) {
+      const int st = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
+      if (!ok) break;
+      tc::fence_after_sync();
+      float x[64];
+      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 64), x);
+      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 64 + 32), x + 32);
+      tc::tmem_wait_ld();
+      tc::fence_before_sync();
+      mbar_arrive(&s_free[st]);
+      // bias or mask of this step's block for my unit
+      const bool is_cur = (j == steps - 1);
+      const bool filler = !is_cur && j >= s_cnt[it];
+      const float bias = (!is_cur && !filler) ? s_bias[it][j] : 0.f;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        float z = fmaf(x[c], qk_scale, bias);
+        if (filler || (is_cur && c > r)) z = -INFINITY;
+        x[c] = z;
+        mx = fmaxf(mx, z);
+      }
+      const float m_new = fmaxf(m_run, mx);
+      const bool rescale = m_run == -INFINITY ? (m_new != -INFINITY) : (m_new > m_run + kRescale);
+      float corr = 1.f;
+      if (rescale) {
+        corr = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+        m_run = m_new;
+      }
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_run);
+        const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_run);
+        sum += p0 + p1;
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      l_run = l_run * corr + sum;
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
+        if (!ok) break;
+        tc::fence_after_sync();
+        // O row *= corr; the TMEM round trip is warp-wide (.sync.aligned), lanes that keep their
+        // max multiply by 1
+        if (__any_sync(0xffffffffu, rescale)) {
+          if (!rescale) corr = 1.f;
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            float ov[32];
+            tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] *= corr;
+            tc::tmem_st32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+          }
+          tc::tmem_wait_st();
+        }
+      }
+      // P row -> shared memory, 128-byte swizzled K-major [64 x 64]
+      unsigned char* prow = sp[it];
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint4 w4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(prow + tc::sw128_offset(r, ch)) = w4;
+      }
+      fence_proxy_async();
+      tc::fence_before_sync();
+      mbar_arrive(p_full);
+    }
+    // epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (steps - 1) & 1));
+    if (ok) {
+      tc::fence_after_sync();
+      const bool live = i < p.n;
+      const size_t orow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
+      const float inv = 1.f / l_run;
+      __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow * D;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        float ov[32];
+        tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+        tc::tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint4 w4;
+            __nv_bfloat162 h;
+            h = __floats2bfloat162_rn(ov[c] * inv, ov[c + 1] * inv);
+            w4.x = *reinterpret_cast<uint32_t*>(&h);
+            h = __floats2bfloat162_rn(ov[c + 2] * inv, ov[c + 3] * inv);
+            w4.y = *reinterpret_cast<uint32_t*>(&h);
+            h = __floats2bfloat162_rn(ov[c + 4] * inv, ov[c + 5] * inv);
+            w4.z = *reinterpret_cast<uint32_t*>(&h);
+            h = __floats2bfloat162_rn(ov[c + 6] * inv, ov[c + 7] * inv);
+            w4.w = *reinterpret_cast<uint32_t*>(&h);
+            *reinterpret_cast<uint4*>(op + c0 + c) = w4;
+          }
+        }
+      }
+      if (live && p.lse) p.lse[orow] = (m_run + log2f(l_run)) * kLn2;
+    } else {
+      ok = false;
+    }
+    if (!ok) s_abort = 1;
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (s_abort && tid == 0) report_timeout(p.status, 3);
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
 }
 
-bsa_status prefill_tc(const void*, const void*, const void*, int, int, int, int, int, int,
-                      const int*, const int*, int, int, int, const float*, int, void*, float*,
-                      int*, cudaStream_t) {
-  return BSA_ERR_UNSUPPORTED;
+// ---- host side -----------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D map over a [rows, D] bf16 row-major tensor, 64x64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams& p,
+                     cudaStream_t st) {
+  CUtensorMap tmq, tmk, tmv;
+  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D) ||
+      !make_map(&tmk, k, (long long)p.B * p.Hk * p.n, D) ||
+      !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
+    return BSA_ERR_CUDA;
+  const int smem = TcSmem<D>::kTotal + 1024;  // + alignment slack
+  auto kern = prefill_tc_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  dim3 grid(p.U, p.Hq / 2, p.B);
+  kern<<<grid, kThreadsTc, smem, st>>>(tmq, tmk, tmv, p);
+  return BSA_OK;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq, int Hk) {
+  if (dt != BSA_BF16 || b != kTiles || q_block != kTiles || K > kMaxKtc) return false;
+  if (d != 64 && d != 128) return false;
+  const int G = Hq / Hk;
+  return G % 2 == 0;  // units are paired by head within one kv group
+}
+
+bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hk, int n,
+                      int d, int b, const int* idx, const int* count, int K, int gate, int norm,
+                      const float* scores, int scores_ld, void* o, float* lse, int* status,
+                      cudaStream_t st) {
+  (void)b;
+  TcParams p{};
+  p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = K;
+  p.idx = idx; p.count = count; p.gate = gate; p.norm = norm;
+  p.scores = scores; p.scores_ld = scores_ld; p.o = o; p.lse = lse; p.status = status;
+  bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
+  if (rc != BSA_OK) return rc;
+  BSA_LAUNCH_CHECK();
+  return BSA_OK;
 }
 
 }  // namespace bsa

@@ -131,6 +131,33 @@ bsa_status bsa_topk_blocks(const float* scores, int rows, int C, int ld, const i
                            void* stream);
 
 /*
+ * bsa_decode_step -- one whole decode step in a single launch: the composition of
+ * bsa_score_blocks, bsa_topk_blocks and bsa_sparse_attn_fwd (nq = 1, no gate), plus the summary
+ * append of the block holding each row's newest token ([SAS] "How it works" step 6: score the
+ * history blocks, keep Top-K and the current block, exact softmax over their tokens).
+ * Selection is per query head; the scores are those bsa_score_blocks writes (same arithmetic),
+ * the Top-K the exact order of bsa_topk_blocks.
+ *
+ *   q [B, Hq, d], k/v [B, Hk, n, d]; query of row b at seq_lens[b] - 1 (n - 1 if NULL).
+ *   mean_k, max_norm, centre: block summaries [B, Hk, C, *] of all history blocks (read); with
+ *             append != 0 the entry of each row's current block is rewritten from its keys.
+ *             max_norm / centre may be NULL unless lambda_h is given.
+ *   lambda_h, sigma_h, prefix_block: optional FreeSolo score bias and candidate rule, as in
+ *             bsa_score_blocks.
+ *   K         history blocks per head, 1..32.
+ *   o [B, Hq, d] out, lse [B, Hq] optional out, idx [B, Hq, K] optional out (ascending, -1
+ *   padded), count [B, Hq] optional out.
+ *   status    optional device int: a bounded wait that runs out writes a nonzero value there.
+ * Needs no workspace: the CTAs of one (batch, kv head) group form a thread-block cluster and
+ * exchange candidates and partial results through distributed shared memory.
+ */
+bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                           int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                           float* mean_k, float* max_norm, float* centre, int append,
+                           const float* lambda_h, const float* sigma_h, int prefix_block, int K,
+                           void* o, float* lse, int* idx, int* count, int* status, void* stream);
+
+/*
  * bsa_sparse_attn_fwd -- exact causal softmax over the gathered tokens
  * ([SAS] Eq. 2 and "How it works" step 6; [Monodratic]), optionally with the log-gate of
  * [SAS] Eq. 9.

@@ -1,0 +1,134 @@
+"""GPU parity of the fused single-launch decode step (bsa_decode_step).
+
+Checked three ways: against the fp64 oracle (selection by the near-tie rule, outputs within the
+bf16 bar of 2e-2), against the chain of separate calls on the GPU (which computes the scores with
+the same arithmetic, so the selected indices must be identical), and for the summary append.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_summaries_b200 as bsa
+from block_sparse_attention_summaries_b200 import inputs
+from oracle import bsa_oracle as orc
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(bsa_lib):
+    return bsa_lib
+
+
+def upload(case):
+    dt = torch.bfloat16 if case.bf16 else torch.float32
+    q, k, v = (torch.from_numpy(x).to(DEV, dt) for x in (case.q, case.k, case.v))
+    sl = torch.from_numpy(case.seq_lens).to(DEV)
+    return q, k, v, sl
+
+
+def oracle_check(case, idx, o, lse, rows, tol):
+    summ = {}
+    G = case.Hq // case.Hk
+    for bi, h in rows:
+        kh = h // G
+        L = int(case.seq_lens[bi])
+        if (bi, kh) not in summ:
+            summ[(bi, kh)] = orc.block_summaries(case.k[bi, kh, :L], case.b)
+        nc = orc.sas_num_candidates(L - 1, case.b)
+        s = orc.round_f32(orc.dot_scores(case.q[bi, h], summ[(bi, kh)][0], nc))
+        sets = orc.valid_selections(s, nc, case.K)
+        gsel = sorted(int(x) for x in idx[bi, h] if x >= 0)
+        assert sets is not None and gsel in sets, (bi, h, gsel)
+        ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, kh, :L], case.v[bi, kh, :L],
+                                          L - 1, case.b, gsel)
+        assert np.max(np.abs(o[bi, h] - ro)) < tol, (bi, h)
+        assert abs(lse[bi, h] - rl) < tol, (bi, h)
+
+
+@pytest.mark.parametrize("G,K,b,d,bf16", [(4, 15, 64, 128, True), (1, 3, 32, 64, True),
+                                          (8, 7, 128, 128, True), (2, 31, 16, 64, True),
+                                          (4, 5, 64, 128, False), (8, 32, 64, 64, True)])
+def test_fused_matches_chain_and_oracle(G, K, b, d, bf16):
+    Hk, n = 2, 3000
+    seq = [3000, 1025, b, 777]
+    case = inputs.decode_case(50 + G + K, B=4, Hq=Hk * G, Hk=Hk, d=d, n=n, b=b, K=K, needles=5,
+                              bf16=bf16, seq_lens=seq)
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, b, sl)
+    o1, lse1, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, b, K, seq_lens=sl, append=False)
+    o2, lse2, idx2 = bsa.decode_step(q, k, v, mean_k, b, K, seq_lens=sl, append=False)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2), "fused and separate selections differ"
+    assert (o1.float() - o2.float()).abs().max().item() < (1e-2 if bf16 else 1e-5)
+    rows = [(bi, h) for bi in range(4) for h in range(case.Hq)]
+    oracle_check(case, idx1.cpu().numpy(), o1.float().cpu().numpy(), lse1.cpu().numpy(), rows,
+                 2e-2 if bf16 else 1e-4)
+    exp_cnt = np.minimum(K, (case.seq_lens - 1) // b)
+    assert (cnt1.cpu().numpy() == exp_cnt[:, None]).all()
+
+
+def test_fused_appends_current_block_summary():
+    case = inputs.decode_case(61, B=3, Hq=8, Hk=2, d=128, n=2000, b=64, K=6, needles=3,
+                              seq_lens=[2000, 1100, 64])
+    q, k, v, sl = upload(case)
+    mean_k, mx, ce = bsa.build_block_summaries(k, 64, sl)
+    ref_m, ref_x, ref_c = mean_k.clone(), mx.clone(), ce.clone()
+    cur = (sl - 1) // 64
+    for bi in range(3):  # spoil the current block's summary; the step must restore it
+        mean_k[bi, :, cur[bi]] = 99.0
+        mx[bi, :, cur[bi]] = 99.0
+        ce[bi, :, cur[bi]] = 99.0
+    bsa.decode_step_fused(q, k, v, mean_k, 64, 6, seq_lens=sl, append=True, max_norm=mx, centre=ce)
+    torch.cuda.synchronize()
+    assert (mean_k - ref_m).abs().max().item() < 1e-5
+    assert ((mx - ref_x).abs() / ref_x.clamp_min(1e-6)).max().item() < 1e-5
+    assert torch.equal(ce, ref_c)
+
+
+def test_fused_freesolo_bias_matches_separate_scoring():
+    case = inputs.decode_case(62, B=2, Hq=8, Hk=2, d=64, n=4096, b=32, K=4, needles=4)
+    q, k, v, sl = upload(case)
+    lam = torch.linspace(0.2, 0.9, 8, device=DEV)
+    sig = torch.linspace(100, 900, 8, device=DEV)
+    mean_k, mx, ce = bsa.build_block_summaries(k, 32, sl)
+    _, _, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, 32, 4, seq_lens=sl, append=False,
+                                             max_norm=mx, centre=ce, lambda_h=lam, sigma_h=sig,
+                                             prefix_block=128)
+    s, nc = bsa.score_blocks(q, mean_k, case.n, 32, sl, mx, ce, lam, sig, 128)
+    idx2, cnt2 = bsa.topk_blocks(s, 4, n_cand=nc)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2) and torch.equal(cnt1, cnt2.view_as(cnt1))
+
+
+@pytest.mark.parametrize("wl", ["sas_gqa_decode_32k", "long_decode_512k"])
+def test_fused_full_size(wl):
+    """Full decode workloads (32K context x batch 8; 512K context): every row against the separate
+    calls, sampled rows against the oracle."""
+    w = dict(sas_gqa_decode_32k=dict(seed=2000, B=8, n=32768, K=15, needles=16,
+                                     needle_layout="random"),
+             long_decode_512k=dict(seed=3000, B=1, n=524288, K=31, needles=64,
+                                   needle_layout="stride"))[wl]
+    case = inputs.decode_case(w["seed"], B=w["B"], Hq=32, Hk=8, d=128, n=w["n"], b=64, K=w["K"],
+                              needles=w["needles"], needle_layout=w["needle_layout"])
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, 64)
+    o1, lse1, idx1, _ = bsa.decode_step_fused(q, k, v, mean_k, 64, w["K"], append=False)
+    o2, lse2, idx2 = bsa.decode_step(q, k, v, mean_k, 64, w["K"], append=False)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2)
+    assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+    rng = np.random.default_rng(7)
+    rows = sorted({(int(bi), int(h)) for bi, h in zip(rng.integers(0, w["B"], 6),
+                                                        rng.integers(0, 32, 6))} | {(0, 0)})
+    oracle_check(case, idx1.cpu().numpy(), o1.float().cpu().numpy(), lse1.cpu().numpy(), rows,
+                 2e-2)
+    # needle recall: every head of a group sees its planted blocks first
+    idx_np = idx1.cpu().numpy()
+    hits = tot = 0
+    for (bi, kh), blocks in case.needles.items():
+        sel = set(idx_np[bi, kh * 4:(kh + 1) * 4].ravel().tolist())
+        hits += len(sel & set(int(c) for c in blocks))
+        tot += len(blocks)
+    assert hits / tot > 0.9

@@ -353,3 +353,57 @@ def test_errors_on_device_tensors():
     with pytest.raises(bsa.BsaError) as e:
         bsa.build_block_summaries(k, 16)
     assert e.value.code == 4
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_bf16_tensor_core_shapes(d):
+    """bf16, 64-query units over 64-token blocks, even GQA groups: the tcgen05 kernel's shapes."""
+    B, Hq, Hk, n, b, K = 2, 8, 2, 2048 + 21, 64, 9
+    case = inputs.prefill_case(18 + d, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, q_block=64)
+    s_gpu = up(case.scores, False)
+    q, k, v = up(case.q, True), up(case.k, True), up(case.v, True)
+    idx, cnt = bsa.topk_blocks(s_gpu, K, units=case.U, q_block=64, b=b)
+    for gate in [None, "selected", "all"]:
+        o, lse = bsa.sparse_attn_fwd(q, k, v, idx, b, count=cnt, q_block=64,
+                                     gate=gate is not None, norm=gate or "selected", scores=s_gpu)
+        o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+        for bi in range(B):
+            for h in [0, 3, 4, 7]:
+                for u in [0, 1, 8, 9, 17, 31, case.U - 1]:
+                    r = orc.prefill_unit_reference(case.q, case.k, case.v, case.scores, b, 64, K,
+                                                   bi, h, u, gate)
+                    lo = u * 64
+                    m = len(r["o"])
+                    assert np.max(np.abs(o[bi, h, lo:lo + m] - r["o"])) < 2e-2, (gate, bi, h, u)
+                    assert np.max(np.abs(lse[bi, h, lo:lo + m] - r["lse"])) < 2e-2
+
+
+def test_prefill_gated_full_size_sampled():
+    """The SAS training-mode prefill workload (batch 2, 32/8 heads, d = 128, 16K context, top-16
+    blocks per 64-query unit, log-softmax gate over the selected blocks): output, lse and the
+    gate gradient on sampled units."""
+    case = inputs.prefill_case(5000)
+    s_gpu = up(case.scores, False)
+    q, k, v = up(case.q, True), up(case.k, True), up(case.v, True)
+    idx, cnt = bsa.topk_blocks(s_gpu, case.K, units=case.U, q_block=64, b=64)
+    o, lse = bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate=True,
+                                 norm="selected", scores=s_gpu)
+    dg = bsa.gate_grad(q, k, v, o, lse, up(case.dout, True), idx, 64, s_gpu, q_block=64,
+                       count=cnt, norm="selected")
+    o, lse, dg, idx = (x.float().cpu().numpy() if x.dtype != torch.int32 else x.cpu().numpy()
+                       for x in (o, lse, dg, idx))
+    rng = np.random.default_rng(11)
+    units = [(0, 0, 0), (1, 31, 255), (0, 5, 16), (1, 12, 17)] + \
+        [(int(a), int(c), int(e)) for a, c, e in zip(rng.integers(0, 2, 8),
+                                                     rng.integers(0, 32, 8),
+                                                     rng.integers(0, 256, 8))]
+    for bi, h, u in units:
+        r = orc.prefill_unit_reference(case.q, case.k, case.v, case.scores, 64, 64, case.K, bi, h,
+                                       u, "selected", case.dout)
+        lo = u * 64
+        assert list(idx[bi, h, u][:len(r["idx"])]) == r["idx"]
+        assert np.max(np.abs(o[bi, h, lo:lo + 64] - r["o"])) < 2e-2, (bi, h, u)
+        assert np.max(np.abs(lse[bi, h, lo:lo + 64] - r["lse"])) < 2e-2
+        if len(r["idx"]):
+            err = np.max(np.abs(dg[bi, h, u, :len(r["idx"])] - r["dg"]))
+            assert err <= 1e-2 * np.max(np.abs(r["dg"])), (bi, h, u, err)
