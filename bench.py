@@ -177,6 +177,101 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def time_cuda(fn, reps, stream):
+    """Average milliseconds of fn() over reps launches (CUDA events on `stream`, one warm-up)."""
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record(stream)
+        for i in range(reps):
+            fn()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
+
+
+def run_prefill(dev, peaks, reps=5):
+    """Prefill rows: SAS gated training prefill (forward on tcgen05 + gate gradient) and FreeSolo
+    two-branch prefill, each as TFLOP/s on the gathered FLOPs (4 d per attended query-key pair)."""
+    import torch
+
+    import block_sparse_attention_summaries_b200 as bsa
+    from block_sparse_attention_summaries_b200 import inputs
+
+    out = {}
+    stream = torch.cuda.Stream(dev)
+    pc = inputs.prefill_case(5000)
+    bf = lambda x: torch.from_numpy(x).to(dev, torch.bfloat16)
+    q, k, v, do = bf(pc.q), bf(pc.k), bf(pc.v), bf(pc.dout)
+    s = torch.from_numpy(pc.scores).to(dev)
+    idx, cnt = bsa.topk_blocks(s, pc.K, units=pc.U, q_block=64, b=64)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
+    dg = torch.empty(pc.B, pc.Hq, pc.U, pc.K, device=dev, dtype=torch.float32)
+    cnt_h = cnt.cpu().numpy().astype(np.int64)  # [B, Hq, U]
+    d = pc.d
+    per_unit = cnt_h * 64 * 64 + 64 * 65 // 2  # attended pairs per unit (history + causal diag)
+    fwd_flops = float(4 * d * per_unit.sum())
+    grad_flops = float(4 * d * (cnt_h * 64 * 64).sum())
+    fwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate=True,
+                                      norm="selected", scores=s, o=o, lse=lse)
+    grad = lambda: bsa.gate_grad(q, k, v, o, lse, do, idx, 64, s, q_block=64, count=cnt,
+                                 norm="selected", dg=dg)
+    t_fwd = statistics.fmean(time_cuda(fwd, reps, stream))
+    t_grad = statistics.fmean(time_cuda(grad, max(2, reps // 2), stream))
+    peak = peaks["bf16_tflops"]
+    out["sas_gated_prefill_16k"] = {
+        "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
+                   "q_block": 64, "K": pc.K, "gate": "log-softmax over the selected blocks"},
+        "forward": {"kernel": "prefill_tc_kernel (tcgen05)", "ms": t_fwd,
+                    "gathered_gflop": fwd_flops / 1e9, "tflops": fwd_flops / t_fwd / 1e9,
+                    "roofline": {"bound": "tensor", "achieved": fwd_flops / t_fwd / 1e9,
+                                 "peak": peak, "unit": "TFLOP/s",
+                                 "frac": fwd_flops / t_fwd / 1e9 / peak,
+                                 "peak_source": peaks["source"] + " bf16 (burst)"}},
+        "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
+                      "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
+                      "frac_of_bf16_peak": grad_flops / t_grad / 1e9 / peak},
+    }
+    del q, k, v, do, o, s, idx, cnt, lse, dg
+    torch.cuda.empty_cache()
+
+    fc = inputs.freesolo_case(4000)
+    q, k, v = bf(fc.q), bf(fc.k), bf(fc.v)
+    lam, sig, alpha = (torch.from_numpy(x).to(dev) for x in (fc.lam, fc.sigma, fc.alpha))
+    mk, mx, ce = bsa.build_block_summaries(k, fc.cell)
+    idx, cnt = bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K)
+    o = torch.empty_like(q)
+    ws = torch.empty(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
+                                                                  fc.d)),
+                     dtype=torch.uint8, device=dev)
+    sel = lambda: bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K,
+                                      idx=idx, count=cnt)
+    att = lambda: bsa.freesolo_attn(q, k, v, alpha, idx, cnt, fc.cell, fc.window, fc.rope_theta,
+                                    o=o, ws=ws)
+    t_sel = statistics.fmean(time_cuda(sel, 2, stream))
+    t_att = statistics.fmean(time_cuda(att, 2, stream))
+    cnt_h = cnt.cpu().numpy().astype(np.int64)
+    pos = np.arange(fc.n)
+    win = np.minimum(pos + 1, fc.window).sum() * fc.B * fc.H
+    att_flops = float(4 * fc.d * (win + (cnt_h * fc.cell).sum()))
+    ncand = ((pos // fc.q_block) * fc.q_block) // fc.cell
+    score_flops = float(2 * fc.d * ncand.sum() * fc.B * fc.H)
+    out["freesolo_prefill_64k"] = {
+        "config": {"B": fc.B, "H": fc.H, "d": fc.d, "n": fc.n, "cell": fc.cell,
+                   "q_block": fc.q_block, "K": fc.K, "window": fc.window},
+        "select": {"kernel": "freesolo_select_kernel (CUDA cores)", "ms": t_sel,
+                   "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9},
+        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode (tcgen05) + freesolo_attn_kernel long branch (CUDA cores)", "ms": t_att,
+                      "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,
+                      "frac_of_bf16_peak": att_flops / t_att / 1e9 / peak},
+        "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),
+    }
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -395,6 +490,10 @@ def run_gpu(args):
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],
     }
+    if not args.no_prefill:
+        del layers
+        torch.cuda.empty_cache()
+        line["prefill"] = run_prefill(dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         summ = oracle_summaries(case, range(case.B))
         tsec, done = 0.0, 0
@@ -422,6 +521,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -7,22 +7,32 @@
 // steps.  [FreeSolo] summary page, "How it works": optional erf distance bias of the cell score.
 //
 // B200 design.  The step is HBM-bound (summaries + selected K/V) and short (~10 us), so launch
-// boundaries and global round trips cost as much as the data.  The CL CTAs of a cluster (CL <= 16)
-// cooperate through distributed shared memory (DSMEM) instead of global scratch:
+// boundaries, global round trips and serial latency chains cost as much as the bytes.  The CL
+// CTAs of a cluster (CL <= 16) cooperate through distributed shared memory (DSMEM):
 //   1. CTA r scores its slice of the history blocks: the mean-key rows stream through a
-//      shared-memory ring filled by bulk copies (TMA engine); the G query heads of the group
-//      share every row (one 31-shuffle transpose-reduce per 32/G rows); a per-head warp radix
-//      select keeps the slice's local Top-K.
-//   2. cluster barrier; every CTA reads all CL local lists over DSMEM and selects the global Top-K
-//      per head (the same exact order everywhere: larger score, then lower index), then the
-//      sorted union of the G heads' selections plus the current block.
-//   3. CTA r attends union entries r, r+CL, ...: each K/V block is one contiguous bulk copy,
-//      double-buffered; logits for all G heads, per-head masks for blocks a head did not select;
-//      the CTA holding the current block also rewrites that block's summary from shared memory.
-//   4. cluster barrier; CTA r merges the CL partial (m, l, o) for its slice of the output columns
-//      over DSMEM and writes o (and lse).
+//      two-stage shared-memory ring filled by bulk copies (TMA engine); the G query heads of the
+//      group share every row (one 31-shuffle transpose-reduce per 32/G rows).  Per head, a warp
+//      selects the slice's local Top-K (bisection on order-preserving keys with warp reductions)
+//      and PUSHES the candidates into every peer's merge buffer with DSMEM stores.
+//   2. cluster barrier; each CTA selects the global Top-K per head from its own merge buffer
+//      (same exact order everywhere: larger score, then lower index) and builds the sorted union
+//      of the G heads' selections (a bitmap over the history blocks, compacted by one warp), plus
+//      the current block, with a head mask per entry.
+//   3. CTA r attends union entries r, r+CL, ...  bf16: each K/V block arrives as 128-byte swizzled
+//      64x64 TMA tiles; two groups of four warps take alternate entries; a warp owns 16 tokens of
+//      a block and computes S = Q K^T and O += P V with warp-level MMAs (the G heads padded to 16
+//      rows), keeping its own online-softmax state, so the per-block work is ~30 MMAs per warp
+//      instead of ~1,200 scalar FMAs/shuffles.  fp32: the same split with scalar FMAs.  The CTA
+//      holding the current block also rewrites that block's summary from shared memory.
+//   4. Each CTA merges its warps, then pushes to CTA r' the partial (m, l, o) of the output columns
+//      CTA r' owns; cluster barrier; each CTA finishes its columns and writes o (and lse).
 // Every CTA reaches every cluster barrier (no early exit); every mbarrier wait is bounded.
-#include "bsa_common.cuh"
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "tc_common.cuh"
 
 namespace bsa {
 namespace {
@@ -32,9 +42,11 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCL = 16;
 constexpr int kMaxKf = 32;        // Top-K bound of the fused path
 constexpr int kMaxUnion = 8 * kMaxKf + 1;
+constexpr int kMaxWords = 512;    // history bitmap words: C <= 16384
 constexpr int kSub = 64;          // summary rows per ring stage
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.f;   // lazy rescale threshold (log2 units)
 
 struct FusedParams {
   const void* q;
@@ -55,7 +67,6 @@ struct FusedParams {
   int* count;
   int* status;
   int chunk;  // history blocks scored per CTA (multiple of kSub)
-  int ns;     // ring stages
 };
 
 // ---- cluster helpers ---------------------------------------------------------------------
@@ -74,21 +85,16 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }
-// Address of `p` (this CTA's shared memory) in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
   uint32_t out;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
   return out;
 }
-__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
+__device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -98,11 +104,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Top-K of N keys held in shared memory, by one warp: exact radix select of the K-th largest key
-// (8-bit digits, the warp's own 256-bin histogram), then one ordered pass that takes every key
-// above it and the lowest-indexed keys equal to it.  Writes the positions of the selected keys in
-// ascending order to `out` and returns their number min(K, N).
-__device__ int warp_topk(const uint32_t* keys, int N, int K, uint32_t* hist, int lane, int* out) {
+// Top-K of N order keys (shared memory, index order) by one warp.  Bisection finds the largest T
+// with count(key >= T) >= K (32 steps of a warp-wide count), then one ordered pass takes every key
+// above T and the lowest-indexed keys equal to T.  Writes the selected positions ascending to
+// `out`; returns min(K, N).  N <= 32 * kSelItems.
+constexpr int kSelItems = 16;
+__device__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
   if (kk == N) {
@@ -110,59 +117,40 @@ __device__ int warp_topk(const uint32_t* keys, int N, int K, uint32_t* hist, int
     __syncwarp();
     return N;
   }
-  uint32_t prefix = 0, mask = 0;
-  int rem = kk;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  uint32_t r[kSelItems];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
-    __syncwarp();
-    for (int i = lane; i < N; i += 32) {
-      const uint32_t x = keys[i];
-      if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    uint32_t hb[8], local = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      hb[j] = hist[lane * 8 + j];
-      local += hb[j];
-    }
-    uint32_t incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-      if (lane + o < 32) incl += y;
-    }
-    uint32_t running = incl - local;
-    int digit = -1, above = 0;
-#pragma unroll
-    for (int j = 7; j >= 0; --j) {
-      if (running < (uint32_t)rem && running + hb[j] >= (uint32_t)rem) {
-        digit = lane * 8 + j;
-        above = (int)running;
-      }
-      running += hb[j];
-    }
-    const unsigned who = __ballot_sync(0xffffffffu, digit >= 0);
-    const int src = __ffs(who) - 1;
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    above = __shfl_sync(0xffffffffu, above, src);
-    prefix |= (uint32_t)digit << shift;
-    mask |= 255u << shift;
-    rem -= above;
-    __syncwarp();
+  for (int e = 0; e < kSelItems; ++e) {
+    const int i = lane + 32 * e;
+    r[e] = i < N ? keys[i] : 0u;
   }
-  const uint32_t T = prefix;
+  const int items = (N + 31) / 32;
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < kSelItems; ++e)
+      if (e < items && lane + 32 * e < N) c += (r[e] >= cand);
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= kk) T = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int e = 0; e < kSelItems; ++e)
+    if (e < items && lane + 32 * e < N) gt += (r[e] > T);
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  const int rem = kk - gt;
   int taken = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < N; base += 32) {
-    const int i = base + lane;
-    const uint32_t x = i < N ? keys[i] : 0u;
+#pragma unroll
+  for (int e = 0; e < kSelItems; ++e) {
+    if (e >= items) break;
+    const int i = lane + 32 * e;
     const bool valid = i < N;
-    const bool gt = valid && x > T;
-    const bool eq = valid && x == T;
+    const bool gtb = valid && r[e] > T;
+    const bool eq = valid && r[e] == T;
     const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < rem);
+    const bool take = gtb || (eq && eq_seen + __popc(eqb & lt) < rem);
     const unsigned tb = __ballot_sync(0xffffffffu, take);
     if (take) out[taken + __popc(tb & lt)] = i;
     taken += __popc(tb);
@@ -172,50 +160,74 @@ __device__ int warp_topk(const uint32_t* keys, int N, int K, uint32_t* hist, int
   return taken;
 }
 
-template <typename T, int D, int G>
+// ---- warp MMA (legacy mma.sync, bf16 in, fp32 accumulate) ---------------------------------
+__device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Shared-memory layout (dynamic part).  MMA: the bf16 warp-MMA path over 64-token blocks.
+template <typename T, int D, int G, bool MMA>
 struct FusedSmem {
-  // region A: summary ring (ns x kSub x D floats) / K,V stages (2 x 2 x b x D x T) / partials
-  __host__ __device__ static size_t tile(int b) { return align_up((size_t)b * D * sizeof(T), 128); }
-  __host__ __device__ static size_t region_a(int b, int ns) {
-    size_t x = (size_t)ns * kSub * D * sizeof(float);
+  // region A: summary ring (2 x kSub x D fp32) / K,V stages (2 x {K,V} tile) / warp partials
+  __host__ __device__ static size_t tile(int b) {
+    return align_up((size_t)(MMA ? 64 : b) * D * sizeof(T), 1024);
+  }
+  __host__ __device__ static size_t region_a(int b) {
+    size_t x = (size_t)2 * kSub * D * sizeof(float);
     x = max_sz(x, 4 * tile(b));
-    x = max_sz(x, (size_t)G * kMaxCL * kMaxKf * 8);                  // merge buffers
-    x = max_sz(x, (size_t)(kThreads / (D / 2) + 1) * G * D * 4);     // split reduction, partials
+    x = max_sz(x, (size_t)kWarps * G * (D + 2) * 4 + 4096);  // warp partials
     return align_up(x, 1024);
   }
   __host__ __device__ static size_t scores(int chunk) { return align_up((size_t)G * chunk * 4, 16); }
-  __host__ __device__ static size_t bytes(int b, int ns, int chunk) {
-    return region_a(b, ns) + scores(chunk) + 2 * align_up((size_t)b * G * 4, 16) + 1024;
+  __host__ __device__ static size_t merge(int CL, int K) { return align_up((size_t)G * CL * K * 8, 16); }
+  __host__ __device__ static size_t recv(int CL) {
+    return align_up((size_t)CL * G * (D / CL + 2) * 4, 16);
+  }
+  __host__ __device__ static size_t zp(int b) { return 2 * align_up((size_t)b * G * 4, 16); }
+  __host__ __device__ static size_t bytes(int b, int chunk, int CL, int K) {
+    return region_a(b) + scores(chunk) + merge(CL, K) + recv(CL) + zp(b) + 256 + 1024;
   }
 };
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParams p) {
+template <typename T, int D, int G, bool MMA>
+__global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
+    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+    const FusedParams p) {
+  constexpr bool kMma = MMA;
+  static_assert(!MMA || std::is_same<T, __nv_bfloat16>::value, "warp MMAs take bf16");
   constexpr int EPL = D / 32;
   constexpr int R = 32 / G;
-  constexpr int CG = D / 2;
-  constexpr int TP = kThreads / CG;
 
-  extern __shared__ __align__(1024) unsigned char smem[];
-  // static shared state
-  __shared__ uint32_t s_hist[kWarps][256];
-  __shared__ uint32_t s_ckey[G][kMaxKf];   // local Top-K keys (read by the cluster)
-  __shared__ int s_cidx[G][kMaxKf];        // and their global block indices
-  __shared__ int s_ccnt[G];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ int s_pick[G][kMaxKf];
   __shared__ int s_sel[G][kMaxKf];
   __shared__ int s_nsel[G];
-  __shared__ int s_list[kMaxUnion];
-  __shared__ unsigned char s_first[kMaxUnion];
+  __shared__ uint32_t s_bits[kMaxWords];
   __shared__ int s_ublk[kMaxUnion];
   __shared__ unsigned s_umask[kMaxUnion];
   __shared__ int s_U;
-  __shared__ float s_m[G], s_l[G], s_corr[G];
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
+  __shared__ float s_m[G], s_l[G], s_corr[G];
 
-  const int b = p.b, K = p.K, Hq = p.Hq, D2 = D;
-  (void)D2;
+  const int b = p.b, K = p.K, Hq = p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = (int)cluster_rank();
   const int CL = (int)cluster_size();
@@ -227,17 +239,21 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
   int nc = p.prefix_block > 0 ? ((pos / p.prefix_block) * p.prefix_block) / b : cur;
   nc = max(0, min(nc, cur));
 
-  const size_t ra = FusedSmem<T, D, G>::region_a(b, p.ns);
+  using SM = FusedSmem<T, D, G, MMA>;
   float* ring = reinterpret_cast<float*>(smem);
-  float* s_sc = reinterpret_cast<float*>(smem + ra);  // [G][chunk]
-  float* zs = reinterpret_cast<float*>(smem + ra + FusedSmem<T, D, G>::scores(p.chunk));
+  unsigned char* after_a = smem + SM::region_a(b);
+  uint32_t* s_keys = reinterpret_cast<uint32_t*>(after_a);                  // [G][chunk]
+  unsigned char* merge = after_a + SM::scores(p.chunk);                        // [G][CL*K] x 2
+  uint32_t* m_key = reinterpret_cast<uint32_t*>(merge);
+  int* m_idx = reinterpret_cast<int*>(merge) + G * CL * K;
+  float* recv = reinterpret_cast<float*>(merge + SM::merge(CL, K));          // [CL][G][cols+2]
+  float* zs = reinterpret_cast<float*>(merge + SM::merge(CL, K) + SM::recv(CL));
   float* ps = zs + align_up((size_t)b * G, 4);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + FusedSmem<T, D, G>::bytes(b, p.ns, p.chunk) -
-                                              1024);
-  // bar[0 .. ns): summary ring; bar[ns], bar[ns+1]: K/V stages
+  uint64_t* bar = reinterpret_cast<uint64_t*>(merge + SM::merge(CL, K) + SM::recv(CL) + SM::zp(b));
+  // bar[0], bar[1]: summary ring; bar[2], bar[3]: K/V stages
 
   if (tid == 0) {
-    for (int i = 0; i < p.ns + 2; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     s_abort = 0;
     s_U = 0;
@@ -248,7 +264,7 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
   }
   __syncthreads();
 
-  // query slices (pre-scaled by 1/sqrt(d) for scoring)
+  // ---- 1. score my slice of the history blocks --------------------------------------------
   float qv[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -258,8 +274,6 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
   }
-
-  // ---- 1. score my slice of the history blocks --------------------------------------------
   const int c_lo = min(nc, rank * p.chunk);
   const int c_hi = min(nc, c_lo + p.chunk);
   const int rows = c_hi - c_lo;
@@ -268,25 +282,23 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
   auto issue_sub = [&](int j) {
     const int r0 = c_lo + j * kSub;
     const int nr = min(kSub, c_hi - r0);
-    const int st = j % p.ns;
     const uint32_t bytes = (uint32_t)(nr * D * sizeof(float));
-    mbar_arrive_expect_tx(&bar[st], bytes);
-    bulk_g2s(ring + (size_t)st * kSub * D, mk + (size_t)r0 * D, bytes, &bar[st]);
+    mbar_arrive_expect_tx(&bar[j & 1], bytes);
+    bulk_g2s(ring + (size_t)(j & 1) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j & 1]);
   };
   if (tid == 0)
-    for (int j = 0; j < min(nsub, p.ns); ++j) issue_sub(j);
+    for (int j = 0; j < min(nsub, 2); ++j) issue_sub(j);
   const float scale = rsqrtf((float)D);
   const int my_r = lane / G, my_g = lane % G;
   const float lam_h = p.lam ? p.lam[h0 + my_g] : 0.f;
   const float inv2sig = p.lam ? 0.5f / p.sig[h0 + my_g] : 0.f;
   for (int j = 0; j < nsub; ++j) {
-    const int st = j % p.ns;
-    if (!s_abort && !mbar_wait_bounded(&bar[st], (j / p.ns) & 1)) s_abort = 1;
+    if (!s_abort && !mbar_wait_bounded(&bar[j & 1], (j >> 1) & 1)) s_abort = 1;
     __syncthreads();
     if (!s_abort) {
       const int r0 = j * kSub;
       const int nr = min(kSub, rows - r0);
-      const float* base = ring + (size_t)st * kSub * D;
+      const float* base = ring + (size_t)(j & 1) * kSub * D;
       for (int t0 = warp * R; t0 < nr; t0 += kWarps * R) {
         float a[32];
 #pragma unroll
@@ -314,45 +326,53 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
             const size_t row = (size_t)(bi * p.Hk + kh) * p.C + c_lo + r0 + t;
             s += lam_h * p.max_norm[row] * erff(((float)pos - p.centre[row]) * inv2sig);
           }
-          reinterpret_cast<uint32_t*>(s_sc)[my_g * p.chunk + r0 + t] = order_key(s);
+          s_keys[my_g * p.chunk + r0 + t] = order_key(s);
         }
       }
     }
     __syncthreads();
-    if (tid == 0 && j + p.ns < nsub && !s_abort) issue_sub(j + p.ns);
+    if (tid == 0 && j + 2 < nsub && !s_abort) issue_sub(j + 2);
   }
-  // local Top-K per head (warp g)
+  // local Top-K per head, pushed into every CTA's merge buffer at slot rank*K
   for (int g = warp; g < G; g += kWarps) {
-    const uint32_t* keys = reinterpret_cast<const uint32_t*>(s_sc) + g * p.chunk;
-    const int cnt = warp_topk(keys, rows, K, s_hist[warp], lane, s_pick[g]);
-    for (int j = lane; j < cnt; j += 32) {
-      const int i = s_pick[g][j];
-      s_ckey[g][j] = keys[i];
-      s_cidx[g][j] = c_lo + i;
+    const uint32_t* keys = s_keys + g * p.chunk;
+    const int cnt = warp_select(keys, rows, K, lane, s_pick[g]);
+    for (int e = lane; e < CL * K; e += 32) {
+      const int r = e / K, j = e % K;
+      const uint32_t key = j < cnt ? keys[s_pick[g][j]] : 0u;
+      const int gi = j < cnt ? c_lo + s_pick[g][j] : -1;  // -1: empty slot
+      const int slot = g * CL * K + rank * K + j;
+      st_dsmem_u32(dsmem_addr(&m_key[slot], r), key);
+      st_dsmem_u32(dsmem_addr(&m_idx[slot], r), (uint32_t)gi);
     }
-    if (lane == 0) s_ccnt[g] = cnt;
   }
   cluster_sync();
 
-  // ---- 2. global Top-K per head over all CTAs' lists, then the union ----------------------
-  // merge buffers [G][CL*K] keys and block indices, in region A (the ring is idle now)
-  uint32_t* mkey_all = reinterpret_cast<uint32_t*>(smem);
-  int* midx_all = reinterpret_cast<int*>(smem) + G * kMaxCL * kMaxKf;
+  // ---- 2. global Top-K per head, then the union -------------------------------------------
+  const int nwords = (nc + 31) / 32;
+  for (int w = tid; w < nwords; w += kThreads) s_bits[w] = 0u;
   for (int g = warp; g < G; g += kWarps) {
-    uint32_t* s_mkey_g = mkey_all + g * kMaxCL * kMaxKf;
-    int* s_midx_g = midx_all + g * kMaxCL * kMaxKf;
-    int tot = 0;
-    for (int r = 0; r < CL; ++r) {
-      const int cnt = (int)ld_dsmem_u32(dsmem_addr(&s_ccnt[g], r));
-      for (int j = lane; j < cnt; j += 32) {
-        s_mkey_g[tot + j] = ld_dsmem_u32(dsmem_addr(&s_ckey[g][j], r));
-        s_midx_g[tot + j] = (int)ld_dsmem_u32(dsmem_addr(&s_cidx[g][j], r));
+    // empty slots carry key 0 and index -1: compact the valid ones first (index order kept)
+    uint32_t* mk_g = m_key + g * CL * K;
+    int* mi_g = m_idx + g * CL * K;
+    int nvalid = 0;
+    for (int e0 = 0; e0 < CL * K; e0 += 32) {
+      const int e = e0 + lane;
+      const bool ok = e < CL * K && mi_g[e] >= 0;
+      const uint32_t kk2 = ok ? mk_g[e] : 0u;
+      const int ii = ok ? mi_g[e] : 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, ok);
+      __syncwarp();
+      if (ok) {
+        const int at = nvalid + __popc(bal & ((1u << lane) - 1u));
+        mk_g[at] = kk2;
+        mi_g[at] = ii;
       }
-      tot += cnt;
+      nvalid += __popc(bal);
+      __syncwarp();
     }
-    __syncwarp();
-    const int cnt = warp_topk(s_mkey_g, tot, K, s_hist[warp], lane, s_pick[g]);
-    for (int j = lane; j < cnt; j += 32) s_sel[g][j] = s_midx_g[s_pick[g][j]];
+    const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[g]);
+    for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[g][j]];
     if (lane == 0) s_nsel[g] = cnt;
   }
   __syncthreads();
@@ -364,249 +384,545 @@ __global__ void __launch_bounds__(kThreads) decode_fused_kernel(const FusedParam
       if (p.count && j == 0) p.count[row] = s_nsel[g];
     }
   }
-  const int nlist = G * K + 1;
-  for (int t = tid; t < nlist; t += kThreads) {
-    int x = INT_MAX;
-    if (t == nlist - 1) {
-      x = cur;
-    } else {
-      const int g = t / K, j = t % K;
-      if (j < s_nsel[g]) x = s_sel[g][j];
+  for (int e = tid; e < G * K; e += kThreads) {
+    const int g = e / K, j = e % K;
+    if (j < s_nsel[g]) {
+      const int x = s_sel[g][j];
+      atomicOr(&s_bits[x >> 5], 1u << (x & 31));
     }
-    s_list[t] = x;
-    s_umask[t] = 0u;
   }
+  for (int e = tid; e < kMaxUnion; e += kThreads) s_umask[e] = 0u;
   __syncthreads();
-  {
-    int nf = 0;
-    for (int t = tid; t < nlist; t += kThreads) {
-      const int x = s_list[t];
-      bool first = x != INT_MAX;
-      for (int u = 0; u < t && first; ++u) first = s_list[u] != x;
-      s_first[t] = first;
-      nf += first;
+  if (warp == 0) {  // compact the bitmap into the sorted union
+    const int per = (nwords + 31) / 32;
+    int mine = 0;
+    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) mine += __popc(s_bits[w]);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    nf = __reduce_add_sync(0xffffffffu, nf);
-    if (lane == 0 && nf) atomicAdd(&s_U, nf);
-  }
-  __syncthreads();
-  for (int t = tid; t < nlist; t += kThreads) {
-    const int x = s_list[t];
-    if (x == INT_MAX) continue;
-    int rk = 0;
-    for (int u = 0; u < nlist; ++u) rk += (s_first[u] && s_list[u] < x);
-    if (s_first[t]) s_ublk[rk] = x;
-    atomicOr(&s_umask[rk], (t == nlist - 1) ? ((1u << G) - 1u) : (1u << (t / K)));
+    int at = incl - mine;
+    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) {
+      uint32_t bits = s_bits[w];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        s_ublk[at++] = w * 32 + bit;
+      }
+    }
+    if (lane == 31) {
+      s_ublk[incl] = cur;  // the current block, always kept, follows every history block
+      s_umask[incl] = (1u << G) - 1u;
+      s_U = incl + 1;
+    }
   }
   __syncthreads();
   const int U = s_U;
+  for (int e = tid; e < G * K; e += kThreads) {  // head masks by binary search in the union
+    const int g = e / K, j = e % K;
+    if (j < s_nsel[g]) {
+      const int x = s_sel[g][j];
+      int lo = 0, hi = U - 2;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (s_ublk[mid] < x) lo = mid + 1; else hi = mid;
+      }
+      atomicOr(&s_umask[lo], 1u << g);
+    }
+  }
+  __syncthreads();
 
   // ---- 3. attend my union entries -----------------------------------------------------------
-  const size_t tl = FusedSmem<T, D, G>::tile(b);
-  T* kbuf[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem + tl)};
-  T* vbuf[2] = {reinterpret_cast<T*>(smem + 2 * tl), reinterpret_cast<T*>(smem + 3 * tl)};
-  uint64_t* kvbar = bar + p.ns;
-  const T* kbase = static_cast<const T*>(p.k) + (size_t)(bi * p.Hk + kh) * p.n * D;
-  const T* vbase = static_cast<const T*>(p.v) + (size_t)(bi * p.Hk + kh) * p.n * D;
   const int ne = rank < U ? (U - rank + CL - 1) / CL : 0;
-  auto block_tokens = [&](int m) { return m == cur ? pos - cur * b + 1 : b; };
-  auto issue_kv = [&](int i) {
-    const int m = s_ublk[rank + i * CL];
-    const uint32_t bytes = (uint32_t)(block_tokens(m) * D * sizeof(T));
-    const int st = i & 1;
-    mbar_arrive_expect_tx(&kvbar[st], 2 * bytes);
-    bulk_g2s(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st]);
-    bulk_g2s(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st]);
-  };
-  if (tid == 0 && !s_abort) {
-    fence_proxy_async();  // ring reads of phase 1 precede the async writes into region A
-    if (ne > 0) issue_kv(0);
-    if (ne > 1) issue_kv(1);
-  }
-  const float qs2 = kLog2e;  // qv already carries nothing but raw q; logits in log2 units
-  float qa[G][EPL];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) qa[g][e] = qv[g][e] * scale * qs2;
-  const int cg = tid % CG, tp = tid / CG;
-  float acc[G][2];
-#pragma unroll
-  for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
+  auto entry_tokens = [&](int m) { return m == cur ? pos - cur * b + 1 : b; };
+  float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 3: [warp][G][D+2]
 
-  for (int i = 0; i < ne; ++i) {
-    const int st = i & 1;
-    const int m = s_ublk[rank + i * CL];
-    const unsigned hm = s_umask[rank + i * CL];
-    const int tok = block_tokens(m);
-    if (!s_abort && !mbar_wait_bounded(&kvbar[st], (i >> 1) & 1)) s_abort = 1;
-    __syncthreads();
-    if (s_abort) break;
-    const T* kt = kbuf[st];
-    const T* vt = vbuf[st];
-    for (int t0 = warp * R; t0 < tok; t0 += kWarps * R) {
-      float a[32];
+  if constexpr (kMma) {
+    // two groups of four warps take alternate entries; stage st = entry & 1 holds K then V
+    const int grp = warp >> 2, wg = warp & 3;
+    const size_t tl = SM::tile(b);
+    auto ktile = [&](int st) { return smem + (size_t)st * 2 * tl; };
+    auto vtile = [&](int st) { return smem + (size_t)st * 2 * tl + tl; };
+    uint64_t* kvbar = bar + 2;
+    const int row0 = (bi * p.Hk + kh) * p.n;
+    auto issue_kv = [&](int i) {
+      const int m = s_ublk[rank + i * CL];
+      const int st = i & 1;
+      mbar_arrive_expect_tx(&kvbar[st], 2 * 64 * D * 2);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float x[EPL];
-        if (t0 + r < tok) {
-          load_vec<T, EPL>(kt + (size_t)(t0 + r) * D + lane * EPL, x);
-        } else {
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tc::tma_load_2d(ktile(st) + hf * 8192, &tmk, hf * 64, row0 + m * b, &kvbar[st]);
+        tc::tma_load_2d(vtile(st) + hf * 8192, &tmv, hf * 64, row0 + m * b, &kvbar[st]);
+      }
+    };
+    if (tid == 0 && !s_abort) {
+      fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
+      if (ne > 0) issue_kv(0);
+      if (ne > 1) issue_kv(1);
+    }
+    // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
+    const int grow = lane >> 2, tig = lane & 3;
+    uint32_t qa0[D / 16], qa1[D / 16];
+    {
+      const float qs = scale * kLog2e;
+      const T* qrow = static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + min(grow, G - 1)) * D;
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+      for (int ks = 0; ks < D / 16; ++ks) {
+        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+        if (grow < G) {
+          x0 = Elem<T>::to_f(qrow[16 * ks + 2 * tig]) * qs;
+          x1 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 1]) * qs;
+          x2 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 8]) * qs;
+          x3 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 9]) * qs;
         }
+        qa0[ks] = pack_bf16(x0, x1);
+        qa1[ks] = pack_bf16(x2, x3);
+      }
+    }
+    // O^T accumulators: m-tile mt covers d rows 16 mt .. 16 mt + 15, columns are heads
+    float oacc[D / 16][4];
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
+    float m_run = -INFINITY, l_part = 0.f;
+    for (int i = grp; i < ne; i += 2) {
+      const int st = i & 1;
+      const int m = s_ublk[rank + i * CL];
+      const unsigned hm = s_umask[rank + i * CL];
+      const int tok = entry_tokens(m);
+      // group-uniform decision: the OR over the group's four warps of "my wait ran out"
+      const int bad = mbar_wait_bounded(&kvbar[st], (i >> 1) & 1) ? 0 : 1;
+      int any_bad;
+      asm volatile(
+          "{\n\t.reg .pred pin, pout;\n\t"
+          "setp.ne.s32 pin, %1, 0;\n\t"
+          "barrier.red.or.pred pout, %2, 128, pin;\n\t"
+          "selp.s32 %0, 1, 0, pout;\n\t}"
+          : "=r"(any_bad)
+          : "r"(bad), "r"(1 + grp)
+          : "memory");
+      if (any_bad) {
+        s_abort = 1;
+        break;
+      }
+      const unsigned char* kt = ktile(st);
+      const unsigned char* vt = vtile(st);
+      const int t0 = wg * 16;  // this warp's 16 tokens
+      // S = Q K^T over two 8-token tiles
+      float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int hf = ks >> 2, ch = (ks & 3) * 2;
+          const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
+          const uint32_t b0 =
+              *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
+          const uint32_t b1 =
+              *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
+          mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+        }
+      }
+      // masks, per-row online softmax (row = head grow; the quad shares the row)
+      const bool head_on = grow < G && ((hm >> grow) & 1u);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = t0 + 8 * nt + 2 * tig + e;
+          if (!head_on || t >= tok) sfr[nt][e] = -INFINITY;
+          mx = fmaxf(mx, sfr[nt][e]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
+      if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
+        corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
+        m_run = mx;
+        l_part *= corr;
+      }
+      // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
+      const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
+      const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
+      if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          oacc[c][0] *= corr_a;
+          oacc[c][1] *= corr_b;
+          oacc[c][2] *= corr_a;
+          oacc[c][3] *= corr_b;
+        }
+      }
+      float pv[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float z = sfr[nt][e];
+          pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
+          l_part += pv[nt][e];
+        }
+      // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
+      const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
+      const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+      // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int tokr = t0 + (mi >> 1) * 8 + rr;
+        const int chunk = 2 * mt + (mi & 1);  // 16-byte chunk along d (0..D/8-1)
+        const int hf = chunk >> 3, cin = chunk & 7;
+        const uint32_t addr =
+            smem_u32(vt + hf * 8192 + tokr * 128 + ((cin ^ (tokr & 7)) << 4));
+        uint32_t v0, v1, v2, v3;
+        ldsm_x4_trans(addr, v0, v1, v2, v3);
+        mma_16816(oacc[mt], v0, v1, v2, v3, pb0, pb1);
+      }
+      // the block being filled: rewrite its summary from the swizzled K tile
+      if (p.append && m == cur) {  // taken by the whole group that holds the current block
+        const int gt = tid & 127;
+        const int col = gt;  // one column per thread (D <= 128)
+        if (col < D) {
+          float sum = 0.f;
+          const int hf = col >> 6, cin = (col & 63) >> 3, e8 = col & 7;
+          for (int t = 0; t < tok; ++t)
+            sum += Elem<T>::to_f(*reinterpret_cast<const T*>(
+                kt + hf * 8192 + t * 128 + ((cin ^ (t & 7)) << 4) + e8 * 2));
+          p.mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = sum / (float)tok;
+        }
+        // max key norm: thread t < tok takes token t
+        float nrm = 0.f;
+        if (gt < tok) {
+          float sq = 0.f;
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const int hf = c8 >> 3, cin = c8 & 7;
+            float xx[8];
+            load_vec<T, 8>(reinterpret_cast<const T*>(kt + hf * 8192 + gt * 128 +
+                                                      ((cin ^ (gt & 7)) << 4)),
+                           xx);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sq = fmaf(xx[e], xx[e], sq);
+          }
+          nrm = sqrtf(sq);
+        }
+        nrm = warp_max(nrm);
+        if (lane == 0) s_red[4 * grp + wg] = nrm;
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));
+        if (gt == 0) {
+          const float* rr = s_red + 4 * grp;
+          float nm = fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3]));
+          const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+          if (p.max_norm) p.max_norm[row] = nm;
+          if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
+        }
+      }
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
+      if (wg == 0 && lane == 0 && i + 2 < ne) issue_kv(i + 2);
+    }
+    if (s_abort && tid == 0) {
+      for (int i = 0; i < 2; ++i) (void)mbar_wait_bounded(&kvbar[i], 0, 1u << 12);
+      report_timeout(p.status, 2);
+    }
+    __syncthreads();
+    // warp partials (rows < G): m, l and o
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    if (grow < G && tig == 0) {
+      float* wp = wpart + ((size_t)warp * G + grow) * (D + 2);
+      wp[D] = m_run;
+      wp[D + 1] = l_part;
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {  // O^T element (d, head 2 tig + e)
+      const int hh = 2 * tig + e;
+      if (hh < G) {
+        float* wp = wpart + ((size_t)warp * G + hh) * (D + 2);
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          wp[16 * mt + grow] = oacc[mt][e];
+          wp[16 * mt + grow + 8] = oacc[mt][2 + e];
+        }
+      }
+    }
+    __syncthreads();
+  } else {
+    // fp32: scalar FMAs; warps split each block's tokens, one CTA-wide softmax per block
+    const size_t tl = SM::tile(b);
+    T* kbuf[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem + 2 * tl)};
+    T* vbuf[2] = {reinterpret_cast<T*>(smem + tl), reinterpret_cast<T*>(smem + 3 * tl)};
+    uint64_t* kvbar = bar + 2;
+    const T* kbase = static_cast<const T*>(p.k) + (size_t)(bi * p.Hk + kh) * p.n * D;
+    const T* vbase = static_cast<const T*>(p.v) + (size_t)(bi * p.Hk + kh) * p.n * D;
+    auto issue_kv = [&](int i) {
+      const int m = s_ublk[rank + i * CL];
+      const uint32_t bytes = (uint32_t)(entry_tokens(m) * D * sizeof(T));
+      const int st = i & 1;
+      mbar_arrive_expect_tx(&kvbar[st], 2 * bytes);
+      bulk_g2s(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st]);
+      bulk_g2s(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st]);
+    };
+    if (tid == 0 && !s_abort) {
+      fence_proxy_async();
+      if (ne > 0) issue_kv(0);
+      if (ne > 1) issue_kv(1);
+    }
+    constexpr int CG = D / 2;
+    constexpr int TP = kThreads / CG;
+    float qa[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) qa[g][e] = qv[g][e] * scale * kLog2e;
+    const int cg = tid % CG, tp = tid / CG;
+    float acc[G][2];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
+    for (int i = 0; i < ne; ++i) {
+      const int st = i & 1;
+      const int m = s_ublk[rank + i * CL];
+      const unsigned hm = s_umask[rank + i * CL];
+      const int tok = entry_tokens(m);
+      if (!s_abort && !mbar_wait_bounded(&kvbar[st], (i >> 1) & 1)) s_abort = 1;
+      __syncthreads();
+      if (s_abort) break;
+      const T* kt = kbuf[st];
+      const T* vt = vbuf[st];
+      for (int t0 = warp * R; t0 < tok; t0 += kWarps * R) {
+        float a[32];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float x[EPL];
+          if (t0 + r < tok) {
+            load_vec<T, EPL>(kt + (size_t)(t0 + r) * D + lane * EPL, x);
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float sacc = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) sacc = fmaf(qa[g][e], x[e], sacc);
+            a[r * G + g] = sacc;
+          }
+        }
+        warp_transpose_reduce32(a, lane);
+        const int t = t0 + lane / G, g = lane % G;
+        if (t < tok) zs[t * G + g] = ((hm >> g) & 1u) ? a[0] : -INFINITY;
+      }
+      if (p.append && m == cur) {
+        for (int col = tid; col < D; col += kThreads) {
+          float sum = 0.f;
+          for (int t = 0; t < tok; ++t) sum += Elem<T>::to_f(kt[(size_t)t * D + col]);
+          p.mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = sum / (float)tok;
+        }
+        float nmax = 0.f;
+        for (int t = warp; t < tok; t += kWarps) {
+          float x[EPL];
+          load_vec<T, EPL>(kt + (size_t)t * D + lane * EPL, x);
+          float sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) sq = fmaf(x[e], x[e], sq);
+          nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
+        }
+        if (lane == 0) s_red[warp] = nmax;
+      }
+      __syncthreads();
+      if (p.append && m == cur && tid == 0) {
+        float nm = 0.f;
+        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
+        const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+        if (p.max_norm) p.max_norm[row] = nm;
+        if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
+      }
+      for (int g = warp; g < G; g += kWarps) {
+        float mx = -INFINITY;
+        for (int t = lane; t < tok; t += 32) mx = fmaxf(mx, zs[t * G + g]);
+        mx = warp_max(mx);
+        const float m_old = s_m[g];
+        const float m_new = fmaxf(m_old, mx);
+        float sum = 0.f;
+        for (int t = lane; t < tok; t += 32) {
+          const float pvv = (m_new == -INFINITY) ? 0.f : exp2f(zs[t * G + g] - m_new);
+          ps[t * G + g] = pvv;
+          sum += pvv;
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) {
+          const float corr = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
+          s_corr[g] = corr;
+          s_l[g] = s_l[g] * corr + sum;
+          s_m[g] = m_new;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        acc[g][0] *= s_corr[g];
+        acc[g][1] *= s_corr[g];
+      }
+      for (int t = tp; t < tok; t += TP) {
+        float vv[2];
+        load_vec<T, 2>(vt + (size_t)t * D + 2 * cg, vv);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          float sacc = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) sacc = fmaf(qa[g][e], x[e], sacc);
-          a[r * G + g] = sacc;
+          const float pw = ps[t * G + g];
+          acc[g][0] = fmaf(pw, vv[0], acc[g][0]);
+          acc[g][1] = fmaf(pw, vv[1], acc[g][1]);
         }
       }
-      warp_transpose_reduce32(a, lane);
-      const int t = t0 + lane / G, g = lane % G;
-      if (t < tok) zs[t * G + g] = ((hm >> g) & 1u) ? a[0] : -INFINITY;
+      __syncthreads();
+      if (tid == 0 && i + 2 < ne) issue_kv(i + 2);
     }
-    // the block being filled: rewrite its summary from the tile already in shared memory
-    if (p.append && m == cur) {
-      for (int col = tid; col < D; col += kThreads) {
-        float sum = 0.f;
-        for (int t = 0; t < tok; ++t) sum += Elem<T>::to_f(kt[(size_t)t * D + col]);
-        p.mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = sum / (float)tok;
-      }
-      float nmax = 0.f;
-      for (int t = warp; t < tok; t += kWarps) {
-        float x[EPL];
-        load_vec<T, EPL>(kt + (size_t)t * D + lane * EPL, x);
-        float sq = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) sq = fmaf(x[e], x[e], sq);
-        nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
-      }
-      if (lane == 0) s_red[warp] = nmax;
+    if (s_abort && tid == 0) {
+      for (int i = 0; i < 2; ++i) (void)mbar_wait_bounded(&kvbar[i], 0, 1u << 12);
+      report_timeout(p.status, 2);
     }
     __syncthreads();
-    if (p.append && m == cur && tid == 0) {
-      float nm = 0.f;
-      for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
-      const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
-      if (p.max_norm) p.max_norm[row] = nm;
-      if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
-    }
-    for (int g = warp; g < G; g += kWarps) {
-      float mx = -INFINITY;
-      for (int t = lane; t < tok; t += 32) mx = fmaxf(mx, zs[t * G + g]);
-      mx = warp_max(mx);
-      const float m_old = s_m[g];
-      const float m_new = fmaxf(m_old, mx);
-      float sum = 0.f;
-      for (int t = lane; t < tok; t += 32) {
-        const float pv = (m_new == -INFINITY) ? 0.f : exp2f(zs[t * G + g] - m_new);
-        ps[t * G + g] = pv;
-        sum += pv;
-      }
-      sum = warp_sum(sum);
-      if (lane == 0) {
-        const float corr = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
-        s_corr[g] = corr;
-        s_l[g] = s_l[g] * corr + sum;
-        s_m[g] = m_new;
-      }
-    }
+    // token partitions tp -> "warp partial" slots 0..TP-1 with the shared (m, l)
+    for (int e = tid; e < kWarps * G * (D + 2); e += kThreads) wpart[e] = 0.f;
     __syncthreads();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      acc[g][0] *= s_corr[g];
-      acc[g][1] *= s_corr[g];
-    }
-    for (int t = tp; t < tok; t += TP) {
-      float vv[2];
-      load_vec<T, 2>(vt + (size_t)t * D + 2 * cg, vv);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pw = ps[t * G + g];
-        acc[g][0] = fmaf(pw, vv[0], acc[g][0]);
-        acc[g][1] = fmaf(pw, vv[1], acc[g][1]);
+      float* wp = wpart + ((size_t)tp * G + g) * (D + 2);
+      wp[2 * cg] = acc[g][0];
+      wp[2 * cg + 1] = acc[g][1];
+      if (cg == 0) {
+        wp[D] = s_m[g];
+        wp[D + 1] = tp == 0 ? s_l[g] : 0.f;
       }
     }
+    for (int w = TP + tid; w < kWarps; w += kThreads)  // unused slots: empty
+      for (int g = 0; g < G; ++g) wpart[((size_t)w * G + g) * (D + 2) + D] = -INFINITY;
     __syncthreads();
-    if (tid == 0 && i + 2 < ne) issue_kv(i + 2);
   }
-  if (s_abort && tid == 0) {
-    for (int i = 0; i < 2; ++i) (void)mbar_wait_bounded(&kvbar[i], 0, 1u << 12);
-    report_timeout(p.status, 2);
-  }
-  __syncthreads();
 
-  // ---- 4. partials in shared memory, merged across the cluster -----------------------------
-  float* red = reinterpret_cast<float*>(smem);  // [TP][G][D], then the partial o [G][D]
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    red[((size_t)tp * G + g) * D + 2 * cg] = acc[g][0];
-    red[((size_t)tp * G + g) * D + 2 * cg + 1] = acc[g][1];
+  // ---- 4. merge the warps, push column slices to their owners, finish -----------------------
+  const int cols = D / CL;
+  // per head: combined max over warps, then weights
+  for (int g = warp; g < G; g += kWarps) {
+    float M = -INFINITY;
+    if (lane < kWarps) M = wpart[((size_t)lane * G + g) * (D + 2) + D];
+    M = warp_max(M);
+    float lsum = 0.f;
+    if (lane < kWarps) {
+      const float mw = wpart[((size_t)lane * G + g) * (D + 2) + D];
+      const float w = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      lsum = w * wpart[((size_t)lane * G + g) * (D + 2) + D + 1];
+    }
+    lsum = warp_sum(lsum);
+    if (lane == 0) {
+      s_m[g] = M;
+      s_l[g] = lsum;
+    }
   }
   __syncthreads();
-  float* part = red + (size_t)TP * G * D;  // [G][D]
   for (int e = tid; e < G * D; e += kThreads) {
-    float sum = 0.f;
-    for (int u = 0; u < TP; ++u) sum += red[(size_t)u * G * D + e];
-    part[e] = sum;
+    const int g = e / D, col = e % D;
+    const float M = s_m[g];
+    float osum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wpart[((size_t)w * G + g) * (D + 2) + D];
+      if (mw != -INFINITY) osum = fmaf(exp2f(mw - M), wpart[((size_t)w * G + g) * (D + 2) + col], osum);
+    }
+    // push to the owner of this column: recv[rank][g][col % cols], plus (m, l)
+    const int owner = col / cols;
+    float* slot = recv + ((size_t)rank * G + g) * (cols + 2);
+    st_dsmem_f32(dsmem_addr(&slot[col % cols], owner), osum);
+    if (col % cols == 0) {
+      st_dsmem_f32(dsmem_addr(&slot[cols], owner), M);
+      st_dsmem_f32(dsmem_addr(&slot[cols + 1], owner), s_l[g]);
+    }
   }
   cluster_sync();
-  const int cols = D / CL;  // output columns merged by this CTA
   for (int e = tid; e < G * cols; e += kThreads) {
-    const int g = e / cols, col = rank * cols + e % cols;
+    const int g = e / cols, cc = e % cols, col = rank * cols + cc;
     float M = -INFINITY;
-    for (int r = 0; r < CL; ++r) M = fmaxf(M, ld_dsmem_f32(dsmem_addr(&s_m[g], r)));
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, recv[((size_t)r * G + g) * (cols + 2) + cols]);
     float lsum = 0.f, osum = 0.f;
     for (int r = 0; r < CL; ++r) {
-      const float mr = ld_dsmem_f32(dsmem_addr(&s_m[g], r));
-      const float w = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
-      if (w != 0.f) {
-        lsum = fmaf(w, ld_dsmem_f32(dsmem_addr(&s_l[g], r)), lsum);
-        osum = fmaf(w, ld_dsmem_f32(dsmem_addr(&part[g * D + col], r)), osum);
-      }
+      const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
+      const float mr = slot[cols];
+      if (mr == -INFINITY) continue;
+      const float w = exp2f(mr - M);
+      lsum = fmaf(w, slot[cols + 1], lsum);
+      osum = fmaf(w, slot[cc], osum);
     }
     const size_t row = (size_t)bi * Hq + h0 + g;
     static_cast<T*>(p.o)[row * D + col] = Elem<T>::from_f(osum / lsum);
     if (col == 0 && p.lse) p.lse[row] = (M + log2f(lsum)) * kLn2;
   }
-  cluster_sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
 int pick_cluster(int groups) {
-  // the largest power of two (2..16) keeping all clusters resident at about two CTAs per SM
+  // the largest power of two (2..16) keeping every cluster resident at two CTAs per SM
   int cl = 2;
   while (cl * 2 <= kMaxCL && groups * cl * 2 <= 2 * kSMs) cl <<= 1;
   return cl;
 }
 
-template <typename T, int D, int G>
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+bool kv_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
+  using SM = FusedSmem<T, D, G, MMA>;
+  CUtensorMap tmk{}, tmv{};
+  if (MMA) {
+    const long long rows = (long long)p.B * p.Hk * p.n;
+    if (!kv_map(&tmk, p.k, rows, D) || !kv_map(&tmv, p.v, rows, D)) return BSA_ERR_CUDA;
+  }
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
-  if (D / CL < 1) CL = D;
-  const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
-  p.chunk = chunk;
-  p.ns = 3;
-  auto kern = decode_fused_kernel<T, D, G>;
-  size_t smem = FusedSmem<T, D, G>::bytes(p.b, p.ns, chunk);
-  if (smem > 200 * 1024) {
-    p.ns = 2;
-    smem = FusedSmem<T, D, G>::bytes(p.b, p.ns, chunk);
-  }
-  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess) {
-    (void)cudaGetLastError();
-    return BSA_ERR_CUDA;
-  }
-  if (CL > 8 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-    (void)cudaGetLastError();
-    CL = 8;
-  }
+  auto kern = decode_fused_kernel<T, D, G, MMA>;
   for (;;) {
+    const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
+    if (chunk > 32 * kSelItems) {  // the local select holds at most 512 keys per head
+      if (CL < kMaxCL) { CL <<= 1; continue; }
+      return BSA_ERR_UNSUPPORTED;
+    }
+    p.chunk = chunk;
+    const size_t smem = SM::bytes(p.b, chunk, CL, p.K) + 1024;  // + alignment slack
+    if (smem > 220 * 1024) return BSA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      return BSA_ERR_CUDA;
+    }
+    if (CL > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                      cudaSuccess) {
+      (void)cudaGetLastError();
+      return BSA_ERR_UNSUPPORTED;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, p.Hk, p.B);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -624,18 +940,9 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
       (void)cudaGetLastError();
       if (CL <= 2) return BSA_ERR_UNSUPPORTED;
       CL >>= 1;
-      const int ch = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
-      p.chunk = ch;
-      smem = FusedSmem<T, D, G>::bytes(p.b, p.ns, ch);
-      if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess) {
-        (void)cudaGetLastError();
-        return BSA_ERR_CUDA;
-      }
       continue;
     }
-    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) {
       (void)cudaGetLastError();
       return BSA_ERR_CUDA;
     }
@@ -643,13 +950,13 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool MMA>
 bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_fused<T, D, 1>(p, st);
-    case 2: return launch_fused<T, D, 2>(p, st);
-    case 4: return launch_fused<T, D, 4>(p, st);
-    case 8: return launch_fused<T, D, 8>(p, st);
+    case 1: return launch_fused<T, D, 1, MMA>(p, st);
+    case 2: return launch_fused<T, D, 2, MMA>(p, st);
+    case 4: return launch_fused<T, D, 4, MMA>(p, st);
+    case 8: return launch_fused<T, D, 8, MMA>(p, st);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }
@@ -679,7 +986,7 @@ extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* 
   BSA_REQUIRE(B <= 65535 && Hk <= 65535, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(all_aligned16(q, k, v, o, mean_k), BSA_ERR_ARG);
   const int C = ceil_div(n, b);
-  BSA_REQUIRE(ceil_div(C, kMaxCL) <= 1024 * 1024, BSA_ERR_UNSUPPORTED);
+  BSA_REQUIRE(C <= kMaxWords * 32, BSA_ERR_UNSUPPORTED);
   FusedParams p{};
   p.q = q; p.k = k; p.v = v;
   p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.b = b; p.C = C; p.K = K;
@@ -688,12 +995,15 @@ extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* 
   p.o = o; p.lse = lse; p.idx = idx; p.count = count; p.status = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   bsa_status rc;
-  if (dt == BSA_BF16)
-    rc = d == 64 ? dispatch_fused<__nv_bfloat16, 64>(Hq / Hk, p, st)
-                 : dispatch_fused<__nv_bfloat16, 128>(Hq / Hk, p, st);
+  if (dt == BSA_BF16 && b == 64)  // 64-token blocks: warp MMAs over swizzled TMA tiles
+    rc = d == 64 ? dispatch_fused<__nv_bfloat16, 64, true>(Hq / Hk, p, st)
+                 : dispatch_fused<__nv_bfloat16, 128, true>(Hq / Hk, p, st);
+  else if (dt == BSA_BF16)
+    rc = d == 64 ? dispatch_fused<__nv_bfloat16, 64, false>(Hq / Hk, p, st)
+                 : dispatch_fused<__nv_bfloat16, 128, false>(Hq / Hk, p, st);
   else
-    rc = d == 64 ? dispatch_fused<float, 64>(Hq / Hk, p, st)
-                 : dispatch_fused<float, 128>(Hq / Hk, p, st);
+    rc = d == 64 ? dispatch_fused<float, 64, false>(Hq / Hk, p, st)
+                 : dispatch_fused<float, 128, false>(Hq / Hk, p, st);
   if (rc != BSA_OK) return rc;
   BSA_LAUNCH_CHECK();
   return BSA_OK;

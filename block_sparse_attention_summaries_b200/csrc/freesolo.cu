@@ -24,6 +24,10 @@
 #include "bsa_common.cuh"
 
 namespace bsa {
+
+bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, int H, int Hk,
+                          int n, int d, int window, void* o, int* status, cudaStream_t st);
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -170,6 +174,7 @@ struct FsParams {
   const void* k;
   const void* v;
   const void* k_rot;
+  int short_in_o;  // 1: o already holds the short branch (tensor-core window kernel)
   int H, n, cell, window, K;
   double log_theta;
   const float* alpha;
@@ -266,11 +271,17 @@ __global__ void __launch_bounds__(128) freesolo_attn_kernel(const FsParams p) {
     }
   };
 
-  float ms, ls, os[E];
-  attend(krb, qrot, max(0, i - p.window + 1), i + 1, nullptr, 0, ms, ls, os);
   float out[E];
+  if (p.short_in_o) {
+    const T* orow = static_cast<const T*>(p.o) + (hrow + i) * D;
 #pragma unroll
-  for (int e = 0; e < E; ++e) out[e] = os[e] / ls;
+    for (int e = 0; e < E; ++e) out[e] = Elem<T>::to_f(orow[lane + 32 * e]);
+  } else {
+    float ms, ls, os[E];
+    attend(krb, qrot, max(0, i - p.window + 1), i + 1, nullptr, 0, ms, ls, os);
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = os[e] / ls;
+  }
 
   const size_t qrow = hrow + i;
   const int cnt = min(p.count ? p.count[qrow] : p.K, p.K);
@@ -281,6 +292,7 @@ __global__ void __launch_bounds__(128) freesolo_attn_kernel(const FsParams p) {
     // only cells wholly at or before the query are read (no future token, no out-of-range row)
     if (c >= 0 && (c + 1) * p.cell <= i + 1 && nsel < kMaxK) cells[nsel++] = c;
   }
+  if (nsel == 0 && p.short_in_o) return;  // o already final
   if (nsel > 0) {
     float ml, ll, ol[E];
     attend(kb, qraw, 0, 0, cells, nsel, ml, ll, ol);
@@ -343,7 +355,8 @@ extern "C" bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, in
 
 extern "C" size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d) {
   if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return 0;
-  return (size_t)B * H * n * d * (dt == BSA_BF16 ? 2 : 4) + 256;
+  // rotated keys, and (bf16) rotated queries for the tensor-core window branch
+  return (size_t)B * H * n * d * (dt == BSA_BF16 ? 2 : 4) * (dt == BSA_BF16 ? 2 : 1) + 256;
 }
 
 extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt,
@@ -366,11 +379,41 @@ extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void
   FsParams p;
   p.q = q; p.k = k; p.v = v;
   p.k_rot = static_cast<unsigned char*>(workspace) + 256;
+  p.short_in_o = 0;
   p.H = H; p.n = n; p.cell = cell; p.window = window; p.K = K;
   p.log_theta = log((double)rope_theta);
   p.alpha = alpha_h; p.idx = idx; p.count = count; p.o = o;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* kr = const_cast<void*>(p.k_rot);
+  if (dt == BSA_BF16) {
+    // short branch on the tensor cores: rotate q and k once, sliding-window tiles over them
+    const long long rows = (long long)B * H * n;
+    void* qr = static_cast<unsigned char*>(workspace) + 256 + (size_t)rows * d * 2;
+    const long long pairs = rows * (d / 2);
+    const unsigned nblk = (unsigned)((pairs + 255) / 256);
+    if (d == 64) {
+      rope_keys_kernel<__nv_bfloat16, 64><<<nblk, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(kr), rows, n, p.log_theta);
+      rope_keys_kernel<__nv_bfloat16, 64><<<nblk, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(qr), rows, n, p.log_theta);
+    } else {
+      rope_keys_kernel<__nv_bfloat16, 128><<<nblk, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(kr), rows, n, p.log_theta);
+      rope_keys_kernel<__nv_bfloat16, 128><<<nblk, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(qr), rows, n, p.log_theta);
+    }
+    BSA_LAUNCH_CHECK();
+    bsa_status rc = window_attn_tc(qr, kr, v, B, H, H, n, d, window, o, nullptr, st);
+    if (rc == BSA_OK) {
+      p.short_in_o = 1;
+      dim3 grid(ceil_div(n, 4), H, B);
+      if (d == 64) freesolo_attn_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(p);
+      else freesolo_attn_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(p);
+      BSA_LAUNCH_CHECK();
+      return BSA_OK;
+    }
+    if (rc != BSA_ERR_UNSUPPORTED) return rc;
+  }
   if (dt == BSA_BF16) {
     if (d == 64) launch_attn<__nv_bfloat16, 64>(p, B, st, kr);
     else launch_attn<__nv_bfloat16, 128>(p, B, st, kr);

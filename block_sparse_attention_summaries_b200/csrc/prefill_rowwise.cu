@@ -23,6 +23,10 @@ bsa_status decode_attn(const void* q, const void* k, const void* v, bsa_dtype dt
                        int scores_ld, void* o, float* lse, void* ws, size_t ws_bytes,
                        cudaStream_t st);
 bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq, int Hk);
+bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, int B, int Hq, int Hk, int n, int d,
+                        const int* idx, const int* count, int K, int norm, const float* scores,
+                        int scores_ld, float* dg, int* status, cudaStream_t st);
 bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hk, int n,
                       int d, int b, const int* idx, const int* count, int K, int gate, int norm,
                       const float* scores, int scores_ld, void* o, float* lse, int* status,
@@ -361,6 +365,11 @@ extern "C" bsa_status bsa_gate_grad(const void* q, const void* k, const void* v,
   BSA_REQUIRE(q_block > 0 && q_block <= n, BSA_ERR_ARG);
   BSA_REQUIRE(scores_ld >= ceil_div(n, b), BSA_ERR_SHAPE);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (prefill_tc_supported(dt, d, b, q_block, K, Hq, Hk)) {
+    // the gradient of the gated forward: the gate enters only through lse and o here
+    return gate_grad_tc(q, k, v, o, lse, dout, B, Hq, Hk, n, d, idx, count, K, norm, scores,
+                        scores_ld, dg, nullptr, st);
+  }
   RowParams p{};
   p.q = q; p.k = k; p.v = v; p.o_in = o; p.lse_in = lse; p.dout = dout;
   p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.b = b; p.q_block = q_block;

@@ -49,6 +49,8 @@ struct TcParams {
   void* o;
   float* lse;
   int* status;
+  int mode;    // 0: heads 2hp, 2hp+1 at unit u (selected blocks); 1: units 2up, 2up+1 of head h
+  int window;  // mode 1: keys j >= i - window + 1 of a sliding window (blocks of the window)
 };
 
 template <int D>
@@ -92,15 +94,33 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u = blockIdx.x, hp = blockIdx.y, bi = blockIdx.z;
-  const int hq[2] = {2 * hp, 2 * hp + 1};
+  const int bi = blockIdx.z;
+  const bool win = p.mode == 1;
+  // the two work items: (head, unit) pairs sharing one kv head
+  const int hq[2] = {win ? (int)blockIdx.y : 2 * (int)blockIdx.y,
+                     win ? (int)blockIdx.y : 2 * (int)blockIdx.y + 1};
+  const int uu[2] = {win ? 2 * (int)blockIdx.x : (int)blockIdx.x,
+                     win ? 2 * (int)blockIdx.x + 1 : (int)blockIdx.x};
+  const bool item_ok[2] = {uu[0] < p.U, uu[1] < p.U};
   const int G = p.Hq / p.Hk;
-  const int kh = hq[0] / G;  // both heads of the pair share the kv head (G is even)
-  const int nc = u;          // history blocks before unit u (q_block == b)
+  const int kh = hq[0] / G;  // both items read the same kv head
+  const int wblocks = win ? (p.window - 1 + kTiles - 1) / kTiles : 0;
 
-  // ---- prologue: block lists and gate biases of both units (warps 0 and 1) -----------------
-  if (warp < 2) {
+  // ---- prologue: block lists and gate biases of both items (warps 0 and 1) -----------------
+  if (warp < 2 && win) {  // sliding window: blocks u - wblocks .. u - 1 before the diagonal one
     const int it = warp;
+    const int u = uu[it];
+    const int first = item_ok[it] ? max(0, u - wblocks) : 0;
+    const int cnt = item_ok[it] ? u - first : 0;
+    for (int j = lane; j < cnt && j < kMaxKtc; j += 32) {
+      s_blk[it][j] = first + j;
+      s_bias[it][j] = 0.f;
+    }
+    if (lane == 0) s_cnt[it] = min(cnt, kMaxKtc);
+  } else if (warp < 2) {
+    const int it = warp;
+    const int u = uu[it];
+    const int nc = u;  // history blocks before unit u (q_block == b)
     const size_t row = ((size_t)bi * p.Hq + hq[it]) * p.U + u;
     const int cnt_in = p.count ? min(p.count[row], p.K) : p.K;
     int base = 0;
@@ -165,7 +185,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int steps = max(s_cnt[0], s_cnt[1]) + 1;
   const uint32_t tmem = s_tmem;
   // step j of unit it: history block, filler (fully masked) or the current block (last step)
-  auto step_block = [&](int it, int j) { return j < s_cnt[it] ? s_blk[it][j] : u; };
+  auto step_block = [&](int it, int j) {
+    return j < s_cnt[it] ? s_blk[it][j] : (item_ok[it] ? uu[it] : uu[0]);
+  };
 
   unsigned char* sq[2] = {smem + L::kQ, smem + L::kQ + L::kTileBytes};
   auto stage_tile = [&](int st, int which) {  // which: 0 K0, 1 V0, 2 K1, 3 V1
@@ -178,7 +200,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
       for (int it = 0; it < 2; ++it) {
-        const int y = ((bi * p.Hq + hq[it]) * p.n) + u * kTiles;
+        const int y = ((bi * p.Hq + hq[it]) * p.n) + uu[it] * kTiles;
         for (int hf = 0; hf < L::kHalves; ++hf)
           tc::tma_load_2d(sq[it] + hf * 8192, &tmq, hf * 64, y, q_full);
       }
@@ -265,9 +287,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax warps 0-3
-    const int it = lane >> 4;                  // unit of this thread's row
+    const int it = lane >> 4;                  // item of this thread's row
     const int r = 16 * warp + (lane & 15);     // row within the unit
-    const int i = u * kTiles + r;              // query position
+    const int i = uu[it] * kTiles + r;         // query position
+    const int wlo = win ? i - p.window + 1 : INT_MIN;  // lowest key of the window
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     const float qk_scale = rsqrtf((float)D) * kLog2e;
     float m_run = -INFINITY, l_run = 0.f;
@@ -287,11 +310,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const bool is_cur = (j == steps - 1);
       const bool filler = !is_cur && j >= s_cnt[it];
       const float bias = (!is_cur && !filler) ? s_bias[it][j] : 0.f;
+      const int kpos0 = step_block(it, j) * kTiles;  // position of this block's first key
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         float z = fmaf(x[c], qk_scale, bias);
-        if (filler || (is_cur && c > r)) z = -INFINITY;
+        if (filler || (is_cur && c > r) || kpos0 + c < wlo) z = -INFINITY;
         x[c] = z;
         mx = fmaxf(mx, z);
       }
@@ -347,7 +371,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (steps - 1) & 1));
     if (ok) {
       tc::fence_after_sync();
-      const bool live = i < p.n;
+      const bool live = i < p.n && item_ok[it];
       const size_t orow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
       const float inv = 1.f / l_run;
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow * D;
@@ -382,6 +406,253 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   tc::fence_before_sync();
   __syncthreads();
   if (s_abort && tid == 0) report_timeout(p.status, 3);
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---- gate gradient on the tensor cores -----------------------------------------------------
+//
+// [SAS] review, "Why the four design choices matter", Eq. 5 (inner gate):
+//     dg_m = sum_{i in B_m} (ptilde_i / g_m) do^T (v_i - o),
+// summed over the unit's queries, in the stable form
+//     dg_m = sum_q sum_{j in B_m} exp(z_qj - lse_q) (do_q . v_j - do_q . o_q),   z = q . k / sqrt(d).
+// Same CTA shape as the forward: heads h and h+1 at unit u in interleaved M = 64 TMEM lanes.
+// Per selected history block j the MMA thread computes Z_j = Q K_j^T and DV_j = dO V_j^T into a
+// double-buffered TMEM pair; each softmax-warp thread reduces its row, and the 64 rows of a unit
+// are summed with shuffles and shared-memory atomics into dg of that block.
+template <int D>
+struct GgSmem {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kTiles * D * 2;
+  static constexpr int kQ = 0;                        // Q0, dO0, Q1, dO1
+  static constexpr int kStage = 4 * kTileBytes;       // stages: K0 V0 K1 V1
+  static constexpr int kStageBytes = 4 * kTileBytes;
+  static constexpr int kBars = kStage + 2 * kStageBytes;
+  static constexpr int kTotal = kBars + 1024;
+};
+
+struct GgParams {
+  int B, Hq, Hk, n, U, K;
+  const int* idx;
+  const int* count;
+  int norm;
+  const float* scores;
+  int scores_ld;
+  const void* o;
+  const float* lse;
+  const void* dout;
+  float* dg;
+  int* status;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    gate_grad_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tmdo,
+                        const __grid_constant__ CUtensorMap tmk,
+                        const __grid_constant__ CUtensorMap tmv, const GgParams p) {
+  using L = GgSmem<D>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* fin = bars + 9;
+
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_blk[2][kMaxKtc];
+  __shared__ int s_slot[2][kMaxKtc];
+  __shared__ float s_dg[2][kMaxKtc];
+  __shared__ int s_cnt[2];
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.x, hp = blockIdx.y, bi = blockIdx.z;
+  const int hq[2] = {2 * hp, 2 * hp + 1};
+  const int G = p.Hq / p.Hk;
+  const int kh = hq[0] / G;
+  const int nc = u;
+
+  if (warp < 2) {  // block lists (with their idx slots) of both units
+    const int it = warp;
+    const size_t row = ((size_t)bi * p.Hq + hq[it]) * p.U + u;
+    const int cnt_in = p.count ? min(p.count[row], p.K) : p.K;
+    int base = 0;
+    for (int j0 = 0; j0 < cnt_in; j0 += 32) {
+      const int j = j0 + lane;
+      const int m = j < cnt_in ? p.idx[row * p.K + j] : -1;
+      const bool ok = j < cnt_in && m >= 0 && m < nc;
+      const unsigned bal = __ballot_sync(0xffffffffu, ok);
+      const int at = base + __popc(bal & ((1u << lane) - 1u));
+      if (ok && at < kMaxKtc) {
+        s_blk[it][at] = m;
+        s_slot[it][at] = j;
+      }
+      base += __popc(bal);
+    }
+    base = min(base, kMaxKtc);
+    for (int j = lane; j < kMaxKtc; j += 32) s_dg[it][j] = 0.f;
+    if (lane == 0) s_cnt[it] = base;
+  }
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    mbar_init(fin, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(&s_tmem, 256);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int steps = max(s_cnt[0], s_cnt[1]);
+  const uint32_t tmem = s_tmem;
+  auto step_block = [&](int it, int j) { return j < s_cnt[it] ? s_blk[it][j] : u; };
+  auto qtile = [&](int it, int which) { return smem + L::kQ + (2 * it + which) * L::kTileBytes; };
+  auto stage_tile = [&](int st, int which) {
+    return smem + L::kStage + st * L::kStageBytes + which * L::kTileBytes;
+  };
+
+  if (steps > 0) {
+    if (warp == 4) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, 4 * L::kTileBytes);
+        for (int it = 0; it < 2; ++it) {
+          const int y = ((bi * p.Hq + hq[it]) * p.n) + u * kTiles;
+          for (int hf = 0; hf < L::kHalves; ++hf) {
+            tc::tma_load_2d(qtile(it, 0) + hf * 8192, &tmq, hf * 64, y, q_full);
+            tc::tma_load_2d(qtile(it, 1) + hf * 8192, &tmdo, hf * 64, y, q_full);
+          }
+        }
+        int issued = 0;
+        for (int j = 0; j < steps; ++j) {
+          const int st = j & 1;
+          if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) - 1) & 1)) {
+            s_abort = 1;
+            break;
+          }
+          issued = j + 1;
+          mbar_arrive_expect_tx(&kv_full[st], 4 * L::kTileBytes);
+          for (int it = 0; it < 2; ++it) {
+            const int y = ((bi * p.Hk + kh) * p.n) + step_block(it, j) * kTiles;
+            for (int hf = 0; hf < L::kHalves; ++hf) {
+              tc::tma_load_2d(stage_tile(st, 2 * it) + hf * 8192, &tmk, hf * 64, y, &kv_full[st]);
+              tc::tma_load_2d(stage_tile(st, 2 * it + 1) + hf * 8192, &tmv, hf * 64, y,
+                              &kv_full[st]);
+            }
+          }
+        }
+        if (s_abort)
+          for (int j = max(0, issued - 2); j < issued; ++j)
+            (void)mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, 1u << 16);
+      }
+    } else if (warp == 5) {
+      if (lane == 0) {
+        constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+        bool ok = mbar_wait_bounded(q_full, 0);
+        for (int j = 0; ok && j < steps; ++j) {
+          const int st = j & 1;
+          ok = mbar_wait_bounded(&kv_full[st], (j >> 1) & 1);
+          if (ok && j >= 2) ok = mbar_wait_bounded(&s_free[st], ((j >> 1) - 1) & 1);
+          if (!ok) break;
+          tc::fence_after_sync();
+          for (int it = 0; it < 2; ++it) {
+            const uint32_t lane_off = (uint32_t)(16 * it) << 16;
+            const uint32_t d_z = tmem + (uint32_t)(st * 128) + lane_off;
+            const uint32_t d_dv = d_z + 64u;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int hf = kk >> 2, off = (kk & 3) * 32;
+              tc::mma_f16_ss(d_z, tc::smem_desc_sw128(qtile(it, 0) + hf * 8192 + off, 16, 1024),
+                             tc::smem_desc_sw128(stage_tile(st, 2 * it) + hf * 8192 + off, 16,
+                                                 1024),
+                             idS, kk > 0);
+              tc::mma_f16_ss(d_dv, tc::smem_desc_sw128(qtile(it, 1) + hf * 8192 + off, 16, 1024),
+                             tc::smem_desc_sw128(stage_tile(st, 2 * it + 1) + hf * 8192 + off, 16,
+                                                 1024),
+                             idS, kk > 0);
+            }
+          }
+          tc::mma_commit(&s_full[st]);
+          tc::mma_commit(&kv_empty[st]);
+        }
+        if (!ok) s_abort = 1;
+        tc::mma_commit(fin);
+        if (!mbar_wait_bounded(fin, 0)) s_abort = 1;
+      }
+    } else {
+      // reduction warps: thread = one query row of one unit
+      const int it = lane >> 4;
+      const int r = 16 * warp + (lane & 15);
+      const int i = u * kTiles + r;
+      const bool live = i < p.n;
+      const size_t qrow = ((size_t)bi * p.Hq + hq[it]) * p.n + (live ? i : 0);
+      float Di = 0.f, lse2 = 0.f;
+      if (live) {
+        const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + qrow * D;
+        const __nv_bfloat16* drow = static_cast<const __nv_bfloat16*>(p.dout) + qrow * D;
+        for (int c = 0; c < D; c += 8) {
+          float a[8], bb[8];
+          load_vec<__nv_bfloat16, 8>(orow + c, a);
+          load_vec<__nv_bfloat16, 8>(drow + c, bb);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) Di = fmaf(a[e], bb[e], Di);
+        }
+        lse2 = p.lse[qrow] * kLog2e;
+      }
+      const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+      const float zs = rsqrtf((float)D) * kLog2e;
+      bool ok = true;
+      for (int j = 0; j < steps; ++j) {
+        const int st = j & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
+        if (!ok) break;
+        tc::fence_after_sync();
+        float z[64], dv[64];
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128), z);
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 32), z + 32);
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 64), dv);
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 96), dv + 32);
+        tc::tmem_wait_ld();
+        tc::fence_before_sync();
+        mbar_arrive(&s_free[st]);
+        float t = 0.f;
+        if (live && j < s_cnt[it]) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) t = fmaf(exp2f(fmaf(z[c], zs, -lse2)), dv[c] - Di, t);
+        }
+        // sum over the 16 rows of this unit held by this warp, then across warps
+#pragma unroll
+        for (int o2 = 8; o2 > 0; o2 >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o2);
+        if ((lane & 15) == 0 && j < s_cnt[it]) atomicAdd(&s_dg[it][j], t);
+      }
+      if (!ok) s_abort = 1;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp < 2) {  // results of both units, every idx slot (0 where nothing was selected)
+    const int it = warp;
+    const size_t row = ((size_t)bi * p.Hq + hq[it]) * p.U + u;
+    for (int j = lane; j < p.K; j += 32) p.dg[row * p.K + j] = 0.f;
+    __syncwarp();
+    for (int j = lane; j < s_cnt[it]; j += 32) p.dg[row * p.K + s_slot[it][j]] = s_dg[it][j];
+  }
+  if (s_abort && tid == 0) report_timeout(p.status, 4);
   if (warp == 5) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 256);
@@ -434,12 +705,62 @@ bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
-  dim3 grid(p.U, p.Hq / 2, p.B);
+  dim3 grid = p.mode == 1 ? dim3((p.U + 1) / 2, p.Hq, p.B) : dim3(p.U, p.Hq / 2, p.B);
   kern<<<grid, kThreadsTc, smem, st>>>(tmq, tmk, tmv, p);
   return BSA_OK;
 }
 
+template <int D>
+bsa_status launch_gg(const void* q, const void* k, const void* v, const void* dout,
+                     const GgParams& p, cudaStream_t st) {
+  CUtensorMap tmq, tmdo, tmk, tmv;
+  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D) ||
+      !make_map(&tmdo, dout, (long long)p.B * p.Hq * p.n, D) ||
+      !make_map(&tmk, k, (long long)p.B * p.Hk * p.n, D) ||
+      !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
+    return BSA_ERR_CUDA;
+  const int smem = GgSmem<D>::kTotal + 1024;
+  auto kern = gate_grad_tc_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  dim3 grid(p.U, p.Hq / 2, p.B);
+  kern<<<grid, kThreadsTc, smem, st>>>(tmq, tmdo, tmk, tmv, p);
+  return BSA_OK;
+}
+
 }  // namespace
+
+bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, int B, int Hq, int Hk, int n, int d,
+                        const int* idx, const int* count, int K, int norm, const float* scores,
+                        int scores_ld, float* dg, int* status, cudaStream_t st) {
+  GgParams p{};
+  p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = K;
+  p.idx = idx; p.count = count; p.norm = norm; p.scores = scores; p.scores_ld = scores_ld;
+  p.o = o; p.lse = lse; p.dout = dout; p.dg = dg; p.status = status;
+  bsa_status rc = d == 64 ? launch_gg<64>(q, k, v, dout, p, st)
+                          : launch_gg<128>(q, k, v, dout, p, st);
+  if (rc != BSA_OK) return rc;
+  BSA_LAUNCH_CHECK();
+  return BSA_OK;
+}
+
+// Sliding-window causal attention (window keys j in [i - window + 1, i]) of already rotated q/k
+// on the tensor cores: the short branch of the FreeSolo prefill, written to o.
+bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, int H, int Hk,
+                          int n, int d, int window, void* o, int* status, cudaStream_t st) {
+  TcParams p{};
+  p.B = B; p.Hq = H; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = 0;
+  p.o = o; p.lse = nullptr; p.status = status; p.mode = 1; p.window = window;
+  if (ceil_div(window - 1, kTiles) > kMaxKtc) return BSA_ERR_UNSUPPORTED;
+  bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
+  if (rc != BSA_OK) return rc;
+  BSA_LAUNCH_CHECK();
+  return BSA_OK;
+}
 
 bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq, int Hk) {
   if (dt != BSA_BF16 || b != kTiles || q_block != kTiles || K > kMaxKtc) return false;
