@@ -278,6 +278,13 @@ def run_gpu(args):
 
     import block_sparse_attention_summaries_b200 as bsa
 
+    if args.prefill_only:
+        torch.cuda.set_device(0)
+        bsa.lib()
+        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), load_peaks())}),
+              flush=True)
+        return
+
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -522,6 +529,8 @@ def main():
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill rows (profiling the prefill kernels)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

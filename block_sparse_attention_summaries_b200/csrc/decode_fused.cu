@@ -104,12 +104,16 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Top-K of N order keys (shared memory, index order) by one warp.  Bisection finds the largest T
-// with count(key >= T) >= K (32 steps of a warp-wide count), then one ordered pass takes every key
-// above T and the lowest-indexed keys equal to T.  Writes the selected positions ascending to
-// `out`; returns min(K, N).  N <= 32 * kSelItems.
-constexpr int kSelItems = 16;
-__device__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
+// Top-K of N order keys (shared memory, index order) by one warp: an exact radix select with
+// 4-bit digits.  Each pass builds the 16-bin histogram of the next digit among the keys that
+// share the prefix found so far (per-lane counts packed two bins per 32-bit word, then eight
+// independent warp reductions), and keeps the digit at which the count of keys at or above the
+// threshold reaches K.  It stops as soon as that count is exactly K ({key >= T} is then the
+// answer); otherwise after the last digit T is the K-th largest key and the lowest-indexed keys
+// equal to T fill the remaining places.  Eight short passes instead of a 32-step bisection.
+// Writes the selected positions ascending to `out`; returns min(K, N).
+constexpr int kSelItems = 16;  // N <= 32 * kSelItems
+__device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
   if (kk == N) {
@@ -117,40 +121,63 @@ __device__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* ou
     __syncwarp();
     return N;
   }
-  uint32_t r[kSelItems];
+  uint32_t T = 0;      // digits fixed so far (higher bits)
+  int above = 0;       // keys strictly above the prefix (they are selected)
+  bool exact = false;
+  for (int shift = 28; shift >= 0 && !exact; shift -= 4) {
+    const uint32_t hi_mask = shift == 28 ? 0u : (0xFFFFFFFFu << (shift + 4));
+    uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bins 2j (low 16 bits), 2j+1 (high)
+    for (int i = lane; i < N; i += 32) {
+      const uint32_t x = keys[i];
+      if ((x & hi_mask) == T) {
+        const uint32_t d = (x >> shift) & 15u;
+        const uint32_t inc = 1u << ((d & 1u) * 16u);
 #pragma unroll
-  for (int e = 0; e < kSelItems; ++e) {
-    const int i = lane + 32 * e;
-    r[e] = i < N ? keys[i] : 0u;
+        for (int j = 0; j < 8; ++j) h[j] += (d >> 1) == (uint32_t)j ? inc : 0u;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) h[j] = __reduce_add_sync(0xffffffffu, h[j]);
+    // largest digit v with above + count(digit >= v) >= kk
+    int run = above, v = 0, run_at_v = 0;
+#pragma unroll
+    for (int d = 15; d >= 0; --d) {
+      const int c = (int)((h[d >> 1] >> ((d & 1) * 16)) & 0xFFFFu);
+      if (run < kk && run + c >= kk) {
+        v = d;
+        run_at_v = run + c;
+      }
+      run += c;
+    }
+    // keys with a digit above v are selected outright
+    int up = above;
+#pragma unroll
+    for (int d = 15; d >= 0; --d) {
+      const int c = (int)((h[d >> 1] >> ((d & 1) * 16)) & 0xFFFFu);
+      if (d > v) up += c;
+    }
+    T |= (uint32_t)v << shift;
+    above = up;
+    exact = (run_at_v == kk);
   }
-  const int items = (N + 31) / 32;
-  uint32_t T = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = T | (1u << bit);
-    int c = 0;
-#pragma unroll
-    for (int e = 0; e < kSelItems; ++e)
-      if (e < items && lane + 32 * e < N) c += (r[e] >= cand);
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= kk) T = cand;
-  }
-  int gt = 0;
-#pragma unroll
-  for (int e = 0; e < kSelItems; ++e)
-    if (e < items && lane + 32 * e < N) gt += (r[e] > T);
-  gt = __reduce_add_sync(0xffffffffu, gt);
-  const int rem = kk - gt;
+  const int rem = kk - above;  // keys equal to the full threshold still to take (if not exact)
+  const uint32_t cmp_mask = 0xFFFFFFFFu;
   int taken = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int e = 0; e < kSelItems; ++e) {
-    if (e >= items) break;
-    const int i = lane + 32 * e;
+  for (int base = 0; base < N; base += 32) {
+    const int i = base + lane;
     const bool valid = i < N;
-    const bool gtb = valid && r[e] > T;
-    const bool eq = valid && r[e] == T;
-    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
-    const bool take = gtb || (eq && eq_seen + __popc(eqb & lt) < rem);
+    const uint32_t x = valid ? keys[i] : 0u;
+    bool take;
+    unsigned eqb = 0u;
+    if (exact) {
+      // T holds the digits down to the stopping pass; compare on those bits only
+      take = valid && x >= T;
+    } else {
+      const bool eq = valid && (x & cmp_mask) == T;
+      eqb = __ballot_sync(0xffffffffu, eq);
+      take = (valid && x > T) || (eq && eq_seen + __popc(eqb & lt) < rem);
+    }
     const unsigned tb = __ballot_sync(0xffffffffu, take);
     if (take) out[taken + __popc(tb & lt)] = i;
     taken += __popc(tb);

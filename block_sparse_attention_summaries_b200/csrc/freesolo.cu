@@ -201,8 +201,9 @@ __global__ void __launch_bounds__(128) freesolo_attn_kernel(const FsParams p) {
 #pragma unroll
   for (int e = 0; e < E; ++e) qraw[e] = Elem<T>::to_f(qp[lane + 32 * e]);
   // rotate q at position i: pairs (t, t + D/2) live in this lane as (e, e + E/2)
+  // (not needed when the short branch already ran on the tensor cores)
 #pragma unroll
-  for (int e = 0; e < E / 2; ++e) {
+  for (int e = 0; e < (p.short_in_o ? 0 : E / 2); ++e) {
     const int t = lane + 32 * e;
     const double inv_freq = exp(-2.0 * t / D * p.log_theta);
     double ang = (double)i * inv_freq;
