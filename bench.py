@@ -247,8 +247,11 @@ def run_prefill(dev, peaks, reps=5):
     ws = torch.empty(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
                                                                   fc.d)),
                      dtype=torch.uint8, device=dev)
+    sws = torch.zeros(max(1, int(bsa.lib().bsa_freesolo_select_workspace_bytes(
+        bsa.BSA_BF16, fc.B, fc.H, fc.n, fc.d, fc.cell, fc.q_block, fc.K))), dtype=torch.uint8,
+        device=dev)
     sel = lambda: bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K,
-                                      idx=idx, count=cnt)
+                                      idx=idx, count=cnt, ws=sws)
     att = lambda: bsa.freesolo_attn(q, k, v, alpha, idx, cnt, fc.cell, fc.window, fc.rope_theta,
                                     o=o, ws=ws)
     t_sel = statistics.fmean(time_cuda(sel, 2, stream))
@@ -262,7 +265,7 @@ def run_prefill(dev, peaks, reps=5):
     out["freesolo_prefill_64k"] = {
         "config": {"B": fc.B, "H": fc.H, "d": fc.d, "n": fc.n, "cell": fc.cell,
                    "q_block": fc.q_block, "K": fc.K, "window": fc.window},
-        "select": {"kernel": "freesolo_select_kernel (CUDA cores)", "ms": t_sel,
+        "select": {"kernel": "split_hi_lo + freesolo_select_tc_kernel (tcgen05)", "ms": t_sel,
                    "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9},
         "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode (tcgen05) + freesolo_attn_kernel long branch (CUDA cores)", "ms": t_att,
                       "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,

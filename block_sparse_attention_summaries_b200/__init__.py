@@ -42,7 +42,8 @@ SIGNATURES = [
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
     ("bsa_freesolo_select", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P,
-                                 _P]),
+                                 _P, _Z, _P]),
+    ("bsa_freesolo_select_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     ("bsa_freesolo_attn", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P,
                                _P, _I, _P, _P, _Z, _P]),
     ("bsa_freesolo_workspace_bytes", _Z, [_I, _I, _I, _I, _I]),
@@ -271,17 +272,25 @@ def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, n
 
 
 def freesolo_select(q, mean_k, max_norm, centre, lambda_h, sigma_h, cell, q_block, K,
-                    idx=None, count=None):
-    """Per-query top-K cells of the FreeSolo long branch: idx [B, H, n, K], count [B, H, n]."""
-    _cuda(q, mean_k, max_norm, centre, lambda_h, sigma_h, idx, count)
+                    idx=None, count=None, ws=None):
+    """Per-query top-K cells of the FreeSolo long branch: idx [B, H, n, K], count [B, H, n].
+
+    ``ws``: a zero-filled uint8 device tensor of at least
+    ``bsa_freesolo_select_workspace_bytes`` bytes (allocated here when omitted)."""
+    _cuda(q, mean_k, max_norm, centre, lambda_h, sigma_h, idx, count, ws)
     B, H, n, d = q.shape
     if idx is None:
         idx = torch.empty(B, H, n, K, device=q.device, dtype=torch.int32)
     if count is None:
         count = torch.empty(B, H, n, device=q.device, dtype=torch.int32)
+    need = int(lib().bsa_freesolo_select_workspace_bytes(_dtype_code(q), B, H, n, d, cell,
+                                                         q_block, K))
+    if ws is None and need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=q.device)
     _check(lib().bsa_freesolo_select(_ptr(q), _dtype_code(q), B, H, n, d, cell, q_block,
                                      _ptr(mean_k), _ptr(max_norm), _ptr(centre), _ptr(lambda_h),
-                                     _ptr(sigma_h), K, _ptr(idx), _ptr(count), _stream(q.device)),
+                                     _ptr(sigma_h), K, _ptr(idx), _ptr(count), _ptr(ws),
+                                     0 if ws is None else ws.numel(), _stream(q.device)),
            "bsa_freesolo_select")
     return idx, count
 

@@ -105,14 +105,34 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 // Top-K of N order keys (shared memory, index order) by one warp: an exact radix select with
-// 4-bit digits.  Each pass builds the 16-bin histogram of the next digit among the keys that
-// share the prefix found so far (per-lane counts packed two bins per 32-bit word, then eight
-// independent warp reductions), and keeps the digit at which the count of keys at or above the
-// threshold reaches K.  It stops as soon as that count is exactly K ({key >= T} is then the
-// answer); otherwise after the last digit T is the K-th largest key and the lowest-indexed keys
-// equal to T fill the remaining places.  Eight short passes instead of a 32-step bisection.
+// 4-bit digits.  The keys sit in registers (lane l holds positions l + 32 j).  Each pass counts
+// the next digit of the keys that share the prefix found so far: every lane keeps sixteen 4-bit
+// counters in one 64-bit word (at most 8 keys between two flushes into 16-bit fields), the eight
+// 32-bit words of 16-bit bins are summed over the warp, and the pass keeps the digit at which the
+// count of keys at or above the threshold reaches K.  It stops as soon as that count is exactly K
+// ({key >= T} is then the answer); otherwise after the last digit T is the K-th largest key and
+// the lowest-indexed keys equal to T fill the remaining places.
 // Writes the selected positions ascending to `out`; returns min(K, N).
 constexpr int kSelItems = 16;  // N <= 32 * kSelItems
+
+// count of digit d in the reduced words: parity p = d & 1 picks words 4p.., the byte k = d >> 1
+// of the nibble-split word sits in b[k & 1] as 16-bit field k >> 1 (see flush_nibbles)
+__device__ __forceinline__ int bin_count(const uint32_t (&r)[8], int d) {
+  const int p = d & 1, k = d >> 1, which = k & 1, f = k >> 1;
+  return (int)((r[p * 4 + which * 2 + (f >> 1)] >> ((f & 1) * 16)) & 0xFFFFu);
+}
+// add sixteen 4-bit counters (nibble d = count of digit d) to eight words of 16-bit bins
+__device__ __forceinline__ void flush_nibbles(uint64_t a, uint32_t (&r)[8]) {
+  const uint64_t m4 = 0x0F0F0F0F0F0F0F0Full, m8 = 0x00FF00FF00FF00FFull;
+  const uint64_t n0 = a & m4, n1 = (a >> 4) & m4;  // even digits / odd digits, one per byte
+  const uint64_t b[4] = {n0 & m8, (n0 >> 8) & m8, n1 & m8, (n1 >> 8) & m8};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    r[2 * q] += (uint32_t)b[q];
+    r[2 * q + 1] += (uint32_t)(b[q] >> 32);
+  }
+}
+
 __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
@@ -121,65 +141,69 @@ __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int 
     __syncwarp();
     return N;
   }
-  uint32_t T = 0;      // digits fixed so far (higher bits)
-  int above = 0;       // keys strictly above the prefix (they are selected)
+  const int nv = (N - lane + 31) >> 5;  // keys of this lane: positions lane + 32 j, j < nv
+  uint32_t kr[kSelItems];
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) kr[j] = j < nv ? keys[lane + 32 * j] : 0u;
+  uint32_t T = 0;  // digits fixed so far (higher bits)
+  int above = 0;   // keys strictly above the prefix (they are selected)
   bool exact = false;
   for (int shift = 28; shift >= 0 && !exact; shift -= 4) {
     const uint32_t hi_mask = shift == 28 ? 0u : (0xFFFFFFFFu << (shift + 4));
-    uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // bins 2j (low 16 bits), 2j+1 (high)
-    for (int i = lane; i < N; i += 32) {
-      const uint32_t x = keys[i];
-      if ((x & hi_mask) == T) {
-        const uint32_t d = (x >> shift) & 15u;
-        const uint32_t inc = 1u << ((d & 1u) * 16u);
+    uint32_t r[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] += (d >> 1) == (uint32_t)j ? inc : 0u;
+    for (int j0 = 0; j0 < kSelItems; j0 += 8) {
+      if (j0 > 0 && j0 >= nv) break;
+      uint64_t acc = 0;
+#pragma unroll
+      for (int j = j0; j < j0 + 8; ++j) {
+        const uint32_t x = kr[j];
+        const bool in = j < nv && (x & hi_mask) == T;
+        acc += in ? (1ull << (((x >> shift) & 15u) * 4u)) : 0ull;
       }
+      flush_nibbles(acc, r);
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) h[j] = __reduce_add_sync(0xffffffffu, h[j]);
-    // largest digit v with above + count(digit >= v) >= kk
+    for (int q = 0; q < 8; ++q) r[q] = __reduce_add_sync(0xffffffffu, r[q]);
+    // largest digit v with above + count(digit >= v) >= kk; keys with a larger digit are taken
     int run = above, v = 0, run_at_v = 0;
 #pragma unroll
     for (int d = 15; d >= 0; --d) {
-      const int c = (int)((h[d >> 1] >> ((d & 1) * 16)) & 0xFFFFu);
+      const int c = bin_count(r, d);
       if (run < kk && run + c >= kk) {
         v = d;
         run_at_v = run + c;
       }
       run += c;
     }
-    // keys with a digit above v are selected outright
     int up = above;
 #pragma unroll
-    for (int d = 15; d >= 0; --d) {
-      const int c = (int)((h[d >> 1] >> ((d & 1) * 16)) & 0xFFFFu);
-      if (d > v) up += c;
-    }
+    for (int d = 15; d >= 0; --d)
+      if (d > v) up += bin_count(r, d);
     T |= (uint32_t)v << shift;
     above = up;
     exact = (run_at_v == kk);
   }
   const int rem = kk - above;  // keys equal to the full threshold still to take (if not exact)
-  const uint32_t cmp_mask = 0xFFFFFFFFu;
   int taken = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < N; base += 32) {
-    const int i = base + lane;
-    const bool valid = i < N;
-    const uint32_t x = valid ? keys[i] : 0u;
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) {
+    if (32 * j >= N) break;  // warp-uniform
+    const bool valid = j < nv;
+    const uint32_t x = kr[j];
     bool take;
     unsigned eqb = 0u;
     if (exact) {
-      // T holds the digits down to the stopping pass; compare on those bits only
+      // T holds the digits down to the stopping pass, zeros below: x >= T compares prefixes
       take = valid && x >= T;
     } else {
-      const bool eq = valid && (x & cmp_mask) == T;
+      const bool eq = valid && x == T;
       eqb = __ballot_sync(0xffffffffu, eq);
       take = (valid && x > T) || (eq && eq_seen + __popc(eqb & lt) < rem);
     }
     const unsigned tb = __ballot_sync(0xffffffffu, take);
-    if (take) out[taken + __popc(tb & lt)] = i;
+    if (take) out[taken + __popc(tb & lt)] = 32 * j + lane;
     taken += __popc(tb);
     eq_seen += __popc(eqb);
   }

@@ -27,6 +27,12 @@ namespace bsa {
 
 bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, int H, int Hk,
                           int n, int d, int window, void* o, int* status, cudaStream_t st);
+size_t freesolo_select_tc_workspace(int B, int H, int n, int d, int cell);
+bool freesolo_select_tc_supported(bsa_dtype dt, int d, int q_block, int K);
+bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cell,
+                              const float* mean_k, const float* max_norm, const float* centre,
+                              const float* lam, const float* sig, int K, int* idx, int* count,
+                              void* ws, size_t ws_bytes, cudaStream_t st);
 
 namespace {
 
@@ -331,7 +337,8 @@ extern "C" bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, in
                                           int cell, int q_block, const float* mean_k,
                                           const float* max_norm, const float* centre,
                                           const float* lambda_h, const float* sigma_h, int K,
-                                          int* idx, int* count, void* stream) {
+                                          int* idx, int* count, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
   using namespace bsa;
   BSA_REQUIRE(dtype_ok(dt), BSA_ERR_DTYPE);
   BSA_REQUIRE(q && mean_k && max_norm && centre && lambda_h && sigma_h && idx, BSA_ERR_ARG);
@@ -341,8 +348,11 @@ extern "C" bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, in
   BSA_REQUIRE(B <= 65535 && H <= 65535, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(all_aligned16(q, mean_k), BSA_ERR_ARG);
   const int C = ceil_div(n, cell);
-  dim3 grid(ceil_div(n, kSelThreads), H, B);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (freesolo_select_tc_supported(dt, d, q_block, K))
+    return freesolo_select_tc(q, B, H, n, d, cell, mean_k, max_norm, centre, lambda_h, sigma_h, K,
+                              idx, count, workspace, workspace_bytes, st);
+  dim3 grid(ceil_div(n, kSelThreads), H, B);
   if (dt == BSA_BF16) {
     if (d == 64) launch_select<__nv_bfloat16, 64>(grid, st, q, H, n, cell, q_block, C, mean_k, max_norm, centre, lambda_h, sigma_h, K, idx, count);
     else launch_select<__nv_bfloat16, 128>(grid, st, q, H, n, cell, q_block, C, mean_k, max_norm, centre, lambda_h, sigma_h, K, idx, count);
@@ -352,6 +362,15 @@ extern "C" bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, in
   }
   BSA_LAUNCH_CHECK();
   return BSA_OK;
+}
+
+extern "C" size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d,
+                                                       int cell, int q_block, int K) {
+  using namespace bsa;
+  if (B <= 0 || H <= 0 || n <= 0 || d <= 0 || cell <= 0) return 0;
+  return freesolo_select_tc_supported(dt, d, q_block, K)
+             ? freesolo_select_tc_workspace(B, H, n, d, cell)
+             : 0;
 }
 
 extern "C" size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d) {

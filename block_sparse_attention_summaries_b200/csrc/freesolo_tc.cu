@@ -1,0 +1,438 @@
+// FreeSolo cell selection on the tensor cores: score tile Q_blk x Kbar^T (tcgen05, TMEM) with the
+// erf distance bias and the per-query Top-K in the epilogue.
+//
+// [FreeSolo] summary page, "How it works": the candidate prefix is fixed per query block of 128
+// queries, so all 128 queries of a block score the same cells:
+//     r_ic = q_i . kbar_c / sqrt(d) + lambda_h * a_c * erf((i - p_c) / (2 sigma_h)),
+// and each query keeps its K best cells.
+//
+// * One CTA per (batch, head, query block of 128): an M = 128 tile, full tcgen05 rate.
+// * The fp32 mean keys are split once into bf16 hi + lo (kbar = hi + lo to ~2^-16 relative); the
+//   product q . kbar is accumulated as Q hi^T + Q lo^T in fp32 TMEM, so the scores keep the
+//   precision the 1e-4 index bar needs while the contraction runs on bf16 tensor cores.
+// * Cells stream through a 2-stage TMA ring, 256 cells per chunk, into double-buffered TMEM.
+// * The bias of cell c for row r is a degree-4 Taylor expansion of erf around the tile's middle
+//   row, x0 = (i0 + 63.5 - p_c) / (2 sigma): the derivatives of erf are Hermite polynomials times
+//   2/sqrt(pi) exp(-x^2), so each cell needs one erf and one exp for its five coefficients, and
+//   each (row, cell) pair four FMAs.  The step t = (r - 63.5) / (2 sigma) is at most 64 / (2 sigma);
+//   the truncation error is below |t|^5 / 5! * max|erf^(5)| (about 1e-7 lambda a_c at sigma = 300).
+// * Eight epilogue warps: warp w reads TMEM lanes 32 (w % 4) .. and column half w / 4; each keeps
+//   a register Top-K list ordered by (score desc, index asc); the two halves of a row are merged
+//   at the end.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tc_common.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kRows = 128;  // queries per tile (= query block)
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsFs = (kEpiWarps + 2) * 32;
+constexpr int kTop = 8;     // every row keeps its 8 best cells; K <= 8 takes the first K
+
+struct FsTcParams {
+  int B, H, n, C, cell, K;
+  const float* max_norm;
+  const float* centre;
+  const float* lam;
+  const float* sig;
+  int* idx;
+  int* count;
+  int* status;
+};
+
+template <int D>
+struct FsTcSmem {
+  static constexpr int kNC = D == 64 ? 256 : 128;  // cells per chunk (TMEM: 2 x kNC columns)
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kChunkBytes = kNC * D * 2;  // one of hi / lo
+  static constexpr int kQ = 0;
+  static constexpr int kStage = kQBytes;
+  static constexpr int kStageBytes = 2 * kChunkBytes;
+  static constexpr int kCoef = kStage + 2 * kStageBytes;  // [2][kNC][8] floats
+  static constexpr int kMerge = kCoef + 2 * kNC * 8 * 4;  // [kEpiWarps * 32][kTop] u64
+  static constexpr int kBars = kMerge + kEpiWarps * 32 * kTop * 8;
+  static constexpr int kTotal = kBars + 256;
+};
+
+__device__ __forceinline__ uint32_t okey(float f) {
+  if (f != f) return 0u;
+  if (f == 0.f) f = 0.f;
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// sorted (descending) insertion into a register list of kTop composite keys
+__device__ __forceinline__ void top_insert(uint64_t (&best)[kTop], uint64_t x) {
+#pragma unroll
+  for (int q = 0; q < kTop; ++q) {
+    const bool gt = x > best[q];
+    const uint64_t t = best[q];
+    best[q] = gt ? x : t;
+    x = gt ? t : x;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsFs, 1)
+    freesolo_select_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+                              const __grid_constant__ CUtensorMap tmhi,
+                              const __grid_constant__ CUtensorMap tmlo, const FsTcParams p) {
+  using L = FsTcSmem<D>;
+  constexpr int kNC = L::kNC;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* fin = bars + 9;
+  float* coef = reinterpret_cast<float*>(smem + L::kCoef);
+  uint64_t* merge = reinterpret_cast<uint64_t*>(smem + L::kMerge);
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qb = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+  const int i0 = qb * kRows;
+  const int nc = min(p.C, i0 / p.cell);  // cells wholly before the query block
+  const int nchunks = (nc + kNC - 1) / kNC;
+  const size_t crow0 = ((size_t)bi * p.H + h) * p.C;
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kEpiWarps * 32);
+    }
+    mbar_init(fin, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == kEpiWarps + 1) {
+    tc::tmem_alloc(&s_tmem, 2 * kNC);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == kEpiWarps) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && nchunks > 0) {
+      mbar_arrive_expect_tx(q_full, L::kQBytes);
+      const int yq = (bi * p.H + h) * p.n + i0;
+      for (int hf = 0; hf < D / 64; ++hf)
+        tc::tma_load_2d(smem + L::kQ + hf * (kRows * 128), &tmq, hf * 64, yq, q_full);
+      int issued = 0;
+      for (int j = 0; j < nchunks; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) - 1) & 1)) {
+          s_abort = 1;
+          break;
+        }
+        issued = j + 1;
+        mbar_arrive_expect_tx(&kv_full[st], L::kStageBytes);
+        const int yc = (int)crow0 + j * kNC;
+        unsigned char* base = smem + L::kStage + st * L::kStageBytes;
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tc::tma_load_2d(base + hf * (kNC * 128), &tmhi, hf * 64, yc, &kv_full[st]);
+          tc::tma_load_2d(base + L::kChunkBytes + hf * (kNC * 128), &tmlo, hf * 64, yc,
+                          &kv_full[st]);
+        }
+      }
+      // on abort, let the loads already issued land before the CTA exits
+      if (s_abort) {
+        (void)mbar_wait_bounded(q_full, 0, 1u << 16);
+        for (int j = max(0, issued - 2); j < issued; ++j)
+          (void)mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, 1u << 16);
+      }
+    }
+  } else if (warp == kEpiWarps + 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nchunks > 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(kRows, kNC, false, false);
+      bool ok = mbar_wait_bounded(q_full, 0);
+      for (int j = 0; ok && j < nchunks; ++j) {
+        const int st = j & 1;
+        ok = mbar_wait_bounded(&kv_full[st], (j >> 1) & 1);
+        if (ok && j >= 2) ok = mbar_wait_bounded(&s_free[st], ((j >> 1) - 1) & 1);
+        if (!ok) break;
+        tc::fence_after_sync();
+        const uint32_t d_s = tmem + (uint32_t)(st * kNC);
+        const unsigned char* base = smem + L::kStage + st * L::kStageBytes;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // kbar hi, then kbar lo, into one accumulator
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int hf = kk >> 2, off = (kk & 3) * 32;
+            const uint64_t a =
+                tc::smem_desc_sw128(smem + L::kQ + hf * (kRows * 128) + off, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(
+                base + part * L::kChunkBytes + hf * (kNC * 128) + off, 16, 1024);
+            tc::mma_f16_ss(d_s, a, b, idS, (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(&s_full[st]);
+        tc::mma_commit(&kv_empty[st]);
+      }
+      if (!ok) s_abort = 1;
+      tc::mma_commit(fin);
+      if (!mbar_wait_bounded(fin, 0)) s_abort = 1;
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps
+    const int sub = warp & 3, half = warp >> 2;
+    const int row = 32 * sub + lane;
+    const int i = i0 + row;
+    const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
+    const float scale = rsqrtf((float)D);
+    const float lam = p.lam[h];
+    const float inv2s = 0.5f / p.sig[h];
+    // Taylor expansion about the tile's middle row while the step stays small (|t| <= 1/8, where
+    // the truncation is below 14 |t|^5 / 120 * lambda a_c = 4e-6 lambda a_c), else erf per pair.
+    const bool taylor = 64.f * fabsf(inv2s) <= 0.125f;
+    const float t = ((float)row - 63.5f) * inv2s;
+    auto score = [&](float s, const float* cf) -> float {
+      float bias;
+      if (taylor) {
+        const float4 c03 = *reinterpret_cast<const float4*>(cf);
+        bias = fmaf(t, fmaf(t, fmaf(t, fmaf(t, cf[4], c03.w), c03.z), c03.y), c03.x);
+      } else {
+        const float2 lp = *reinterpret_cast<const float2*>(cf + 6);
+        bias = lp.x * erff(((float)i - lp.y) * inv2s);
+      }
+      return fmaf(s, scale, bias);
+    };
+    // best: this row's 8 best (score, cell) so far as composite keys (order key << 32 | ~cell),
+    // descending; thr: the score of best[7] (-inf while a slot is empty).  The hot loop only
+    // flags cells with score >= thr; the flagged ones are re-read (one TMEM column each) and
+    // inserted exactly in a warp-uniform loop.
+    uint64_t best[kTop];
+#pragma unroll
+    for (int e = 0; e < kTop; ++e) best[e] = 0ull;
+    float thr = -INFINITY;
+    auto scan32 = [&](const float (&sv)[32], const float* cfb, int cbase) -> uint32_t {
+      uint32_t hit = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float r = score(sv[e], cfb + e * 8);
+        hit |= !(r < thr) ? (1u << e) : 0u;
+      }
+      const int left = nc - cbase;
+      return left >= 32 ? hit : (hit & ((1u << left) - 1u));
+    };
+    auto insert_flagged = [&](uint32_t hit, uint32_t col, const float* cfb, int cbase) {
+      unsigned any = __reduce_or_sync(0xffffffffu, hit);
+      while (any) {
+        const int e = __ffs(any) - 1;
+        any &= any - 1u;
+        float s1 = tc::tmem_ld1(tmem + lane_base + col + (uint32_t)e);
+        tc::tmem_wait_ld();
+        tc::reg_fence1(s1);
+        if ((hit >> e) & 1u) {
+          const float r = score(s1, cfb + e * 8);
+          const uint32_t c = (uint32_t)(cbase + e);
+          const uint64_t comp = ((uint64_t)okey(r) << 32) | (uint64_t)(0xFFFFFFFFu - c);
+          if (comp > best[kTop - 1]) {
+            top_insert(best, comp);
+            const uint32_t k7 = (uint32_t)(best[kTop - 1] >> 32);
+            thr = k7 == 0u ? -INFINITY
+                           : __uint_as_float((k7 & 0x80000000u) ? (k7 & 0x7FFFFFFFu) : ~k7);
+          }
+        }
+      }
+    };
+    bool ok = true;
+    for (int j = 0; j < nchunks; ++j) {
+      const int st = j & 1;
+      // coefficients of this chunk's cells, one cell per thread (kNC <= 256 epilogue threads);
+      // slot k < 5 holds lambda a_c erf^(k)(x0) / k!, slot 6 lambda a_c, slot 7 p_c
+      if (tid < kNC) {
+        const int c = j * kNC + tid;
+        float* cf = coef + ((size_t)st * kNC + tid) * 8;
+        if (c < nc) {
+          const float la = lam * p.max_norm[crow0 + c];
+          const float pc = p.centre[crow0 + c];
+          if (taylor) {
+            const float x = ((float)i0 + 63.5f - pc) * inv2s;
+            const float x2 = x * x;
+            const float e = 1.1283791670955126f * expf(-x2);  // first derivative of erf
+            cf[0] = la * erff(x);
+            cf[1] = la * e;
+            cf[2] = la * (-x * e);
+            cf[3] = la * ((4.f * x2 - 2.f) * e) * (1.f / 6.f);
+            cf[4] = la * ((12.f * x - 8.f * x2 * x) * e) * (1.f / 24.f);
+          }
+          cf[6] = la;
+          cf[7] = pc;
+        }
+      }
+      // every epilogue warp passes this barrier once per chunk, also after a failed wait
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
+      ok = __all_sync(0xffffffffu, ok && !*reinterpret_cast<volatile int*>(&s_abort));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
+      tc::fence_after_sync();
+      const int colh = half * (kNC / 2);
+      // two 32-column groups per step: the second group's TMEM load overlaps the first's scan
+#pragma unroll 1
+      for (int c0 = 0; c0 < kNC / 2; c0 += 64) {
+        const int cbA = j * kNC + colh + c0;
+        if (!ok || cbA >= nc) break;  // warp-uniform
+        const uint32_t colA = (uint32_t)(st * kNC + colh + c0);
+        const float* cfA = coef + ((size_t)st * kNC + colh + c0) * 8;
+        const bool hasB = cbA + 32 < nc;
+        float svA[32], svB[32];
+        tc::tmem_ld32(tmem + lane_base + colA, svA);
+        tc::tmem_wait_ld();
+        tc::reg_fence(svA);
+        if (hasB) tc::tmem_ld32(tmem + lane_base + colA + 32u, svB);
+        insert_flagged(scan32(svA, cfA, cbA), colA, cfA, cbA);
+        if (hasB) {
+          tc::tmem_wait_ld();
+          tc::reg_fence(svB);
+          insert_flagged(scan32(svB, cfA + 32 * 8, cbA + 32), colA + 32u, cfA + 32 * 8, cbA + 32);
+        }
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&s_free[st]);
+    }
+    if (!ok) s_abort = 1;
+    // merge the two column halves of each row, order the winners by index, write
+    uint64_t* mine = merge + (size_t)tid * kTop;
+#pragma unroll
+    for (int e = 0; e < kTop; ++e) mine[e] = best[e];
+    asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
+    if (half == 0 && i < p.n) {
+      const uint64_t* other = merge + (size_t)(tid + 128) * kTop;
+#pragma unroll
+      for (int e = 0; e < kTop; ++e) top_insert(best, other[e]);
+      const int kk = min(p.K, nc);
+      int sel[kTop];
+#pragma unroll
+      for (int e = 0; e < kTop; ++e)
+        sel[e] = e < kk ? (int)(0xFFFFFFFFu - (uint32_t)(best[e] & 0xFFFFFFFFu)) : INT_MAX;
+#pragma unroll
+      for (int a = 0; a < kTop; ++a)
+#pragma unroll
+        for (int b2 = 0; b2 + 1 < kTop - a; ++b2) {
+          const int lo = min(sel[b2], sel[b2 + 1]), hi = max(sel[b2], sel[b2 + 1]);
+          sel[b2] = lo;
+          sel[b2 + 1] = hi;
+        }
+      int* out = p.idx + (((size_t)bi * p.H + h) * p.n + i) * p.K;
+#pragma unroll
+      for (int e = 0; e < kTop; ++e)
+        if (e < p.K) out[e] = e < kk ? sel[e] : -1;
+      if (p.count) p.count[((size_t)bi * p.H + h) * p.n + i] = kk;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (s_abort && tid == 0) report_timeout(p.status, 5);
+  if (warp == kEpiWarps + 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kNC);
+  }
+}
+
+// kbar (fp32) -> bf16 hi, lo with kbar ~ hi + lo
+__global__ void split_hi_lo_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ hi,
+                                   __nv_bfloat16* __restrict__ lo, long long count) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  const float v = x[i];
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[i] = h;
+  lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fs() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    else
+      (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+bool map2d(CUtensorMap* m, const void* base, long long rows, int D, int box_rows) {
+  auto enc = encode_fs();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t freesolo_select_tc_workspace(int B, int H, int n, int d, int cell) {
+  const long long C = (n + cell - 1) / cell;
+  return (size_t)256 + (size_t)2 * B * H * C * d * 2 + 256;
+}
+
+bool freesolo_select_tc_supported(bsa_dtype dt, int d, int q_block, int K) {
+  return dt == BSA_BF16 && (d == 64 || d == 128) && q_block == kRows && K <= kTop;
+}
+
+// Workspace: [0, 256) status word (zeroed by the caller before first use), then kbar hi, kbar lo.
+bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cell,
+                              const float* mean_k, const float* max_norm, const float* centre,
+                              const float* lam, const float* sig, int K, int* idx, int* count,
+                              void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int C = (n + cell - 1) / cell;
+  if (!ws || ws_bytes < freesolo_select_tc_workspace(B, H, n, d, cell)) return BSA_ERR_WORKSPACE;
+  if ((long long)B * H * n >= (1ll << 31) || (long long)B * H * C >= (1ll << 31))
+    return BSA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit
+  const long long cnt = (long long)B * H * C * d;
+  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(
+      align_up(reinterpret_cast<uintptr_t>(ws) + 256, (uintptr_t)256));
+  __nv_bfloat16* lo = hi + cnt;
+  split_hi_lo_kernel<<<(unsigned)((cnt + 255) / 256), 256, 0, st>>>(mean_k, hi, lo, cnt);
+  BSA_LAUNCH_CHECK();
+  const int nc_box = d == 64 ? FsTcSmem<64>::kNC : FsTcSmem<128>::kNC;
+  CUtensorMap tmq, tmhi, tmlo;
+  if (!map2d(&tmq, q, (long long)B * H * n, d, kRows) ||
+      !map2d(&tmhi, hi, (long long)B * H * C, d, nc_box) ||
+      !map2d(&tmlo, lo, (long long)B * H * C, d, nc_box))
+    return BSA_ERR_CUDA;
+  FsTcParams p{};
+  p.B = B; p.H = H; p.n = n; p.C = C; p.cell = cell; p.K = K;
+  p.max_norm = max_norm; p.centre = centre; p.lam = lam; p.sig = sig;
+  p.idx = idx; p.count = count; p.status = static_cast<int*>(ws);
+  const dim3 grid((n + kRows - 1) / kRows, H, B);
+  auto run = [&](auto kern, int smem) -> bsa_status {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      return BSA_ERR_CUDA;
+    }
+    kern<<<grid, kThreadsFs, smem, st>>>(tmq, tmhi, tmlo, p);
+    BSA_LAUNCH_CHECK();
+    return BSA_OK;
+  };
+  return d == 64 ? run(freesolo_select_tc_kernel<64>, FsTcSmem<64>::kTotal + 1024)
+                 : run(freesolo_select_tc_kernel<128>, FsTcSmem<128>::kTotal + 1024);
+}
+
+}  // namespace bsa

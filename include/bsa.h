@@ -218,11 +218,22 @@ bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void
  *   lambda_h, sigma_h: [H] float32 device arrays.
  *   idx       [B, H, n, K] int32 out, ascending, -1 padded; count optional [B, H, n] out.
  *   K <= 8.
+ *   workspace device scratch of bsa_freesolo_select_workspace_bytes() bytes, its first int zeroed
+ *             before first use (the status word: a bounded wait that runs out writes a nonzero
+ *             value there; bsa_workspace_status reads and clears it).  Required (else
+ *             BSA_ERR_WORKSPACE) for the tensor-core form: bf16, d in {64, 128}, q_block = 128;
+ *             it then holds the mean keys split into bf16 high and low parts.  Other forms take
+ *             no workspace (size 0; the pointer may be NULL).
  */
 bsa_status bsa_freesolo_select(const void* q, bsa_dtype dt, int B, int H, int n, int d,
                                int cell, int q_block, const float* mean_k, const float* max_norm,
                                const float* centre, const float* lambda_h, const float* sigma_h,
-                               int K, int* idx, int* count, void* stream);
+                               int K, int* idx, int* count, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Workspace bytes bsa_freesolo_select needs for these arguments (0: none). */
+size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d, int cell,
+                                           int q_block, int K);
 
 /*
  * bsa_freesolo_attn -- FreeSolo two-branch prefill output ([FreeSolo] "How it works"):

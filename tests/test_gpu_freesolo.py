@@ -63,9 +63,15 @@ def check_rows(case, idx, cnt, o, rows):
     return worst
 
 
-@pytest.mark.parametrize("window,sigma", [(100, 300.0), (512, 4096.0)])
-def test_freesolo_small(window, sigma):
-    case = inputs.freesolo_case(41, B=1, H=2, d=64, n=1000, cell=32, q_block=128, K=4,
+# sigma 300 / 4096: the tensor-core select expands erf about the tile's middle row; sigma 50:
+# erf per (query, cell) pair; d = 128: the 128-cell chunk form; q_block 64 / K 8 / fp32 paths too.
+@pytest.mark.parametrize("window,sigma,d,q_block,K", [(100, 300.0, 64, 128, 4),
+                                                      (512, 4096.0, 64, 128, 4),
+                                                      (64, 50.0, 64, 128, 8),
+                                                      (256, 1000.0, 128, 128, 3),
+                                                      (100, 300.0, 64, 64, 4)])
+def test_freesolo_small(window, sigma, d, q_block, K):
+    case = inputs.freesolo_case(41, B=1, H=2, d=d, n=1000, cell=32, q_block=q_block, K=K,
                                 window=window, sigma=sigma)
     idx, cnt, o = run_gpu(case)
     rng = np.random.default_rng(5)
@@ -73,6 +79,36 @@ def test_freesolo_small(window, sigma):
             sorted(set([0, 1, 127, 128, 129, 255, 256, 511, 640, 999]) |
                    set(rng.integers(0, 1000, 30).tolist()))]
     check_rows(case, idx, cnt, o, rows)
+
+
+def test_freesolo_select_two_batches_many_cells():
+    """B = 2, 40 cells of 16 per query block: several 256-cell chunks and a ragged last chunk."""
+    case = inputs.freesolo_case(43, B=2, H=3, d=64, n=5000, cell=16, q_block=128, K=5,
+                                window=128, sigma=2000.0)
+    idx, cnt, o = run_gpu(case)
+    rng = np.random.default_rng(9)
+    rows = [(int(b), int(h), int(i)) for b, h, i in
+            zip(rng.integers(0, 2, 24), rng.integers(0, 3, 24), rng.integers(0, 5000, 24))]
+    rows += [(1, 2, 4999), (0, 0, 4096), (1, 1, 4224)]
+    check_rows(case, idx, cnt, o, rows)
+
+
+def test_freesolo_select_status_clean():
+    case = inputs.freesolo_case(44, B=1, H=2, d=64, n=2048, cell=32, q_block=128, K=4)
+    q = torch.from_numpy(case.q).to(DEV, torch.bfloat16)
+    k = torch.from_numpy(case.k).to(DEV, torch.bfloat16)
+    lam = torch.from_numpy(case.lam).to(DEV)
+    sig = torch.from_numpy(case.sigma).to(DEV)
+    mean_k, mx, ce = bsa.build_block_summaries(k, case.cell)
+    need = int(bsa.lib().bsa_freesolo_select_workspace_bytes(bsa.BSA_BF16, 1, 2, 2048, 64, 32,
+                                                             128, 4))
+    assert need > 0
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    bsa.freesolo_select(q, mean_k, mx, ce, lam, sig, case.cell, case.q_block, case.K, ws=ws)
+    assert bsa.workspace_status(ws) == 0
+    with pytest.raises(RuntimeError):
+        bsa.freesolo_select(q, mean_k, mx, ce, lam, sig, case.cell, case.q_block, case.K,
+                            ws=ws[:need - 1])
 
 
 def test_freesolo_full_size_sampled():
