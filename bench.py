@@ -22,6 +22,8 @@ import sys
 import threading
 import time
 
+import hashlib
+
 import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +38,27 @@ WORKLOADS = {
                              needle_layout="stride", seed=3000),
 }
 
+
+
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the kernel
+# built from the source whose hash is given (the capture command is in the profile summary
+# decode_fused_kernel__sas_gqa_decode_32k.md).  Reported only while the source is unchanged.
+MEASURED_TRAFFIC = {
+    ("sas_gqa_decode_32k", "decode_fused_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
+        "sha256_16": "3a64f74fc534e67e", "bytes": 52_587_520 + 378_112},
+}
+
+
+def measured_traffic(workload: str, kernel: str):
+    rec = MEASURED_TRAFFIC.get((workload, kernel))
+    if rec is None:
+        return None
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), rec["source"])
+    with open(path, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+            return None
+    return rec["bytes"]
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -484,7 +507,8 @@ def run_gpu(args):
                    "graphs": "one CUDA graph (one fused kernel) per step"},
         "roofline": {"bound": "hbm", "kernel": "decode_fused_kernel",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": measured_traffic(args.workload, "decode_fused_kernel"),
                      "algorithmic_bytes": step_bytes + io_bytes,
                      "peak_source": peaks["source"] + " (burst copy)"},
         "hbm": {"north_star_bytes": step_bytes, "gbs": step_bytes / (avg_ms / 1e3) / 1e9,

@@ -31,7 +31,7 @@ namespace {
 constexpr int kRows = 128;  // queries per tile (= query block)
 constexpr int kEpiWarps = 8;
 constexpr int kThreadsFs = (kEpiWarps + 2) * 32;
-constexpr int kTop = 8;     // every row keeps its 8 best cells; K <= 8 takes the first K
+constexpr int kMaxTop = 8;  // K <= 8: rows keep a list of 4 (K <= 4) or 8 slots
 
 struct FsTcParams {
   int B, H, n, C, cell, K;
@@ -53,30 +53,74 @@ struct FsTcSmem {
   static constexpr int kStage = kQBytes;
   static constexpr int kStageBytes = 2 * kChunkBytes;
   static constexpr int kCoef = kStage + 2 * kStageBytes;  // [2][kNC][8] floats
-  static constexpr int kMerge = kCoef + 2 * kNC * 8 * 4;  // [kEpiWarps * 32][kTop] u64
-  static constexpr int kBars = kMerge + kEpiWarps * 32 * kTop * 8;
+  // [32][kEpiWarps * 32] floats: the scores of a thread's current 32-cell group, column tid
+  // (also the merge buffer at the end: [kMaxTop][kEpiWarps * 32] keys, then as many indices)
+  static constexpr int kStash = kCoef + 2 * kNC * 8 * 4;
+  static constexpr int kBars = kStash + 32 * kEpiWarps * 32 * 4;
   static constexpr int kTotal = kBars + 256;
 };
 
-__device__ __forceinline__ uint32_t okey(float f) {
-  if (f != f) return 0u;
+// Order key of a score plus one: 0 marks an empty slot, NaN ranks just above it (below every
+// number), -0 counts as +0; larger keys are larger scores.
+__device__ __forceinline__ uint32_t okey1(float f) {
+  if (f != f) return 1u;
   if (f == 0.f) f = 0.f;
   const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) + 1u;
+}
+__device__ __forceinline__ float okey1_to_float(uint32_t k1) {
+  const uint32_t k = k1 - 1u;
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// sorted (descending) insertion into a register list of kTop composite keys
-__device__ __forceinline__ void top_insert(uint64_t (&best)[kTop], uint64_t x) {
+// A row's KT best cells, descending by (score, then lower cell index).
+template <int KT>
+struct TopList {
+  uint32_t key[KT];
+  int idx[KT];
+  float thr;  // NaN while a slot is empty, else the score of the last slot
+  __device__ __forceinline__ void init() {
 #pragma unroll
-  for (int q = 0; q < kTop; ++q) {
-    const bool gt = x > best[q];
-    const uint64_t t = best[q];
-    best[q] = gt ? x : t;
-    x = gt ? t : x;
+    for (int q = 0; q < KT; ++q) {
+      key[q] = 0u;
+      idx[q] = -1;
+    }
+    thr = __int_as_float(0x7fc00000);
   }
-}
+  // cells offered in increasing index order: an equal key never displaces an entry
+  __device__ __forceinline__ void offer_in_order(float r, int c) {
+    uint32_t k = okey1(r);
+    if (k <= key[KT - 1]) return;
+    int ci = c;
+#pragma unroll
+    for (int q = 0; q < KT; ++q) {
+      const bool gt = k > key[q];
+      const uint32_t tk = key[q];
+      const int ti = idx[q];
+      key[q] = gt ? k : tk;
+      idx[q] = gt ? ci : ti;
+      k = gt ? tk : k;
+      ci = gt ? ti : ci;
+    }
+    thr = key[KT - 1] == 0u ? __int_as_float(0x7fc00000) : okey1_to_float(key[KT - 1]);
+  }
+  // any order: ties go to the lower index
+  __device__ __forceinline__ void offer(uint32_t k, int c) {
+    int ci = c;
+#pragma unroll
+    for (int q = 0; q < KT; ++q) {
+      const bool gt = k > key[q] || (k == key[q] && k != 0u && (unsigned)ci < (unsigned)idx[q]);
+      const uint32_t tk = key[q];
+      const int ti = idx[q];
+      key[q] = gt ? k : tk;
+      idx[q] = gt ? ci : ti;
+      k = gt ? tk : k;
+      ci = gt ? ti : ci;
+    }
+  }
+};
 
-template <int D>
+template <int D, int KT>
 __global__ void __launch_bounds__(kThreadsFs, 1)
     freesolo_select_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                               const __grid_constant__ CUtensorMap tmhi,
@@ -94,7 +138,9 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
   uint64_t* s_free = bars + 7;    // [2]
   uint64_t* fin = bars + 9;
   float* coef = reinterpret_cast<float*>(smem + L::kCoef);
-  uint64_t* merge = reinterpret_cast<uint64_t*>(smem + L::kMerge);
+  float* stash = reinterpret_cast<float*>(smem + L::kStash);
+  uint32_t* merge_key = reinterpret_cast<uint32_t*>(smem + L::kStash);
+  int* merge_idx = reinterpret_cast<int*>(smem + L::kStash) + kMaxTop * kEpiWarps * 32;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -202,55 +248,47 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
     // the truncation is below 14 |t|^5 / 120 * lambda a_c = 4e-6 lambda a_c), else erf per pair.
     const bool taylor = 64.f * fabsf(inv2s) <= 0.125f;
     const float t = ((float)row - 63.5f) * inv2s;
-    auto score = [&](float s, const float* cf) -> float {
-      float bias;
-      if (taylor) {
-        const float4 c03 = *reinterpret_cast<const float4*>(cf);
-        bias = fmaf(t, fmaf(t, fmaf(t, fmaf(t, cf[4], c03.w), c03.z), c03.y), c03.x);
-      } else {
-        const float2 lp = *reinterpret_cast<const float2*>(cf + 6);
-        bias = lp.x * erff(((float)i - lp.y) * inv2s);
-      }
-      return fmaf(s, scale, bias);
-    };
-    // best: this row's 8 best (score, cell) so far as composite keys (order key << 32 | ~cell),
-    // descending; thr: the score of best[7] (-inf while a slot is empty).  The hot loop only
-    // flags cells with score >= thr; the flagged ones are re-read (one TMEM column each) and
-    // inserted exactly in a warp-uniform loop.
-    uint64_t best[kTop];
+    // The row's list; a scan flags the cells of a 32-cell group with score above the list's
+    // threshold (all of them while a slot is empty), parks the group's scores in this thread's
+    // stash column, and the lane offers its own flagged cells in index order.
+    TopList<KT> top;
+    top.init();
+    auto insert_hits = [&](uint32_t hit, const float (&rr)[32], int cbase) {
+      const int left = nc - cbase;
+      if (left < 32) hit &= (1u << left) - 1u;
+      if (!hit) return;
 #pragma unroll
-    for (int e = 0; e < kTop; ++e) best[e] = 0ull;
-    float thr = -INFINITY;
-    auto scan32 = [&](const float (&sv)[32], const float* cfb, int cbase) -> uint32_t {
+      for (int e = 0; e < 32; ++e) stash[e * (kEpiWarps * 32) + tid] = rr[e];
+      while (hit) {
+        const int e = __ffs(hit) - 1;
+        hit &= hit - 1u;
+        top.offer_in_order(stash[e * (kEpiWarps * 32) + tid], cbase + e);
+      }
+    };
+    // the two bias forms are separate straight-line loops so the one that runs stays small
+    auto scan_taylor = [&](const float (&sv)[32], const float* cfb, int cbase) {
+      float rr[32];
       uint32_t hit = 0u;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float r = score(sv[e], cfb + e * 8);
-        hit |= !(r < thr) ? (1u << e) : 0u;
+        const float* cf = cfb + e * 8;
+        const float4 c03 = *reinterpret_cast<const float4*>(cf);
+        const float bias = fmaf(t, fmaf(t, fmaf(t, fmaf(t, cf[4], c03.w), c03.z), c03.y), c03.x);
+        rr[e] = fmaf(sv[e], scale, bias);
+        hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
       }
-      const int left = nc - cbase;
-      return left >= 32 ? hit : (hit & ((1u << left) - 1u));
+      insert_hits(hit, rr, cbase);
     };
-    auto insert_flagged = [&](uint32_t hit, uint32_t col, const float* cfb, int cbase) {
-      unsigned any = __reduce_or_sync(0xffffffffu, hit);
-      while (any) {
-        const int e = __ffs(any) - 1;
-        any &= any - 1u;
-        float s1 = tc::tmem_ld1(tmem + lane_base + col + (uint32_t)e);
-        tc::tmem_wait_ld();
-        tc::reg_fence1(s1);
-        if ((hit >> e) & 1u) {
-          const float r = score(s1, cfb + e * 8);
-          const uint32_t c = (uint32_t)(cbase + e);
-          const uint64_t comp = ((uint64_t)okey(r) << 32) | (uint64_t)(0xFFFFFFFFu - c);
-          if (comp > best[kTop - 1]) {
-            top_insert(best, comp);
-            const uint32_t k7 = (uint32_t)(best[kTop - 1] >> 32);
-            thr = k7 == 0u ? -INFINITY
-                           : __uint_as_float((k7 & 0x80000000u) ? (k7 & 0x7FFFFFFFu) : ~k7);
-          }
-        }
+    auto scan_direct = [&](const float (&sv)[32], const float* cfb, int cbase) {
+      float rr[32];
+      uint32_t hit = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2 lp = *reinterpret_cast<const float2*>(cfb + e * 8 + 6);
+        rr[e] = fmaf(sv[e], scale, lp.x * erff(((float)i - lp.y) * inv2s));
+        hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
       }
+      insert_hits(hit, rr, cbase);
     };
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
@@ -283,55 +321,53 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       tc::fence_after_sync();
       const int colh = half * (kNC / 2);
-      // two 32-column groups per step: the second group's TMEM load overlaps the first's scan
 #pragma unroll 1
-      for (int c0 = 0; c0 < kNC / 2; c0 += 64) {
-        const int cbA = j * kNC + colh + c0;
-        if (!ok || cbA >= nc) break;  // warp-uniform
-        const uint32_t colA = (uint32_t)(st * kNC + colh + c0);
-        const float* cfA = coef + ((size_t)st * kNC + colh + c0) * 8;
-        const bool hasB = cbA + 32 < nc;
-        float svA[32], svB[32];
-        tc::tmem_ld32(tmem + lane_base + colA, svA);
+      for (int c0 = 0; c0 < kNC / 2; c0 += 32) {
+        const int cb = j * kNC + colh + c0;
+        if (!ok || cb >= nc) break;  // warp-uniform
+        const uint32_t col = (uint32_t)(st * kNC + colh + c0);
+        const float* cfb = coef + ((size_t)st * kNC + colh + c0) * 8;
+        float sv[32];
+        tc::tmem_ld32(tmem + lane_base + col, sv);
         tc::tmem_wait_ld();
-        tc::reg_fence(svA);
-        if (hasB) tc::tmem_ld32(tmem + lane_base + colA + 32u, svB);
-        insert_flagged(scan32(svA, cfA, cbA), colA, cfA, cbA);
-        if (hasB) {
-          tc::tmem_wait_ld();
-          tc::reg_fence(svB);
-          insert_flagged(scan32(svB, cfA + 32 * 8, cbA + 32), colA + 32u, cfA + 32 * 8, cbA + 32);
-        }
+        tc::reg_fence(sv);
+        if (taylor)
+          scan_taylor(sv, cfb, cb);
+        else
+          scan_direct(sv, cfb, cb);
       }
       tc::fence_before_sync();
       mbar_arrive(&s_free[st]);
     }
     if (!ok) s_abort = 1;
     // merge the two column halves of each row, order the winners by index, write
-    uint64_t* mine = merge + (size_t)tid * kTop;
+    asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));  // stash free: merge reuses it
 #pragma unroll
-    for (int e = 0; e < kTop; ++e) mine[e] = best[e];
+    for (int e = 0; e < KT; ++e) {
+      merge_key[e * (kEpiWarps * 32) + tid] = top.key[e];
+      merge_idx[e * (kEpiWarps * 32) + tid] = top.idx[e];
+    }
     asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
     if (half == 0 && i < p.n) {
-      const uint64_t* other = merge + (size_t)(tid + 128) * kTop;
 #pragma unroll
-      for (int e = 0; e < kTop; ++e) top_insert(best, other[e]);
+      for (int e = 0; e < KT; ++e)
+        top.offer(merge_key[e * (kEpiWarps * 32) + tid + 128],
+                  merge_idx[e * (kEpiWarps * 32) + tid + 128]);
       const int kk = min(p.K, nc);
-      int sel[kTop];
+      int sel[KT];
 #pragma unroll
-      for (int e = 0; e < kTop; ++e)
-        sel[e] = e < kk ? (int)(0xFFFFFFFFu - (uint32_t)(best[e] & 0xFFFFFFFFu)) : INT_MAX;
+      for (int e = 0; e < KT; ++e) sel[e] = e < kk ? top.idx[e] : INT_MAX;
 #pragma unroll
-      for (int a = 0; a < kTop; ++a)
+      for (int a = 0; a < KT; ++a)
 #pragma unroll
-        for (int b2 = 0; b2 + 1 < kTop - a; ++b2) {
+        for (int b2 = 0; b2 + 1 < KT - a; ++b2) {
           const int lo = min(sel[b2], sel[b2 + 1]), hi = max(sel[b2], sel[b2 + 1]);
           sel[b2] = lo;
           sel[b2 + 1] = hi;
         }
       int* out = p.idx + (((size_t)bi * p.H + h) * p.n + i) * p.K;
 #pragma unroll
-      for (int e = 0; e < kTop; ++e)
+      for (int e = 0; e < KT; ++e)
         if (e < p.K) out[e] = e < kk ? sel[e] : -1;
       if (p.count) p.count[((size_t)bi * p.H + h) * p.n + i] = kk;
     }
@@ -392,7 +428,7 @@ size_t freesolo_select_tc_workspace(int B, int H, int n, int d, int cell) {
 }
 
 bool freesolo_select_tc_supported(bsa_dtype dt, int d, int q_block, int K) {
-  return dt == BSA_BF16 && (d == 64 || d == 128) && q_block == kRows && K <= kTop;
+  return dt == BSA_BF16 && (d == 64 || d == 128) && q_block == kRows && K <= kMaxTop;
 }
 
 // Workspace: [0, 256) status word (zeroed by the caller before first use), then kbar hi, kbar lo.
@@ -431,8 +467,11 @@ bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cel
     BSA_LAUNCH_CHECK();
     return BSA_OK;
   };
-  return d == 64 ? run(freesolo_select_tc_kernel<64>, FsTcSmem<64>::kTotal + 1024)
-                 : run(freesolo_select_tc_kernel<128>, FsTcSmem<128>::kTotal + 1024);
+  if (d == 64)
+    return K <= 4 ? run(freesolo_select_tc_kernel<64, 4>, FsTcSmem<64>::kTotal + 1024)
+                  : run(freesolo_select_tc_kernel<64, 8>, FsTcSmem<64>::kTotal + 1024);
+  return K <= 4 ? run(freesolo_select_tc_kernel<128, 4>, FsTcSmem<128>::kTotal + 1024)
+                : run(freesolo_select_tc_kernel<128, 8>, FsTcSmem<128>::kTotal + 1024);
 }
 
 }  // namespace bsa

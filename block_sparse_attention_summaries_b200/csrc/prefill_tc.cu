@@ -311,31 +311,47 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const bool filler = !is_cur && j >= s_cnt[it];
       const float bias = (!is_cur && !filler) ? s_bias[it][j] : 0.f;
       const int kpos0 = step_block(it, j) * kTiles;  // position of this block's first key
-      float mx = -INFINITY;
+      // keys of this block the row may see: all of a history block; none of a filler; c <= r on
+      // the diagonal; c >= wlo - kpos0 inside a sliding window
+      uint64_t keep = filler ? 0ull : ~0ull;
+      if (is_cur) keep &= r >= 63 ? ~0ull : ((2ull << r) - 1ull);
+      if (wlo - kpos0 > 0) keep &= wlo - kpos0 >= 64 ? 0ull : (~0ull << (wlo - kpos0));
+      // z in log2 units; the row max by a 4-way tree
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (keep == ~0ull) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float z = fmaf(x[c], qk_scale, bias);
-        if (filler || (is_cur && c > r) || kpos0 + c < wlo) z = -INFINITY;
-        x[c] = z;
-        mx = fmaxf(mx, z);
+        for (int c = 0; c < 64; ++c) {
+          x[c] = fmaf(x[c], qk_scale, bias);
+          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = ((keep >> c) & 1ull) ? fmaf(x[c], qk_scale, bias) : -INFINITY;
+          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+        }
       }
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_new = fmaxf(m_run, mx);
       const bool rescale = m_run == -INFINITY ? (m_new != -INFINITY) : (m_new > m_run + kRescale);
       float corr = 1.f;
       if (rescale) {
-        corr = m_run == -INFINITY ? 0.f : exp2f(m_run - m_new);
+        corr = m_run == -INFINITY ? 0.f : tc::ex2_approx(m_run - m_new);
         m_run = m_new;
       }
-      float sum = 0.f;
+      // masked keys hold -inf and give 2^-inf = 0; a row with nothing seen yet subtracts 0
+      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_run);
-        const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_run);
-        sum += p0 + p1;
+        const float p0 = tc::ex2_approx(x[c] - m_use);
+        const float p1 = tc::ex2_approx(x[c + 1] - m_use);
+        sum4[(c >> 1) & 3] += p0 + p1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run = l_run * corr + sum;
       if (j > 0) {
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
@@ -632,8 +648,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         mbar_arrive(&s_free[st]);
         float t = 0.f;
         if (live && j < s_cnt[it]) {
+          float t4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 64; ++c) t = fmaf(exp2f(fmaf(z[c], zs, -lse2)), dv[c] - Di, t);
+          for (int c = 0; c < 64; ++c)
+            t4[c & 3] = fmaf(tc::ex2_approx(fmaf(z[c], zs, -lse2)), dv[c] - Di, t4[c & 3]);
+          t = (t4[0] + t4[1]) + (t4[2] + t4[3]);
         }
         // sum over the 16 rows of this unit held by this warp, then across warps
 #pragma unroll

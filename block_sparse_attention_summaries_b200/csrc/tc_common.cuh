@@ -88,6 +88,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// 2^x by the MUFU approximation (relative error about 2^-22; 2^-inf = +0), flushing subnormals.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // One column: lane i of the warp's 32-lane group gets column `taddr` of its lane.
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   uint32_t r;
