@@ -34,7 +34,8 @@ namespace {
 
 constexpr int kTiles = 64;         // queries per unit = keys per block
 constexpr int kMaxKtc = 64;        // selected history blocks per unit
-constexpr int kThreadsTc = 192;    // 4 softmax warps + producer + MMA
+constexpr int kThreadsTc = 192;    // gate gradient: 4 reduction warps + producer + MMA
+constexpr int kThreadsFwd = 224;   // forward: 4 softmax warps + K producer + MMA + V producer
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.f;    // lazy rescale threshold (log2 units)
@@ -57,17 +58,18 @@ template <int D>
 struct TcSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTiles * D * 2;  // one [64 x D] bf16 tile
+  static constexpr int kKSlots = 3;                  // K ring: freed when S_j completes
+  static constexpr int kVSlots = 2;                  // V ring: freed when P_j V_j completes
   static constexpr int kQ = 0;                       // 2 query tiles
-  static constexpr int kStage = 2 * kTileBytes;      // stages: K0 V0 K1 V1
-  static constexpr int kStageBytes = 4 * kTileBytes;
-  static constexpr int kP = kStage + 2 * kStageBytes;  // 2 P tiles [64 x 64] bf16
+  static constexpr int kK = 2 * kTileBytes;          // [kKSlots][2 units]
+  static constexpr int kV = kK + kKSlots * 2 * kTileBytes;  // [kVSlots][2 units]
+  static constexpr int kP = kV + kVSlots * 2 * kTileBytes;  // [2 buffers][2 units] [64 x 64] bf16
   static constexpr int kPBytes = kTiles * 64 * 2;
-  static constexpr int kBars = kP + 2 * kPBytes;
-  static constexpr int kTotal = kBars + 1024;
+  static constexpr int kTotal = kP + 4 * kPBytes;  // mbarriers live in static shared memory
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(kThreadsFwd, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const TcParams p) {
@@ -76,21 +78,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   // 1024-byte alignment of the swizzled tiles
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  __shared__ __align__(8) uint64_t bars[20];
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* o_done = bars + 10;
-  uint64_t* fin = bars + 11;
+  uint64_t* k_full = bars + 1;    // [3]
+  uint64_t* k_empty = bars + 4;   // [3]
+  uint64_t* v_full = bars + 7;    // [2]
+  uint64_t* v_empty = bars + 9;   // [2]
+  uint64_t* s_full = bars + 11;   // [2]
+  uint64_t* s_free = bars + 13;   // [2]
+  uint64_t* p_full = bars + 15;   // [2] per P buffer
+  uint64_t* o_done = bars + 17;   // [2] P_j V_j done, per P buffer
+  uint64_t* fin = bars + 19;
 
   __shared__ uint32_t s_tmem;
   __shared__ int s_blk[2][kMaxKtc + 1];
   __shared__ float s_bias[2][kMaxKtc + 1];
   __shared__ int s_cnt[2];
-  __shared__ int s_steps;
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -158,14 +161,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
   if (tid == 0) {
     mbar_init(q_full, 1);
+    for (int i = 0; i < L::kKSlots; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     fence_mbar_init();
     s_abort = 0;
@@ -190,42 +197,47 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   };
 
   unsigned char* sq[2] = {smem + L::kQ, smem + L::kQ + L::kTileBytes};
-  auto stage_tile = [&](int st, int which) {  // which: 0 K0, 1 V0, 2 K1, 3 V1
-    return smem + L::kStage + st * L::kStageBytes + which * L::kTileBytes;
-  };
-  unsigned char* sp[2] = {smem + L::kP, smem + L::kP + L::kPBytes};
+  auto ktile = [&](int slot, int it) { return smem + L::kK + (2 * slot + it) * L::kTileBytes; };
+  auto vtile = [&](int slot, int it) { return smem + L::kV + (2 * slot + it) * L::kTileBytes; };
+  auto ptile = [&](int buf, int it) { return smem + L::kP + (2 * buf + it) * L::kPBytes; };
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- TMA producer
+  if (warp == 4 || warp == 6) {
+    // ------------------------------------------------ TMA producers: warp 4 Q and K, warp 6 V
+    // Each runs ahead as far as its ring allows: K_j once S_{j-3} completed, V_j once
+    // P_{j-2} V_{j-2} completed.
     if (lane == 0) {
-      mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
-      for (int it = 0; it < 2; ++it) {
-        const int y = ((bi * p.Hq + hq[it]) * p.n) + uu[it] * kTiles;
-        for (int hf = 0; hf < L::kHalves; ++hf)
-          tc::tma_load_2d(sq[it] + hf * 8192, &tmq, hf * 64, y, q_full);
+      const bool is_k = warp == 4;
+      if (is_k) {
+        mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+        for (int it = 0; it < 2; ++it) {
+          const int y = ((bi * p.Hq + hq[it]) * p.n) + uu[it] * kTiles;
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            tc::tma_load_2d(sq[it] + hf * 8192, &tmq, hf * 64, y, q_full);
+        }
       }
+      const int nslots = is_k ? L::kKSlots : L::kVSlots;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const CUtensorMap* tm = is_k ? &tmk : &tmv;
       int issued = 0;
       for (int j = 0; j < steps; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) - 1) & 1)) {
+        const int sl = j % nslots;
+        if (j >= nslots && !mbar_wait_bounded(&empty[sl], ((j / nslots) - 1) & 1)) {
           s_abort = 1;
           break;
         }
-        issued = j + 1;
-        mbar_arrive_expect_tx(&kv_full[st], 4 * L::kTileBytes);
+        mbar_arrive_expect_tx(&full[sl], 2 * L::kTileBytes);
         for (int it = 0; it < 2; ++it) {
           const int y = ((bi * p.Hk + kh) * p.n) + step_block(it, j) * kTiles;
-          for (int hf = 0; hf < L::kHalves; ++hf) {
-            tc::tma_load_2d(stage_tile(st, 2 * it) + hf * 8192, &tmk, hf * 64, y, &kv_full[st]);
-            tc::tma_load_2d(stage_tile(st, 2 * it + 1) + hf * 8192, &tmv, hf * 64, y,
-                            &kv_full[st]);
-          }
+          unsigned char* dst = is_k ? ktile(sl, it) : vtile(sl, it);
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            tc::tma_load_2d(dst + hf * 8192, tm, hf * 64, y, &full[sl]);
         }
+        issued = j + 1;
       }
-      if (s_abort) {  // loads still in flight land before the CTA leaves
-        for (int j = max(0, issued - 2); j < issued; ++j)
-          (void)mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1, 1u << 16);
-      }
+      if (s_abort)  // loads still in flight land before the CTA leaves
+        for (int j = max(0, issued - nslots); j < issued; ++j)
+          (void)mbar_wait_bounded(&full[j % nslots], (j / nslots) & 1, 1u << 16);
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
@@ -233,10 +245,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(64, D, false, true);
       auto issue_s = [&](int j) {
-        const int st = j & 1;
+        const int st = j & 1, sl = j % L::kKSlots;
         for (int it = 0; it < 2; ++it) {
           const uint32_t d_s = tmem + (uint32_t)(st * 64) + ((uint32_t)(16 * it) << 16);
-          const unsigned char* kt = stage_tile(st, 2 * it);
+          const unsigned char* kt = ktile(sl, it);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const int hf = kk >> 2, off = (kk & 3) * 32;
@@ -246,39 +258,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
         tc::mma_commit(&s_full[st]);
+        tc::mma_commit(&k_empty[sl]);
       };
-      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&kv_full[0], 0);
+      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
       if (ok) {
         tc::fence_after_sync();
         issue_s(0);
       }
       for (int j = 0; ok && j < steps; ++j) {
-        if (j + 1 < steps) {
-          const int st1 = (j + 1) & 1;
-          ok = mbar_wait_bounded(&kv_full[st1], ((j + 1) >> 1) & 1);
-          if (ok && j + 1 >= 2) ok = mbar_wait_bounded(&s_free[st1], (((j + 1) >> 1) - 1) & 1);
+        if (j + 1 < steps) {  // S_{j+1} one step ahead of the softmax
+          const int j1 = j + 1;
+          ok = mbar_wait_bounded(&k_full[j1 % L::kKSlots], (j1 / L::kKSlots) & 1);
+          if (ok && j1 >= 2) ok = mbar_wait_bounded(&s_free[j1 & 1], ((j1 >> 1) - 1) & 1);
           if (!ok) break;
           tc::fence_after_sync();
-          issue_s(j + 1);
+          issue_s(j1);
         }
-        if (!mbar_wait_bounded(p_full, j & 1)) {
-          ok = false;
-          break;
-        }
+        const int pb = j & 1;
+        ok = mbar_wait_bounded(&p_full[pb], (j >> 1) & 1) &&
+             mbar_wait_bounded(&v_full[pb], (j >> 1) & 1);
+        if (!ok) break;
         tc::fence_after_sync();
-        const int st = j & 1;
         for (int it = 0; it < 2; ++it) {
           const uint32_t d_o = tmem + 128u + ((uint32_t)(16 * it) << 16);
-          const unsigned char* vt = stage_tile(st, 2 * it + 1);
+          const unsigned char* vt = vtile(pb, it);
+          const unsigned char* pt = ptile(pb, it);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 64 keys in steps of 16
-            const uint64_t a = tc::smem_desc_sw128(sp[it] + kk * 32, 16, 1024);
+            const uint64_t a = tc::smem_desc_sw128(pt + kk * 32, 16, 1024);
             const uint64_t b = tc::smem_desc_sw128(vt + kk * 2048, 8192, 1024);
             tc::mma_f16_ss(d_o, a, b, idO, (j > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        tc::mma_commit(o_done);
-        tc::mma_commit(&kv_empty[st]);
+        tc::mma_commit(&o_done[pb]);
+        tc::mma_commit(&v_empty[pb]);
       }
       if (!ok) s_abort = 1;
       // drain: every MMA this thread issued has completed before TMEM is released
@@ -353,13 +366,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run = l_run * corr + sum;
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
-        if (!ok) break;
-        tc::fence_after_sync();
+      // O may be rescaled only after P_{j-1} V_{j-1} completed; P buffer j & 1 may be rewritten
+      // once P_{j-2} V_{j-2} completed (implied by the former)
+      const bool any_rescale = j > 0 && __any_sync(0xffffffffu, rescale);
+      if (any_rescale) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
+      } else if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_done[j & 1], ((j - 2) >> 1) & 1));
+      }
+      if (!ok) break;
+      tc::fence_after_sync();
+      {
         // O row *= corr; the TMEM round trip is warp-wide (.sync.aligned), lanes that keep their
         // max multiply by 1
-        if (__any_sync(0xffffffffu, rescale)) {
+        if (any_rescale) {
           if (!rescale) corr = 1.f;
           for (int c0 = 0; c0 < D; c0 += 32) {
             float ov[32];
@@ -373,7 +393,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
       }
       // P row -> shared memory, 128-byte swizzled K-major [64 x 64]
-      unsigned char* prow = sp[it];
+      unsigned char* prow = ptile(j & 1, it);
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         const uint4 w4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
@@ -381,10 +401,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       fence_proxy_async();
       tc::fence_before_sync();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
     // epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (steps - 1) & 1));
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&o_done[(steps - 1) & 1], ((steps - 1) >> 1) & 1));
     if (ok) {
       tc::fence_after_sync();
       const bool live = i < p.n && item_ok[it];
@@ -725,7 +747,7 @@ bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams
     return BSA_ERR_CUDA;
   }
   dim3 grid = p.mode == 1 ? dim3((p.U + 1) / 2, p.Hq, p.B) : dim3(p.U, p.Hq / 2, p.B);
-  kern<<<grid, kThreadsTc, smem, st>>>(tmq, tmk, tmv, p);
+  kern<<<grid, kThreadsFwd, smem, st>>>(tmq, tmk, tmv, p);
   return BSA_OK;
 }
 
