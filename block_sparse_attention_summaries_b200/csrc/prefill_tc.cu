@@ -60,8 +60,11 @@ struct TcSmem {
   static constexpr int kTileBytes = kTiles * D * 2;  // one [64 x D] bf16 tile
   static constexpr int kKSlots = 3;                  // K ring: freed when S_j completes
   static constexpr int kVSlots = 2;                  // V ring: freed when P_j V_j completes
-  static constexpr int kQ = 0;                       // 2 query tiles
-  static constexpr int kK = 2 * kTileBytes;          // [kKSlots][2 units]
+  // queries: [half][128 rows x 128 B], unit it's row r at row 32 (r / 16) + 16 it + r % 16, the
+  // lane order of the M = 64 accumulators; K slot: [half][128 rows], unit 0 rows 0-63, unit 1
+  // rows 64-127 -- so one M = 128, N = 128 MMA chain gives both units' scores
+  static constexpr int kQ = 0;
+  static constexpr int kK = 2 * kTileBytes;          // [kKSlots][half][2 units x 64 rows]
   static constexpr int kV = kK + kKSlots * 2 * kTileBytes;  // [kVSlots][2 units]
   static constexpr int kP = kV + kVSlots * 2 * kTileBytes;  // [2 buffers][2 units] [64 x 64] bf16
   static constexpr int kPBytes = kTiles * 64 * 2;
@@ -177,8 +180,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     fence_mbar_init();
     s_abort = 0;
   }
-  if (warp == 5) {
-    tc::tmem_alloc(&s_tmem, 256);
+  if (warp == 5) {  // S: 2 x 128 columns, O: D columns at 256
+    tc::tmem_alloc(&s_tmem, 512);
     tc::tmem_relinquish();
   }
   if (warp == 4 && lane == 0) {
@@ -196,8 +199,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     return j < s_cnt[it] ? s_blk[it][j] : (item_ok[it] ? uu[it] : uu[0]);
   };
 
-  unsigned char* sq[2] = {smem + L::kQ, smem + L::kQ + L::kTileBytes};
-  auto ktile = [&](int slot, int it) { return smem + L::kK + (2 * slot + it) * L::kTileBytes; };
+  auto kslot = [&](int slot) { return smem + L::kK + slot * 2 * L::kTileBytes; };
   auto vtile = [&](int slot, int it) { return smem + L::kV + (2 * slot + it) * L::kTileBytes; };
   auto ptile = [&](int buf, int it) { return smem + L::kP + (2 * buf + it) * L::kPBytes; };
 
@@ -207,12 +209,14 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // P_{j-2} V_{j-2} completed.
     if (lane == 0) {
       const bool is_k = warp == 4;
-      if (is_k) {
+      if (is_k) {  // 16-row boxes into the accumulator lane order
         mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
         for (int it = 0; it < 2; ++it) {
           const int y = ((bi * p.Hq + hq[it]) * p.n) + uu[it] * kTiles;
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tc::tma_load_2d(sq[it] + hf * 8192, &tmq, hf * 64, y, q_full);
+            for (int b4 = 0; b4 < 4; ++b4)
+              tc::tma_load_2d(smem + L::kQ + hf * 16384 + (32 * b4 + 16 * it) * 128, &tmq,
+                              hf * 64, y + 16 * b4, q_full);
         }
       }
       const int nslots = is_k ? L::kKSlots : L::kVSlots;
@@ -229,9 +233,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         mbar_arrive_expect_tx(&full[sl], 2 * L::kTileBytes);
         for (int it = 0; it < 2; ++it) {
           const int y = ((bi * p.Hk + kh) * p.n) + step_block(it, j) * kTiles;
-          unsigned char* dst = is_k ? ktile(sl, it) : vtile(sl, it);
+          unsigned char* dst = is_k ? kslot(sl) + it * 8192 : vtile(sl, it);
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tc::tma_load_2d(dst + hf * 8192, tm, hf * 64, y, &full[sl]);
+            tc::tma_load_2d(dst + hf * (is_k ? 16384 : 8192), tm, hf * 64, y, &full[sl]);
         }
         issued = j + 1;
       }
@@ -242,20 +246,20 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+      constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(64, D, false, true);
+      // S_j = [Q_0; Q_1] [K_0; K_1]^T as one M = 128, N = 128 chain (full tensor-core rate);
+      // the cross products Q_0 K_1^T, Q_1 K_0^T land in columns the softmax ignores
       auto issue_s = [&](int j) {
         const int st = j & 1, sl = j % L::kKSlots;
-        for (int it = 0; it < 2; ++it) {
-          const uint32_t d_s = tmem + (uint32_t)(st * 64) + ((uint32_t)(16 * it) << 16);
-          const unsigned char* kt = ktile(sl, it);
+        const uint32_t d_s = tmem + (uint32_t)(st * 128);
+        const unsigned char* kb = kslot(sl);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int hf = kk >> 2, off = (kk & 3) * 32;
-            const uint64_t a = tc::smem_desc_sw128(sq[it] + hf * 8192 + off, 16, 1024);
-            const uint64_t b = tc::smem_desc_sw128(kt + hf * 8192 + off, 16, 1024);
-            tc::mma_f16_ss(d_s, a, b, idS, kk > 0);
-          }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int hf = kk >> 2, off = (kk & 3) * 32;
+          const uint64_t a = tc::smem_desc_sw128(smem + L::kQ + hf * 16384 + off, 16, 1024);
+          const uint64_t b = tc::smem_desc_sw128(kb + hf * 16384 + off, 16, 1024);
+          tc::mma_f16_ss(d_s, a, b, idS, kk > 0);
         }
         tc::mma_commit(&s_full[st]);
         tc::mma_commit(&k_empty[sl]);
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         if (!ok) break;
         tc::fence_after_sync();
         for (int it = 0; it < 2; ++it) {
-          const uint32_t d_o = tmem + 128u + ((uint32_t)(16 * it) << 16);
+          const uint32_t d_o = tmem + 256u + ((uint32_t)(16 * it) << 16);
           const unsigned char* vt = vtile(pb, it);
           const unsigned char* pt = ptile(pb, it);
 #pragma unroll
@@ -313,10 +317,19 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       if (!ok) break;
       tc::fence_after_sync();
+      // this row's 64 scores: columns 64 it .. 64 it + 63 of the score tile (the load is
+      // warp-wide, so both units' column ranges are read and each lane keeps its own)
       float x[64];
-      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 64), x);
-      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 64 + 32), x + 32);
-      tc::tmem_wait_ld();
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float t[32];
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 32 * hh), x + 32 * hh);
+        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 64 + 32 * hh), t);
+        tc::tmem_wait_ld();
+        tc::reg_fence(t);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) x[32 * hh + c] = it ? t[c] : x[32 * hh + c];
+      }
       tc::fence_before_sync();
       mbar_arrive(&s_free[st]);
       // bias or mask of this step's block for my unit
@@ -383,11 +396,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           if (!rescale) corr = 1.f;
           for (int c0 = 0; c0 < D; c0 += 32) {
             float ov[32];
-            tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+            tc::tmem_ld32(tmem + lane_base + 256u + (uint32_t)c0, ov);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) ov[c] *= corr;
-            tc::tmem_st32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+            tc::tmem_st32(tmem + lane_base + 256u + (uint32_t)c0, ov);
           }
           tc::tmem_wait_st();
         }
@@ -415,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow * D;
       for (int c0 = 0; c0 < D; c0 += 32) {
         float ov[32];
-        tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+        tc::tmem_ld32(tmem + lane_base + 256u + (uint32_t)c0, ov);
         tc::tmem_wait_ld();
         if (live) {
 #pragma unroll
@@ -446,7 +459,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   if (s_abort && tid == 0) report_timeout(p.status, 3);
   if (warp == 5) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -718,13 +731,14 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D map over a [rows, D] bf16 row-major tensor, 64x64 boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int D) {
+// 2-D map over a [rows, D] bf16 row-major tensor, boxes of 64 columns x box_rows rows,
+// 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int D, int box_rows = 64) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -735,7 +749,7 @@ template <int D>
 bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams& p,
                      cudaStream_t st) {
   CUtensorMap tmq, tmk, tmv;
-  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D) ||
+  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D, 16) ||
       !make_map(&tmk, k, (long long)p.B * p.Hk * p.n, D) ||
       !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
     return BSA_ERR_CUDA;
