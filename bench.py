@@ -267,7 +267,7 @@ def run_prefill(dev, peaks, reps=5):
     mk, mx, ce = bsa.build_block_summaries(k, fc.cell)
     idx, cnt = bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K)
     o = torch.empty_like(q)
-    ws = torch.empty(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
+    ws = torch.zeros(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
                                                                   fc.d)),
                      dtype=torch.uint8, device=dev)
     sws = torch.zeros(max(1, int(bsa.lib().bsa_freesolo_select_workspace_bytes(
@@ -290,7 +290,7 @@ def run_prefill(dev, peaks, reps=5):
                    "q_block": fc.q_block, "K": fc.K, "window": fc.window},
         "select": {"kernel": "split_hi_lo + freesolo_select_tc_kernel (tcgen05)", "ms": t_sel,
                    "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9},
-        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode (tcgen05) + freesolo_attn_kernel long branch (CUDA cores)", "ms": t_att,
+        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode + block unions + prefill_tc_kernel long-branch mode (tcgen05)", "ms": t_att,
                       "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,
                       "frac_of_bf16_peak": att_flops / t_att / 1e9 / peak},
         "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),

@@ -305,7 +305,7 @@ def freesolo_attn(q, k, v, alpha_h, idx, count, cell, window, rope_theta=10000.0
         o = torch.empty_like(q)
     need = int(lib().bsa_freesolo_workspace_bytes(_dtype_code(q), B, H, n, d))
     if ws is None:
-        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws = torch.zeros(need, dtype=torch.uint8, device=q.device)
     _check(lib().bsa_freesolo_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, H, n, d, cell,
                                    window, float(rope_theta), _ptr(alpha_h), _ptr(_i32(idx)),
                                    _ptr(_i32(count)), K, _ptr(o), _ptr(ws), ws.numel(),

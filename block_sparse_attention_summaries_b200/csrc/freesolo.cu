@@ -27,6 +27,12 @@ namespace bsa {
 
 bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, int H, int Hk,
                           int n, int d, int window, void* o, int* status, cudaStream_t st);
+size_t long_attn_tc_workspace(int B, int H, int n);
+bool long_attn_tc_supported(int d, int cell, int ksel);
+bsa_status long_attn_tc(const void* q, const void* k, const void* v, int B, int H, int n, int d,
+                        int cell, const int* sel, const int* sel_cnt, int ksel,
+                        const float* alpha, void* o, void* ws, size_t ws_bytes, int* status,
+                        cudaStream_t st);
 size_t freesolo_select_tc_workspace(int B, int H, int n, int d, int cell);
 bool freesolo_select_tc_supported(bsa_dtype dt, int d, int q_block, int K);
 bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cell,
@@ -374,9 +380,13 @@ extern "C" size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H
 }
 
 extern "C" size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d) {
+  using namespace bsa;
   if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return 0;
-  // rotated keys, and (bf16) rotated queries for the tensor-core window branch
-  return (size_t)B * H * n * d * (dt == BSA_BF16 ? 2 : 4) * (dt == BSA_BF16 ? 2 : 1) + 256;
+  // status word, rotated keys; bf16 adds the rotated queries of the tensor-core window branch and
+  // the per-unit block unions of the tensor-core long branch
+  const size_t rows = (size_t)B * H * n;
+  if (dt != BSA_BF16) return 256 + rows * d * 4;
+  return 256 + 2 * rows * d * 2 + long_attn_tc_workspace(B, H, n);
 }
 
 extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt,
@@ -423,7 +433,15 @@ extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void
           static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(qr), rows, n, p.log_theta);
     }
     BSA_LAUNCH_CHECK();
-    bsa_status rc = window_attn_tc(qr, kr, v, B, H, H, n, d, window, o, nullptr, st);
+    int* status = static_cast<int*>(workspace);
+    bsa_status rc = window_attn_tc(qr, kr, v, B, H, H, n, d, window, o, status, st);
+    if (rc == BSA_OK && long_attn_tc_supported(d, cell, K)) {
+      // long branch on the tensor cores over each unit's union of selected blocks
+      unsigned char* lws = static_cast<unsigned char*>(qr) + (size_t)rows * d * 2;
+      const size_t used = (size_t)(lws - static_cast<unsigned char*>(workspace));
+      return long_attn_tc(q, k, v, B, H, n, d, cell, idx, count, K, alpha_h, o, lws,
+                          workspace_bytes - used, status, st);
+    }
     if (rc == BSA_OK) {
       p.short_in_o = 1;
       dim3 grid(ceil_div(n, 4), H, B);

@@ -51,7 +51,17 @@ struct TcParams {
   float* lse;
   int* status;
   int mode;    // 0: heads 2hp, 2hp+1 at unit u (selected blocks); 1: units 2up, 2up+1 of head h
+               // over a sliding window; 2: units 2up, 2up+1 of head h over their selected cells
   int window;  // mode 1: keys j >= i - window + 1 of a sliding window (blocks of the window)
+  // mode 2 (FreeSolo long branch): each unit walks the sorted union of the 64-key blocks that
+  // hold its rows' selected cells; a row sees only the keys of its own cells
+  const int* ulist;    // [B * Hq * U][ucap] union blocks of each unit
+  const int* ucnt;     // [B * Hq * U]
+  int ucap;
+  const int* sel;      // [B, Hq, n, ksel] selected cells, -1 padded
+  const int* sel_cnt;  // [B, Hq, n] or null
+  int ksel, cell;
+  const float* alpha;  // [Hq] mixing weight of the long branch
 };
 
 template <int D>
@@ -102,18 +112,26 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bi = blockIdx.z;
   const bool win = p.mode == 1;
+  const bool fsl = p.mode == 2;
+  const bool unit_pairs = p.mode != 0;
   // the two work items: (head, unit) pairs sharing one kv head
-  const int hq[2] = {win ? (int)blockIdx.y : 2 * (int)blockIdx.y,
-                     win ? (int)blockIdx.y : 2 * (int)blockIdx.y + 1};
-  const int uu[2] = {win ? 2 * (int)blockIdx.x : (int)blockIdx.x,
-                     win ? 2 * (int)blockIdx.x + 1 : (int)blockIdx.x};
+  const int hq[2] = {unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y,
+                     unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y + 1};
+  const int uu[2] = {unit_pairs ? 2 * (int)blockIdx.x : (int)blockIdx.x,
+                     unit_pairs ? 2 * (int)blockIdx.x + 1 : (int)blockIdx.x};
   const bool item_ok[2] = {uu[0] < p.U, uu[1] < p.U};
   const int G = p.Hq / p.Hk;
   const int kh = hq[0] / G;  // both items read the same kv head
   const int wblocks = win ? (p.window - 1 + kTiles - 1) / kTiles : 0;
 
   // ---- prologue: block lists and gate biases of both items (warps 0 and 1) -----------------
-  if (warp < 2 && win) {  // sliding window: blocks u - wblocks .. u - 1 before the diagonal one
+  if (warp < 2 && fsl) {  // union lists come from global memory
+    if (lane == 0) {
+      const int it = warp;
+      const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
+      s_cnt[it] = item_ok[it] ? min(p.ucnt[urow], p.ucap) : 0;
+    }
+  } else if (warp < 2 && win) {  // sliding window: blocks u - wblocks .. u - 1 before the diagonal one
     const int it = warp;
     const int u = uu[it];
     const int first = item_ok[it] ? max(0, u - wblocks) : 0;
@@ -192,10 +210,15 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const int steps = max(s_cnt[0], s_cnt[1]) + 1;
+  // modes 0 and 1 end on the diagonal block; the long branch has none
+  const int steps = max(s_cnt[0], s_cnt[1]) + (fsl ? 0 : 1);
   const uint32_t tmem = s_tmem;
   // step j of unit it: history block, filler (fully masked) or the current block (last step)
   auto step_block = [&](int it, int j) {
+    if (fsl) {
+      const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
+      return j < s_cnt[it] ? p.ulist[urow * p.ucap + j] : 0;
+    }
     return j < s_cnt[it] ? s_blk[it][j] : (item_ok[it] ? uu[it] : uu[0]);
   };
 
@@ -207,7 +230,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     // ------------------------------------------------ TMA producers: warp 4 Q and K, warp 6 V
     // Each runs ahead as far as its ring allows: K_j once S_{j-3} completed, V_j once
     // P_{j-2} V_{j-2} completed.
-    if (lane == 0) {
+    if (lane == 0 && steps > 0) {
       const bool is_k = warp == 4;
       if (is_k) {  // 16-row boxes into the accumulator lane order
         mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
@@ -245,7 +268,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     }
   } else if (warp == 5) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && steps > 0) {
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(64, D, false, true);
       // S_j = [Q_0; Q_1] [K_0; K_1]^T as one M = 128, N = 128 chain (full tensor-core rate);
@@ -310,6 +333,25 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const int wlo = win ? i - p.window + 1 : INT_MIN;  // lowest key of the window
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     const float qk_scale = rsqrtf((float)D) * kLog2e;
+    // long branch: this row's cells that lie wholly at or before it (never a future key)
+    constexpr int kSelMax = 8;
+    int my_cells[kSelMax];
+    int nmine = 0;
+#pragma unroll
+    for (int k = 0; k < kSelMax; ++k) my_cells[k] = -1;
+    if (fsl && item_ok[it] && i < p.n) {
+      const size_t qrow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
+      const int cnt = p.sel_cnt ? min(p.sel_cnt[qrow], p.ksel) : p.ksel;
+#pragma unroll
+      for (int k = 0; k < kSelMax; ++k) {
+        const int c = k < cnt ? p.sel[qrow * p.ksel + k] : -1;
+        if (c >= 0 && (long long)(c + 1) * p.cell <= i + 1) {
+          my_cells[k] = c;
+          ++nmine;
+        }
+      }
+    }
+    const uint64_t cell_bits = p.cell >= 64 ? ~0ull : ((1ull << p.cell) - 1ull);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < steps && ok; ++j) {
@@ -333,15 +375,25 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       tc::fence_before_sync();
       mbar_arrive(&s_free[st]);
       // bias or mask of this step's block for my unit
-      const bool is_cur = (j == steps - 1);
+      const bool is_cur = !fsl && (j == steps - 1);
       const bool filler = !is_cur && j >= s_cnt[it];
-      const float bias = (!is_cur && !filler) ? s_bias[it][j] : 0.f;
+      const float bias = (!is_cur && !filler && !fsl) ? s_bias[it][j] : 0.f;
       const int kpos0 = step_block(it, j) * kTiles;  // position of this block's first key
       // keys of this block the row may see: all of a history block; none of a filler; c <= r on
-      // the diagonal; c >= wlo - kpos0 inside a sliding window
+      // the diagonal; c >= wlo - kpos0 inside a sliding window; the keys of the row's own cells
+      // in the long branch
       uint64_t keep = filler ? 0ull : ~0ull;
       if (is_cur) keep &= r >= 63 ? ~0ull : ((2ull << r) - 1ull);
       if (wlo - kpos0 > 0) keep &= wlo - kpos0 >= 64 ? 0ull : (~0ull << (wlo - kpos0));
+      if (fsl && !filler) {
+        uint64_t mine = 0ull;
+#pragma unroll
+        for (int k = 0; k < kSelMax; ++k) {
+          const long long t0 = (long long)my_cells[k] * p.cell - kpos0;
+          if (my_cells[k] >= 0 && t0 >= 0 && t0 < 64) mine |= cell_bits << t0;
+        }
+        keep &= mine;
+      }
       // z in log2 units; the row max by a 4-way tree
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (keep == ~0ull) {
@@ -416,15 +468,17 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       tc::fence_before_sync();
       mbar_arrive(&p_full[j & 1]);
     }
-    // epilogue
-    if (ok)
+    // epilogue (nothing to do without a step: the long branch of units that selected nothing)
+    if (ok && steps > 0)
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded(&o_done[(steps - 1) & 1], ((steps - 1) >> 1) & 1));
-    if (ok) {
+    if (ok && steps > 0) {
       tc::fence_after_sync();
-      const bool live = i < p.n && item_ok[it];
+      // the long branch mixes into the short branch already in o, for rows that saw a cell
+      const bool live = i < p.n && item_ok[it] && (!fsl || nmine > 0);
       const size_t orow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
-      const float inv = 1.f / l_run;
+      const float a_mix = fsl ? p.alpha[hq[it]] : 1.f;
+      const float inv = (fsl ? a_mix : 1.f) / l_run;
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow * D;
       for (int c0 = 0; c0 < D; c0 += 32) {
         float ov[32];
@@ -433,22 +487,31 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         if (live) {
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
+            if (fsl) {  // o = (1 - alpha) o_short + alpha o_long
+              float sh[8];
+              load_vec<__nv_bfloat16, 8>(op + c0 + c, sh);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ov[c + e] = fmaf(ov[c + e], inv, (1.f - a_mix) * sh[e]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ov[c + e] *= inv;
+            }
             uint4 w4;
             __nv_bfloat162 h;
-            h = __floats2bfloat162_rn(ov[c] * inv, ov[c + 1] * inv);
+            h = __floats2bfloat162_rn(ov[c], ov[c + 1]);
             w4.x = *reinterpret_cast<uint32_t*>(&h);
-            h = __floats2bfloat162_rn(ov[c + 2] * inv, ov[c + 3] * inv);
+            h = __floats2bfloat162_rn(ov[c + 2], ov[c + 3]);
             w4.y = *reinterpret_cast<uint32_t*>(&h);
-            h = __floats2bfloat162_rn(ov[c + 4] * inv, ov[c + 5] * inv);
+            h = __floats2bfloat162_rn(ov[c + 4], ov[c + 5]);
             w4.z = *reinterpret_cast<uint32_t*>(&h);
-            h = __floats2bfloat162_rn(ov[c + 6] * inv, ov[c + 7] * inv);
+            h = __floats2bfloat162_rn(ov[c + 6], ov[c + 7]);
             w4.w = *reinterpret_cast<uint32_t*>(&h);
             *reinterpret_cast<uint4*>(op + c0 + c) = w4;
           }
         }
       }
       if (live && p.lse) p.lse[orow] = (m_run + log2f(l_run)) * kLn2;
-    } else {
+    } else if (steps > 0) {
       ok = false;
     }
     if (!ok) s_abort = 1;
@@ -713,6 +776,59 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
 }
 
+// ---- FreeSolo long branch: union of each unit's selected blocks -----------------------------
+//
+// One CTA of 64 threads per (unit of 64 queries, head, batch): every query marks the 64-key blocks
+// holding its selected cells (only cells wholly at or before the query) in a bitmap; warp 0 then
+// writes the marked blocks in increasing order.
+__global__ void __launch_bounds__(64)
+    freesolo_union_kernel(const int* __restrict__ sel, const int* __restrict__ sel_cnt, int H,
+                          int n, int U, int ksel, int cell, int ucap, int* __restrict__ ucnt,
+                          int* __restrict__ ulist) {
+  extern __shared__ uint32_t ubits[];
+  const int u = blockIdx.x, h = blockIdx.y, bi = blockIdx.z, tid = threadIdx.x;
+  const int nblk = (n + kTiles - 1) / kTiles, nwords = (nblk + 31) / 32;
+  for (int w = tid; w < nwords; w += 64) ubits[w] = 0u;
+  __syncthreads();
+  const int i = u * kTiles + tid;
+  if (i < n) {
+    const size_t row = ((size_t)bi * H + h) * n + i;
+    const int cnt = sel_cnt ? min(sel_cnt[row], ksel) : ksel;
+    for (int k = 0; k < cnt; ++k) {
+      const int c = sel[row * ksel + k];
+      if (c >= 0 && (long long)(c + 1) * cell <= i + 1) {
+        const int blk = (int)((long long)c * cell / kTiles);
+        atomicOr(&ubits[blk >> 5], 1u << (blk & 31));
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const size_t urow = ((size_t)bi * H + h) * U + u;
+    int base = 0;
+    for (int w0 = 0; w0 < nwords; w0 += 32) {
+      const int w = w0 + tid;
+      uint32_t b = w < nwords ? ubits[w] : 0u;
+      const int cw = __popc(b);
+      int incl = cw;
+#pragma unroll
+      for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o2);
+        if (tid >= o2) incl += y;
+      }
+      int pos = base + incl - cw;
+      while (b) {
+        const int t = __ffs(b) - 1;
+        b &= b - 1u;
+        if (pos < ucap) ulist[urow * ucap + pos] = w * 32 + t;
+        ++pos;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (tid == 0) ucnt[urow] = min(base, ucap);
+  }
+}
+
 // ---- host side -----------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -760,7 +876,7 @@ bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
-  dim3 grid = p.mode == 1 ? dim3((p.U + 1) / 2, p.Hq, p.B) : dim3(p.U, p.Hq / 2, p.B);
+  dim3 grid = p.mode != 0 ? dim3((p.U + 1) / 2, p.Hq, p.B) : dim3(p.U, p.Hq / 2, p.B);
   kern<<<grid, kThreadsFwd, smem, st>>>(tmq, tmk, tmv, p);
   return BSA_OK;
 }
@@ -811,6 +927,45 @@ bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, in
   p.B = B; p.Hq = H; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = 0;
   p.o = o; p.lse = nullptr; p.status = status; p.mode = 1; p.window = window;
   if (ceil_div(window - 1, kTiles) > kMaxKtc) return BSA_ERR_UNSUPPORTED;
+  bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
+  if (rc != BSA_OK) return rc;
+  BSA_LAUNCH_CHECK();
+  return BSA_OK;
+}
+
+// Long branch of the FreeSolo prefill on the tensor cores (mode 2), mixing into o.
+// Workspace: union counts [B * H * U] then lists [B * H * U][ucap], ucap = min(64 * 8, blocks).
+static int long_ucap(int n) { return min(64 * 8, ceil_div(n, kTiles)); }
+
+size_t long_attn_tc_workspace(int B, int H, int n) {
+  const size_t units = (size_t)B * H * ceil_div(n, kTiles);
+  return units * sizeof(int) * (1 + (size_t)long_ucap(n)) + 256;
+}
+
+bool long_attn_tc_supported(int d, int cell, int ksel) {
+  // cells must tile the 64-key blocks: a power of two up to 64
+  return (d == 64 || d == 128) && cell >= 1 && cell <= kTiles && (kTiles % cell) == 0 &&
+         ((cell & (cell - 1)) == 0) && ksel >= 1 && ksel <= 8;
+}
+
+bsa_status long_attn_tc(const void* q, const void* k, const void* v, int B, int H, int n, int d,
+                        int cell, const int* sel, const int* sel_cnt, int ksel,
+                        const float* alpha, void* o, void* ws, size_t ws_bytes, int* status,
+                        cudaStream_t st) {
+  if (!ws || ws_bytes < long_attn_tc_workspace(B, H, n)) return BSA_ERR_WORKSPACE;
+  const int U = ceil_div(n, kTiles);
+  const int ucap = long_ucap(n);
+  int* ucnt = reinterpret_cast<int*>(align_up(reinterpret_cast<uintptr_t>(ws), (uintptr_t)256));
+  int* ulist = ucnt + (size_t)B * H * U;
+  const int nwords = ceil_div(ceil_div(n, kTiles), 32);
+  freesolo_union_kernel<<<dim3(U, H, B), 64, nwords * sizeof(uint32_t), st>>>(
+      sel, sel_cnt, H, n, U, ksel, cell, ucap, ucnt, ulist);
+  BSA_LAUNCH_CHECK();
+  TcParams p{};
+  p.B = B; p.Hq = H; p.Hk = H; p.n = n; p.U = U; p.K = 0;
+  p.o = o; p.lse = nullptr; p.status = status; p.mode = 2; p.window = 0;
+  p.ulist = ulist; p.ucnt = ucnt; p.ucap = ucap;
+  p.sel = sel; p.sel_cnt = sel_cnt; p.ksel = ksel; p.cell = cell; p.alpha = alpha;
   bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
   if (rc != BSA_OK) return rc;
   BSA_LAUNCH_CHECK();

@@ -243,7 +243,12 @@ size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H, int n, in
  * o_long: softmax attention of the raw q_i over the raw tokens of its selected cells (NoPE).
  *   idx/count as written by bsa_freesolo_select (cells not wholly at or before i are ignored).
  *   alpha_h   [H] float32 device array.   o  [B, H, n, d] out (dtype dt).
- *   workspace device scratch of bsa_freesolo_workspace_bytes() bytes (holds the rotated keys).
+ *   workspace device scratch of bsa_freesolo_workspace_bytes() bytes, its first int zeroed before
+ *             first use (the status word of the bounded waits, read and cleared by
+ *             bsa_workspace_status).  It holds the rotated keys; for bf16 also the rotated queries
+ *             and, per 64-query unit, the sorted union of the 64-key blocks holding the unit's
+ *             selected cells (the long branch then runs on the tensor cores when cell is a power
+ *             of two up to 64 and K <= 8).
  */
 bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
                              int H, int n, int d, int cell, int window, float rope_theta,

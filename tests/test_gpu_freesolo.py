@@ -111,6 +111,22 @@ def test_freesolo_select_status_clean():
                             ws=ws[:need - 1])
 
 
+def test_freesolo_attn_status_clean():
+    """The tensor-core window and long branches leave the workspace status word at zero."""
+    case = inputs.freesolo_case(45, B=1, H=2, d=64, n=3000, cell=32, q_block=128, K=4,
+                                window=256, sigma=1000.0)
+    q, k, v = (torch.from_numpy(x).to(DEV, torch.bfloat16) for x in (case.q, case.k, case.v))
+    lam = torch.from_numpy(case.lam).to(DEV)
+    sig = torch.from_numpy(case.sigma).to(DEV)
+    alpha = torch.from_numpy(case.alpha).to(DEV)
+    mean_k, mx, ce = bsa.build_block_summaries(k, case.cell)
+    idx, cnt = bsa.freesolo_select(q, mean_k, mx, ce, lam, sig, case.cell, case.q_block, case.K)
+    need = int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, 1, 2, 3000, 64))
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    bsa.freesolo_attn(q, k, v, alpha, idx, cnt, case.cell, case.window, case.rope_theta, ws=ws)
+    assert bsa.workspace_status(ws) == 0
+
+
 def test_freesolo_full_size_sampled():
     """The 64K-token, 16-head FreeSolo workload, checked on sampled queries of three heads."""
     case = inputs.freesolo_case(4000)
