@@ -112,7 +112,8 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // count of keys at or above the threshold reaches K.  It stops as soon as that count is exactly K
 // ({key >= T} is then the answer); otherwise after the last digit T is the K-th largest key and
 // the lowest-indexed keys equal to T fill the remaining places.
-// Writes the selected positions ascending to `out`; returns min(K, N).
+// Writes the selected positions ascending to `out`; returns min(K, N).  Up to 64 keys an exact
+// rank count (below) is cheaper than the radix passes.
 constexpr int kSelItems = 16;  // N <= 32 * kSelItems
 
 // count of digit d in the reduced words: parity p = d & 1 picks words 4p.., the byte k = d >> 1
@@ -133,6 +134,36 @@ __device__ __forceinline__ void flush_nibbles(uint64_t a, uint32_t (&r)[8]) {
   }
 }
 
+// Small N (<= 32 R): rank every key by counting the keys above it (ties: the lower position
+// ranks higher) and keep ranks below K -- N broadcast loads per lane, no passes.
+template <int R>
+__device__ __forceinline__ int warp_select_rank(const uint32_t* keys, int N, int kk, int lane,
+                                                int* out) {
+  uint32_t mk[R];
+  int rk[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    mk[q] = lane + 32 * q < N ? keys[lane + 32 * q] : 0u;
+    rk[q] = 0;
+  }
+  for (int j = 0; j < N; ++j) {
+    const uint32_t kj = keys[j];
+#pragma unroll
+    for (int q = 0; q < R; ++q) rk[q] += (kj > mk[q] || (kj == mk[q] && j < lane + 32 * q)) ? 1 : 0;
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  int taken = 0;
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const bool take = lane + 32 * q < N && rk[q] < kk;
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) out[taken + __popc(tb & lt)] = lane + 32 * q;
+    taken += __popc(tb);
+  }
+  __syncwarp();
+  return taken;
+}
+
 __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
@@ -141,6 +172,7 @@ __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int 
     __syncwarp();
     return N;
   }
+  if (N <= 64) return warp_select_rank<2>(keys, N, kk, lane, out);
   const int nv = (N - lane + 31) >> 5;  // keys of this lane: positions lane + 32 j, j < nv
   uint32_t kr[kSelItems];
 #pragma unroll
@@ -444,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   }
   for (int e = tid; e < kMaxUnion; e += kThreads) s_umask[e] = 0u;
   __syncthreads();
-  if (warp == 0) {  // compact the bitmap into the sorted union
+  if (warp == 0) {  // compact the bitmap into the sorted union (one word per lane up to 32)
     const int per = (nwords + 31) / 32;
     int mine = 0;
     for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) mine += __popc(s_bits[w]);

@@ -532,17 +532,19 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
 //     dg_m = sum_{i in B_m} (ptilde_i / g_m) do^T (v_i - o),
 // summed over the unit's queries, in the stable form
 //     dg_m = sum_q sum_{j in B_m} exp(z_qj - lse_q) (do_q . v_j - do_q . o_q),   z = q . k / sqrt(d).
-// Same CTA shape as the forward: heads h and h+1 at unit u in interleaved M = 64 TMEM lanes.
-// Per selected history block j the MMA thread computes Z_j = Q K_j^T and DV_j = dO V_j^T into a
-// double-buffered TMEM pair; each softmax-warp thread reduces its row, and the 64 rows of a unit
-// are summed with shuffles and shared-memory atomics into dg of that block.
+// Same CTA shape as the forward: heads h and h+1 at unit u, rows in the lane order of the M = 64
+// accumulators.  Per selected history block j the MMA thread computes Z_j = [Q_0; Q_1] [K_0; K_1]^T
+// and DV_j = [dO_0; dO_1] [V_0; V_1]^T as M = 128, N = 128 chains (the cross products are never
+// read) into a double-buffered TMEM pair; each reduction-warp thread reduces its row, and the 64
+// rows of a unit are summed with shuffles and shared-memory atomics into dg of that block.
 template <int D>
 struct GgSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTiles * D * 2;
-  static constexpr int kQ = 0;                        // Q0, dO0, Q1, dO1
-  static constexpr int kStage = 4 * kTileBytes;       // stages: K0 V0 K1 V1
-  static constexpr int kStageBytes = 4 * kTileBytes;
+  static constexpr int kPair = 2 * kTileBytes;        // [half][2 units x 64 rows x 128 B]
+  static constexpr int kQ = 0;                        // Q pair, then dO pair
+  static constexpr int kStage = 2 * kPair;            // stages: K pair, V pair
+  static constexpr int kStageBytes = 2 * kPair;
   static constexpr int kBars = kStage + 2 * kStageBytes;
   static constexpr int kTotal = kBars + 1024;
 };
@@ -626,8 +628,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     fence_mbar_init();
     s_abort = 0;
   }
-  if (warp == 5) {
-    tc::tmem_alloc(&s_tmem, 256);
+  if (warp == 5) {  // two stages of (Z: 128 columns, DV: 128 columns)
+    tc::tmem_alloc(&s_tmem, 512);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
@@ -636,21 +638,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int steps = max(s_cnt[0], s_cnt[1]);
   const uint32_t tmem = s_tmem;
   auto step_block = [&](int it, int j) { return j < s_cnt[it] ? s_blk[it][j] : u; };
-  auto qtile = [&](int it, int which) { return smem + L::kQ + (2 * it + which) * L::kTileBytes; };
-  auto stage_tile = [&](int st, int which) {
-    return smem + L::kStage + st * L::kStageBytes + which * L::kTileBytes;
+  // pairs: which 0 = Q, 1 = dO; in a stage which 0 = K, 1 = V; half hf at + hf * 16384
+  auto qpair = [&](int which) { return smem + L::kQ + which * L::kPair; };
+  auto stage_pair = [&](int st, int which) {
+    return smem + L::kStage + st * L::kStageBytes + which * L::kPair;
   };
 
   if (steps > 0) {
     if (warp == 4) {
       if (lane == 0) {
+        // 16-row boxes: unit it's row r at row 32 (r / 16) + 16 it + r % 16 of the pair
         mbar_arrive_expect_tx(q_full, 4 * L::kTileBytes);
         for (int it = 0; it < 2; ++it) {
           const int y = ((bi * p.Hq + hq[it]) * p.n) + u * kTiles;
-          for (int hf = 0; hf < L::kHalves; ++hf) {
-            tc::tma_load_2d(qtile(it, 0) + hf * 8192, &tmq, hf * 64, y, q_full);
-            tc::tma_load_2d(qtile(it, 1) + hf * 8192, &tmdo, hf * 64, y, q_full);
-          }
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            for (int b4 = 0; b4 < 4; ++b4) {
+              const int off = hf * 16384 + (32 * b4 + 16 * it) * 128;
+              tc::tma_load_2d(qpair(0) + off, &tmq, hf * 64, y + 16 * b4, q_full);
+              tc::tma_load_2d(qpair(1) + off, &tmdo, hf * 64, y + 16 * b4, q_full);
+            }
         }
         int issued = 0;
         for (int j = 0; j < steps; ++j) {
@@ -664,9 +670,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int it = 0; it < 2; ++it) {
             const int y = ((bi * p.Hk + kh) * p.n) + step_block(it, j) * kTiles;
             for (int hf = 0; hf < L::kHalves; ++hf) {
-              tc::tma_load_2d(stage_tile(st, 2 * it) + hf * 8192, &tmk, hf * 64, y, &kv_full[st]);
-              tc::tma_load_2d(stage_tile(st, 2 * it + 1) + hf * 8192, &tmv, hf * 64, y,
-                              &kv_full[st]);
+              const int off = hf * 16384 + it * 8192;
+              tc::tma_load_2d(stage_pair(st, 0) + off, &tmk, hf * 64, y, &kv_full[st]);
+              tc::tma_load_2d(stage_pair(st, 1) + off, &tmv, hf * 64, y, &kv_full[st]);
             }
           }
         }
@@ -676,7 +682,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
     } else if (warp == 5) {
       if (lane == 0) {
-        constexpr uint32_t idS = tc::idesc_bf16(64, 64, false, false);
+        constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
         bool ok = mbar_wait_bounded(q_full, 0);
         for (int j = 0; ok && j < steps; ++j) {
           const int st = j & 1;
@@ -684,22 +690,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           if (ok && j >= 2) ok = mbar_wait_bounded(&s_free[st], ((j >> 1) - 1) & 1);
           if (!ok) break;
           tc::fence_after_sync();
-          for (int it = 0; it < 2; ++it) {
-            const uint32_t lane_off = (uint32_t)(16 * it) << 16;
-            const uint32_t d_z = tmem + (uint32_t)(st * 128) + lane_off;
-            const uint32_t d_dv = d_z + 64u;
+          const uint32_t d_z = tmem + (uint32_t)(st * 256);
+          const uint32_t d_dv = d_z + 128u;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const int hf = kk >> 2, off = (kk & 3) * 32;
-              tc::mma_f16_ss(d_z, tc::smem_desc_sw128(qtile(it, 0) + hf * 8192 + off, 16, 1024),
-                             tc::smem_desc_sw128(stage_tile(st, 2 * it) + hf * 8192 + off, 16,
-                                                 1024),
-                             idS, kk > 0);
-              tc::mma_f16_ss(d_dv, tc::smem_desc_sw128(qtile(it, 1) + hf * 8192 + off, 16, 1024),
-                             tc::smem_desc_sw128(stage_tile(st, 2 * it + 1) + hf * 8192 + off, 16,
-                                                 1024),
-                             idS, kk > 0);
-            }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            tc::mma_f16_ss(d_z, tc::smem_desc_sw128(qpair(0) + off, 16, 1024),
+                           tc::smem_desc_sw128(stage_pair(st, 0) + off, 16, 1024), idS, kk > 0);
+            tc::mma_f16_ss(d_dv, tc::smem_desc_sw128(qpair(1) + off, 16, 1024),
+                           tc::smem_desc_sw128(stage_pair(st, 1) + off, 16, 1024), idS, kk > 0);
           }
           tc::mma_commit(&s_full[st]);
           tc::mma_commit(&kv_empty[st]);
@@ -736,22 +735,35 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
         if (!ok) break;
         tc::fence_after_sync();
-        float z[64], dv[64];
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128), z);
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 32), z + 32);
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 64), dv);
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 96), dv + 32);
-        tc::tmem_wait_ld();
+        // this row's 64 columns of Z and DV: unit it's block (the loads are warp-wide, so each
+        // lane keeps its own unit's half); 32 columns at a time
+        const bool use = live && j < s_cnt[it];
+        float t4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float za[32], zb[32], da[32], db[32];
+          const uint32_t base = tmem + lane_base + (uint32_t)(st * 256 + 32 * hh);
+          tc::tmem_ld32(base, za);
+          tc::tmem_ld32(base + 64u, zb);
+          tc::tmem_ld32(base + 128u, da);
+          tc::tmem_ld32(base + 192u, db);
+          tc::tmem_wait_ld();
+          tc::reg_fence(za);
+          tc::reg_fence(zb);
+          tc::reg_fence(da);
+          tc::reg_fence(db);
+          if (use) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float z = it ? zb[c] : za[c];
+              const float dv = it ? db[c] : da[c];
+              t4[c & 3] = fmaf(tc::ex2_approx(fmaf(z, zs, -lse2)), dv - Di, t4[c & 3]);
+            }
+          }
+        }
         tc::fence_before_sync();
         mbar_arrive(&s_free[st]);
-        float t = 0.f;
-        if (live && j < s_cnt[it]) {
-          float t4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            t4[c & 3] = fmaf(tc::ex2_approx(fmaf(z[c], zs, -lse2)), dv[c] - Di, t4[c & 3]);
-          t = (t4[0] + t4[1]) + (t4[2] + t4[3]);
-        }
+        float t = (t4[0] + t4[1]) + (t4[2] + t4[3]);
         // sum over the 16 rows of this unit held by this warp, then across warps
 #pragma unroll
         for (int o2 = 8; o2 > 0; o2 >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o2);
@@ -772,7 +784,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   if (s_abort && tid == 0) report_timeout(p.status, 4);
   if (warp == 5) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 256);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
@@ -885,8 +897,8 @@ template <int D>
 bsa_status launch_gg(const void* q, const void* k, const void* v, const void* dout,
                      const GgParams& p, cudaStream_t st) {
   CUtensorMap tmq, tmdo, tmk, tmv;
-  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D) ||
-      !make_map(&tmdo, dout, (long long)p.B * p.Hq * p.n, D) ||
+  if (!make_map(&tmq, q, (long long)p.B * p.Hq * p.n, D, 16) ||
+      !make_map(&tmdo, dout, (long long)p.B * p.Hq * p.n, D, 16) ||
       !make_map(&tmk, k, (long long)p.B * p.Hk * p.n, D) ||
       !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
     return BSA_ERR_CUDA;
