@@ -359,21 +359,6 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       if (!ok) break;
       tc::fence_after_sync();
-      // this row's 64 scores: columns 64 it .. 64 it + 63 of the score tile (the load is
-      // warp-wide, so both units' column ranges are read and each lane keeps its own)
-      float x[64];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float t[32];
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 32 * hh), x + 32 * hh);
-        tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 64 + 32 * hh), t);
-        tc::tmem_wait_ld();
-        tc::reg_fence(t);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) x[32 * hh + c] = it ? t[c] : x[32 * hh + c];
-      }
-      tc::fence_before_sync();
-      mbar_arrive(&s_free[st]);
       // bias or mask of this step's block for my unit
       const bool is_cur = !fsl && (j == steps - 1);
       const bool filler = !is_cur && j >= s_cnt[it];
@@ -394,19 +379,40 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         }
         keep &= mine;
       }
-      // z in log2 units; the row max by a 4-way tree
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (keep == ~0ull) {
+      // a warp none of whose rows sees a key of this block skips the scores entirely (most steps
+      // of the long branch, where a row's few cells sit in a handful of the unit's blocks)
+      const bool warp_live = __any_sync(0xffffffffu, keep != 0ull);
+      // this row's 64 scores: columns 64 it .. 64 it + 63 of the score tile (the load is
+      // warp-wide, so both units' column ranges are read and each lane keeps its own)
+      float x[64];
+      if (warp_live) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = fmaf(x[c], qk_scale, bias);
-          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+        for (int hh = 0; hh < 2; ++hh) {
+          float t[32];
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 32 * hh), x + 32 * hh);
+          tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * 128 + 64 + 32 * hh), t);
+          tc::tmem_wait_ld();
+          tc::reg_fence(t);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[32 * hh + c] = it ? t[c] : x[32 * hh + c];
         }
-      } else {
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&s_free[st]);
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (warp_live) {
+        if (keep == ~0ull) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = ((keep >> c) & 1ull) ? fmaf(x[c], qk_scale, bias) : -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+          for (int c = 0; c < 64; ++c) {
+            x[c] = fmaf(x[c], qk_scale, bias);
+            mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            x[c] = ((keep >> c) & 1ull) ? fmaf(x[c], qk_scale, bias) : -INFINITY;
+            mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+          }
         }
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
@@ -421,13 +427,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
+      if (warp_live) {
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = tc::ex2_approx(x[c] - m_use);
-        const float p1 = tc::ex2_approx(x[c + 1] - m_use);
-        sum4[(c >> 1) & 3] += p0 + p1;
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = tc::ex2_approx(x[c] - m_use);
+          const float p1 = tc::ex2_approx(x[c + 1] - m_use);
+          sum4[(c >> 1) & 3] += p0 + p1;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
       const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run = l_run * corr + sum;
