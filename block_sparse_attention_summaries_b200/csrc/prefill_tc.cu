@@ -68,8 +68,10 @@ template <int D>
 struct TcSmem {
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kTiles * D * 2;  // one [64 x D] bf16 tile
-  static constexpr int kKSlots = 3;                  // K ring: freed when S_j completes
-  static constexpr int kVSlots = 2;                  // V ring: freed when P_j V_j completes
+  // K ring slots are freed when S_j completes, V ring slots when P_j V_j completes; gathers take
+  // a few microseconds to land, so the rings run as deep as shared memory allows
+  static constexpr int kKSlots = D == 64 ? 6 : 3;
+  static constexpr int kVSlots = D == 64 ? 4 : 2;
   // queries: [half][128 rows x 128 B], unit it's row r at row 32 (r / 16) + 16 it + r % 16, the
   // lane order of the M = 64 accumulators; K slot: [half][128 rows], unit 0 rows 0-63, unit 1
   // rows 64-127 -- so one M = 128, N = 128 MMA chain gives both units' scores
@@ -91,17 +93,17 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   // 1024-byte alignment of the swizzled tiles
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[20];
+  __shared__ __align__(8) uint64_t bars[30];
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [3]
-  uint64_t* k_empty = bars + 4;   // [3]
-  uint64_t* v_full = bars + 7;    // [2]
-  uint64_t* v_empty = bars + 9;   // [2]
-  uint64_t* s_full = bars + 11;   // [2]
-  uint64_t* s_free = bars + 13;   // [2]
-  uint64_t* p_full = bars + 15;   // [2] per P buffer
-  uint64_t* o_done = bars + 17;   // [2] P_j V_j done, per P buffer
-  uint64_t* fin = bars + 19;
+  uint64_t* k_full = bars + 1;    // [kKSlots <= 6]
+  uint64_t* k_empty = bars + 7;   // [kKSlots]
+  uint64_t* v_full = bars + 13;   // [kVSlots <= 4]
+  uint64_t* v_empty = bars + 17;  // [kVSlots]
+  uint64_t* s_full = bars + 21;   // [2]
+  uint64_t* s_free = bars + 23;   // [2]
+  uint64_t* p_full = bars + 25;   // [2] per P buffer
+  uint64_t* o_done = bars + 27;   // [2] P_j V_j done, per P buffer
+  uint64_t* fin = bars + 29;
 
   __shared__ uint32_t s_tmem;
   __shared__ int s_blk[2][kMaxKtc + 1];
@@ -186,9 +188,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < L::kVSlots; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
@@ -303,12 +307,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         }
         const int pb = j & 1;
         ok = mbar_wait_bounded(&p_full[pb], (j >> 1) & 1) &&
-             mbar_wait_bounded(&v_full[pb], (j >> 1) & 1);
+             mbar_wait_bounded(&v_full[j % L::kVSlots], (j / L::kVSlots) & 1);
         if (!ok) break;
         tc::fence_after_sync();
         for (int it = 0; it < 2; ++it) {
           const uint32_t d_o = tmem + 256u + ((uint32_t)(16 * it) << 16);
-          const unsigned char* vt = vtile(pb, it);
+          const unsigned char* vt = vtile(j % L::kVSlots, it);
           const unsigned char* pt = ptile(pb, it);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 64 keys in steps of 16
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           }
         }
         tc::mma_commit(&o_done[pb]);
-        tc::mma_commit(&v_empty[pb]);
+        tc::mma_commit(&v_empty[j % L::kVSlots]);
       }
       if (!ok) s_abort = 1;
       // drain: every MMA this thread issued has completed before TMEM is released
