@@ -378,8 +378,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         uint64_t mine = 0ull;
 #pragma unroll
         for (int k = 0; k < kSelMax; ++k) {
-          const long long t0 = (long long)my_cells[k] * p.cell - kpos0;
-          if (my_cells[k] >= 0 && t0 >= 0 && t0 < 64) mine |= cell_bits << t0;
+          if (k < p.ksel && my_cells[k] >= 0) {
+            const long long t0 = (long long)my_cells[k] * p.cell - kpos0;
+            if (t0 >= 0 && t0 < 64) mine |= cell_bits << t0;
+          }
         }
         keep &= mine;
       }
@@ -405,7 +407,22 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       mbar_arrive(&s_free[st]);
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (warp_live) {
-        if (keep == ~0ull) {
+        if (fsl && p.cell >= 8) {
+          // cell masks are whole 8-key chunks: per chunk a (scale, bias) of (0, -inf) masks it
+          // with the same one FMA per key as the unmasked path (scores are finite); every lane
+          // takes this path, so a warp whose rows see different cells does not diverge
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const bool kc = ((keep >> (8 * ch)) & 0xFFull) != 0ull;
+            const float sc_c = kc ? qk_scale : 0.f, b_c = kc ? bias : -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = 8 * ch + e;
+              x[c] = fmaf(x[c], sc_c, b_c);
+              mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
+            }
+          }
+        } else if (keep == ~0ull) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
             x[c] = fmaf(x[c], qk_scale, bias);
