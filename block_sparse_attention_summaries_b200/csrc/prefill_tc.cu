@@ -356,10 +356,25 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       }
     }
     const uint64_t cell_bits = p.cell >= 64 ? ~0ull : ((1ull << p.cell) - 1ull);
+    // per cell of this row, once: its 64-key block and its keys' bits in that block (a cell
+    // never straddles two blocks: its size divides 64); block -1 for an empty slot
+    int cell_blk[kSelMax];
+    uint64_t cell_keys[kSelMax];
+#pragma unroll
+    for (int k = 0; k < kSelMax; ++k) {
+      const long long first = (long long)my_cells[k] * p.cell;
+      cell_blk[k] = my_cells[k] >= 0 ? (int)(first / kTiles) : -1;
+      cell_keys[k] = my_cells[k] >= 0 ? cell_bits << (int)(first % kTiles) : 0ull;
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    // the step's block index is read one step ahead (in the long branch it comes from global
+    // memory and its latency would otherwise sit on every step)
+    int blk_next = steps > 0 ? step_block(it, 0) : 0;
     for (int j = 0; j < steps && ok; ++j) {
       const int st = j & 1;
+      const int blk = blk_next;
+      if (j + 1 < steps) blk_next = step_block(it, j + 1);
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       if (!ok) break;
       tc::fence_after_sync();
@@ -367,7 +382,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       const bool is_cur = !fsl && (j == steps - 1);
       const bool filler = !is_cur && j >= s_cnt[it];
       const float bias = (!is_cur && !filler && !fsl) ? s_bias[it][j] : 0.f;
-      const int kpos0 = step_block(it, j) * kTiles;  // position of this block's first key
+      const int kpos0 = blk * kTiles;  // position of this block's first key
       // keys of this block the row may see: all of a history block; none of a filler; c <= r on
       // the diagonal; c >= wlo - kpos0 inside a sliding window; the keys of the row's own cells
       // in the long branch
@@ -377,12 +392,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       if (fsl && !filler) {
         uint64_t mine = 0ull;
 #pragma unroll
-        for (int k = 0; k < kSelMax; ++k) {
-          if (k < p.ksel && my_cells[k] >= 0) {
-            const long long t0 = (long long)my_cells[k] * p.cell - kpos0;
-            if (t0 >= 0 && t0 < 64) mine |= cell_bits << t0;
-          }
-        }
+        for (int k = 0; k < kSelMax; ++k) mine |= cell_blk[k] == blk ? cell_keys[k] : 0ull;
         keep &= mine;
       }
       // a warp none of whose rows sees a key of this block skips the scores entirely (most steps
@@ -438,12 +448,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       const float m_new = fmaxf(m_run, mx);
-      const bool rescale = m_run == -INFINITY ? (m_new != -INFINITY) : (m_new > m_run + kRescale);
+      // the first finite max needs no O scaling (the row's O and l are still 0); later ones
+      // rescale O only when the max grows by more than 2^8
+      const bool rescale = m_run != -INFINITY && m_new > m_run + kRescale;
       float corr = 1.f;
-      if (rescale) {
-        corr = m_run == -INFINITY ? 0.f : tc::ex2_approx(m_run - m_new);
-        m_run = m_new;
-      }
+      if (rescale) corr = tc::ex2_approx(m_run - m_new);
+      if (rescale || m_run == -INFINITY) m_run = m_new;
       // masked keys hold -inf and give 2^-inf = 0; a row with nothing seen yet subtracts 0
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};

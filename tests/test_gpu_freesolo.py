@@ -81,6 +81,19 @@ def test_freesolo_small(window, sigma, d, q_block, K):
     check_rows(case, idx, cnt, o, rows)
 
 
+@pytest.mark.parametrize("cell", [4, 64])
+def test_freesolo_cell_sizes(cell):
+    """Cells of 4 keys (per-key masks in the tensor-core long branch) and of 64 (a cell fills a
+    block); ragged n."""
+    case = inputs.freesolo_case(46, B=1, H=2, d=64, n=1500, cell=cell, q_block=128, K=4,
+                                window=200, sigma=600.0)
+    idx, cnt, o = run_gpu(case)
+    rng = np.random.default_rng(11)
+    rows = [(0, h, i) for h in range(2) for i in
+            sorted(set([0, 127, 128, 700, 1499]) | set(rng.integers(0, 1500, 12).tolist()))]
+    check_rows(case, idx, cnt, o, rows)
+
+
 def test_freesolo_select_two_batches_many_cells():
     """B = 2, 40 cells of 16 per query block: several 256-cell chunks and a ragged last chunk."""
     case = inputs.freesolo_case(43, B=2, H=3, d=64, n=5000, cell=16, q_block=128, K=5,
