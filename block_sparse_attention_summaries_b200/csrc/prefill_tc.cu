@@ -83,7 +83,8 @@ struct TcSmem {
   static constexpr int kTotal = kP + 4 * kPBytes;  // mbarriers live in static shared memory
 };
 
-template <int D>
+// MODE (p.mode) is a template argument so that each mode compiles without the others' code.
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
@@ -113,9 +114,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bi = blockIdx.z;
-  const bool win = p.mode == 1;
-  const bool fsl = p.mode == 2;
-  const bool unit_pairs = p.mode != 0;
+  constexpr bool win = MODE == 1;
+  constexpr bool fsl = MODE == 2;
+  constexpr bool unit_pairs = MODE != 0;
   // the two work items: (head, unit) pairs sharing one kv head
   const int hq[2] = {unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y,
                      unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y + 1};
@@ -924,7 +925,8 @@ bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams
       !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
     return BSA_ERR_CUDA;
   const int smem = TcSmem<D>::kTotal + 1024;  // + alignment slack
-  auto kern = prefill_tc_kernel<D>;
+  auto kern = p.mode == 0 ? prefill_tc_kernel<D, 0>
+                          : (p.mode == 1 ? prefill_tc_kernel<D, 1> : prefill_tc_kernel<D, 2>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess) {
     (void)cudaGetLastError();
