@@ -322,6 +322,33 @@ def gate_grad_rows(qs, k, v, positions, b, selected, gate, douts):
     return dg
 
 
+def selector_grad_row(s, n_cand: int, selected, dg, norm: str):
+    """ds_c = dL/ds_c for every history block c < n_cand, from dg_m = dL/dg_m of the selected.
+
+    [SAS] "Why the four design choices matter": log g_m = s_m - LSE(s) over the normaliser set
+    (R1), g_m = exp(log g_m).  By the chain rule, dL/dlog g_m = g_m dg_m and
+    dlog g_m / ds_c = [c = m] - pi_c, with pi the softmax of s over the normaliser set (0 outside
+    it), so ds_c = sum over selected m of g_m dg_m ([c = m] - pi_c).  Returns an array of n_cand.
+    """
+    s = np.asarray(s, dtype=np.float64)
+    sel = [int(m) for m in selected]
+    lg = log_gates(s, n_cand, sel, norm)
+    if norm == "all":
+        norm_set = list(range(n_cand))
+    else:
+        norm_set = sel
+    L = logsumexp(s[norm_set]) if norm_set else 0.0
+    pi = np.zeros(n_cand)
+    for c in norm_set:
+        pi[c] = math.exp(float(s[c]) - L)
+    ds = np.zeros(n_cand)
+    for m in sel:
+        w = math.exp(lg[m]) * float(dg[m])
+        for c in range(n_cand):
+            ds[c] += w * ((1.0 if c == m else 0.0) - pi[c])
+    return ds
+
+
 def gated_loss(qs, k, v, positions, b, selected, g, douts) -> float:
     """L = sum_i do_i . o_i(g) for gates g (dict m -> g_m > 0); used for finite differences."""
     gate = {m: math.log(gm) for m, gm in g.items()}

@@ -293,6 +293,60 @@ def test_gate_gradient_matches_finite_differences():
             assert abs(dg[m] - fd) <= 1e-6 * max(1.0, abs(fd))
 
 
+def _loss_of_scores(s, nc, sel, norm, q, k, v, pos, b, do):
+    gate = orc.log_gates(s, nc, sel, norm)
+    g = {m: math.exp(gate[m]) for m in sel}
+    return orc.gated_loss(q, k, v, pos, b, sel, g, do)
+
+
+def test_selector_gradient_matches_finite_differences():
+    """ds through the log-softmax gate equals central differences of the gated loss in every
+    history score -- the unselected ones included when the normaliser runs over all history."""
+    n, b, d = 256, 32, 8
+    rng = np.random.default_rng(29)
+    q, k, v = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    do = rng.standard_normal((n, d))
+    lo, hi = 192, 224
+    nc = orc.sas_num_candidates(lo, b)
+    s = rng.standard_normal(nc)
+    sel = orc.topk_blocks(s, nc, 3)
+    pos = list(range(lo, hi))
+    for norm in ["selected", "all"]:
+        gate = orc.log_gates(s, nc, sel, norm)
+        dg = orc.gate_grad_rows(q[lo:hi], k, v, pos, b, sel, gate, do[lo:hi])
+        ds = orc.selector_grad_row(s, nc, sel, dg, norm)
+        for c in range(nc):
+            h = 1e-6
+            sp, sm = s.copy(), s.copy()
+            sp[c] += h
+            sm[c] -= h
+            fd = (_loss_of_scores(sp, nc, sel, norm, q[lo:hi], k, v, pos, b, do[lo:hi]) -
+                  _loss_of_scores(sm, nc, sel, norm, q[lo:hi], k, v, pos, b, do[lo:hi])) / (2 * h)
+            assert abs(ds[c] - fd) <= 1e-6 * max(1.0, abs(fd)), (norm, c, ds[c], fd)
+        if norm == "selected":
+            assert all(ds[c] == 0.0 for c in range(nc) if c not in sel)
+
+
+def test_selector_gradient_sums_to_zero():
+    """Adding one constant to every score of the normaliser set leaves the gates unchanged, so
+    the gradient sums to zero over that set."""
+    rng = np.random.default_rng(30)
+    nc, K = 40, 6
+    s = rng.standard_normal(nc)
+    sel = orc.topk_blocks(s, nc, K)
+    dg = {m: float(rng.standard_normal()) for m in sel}
+    ds_all = orc.selector_grad_row(s, nc, sel, dg, "all")
+    ds_sel = orc.selector_grad_row(s, nc, sel, dg, "selected")
+    assert abs(ds_all.sum()) < 1e-12 * max(1.0, np.abs(ds_all).max() * nc)
+    assert abs(ds_sel.sum()) < 1e-12 * max(1.0, np.abs(ds_sel).max() * nc)
+    # a planted sign error in the normaliser term breaks the invariant
+    g = {m: math.exp(v) for m, v in orc.log_gates(s, nc, sel, "all").items()}
+    wrong = ds_all.copy()
+    for m in sel:
+        wrong[m] += 2 * g[m] * dg[m]
+    assert abs(wrong.sum()) > 1e-6
+
+
 def test_prefill_unit_dg_matches_rows():
     """The unit driver sums Eq. 5 over the unit's queries (R10) and picks Top-K of its scores."""
     B, Hq, Hk, n, d, b, qb, K = 1, 2, 1, 256, 8, 32, 32, 2
