@@ -41,6 +41,7 @@ SIGNATURES = [
                                             _I, _I, _I, _P, _I, _P, _P, _P]),
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
+    ("bsa_selector_grad", _I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _P, _I, _P]),
     ("bsa_freesolo_select", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P,
                                  _P, _Z, _P]),
     ("bsa_freesolo_select_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -269,6 +270,24 @@ def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, n
                                _ptr(_i32(count)), K, _norm_code(norm), _ptr(scores),
                                scores.shape[-1], _ptr(dg), _stream(q.device)), "bsa_gate_grad")
     return dg
+
+
+def selector_grad(scores, n_cand, idx, count, dg, norm, ds=None):
+    """ds = dL/ds through the log-softmax gate from dg; leading dims flattened into rows.
+
+    scores [..., C] float32, n_cand [...] int32, idx / dg [..., K], count [...] or None.
+    Returns ds [..., C] (0 beyond each row's candidates)."""
+    _cuda(scores, n_cand, idx, count, dg, ds)
+    C = scores.shape[-1]
+    K = idx.shape[-1]
+    rows = scores.numel() // C
+    if ds is None:
+        ds = torch.empty_like(scores)
+    _check(lib().bsa_selector_grad(_ptr(scores), C, _ptr(_i32(n_cand)), _ptr(_i32(idx)),
+                                   _ptr(None if count is None else _i32(count)), K, _ptr(dg),
+                                   int(norm), rows, _ptr(ds), C, _stream(scores.device)),
+           "bsa_selector_grad")
+    return ds
 
 
 def freesolo_select(q, mean_k, max_norm, centre, lambda_h, sigma_h, cell, q_block, K,

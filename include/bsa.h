@@ -206,6 +206,26 @@ bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void
                          float* dg, void* stream);
 
 /*
+ * bsa_selector_grad -- gradient of the loss with respect to the selector scores, through the
+ * log-softmax gate ([SAS] "Why the four design choices matter": log g_m = s_m - LSE(s) over the
+ * normaliser set N).  From dg (bsa_gate_grad):
+ *     ds_c = [c selected] g_c dg_c - pi_c * sum_{m selected} g_m dg_m,   pi = softmax over N,
+ * pi_c = 0 outside N (N = the row's history blocks c < n_cand for BSA_NORM_ALL_HISTORY, the
+ * selected blocks for BSA_NORM_SELECTED).
+ *   scores    [rows, scores_ld] float32, the row's history scores in its first n_cand entries.
+ *   n_cand    [rows] int32 device array: history blocks of the row (prefill unit u with
+ *             q_block = b has u; a decode row at position i has i / b).
+ *   idx, count, K   the row's selection as given to the gated forward (K <= 32; count may be
+ *             NULL); entries outside [0, n_cand) are ignored.
+ *   dg        [rows, K] float32 (per idx slot), as written by bsa_gate_grad.
+ *   ds        [rows, ds_ld] float32 out: ds_c for c < n_cand, 0 for c in [n_cand, ds_ld).
+ * Rows are the flattened leading dimensions ([B, Hq, U] for prefill units).
+ */
+bsa_status bsa_selector_grad(const float* scores, int scores_ld, const int* n_cand,
+                             const int* idx, const int* count, int K, const float* dg,
+                             bsa_gate_norm norm, int rows, float* ds, int ds_ld, void* stream);
+
+/*
  * bsa_freesolo_select -- per-query cell selection of the FreeSolo long branch (prefill),
  * [FreeSolo] "How it works": for the query at position i of head h the candidates are the cells
  * c lying wholly before the start of its query block, (c + 1) * cell <= floor(i / q_block) *

@@ -144,3 +144,19 @@ def test_gate_grad_rejects_bad_arguments(bsa_lib):
     assert f(*bad) == 2
     bad = list(base); bad[17] = 5
     assert f(*bad) == 1
+
+
+def test_selector_grad_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_selector_grad
+    # scores, scores_ld, n_cand, idx, count, K, dg, norm, rows, ds, ds_ld, stream
+    base = [FAKE, 64, FAKE, FAKE, None, 8, FAKE, 1, 100, FAKE, 64, None]
+    bad = list(base); bad[0] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[6] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[5] = 33
+    assert f(*bad) == 4
+    bad = list(base); bad[7] = 2
+    assert f(*bad) == 1
+    bad = list(base); bad[8] = 0
+    assert f(*bad) == 1

@@ -334,6 +334,68 @@ def test_prefill_bf16_units(gate):
 
 
 # -------------------------------------------------------------------------------------------
+# selector gradient through the log-softmax gate
+# -------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("norm", ["selected", "all"])
+def test_selector_grad_rows(norm):
+    """ds from given dg: fp32 kernel against the fp64 chain rule, rows with no, few and many
+    candidates, K up to 32."""
+    rng = np.random.default_rng(31)
+    rows, C = 300, 200
+    s = rng.standard_normal((rows, C)).astype(np.float32) * 2.0
+    n_cand = rng.integers(0, C + 1, rows).astype(np.int32)
+    n_cand[:4] = [0, 1, 3, C]
+    for K in (5, 32):
+        idx = np.full((rows, K), -1, np.int32)
+        dg = np.zeros((rows, K), np.float32)
+        for r in range(rows):
+            sel = orc.topk_blocks(s[r].astype(np.float64), int(n_cand[r]), K)
+            idx[r, :len(sel)] = sel
+            dg[r, :len(sel)] = rng.standard_normal(len(sel))
+        ds = bsa.selector_grad(up(s, False), up_i32(n_cand), up_i32(idx), None,
+                               up(dg, False), bsa.NORM_SELECTED if norm == "selected"
+                               else bsa.NORM_ALL_HISTORY).cpu().numpy()
+        for r in range(rows):
+            nc = int(n_cand[r])
+            sel = [int(m) for m in idx[r] if m >= 0]
+            ref = orc.selector_grad_row(s[r].astype(np.float64), nc, sel,
+                                        {m: float(dg[r, j]) for j, m in enumerate(sel)}, norm)
+            scale = max(1.0, float(np.max(np.abs(ref))) if nc else 1.0)
+            assert np.max(np.abs(ds[r, :nc] - ref), initial=0.0) <= 1e-5 * scale, (K, r)
+            assert np.all(ds[r, nc:] == 0.0)
+
+
+@pytest.mark.parametrize("norm", ["selected", "all"])
+def test_selector_grad_chain_bf16_units(norm):
+    """The training backward o -> g -> s on bf16 units: GPU dg then GPU ds against the oracle's
+    gate gradient and chain rule on sampled units."""
+    B, Hq, Hk, n, d, b, K = 1, 4, 2, 1024 + 37, 128, 64, 6
+    case = inputs.prefill_case(17, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, q_block=64)
+    s_gpu = up(case.scores, False)
+    q, k, v = up(case.q, True), up(case.k, True), up(case.v, True)
+    idx, cnt = bsa.topk_blocks(s_gpu, K, units=case.U, q_block=64, b=b)
+    o, lse = bsa.sparse_attn_fwd(q, k, v, idx, b, count=cnt, q_block=64, gate=True, norm=norm,
+                                 scores=s_gpu)
+    dg = bsa.gate_grad(q, k, v, o, lse, up(case.dout, True), idx, b, s_gpu, q_block=64,
+                       count=cnt, norm=norm)
+    n_cand = torch.arange(case.U, dtype=torch.int32, device=DEV).expand(B, Hq, case.U)
+    ds = bsa.selector_grad(s_gpu, n_cand.contiguous(), idx, cnt, dg,
+                           bsa.NORM_SELECTED if norm == "selected" else bsa.NORM_ALL_HISTORY)
+    ds = ds.cpu().numpy()
+    for h in range(Hq):
+        for u in [1, 2, 5, 9, 15, 16]:
+            r = orc.prefill_unit_reference(case.q, case.k, case.v, case.scores, b, 64, K, 0, h, u,
+                                           norm, case.dout)
+            sel = r["idx"]
+            dgr = {m: float(x) for m, x in zip(sel, r["dg"])}
+            ref = orc.selector_grad_row(case.scores[0, h, u].astype(np.float64), u, sel, dgr, norm)
+            err = np.max(np.abs(ds[0, h, u, :u] - ref))
+            assert err <= 1e-2 * max(1e-6, np.max(np.abs(ref))), (h, u, err)
+
+
+# -------------------------------------------------------------------------------------------
 # failure path
 # -------------------------------------------------------------------------------------------
 
