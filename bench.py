@@ -244,6 +244,13 @@ def run_prefill(dev, peaks, reps=5):
                                  norm="selected", dg=dg)
     t_fwd = statistics.fmean(time_cuda(fwd, reps, stream))
     t_grad = statistics.fmean(time_cuda(grad, max(2, reps // 2), stream))
+    n_cand = torch.arange(pc.U, dtype=torch.int32, device=dev).expand(pc.B, pc.Hq, pc.U).contiguous()
+    ds = torch.empty_like(s)
+    sgrad = lambda: bsa.selector_grad(s, n_cand, idx, cnt, dg, bsa.NORM_SELECTED, ds=ds)
+    t_sgrad = statistics.fmean(time_cuda(sgrad, reps, stream))
+    # selected normaliser: ds written over every candidate slot; idx, dg and the selected scores
+    # read per slot; count and n_cand per unit
+    sgrad_bytes = float(s.numel() * 4 + idx.numel() * 4 * 3 + cnt.numel() * 4 * 2)
     peak = peaks["bf16_tflops"]
     out["sas_gated_prefill_16k"] = {
         "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
@@ -257,6 +264,9 @@ def run_prefill(dev, peaks, reps=5):
         "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
                       "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
                       "frac_of_bf16_peak": grad_flops / t_grad / 1e9 / peak},
+        "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
+                          "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
+                          "frac_of_hbm": sgrad_bytes / t_sgrad / 1e6 / peaks["hbm_gbs"]},
     }
     del q, k, v, do, o, s, idx, cnt, lse, dg
     torch.cuda.empty_cache()
