@@ -161,6 +161,34 @@ def topk_blocks(s, n_cand: int, K: int) -> list[int]:
     return sorted(order[:min(K, n_cand)])
 
 
+def fsl_candidates(max_norm, n_cells: int, W: int, P: int) -> list[int]:
+    """FS-L pre-query pruning: the cells a head keeps before any query arrives.
+
+    [FreeSolo] "How it works", the FS-L variant: each head keeps its W most recent cells and the
+    P cells of largest maximum key norm, and queries pick their top K inside that set.  R18: the
+    P cells are taken among the cells older than the W recent ones (the two parts are disjoint),
+    larger norm first, lower index on ties, NaN last; fewer cells than W + P are all kept.
+    Returns ascending cell indices among c < n_cells.
+    """
+    recent = list(range(max(0, n_cells - W), n_cells))
+    older = n_cells - len(recent)
+    return sorted(topk_blocks(max_norm, older, P) + recent)
+
+
+def fsl_select(q, i, mean_k, max_norm, centre, lam, sigma, cand, K) -> list[int]:
+    """Top-K of the FreeSolo cell score over the pruned candidates only (ascending cells).
+
+    [FreeSolo] "How it works": the FS-L query scores the kept cells with the same r_ic as the
+    full method and reads its K best.  R18 tie rule: larger score, then lower cell index.
+    """
+    cand = [int(c) for c in cand]
+    if not cand:
+        return []
+    r = freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, max(cand) + 1)
+    order = sorted(cand, key=lambda c: _rank_key(float(round_f32(r[c])), c))
+    return sorted(order[:min(K, len(cand))])
+
+
 def round_f32(x):
     """R11: the precision in which a computed score decides the selection."""
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)

@@ -523,3 +523,56 @@ def test_freesolo_explicit_selection_matches_default():
         assert sel2 == sel and np.max(np.abs(o1 - o2)) == 0.0
         o3, _ = orc.freesolo_row(q[i], k, v, i, summ, selection=[0], **args)
         assert np.max(np.abs(o3 - o1)) > 0  # a different set changes the long branch
+
+
+def test_fsl_candidates_against_brute_force():
+    """FS-L pruning = the W newest cells plus, among the older ones, the P largest norms (lower
+    index on ties, NaN last), checked against a direct sort; small and degenerate sizes."""
+    rng = np.random.default_rng(40)
+    for trial in range(200):
+        n_cells = int(rng.integers(0, 40))
+        W, P = int(rng.integers(0, 6)), int(rng.integers(0, 10))
+        a = np.round(rng.standard_normal(n_cells) * 2) / 2  # many ties
+        if n_cells > 3 and trial % 7 == 0:
+            a[1] = np.nan
+        got = orc.fsl_candidates(a, n_cells, W, P)
+        recent = set(range(max(0, n_cells - W), n_cells))
+        older = [c for c in range(n_cells) if c not in recent]
+        keyed = sorted(older, key=lambda c: (1, 0.0, c) if np.isnan(a[c]) else (0, -a[c], c))
+        want = sorted(recent | set(keyed[:P]))
+        assert got == want
+        assert len(got) == min(n_cells, W + P)
+        # properties, independent of how the set is built: the recent cells are kept, and every
+        # kept older cell outranks every dropped older cell
+        assert recent <= set(got)
+        kept_old = [c for c in got if c not in recent]
+        dropped = [c for c in older if c not in got]
+
+        def outranks(x, y):
+            if np.isnan(a[y]):
+                return not np.isnan(a[x]) or x < y
+            if np.isnan(a[x]):
+                return False
+            return a[x] > a[y] or (a[x] == a[y] and x < y)
+        assert all(outranks(x, y) for x in kept_old for y in dropped)
+
+
+def test_fsl_select_with_every_cell_kept_is_the_full_selection():
+    """When the pruned set holds every cell, FS-L selection equals the full method's Top-K."""
+    rng = np.random.default_rng(41)
+    n, d, cell = 2048, 16, 32
+    k = rng.standard_normal((n, d))
+    mean_k, max_norm, centre = orc.block_summaries(k, cell)
+    for i in [300, 1000, 2047]:
+        q = rng.standard_normal(d)
+        nc = orc.freesolo_num_candidates(i, cell, 128)
+        cand = orc.fsl_candidates(max_norm, nc, W=8, P=nc)
+        assert cand == list(range(nc))
+        full = orc.topk_blocks(orc.round_f32(orc.freesolo_scores(q, i, mean_k, max_norm, centre,
+                                                                 0.5, 300.0, nc)), nc, 4)
+        assert orc.fsl_select(q, i, mean_k, max_norm, centre, 0.5, 300.0, cand, 4) == full
+    # a pruned set: the selection stays inside it
+    cand = orc.fsl_candidates(max_norm, 40, W=8, P=5)
+    got = orc.fsl_select(rng.standard_normal(d), 1400, mean_k, max_norm, centre, 0.5, 300.0,
+                         cand, 4)
+    assert set(got) <= set(cand) and len(got) == 4
