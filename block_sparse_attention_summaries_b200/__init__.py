@@ -42,6 +42,9 @@ SIGNATURES = [
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
     ("bsa_selector_grad", _I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _P, _I, _P]),
+    ("bsa_fsl_prune", _I, [_P, _I, _I, _P, _I, _I, _P, _P, _P]),
+    ("bsa_fsl_select", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _P,
+                            _P, _P]),
     ("bsa_freesolo_select", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P,
                                  _P, _Z, _P]),
     ("bsa_freesolo_select_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -288,6 +291,38 @@ def selector_grad(scores, n_cand, idx, count, dg, norm, ds=None):
                                    int(norm), rows, _ptr(ds), C, _stream(scores.device)),
            "bsa_selector_grad")
     return ds
+
+
+def fsl_prune(max_norm, n_cells, W, P):
+    """FS-L kept cells per row: cand [..., W + P] (ascending, -1 padded), count [...].
+
+    max_norm [..., C] float32; n_cells [...] int32 candidate cells per row."""
+    _cuda(max_norm, n_cells)
+    C = max_norm.shape[-1]
+    rows = max_norm.numel() // C
+    lead = max_norm.shape[:-1]
+    cand = torch.empty(*lead, W + P, device=max_norm.device, dtype=torch.int32)
+    cnt = torch.empty(*lead, device=max_norm.device, dtype=torch.int32)
+    _check(lib().bsa_fsl_prune(_ptr(max_norm), rows, C, _ptr(_i32(n_cells)), W, P, _ptr(cand),
+                               _ptr(cnt), _stream(max_norm.device)), "bsa_fsl_prune")
+    return cand, cnt
+
+
+def fsl_select(q, pos, mean_k, max_norm, centre, lambda_h, sigma_h, cand, cand_count, K):
+    """FS-L decode selection: idx [B, H, K] (ascending, -1 padded), count [B, H].
+
+    q [B, H, d]; pos [B] int32; summaries [B, H, C, d] / [B, H, C]; lambda_h, sigma_h [H] or
+    None; cand / cand_count from fsl_prune."""
+    _cuda(q, pos, mean_k, max_norm, centre, lambda_h, sigma_h, cand, cand_count)
+    B, H, d = q.shape
+    C = mean_k.shape[2]
+    idx = torch.empty(B, H, K, device=q.device, dtype=torch.int32)
+    cnt = torch.empty(B, H, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_fsl_select(_ptr(q), _dtype_code(q), B, H, d, _ptr(_i32(pos)), _ptr(mean_k),
+                                _ptr(max_norm), _ptr(centre), C, _ptr(lambda_h), _ptr(sigma_h),
+                                _ptr(_i32(cand)), _ptr(_i32(cand_count)), cand.shape[-1], K,
+                                _ptr(idx), _ptr(cnt), _stream(q.device)), "bsa_fsl_select")
+    return idx, cnt
 
 
 def freesolo_select(q, mean_k, max_norm, centre, lambda_h, sigma_h, cell, q_block, K,

@@ -48,7 +48,7 @@ template <int THREADS, int ITEMS>
 __global__ void __launch_bounds__(THREADS)
     topk_kernel(const float* __restrict__ scores, int C, int ld, const int* __restrict__ n_cand,
                 int units, int q_block, int b, int K, int* __restrict__ idx,
-                int* __restrict__ count) {
+                int* __restrict__ count, int out_ld, int keep_newest) {
   __shared__ uint32_t hist[256];
   __shared__ int warp_tot[THREADS / 32];
   __shared__ uint32_t s_digit;
@@ -64,15 +64,19 @@ __global__ void __launch_bounds__(THREADS)
   else
     nc = C;
   nc = max(0, min(nc, C));
+  // the keep_newest newest candidates are kept outright (FS-L) and follow the K selected among
+  // the older ones; their indices are all larger, so the row stays ascending
+  const int newest = min(keep_newest, nc);
+  nc -= newest;
   const int kk = min(K, nc);
-  int* out = idx + (size_t)row * K;
-  if (count && tid == 0) count[row] = kk;
+  int* out = idx + (size_t)row * out_ld;
+  if (count && tid == 0) count[row] = kk + newest;
+  for (int j = kk + tid; j < out_ld; j += THREADS) out[j] = j - kk < newest ? nc + (j - kk) : -1;
 
   if (kk == nc) {  // every candidate is selected (includes nc == 0)
-    for (int j = tid; j < K; j += THREADS) out[j] = j < nc ? j : -1;
+    for (int j = tid; j < kk; j += THREADS) out[j] = j;
     return;
   }
-  for (int j = kk + tid; j < K; j += THREADS) out[j] = -1;
 
   const float* srow = scores + (size_t)row * ld;
   const int i0 = tid * ITEMS;
@@ -166,6 +170,25 @@ __global__ void __launch_bounds__(THREADS)
 }  // namespace
 }  // namespace bsa
 
+namespace bsa {
+void launch_topk_rows(const float* scores, int rows, int C, int ld, const int* n_cand, int units,
+                      int q_block, int b, int K, int* idx, int* count, int out_ld,
+                      int keep_newest, cudaStream_t st) {
+  if (C <= 256)
+    topk_kernel<256, 1><<<rows, 256, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
+                                              count, out_ld, keep_newest);
+  else if (C <= 1024)
+    topk_kernel<256, 4><<<rows, 256, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
+                                              count, out_ld, keep_newest);
+  else if (C <= 4096)
+    topk_kernel<512, 8><<<rows, 512, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
+                                              count, out_ld, keep_newest);
+  else
+    topk_kernel<1024, 16><<<rows, 1024, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
+                                                 count, out_ld, keep_newest);
+}
+}  // namespace bsa
+
 extern "C" bsa_status bsa_topk_blocks(const float* scores, int rows, int C, int ld,
                                       const int* n_cand, int units, int q_block, int b, int K,
                                       int* idx, int* count, void* stream) {
@@ -175,19 +198,8 @@ extern "C" bsa_status bsa_topk_blocks(const float* scores, int rows, int C, int 
   BSA_REQUIRE(units == 0 || n_cand || (q_block > 0 && b > 0), BSA_ERR_ARG);
   BSA_REQUIRE(C <= 16384 && K <= 256, BSA_ERR_UNSUPPORTED);
   if (rows == 0) return BSA_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (C <= 256)
-    topk_kernel<256, 1><<<rows, 256, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
-                                              count);
-  else if (C <= 1024)
-    topk_kernel<256, 4><<<rows, 256, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
-                                              count);
-  else if (C <= 4096)
-    topk_kernel<512, 8><<<rows, 512, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
-                                              count);
-  else
-    topk_kernel<1024, 16><<<rows, 1024, 0, st>>>(scores, C, ld, n_cand, units, q_block, b, K, idx,
-                                                 count);
+  launch_topk_rows(scores, rows, C, ld, n_cand, units, q_block, b, K, idx, count, K, 0,
+                   static_cast<cudaStream_t>(stream));
   BSA_LAUNCH_CHECK();
   return BSA_OK;
 }

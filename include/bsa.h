@@ -226,6 +226,35 @@ bsa_status bsa_selector_grad(const float* scores, int scores_ld, const int* n_ca
                              bsa_gate_norm norm, int rows, float* ds, int ds_ld, void* stream);
 
 /*
+ * bsa_fsl_prune -- FS-L pre-query pruning ([FreeSolo] "How it works", FS-L variant): before any
+ * query arrives, each (batch, head) row keeps its W most recent candidate cells and the P cells
+ * of largest maximum key norm among the older ones (lower index on ties, NaN last).
+ *   max_norm  [rows, C] float32 (from bsa_build_block_summaries with b = cell).
+ *   n_cells   [rows] int32 device array: candidate cells of the row (c < n_cells).
+ *   cand      [rows, W + P] int32 out: kept cells ascending, -1 padded; cand_count [rows] out,
+ *             min(n_cells, W + P).  Limits: C <= 16384, P <= 256, W + P <= 128.
+ */
+bsa_status bsa_fsl_prune(const float* max_norm, int rows, int C, const int* n_cells, int W, int P,
+                         int* cand, int* cand_count, void* stream);
+
+/*
+ * bsa_fsl_select -- FS-L decode selection: the query of each (batch, head) row scores only its
+ * kept cells with the FreeSolo cell score
+ *     r_c = q . kbar_c / sqrt(d) + lambda_h * a_c * erf((i - p_c) / (2 sigma_h))
+ * (plain q . kbar_c / sqrt(d) when lambda_h is NULL) and keeps the K best (ties to the lower cell
+ * index, NaN last).
+ *   q         [B, H, d] (the decode query of each row); pos [B] int32 device array: its position i.
+ *   mean_k [B, H, C, d], max_norm / centre [B, H, C]: cell summaries; lambda_h, sigma_h [H] or NULL.
+ *   cand, cand_count, cand_ld  as written by bsa_fsl_prune (cand_ld = W + P <= 128).
+ *   idx       [B, H, K] int32 out, ascending, -1 padded; count [B, H] optional out.
+ */
+bsa_status bsa_fsl_select(const void* q, bsa_dtype dt, int B, int H, int d, const int* pos,
+                          const float* mean_k, const float* max_norm, const float* centre, int C,
+                          const float* lambda_h, const float* sigma_h, const int* cand,
+                          const int* cand_count, int cand_ld, int K, int* idx, int* count,
+                          void* stream);
+
+/*
  * bsa_freesolo_select -- per-query cell selection of the FreeSolo long branch (prefill),
  * [FreeSolo] "How it works": for the query at position i of head h the candidates are the cells
  * c lying wholly before the start of its query block, (c + 1) * cell <= floor(i / q_block) *

@@ -160,3 +160,26 @@ def test_selector_grad_rejects_bad_arguments(bsa_lib):
     assert f(*bad) == 1
     bad = list(base); bad[8] = 0
     assert f(*bad) == 1
+
+
+def test_fsl_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_fsl_prune
+    # max_norm, rows, C, n_cells, W, P, cand, cand_count, stream
+    base = [FAKE, 4, 100, FAKE, 8, 64, FAKE, FAKE, None]
+    bad = list(base); bad[0] = None
+    assert f(*bad) == 1
+    bad = list(base); bad[5] = 0
+    assert f(*bad) == 1
+    bad = list(base); bad[4] = 100
+    assert f(*bad) == 4  # W + P > 128
+    g = bsa_lib.bsa_fsl_select
+    # q, dt, B, H, d, pos, mean_k, max_norm, centre, C, lambda, sigma, cand, cand_count, cand_ld,
+    # K, idx, count, stream
+    base = [FAKE, 1, 2, 16, 64, FAKE, FAKE, FAKE, FAKE, 2048, FAKE, FAKE, FAKE, FAKE, 72, 4,
+            FAKE, None, None]
+    bad = list(base); bad[10] = None
+    assert g(*bad) == 1  # lambda without sigma
+    bad = list(base); bad[14] = 200
+    assert g(*bad) == 4
+    bad = list(base); bad[4] = 96
+    assert g(*bad) == 4
