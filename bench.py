@@ -305,6 +305,43 @@ def run_prefill(dev, peaks, reps=5):
                       "frac_of_bf16_peak": att_flops / t_att / 1e9 / peak},
         "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),
     }
+    del q, k, v, o, ws, sws, idx, cnt
+    torch.cuda.empty_cache()
+
+    # FS-L decode selection at 256K: the pruned state (W + P cells) against full O(C) scoring
+    H, d, n, cell, K, W, P = 16, 64, 262144, 32, 4, 8, 64
+    g = torch.Generator(device=dev).manual_seed(4200)
+    kf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
+    qf = torch.randn(1, H, d, device=dev, generator=g).to(torch.bfloat16)
+    mk, mx, ce = bsa.build_block_summaries(kf, cell)
+    del kf
+    C = mk.shape[2]
+    posv = n - 1
+    pos = torch.full((1,), posv, dtype=torch.int32, device=dev)
+    lam = torch.full((H,), 0.5, device=dev)
+    sig = torch.full((H,), 4096.0, device=dev)
+    n_cells = torch.full((1, H), (posv // 128) * 128 // cell, dtype=torch.int32, device=dev)
+    cand, ccnt = bsa.fsl_prune(mx, n_cells, W, P)
+    seq = torch.full((1,), n, dtype=torch.int32, device=dev)
+    sc = torch.empty(1, H, C, device=dev)
+    ncnd = torch.empty(H, device=dev, dtype=torch.int32)
+    full = lambda: bsa.topk_blocks(bsa.score_blocks(qf, mk, n, cell, seq_lens=seq, max_norm=mx,
+                                                    centre=ce, lambda_h=lam, sigma_h=sig,
+                                                    prefix_block=128, scores=sc, n_cand=ncnd)[0],
+                                   K, n_cand=ncnd)
+    fsl = lambda: bsa.fsl_select(qf, pos, mk, mx, ce, lam, sig, cand, ccnt, K)
+    prune = lambda: bsa.fsl_prune(mx, n_cells, W, P)
+    t_full = statistics.fmean(time_cuda(full, reps, stream))
+    t_fsl = statistics.fmean(time_cuda(fsl, reps, stream))
+    t_prune = statistics.fmean(time_cuda(prune, reps, stream))
+    out["fsl_decode_256k"] = {
+        "config": {"B": 1, "H": H, "d": d, "n": n, "cell": cell, "K": K, "W": W, "P": P,
+                   "cells": C},
+        "full_select_ms": t_full, "fsl_select_ms": t_fsl, "fsl_prune_ms": t_prune,
+        "kernels": "full: score_decode_kernel + topk_kernel over every cell; FS-L: "
+                   "fsl_select_kernel over W + P kept cells (prune: topk_kernel over key norms, "
+                   "once per new cell)",
+    }
     return out
 
 
