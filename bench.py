@@ -331,9 +331,29 @@ def run_prefill(dev, peaks, reps=5):
                                    K, n_cand=ncnd)
     fsl = lambda: bsa.fsl_select(qf, pos, mk, mx, ce, lam, sig, cand, ccnt, K)
     prune = lambda: bsa.fsl_prune(mx, n_cells, W, P)
-    t_full = statistics.fmean(time_cuda(full, reps, stream))
-    t_fsl = statistics.fmean(time_cuda(fsl, reps, stream))
-    t_prune = statistics.fmean(time_cuda(prune, reps, stream))
+    def graph_ms(fn, iters=20):
+        """Device time per call: `iters` calls captured in one CUDA graph (these calls are a
+        few microseconds each, far below the cost of launching them one by one from Python)."""
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(iters):
+                fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gr.replay()
+            e0.record(stream)
+            for _ in range(reps):
+                gr.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / (reps * iters)
+
+    t_full = graph_ms(full)
+    t_fsl = graph_ms(fsl)
+    t_prune = graph_ms(prune)
     out["fsl_decode_256k"] = {
         "config": {"B": 1, "H": H, "d": d, "n": n, "cell": cell, "K": K, "W": W, "P": P,
                    "cells": C},

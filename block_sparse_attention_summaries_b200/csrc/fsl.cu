@@ -7,9 +7,10 @@
 // and reads its K best, so the per-query cost is O(W + P) instead of O(C).
 //   * Pruning: the radix select of the Top-K call over the maximum key norms of the older cells,
 //     with the W newest kept outright and written after them (one CTA per (batch, head)).
-//   * Selection: one warp per (batch, head) decode query; lanes own the kept cells, a dot
-//     product per cell (q slice per lane, warp reduction), the erf bias by the owning lane, then
-//     an exact rank count for the top K (ties to the lower cell index, NaN last).
+//   * Selection: one warp per (batch, head) decode query; lane l scores kept cells l, l + 32, ...
+//     by itself (q staged in shared memory and read as broadcasts, the cell's mean key as 16-byte
+//     loads, all of them in flight at once), then an exact rank count for the top K (ties to the
+//     lower cell index, NaN last).
 #include "bsa_common.cuh"
 
 namespace bsa {
@@ -38,32 +39,37 @@ __global__ void __launch_bounds__(32 * kRowsPerCta)
                       const float* __restrict__ sig, const int* __restrict__ cand,
                       const int* __restrict__ cand_count, int cand_ld, int K,
                       int* __restrict__ idx, int* __restrict__ count) {
-  constexpr int EPL = D / 32;
   __shared__ uint32_t s_key[kRowsPerCta][kMaxKept];
+  __shared__ __align__(16) float s_q[kRowsPerCta][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kRowsPerCta + warp;  // (batch, head)
   if (row >= B * H) return;
   const int bi = row / H, h = row % H;
   const int i = pos[bi];
   const int nk = min(max(cand_count[row], 0), min(cand_ld, kMaxKept));
-  float qv[EPL];
-  load_vec<T, EPL>(q + (size_t)row * D + lane * EPL, qv);
+  for (int e = lane; e < D; e += 32) s_q[warp][e] = Elem<T>::to_f(q[(size_t)row * D + e]);
+  __syncwarp();
   const float scale = rsqrtf((float)D);
   const float lm = lam ? lam[h] : 0.f;
   const float inv2s = lam ? 0.5f / sig[h] : 0.f;
   const int* crow = cand + (size_t)row * cand_ld;
   const size_t srow = (size_t)row * C;
   uint32_t* keys = s_key[warp];
-  for (int j = 0; j < nk; ++j) {  // warp-cooperative dot product per kept cell
-    const int c = crow[j];
-    float x[EPL];
-    load_vec<float, EPL>(mean_k + (srow + c) * D + lane * EPL, x);
-    float s = 0.f;
+  const float4* qs = reinterpret_cast<const float4*>(s_q[warp]);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) s = fmaf(qv[e], x[e], s);
-    s = warp_sum(s);
-    if (lane == (j & 31)) {
-      float r = s * scale;
+  for (int t = 0; t < kMaxKept / 32; ++t) {
+    const int j = lane + 32 * t;
+    if (j < nk) {
+      const int c = crow[j];
+      const float4* kp = reinterpret_cast<const float4*>(mean_k + (srow + c) * D);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int e4 = 0; e4 < D / 4; ++e4) {
+        const float4 kv = kp[e4], qv = qs[e4];
+        a0 = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, a0));
+        a1 = fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, a1));
+      }
+      float r = (a0 + a1) * scale;
       if (lam) r += lm * max_norm[srow + c] * erff(((float)i - centre[srow + c]) * inv2s);
       keys[j] = fsl_key(r);
     }
