@@ -29,7 +29,9 @@
 // Every CTA reaches every cluster barrier (no early exit); every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
 
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <type_traits>
 
 #include "tc_common.cuh"
@@ -976,6 +978,18 @@ bool kv_map(CUtensorMap* m, const void* base, long long rows, int D) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Host-side per-call costs kept off the decode path: the occupancy of a (device, kernel, shared
+// memory, cluster size) and the shared-memory attribute of a kernel are looked up once.
+struct LaunchCache {
+  std::mutex mu;
+  std::map<std::tuple<int, const void*, size_t, int>, int> clusters;  // -> max active clusters
+  std::map<std::pair<int, const void*>, size_t> smem_set;              // -> attribute set to
+};
+LaunchCache& launch_cache() {
+  static LaunchCache c;
+  return c;
+}
+
 template <typename T, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   using SM = FusedSmem<T, D, G, MMA>;
@@ -996,15 +1010,26 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     p.chunk = chunk;
     const size_t smem = SM::bytes(p.b, chunk, CL, p.K) + 1024;  // + alignment slack
     if (smem > 220 * 1024) return BSA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
       (void)cudaGetLastError();
       return BSA_ERR_CUDA;
     }
-    if (CL > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                      cudaSuccess) {
-      (void)cudaGetLastError();
-      return BSA_ERR_UNSUPPORTED;
+    LaunchCache& lc = launch_cache();
+    {
+      std::lock_guard<std::mutex> lock(lc.mu);
+      size_t& set_to = lc.smem_set[{dev, reinterpret_cast<const void*>(kern)}];
+      if (set_to < smem) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess) {
+          (void)cudaGetLastError();
+          return BSA_ERR_CUDA;
+        }
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess)
+          (void)cudaGetLastError();  // portable cluster sizes still work
+        set_to = smem;
+      }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(CL, p.Hk, p.B);
@@ -1019,8 +1044,21 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess || nclusters <= 0) {
-      (void)cudaGetLastError();
+    {
+      std::lock_guard<std::mutex> lock(lc.mu);
+      const auto key = std::make_tuple(dev, reinterpret_cast<const void*>(kern), smem, CL);
+      auto it = lc.clusters.find(key);
+      if (it != lc.clusters.end()) {
+        nclusters = it->second;
+      } else {
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+          (void)cudaGetLastError();
+          nclusters = 0;
+        }
+        lc.clusters[key] = nclusters;
+      }
+    }
+    if (nclusters <= 0) {
       if (CL <= 2) return BSA_ERR_UNSUPPORTED;
       CL >>= 1;
       continue;
