@@ -10,15 +10,21 @@
 // * The fp32 mean keys are split once into bf16 hi + lo (kbar = hi + lo to ~2^-16 relative); the
 //   product q . kbar is accumulated as Q hi^T + Q lo^T in fp32 TMEM, so the scores keep the
 //   precision the 1e-4 index bar needs while the contraction runs on bf16 tensor cores.
-// * Cells stream through a 2-stage TMA ring, 256 cells per chunk, into double-buffered TMEM.
+// * Cells stream through a 2-stage TMA ring (128 cells per chunk at d = 64, 64 at d = 128) into
+//   double-buffered TMEM.
 // * The bias of cell c for row r is a degree-4 Taylor expansion of erf around the tile's middle
 //   row, x0 = (i0 + 63.5 - p_c) / (2 sigma): the derivatives of erf are Hermite polynomials times
-//   2/sqrt(pi) exp(-x^2), so each cell needs one erf and one exp for its five coefficients, and
-//   each (row, cell) pair four FMAs.  The step t = (r - 63.5) / (2 sigma) is at most 64 / (2 sigma);
-//   the truncation error is below |t|^5 / 5! * max|erf^(5)| (about 1e-7 lambda a_c at sigma = 300).
+//   2/sqrt(pi) exp(-x^2), so each cell needs one erf and one exp for its five coefficients.  The
+//   step t = (r - 63.5) / (2 sigma) is at most 64 / (2 sigma); the truncation error is below
+//   |t|^5 / 5! * max|erf^(5)|.  The sum over k of t_r^k coef_k(c) is a rank-5 product, so it runs
+//   on the tensor cores too: one extra K = 16 slice per part with A = [t^k high | t^k low] (per
+//   query row, written once) and B = [sqrt(d) coef high | sqrt(d) coef high] for the first part,
+//   [sqrt(d) coef low | 0] for the second (per cell, written by the epilogue one chunk ahead), all
+//   bf16 splits with ~2^-18 relative error.  TMEM then holds q . kbar + bias / scale.
 // * Eight epilogue warps: warp w reads TMEM lanes 32 (w % 4) .. and column half w / 4; each keeps
 //   a register Top-K list ordered by (score desc, index asc); the two halves of a row are merged
-//   at the end.
+//   at the end.  Where the Taylor step is too large (small sigma) the bias MMA is skipped and the
+//   epilogue evaluates erf per pair.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -46,16 +52,18 @@ struct FsTcParams {
 
 template <int D>
 struct FsTcSmem {
-  static constexpr int kNC = D == 64 ? 256 : 128;  // cells per chunk (TMEM: 2 x kNC columns)
+  static constexpr int kNC = D == 64 ? 128 : 64;  // cells per chunk (TMEM: 2 x kNC columns)
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kChunkBytes = kNC * D * 2;  // one of hi / lo
   static constexpr int kQ = 0;
-  static constexpr int kStage = kQBytes;
+  static constexpr int kAx = kQBytes;              // bias A: [128 rows x 128 B] (first 64 B used)
+  static constexpr int kStage = kAx + kRows * 128;
   static constexpr int kStageBytes = 2 * kChunkBytes;
-  static constexpr int kCoef = kStage + 2 * kStageBytes;  // [2][kNC][8] floats
+  static constexpr int kBx = kStage + 2 * kStageBytes;  // bias B: [2][kNC rows x 128 B]
+  static constexpr int kLp = kBx + 2 * kNC * 128;       // [2][kNC] (lambda a_c, p_c), erf path
   // [32][kEpiWarps * 32] floats: the scores of a thread's current 32-cell group, column tid
   // (also the merge buffer at the end: [kMaxTop][kEpiWarps * 32] keys, then as many indices)
-  static constexpr int kStash = kCoef + 2 * kNC * 8 * 4;
+  static constexpr int kStash = kLp + 2 * kNC * 8;
   static constexpr int kBars = kStash + 32 * kEpiWarps * 32 * 4;
   static constexpr int kTotal = kBars + 256;
 };
@@ -137,7 +145,9 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_free = bars + 7;    // [2]
   uint64_t* fin = bars + 9;
-  float* coef = reinterpret_cast<float*>(smem + L::kCoef);
+  uint64_t* ax_full = bars + 10;  // bias A written
+  uint64_t* bx_full = bars + 11;  // [2] bias B of a chunk written
+  float2* lp = reinterpret_cast<float2*>(smem + L::kLp);
   float* stash = reinterpret_cast<float*>(smem + L::kStash);
   uint32_t* merge_key = reinterpret_cast<uint32_t*>(smem + L::kStash);
   int* merge_idx = reinterpret_cast<int*>(smem + L::kStash) + kMaxTop * kEpiWarps * 32;
@@ -158,7 +168,9 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kEpiWarps * 32);
+      mbar_init(&bx_full[i], kNC);
     }
+    mbar_init(ax_full, kRows);
     mbar_init(fin, 1);
     fence_mbar_init();
     s_abort = 0;
@@ -207,15 +219,18 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && nchunks > 0) {
       constexpr uint32_t idS = tc::idesc_bf16(kRows, kNC, false, false);
-      bool ok = mbar_wait_bounded(q_full, 0);
+      const bool taylor = 64.f * fabsf(0.5f / p.sig[h]) <= 0.125f;  // as in the epilogue
+      bool ok = mbar_wait_bounded(q_full, 0) && (!taylor || mbar_wait_bounded(ax_full, 0));
       for (int j = 0; ok && j < nchunks; ++j) {
         const int st = j & 1;
         ok = mbar_wait_bounded(&kv_full[st], (j >> 1) & 1);
         if (ok && j >= 2) ok = mbar_wait_bounded(&s_free[st], ((j >> 1) - 1) & 1);
+        if (ok && taylor) ok = mbar_wait_bounded(&bx_full[st], (j >> 1) & 1);
         if (!ok) break;
         tc::fence_after_sync();
         const uint32_t d_s = tmem + (uint32_t)(st * kNC);
         const unsigned char* base = smem + L::kStage + st * L::kStageBytes;
+        const unsigned char* bx = smem + L::kBx + st * (kNC * 128);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // kbar hi, then kbar lo, into one accumulator
 #pragma unroll
@@ -226,6 +241,11 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
             const uint64_t b = tc::smem_desc_sw128(
                 base + part * L::kChunkBytes + hf * (kNC * 128) + off, 16, 1024);
             tc::mma_f16_ss(d_s, a, b, idS, (part > 0 || kk > 0) ? 1u : 0u);
+          }
+          if (taylor) {  // + [t^k hi | t^k lo] x [coef' hi | coef' hi] (part 0), x [coef' lo | 0]
+            const uint64_t a = tc::smem_desc_sw128(smem + L::kAx + part * 32, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(bx + part * 32, 16, 1024);
+            tc::mma_f16_ss(d_s, a, b, idS, 1u);
           }
         }
         tc::mma_commit(&s_full[st]);
@@ -266,57 +286,105 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       }
     };
     // the two bias forms are separate straight-line loops so the one that runs stays small
-    auto scan_taylor = [&](const float (&sv)[32], const float* cfb, int cbase) {
+    auto scan_mma_bias = [&](const float (&sv)[32], int cbase) {  // bias already in TMEM
       float rr[32];
       uint32_t hit = 0u;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float* cf = cfb + e * 8;
-        const float4 c03 = *reinterpret_cast<const float4*>(cf);
-        const float bias = fmaf(t, fmaf(t, fmaf(t, fmaf(t, cf[4], c03.w), c03.z), c03.y), c03.x);
-        rr[e] = fmaf(sv[e], scale, bias);
+        rr[e] = sv[e] * scale;
         hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
       }
       insert_hits(hit, rr, cbase);
     };
-    auto scan_direct = [&](const float (&sv)[32], const float* cfb, int cbase) {
+    auto scan_direct = [&](const float (&sv)[32], const float2* lpb, int cbase) {
       float rr[32];
       uint32_t hit = 0u;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float2 lp = *reinterpret_cast<const float2*>(cfb + e * 8 + 6);
-        rr[e] = fmaf(sv[e], scale, lp.x * erff(((float)i - lp.y) * inv2s));
+        const float2 l2 = lpb[e];
+        rr[e] = fmaf(sv[e], scale, l2.x * erff(((float)i - l2.y) * inv2s));
         hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
       }
       insert_hits(hit, rr, cbase);
     };
-    bool ok = true;
-    for (int j = 0; j < nchunks; ++j) {
-      const int st = j & 1;
-      // coefficients of this chunk's cells, one cell per thread (kNC <= 256 epilogue threads);
-      // slot k < 5 holds lambda a_c erf^(k)(x0) / k!, slot 6 lambda a_c, slot 7 p_c
+    // bias operands: the A rows (t^k of this row, once) and the B rows of chunk jj (one cell per
+    // thread), 128-byte swizzled like the TMA tiles; slot k < 5 of B is sqrt(d) lambda a_c
+    // erf^(k)(x0) / k! (so that TMEM holds q . kbar + bias / scale)
+    auto pack8 = [](const float (&x)[8], uint4& w) {
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]), h1 = __floats2bfloat162_rn(x[2], x[3]);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(x[4], x[5]), h3 = __floats2bfloat162_rn(x[6], x[7]);
+      w = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                     *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+    };
+    auto split8 = [](const float (&x)[8], float (&hi)[8], float (&lo)[8]) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        hi[k] = __bfloat162float(__float2bfloat16_rn(x[k]));
+        lo[k] = x[k] - hi[k];
+      }
+    };
+    auto write_bx = [&](int jj) {
       if (tid < kNC) {
-        const int c = j * kNC + tid;
-        float* cf = coef + ((size_t)st * kNC + tid) * 8;
+        const int c = jj * kNC + tid;
+        float cf[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float2 l2 = make_float2(0.f, 0.f);
         if (c < nc) {
           const float la = lam * p.max_norm[crow0 + c];
           const float pc = p.centre[crow0 + c];
+          l2 = make_float2(la, pc);
           if (taylor) {
             const float x = ((float)i0 + 63.5f - pc) * inv2s;
             const float x2 = x * x;
             const float e = 1.1283791670955126f * expf(-x2);  // first derivative of erf
-            cf[0] = la * erff(x);
-            cf[1] = la * e;
-            cf[2] = la * (-x * e);
-            cf[3] = la * ((4.f * x2 - 2.f) * e) * (1.f / 6.f);
-            cf[4] = la * ((12.f * x - 8.f * x2 * x) * e) * (1.f / 24.f);
+            const float ls = la * sqrtf((float)D);
+            cf[0] = ls * erff(x);
+            cf[1] = ls * e;
+            cf[2] = ls * (-x * e);
+            cf[3] = ls * ((4.f * x2 - 2.f) * e) * (1.f / 6.f);
+            cf[4] = ls * ((12.f * x - 8.f * x2 * x) * e) * (1.f / 24.f);
           }
-          cf[6] = la;
-          cf[7] = pc;
+        }
+        lp[(jj & 1) * kNC + tid] = l2;
+        if (taylor) {
+          float hi[8], lo[8];
+          split8(cf, hi, lo);
+          uint4 whi, wlo;
+          pack8(hi, whi);
+          pack8(lo, wlo);
+          unsigned char* rowp = smem + L::kBx + (jj & 1) * (kNC * 128);
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 0)) = whi;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 1)) = whi;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 2)) = wlo;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 3)) = make_uint4(0, 0, 0, 0);
+          fence_proxy_async();
+          mbar_arrive(&bx_full[jj & 1]);
         }
       }
-      // every epilogue warp passes this barrier once per chunk, also after a failed wait
-      asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
+    };
+    if (taylor && nchunks > 0) {
+      if (tid < kRows) {  // A rows: powers of this row's Taylor step
+        float pw[8] = {1.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float tr = ((float)tid - 63.5f) * inv2s;
+#pragma unroll
+        for (int k = 1; k < 5; ++k) pw[k] = pw[k - 1] * tr;
+        float hi[8], lo[8];
+        split8(pw, hi, lo);
+        uint4 whi, wlo;
+        pack8(hi, whi);
+        pack8(lo, wlo);
+        unsigned char* ax = smem + L::kAx;
+        *reinterpret_cast<uint4*>(ax + tc::sw128_offset(tid, 0)) = whi;
+        *reinterpret_cast<uint4*>(ax + tc::sw128_offset(tid, 1)) = wlo;
+        *reinterpret_cast<uint4*>(ax + tc::sw128_offset(tid, 2)) = whi;
+        *reinterpret_cast<uint4*>(ax + tc::sw128_offset(tid, 3)) = wlo;
+        fence_proxy_async();
+        mbar_arrive(ax_full);
+      }
+    }
+    for (int jj = 0; jj < 2 && jj < nchunks; ++jj) write_bx(jj);
+    bool ok = true;
+    for (int j = 0; j < nchunks; ++j) {
+      const int st = j & 1;
       ok = __all_sync(0xffffffffu, ok && !*reinterpret_cast<volatile int*>(&s_abort));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       tc::fence_after_sync();
@@ -326,16 +394,19 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
         const int cb = j * kNC + colh + c0;
         if (!ok || cb >= nc) break;  // warp-uniform
         const uint32_t col = (uint32_t)(st * kNC + colh + c0);
-        const float* cfb = coef + ((size_t)st * kNC + colh + c0) * 8;
         float sv[32];
         tc::tmem_ld32(tmem + lane_base + col, sv);
         tc::tmem_wait_ld();
         tc::reg_fence(sv);
         if (taylor)
-          scan_taylor(sv, cfb, cb);
+          scan_mma_bias(sv, cb);
         else
-          scan_direct(sv, cfb, cb);
+          scan_direct(sv, lp + st * kNC + colh + c0, cb);
       }
+      // every epilogue warp passes this barrier once per chunk, also after a failed wait: the
+      // chunk's (lambda a_c, p_c) and bias B rows are free once every warp has scanned it
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
+      if (ok && j + 2 < nchunks) write_bx(j + 2);
       tc::fence_before_sync();
       mbar_arrive(&s_free[st]);
     }
