@@ -21,10 +21,14 @@
 //   query row, written once) and B = [sqrt(d) coef high | sqrt(d) coef high] for the first part,
 //   [sqrt(d) coef low | 0] for the second (per cell, written by the epilogue one chunk ahead), all
 //   bf16 splits with ~2^-18 relative error.  TMEM then holds q . kbar + bias / scale.
-// * Eight epilogue warps: warp w reads TMEM lanes 32 (w % 4) .. and column half w / 4; each keeps
-//   a register Top-K list ordered by (score desc, index asc); the two halves of a row are merged
-//   at the end.  Where the Taylor step is too large (small sigma) the bias MMA is skipped and the
-//   epilogue evaluates erf per pair.
+// * Sixteen epilogue warps at d = 64, eight at d = 128 (chunks of 128 and 64 cells):
+//   warp w reads TMEM lanes 32 (w % 4) .. and the w / 4-th group of 32 columns of a chunk; each
+//   keeps a register Top-K list ordered by (score desc, index asc); the lists of a row are merged
+//   at the end.  A list is seeded with its first K cells; after that a group of 32 cells is
+//   compared raw (TMEM value against the list's threshold times sqrt(d), lowered by 2^-20 so that
+//   no cell above the threshold is missed) and only the flagged cells are scaled and offered.
+//   Where the Taylor step is too large (small sigma) the bias MMA is skipped and the epilogue
+//   evaluates erf per pair.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -35,8 +39,6 @@ namespace bsa {
 namespace {
 
 constexpr int kRows = 128;  // queries per tile (= query block)
-constexpr int kEpiWarps = 8;
-constexpr int kThreadsFs = (kEpiWarps + 2) * 32;
 constexpr int kMaxTop = 8;  // K <= 8: rows keep a list of 4 (K <= 4) or 8 slots
 
 struct FsTcParams {
@@ -53,6 +55,8 @@ struct FsTcParams {
 template <int D>
 struct FsTcSmem {
   static constexpr int kNC = D == 64 ? 128 : 64;  // cells per chunk (TMEM: 2 x kNC columns)
+  static constexpr int kEpiWarps = 4 * (kNC / 32);  // four lane quarters x 32-column groups
+  static constexpr int kThreads = (kEpiWarps + 2) * 32;
   static constexpr int kQBytes = kRows * D * 2;
   static constexpr int kChunkBytes = kNC * D * 2;  // one of hi / lo
   static constexpr int kQ = 0;
@@ -61,7 +65,7 @@ struct FsTcSmem {
   static constexpr int kStageBytes = 2 * kChunkBytes;
   static constexpr int kBx = kStage + 2 * kStageBytes;  // bias B: [2][kNC rows x 128 B]
   static constexpr int kLp = kBx + 2 * kNC * 128;       // [2][kNC] (lambda a_c, p_c), erf path
-  // [32][kEpiWarps * 32] floats: the scores of a thread's current 32-cell group, column tid
+  // [32][kEpiWarps * 32] floats: the values of a thread's current 32-cell group, column tid
   // (also the merge buffer at the end: [kMaxTop][kEpiWarps * 32] keys, then as many indices)
   static constexpr int kStash = kLp + 2 * kNC * 8;
   static constexpr int kBars = kStash + 32 * kEpiWarps * 32 * 4;
@@ -128,13 +132,74 @@ struct TopList {
   }
 };
 
+// NaN-propagating max / min: a comparator that sees a NaN puts NaN on both its outputs, so a
+// network below never duplicates a finite value and a NaN input can only make its result NaN
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+// v[o .. o + N) into descending order when it is bitonic (N a power of two, fixed indices)
+template <int N>
+__device__ __forceinline__ void bitonic_merge_desc(float (&v)[32], int o) {
+#pragma unroll
+  for (int j = N / 2; j > 0; j >>= 1)
+#pragma unroll
+    for (int e = 0; e < N; ++e)
+      if ((e ^ j) > e) {
+        const float x = v[o + e], y = v[o + (e ^ j)];
+        v[o + e] = fmax_nan(x, y);
+        v[o + (e ^ j)] = fmin_nan(x, y);
+      }
+}
+// K-th largest of 32 values (destroys v): sort runs of K with bitonic networks, then halve the
+// runs, keeping the K largest of each pair (elementwise max against the reversed partner is a
+// bitonic sequence holding them)
+template <int K>
+__device__ __forceinline__ float kth_largest32(float (&v)[32]) {
+#pragma unroll
+  for (int g = 0; g < 32 / K; ++g)
+#pragma unroll
+    for (int k = 2; k <= K; k <<= 1)
+#pragma unroll
+      for (int j = k / 2; j > 0; j >>= 1)
+#pragma unroll
+        for (int e = 0; e < K; ++e)
+          if ((e ^ j) > e) {
+            const float x = v[g * K + e], y = v[g * K + (e ^ j)];
+            const bool desc = (e & k) == 0;
+            v[g * K + e] = desc ? fmax_nan(x, y) : fmin_nan(x, y);
+            v[g * K + (e ^ j)] = desc ? fmin_nan(x, y) : fmax_nan(x, y);
+          }
+#pragma unroll
+  for (int w = 32 / K; w > 1; w >>= 1)
+#pragma unroll
+    for (int g = 0; g < w / 2; ++g) {
+#pragma unroll
+      for (int e = 0; e < K; ++e)
+        v[g * K + e] = fmax_nan(v[g * K + e], v[(g + w / 2) * K + K - 1 - e]);
+      bitonic_merge_desc<K>(v, g * K);
+    }
+  return v[K - 1];
+}
+// a little below x, so that a value compared against it is never dropped by rounding
+__device__ __forceinline__ float lowered(float x) {
+  return x - fmaf(fabsf(x), 0x1p-20f, 0x1p-100f);
+}
+
 template <int D, int KT>
-__global__ void __launch_bounds__(kThreadsFs, 1)
+__global__ void __launch_bounds__(FsTcSmem<D>::kThreads, 1)
     freesolo_select_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                               const __grid_constant__ CUtensorMap tmhi,
                               const __grid_constant__ CUtensorMap tmlo, const FsTcParams p) {
   using L = FsTcSmem<D>;
   constexpr int kNC = L::kNC;
+  constexpr int kEpiWarps = L::kEpiWarps;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -153,6 +218,9 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
   int* merge_idx = reinterpret_cast<int*>(smem + L::kStash) + kMaxTop * kEpiWarps * 32;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  // each list's current threshold (its K-th score, NaN while not full), [column group][row]:
+  // any value a list ever held bounds its row's K-th best from below, so reads need no ordering
+  __shared__ float s_thr[kEpiWarps * 32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qb = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
@@ -175,6 +243,7 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
     fence_mbar_init();
     s_abort = 0;
   }
+  if (tid < kEpiWarps * 32) s_thr[tid] = __int_as_float(0x7fc00000);
   if (warp == kEpiWarps + 1) {
     tc::tmem_alloc(&s_tmem, 2 * kNC);
     tc::tmem_relinquish();
@@ -257,55 +326,88 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps
-    const int sub = warp & 3, half = warp >> 2;
+    const int sub = warp & 3, grp = warp >> 2;  // lane quarter, 32-column group of a chunk
     const int row = 32 * sub + lane;
     const int i = i0 + row;
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     const float scale = rsqrtf((float)D);
+    const float sqrt_d = sqrtf((float)D);
     const float lam = p.lam[h];
     const float inv2s = 0.5f / p.sig[h];
     // Taylor expansion about the tile's middle row while the step stays small (|t| <= 1/8, where
     // the truncation is below 14 |t|^5 / 120 * lambda a_c = 4e-6 lambda a_c), else erf per pair.
     const bool taylor = 64.f * fabsf(inv2s) <= 0.125f;
     const float t = ((float)row - 63.5f) * inv2s;
-    // The row's list; a scan flags the cells of a 32-cell group with score above the list's
-    // threshold (all of them while a slot is empty), parks the group's scores in this thread's
-    // stash column, and the lane offers its own flagged cells in index order.
+    // The row's list (one per column group); a scan flags the cells of its 32-cell group that
+    // can still be among the row's K best (score not below the largest threshold any of the
+    // row's lists holds), parks the group's values in this thread's stash column, and the lane
+    // offers its own flagged cells in index order.
     TopList<KT> top;
     top.init();
-    auto insert_hits = [&](uint32_t hit, const float (&rr)[32], int cbase) {
+    auto insert_hits = [&](uint32_t hit, const float (&v)[32], float mul, int cbase) {
       const int left = nc - cbase;
       if (left < 32) hit &= (1u << left) - 1u;
       if (!hit) return;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) stash[e * (kEpiWarps * 32) + tid] = rr[e];
+      for (int e = 0; e < 32; ++e) stash[e * (kEpiWarps * 32) + tid] = v[e];
       while (hit) {
         const int e = __ffs(hit) - 1;
         hit &= hit - 1u;
-        top.offer_in_order(stash[e * (kEpiWarps * 32) + tid], cbase + e);
+        // the same product the unflagged path would have formed
+        top.offer_in_order(stash[e * (kEpiWarps * 32) + tid] * mul, cbase + e);
       }
     };
-    // the two bias forms are separate straight-line loops so the one that runs stays small
-    auto scan_mma_bias = [&](const float (&sv)[32], int cbase) {  // bias already in TMEM
-      float rr[32];
-      uint32_t hit = 0u;
+    // the largest threshold of the row's lists (NaN while none is full)
+    auto row_threshold = [&]() {
+      float t = top.thr;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        rr[e] = sv[e] * scale;
-        hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
+      for (int g = 0; g < kEpiWarps / 4; ++g)
+        t = fmaxf(t, reinterpret_cast<volatile float*>(s_thr)[g * kRows + row]);
+      return t;
+    };
+    // The list of a warp's first full group is still empty (the same for every lane: the test is
+    // warp-uniform); the group's own K-th largest value is then the bound.  The two bias forms
+    // are separate straight-line loops so the one that runs stays small.
+    auto scan_mma_bias = [&](float (&sv)[32], int cbase, uint32_t taddr) {  // bias in TMEM
+      // sv * scale >= t implies sv >= lowered(t * sqrt d)
+      float tv = lowered(row_threshold() * sqrt_d);
+      if (top.key[KT - 1] == 0u && nc - cbase >= 32) {
+        tv = fmaxf(tv, lowered(kth_largest32<KT>(sv)));
+        tc::tmem_ld32(taddr, sv);
+        tc::tmem_wait_ld();
+        tc::reg_fence(sv);
       }
-      insert_hits(hit, rr, cbase);
+      uint32_t hit = 0u;  // NaN bound: every cell
+#pragma unroll
+      for (int e = 0; e < 32; ++e) hit |= !(sv[e] < tv) ? (1u << e) : 0u;
+      insert_hits(hit, sv, scale, cbase);
+      s_thr[tid] = top.thr;
     };
     auto scan_direct = [&](const float (&sv)[32], const float2* lpb, int cbase) {
       float rr[32];
-      uint32_t hit = 0u;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float2 l2 = lpb[e];
         rr[e] = fmaf(sv[e], scale, l2.x * erff(((float)i - l2.y) * inv2s));
-        hit |= !(rr[e] <= top.thr) ? (1u << e) : 0u;
       }
-      insert_hits(hit, rr, cbase);
+      float tv = row_threshold();
+      if (top.key[KT - 1] == 0u && nc - cbase >= 32) {
+        // the K-th largest of K block maxima (blocks of 32 / K cells): K distinct cells reach it
+        float bm = __int_as_float(0x7f800000);
+#pragma unroll
+        for (int g = 0; g < KT; ++g) {
+          float m = rr[g * (32 / KT)];
+#pragma unroll
+          for (int e = 1; e < 32 / KT; ++e) m = fmax_nan(m, rr[g * (32 / KT) + e]);
+          bm = fmin_nan(bm, m);
+        }
+        tv = fmaxf(tv, bm);
+      }
+      uint32_t hit = 0u;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) hit |= !(rr[e] < tv) ? (1u << e) : 0u;
+      insert_hits(hit, rr, 1.f, cbase);
+      s_thr[tid] = top.thr;
     };
     // bias operands: the A rows (t^k of this row, once) and the B rows of chunk jj (one cell per
     // thread), 128-byte swizzled like the TMA tiles; slot k < 5 of B is sqrt(d) lambda a_c
@@ -323,9 +425,12 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
         lo[k] = x[k] - hi[k];
       }
     };
+    // chunk jj's rows are written by the threads of column group jj % (kEpiWarps / 4), one cell
+    // each, so that the work rotates over the warps
     auto write_bx = [&](int jj) {
-      if (tid < kNC) {
-        const int c = jj * kNC + tid;
+      const int wt = tid - kRows * (jj % (kEpiWarps / 4));
+      if (wt >= 0 && wt < kNC) {
+        const int c = jj * kNC + wt;
         float cf[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         float2 l2 = make_float2(0.f, 0.f);
         if (c < nc) {
@@ -344,7 +449,7 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
             cf[4] = ls * ((12.f * x - 8.f * x2 * x) * e) * (1.f / 24.f);
           }
         }
-        lp[(jj & 1) * kNC + tid] = l2;
+        lp[(jj & 1) * kNC + wt] = l2;
         if (taylor) {
           float hi[8], lo[8];
           split8(cf, hi, lo);
@@ -352,10 +457,10 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
           pack8(hi, whi);
           pack8(lo, wlo);
           unsigned char* rowp = smem + L::kBx + (jj & 1) * (kNC * 128);
-          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 0)) = whi;
-          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 1)) = whi;
-          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 2)) = wlo;
-          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(tid, 3)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(wt, 0)) = whi;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(wt, 1)) = whi;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(wt, 2)) = wlo;
+          *reinterpret_cast<uint4*>(rowp + tc::sw128_offset(wt, 3)) = make_uint4(0, 0, 0, 0);
           fence_proxy_async();
           mbar_arrive(&bx_full[jj & 1]);
         }
@@ -388,20 +493,18 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       ok = __all_sync(0xffffffffu, ok && !*reinterpret_cast<volatile int*>(&s_abort));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       tc::fence_after_sync();
-      const int colh = half * (kNC / 2);
-#pragma unroll 1
-      for (int c0 = 0; c0 < kNC / 2; c0 += 32) {
-        const int cb = j * kNC + colh + c0;
-        if (!ok || cb >= nc) break;  // warp-uniform
-        const uint32_t col = (uint32_t)(st * kNC + colh + c0);
+      const int colh = grp * 32;
+      const int cb = j * kNC + colh;
+      if (ok && cb < nc) {  // warp-uniform
+        const uint32_t col = (uint32_t)(st * kNC + colh);
         float sv[32];
         tc::tmem_ld32(tmem + lane_base + col, sv);
         tc::tmem_wait_ld();
         tc::reg_fence(sv);
         if (taylor)
-          scan_mma_bias(sv, cb);
+          scan_mma_bias(sv, cb, tmem + lane_base + col);
         else
-          scan_direct(sv, lp + st * kNC + colh + c0, cb);
+          scan_direct(sv, lp + st * kNC + colh, cb);
       }
       // every epilogue warp passes this barrier once per chunk, also after a failed wait: the
       // chunk's (lambda a_c, p_c) and bias B rows are free once every warp has scanned it
@@ -411,7 +514,7 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       mbar_arrive(&s_free[st]);
     }
     if (!ok) s_abort = 1;
-    // merge the two column halves of each row, order the winners by index, write
+    // merge the column groups' lists of each row, order the winners by index, write
     asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));  // stash free: merge reuses it
 #pragma unroll
     for (int e = 0; e < KT; ++e) {
@@ -419,11 +522,13 @@ __global__ void __launch_bounds__(kThreadsFs, 1)
       merge_idx[e * (kEpiWarps * 32) + tid] = top.idx[e];
     }
     asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32));
-    if (half == 0 && i < p.n) {
+    if (grp == 0 && i < p.n) {
 #pragma unroll
-      for (int e = 0; e < KT; ++e)
-        top.offer(merge_key[e * (kEpiWarps * 32) + tid + 128],
-                  merge_idx[e * (kEpiWarps * 32) + tid + 128]);
+      for (int g = 1; g < kEpiWarps / 4; ++g)
+#pragma unroll
+        for (int e = 0; e < KT; ++e)
+          top.offer(merge_key[e * (kEpiWarps * 32) + tid + kRows * g],
+                    merge_idx[e * (kEpiWarps * 32) + tid + kRows * g]);
       const int kk = min(p.K, nc);
       int sel[KT];
 #pragma unroll
@@ -528,21 +633,23 @@ bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cel
   p.max_norm = max_norm; p.centre = centre; p.lam = lam; p.sig = sig;
   p.idx = idx; p.count = count; p.status = static_cast<int*>(ws);
   const dim3 grid((n + kRows - 1) / kRows, H, B);
-  auto run = [&](auto kern, int smem) -> bsa_status {
+  auto run = [&](auto kern, int smem, int threads) -> bsa_status {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess) {
       (void)cudaGetLastError();
       return BSA_ERR_CUDA;
     }
-    kern<<<grid, kThreadsFs, smem, st>>>(tmq, tmhi, tmlo, p);
+    kern<<<grid, threads, smem, st>>>(tmq, tmhi, tmlo, p);
     BSA_LAUNCH_CHECK();
     return BSA_OK;
   };
+  using S64 = FsTcSmem<64>;
+  using S128 = FsTcSmem<128>;
   if (d == 64)
-    return K <= 4 ? run(freesolo_select_tc_kernel<64, 4>, FsTcSmem<64>::kTotal + 1024)
-                  : run(freesolo_select_tc_kernel<64, 8>, FsTcSmem<64>::kTotal + 1024);
-  return K <= 4 ? run(freesolo_select_tc_kernel<128, 4>, FsTcSmem<128>::kTotal + 1024)
-                : run(freesolo_select_tc_kernel<128, 8>, FsTcSmem<128>::kTotal + 1024);
+    return K <= 4 ? run(freesolo_select_tc_kernel<64, 4>, S64::kTotal + 1024, S64::kThreads)
+                  : run(freesolo_select_tc_kernel<64, 8>, S64::kTotal + 1024, S64::kThreads);
+  return K <= 4 ? run(freesolo_select_tc_kernel<128, 4>, S128::kTotal + 1024, S128::kThreads)
+                : run(freesolo_select_tc_kernel<128, 8>, S128::kTotal + 1024, S128::kThreads);
 }
 
 }  // namespace bsa
