@@ -287,7 +287,7 @@ def run_prefill(dev, peaks, reps=5):
     idx, cnt = bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K)
     o = torch.empty_like(q)
     ws = torch.zeros(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
-                                                                  fc.d)),
+                                                                  fc.d, fc.cell, fc.K)),
                      dtype=torch.uint8, device=dev)
     sws = torch.zeros(max(1, int(bsa.lib().bsa_freesolo_select_workspace_bytes(
         bsa.BSA_BF16, fc.B, fc.H, fc.n, fc.d, fc.cell, fc.q_block, fc.K))), dtype=torch.uint8,

@@ -50,7 +50,7 @@ SIGNATURES = [
     ("bsa_freesolo_select_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     ("bsa_freesolo_attn", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P,
                                _P, _I, _P, _P, _Z, _P]),
-    ("bsa_freesolo_workspace_bytes", _Z, [_I, _I, _I, _I, _I]),
+    ("bsa_freesolo_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I]),
     ("bsa_workspace_status", _I, [_P, _P]),
     ("bsa_selftest_bounded_wait", _I, [_P, _I, _P]),
 ]
@@ -357,7 +357,7 @@ def freesolo_attn(q, k, v, alpha_h, idx, count, cell, window, rope_theta=10000.0
     K = idx.shape[-1]
     if o is None:
         o = torch.empty_like(q)
-    need = int(lib().bsa_freesolo_workspace_bytes(_dtype_code(q), B, H, n, d))
+    need = int(lib().bsa_freesolo_workspace_bytes(_dtype_code(q), B, H, n, d, cell, K))
     if ws is None:
         ws = torch.zeros(need, dtype=torch.uint8, device=q.device)
     _check(lib().bsa_freesolo_attn(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, H, n, d, cell,

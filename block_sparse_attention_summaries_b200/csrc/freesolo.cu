@@ -33,6 +33,11 @@ bsa_status long_attn_tc(const void* q, const void* k, const void* v, int B, int 
                         int cell, const int* sel, const int* sel_cnt, int ksel,
                         const float* alpha, void* o, void* ws, size_t ws_bytes, int* status,
                         cudaStream_t st);
+bool long_cells_supported(int d, int cell, int K, long long rows);
+size_t long_cells_workspace(int B, int H, int n, int d, int cell, int K);
+bsa_status long_cells(const void* q, const void* k, const void* v, int B, int H, int n, int d,
+                      int cell, const int* idx, const int* count, int K, const float* alpha,
+                      void* o, void* ws, size_t ws_bytes, int* status, cudaStream_t st);
 size_t freesolo_select_tc_workspace(int B, int H, int n, int d, int cell);
 bool freesolo_select_tc_supported(bsa_dtype dt, int d, int q_block, int K);
 bsa_status freesolo_select_tc(const void* q, int B, int H, int n, int d, int cell,
@@ -379,14 +384,18 @@ extern "C" size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H
              : 0;
 }
 
-extern "C" size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d) {
+extern "C" size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d,
+                                                int cell, int K) {
   using namespace bsa;
-  if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return 0;
+  if (B <= 0 || H <= 0 || n <= 0 || d <= 0 || cell <= 0 || K <= 0) return 0;
   // status word, rotated keys; bf16 adds the rotated queries of the tensor-core window branch and
-  // the per-unit block unions of the tensor-core long branch
+  // the long branch's scratch: cell-major pair lists and partial outputs, or per-unit block unions
   const size_t rows = (size_t)B * H * n;
   if (dt != BSA_BF16) return 256 + rows * d * 4;
-  return 256 + 2 * rows * d * 2 + long_attn_tc_workspace(B, H, n);
+  const size_t lw = long_cells_supported(d, cell, K, (long long)rows)
+                        ? long_cells_workspace(B, H, n, d, cell, K)
+                        : long_attn_tc_workspace(B, H, n);
+  return 256 + 2 * rows * d * 2 + lw;
 }
 
 extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt,
@@ -404,7 +413,7 @@ extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void
   BSA_REQUIRE(K <= kMaxK, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(B <= 65535 && H <= 65535, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(all_aligned16(q, k, v, o, workspace), BSA_ERR_ARG);
-  if (!workspace || workspace_bytes < bsa_freesolo_workspace_bytes(dt, B, H, n, d))
+  if (!workspace || workspace_bytes < bsa_freesolo_workspace_bytes(dt, B, H, n, d, cell, K))
     return BSA_ERR_WORKSPACE;
   FsParams p;
   p.q = q; p.k = k; p.v = v;
@@ -435,10 +444,15 @@ extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void
     BSA_LAUNCH_CHECK();
     int* status = static_cast<int*>(workspace);
     bsa_status rc = window_attn_tc(qr, kr, v, B, H, H, n, d, window, o, status, st);
+    unsigned char* lws = static_cast<unsigned char*>(qr) + (size_t)rows * d * 2;
+    const size_t used = (size_t)(lws - static_cast<unsigned char*>(workspace));
+    if (rc == BSA_OK && long_cells_supported(d, cell, K, rows)) {
+      // long branch on the tensor cores, regrouped by cell: only the selected pairs are computed
+      return long_cells(q, k, v, B, H, n, d, cell, idx, count, K, alpha_h, o, lws,
+                        workspace_bytes - used, status, st);
+    }
     if (rc == BSA_OK && long_attn_tc_supported(d, cell, K)) {
       // long branch on the tensor cores over each unit's union of selected blocks
-      unsigned char* lws = static_cast<unsigned char*>(qr) + (size_t)rows * d * 2;
-      const size_t used = (size_t)(lws - static_cast<unsigned char*>(workspace));
       return long_attn_tc(q, k, v, B, H, n, d, cell, idx, count, K, alpha_h, o, lws,
                           workspace_bytes - used, status, st);
     }

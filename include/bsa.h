@@ -295,16 +295,22 @@ size_t bsa_freesolo_select_workspace_bytes(bsa_dtype dt, int B, int H, int n, in
  *   workspace device scratch of bsa_freesolo_workspace_bytes() bytes, its first int zeroed before
  *             first use (the status word of the bounded waits, read and cleared by
  *             bsa_workspace_status).  It holds the rotated keys; for bf16 also the rotated queries
- *             and, per 64-query unit, the sorted union of the 64-key blocks holding the unit's
- *             selected cells (the long branch then runs on the tensor cores when cell is a power
- *             of two up to 64 and K <= 8).
+ *             and the long branch's scratch.  With bf16, d in {64, 128}, cell in {16, 32, 64} and
+ *             K <= 8 the long branch is regrouped by cell: each attended (query, cell) pair gets a
+ *             place in its cell's list, tiles of 128 such queries attend to the cell's tokens on
+ *             the tensor cores, and an unnormalised output row with its (max, sum) per pair
+ *             (B * H * n * K * (d + 2) floats) is merged per query at the end.  With other cell
+ *             sizes (powers of two up to 64) the scratch holds, per 64-query unit, the sorted
+ *             union of the 64-key blocks holding the unit's selected cells.  A slot is attended
+ *             once: a cell repeated within a query's slots counts once.
  */
 bsa_status bsa_freesolo_attn(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
                              int H, int n, int d, int cell, int window, float rope_theta,
                              const float* alpha_h, const int* idx, const int* count, int K,
                              void* o, void* workspace, size_t workspace_bytes, void* stream);
 
-size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d);
+/* Workspace bytes bsa_freesolo_attn needs for these arguments (0 for invalid sizes). */
+size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d, int cell, int K);
 
 /*
  * bsa_sparse_attn_decode_noalloc -- the decode form of bsa_sparse_attn_fwd (nq == 1) for callers

@@ -134,7 +134,8 @@ def test_freesolo_attn_status_clean():
     alpha = torch.from_numpy(case.alpha).to(DEV)
     mean_k, mx, ce = bsa.build_block_summaries(k, case.cell)
     idx, cnt = bsa.freesolo_select(q, mean_k, mx, ce, lam, sig, case.cell, case.q_block, case.K)
-    need = int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, 1, 2, 3000, 64))
+    need = int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, 1, 2, 3000, 64,
+                                                         case.cell, case.K))
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     bsa.freesolo_attn(q, k, v, alpha, idx, cnt, case.cell, case.window, case.rope_theta, ws=ws)
     assert bsa.workspace_status(ws) == 0
