@@ -18,9 +18,15 @@
 //  * rope_keys: K rotated once into the workspace.  Angles pos * theta^(-2t/d) are formed and
 //    reduced modulo 2 pi in fp64 (positions reach 2^16 and more, where an fp32 angle would be off
 //    by ~1e-2 rad), then sin/cos are taken in fp32.
+//  * rope_qk (bf16, tensor-core branch): Q and K rotated in one pass, sharing each position's
+//    angles; the frequencies theta^(-2t/d) come from a table formed once on the host in fp64, the
+//    angle is reduced in fp64 as above and its sine and cosine are the fast fp32 ones on
+//    [-pi, pi] (absolute error ~1e-6, far below the bf16 rounding of the result).
 //  * attn: one warp per query, lane l holding elements {l, l+32, ...} so that every rotate-half
 //    pair (t, t + d/2) sits in one lane; online softmax over the window, then over the selected
 //    cells, then the mix.
+#include <cmath>
+
 #include "bsa_common.cuh"
 
 namespace bsa {
@@ -184,6 +190,64 @@ __global__ void rope_keys_kernel(const T* __restrict__ k, T* __restrict__ kr, lo
   T* dst = kr + row * D;
   dst[t] = Elem<T>::from_f(a * c - b * s);
   dst[t + D / 2] = Elem<T>::from_f(b * c + a * s);
+}
+
+// Rotation of q and k for the tensor-core branch: a thread per (row, group of four pairs t),
+// 8-byte loads and stores of both halves.
+template <int D>
+struct InvFreq {
+  double f[D / 2];
+};
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    rope_qk_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                   __nv_bfloat16* __restrict__ qr, __nv_bfloat16* __restrict__ kr, long long rows,
+                   int n, const InvFreq<D> inv) {
+  constexpr int G = D / 8;  // groups of four pairs per row
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= rows * G) return;
+  const long long row = gid / G;
+  const int t0 = (int)(gid % G) * 4;
+  const double pos = (double)(row % n);
+  float c[4], s[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    double ang = pos * inv.f[t0 + e];
+    ang = fma(-6.283185307179586, rint(ang * 0.15915494309189535), ang);
+    __sincosf((float)ang, &s[e], &c[e]);
+  }
+  auto rotate = [&](const __nv_bfloat16* src, __nv_bfloat16* dst) {
+    const uint2 lo = *reinterpret_cast<const uint2*>(src + row * D + t0);
+    const uint2 hi = *reinterpret_cast<const uint2*>(src + row * D + t0 + D / 2);
+    const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&lo);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&hi);
+    uint2 olo, ohi;
+    __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&olo);
+    __nv_bfloat162* y = reinterpret_cast<__nv_bfloat162*>(&ohi);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 fa = __bfloat1622float2(a[e]), fb = __bfloat1622float2(b[e]);
+      const int u = 2 * e, w = 2 * e + 1;
+      x[e] = __floats2bfloat162_rn(fa.x * c[u] - fb.x * s[u], fa.y * c[w] - fb.y * s[w]);
+      y[e] = __floats2bfloat162_rn(fb.x * c[u] + fa.x * s[u], fb.y * c[w] + fa.y * s[w]);
+    }
+    *reinterpret_cast<uint2*>(dst + row * D + t0) = olo;
+    *reinterpret_cast<uint2*>(dst + row * D + t0 + D / 2) = ohi;
+  };
+  rotate(q, qr);
+  rotate(k, kr);
+}
+
+template <int D>
+void launch_rope_qk(const void* q, const void* k, void* qr, void* kr, long long rows, int n,
+                    double log_theta, cudaStream_t st) {
+  InvFreq<D> inv;
+  for (int t = 0; t < D / 2; ++t) inv.f[t] = std::exp(-2.0 * t / D * log_theta);
+  const long long threads = rows * (D / 8);
+  rope_qk_kernel<D><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<__nv_bfloat16*>(qr), static_cast<__nv_bfloat16*>(kr), rows, n, inv);
 }
 
 struct FsParams {
@@ -428,19 +492,8 @@ extern "C" bsa_status bsa_freesolo_attn(const void* q, const void* k, const void
     // short branch on the tensor cores: rotate q and k once, sliding-window tiles over them
     const long long rows = (long long)B * H * n;
     void* qr = static_cast<unsigned char*>(workspace) + 256 + (size_t)rows * d * 2;
-    const long long pairs = rows * (d / 2);
-    const unsigned nblk = (unsigned)((pairs + 255) / 256);
-    if (d == 64) {
-      rope_keys_kernel<__nv_bfloat16, 64><<<nblk, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(kr), rows, n, p.log_theta);
-      rope_keys_kernel<__nv_bfloat16, 64><<<nblk, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(qr), rows, n, p.log_theta);
-    } else {
-      rope_keys_kernel<__nv_bfloat16, 128><<<nblk, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(kr), rows, n, p.log_theta);
-      rope_keys_kernel<__nv_bfloat16, 128><<<nblk, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(qr), rows, n, p.log_theta);
-    }
+    if (d == 64) launch_rope_qk<64>(q, k, qr, kr, rows, n, p.log_theta, st);
+    else launch_rope_qk<128>(q, k, qr, kr, rows, n, p.log_theta, st);
     BSA_LAUNCH_CHECK();
     int* status = static_cast<int*>(workspace);
     bsa_status rc = window_attn_tc(qr, kr, v, B, H, H, n, d, window, o, status, st);

@@ -27,6 +27,7 @@
 
 #include <map>
 #include <mutex>
+#include <type_traits>
 
 #include "tc_common.cuh"
 
@@ -34,7 +35,6 @@ namespace bsa {
 namespace {
 
 constexpr int kRowsL = 128;    // pairs per tile (tcgen05 M)
-constexpr int kThreadsL = 128;
 constexpr int kMaxKL = 8;      // slots per query
 
 struct FsLongWs {
@@ -158,6 +158,13 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---- 4. tiles: 128 gathered queries x one cell ------------------------------------------------
+// Warp roles: 0-3 softmax and epilogue (thread = tile row = TMEM lane); 4 the producer (the tile's
+// query rows by TMA row gathers, four rows per instruction into the 128-byte-swizzled tile, the
+// cell's K and V by tiled TMA, all completing on the stage's barrier; it prefetches the next
+// tile's pair ids meanwhile); 5 the MMA issuer, which issues S of a tile as soon as its stage has
+// landed and P V as soon as its P is written.  S and O (TMEM) and P (shared memory) are
+// double-buffered, so the softmax of one tile overlaps the gathers and MMAs of its neighbours;
+// NS (2 or 3) stages of gathers are in flight per CTA.
 struct LongTileParams {
   const __nv_bfloat16* q;
   const int4* tiles;
@@ -166,61 +173,85 @@ struct LongTileParams {
   float2* part_ml;
   __nv_bfloat16* part_o;
   int* status;
-  int n, C, K;
+  int n, C, K, rows;
   long long tile_cap;
   float c2;  // log2(e) / sqrt(d)
 };
 
-template <int D>
+template <int D, int CELL>
 struct LongSmem {
   static constexpr int kHalves = D / 64;
-  static constexpr int kQ = 0;                        // [half][128 rows x 128 B]
-  static constexpr int kK = kQ + kHalves * 16384;     // [half][64 rows x 128 B]
-  static constexpr int kV = kK + kHalves * 8192;      // [half][64 rows x 128 B]
-  static constexpr int kP = kV + kHalves * 8192;      // [128 rows x 128 B]
-  static constexpr int kTotal = kP + 16384;
-  // TMEM: S in columns [0, 64), O in [64, 64 + D)
-  static constexpr uint32_t kCols = D == 64 ? 128 : 256;
+  static constexpr int kCtasPerSm = D == 64 ? 2 : 1;  // TMEM: 2 x 256 or 1 x 512 columns
+  static constexpr int kQBytes = kHalves * 16384;      // [half][128 rows x 128 B]
+  static constexpr int kKVBytes = kHalves * CELL * 128;  // [half][CELL rows x 128 B]
+  static constexpr int kStageBytes = kQBytes + 2 * kKVBytes;  // Q, K, V
+  static constexpr int kBytes(int ns) { return ns * kStageBytes + 2 * 16384 + ns * 128 * 4; }
+  // three stages where the SM's shared memory still holds kCtasPerSm CTAs, else two
+  static constexpr int kStages = kCtasPerSm * (kBytes(3) + 3 * 1024) <= 233472 ? 3 : 2;
+  static constexpr int kThreads = 6 * 32;
+  static constexpr int kP = kStages * kStageBytes;  // [2][128 rows x 128 B]
+  static constexpr int kPid = kP + 2 * 16384;       // [kStages][128] pair ids
+  static constexpr int kTotal = kPid + kStages * 128 * 4;
+  // TMEM: S[b] at column 64 b, O[b] at 128 + D b
+  static constexpr uint32_t kCols = D == 64 ? 256 : 512;
+  static_assert(kCtasPerSm * kCols <= 512, "resident CTAs must not oversubscribe TMEM");
+  static_assert(kCtasPerSm * (kTotal + 3 * 1024) <= 233472,
+                "resident CTAs must fit the SM's shared memory");
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// Four rows (y0..y3) of a 2-D tensor map whose box is one row high, columns from x, into four
+// consecutive rows of shared memory (with the map's swizzle), completing on `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0,
+                                            int y1, int y2, int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3),
+      "r"(smem_u32(bar))
+      : "memory");
 }
 
-template <int D>
-constexpr int kCtasPerSm = D == 64 ? 4 : 2;  // TMEM: 4 x 128 or 2 x 256 of 512 columns
-static_assert(kCtasPerSm<64> * LongSmem<64>::kCols <= 512 &&
-                  kCtasPerSm<128> * LongSmem<128>::kCols <= 512,
-              "resident CTAs must not oversubscribe TMEM");
-static_assert(kCtasPerSm<64> * (LongSmem<64>::kTotal + 3 * 1024) <= 233472 &&
-                  kCtasPerSm<128> * (LongSmem<128>::kTotal + 3 * 1024) <= 233472,
-              "resident CTAs must fit the SM's shared memory");
-
 template <int D, int CELL>
-__global__ void __launch_bounds__(kThreadsL, kCtasPerSm<D>)
-    fs_long_tile_kernel(const __grid_constant__ CUtensorMap tmk,
+__global__ void __launch_bounds__(LongSmem<D, CELL>::kThreads, LongSmem<D, CELL>::kCtasPerSm)
+    fs_long_tile_kernel(const __grid_constant__ CUtensorMap tmq,
+                        const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv, const LongTileParams p) {
-  using L = LongSmem<D>;
+  using L = LongSmem<D, CELL>;
+  constexpr int NS = L::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t bars[3];
+  __shared__ __align__(8) uint64_t bars[2 * 3 + 9];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  uint64_t* kv_full = bars + 0;
-  uint64_t* s_done = bars + 1;
-  uint64_t* o_done = bars + 2;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  uint64_t* full = bars;                // [NS] the producer's arrival + the stage's bytes
+  uint64_t* empty = bars + NS;          // [NS] P V of the stage's tile done
+  uint64_t* s_full = bars + 2 * NS;     // [2]
+  uint64_t* p_full = bars + 2 * NS + 2; // [2] 128 softmax threads
+  uint64_t* o_full = bars + 2 * NS + 4; // [2]
+  uint64_t* o_free = bars + 2 * NS + 6; // [2] 128 softmax threads
+  uint64_t* fin = bars + 2 * NS + 8;
+  int* pid_s = reinterpret_cast<int*>(smem + L::kPid);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(kv_full, 1);
-    mbar_init(s_done, 1);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_free[i], 128);
+    }
+    mbar_init(fin, 1);
     fence_mbar_init();
     s_abort = 0;
+    tc::prefetch_tmap(&tmq);
     tc::prefetch_tmap(&tmk);
     tc::prefetch_tmap(&tmv);
   }
-  if (warp == 0) {
+  if (warp == 5) {
     tc::tmem_alloc(&s_tmem, L::kCols);
     tc::tmem_relinquish();
   }
@@ -228,189 +259,280 @@ __global__ void __launch_bounds__(kThreadsL, kCtasPerSm<D>)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = s_tmem;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-  const uint32_t sQ = smem_u32(smem + L::kQ);
-  const int ntiles = (int)min((long long)*p.ntiles, p.tile_cap);  // tiles reserved
-  constexpr uint32_t idS = tc::idesc_bf16(kRowsL, CELL, false, false);
-  constexpr uint32_t idO = tc::idesc_bf16(kRowsL, D, false, true);
+  const int ntiles = (int)min((long long)*p.ntiles, p.tile_cap);
+  const int first = blockIdx.x, stride = gridDim.x;
+  const int my = first < ntiles ? (ntiles - first + stride - 1) / stride : 0;  // this CTA's tiles
+  volatile int* abort_flag = &s_abort;
 
-  for (int t = blockIdx.x, it = 0; t < ntiles; t += gridDim.x, ++it) {
-    const int4 tile = p.tiles[t];
-    const int bh = tile.x / p.C, c = tile.x - bh * p.C;
-    const int m = tile.z;
-    const uint32_t ph = (uint32_t)it & 1u;
-    if (tid == 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * L::kHalves * CELL * 128);
-      const int y = bh * p.n + c * CELL;
+  if (warp == 4) {
+    // ---------------------------------------------------------------- producer
+    const int rows_total = p.rows;  // a row coordinate past the end reads zeros
+    // Descriptors run two tiles ahead and pair ids one tile ahead, so that no load issued here
+    // is waited for in the iteration that issued it.
+    auto desc = [&](int j) {
+      return j < my ? p.tiles[first + j * stride] : make_int4(0, 0, 0, 0);
+    };
+    auto ids = [&](const int4& t, int (&out)[4]) {  // rows 4 lane .. 4 lane + 3 of the tile
 #pragma unroll
-      for (int hf = 0; hf < L::kHalves; ++hf) {
-        tc::tma_load_2d(smem + L::kK + hf * 8192, &tmk, hf * 64, y, kv_full);
-        tc::tma_load_2d(smem + L::kV + hf * 8192, &tmv, hf * 64, y, kv_full);
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int r = 4 * lane + q4;
+        out[q4] = r < t.z ? p.pairs[t.y + r] : -1;
       }
-    }
-    // this thread's query row (zeros past the tile's last pair)
-    int pid = -1;
-    if (tid < m) {
-      pid = p.pairs[tile.y + tid];
-      const __nv_bfloat16* src = p.q + (size_t)(pid / p.K) * D;
+    };
+    int4 tile = desc(0), tile_next = desc(1);
+    int pid[4], pid_next[4];
+    ids(tile, pid);
+    for (int j = 0; j < my; ++j) {
+      const int s = j % NS;
+      bool ok = true;
+      if (j >= NS) ok = mbar_wait_bounded(&empty[s], ((j / NS) - 1) & 1);
+      if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      unsigned char* qs = smem + s * L::kStageBytes;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) pid_s[s * 128 + 4 * lane + q4] = pid[q4];
+      __syncwarp();  // the ids are written before the stage's arrival releases them
+      const int bh = tile.x / p.C, c = tile.x - bh * p.C;
+      if (lane == 0)
+        mbar_arrive_expect_tx(&full[s], L::kHalves * 128 * 128 + 2 * L::kHalves * CELL * 128);
+      __syncwarp();
+      int y[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) y[q4] = pid[q4] >= 0 ? pid[q4] / p.K : rows_total;
 #pragma unroll
       for (int hf = 0; hf < L::kHalves; ++hf)
+        tma_gather4(smem_u32(qs + hf * 16384 + 4 * lane * 128), &tmq, hf * 64, y[0], y[1], y[2],
+                    y[3], &full[s]);
+      if (lane == 0) {
+        const int yk = bh * p.n + c * CELL;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          cp_async16(sQ + hf * 16384 + tc::sw128_offset(tid, ch), src + hf * 64 + ch * 8);
-    } else {
+        for (int hf = 0; hf < L::kHalves; ++hf) {
+          tc::tma_load_2d(qs + L::kQBytes + hf * CELL * 128, &tmk, hf * 64, yk, &full[s]);
+          tc::tma_load_2d(qs + L::kQBytes + L::kKVBytes + hf * CELL * 128, &tmv, hf * 64, yk,
+                          &full[s]);
+        }
+      }
+      ids(tile_next, pid_next);
+      const int4 tile_after = desc(j + 2);
+      tile = tile_next;
+      tile_next = tile_after;
 #pragma unroll
-      for (int hf = 0; hf < L::kHalves; ++hf)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(smem + L::kQ + hf * 16384 + tc::sw128_offset(tid, ch)) =
-              make_uint4(0, 0, 0, 0);
+      for (int q4 = 0; q4 < 4; ++q4) pid[q4] = pid_next[q4];
     }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-      tc::fence_after_sync();
-      if (mbar_wait_bounded(kv_full, ph)) {
+  } else if (warp == 5) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && my > 0) {
+      constexpr uint32_t idS = tc::idesc_bf16(kRowsL, CELL, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(kRowsL, D, false, true);
+      auto issue_s = [&](int j) {
+        const unsigned char* st = smem + (j % NS) * L::kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int hf = kk >> 2, off = (kk & 3) * 32;
-          const uint64_t a = tc::smem_desc_sw128(smem + L::kQ + hf * 16384 + off, 16, 1024);
-          const uint64_t b = tc::smem_desc_sw128(smem + L::kK + hf * 8192 + off, 16, 1024);
-          tc::mma_f16_ss(tmem, a, b, idS, kk > 0 ? 1u : 0u);
+          const uint64_t a = tc::smem_desc_sw128(st + hf * 16384 + off, 16, 1024);
+          const uint64_t b =
+              tc::smem_desc_sw128(st + L::kQBytes + hf * CELL * 128 + off, 16, 1024);
+          tc::mma_f16_ss(tmem + 64u * (uint32_t)(j & 1), a, b, idS, kk > 0 ? 1u : 0u);
         }
-      } else {
-        s_abort = 1;
+        tc::mma_commit(&s_full[j & 1]);
+      };
+      // Issue whichever is ready first: S of tile js (its stage loaded, its S / O buffer free) or
+      // P V of tile jp (its P written).  Each barrier polled is at most one phase ahead of the
+      // phase awaited, so a parity test cannot pass early.
+      bool ok = true;
+      int js = 0, jp = 0;
+      uint32_t idle = 0;
+      while (jp < my) {
+        bool progressed = false;
+        if (js < my && mbar_try_wait(&full[js % NS], (js / NS) & 1) &&
+            (js < 2 || mbar_try_wait(&o_free[js & 1], ((js >> 1) - 1) & 1))) {
+          tc::fence_after_sync();
+          issue_s(js);
+          ++js;
+          progressed = true;
+        }
+        if (jp < js && mbar_try_wait(&p_full[jp & 1], (jp >> 1) & 1)) {
+          tc::fence_after_sync();
+          const unsigned char* st = smem + (jp % NS) * L::kStageBytes;
+          const unsigned char* pt = smem + L::kP + (jp & 1) * 16384;
+#pragma unroll
+          for (int kk = 0; kk < CELL / 16; ++kk) {
+            const uint64_t a = tc::smem_desc_sw128(pt + kk * 32, 16, 1024);
+            const uint64_t b = tc::smem_desc_sw128(st + L::kQBytes + L::kKVBytes + kk * 2048,
+                                                   CELL * 128, 1024);
+            tc::mma_f16_ss(tmem + 128u + (uint32_t)(D * (jp & 1)), a, b, idO, kk > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&o_full[jp & 1]);
+          tc::mma_commit(&empty[jp % NS]);
+          ++jp;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle > (1u << 22) || *abort_flag) {
+          ok = false;
+          break;
+        }
       }
-      tc::mma_commit(s_done);  // also when nothing was issued: the others must not wait forever
+      if (!ok) *abort_flag = 1;
+      tc::mma_commit(fin);  // every MMA issued has completed before TMEM is released
+      if (!mbar_wait_bounded(fin, 0)) *abort_flag = 1;
     }
-    bool ok = mbar_wait_bounded(s_done, ph);
-    tc::fence_after_sync();
-    // softmax over the cell, one row per thread (log2 units)
-    constexpr int kLd = CELL < 32 ? 32 : CELL;
-    float s[kLd];
-#pragma unroll
-    for (int cb = 0; cb < kLd; cb += 32) tc::tmem_ld32(tmem + lane_base + cb, s + cb);
-    tc::tmem_wait_ld();
-    tc::reg_fence(s);
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < CELL; ++j) mx = fmaxf(mx, s[j]);
-    const float m2 = mx * p.c2;
-    float l = 0.f;
-#pragma unroll
-    for (int j = 0; j < CELL; ++j) {
-      s[j] = tc::ex2_approx(fmaf(s[j], p.c2, -m2));
-      l += s[j];
-    }
-#pragma unroll
-    for (int ch = 0; ch < CELL / 8; ++ch) {
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(s[8 * ch + 0], s[8 * ch + 1]);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(s[8 * ch + 2], s[8 * ch + 3]);
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(s[8 * ch + 4], s[8 * ch + 5]);
-      __nv_bfloat162 h3 = __floats2bfloat162_rn(s[8 * ch + 6], s[8 * ch + 7]);
-      *reinterpret_cast<uint4*>(smem + L::kP + tc::sw128_offset(tid, ch)) =
-          make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                     *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
-    }
-    fence_proxy_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
+  } else {
+    // ---------------------------------------------------------------- softmax and epilogue
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    for (int j = 0; j < my; ++j) {
+      const int b = j & 1, s = j % NS;
+      bool ok = mbar_wait_bounded(&full[s], (j / NS) & 1);  // the stage's pair ids
+      const int pid = ok ? pid_s[s * 128 + tid] : -1;
+      ok = ok && mbar_wait_bounded(&s_full[b], (j >> 1) & 1);
+      if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
       tc::fence_after_sync();
-      if (ok && !s_abort) {
+      constexpr int kLd = CELL < 32 ? 32 : CELL;
+      float sv[kLd];
 #pragma unroll
-        for (int kk = 0; kk < CELL / 16; ++kk) {
-          const uint64_t a = tc::smem_desc_sw128(smem + L::kP + kk * 32, 16, 1024);
-          const uint64_t b = tc::smem_desc_sw128(smem + L::kV + kk * 2048, 8192, 1024);
-          tc::mma_f16_ss(tmem + 64u, a, b, idO, kk > 0 ? 1u : 0u);
-        }
-      }
-      tc::mma_commit(o_done);
-    }
-    ok = mbar_wait_bounded(o_done, ph) && ok;
-    tc::fence_after_sync();
-    const bool stop = __syncthreads_or(!ok || s_abort);
-    if (stop) {
-      if (tid == 0) s_abort = 1;
-      break;
-    }
-    // normalised output row (bf16) and (max, sum) to the pair's record
-    const float inv_l = 1.f / l;
-#pragma unroll
-    for (int cb = 0; cb < D; cb += 32) {
-      float o[32];
-      tc::tmem_ld32(tmem + lane_base + 64u + cb, o);
+      for (int cb = 0; cb < kLd; cb += 32) tc::tmem_ld32(tmem + lane_base + 64u * b + cb, sv + cb);
       tc::tmem_wait_ld();
-      tc::reg_fence(o);
-      if (pid >= 0) {
-        uint4* dst = reinterpret_cast<uint4*>(p.part_o + (size_t)pid * D + cb);
+      tc::reg_fence(sv);
+      float mx = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * e + 0] * inv_l, o[8 * e + 1] * inv_l);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * e + 2] * inv_l, o[8 * e + 3] * inv_l);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * e + 4] * inv_l, o[8 * e + 5] * inv_l);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * e + 6] * inv_l, o[8 * e + 7] * inv_l);
-          dst[e] = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
-                              *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+      for (int e = 0; e < CELL; ++e) mx = fmaxf(mx, sv[e]);
+      const float m2 = mx * p.c2;
+      float l = 0.f;
+#pragma unroll
+      for (int e = 0; e < CELL; ++e) {
+        sv[e] = tc::ex2_approx(fmaf(sv[e], p.c2, -m2));
+        l += sv[e];
+      }
+      unsigned char* pt = smem + L::kP + b * 16384;
+#pragma unroll
+      for (int ch = 0; ch < CELL / 8; ++ch) {
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(sv[8 * ch + 0], sv[8 * ch + 1]);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(sv[8 * ch + 2], sv[8 * ch + 3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(sv[8 * ch + 4], sv[8 * ch + 5]);
+        __nv_bfloat162 h3 = __floats2bfloat162_rn(sv[8 * ch + 6], sv[8 * ch + 7]);
+        *reinterpret_cast<uint4*>(pt + tc::sw128_offset(tid, ch)) =
+            make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                       *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+      }
+      fence_proxy_async();
+      tc::fence_before_sync();
+      mbar_arrive(&p_full[b]);
+      ok = mbar_wait_bounded(&o_full[b], (j >> 1) & 1);
+      if (!__all_sync(0xffffffffu, ok)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc::fence_after_sync();
+      // normalised output row (bf16) and (max, sum) to the pair's record
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 64) {  // 64 columns per TMEM round trip
+        float o[64];
+        tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)(D * b) + c0, o);
+        tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)(D * b) + c0 + 32, o + 32);
+        tc::tmem_wait_ld();
+        tc::reg_fence(o);
+        if (pid >= 0) {
+          uint4* dst = reinterpret_cast<uint4*>(p.part_o + (size_t)pid * D + c0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(o[8 * e + 0] * inv_l, o[8 * e + 1] * inv_l);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(o[8 * e + 2] * inv_l, o[8 * e + 3] * inv_l);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(o[8 * e + 4] * inv_l, o[8 * e + 5] * inv_l);
+            __nv_bfloat162 h3 = __floats2bfloat162_rn(o[8 * e + 6] * inv_l, o[8 * e + 7] * inv_l);
+            dst[e] =
+                make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                           *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
+          }
         }
       }
+      if (pid >= 0) p.part_ml[pid] = make_float2(m2, l);
+      tc::fence_before_sync();
+      mbar_arrive(&o_free[b]);
     }
-    if (pid >= 0) p.part_ml[pid] = make_float2(m2, l);
-    tc::fence_before_sync();
-    __syncthreads();  // TMEM and shared memory are reused by the next tile
   }
   tc::fence_before_sync();
   __syncthreads();
   if (s_abort && tid == 0) report_timeout(p.status, 7);
-  if (warp == 0) {
+  if (warp == 5) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, L::kCols);
   }
 }
 
 // ---- 5. merge a query's partials and mix into the short-branch output -----------------------
+// Sixteen lanes per query (two queries per warp, d / 16 elements per lane); every load of the
+// query (its slots' positions and (max, sum), all K partial rows, the short-branch row) is issued
+// up front, so each warp waits for memory once.  Slots that were not attended have no record:
+// their loads are in bounds but unused (selected away, never multiplied, so whatever the buffer
+// holds cannot leak into the result).
 template <int D>
 __global__ void __launch_bounds__(256)
     fs_long_combine_kernel(const int* __restrict__ slotpos, const float2* __restrict__ part_ml,
                            const __nv_bfloat16* __restrict__ part_o,
                            const float* __restrict__ alpha, int H, int n, int K, long long rows,
                            __nv_bfloat16* __restrict__ o) {
-  constexpr int E = D / 32;  // elements per lane
-  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  float M = -INFINITY;
-  for (int k = 0; k < K; ++k)
-    if (slotpos[row * K + k] >= 0) M = fmaxf(M, part_ml[row * K + k].x);
-  if (M == -INFINITY) return;  // no cell attended: o keeps the short branch
+  constexpr int E = D / 16;  // elements per lane: 4 (8-byte loads) or 8 (16-byte loads)
+  using V = typename std::conditional<E == 4, uint2, uint4>::type;
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+  const int lane = threadIdx.x & 31, sub = lane & 15, seg = lane & 16;
+  const bool live = row < rows;
+  const long long r0 = (live ? row : 0) * K;
+  const int sp = live && sub < K ? slotpos[r0 + sub] : -1;
+  const float2 ml = live && sub < K ? part_ml[r0 + sub] : make_float2(-INFINITY, 0.f);
+  V part[kMaxKL];
+#pragma unroll
+  for (int k = 0; k < kMaxKL; ++k)
+    if (live && k < K)
+      part[k] = *reinterpret_cast<const V*>(part_o + (size_t)(r0 + k) * D + sub * E);
+  __nv_bfloat16* dst = o + (size_t)(live ? row : 0) * D + sub * E;
+  V sh{};
+  if (live) sh = *reinterpret_cast<const V*>(dst);
+  const bool valid = sp >= 0;
+  float M = valid ? ml.x : -INFINITY;
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  M = __shfl_sync(0xffffffffu, M, seg);  // sub-lanes 0 .. 7 hold the slots
+  const float w = valid ? ml.y * exp2f(ml.x - M) : 0.f;  // the slot's share of the softmax mass
+  float Lsum = w;
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
+  Lsum = __shfl_sync(0xffffffffu, Lsum, seg);
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float Lsum = 0.f;
-  for (int k = 0; k < K; ++k) {
-    if (slotpos[row * K + k] < 0) continue;
-    const float2 ml = part_ml[row * K + k];
-    const float w = ml.y * exp2f(ml.x - M);  // this pair's share of the softmax mass
-    Lsum += w;
-    const __nv_bfloat16* src = part_o + (size_t)(row * K + k) * D + lane * E;
 #pragma unroll
-    for (int e = 0; e < E; e += 2) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + e));
-      acc[e] = fmaf(w, f.x, acc[e]);
-      acc[e + 1] = fmaf(w, f.y, acc[e + 1]);
+  for (int k = 0; k < kMaxKL; ++k) {
+    if (k >= K) break;
+    const float wk = __shfl_sync(0xffffffffu, w, seg + k);
+    const bool vk = __shfl_sync(0xffffffffu, valid ? 1 : 0, seg + k) != 0;
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&part[k]);
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      acc[2 * e] += vk ? wk * f.x : 0.f;
+      acc[2 * e + 1] += vk ? wk * f.y : 0.f;
     }
   }
+  if (!live || M == -INFINITY) return;  // no cell attended: o keeps the short branch
   const float a = alpha[(row / n) % H];
   const float inv = 1.f / Lsum;
-  __nv_bfloat16* dst = o + (size_t)row * D + lane * E;
+  V out;
+  const __nv_bfloat162* hs = reinterpret_cast<const __nv_bfloat162*>(&sh);
+  __nv_bfloat162* ho = reinterpret_cast<__nv_bfloat162*>(&out);
 #pragma unroll
-  for (int e = 0; e < E; e += 2) {
-    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dst + e));
-    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(
-        (1.f - a) * f.x + a * (acc[e] * inv), (1.f - a) * f.y + a * (acc[e + 1] * inv));
+  for (int e = 0; e < E / 2; ++e) {
+    const float2 f = __bfloat1622float2(hs[e]);
+    ho[e] = __floats2bfloat162_rn((1.f - a) * f.x + a * (acc[2 * e] * inv),
+                                  (1.f - a) * f.y + a * (acc[2 * e + 1] * inv));
   }
+  *reinterpret_cast<V*>(dst) = out;
 }
 
 // ---- host side ------------------------------------------------------------------------------
@@ -467,6 +589,11 @@ int persistent_grid(const void* kern, int smem, int per_sm) {
   return sms * per_sm;
 }
 
+template <typename T>
+struct Tag {
+  using type = T;
+};
+
 }  // namespace
 
 bool long_cells_supported(int d, int cell, int K, long long rows) {
@@ -502,36 +629,38 @@ bsa_status long_cells(const void* q, const void* k, const void* v, int B, int H,
   fs_long_scatter_kernel<<<(unsigned)((rows * K + 255) / 256), 256, 0, st>>>(
       idx, w.slotpos, n, K, C, rows, w.cell_off, w.pairs);
   BSA_LAUNCH_CHECK();
-  CUtensorMap tmk, tmv;
-  if (!map_cells(&tmk, k, rows, d, cell) || !map_cells(&tmv, v, rows, d, cell)) return BSA_ERR_CUDA;
+  CUtensorMap tmq, tmk, tmv;
+  if (!map_cells(&tmq, q, rows, d, 1) || !map_cells(&tmk, k, rows, d, cell) ||
+      !map_cells(&tmv, v, rows, d, cell))
+    return BSA_ERR_CUDA;
   LongTileParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.tiles = w.tiles; p.ntiles = w.ntiles; p.pairs = w.pairs;
   p.part_ml = w.part_ml; p.part_o = w.part_o; p.status = status;
-  p.n = n; p.C = C; p.K = K; p.tile_cap = w.tile_cap;
+  p.n = n; p.C = C; p.K = K; p.rows = (int)rows; p.tile_cap = w.tile_cap;
   p.c2 = 1.4426950408889634f / sqrtf((float)d);
-  auto run = [&](auto kern, int smem) -> bsa_status {
-    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), smem,
-                                     d == 64 ? kCtasPerSm<64> : kCtasPerSm<128>);
+  auto run = [&](auto kern, int smem, int threads, int per_sm) -> bsa_status {
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), smem, per_sm);
     if (grid < 1) return BSA_ERR_CUDA;
-    kern<<<grid, kThreadsL, smem, st>>>(tmk, tmv, p);
+    kern<<<grid, threads, smem, st>>>(tmq, tmk, tmv, p);
     BSA_LAUNCH_CHECK();
     return BSA_OK;
   };
+  auto run_dc = [&](auto kern, auto tag) -> bsa_status {
+    using L = typename decltype(tag)::type;
+    return run(kern, L::kTotal + 1024, L::kThreads, L::kCtasPerSm);
+  };
   bsa_status rc;
-  if (d == 64) {
-    constexpr int sm = LongSmem<64>::kTotal + 1024;
-    rc = cell == 16 ? run(fs_long_tile_kernel<64, 16>, sm)
-         : cell == 32 ? run(fs_long_tile_kernel<64, 32>, sm)
-                      : run(fs_long_tile_kernel<64, 64>, sm);
-  } else {
-    constexpr int sm = LongSmem<128>::kTotal + 1024;
-    rc = cell == 16 ? run(fs_long_tile_kernel<128, 16>, sm)
-         : cell == 32 ? run(fs_long_tile_kernel<128, 32>, sm)
-                      : run(fs_long_tile_kernel<128, 64>, sm);
-  }
+  if (d == 64)
+    rc = cell == 16   ? run_dc(fs_long_tile_kernel<64, 16>, Tag<LongSmem<64, 16>>{})
+         : cell == 32 ? run_dc(fs_long_tile_kernel<64, 32>, Tag<LongSmem<64, 32>>{})
+                      : run_dc(fs_long_tile_kernel<64, 64>, Tag<LongSmem<64, 64>>{});
+  else
+    rc = cell == 16   ? run_dc(fs_long_tile_kernel<128, 16>, Tag<LongSmem<128, 16>>{})
+         : cell == 32 ? run_dc(fs_long_tile_kernel<128, 32>, Tag<LongSmem<128, 32>>{})
+                      : run_dc(fs_long_tile_kernel<128, 64>, Tag<LongSmem<128, 64>>{});
   if (rc != BSA_OK) return rc;
-  const unsigned cblocks = (unsigned)((rows * 32 + 255) / 256);
+  const unsigned cblocks = (unsigned)((rows * 16 + 255) / 256);
   if (d == 64)
     fs_long_combine_kernel<64><<<cblocks, 256, 0, st>>>(w.slotpos, w.part_ml, w.part_o, alpha, H,
                                                          n, K, rows,

@@ -94,6 +94,50 @@ def test_freesolo_cell_sizes(cell):
     check_rows(case, idx, cnt, o, rows)
 
 
+@pytest.mark.parametrize("cell", [16, 64])
+def test_freesolo_cell_sizes_d128(cell):
+    """d = 128 with the smallest and largest cells the cell-major long branch tiles (three and
+    two gather stages)."""
+    case = inputs.freesolo_case(48, B=1, H=2, d=128, n=1300, cell=cell, q_block=128, K=4,
+                                window=150, sigma=700.0)
+    idx, cnt, o = run_gpu(case)
+    rng = np.random.default_rng(12)
+    rows = [(0, h, i) for h in range(2) for i in
+            sorted(set([0, 127, 128, 640, 1299]) | set(rng.integers(0, 1300, 12).tolist()))]
+    check_rows(case, idx, cnt, o, rows)
+
+
+def test_freesolo_attn_repeated_and_late_cells():
+    """Caller-given slots: a cell repeated within a query's slots counts once, and a cell that
+    is not wholly at or before the query is ignored; the long branch uses the rest."""
+    case = inputs.freesolo_case(47, B=1, H=2, d=64, n=1024, cell=32, q_block=128, K=4,
+                                window=128, sigma=500.0)
+    q, k, v = (torch.from_numpy(x).to(DEV, torch.bfloat16) for x in (case.q, case.k, case.v))
+    lam = torch.from_numpy(case.lam).to(DEV)
+    sig = torch.from_numpy(case.sigma).to(DEV)
+    alpha = torch.from_numpy(case.alpha).to(DEV)
+    mean_k, mx, ce = bsa.build_block_summaries(k, case.cell)
+    idx, cnt = bsa.freesolo_select(q, mean_k, mx, ce, lam, sig, case.cell, case.q_block, case.K)
+    rows = [(0, h, i) for h in range(2) for i in (300, 517, 700, 1000)]
+    for (bi, h, i) in rows:
+        idx[bi, h, i, 1] = idx[bi, h, i, 0]   # repeated
+        idx[bi, h, i, 2] = i // case.cell     # the query's own cell: ends after i
+    o = bsa.freesolo_attn(q, k, v, alpha, idx, cnt, case.cell, case.window, case.rope_theta)
+    torch.cuda.synchronize()
+    idx_h, o_h = idx.cpu().numpy(), o.float().cpu().numpy()
+    for (bi, h, i) in rows:
+        keep = sorted({int(c) for c in idx_h[bi, h, i] if c >= 0 and (c + 1) * case.cell <= i + 1})
+        assert len(keep) == 2
+        summ = orc.block_summaries(case.k[bi, h], case.cell)
+        ref, _ = orc.freesolo_row(case.q[bi, h, i], case.k[bi, h], case.v[bi, h], i, summ,
+                                  cell=case.cell, q_block=case.q_block, K=case.K,
+                                  window=case.window, lam=float(case.lam[h]),
+                                  sigma=float(case.sigma[h]), alpha=float(case.alpha[h]),
+                                  theta=case.rope_theta, selection=keep)
+        err = float(np.max(np.abs(o_h[bi, h, i] - ref)))
+        assert err < 2e-2, (bi, h, i, err)
+
+
 def test_freesolo_select_two_batches_many_cells():
     """B = 2, 40 cells of 16 per query block: several 256-cell chunks and a ragged last chunk."""
     case = inputs.freesolo_case(43, B=2, H=3, d=64, n=5000, cell=16, q_block=128, K=5,
