@@ -472,18 +472,19 @@ def run_gpu(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
         sampler.mark("t0")
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        # events bracket the K steps only: an event recorded between two replays costs the step
+        # about 2 us (it ends the overlap of one launch's tail with the next one's start)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record(stream)
         for i in range(args.steps):
             graphs[i % R].replay()
-            ev[i + 1].record(stream)
+        ev[1].record(stream)
         torch.cuda.synchronize(dev)
         sampler.mark("t1")
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
-    step_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[args.steps])
+    total_ms = ev[0].elapsed_time(ev[1])
 
     # the same step through the separate calls (score, Top-K, attention), for the breakdown
     sep = []
@@ -534,6 +535,69 @@ def run_gpu(args):
     sep_attn = statistics.fmean(e[2].elapsed_time(e[3]) for e in sep) * 1e3
     sep_step = statistics.fmean(e[0].elapsed_time(e[3]) for e in sep) * 1e3
 
+    # GQA-shared selection and bf16 summaries (bsa_decode_step_ex flags): time per step on the same
+    # rotated layers, algorithmic bytes, and how far the selection moves from the per-head fp32 one
+    variants = {}
+    ref_sets = [set(int(x) for x in row if x >= 0) for row in idx_h.reshape(-1, K)]
+    for name, flags in (("bf16_summaries", bsa.DECODE_BF16_SUMMARIES),
+                        ("per_head_fp32_control", 0),
+                        ("shared_selection", bsa.DECODE_SHARED_SELECTION),
+                        ("shared_bf16", bsa.DECODE_SHARED_SELECTION | bsa.DECODE_BF16_SUMMARIES)):
+        bf16_sum = bool(flags & bsa.DECODE_BF16_SUMMARIES)
+        # every buffer a captured graph uses stays referenced as long as the graphs live:
+        # entering a capture empties the allocator's cache, so a buffer kept alive only by a
+        # replaced closure would go back to the driver and its graph would replay into freed memory
+        vgraphs, vbufs, vidx = [], [], None
+        with torch.cuda.stream(stream):
+            for r, L in enumerate(layers):
+                mk = bsa.round_summaries_bf16(L["mean_k"]) if bf16_sum else L["mean_k"].clone()
+                ix = torch.empty(B, Hq, K, device=dev, dtype=torch.int32)
+                vbufs.append((mk, ix))
+
+                def vstep(L=L, mk=mk, ix=ix):
+                    bsa.decode_step_ex(L["q"], L["k"], L["v"], mk, b, K, flags, append=True,
+                                       max_norm=L["max_norm"], centre=L["centre"], o=L["o"],
+                                       lse=L["lse"], idx=ix, count=L["count"], status=status)
+                vstep()
+                torch.cuda.synchronize(dev)
+                if r == 0:
+                    vidx = ix.cpu().numpy()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    vstep()
+                vgraphs.append(g)
+            nv = max(50, min(args.steps, 400))
+            for i in range(args.warmup):
+                vgraphs[i % R].replay()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for i in range(nv):
+                vgraphs[i % R].replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        v_us = e0.elapsed_time(e1) / nv * 1e3
+        del vgraphs  # graphs first, then the buffers they replay into
+        del vbufs
+        v_union = v_hits = 0
+        for bi in range(B):
+            for kh in range(Hk):
+                sel = set(int(x) for x in vidx[bi, kh * G:(kh + 1) * G].ravel() if x >= 0)
+                v_union += len(sel) + 1
+                blocks = case.needles.get((bi, kh), [])
+                v_hits += len(sel & set(int(c) for c in blocks))
+        v_kv = (v_union - B * Hk) * b * d * 2 * 2 + B * Hk * cur_tokens * d * 2 * 2
+        v_sum = B * Hk * cur * d * (2 if bf16_sum else 4)
+        v_bytes = v_kv + v_sum + io_bytes
+        agree = statistics.fmean(
+            len(ref & set(int(x) for x in row if x >= 0)) / max(1, len(ref))
+            for ref, row in zip(ref_sets, vidx.reshape(-1, K)))
+        variants[name] = {"us_per_step": v_us, "tokens_per_s": B / (v_us / 1e6),
+                          "algorithmic_bytes": v_bytes, "gbs": v_bytes / (v_us / 1e6) / 1e9,
+                          "frac_of_hbm": v_bytes / (v_us / 1e6) / 1e9 / load_peaks()["hbm_gbs"],
+                          "union_blocks": v_union, "needle_recall": v_hits / max(1, tot),
+                          "index_agreement_vs_per_head_fp32": agree}
+
     # end to end through the public API: pinned host q in, the bsa_decode_step call (binding ->
     # C-ABI, no graph), o out, every step
     q_host = [torch.from_numpy(np.ascontiguousarray(L["q"].float().cpu().numpy()))
@@ -569,7 +633,7 @@ def run_gpu(args):
     e2e_value = tokens / (e2e_total / 1e3)
 
     peaks = load_peaks()
-    avg_ms = statistics.fmean(step_ms)
+    avg_ms = total_ms / args.steps  # one fused kernel per step
     achieved = (step_bytes + io_bytes) / (avg_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -593,6 +657,7 @@ def run_gpu(args):
                 "what": "selected K/V (union per GQA group) + summaries, per step time"},
         "separate_calls_us": {"append+score": sep_sel, "topk": sep_topk, "attention": sep_attn,
                               "step": sep_step},
+        "variants": variants,
         "union_blocks": union_blocks, "per_head_blocks": per_head_blocks,
         "needle_recall": hits / max(1, tot), "status_word": st_word,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * Hq * d * 2,

@@ -34,6 +34,9 @@ SIGNATURES = [
     ("bsa_topk_blocks", _I, [_P, _I, _I, _I, _P, _I, _I, _I, _I, _P, _P, _P]),
     ("bsa_decode_step", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P,
                              _I, _I, _P, _P, _P, _P, _P, _P]),
+    ("bsa_decode_step_ex", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P,
+                                _P, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
+    ("bsa_round_summaries_bf16", _I, [_P, _P, ctypes.c_longlong, _P]),
     ("bsa_sparse_attn_fwd", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _I,
                                  _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
     ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -399,6 +402,45 @@ def decode_step_fused(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_nor
                                  K, _ptr(o), _ptr(lse), _ptr(idx), _ptr(count), _ptr(status),
                                  _stream(q.device)), "bsa_decode_step")
     return o, lse, idx, count
+
+
+DECODE_SHARED_SELECTION = 1
+DECODE_BF16_SUMMARIES = 2
+
+
+def decode_step_ex(q, k, v, mean_k, b, K, flags, seq_lens=None, append=True, max_norm=None,
+                   centre=None, lambda_h=None, sigma_h=None, prefix_block=0, o=None, lse=None,
+                   idx=None, count=None, status=None):
+    """bsa_decode_step_ex: the fused decode step with the variants of DECODE_* flags (shared
+    selection per kv head; bf16 mean keys).  Returns (o, lse, idx, count)."""
+    _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    if idx is None:
+        idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b,
+                                    _ptr(_i32(seq_lens)), _ptr(mean_k), _ptr(max_norm),
+                                    _ptr(centre), 1 if append else 0, _ptr(lambda_h),
+                                    _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse), _ptr(idx),
+                                    _ptr(count), _ptr(status), int(flags), _stream(q.device)),
+           "bsa_decode_step_ex")
+    return o, lse, idx, count
+
+
+def round_summaries_bf16(mean_k, out=None):
+    """bf16 copy of float32 mean keys (round to nearest even), for DECODE_BF16_SUMMARIES."""
+    _cuda(mean_k, out)
+    if out is None:
+        out = torch.empty(mean_k.shape, device=mean_k.device, dtype=torch.bfloat16)
+    _check(lib().bsa_round_summaries_bf16(_ptr(mean_k), _ptr(out), mean_k.numel(),
+                                          _stream(mean_k.device)), "bsa_round_summaries_bf16")
+    return out
 
 
 def decode_step(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_norm=None, centre=None,

@@ -26,6 +26,10 @@
 //      holding the current block also rewrites that block's summary from shared memory.
 //   4. Each CTA merges its warps, then pushes to CTA r' the partial (m, l, o) of the output columns
 //      CTA r' owns; cluster barrier; each CTA finishes its columns and writes o (and lse).
+// Variants (flags of bsa_decode_step_ex): shared selection -- the group's score of a block is the
+// mean of its G heads' scores, ranked once and attended by every head (one selection per kv
+// head instead of G); bf16 summaries -- the mean keys are read (and appended) in bf16, halving the
+// summary bytes, with fp32 accumulation of the dot products.
 // Every CTA reaches every cluster barrier (no early exit); every mbarrier wait is bounded.
 #include <cudaTypedefs.h>
 
@@ -56,7 +60,7 @@ struct FusedParams {
   const void* v;
   int B, Hq, Hk, n, b, C, K;
   const int* seq_lens;
-  float* mean_k;
+  void* mean_k;  // [B, Hk, C, d] in the summary type (fp32, or bf16 on the 64-token bf16 path)
   float* max_norm;
   float* centre;
   int append;
@@ -69,6 +73,7 @@ struct FusedParams {
   int* count;
   int* status;
   int chunk;  // history blocks scored per CTA (multiple of kSub)
+  int shared;  // one selection per kv head from the mean of its heads' scores
 };
 
 // ---- cluster helpers ---------------------------------------------------------------------
@@ -289,7 +294,7 @@ struct FusedSmem {
   }
 };
 
-template <typename T, int D, int G, bool MMA>
+template <typename T, typename TS, int D, int G, bool MMA>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const FusedParams p) {
@@ -325,7 +330,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   nc = max(0, min(nc, cur));
 
   using SM = FusedSmem<T, D, G, MMA>;
-  float* ring = reinterpret_cast<float*>(smem);
+  TS* ring = reinterpret_cast<TS*>(smem);  // fits: region A holds 2 x kSub fp32 rows
+  TS* mean_k = static_cast<TS*>(p.mean_k);
+  const int Gs = p.shared ? 1 : G;  // selections made per group
   unsigned char* after_a = smem + SM::region_a(b);
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(after_a);                  // [G][chunk]
   unsigned char* merge = after_a + SM::scores(p.chunk);                        // [G][CL*K] x 2
@@ -363,11 +370,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int c_hi = min(nc, c_lo + p.chunk);
   const int rows = c_hi - c_lo;
   const int nsub = (rows + kSub - 1) / kSub;
-  const float* mk = p.mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
+  const TS* mk = mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
   auto issue_sub = [&](int j) {
     const int r0 = c_lo + j * kSub;
     const int nr = min(kSub, c_hi - r0);
-    const uint32_t bytes = (uint32_t)(nr * D * sizeof(float));
+    const uint32_t bytes = (uint32_t)(nr * D * sizeof(TS));
     mbar_arrive_expect_tx(&bar[j & 1], bytes);
     bulk_g2s(ring + (size_t)(j & 1) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j & 1]);
   };
@@ -383,14 +390,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     if (!s_abort) {
       const int r0 = j * kSub;
       const int nr = min(kSub, rows - r0);
-      const float* base = ring + (size_t)(j & 1) * kSub * D;
+      const TS* base = ring + (size_t)(j & 1) * kSub * D;
       for (int t0 = warp * R; t0 < nr; t0 += kWarps * R) {
         float a[32];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           float x[EPL];
           if (t0 + r < nr) {
-            load_vec<float, EPL>(base + (size_t)(t0 + r) * D + lane * EPL, x);
+            load_vec<TS, EPL>(base + (size_t)(t0 + r) * D + lane * EPL, x);
           } else {
 #pragma unroll
             for (int e = 0; e < EPL; ++e) x[e] = 0.f;
@@ -405,21 +412,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         }
         warp_transpose_reduce32(a, lane);
         const int t = t0 + my_r;
-        if (t < nr) {
-          float s = a[0] * scale;
-          if (p.lam) {
-            const size_t row = (size_t)(bi * p.Hk + kh) * p.C + c_lo + r0 + t;
-            s += lam_h * p.max_norm[row] * erff(((float)pos - p.centre[row]) * inv2sig);
-          }
-          s_keys[my_g * p.chunk + r0 + t] = order_key(s);
+        float s = a[0] * scale;
+        if (p.lam && t < nr) {
+          const size_t row = (size_t)(bi * p.Hk + kh) * p.C + c_lo + r0 + t;
+          s += lam_h * p.max_norm[row] * erff(((float)pos - p.centre[row]) * inv2sig);
         }
+        if (p.shared) {  // mean over the G lanes of this row (lane = my_r * G + my_g)
+#pragma unroll
+          for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          s *= 1.f / (float)G;
+        }
+        if (t < nr && my_g < Gs) s_keys[my_g * p.chunk + r0 + t] = order_key(s);
       }
     }
     __syncthreads();
     if (tid == 0 && j + 2 < nsub && !s_abort) issue_sub(j + 2);
   }
-  // local Top-K per head, pushed into every CTA's merge buffer at slot rank*K
-  for (int g = warp; g < G; g += kWarps) {
+  // local Top-K per head (per group when shared), pushed into every CTA's merge buffer at slot
+  // rank*K
+  for (int g = warp; g < Gs; g += kWarps) {
     const uint32_t* keys = s_keys + g * p.chunk;
     const int cnt = warp_select(keys, rows, K, lane, s_pick[g]);
     for (int e = lane; e < CL * K; e += 32) {
@@ -436,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   // ---- 2. global Top-K per head, then the union -------------------------------------------
   const int nwords = (nc + 31) / 32;
   for (int w = tid; w < nwords; w += kThreads) s_bits[w] = 0u;
-  for (int g = warp; g < G; g += kWarps) {
+  for (int g = warp; g < Gs; g += kWarps) {
     // empty slots carry key 0 and index -1: compact the valid ones first (index order kept)
     uint32_t* mk_g = m_key + g * CL * K;
     int* mi_g = m_idx + g * CL * K;
@@ -463,13 +474,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __syncthreads();
   if (rank == 0) {  // optional outputs: the selection of every head
     for (int e = tid; e < G * K; e += kThreads) {
-      const int g = e / K, j = e % K;
+      const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
       const size_t row = (size_t)bi * Hq + h0 + g;
-      if (p.idx) p.idx[row * K + j] = j < s_nsel[g] ? s_sel[g][j] : -1;
-      if (p.count && j == 0) p.count[row] = s_nsel[g];
+      if (p.idx) p.idx[row * K + j] = j < s_nsel[gs] ? s_sel[gs][j] : -1;
+      if (p.count && j == 0) p.count[row] = s_nsel[gs];
     }
   }
-  for (int e = tid; e < G * K; e += kThreads) {
+  for (int e = tid; e < Gs * K; e += kThreads) {
     const int g = e / K, j = e % K;
     if (j < s_nsel[g]) {
       const int x = s_sel[g][j];
@@ -505,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   }
   __syncthreads();
   const int U = s_U;
-  for (int e = tid; e < G * K; e += kThreads) {  // head masks by binary search in the union
+  for (int e = tid; e < Gs * K; e += kThreads) {  // head masks by binary search in the union
     const int g = e / K, j = e % K;
     if (j < s_nsel[g]) {
       const int x = s_sel[g][j];
@@ -514,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         const int mid = (lo + hi) >> 1;
         if (s_ublk[mid] < x) lo = mid + 1; else hi = mid;
       }
-      atomicOr(&s_umask[lo], 1u << g);
+      atomicOr(&s_umask[lo], p.shared ? (1u << G) - 1u : 1u << g);
     }
   }
   __syncthreads();
@@ -676,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
           for (int t = 0; t < tok; ++t)
             sum += Elem<T>::to_f(*reinterpret_cast<const T*>(
                 kt + hf * 8192 + t * 128 + ((cin ^ (t & 7)) << 4) + e8 * 2));
-          p.mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = sum / (float)tok;
+          mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = Elem<TS>::from_f(sum / (float)tok);
         }
         // max key norm: thread t < tok takes token t
         float nrm = 0.f;
@@ -802,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         for (int col = tid; col < D; col += kThreads) {
           float sum = 0.f;
           for (int t = 0; t < tok; ++t) sum += Elem<T>::to_f(kt[(size_t)t * D + col]);
-          p.mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = sum / (float)tok;
+          mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = Elem<TS>::from_f(sum / (float)tok);
         }
         float nmax = 0.f;
         for (int t = warp; t < tok; t += kWarps) {
@@ -990,7 +1001,7 @@ LaunchCache& launch_cache() {
   return c;
 }
 
-template <typename T, int D, int G, bool MMA>
+template <typename T, typename TS, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   using SM = FusedSmem<T, D, G, MMA>;
   CUtensorMap tmk{}, tmv{};
@@ -1000,7 +1011,7 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   }
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
-  auto kern = decode_fused_kernel<T, D, G, MMA>;
+  auto kern = decode_fused_kernel<T, TS, D, G, MMA>;
   for (;;) {
     const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
     if (chunk > 32 * kSelItems) {  // the local select holds at most 512 keys per head
@@ -1071,13 +1082,13 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   }
 }
 
-template <typename T, int D, bool MMA>
+template <typename T, typename TS, int D, bool MMA>
 bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_fused<T, D, 1, MMA>(p, st);
-    case 2: return launch_fused<T, D, 2, MMA>(p, st);
-    case 4: return launch_fused<T, D, 4, MMA>(p, st);
-    case 8: return launch_fused<T, D, 8, MMA>(p, st);
+    case 1: return launch_fused<T, TS, D, 1, MMA>(p, st);
+    case 2: return launch_fused<T, TS, D, 2, MMA>(p, st);
+    case 4: return launch_fused<T, TS, D, 4, MMA>(p, st);
+    case 8: return launch_fused<T, TS, D, 8, MMA>(p, st);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }
@@ -1085,17 +1096,19 @@ bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st) {
 }  // namespace
 }  // namespace bsa
 
-extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtype dt,
-                                      int B, int Hq, int Hk, int n, int d, int b,
-                                      const int* seq_lens, float* mean_k, float* max_norm,
-                                      float* centre, int append, const float* lambda_h,
-                                      const float* sigma_h, int prefix_block, int K, void* o,
-                                      float* lse, int* idx, int* count, int* status,
-                                      void* stream) {
+extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v,
+                                         bsa_dtype dt, int B, int Hq, int Hk, int n, int d, int b,
+                                         const int* seq_lens, void* mean_k, float* max_norm,
+                                         float* centre, int append, const float* lambda_h,
+                                         const float* sigma_h, int prefix_block, int K, void* o,
+                                         float* lse, int* idx, int* count, int* status,
+                                         int flags, void* stream) {
   using namespace bsa;
   BSA_REQUIRE(dtype_ok(dt), BSA_ERR_DTYPE);
   BSA_REQUIRE(q && k && v && mean_k && o, BSA_ERR_ARG);
   BSA_REQUIRE(B > 0 && Hq > 0 && Hk > 0 && n > 0 && d > 0 && b > 0 && K > 0 && prefix_block >= 0,
+              BSA_ERR_ARG);
+  BSA_REQUIRE((flags & ~(BSA_DECODE_SHARED_SELECTION | BSA_DECODE_BF16_SUMMARIES)) == 0,
               BSA_ERR_ARG);
   BSA_REQUIRE((lambda_h == nullptr) == (sigma_h == nullptr), BSA_ERR_ARG);
   BSA_REQUIRE(!lambda_h || (max_norm && centre), BSA_ERR_ARG);
@@ -1106,6 +1119,9 @@ extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* 
   BSA_REQUIRE((size_t)b * d * (dt == BSA_BF16 ? 2 : 4) <= 32768, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(B <= 65535 && Hk <= 65535, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(all_aligned16(q, k, v, o, mean_k), BSA_ERR_ARG);
+  const bool bf16_sum = (flags & BSA_DECODE_BF16_SUMMARIES) != 0;
+  // bf16 summaries ride on the 64-token bf16 path (warp MMAs over TMA tiles)
+  BSA_REQUIRE(!bf16_sum || (dt == BSA_BF16 && b == 64), BSA_ERR_UNSUPPORTED);
   const int C = ceil_div(n, b);
   BSA_REQUIRE(C <= kMaxWords * 32, BSA_ERR_UNSUPPORTED);
   FusedParams p{};
@@ -1114,18 +1130,35 @@ extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* 
   p.seq_lens = seq_lens; p.mean_k = mean_k; p.max_norm = max_norm; p.centre = centre;
   p.append = append; p.lam = lambda_h; p.sig = sigma_h; p.prefix_block = prefix_block;
   p.o = o; p.lse = lse; p.idx = idx; p.count = count; p.status = status;
+  p.shared = (flags & BSA_DECODE_SHARED_SELECTION) != 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  using bf = __nv_bfloat16;
   bsa_status rc;
-  if (dt == BSA_BF16 && b == 64)  // 64-token blocks: warp MMAs over swizzled TMA tiles
-    rc = d == 64 ? dispatch_fused<__nv_bfloat16, 64, true>(Hq / Hk, p, st)
-                 : dispatch_fused<__nv_bfloat16, 128, true>(Hq / Hk, p, st);
+  if (dt == BSA_BF16 && b == 64 && bf16_sum)
+    rc = d == 64 ? dispatch_fused<bf, bf, 64, true>(Hq / Hk, p, st)
+                 : dispatch_fused<bf, bf, 128, true>(Hq / Hk, p, st);
+  else if (dt == BSA_BF16 && b == 64)  // 64-token blocks: warp MMAs over swizzled TMA tiles
+    rc = d == 64 ? dispatch_fused<bf, float, 64, true>(Hq / Hk, p, st)
+                 : dispatch_fused<bf, float, 128, true>(Hq / Hk, p, st);
   else if (dt == BSA_BF16)
-    rc = d == 64 ? dispatch_fused<__nv_bfloat16, 64, false>(Hq / Hk, p, st)
-                 : dispatch_fused<__nv_bfloat16, 128, false>(Hq / Hk, p, st);
+    rc = d == 64 ? dispatch_fused<bf, float, 64, false>(Hq / Hk, p, st)
+                 : dispatch_fused<bf, float, 128, false>(Hq / Hk, p, st);
   else
-    rc = d == 64 ? dispatch_fused<float, 64, false>(Hq / Hk, p, st)
-                 : dispatch_fused<float, 128, false>(Hq / Hk, p, st);
+    rc = d == 64 ? dispatch_fused<float, float, 64, false>(Hq / Hk, p, st)
+                 : dispatch_fused<float, float, 128, false>(Hq / Hk, p, st);
   if (rc != BSA_OK) return rc;
   BSA_LAUNCH_CHECK();
   return BSA_OK;
+}
+
+extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtype dt,
+                                      int B, int Hq, int Hk, int n, int d, int b,
+                                      const int* seq_lens, float* mean_k, float* max_norm,
+                                      float* centre, int append, const float* lambda_h,
+                                      const float* sigma_h, int prefix_block, int K, void* o,
+                                      float* lse, int* idx, int* count, int* status,
+                                      void* stream) {
+  return bsa_decode_step_ex(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, mean_k, max_norm, centre,
+                            append, lambda_h, sigma_h, prefix_block, K, o, lse, idx, count,
+                            status, 0, stream);
 }

@@ -163,3 +163,36 @@ extern "C" bsa_status bsa_build_block_summaries(const void* k, bsa_dtype dt, int
   BSA_LAUNCH_CHECK();
   return BSA_OK;
 }
+
+namespace bsa {
+namespace {
+
+// fp32 -> bf16 with round-to-nearest-even, four values per thread
+__global__ void __launch_bounds__(256)
+    round_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, long long count) {
+  const long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (i + 4 <= count) {
+    const float4 v = *reinterpret_cast<const float4*>(x + i);
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    *reinterpret_cast<uint2*>(y + i) =
+        make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+  } else {
+    for (long long j = i; j < count; ++j) y[j] = __float2bfloat16_rn(x[j]);
+  }
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" bsa_status bsa_round_summaries_bf16(const float* mean_k, void* out, long long count,
+                                               void* stream) {
+  using namespace bsa;
+  BSA_REQUIRE(mean_k && out && count >= 0, BSA_ERR_ARG);
+  BSA_REQUIRE(all_aligned16(mean_k, out), BSA_ERR_ARG);
+  if (count == 0) return BSA_OK;
+  const long long threads = (count + 3) / 4;
+  round_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      mean_k, static_cast<__nv_bfloat16*>(out), count);
+  BSA_LAUNCH_CHECK();
+  return BSA_OK;
+}

@@ -62,6 +62,18 @@ typedef enum { BSA_GATE_NONE = 0, BSA_GATE_LOG_SOFTMAX = 1 } bsa_gate_mode;
  * SELECTED = LSE over the selected history blocks, ALL_HISTORY = LSE over every history block. */
 typedef enum { BSA_NORM_SELECTED = 0, BSA_NORM_ALL_HISTORY = 1 } bsa_gate_norm;
 
+/* Variants of bsa_decode_step_ex (bit flags). */
+typedef enum {
+  /* One selection per kv head: the group's score of a block is the mean of its G query heads'
+   * scores (the bsa_score_blocks scores); its Top-K (plus the current block) is attended by every
+   * head of the group.  The pages leave per-head versus shared selection under GQA open; the
+   * per-head rule is the default. */
+  BSA_DECODE_SHARED_SELECTION = 1,
+  /* mean_k is bf16 [B, Hk, C, d] (see bsa_round_summaries_bf16): half the summary bytes; the dot
+   * products still accumulate in fp32.  Needs dt = BSA_BF16 and b = 64. */
+  BSA_DECODE_BF16_SUMMARIES = 2
+} bsa_decode_flags;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* bsa_status_string(bsa_status s);
 
@@ -89,6 +101,14 @@ int bsa_version(void);
 bsa_status bsa_build_block_summaries(const void* k, bsa_dtype dt, int B, int Hk, int n, int d,
                                      int b, const int* seq_lens, int first_block, int num_blocks,
                                      float* mean_k, float* max_norm, float* centre, void* stream);
+
+/*
+ * bsa_round_summaries_bf16 -- mean keys for BSA_DECODE_BF16_SUMMARIES: out[i] = bf16(mean_k[i])
+ * with round-to-nearest-even (NaN stays NaN, infinities stay infinite).
+ *   mean_k    count float32 values (device);  out  count bf16 values (device), 16-byte aligned.
+ */
+bsa_status bsa_round_summaries_bf16(const float* mean_k, void* out, long long count,
+                                    void* stream);
 
 /*
  * bsa_score_blocks -- decode block scores of one query per (batch, query head).
@@ -156,6 +176,20 @@ bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtyp
                            float* mean_k, float* max_norm, float* centre, int append,
                            const float* lambda_h, const float* sigma_h, int prefix_block, int K,
                            void* o, float* lse, int* idx, int* count, int* status, void* stream);
+
+/*
+ * bsa_decode_step_ex -- bsa_decode_step with the variants of bsa_decode_flags: flags = 0 is
+ * bsa_decode_step.  With BSA_DECODE_SHARED_SELECTION every head of a group writes the group's
+ * selection to idx / count; with BSA_DECODE_BF16_SUMMARIES mean_k is bf16 (read, and with
+ * append != 0 the current block's entry rewritten as bf16 of its fp32 mean).  Unknown flag bits
+ * are BSA_ERR_ARG; bf16 summaries with dt != BSA_BF16 or b != 64 are BSA_ERR_UNSUPPORTED.
+ */
+bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                              int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                              void* mean_k, float* max_norm, float* centre, int append,
+                              const float* lambda_h, const float* sigma_h, int prefix_block, int K,
+                              void* o, float* lse, int* idx, int* count, int* status, int flags,
+                              void* stream);
 
 /*
  * bsa_sparse_attn_fwd -- exact causal softmax over the gathered tokens

@@ -41,6 +41,10 @@ Readings where the pages are silent or garbled (each listed with its reason in D
   history block); with per-query-block selection it sums over the unit's queries.
 * R11 a computed selector score is rounded to float32 before top-K, the precision in which the
   CUDA kernels take the same decision; supplied scores are float32 already.
+* R19 GQA-shared selection (a variant; the pages leave per-head versus shared selection open):
+  the group's score of a block is the mean of its query heads' scores, its top-K is attended by
+  every head of the group; bf16 summaries are the float32 mean keys rounded to the nearest
+  bfloat16 (ties to even).
 """
 from __future__ import annotations
 
@@ -192,6 +196,59 @@ def fsl_select(q, i, mean_k, max_norm, centre, lam, sigma, cand, K) -> list[int]
 def round_f32(x):
     """R11: the precision in which a computed score decides the selection."""
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def round_bf16(x):
+    """Nearest bfloat16 of each float32 value, ties to the even significand; NaN stays NaN (R19).
+
+    bfloat16 keeps the sign, the 8 exponent bits and the top 7 fraction bits of a float32.  The
+    16 dropped bits decide: above half of the last kept bit rounds the magnitude up, below half
+    truncates, exactly half rounds to the even kept pattern (a carry may reach the exponent,
+    overflowing to infinity as IEEE rounding does).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    u = x32.view(np.uint32).astype(np.uint64)
+    kept, dropped = u >> 16, u & 0xFFFF
+    up = (dropped > 0x8000) | ((dropped == 0x8000) & ((kept & 1) == 1))
+    out = ((kept + up.astype(np.uint64)) << 16).astype(np.uint32).view(np.float32)
+    return np.where(np.isnan(x32), np.float32(np.nan), out).astype(np.float64)
+
+
+def shared_block_scores(per_head_scores) -> np.ndarray:
+    """Group score of every block for GQA-shared selection (R19): the mean over the group's
+    query heads of their block scores ([G, n_cand] -> [n_cand])."""
+    return np.asarray(per_head_scores, dtype=np.float64).mean(axis=0)
+
+
+def decode_reference_shared(q, k, v, seq_lens, b, K, summaries=None):
+    """Decode step with one selection per (batch, kv head) (R19).
+
+    For every kv group: the query heads' scores q . kbar / sqrt(d) over the history blocks, their
+    mean (shared_block_scores, rounded to float32 as a decision precision, R11), its top-K, and
+    for every head of the group the exact softmax over the selected blocks plus the current one.
+    ``summaries`` maps (bi, kh) to (mean_k, ...) to use instead of the fp64 block means.
+    Returns dict (bi, h) -> {"idx", "scores", "o", "lse"}.
+    """
+    B, Hq, d = q.shape
+    Hk = k.shape[1]
+    G = Hq // Hk
+    out = {}
+    for bi in range(B):
+        L = int(seq_lens[bi])
+        i = L - 1
+        nc = sas_num_candidates(i, b)
+        for kh in range(Hk):
+            kk = k[bi, kh, :L]
+            vv = v[bi, kh, :L]
+            mean_k = (summaries[(bi, kh)] if summaries is not None else block_summaries(kk, b))[0]
+            per_head = [dot_scores(q[bi, kh * G + g], mean_k, nc) for g in range(G)]
+            s = round_f32(shared_block_scores(per_head))
+            sel = topk_blocks(s, nc, K)
+            for g in range(G):
+                h = kh * G + g
+                o, lse = sparse_attention_row(q[bi, h], kk, vv, i, b, sel)
+                out[(bi, h)] = {"idx": sel, "scores": s, "o": o, "lse": lse}
+    return out
 
 
 # ----------------------------------------------------------------------------------------------

@@ -17,7 +17,7 @@ FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails val
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(bsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_hot_path():
@@ -183,3 +183,19 @@ def test_fsl_rejects_bad_arguments(bsa_lib):
     assert g(*bad) == 4
     bad = list(base); bad[4] = 96
     assert g(*bad) == 4
+
+
+def test_decode_step_ex_rejects_bad_arguments(bsa_lib):
+    f = bsa_lib.bsa_decode_step_ex
+    base = [FAKE, FAKE, FAKE, 1, 2, 8, 2, 2048, 128, 64, None, FAKE, None, None, 0, None, None, 0,
+            15, FAKE, None, None, None, None, 0, None]
+    bad = list(base); bad[24] = 4      # unknown flag bit
+    assert f(*bad) == 1
+    bad = list(base); bad[24] = 2; bad[3] = 0    # bf16 summaries need bf16 K/V
+    assert f(*bad) == 4
+    bad = list(base); bad[24] = 2; bad[9] = 32   # ... and 64-token blocks
+    assert f(*bad) == 4
+    bad = list(base); bad[0] = None
+    assert f(*bad) == 1
+    assert bsa_lib.bsa_round_summaries_bf16(None, FAKE, 16, None) == 1
+    assert bsa_lib.bsa_round_summaries_bf16(FAKE, FAKE, -1, None) == 1

@@ -132,3 +132,141 @@ def test_fused_full_size(wl):
         hits += len(sel & set(int(c) for c in blocks))
         tot += len(blocks)
     assert hits / tot > 0.9
+
+
+# ---- variants: GQA-shared selection and bf16 summaries (bsa_decode_step_ex) ------------------
+
+
+def test_round_summaries_bf16_bit_exact():
+    rng = np.random.default_rng(70)
+    x = (rng.standard_normal(100_003) * 10.0 ** rng.integers(-20, 20, 100_003)).astype(np.float32)
+    grid = orc.round_bf16(x[:4000]).astype(np.float32)     # ties: halfway between grid points
+    x[:4000] = grid + np.float32(2.0 ** -8) * np.abs(grid)
+    x[-5:] = [np.inf, -np.inf, np.nan, 0.0, np.finfo(np.float32).max]
+    out = bsa.round_summaries_bf16(torch.from_numpy(x).to(DEV))
+    torch.cuda.synchronize()
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = orc.round_bf16(x)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), np.flatnonzero(~same)[:5]
+
+
+def shared_oracle_check(case, idx, o, lse, summaries=None):
+    ref = orc.decode_reference_shared(case.q, case.k, case.v, case.seq_lens, case.b, case.K,
+                                      summaries=summaries)
+    G = case.Hq // case.Hk
+    for (bi, h), r in ref.items():
+        L = int(case.seq_lens[bi])
+        nc = orc.sas_num_candidates(L - 1, case.b)
+        sets = orc.valid_selections(r["scores"], nc, case.K)
+        gsel = sorted(int(x) for x in idx[bi, h] if x >= 0)
+        assert sets is not None and gsel in sets, (bi, h, gsel)
+        # every head of the group holds the group's selection
+        assert gsel == sorted(int(x) for x in idx[bi, (h // G) * G] if x >= 0)
+        kh = h // G
+        ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, kh, :L], case.v[bi, kh, :L],
+                                          L - 1, case.b, gsel)
+        assert np.max(np.abs(o[bi, h] - ro)) < 2e-2, (bi, h)
+        assert abs(lse[bi, h] - rl) < 2e-2, (bi, h)
+
+
+@pytest.mark.parametrize("G,K,d", [(4, 15, 128), (8, 7, 64)])
+def test_fused_shared_selection_matches_oracle(G, K, d):
+    Hk = 2
+    case = inputs.decode_case(80 + G, B=3, Hq=Hk * G, Hk=Hk, d=d, n=2500, b=64, K=K, needles=5,
+                              seq_lens=[2500, 1111, 300])
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, 64, sl)
+    o, lse, idx, cnt = bsa.decode_step_ex(q, k, v, mean_k, 64, K, bsa.DECODE_SHARED_SELECTION,
+                                          seq_lens=sl, append=False)
+    torch.cuda.synchronize()
+    shared_oracle_check(case, idx.cpu().numpy(), o.float().cpu().numpy(), lse.cpu().numpy())
+    exp_cnt = np.minimum(K, (case.seq_lens - 1) // 64)
+    assert (cnt.cpu().numpy() == exp_cnt[:, None]).all()
+
+
+def oracle_bf16_summaries(case):
+    """fp64 block means rounded to float32, then to bfloat16: the caller's bf16 mean keys."""
+    summ, arr = {}, np.zeros((case.B, case.Hk, -(-case.n // case.b), case.d), np.float32)
+    for bi in range(case.B):
+        L = int(case.seq_lens[bi])
+        for kh in range(case.Hk):
+            m = orc.round_bf16(orc.round_f32(orc.block_summaries(case.k[bi, kh, :L], case.b)[0]))
+            summ[(bi, kh)] = (m,)
+            arr[bi, kh, :m.shape[0]] = m
+    return summ, torch.from_numpy(arr).to(DEV, torch.bfloat16)
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_fused_bf16_summaries_match_oracle(shared):
+    case = inputs.decode_case(85, B=2, Hq=8, Hk=2, d=128, n=3000, b=64, K=9, needles=4,
+                              seq_lens=[3000, 1400])
+    q, k, v, sl = upload(case)
+    summ, mk16 = oracle_bf16_summaries(case)
+    flags = bsa.DECODE_BF16_SUMMARIES | (bsa.DECODE_SHARED_SELECTION if shared else 0)
+    o, lse, idx, _ = bsa.decode_step_ex(q, k, v, mk16, 64, case.K, flags, seq_lens=sl,
+                                        append=False)
+    torch.cuda.synchronize()
+    idx, o, lse = idx.cpu().numpy(), o.float().cpu().numpy(), lse.cpu().numpy()
+    if shared:
+        shared_oracle_check(case, idx, o, lse, summaries=summ)
+        return
+    ref = orc.decode_reference(case.q, case.k, case.v, case.seq_lens, case.b, case.K,
+                               summaries=dict(summ))
+    for (bi, h), r in ref.items():
+        L = int(case.seq_lens[bi])
+        sets = orc.valid_selections(r["scores"], orc.sas_num_candidates(L - 1, 64), case.K)
+        gsel = sorted(int(x) for x in idx[bi, h] if x >= 0)
+        assert sets is not None and gsel in sets, (bi, h, gsel)
+        kh = h // 4
+        ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, kh, :L], case.v[bi, kh, :L],
+                                          L - 1, 64, gsel)
+        assert np.max(np.abs(o[bi, h] - ro)) < 2e-2 and abs(lse[bi, h] - rl) < 2e-2, (bi, h)
+
+
+def test_fused_bf16_summary_append():
+    """The step rewrites the current block's bf16 mean key: bf16 of its float32 mean (within one
+    bf16 step of the oracle's rounding of the exact mean)."""
+    case = inputs.decode_case(86, B=2, Hq=8, Hk=2, d=128, n=2000, b=64, K=6, needles=3,
+                              seq_lens=[2000, 1100])
+    q, k, v, sl = upload(case)
+    summ, mk16 = oracle_bf16_summaries(case)
+    cur = (case.seq_lens - 1) // 64
+    for bi in range(2):
+        mk16[bi, :, int(cur[bi])] = 99.0
+    bsa.decode_step_ex(q, k, v, mk16, 64, 6, bsa.DECODE_BF16_SUMMARIES, seq_lens=sl, append=True)
+    torch.cuda.synchronize()
+    got = mk16.float().cpu().numpy()
+    for bi in range(2):
+        for kh in range(2):
+            ref = summ[(bi, kh)][0][int(cur[bi])]
+            step = np.maximum(np.abs(ref), 1e-30) * 2.0 ** -7
+            assert np.all(np.abs(got[bi, kh, int(cur[bi])] - ref) <= step), (bi, kh)
+
+
+def test_fused_shared_bf16_full_size():
+    """The 32K decode workload with both variants: sampled rows against the oracle."""
+    case = inputs.decode_case(2000, B=8, Hq=32, Hk=8, d=128, n=32768, b=64, K=15, needles=16,
+                              needle_layout="random")
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, 64)
+    mk16 = bsa.round_summaries_bf16(mean_k)
+    o, lse, idx, _ = bsa.decode_step_ex(q, k, v, mk16, 64, 15,
+                                        bsa.DECODE_SHARED_SELECTION | bsa.DECODE_BF16_SUMMARIES,
+                                        append=False)
+    o2, _, idx2, _ = bsa.decode_step_ex(q, k, v, mean_k, 64, 15, bsa.DECODE_SHARED_SELECTION,
+                                        append=False)
+    torch.cuda.synchronize()
+    # within a group every head holds one selection, and bf16 summaries keep almost all of it
+    idx_h = idx.cpu().numpy()
+    assert (idx_h.reshape(8, 8, 4, 15) == idx_h.reshape(8, 8, 4, 15)[:, :, :1]).all()
+    agree = np.mean([len(set(a) & set(b)) / 15.0 for a, b in
+                     zip(idx_h.reshape(-1, 15), idx2.cpu().numpy().reshape(-1, 15))])
+    assert agree > 0.9, agree
+    rows = [(bi, h) for bi in range(0, 8, 3) for h in range(0, 32, 5)]
+    for bi, h in rows:
+        L = int(case.seq_lens[bi])
+        gsel = sorted(int(x) for x in idx_h[bi, h] if x >= 0)
+        ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, h // 4, :L],
+                                          case.v[bi, h // 4, :L], L - 1, 64, gsel)
+        assert np.max(np.abs(o[bi, h].float().cpu().numpy() - ro)) < 2e-2, (bi, h)

@@ -576,3 +576,78 @@ def test_fsl_select_with_every_cell_kept_is_the_full_selection():
     got = orc.fsl_select(rng.standard_normal(d), 1400, mean_k, max_norm, centre, 0.5, 300.0,
                          cand, 4)
     assert set(got) <= set(cand) and len(got) == 4
+
+
+# ------------------------------------------------------------------------------------------
+# bf16 summaries and GQA-shared selection (R19)
+# ------------------------------------------------------------------------------------------
+
+
+def _bf16_by_grid(x: float) -> float:
+    """bfloat16 rounding rebuilt from the number line: the grid spacing at |x| is 2^(e - 7) with
+    e = max(floor(log2 |x|), -126); take the nearer grid neighbour, the even multiple on a tie."""
+    if x == 0.0 or math.isinf(x):
+        return x
+    a = abs(x)
+    e = max(math.floor(math.log2(a)), -126)
+    ulp = 2.0 ** (e - 7)
+    lo = math.floor(a / ulp)
+    r = a / ulp - lo
+    m = lo + 1 if (r > 0.5 or (r == 0.5 and lo % 2 == 1)) else lo
+    return math.copysign(m * ulp, x)
+
+
+def test_round_bf16_matches_grid_construction():
+    rng = np.random.default_rng(90)
+    x = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-30, 30, 20000),
+        rng.standard_normal(2000) * 1e-39,            # float32 subnormals
+    ]).astype(np.float32)
+    got = orc.round_bf16(x)
+    ref = np.array([_bf16_by_grid(float(v)) for v in x])
+    assert np.array_equal(got, ref)
+
+
+def test_round_bf16_ties_and_specials():
+    # ties: exactly half a bf16 step above a grid point round to the even significand
+    assert orc.round_bf16(1.0 + 2.0 ** -8) == 1.0             # 1.0000000|1 -> even 1.0
+    assert orc.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert orc.round_bf16(-(1.0 + 2.0 ** -8)) == -1.0
+    assert orc.round_bf16(1.0 + 2.0 ** -8 + 2.0 ** -20) == 1.0 + 2.0 ** -7  # just above half
+    # representable values are kept; infinities stay; the largest float32 overflows to infinity
+    for v in [0.0, -0.0, 1.5, -3.25, 2.0 ** -133, np.inf, -np.inf]:
+        assert orc.round_bf16(v) == v
+    assert orc.round_bf16(np.finfo(np.float32).max) == np.inf
+    assert np.isnan(orc.round_bf16(np.nan))
+
+
+def test_shared_scores_are_the_mean_query_scores():
+    """Mean over heads of q_g . kbar / sqrt(d) equals the mean query's score (linearity)."""
+    rng = np.random.default_rng(91)
+    G, d, C = 4, 64, 40
+    qs = rng.standard_normal((G, d))
+    mean_k = rng.standard_normal((C, d))
+    per_head = [orc.dot_scores(qs[g], mean_k, C) for g in range(G)]
+    shared = orc.shared_block_scores(per_head)
+    assert np.allclose(shared, orc.dot_scores(qs.mean(axis=0), mean_k, C), rtol=0, atol=1e-12)
+    assert np.allclose(orc.shared_block_scores(per_head[::-1]), shared, rtol=0, atol=1e-14)
+
+
+def test_shared_selection_reduces_to_per_head():
+    """One query head per kv head: the shared decode step is the per-head decode step; identical
+    heads in a group: every head keeps its own selection."""
+    rng = np.random.default_rng(92)
+    B, Hk, n, d, b, K = 2, 2, 700, 32, 32, 4
+    k = rng.standard_normal((B, Hk, n, d))
+    v = rng.standard_normal((B, Hk, n, d))
+    seq = np.array([700, 333])
+    q1 = rng.standard_normal((B, Hk, d))
+    a = orc.decode_reference_shared(q1, k, v, seq, b, K)
+    r = orc.decode_reference(q1, k, v, seq, b, K)
+    for key in r:
+        assert a[key]["idx"] == r[key]["idx"]
+        assert np.allclose(a[key]["o"], r[key]["o"], rtol=0, atol=1e-12)
+    q4 = np.repeat(q1, 4, axis=1)   # four identical heads per group
+    a4 = orc.decode_reference_shared(q4, k, v, seq, b, K)
+    for (bi, h), row in a4.items():
+        assert row["idx"] == r[(bi, h // 4)]["idx"]
