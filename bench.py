@@ -48,8 +48,8 @@ WORKLOADS = {
 MEASURED_TRAFFIC = {
     ("sas_gqa_decode_32k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "b3d41af8ef3e40b3",
-        "bytes": 52_589_312 + 413_184},
+        "device_end": "int pick_cluster(", "sha256_16": "655f3f3d4f809aee",
+        "bytes": 52_592_384 + 344_320},
 }
 
 
