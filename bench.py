@@ -260,6 +260,16 @@ def run_prefill(dev, peaks, reps=5):
     # selected normaliser: ds written over every candidate slot; idx, dg and the selected scores
     # read per slot; count and n_cand per unit
     sgrad_bytes = float(s.numel() * 4 + idx.numel() * 4 * 3 + cnt.numel() * 4 * 2)
+    # the outer-gate variant (gate outside the softmax) on the CUDA-core row kernels
+    o2 = torch.empty_like(q)
+    lse2 = torch.empty_like(lse)
+    dg2 = torch.empty_like(dg)
+    ofwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate="outer",
+                                       norm="selected", scores=s, o=o2, lse=lse2)
+    ograd = lambda: bsa.gate_grad(q, k, v, o2, lse2, do, idx, 64, s, q_block=64, count=cnt,
+                                  norm="selected", dg=dg2, outer=True)
+    t_ofwd = statistics.fmean(time_cuda(ofwd, max(2, reps // 2), stream))
+    t_ograd = statistics.fmean(time_cuda(ograd, max(2, reps // 2), stream))
     peak = peaks["bf16_tflops"]
     out["sas_gated_prefill_16k"] = {
         "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
@@ -276,8 +286,11 @@ def run_prefill(dev, peaks, reps=5):
         "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
                           "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
                           "frac_of_hbm": sgrad_bytes / t_sgrad / 1e6 / peaks["hbm_gbs"]},
+        "outer_gate": {"kernels": "prefill_tc_kernel, gate_grad_tc_kernel (tcgen05)",
+                       "forward_ms": t_ofwd, "forward_tflops": fwd_flops / t_ofwd / 1e9,
+                       "grad_ms": t_ograd, "grad_tflops": grad_flops / t_ograd / 1e9},
     }
-    del q, k, v, do, o, s, idx, cnt, lse, dg
+    del q, k, v, do, o, s, idx, cnt, lse, dg, o2, lse2, dg2
     torch.cuda.empty_cache()
 
     fc = inputs.freesolo_case(4000)

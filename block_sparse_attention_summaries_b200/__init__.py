@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsa.so")
 
 BSA_F32, BSA_BF16 = 0, 1
-GATE_NONE, GATE_LOG_SOFTMAX = 0, 1
+GATE_NONE, GATE_LOG_SOFTMAX, GATE_OUTER = 0, 1, 2
 NORM_SELECTED, NORM_ALL_HISTORY = 0, 1
 STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_ARG", 2: "BSA_ERR_SHAPE", 3: "BSA_ERR_DTYPE",
                 4: "BSA_ERR_UNSUPPORTED", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_TIMEOUT",
@@ -42,6 +42,8 @@ SIGNATURES = [
     ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     ("bsa_sparse_attn_decode_noalloc", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                                             _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("bsa_gate_grad_outer", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P,
+                                 _I, _I, _P, _I, _P, _P]),
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
                            _P, _I, _P, _P]),
     ("bsa_selector_grad", _I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _P, _I, _P]),
@@ -203,6 +205,13 @@ def sparse_attn_workspace_bytes(B, Hq, Hk, nq, n, d, b, K) -> int:
     return int(lib().bsa_sparse_attn_workspace_bytes(B, Hq, Hk, nq, n, d, b, K))
 
 
+def _gate_code(gate):
+    """gate: False / None (no gate), True (inner log-gate) or "outer" (gate outside the softmax)."""
+    if gate == "outer":
+        return GATE_OUTER
+    return GATE_LOG_SOFTMAX if gate else GATE_NONE
+
+
 def sparse_attn_fwd(q, k, v, idx, b, count=None, seq_lens=None, q_block=None, gate=False,
                     norm="selected", scores=None, o=None, lse=None, ws=None):
     """Exact causal softmax over the gathered tokens.
@@ -230,7 +239,7 @@ def sparse_attn_fwd(q, k, v, idx, b, count=None, seq_lens=None, q_block=None, ga
     _check(lib().bsa_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, nq, n,
                                      d, b, _ptr(_i32(seq_lens)), q_block, _ptr(_i32(idx)),
                                      _ptr(_i32(count)), K,
-                                     GATE_LOG_SOFTMAX if gate else GATE_NONE, _norm_code(norm),
+                                     _gate_code(gate), _norm_code(norm),
                                      _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _ptr(ws),
                                      ws.numel(), _stream(q.device)), "bsa_sparse_attn_fwd")
     return o, lse
@@ -253,15 +262,16 @@ def sparse_attn_decode_noalloc(q, k, v, idx, b, count=None, seq_lens=None, gate=
     scores_ld = scores.shape[-1] if scores is not None else 0
     _check(lib().bsa_sparse_attn_decode_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b, _ptr(_i32(seq_lens)),
-        _ptr(_i32(idx)), _ptr(_i32(count)), K, GATE_LOG_SOFTMAX if gate else GATE_NONE,
+        _ptr(_i32(idx)), _ptr(_i32(count)), K, _gate_code(gate),
         _norm_code(norm), _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _stream(q.device)),
         "bsa_sparse_attn_decode_noalloc")
     return o, lse
 
 
 def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, norm="selected",
-              dg=None):
-    """dg [B, Hq, U, K] of the inner log-gates (closed form, Eq. 5 of the SAS review)."""
+              dg=None, outer=False):
+    """dg [B, Hq, U, K] of the inner log-gates (closed form, Eq. 5 of the SAS review), or with
+    outer=True of the gates outside the softmax (bsa_gate_grad_outer)."""
     _cuda(q, k, v, o, lse, dout, idx, scores, count, dg)
     B, Hk, n, d = k.shape
     Hq = q.shape[1]
@@ -271,10 +281,10 @@ def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, n
     U = (n + q_block - 1) // q_block
     if dg is None:
         dg = torch.empty(B, Hq, U, K, device=q.device, dtype=torch.float32)
-    _check(lib().bsa_gate_grad(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
-                               _dtype_code(q), B, Hq, Hk, n, d, b, q_block, _ptr(_i32(idx)),
-                               _ptr(_i32(count)), K, _norm_code(norm), _ptr(scores),
-                               scores.shape[-1], _ptr(dg), _stream(q.device)), "bsa_gate_grad")
+    fn = lib().bsa_gate_grad_outer if outer else lib().bsa_gate_grad
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _dtype_code(q), B, Hq,
+              Hk, n, d, b, q_block, _ptr(_i32(idx)), _ptr(_i32(count)), K, _norm_code(norm),
+              _ptr(scores), scores.shape[-1], _ptr(dg), _stream(q.device)), "bsa_gate_grad")
     return dg
 
 

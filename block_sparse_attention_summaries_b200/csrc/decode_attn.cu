@@ -534,7 +534,9 @@ extern "C" bsa_status bsa_sparse_attn_decode_noalloc(
   BSA_REQUIRE(head_dim_ok(d), BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(B <= 65535 && Hk <= 65535 && b <= 128, BSA_ERR_UNSUPPORTED);
   BSA_REQUIRE(all_aligned16(q, k, v, o), BSA_ERR_ARG);
-  BSA_REQUIRE(gate == BSA_GATE_NONE || gate == BSA_GATE_LOG_SOFTMAX, BSA_ERR_ARG);
+  BSA_REQUIRE(gate == BSA_GATE_NONE || gate == BSA_GATE_LOG_SOFTMAX || gate == BSA_GATE_OUTER,
+              BSA_ERR_ARG);
+  BSA_REQUIRE(gate != BSA_GATE_OUTER, BSA_ERR_UNSUPPORTED);  // a training-mode (prefill) gate
   BSA_REQUIRE(norm == BSA_NORM_SELECTED || norm == BSA_NORM_ALL_HISTORY, BSA_ERR_ARG);
   if (gate == BSA_GATE_LOG_SOFTMAX) {
     BSA_REQUIRE(scores != nullptr, BSA_ERR_ARG);

@@ -11,6 +11,10 @@
 // are in flight per step.  Gate gradient is computed in the stable form
 //     dg_m = sum_i sum_{j in B_m} exp(z_ij - lse_i) (do_i . v_j - do_i . o_i),
 // (ptilde_j / g_m = exp(z_j + log g_m - lse) / g_m = exp(z_j - lse), z without the gate).
+// Outer gate (the gate outside the softmax, the ablation of "Why the four design choices
+// matter"): o_i = sum_j g_m(j) p_j v_j with p the ungated softmax, so the forward scales each
+// block's value contributions by g_m (the normaliser stays ungated) and
+//     dg_m = sum_i sum_{j in B_m} exp(z_ij - lse_i) do_i . v_j.
 #include "bsa_common.cuh"
 
 namespace bsa {
@@ -26,7 +30,7 @@ bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq
 bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, int B, int Hq, int Hk, int n, int d,
                         const int* idx, const int* count, int K, int norm, const float* scores,
-                        int scores_ld, float* dg, int* status, cudaStream_t st);
+                        int scores_ld, float* dg, int* status, int outer, cudaStream_t st);
 bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hk, int n,
                       int d, int b, const int* idx, const int* count, int K, int gate, int norm,
                       const float* scores, int scores_ld, void* o, float* lse, int* status,
@@ -91,7 +95,7 @@ __device__ float load_unit(const RowParams& p, int bi, int h, int u, UnitSel& se
   }
   if (lane == 0) sel.cnt = base;
   __syncwarp();
-  if (p.gate != BSA_GATE_LOG_SOFTMAX) return 0.f;
+  if (p.gate == BSA_GATE_NONE) return 0.f;
   const float* srow = p.scores + row * p.scores_ld;
   float mx = -INFINITY, acc = 0.f;
   if (p.norm == BSA_NORM_ALL_HISTORY) {
@@ -121,7 +125,8 @@ __global__ void __launch_bounds__(kThreads) prefill_rowwise_kernel(const RowPara
   UnitSel& S = sel[warp];
   const float lse_norm = load_unit(p, bi, h, u, S, lane);
   const size_t urow = ((size_t)bi * p.Hq + h) * p.U + u;
-  const float* srow = p.gate == BSA_GATE_LOG_SOFTMAX ? p.scores + urow * p.scores_ld : nullptr;
+  const float* srow = p.gate != BSA_GATE_NONE ? p.scores + urow * p.scores_ld : nullptr;
+  const bool outer = p.gate == BSA_GATE_OUTER;
 
   const T* qp = static_cast<const T*>(p.q) + (((size_t)bi * p.Hq + h) * p.n + i) * D + lane * EPL;
   const T* kb = static_cast<const T*>(p.k) + ((size_t)bi * p.Hk + kh) * p.n * D + lane * EPL;
@@ -136,8 +141,9 @@ __global__ void __launch_bounds__(kThreads) prefill_rowwise_kernel(const RowPara
 #pragma unroll
   for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
 
-  // token stream: selected history blocks (with their gate bias), then the current block
-  auto run = [&](int lo, int hi, float bias) {
+  // token stream: selected history blocks (with their gate: a logit bias inside the softmax, or
+  // a value scale outside it), then the current block
+  auto run = [&](int lo, int hi, float bias, float vscale) {
     for (int j0 = lo; j0 < hi; j0 += 4) {
       float z[4], vv[4][EPL];
 #pragma unroll
@@ -174,18 +180,19 @@ __global__ void __launch_bounds__(kThreads) prefill_rowwise_kernel(const RowPara
       for (int r = 0; r < 4; ++r) {
         const float pw = z[r] == -INFINITY ? 0.f : exp2f(z[r] - mx);
         l_run += pw;
+        const float pv = pw * vscale;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pw, vv[r][e], acc[e]);
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(pv, vv[r][e], acc[e]);
       }
       m_run = mx;
     }
   };
   for (int j = 0; j < S.cnt; ++j) {
     const int m = S.m[j];
-    const float bias = srow ? srow[m] * kLog2e - lse_norm : 0.f;
-    run(m * p.b, min((m + 1) * p.b, p.n), bias);
+    const float lg = srow ? srow[m] * kLog2e - lse_norm : 0.f;  // log2 g_m
+    run(m * p.b, min((m + 1) * p.b, p.n), outer ? 0.f : lg, outer ? exp2f(lg) : 1.f);
   }
-  run(cur * p.b, i + 1, 0.f);
+  run(cur * p.b, i + 1, 0.f, 1.f);
 
   T* op = static_cast<T*>(p.o) + (((size_t)bi * p.Hq + h) * p.n + i) * D + lane * EPL;
   const float inv = 1.f / l_run;
@@ -208,6 +215,7 @@ __global__ void __launch_bounds__(kThreads) gate_grad_rowwise_kernel(const RowPa
   (void)load_unit(p, bi, h, u, S, lane);
   const size_t urow = ((size_t)bi * p.Hq + h) * p.U + u;
   const size_t qrow = ((size_t)bi * p.Hq + h) * p.n + i;
+  const bool outer = p.gate == BSA_GATE_OUTER;
 
   float qv[EPL], dov[EPL], ov[EPL];
   load_vec<T, EPL>(static_cast<const T*>(p.q) + qrow * D + lane * EPL, qv);
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(kThreads) gate_grad_rowwise_kernel(const RowPa
         }
 #pragma unroll
       for (int r = 0; r < 4; ++r)
-        if (t0 + r < hi) tot += exp2f(z[r] - lse2) * (dv[r] - Di);
+        if (t0 + r < hi) tot += exp2f(z[r] - lse2) * (outer ? dv[r] : dv[r] - Di);
     }
     if (lane == 0) atomicAdd(&p.dg[urow * p.K + S.slot[j]], tot);
   }
@@ -318,14 +326,16 @@ extern "C" bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const vo
   if (rc != BSA_OK) return rc;
   BSA_REQUIRE(o, BSA_ERR_ARG);
   BSA_REQUIRE(all_aligned16(o), BSA_ERR_ARG);
-  BSA_REQUIRE(gate == BSA_GATE_NONE || gate == BSA_GATE_LOG_SOFTMAX, BSA_ERR_ARG);
+  BSA_REQUIRE(gate == BSA_GATE_NONE || gate == BSA_GATE_LOG_SOFTMAX || gate == BSA_GATE_OUTER,
+              BSA_ERR_ARG);
   BSA_REQUIRE(norm == BSA_NORM_SELECTED || norm == BSA_NORM_ALL_HISTORY, BSA_ERR_ARG);
-  if (gate == BSA_GATE_LOG_SOFTMAX) {
+  if (gate != BSA_GATE_NONE) {
     BSA_REQUIRE(scores != nullptr, BSA_ERR_ARG);
     BSA_REQUIRE(scores_ld >= ceil_div(n, b), BSA_ERR_SHAPE);
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (nq == 1) {
+    BSA_REQUIRE(gate != BSA_GATE_OUTER, BSA_ERR_UNSUPPORTED);  // a training-mode (prefill) gate
     BSA_REQUIRE(b <= 128, BSA_ERR_UNSUPPORTED);
     return decode_attn(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, idx, count, K, gate, norm,
                        scores, scores_ld, o, lse, workspace, workspace_bytes, st);
@@ -350,13 +360,14 @@ extern "C" bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const vo
   return BSA_OK;
 }
 
-extern "C" bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void* o,
-                                    const float* lse, const void* dout, bsa_dtype dt, int B,
-                                    int Hq, int Hk, int n, int d, int b, int q_block,
-                                    const int* idx, const int* count, int K, bsa_gate_norm norm,
-                                    const float* scores, int scores_ld, float* dg,
-                                    void* stream) {
-  using namespace bsa;
+namespace bsa {
+namespace {
+
+bsa_status gate_grad_impl(const void* q, const void* k, const void* v, const void* o,
+                          const float* lse, const void* dout, bsa_dtype dt, int B, int Hq, int Hk,
+                          int n, int d, int b, int q_block, const int* idx, const int* count,
+                          int K, bsa_gate_norm norm, const float* scores, int scores_ld,
+                          float* dg, bool outer, void* stream) {
   bsa_status rc = check_common(q, k, v, dt, B, Hq, Hk, n, d, b, idx, K);
   if (rc != BSA_OK) return rc;
   BSA_REQUIRE(o && lse && dout && dg && scores, BSA_ERR_ARG);
@@ -368,14 +379,14 @@ extern "C" bsa_status bsa_gate_grad(const void* q, const void* k, const void* v,
   if (prefill_tc_supported(dt, d, b, q_block, K, Hq, Hk)) {
     // the gradient of the gated forward: the gate enters only through lse and o here
     return gate_grad_tc(q, k, v, o, lse, dout, B, Hq, Hk, n, d, idx, count, K, norm, scores,
-                        scores_ld, dg, nullptr, st);
+                        scores_ld, dg, nullptr, outer ? 1 : 0, st);
   }
   RowParams p{};
   p.q = q; p.k = k; p.v = v; p.o_in = o; p.lse_in = lse; p.dout = dout;
   p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.b = b; p.q_block = q_block;
   p.U = ceil_div(n, q_block); p.K = K;
-  p.idx = idx; p.count = count; p.gate = BSA_GATE_LOG_SOFTMAX; p.norm = norm;
-  p.scores = scores; p.scores_ld = scores_ld; p.dg = dg;
+  p.idx = idx; p.count = count; p.gate = outer ? BSA_GATE_OUTER : BSA_GATE_LOG_SOFTMAX;
+  p.norm = norm; p.scores = scores; p.scores_ld = scores_ld; p.dg = dg;
   if (cudaMemsetAsync(dg, 0, (size_t)B * Hq * p.U * K * sizeof(float), st) != cudaSuccess) {
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
@@ -384,6 +395,29 @@ extern "C" bsa_status bsa_gate_grad(const void* q, const void* k, const void* v,
   else launch_rowwise<float>(true, d, p, st);
   BSA_LAUNCH_CHECK();
   return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void* o,
+                                    const float* lse, const void* dout, bsa_dtype dt, int B,
+                                    int Hq, int Hk, int n, int d, int b, int q_block,
+                                    const int* idx, const int* count, int K, bsa_gate_norm norm,
+                                    const float* scores, int scores_ld, float* dg,
+                                    void* stream) {
+  return bsa::gate_grad_impl(q, k, v, o, lse, dout, dt, B, Hq, Hk, n, d, b, q_block, idx, count,
+                             K, norm, scores, scores_ld, dg, false, stream);
+}
+
+extern "C" bsa_status bsa_gate_grad_outer(const void* q, const void* k, const void* v,
+                                          const void* o, const float* lse, const void* dout,
+                                          bsa_dtype dt, int B, int Hq, int Hk, int n, int d,
+                                          int b, int q_block, const int* idx, const int* count,
+                                          int K, bsa_gate_norm norm, const float* scores,
+                                          int scores_ld, float* dg, void* stream) {
+  return bsa::gate_grad_impl(q, k, v, o, lse, dout, dt, B, Hq, Hk, n, d, b, q_block, idx, count,
+                             K, norm, scores, scores_ld, dg, true, stream);
 }
 
 extern "C" bsa_status bsa_workspace_status(void* workspace, void* stream) {

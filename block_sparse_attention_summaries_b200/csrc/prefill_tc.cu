@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     }
     base = min(base, kMaxKtc);
     float lnorm = 0.f;
-    if (p.gate == BSA_GATE_LOG_SOFTMAX) {
+    if (p.gate != BSA_GATE_NONE) {  // log2 g_m of the softmax gate, inside or outside the softmax
       const float* srow = p.scores + row * p.scores_ld;
       __syncwarp();
       float mx = -INFINITY, acc = 0.f;
@@ -382,7 +382,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       // bias or mask of this step's block for my unit
       const bool is_cur = !fsl && (j == steps - 1);
       const bool filler = !is_cur && j >= s_cnt[it];
-      const float bias = (!is_cur && !filler && !fsl) ? s_bias[it][j] : 0.f;
+      const float lg = (!is_cur && !filler && !fsl) ? s_bias[it][j] : 0.f;  // log2 g_m
+      // inner gate: a logit bias; outer gate: P scaled by g_m for P V (the row sum stays ungated)
+      const bool outer = p.gate == BSA_GATE_OUTER;
+      const float bias = outer ? 0.f : lg;
+      const float vs = outer ? tc::ex2_approx(lg) : 1.f;
       const int kpos0 = blk * kTiles;  // position of this block's first key
       // keys of this block the row may see: all of a history block; none of a filler; c <= r on
       // the diagonal; c >= wlo - kpos0 inside a sliding window; the keys of the row's own cells
@@ -459,13 +463,13 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
-      if (warp_live) {
+      if (warp_live) {  // outer gate: P V takes g_m p (vs = g_m), the row sum p; inner: vs = 1
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float p0 = tc::ex2_approx(x[c] - m_use);
           const float p1 = tc::ex2_approx(x[c + 1] - m_use);
           sum4[(c >> 1) & 3] += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0 * vs, p1 * vs);
           pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
         }
       } else {
@@ -604,6 +608,7 @@ struct GgParams {
   const void* dout;
   float* dg;
   int* status;
+  int outer;  // outer gate: dg_m = sum p do . v_j (no do . o term)
 };
 
 template <int D>
@@ -761,7 +766,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (live) {
         const __nv_bfloat16* orow = static_cast<const __nv_bfloat16*>(p.o) + qrow * D;
         const __nv_bfloat16* drow = static_cast<const __nv_bfloat16*>(p.dout) + qrow * D;
-        for (int c = 0; c < D; c += 8) {
+        for (int c = 0; !p.outer && c < D; c += 8) {
           float a[8], bb[8];
           load_vec<__nv_bfloat16, 8>(orow + c, a);
           load_vec<__nv_bfloat16, 8>(drow + c, bb);
@@ -963,8 +968,9 @@ bsa_status launch_gg(const void* q, const void* k, const void* v, const void* do
 bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, int B, int Hq, int Hk, int n, int d,
                         const int* idx, const int* count, int K, int norm, const float* scores,
-                        int scores_ld, float* dg, int* status, cudaStream_t st) {
+                        int scores_ld, float* dg, int* status, int outer, cudaStream_t st) {
   GgParams p{};
+  p.outer = outer;
   p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = K;
   p.idx = idx; p.count = count; p.norm = norm; p.scores = scores; p.scores_ld = scores_ld;
   p.o = o; p.lse = lse; p.dout = dout; p.dg = dg; p.status = status;

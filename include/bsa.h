@@ -56,7 +56,10 @@ typedef enum {
 typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
 
 /* Training-mode gate of [SAS] "The new approach", Eq. 9. */
-typedef enum { BSA_GATE_NONE = 0, BSA_GATE_LOG_SOFTMAX = 1 } bsa_gate_mode;
+/* BSA_GATE_OUTER is the outer-gate variant ([SAS] "Why the four design choices matter", the gate
+ * placed outside the softmax): o_i = sum_j g_m(j) p_j v_j with p the ungated softmax and g the
+ * same softmax gate; prefill (training) form only. */
+typedef enum { BSA_GATE_NONE = 0, BSA_GATE_LOG_SOFTMAX = 1, BSA_GATE_OUTER = 2 } bsa_gate_mode;
 
 /* Set the softmax gate normalises over ([SAS] "Why the four design choices matter"):
  * SELECTED = LSE over the selected history blocks, ALL_HISTORY = LSE over every history block. */
@@ -210,6 +213,9 @@ bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v, bsa_d
  *   count     optional per-row/per-unit int32 count of valid idx entries; NULL = up to first -1.
  *   gate      BSA_GATE_LOG_SOFTMAX adds log g_m = s_m - LSE(normaliser set) to the logits of
  *             selected history block m; the current block gets 0 ([SAS] Eq. 4).
+ *             BSA_GATE_OUTER (prefill only; decode returns BSA_ERR_UNSUPPORTED) multiplies the
+ *             value contributions of block m by g_m outside the softmax; lse is then the
+ *             log-sum-exp of the ungated logits.
  *   o         [B, Hq, nq, d] out (dtype dt);  lse  optional [B, Hq, nq] float32 out.
  *   workspace device scratch of bsa_sparse_attn_workspace_bytes() bytes, zero-filled before its
  *             first use; each successful call leaves it reusable.  Calls sharing one workspace
@@ -233,6 +239,18 @@ size_t bsa_sparse_attn_workspace_bytes(int B, int Hq, int Hk, int nq, int n, int
  * bsa_sparse_attn_fwd; o and lse are that call's gated outputs, dout the upstream gradient.
  *   dg        [B, Hq, U, K] float32 out (0 in padded slots).
  */
+/*
+ * bsa_gate_grad_outer -- the gradient for the outer gate (BSA_GATE_OUTER forward):
+ *     dg_m = sum_{queries i of the unit} sum_{j in B_m} p_ij do_i^T v_j,
+ * p the ungated softmax of query i over its token set (lse as written by the outer-gate
+ * forward).  Arguments as bsa_gate_grad (o is not read but must be given).
+ */
+bsa_status bsa_gate_grad_outer(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, bsa_dtype dt, int B, int Hq,
+                               int Hk, int n, int d, int b, int q_block, const int* idx,
+                               const int* count, int K, bsa_gate_norm norm, const float* scores,
+                               int scores_ld, float* dg, void* stream);
+
 bsa_status bsa_gate_grad(const void* q, const void* k, const void* v, const void* o,
                          const float* lse, const void* dout, bsa_dtype dt, int B, int Hq, int Hk,
                          int n, int d, int b, int q_block, const int* idx, const int* count,

@@ -41,6 +41,9 @@ Readings where the pages are silent or garbled (each listed with its reason in D
   history block); with per-query-block selection it sums over the unit's queries.
 * R11 a computed selector score is rounded to float32 before top-K, the precision in which the
   CUDA kernels take the same decision; supplied scores are float32 already.
+* R20 outer gate (f1 variant): the gate multiplies the value contributions of its block outside
+  the softmax, o = sum_j g_m(j) p_j v_j with p the ungated softmax; the current block has gate 1;
+  g = softmax of the scores over the normaliser set, as for the inner gate.
 * R19 GQA-shared selection (a variant; the pages leave per-head versus shared selection open):
   the group's score of a block is the mean of its query heads' scores, its top-K is attended by
   every head of the group; bf16 summaries are the float32 mean keys rounded to the nearest
@@ -351,6 +354,38 @@ def sparse_attention_row(q, k, v, i, b, selected, gate=None, keep_current=True):
     return o, lse
 
 
+def outer_gated_row(q, k, v, i, b, selected, g):
+    """Outer-gate forward of one query ([SAS] "Why the four design choices matter", the gate
+    placed outside the softmax, R20): p = softmax of the ungated logits over the token set,
+    o = sum_j g_m(j) p_j v_j with g_m the gate of history block m (a dict m -> g_m) and 1 for the
+    current block; lse is the log-sum-exp of the ungated logits.
+    """
+    n = k.shape[0]
+    toks, owner = token_set(i, b, selected, n)
+    _, lse, p = attend(q, k, v, toks, np.zeros(len(toks)))
+    w = np.array([p[t] * (g[int(m)] if m >= 0 else 1.0) for t, m in enumerate(owner)])
+    o = w @ np.asarray(v[toks], dtype=np.float64)
+    return o, lse
+
+
+def gate_grad_rows_outer(qs, k, v, positions, b, selected, douts):
+    """dg_m of the outer gate, summed over the given queries (R20):
+        dg_m = sum_{i} sum_{j in B_m} p_ij do_i^T v_j,
+    p the ungated softmax of query i over its token set (the gate multiplies the values only, so
+    the derivative of o_i with respect to g_m is sum_{j in B_m} p_ij v_j).  Returns dict m -> dg_m.
+    """
+    n = k.shape[0]
+    dg = {int(m): 0.0 for m in selected}
+    for q, i, do in zip(qs, positions, douts):
+        toks, owner = token_set(int(i), b, selected, n)
+        _, _, p = attend(q, k, v, toks, np.zeros(len(toks)))
+        do = np.asarray(do, dtype=np.float64)
+        for t, m in enumerate(owner):
+            if m >= 0:
+                dg[int(m)] += p[t] * float(np.dot(do, np.asarray(v[toks[t]], dtype=np.float64)))
+    return dg
+
+
 def masked_attention_row(q, k, v, i, b, selected, gate=None, keep_current=True):
     """The same quantity written as dense attention over all n keys with a -inf mask.
 
@@ -517,6 +552,31 @@ def prefill_unit_reference(q, k, v, scores, b, q_block, K, bi, h, u, gate_norm=N
     if dout is not None and gate is not None:
         dg = gate_grad_rows(q[bi, h, lo:hi], kk, vv, range(lo, hi), b, sel, gate,
                             dout[bi, h, lo:hi])
+        res["dg"] = np.array([dg[m] for m in sel])
+    return res
+
+
+def prefill_unit_reference_outer(q, k, v, scores, b, q_block, K, bi, h, u, gate_norm, dout=None):
+    """prefill_unit_reference with the outer gate (R20): the same selection and softmax gate
+    g_m = exp(log g_m), placed outside the softmax; dg of the outer gate with ``dout``."""
+    Hk = k.shape[1]
+    G = q.shape[1] // Hk
+    kk, vv = k[bi, h // G], v[bi, h // G]
+    n = k.shape[2]
+    lo = u * q_block
+    hi = min(n, lo + q_block)
+    nc = sas_num_candidates(lo, b)
+    s = np.asarray(scores[bi, h, u, :nc], dtype=np.float64)
+    sel = topk_blocks(s, nc, K)
+    g = {m: math.exp(lg) for m, lg in log_gates(s, nc, sel, gate_norm).items()}
+    o = np.zeros((hi - lo, q.shape[3]))
+    lse = np.zeros(hi - lo)
+    for t, i in enumerate(range(lo, hi)):
+        o[t], lse[t] = outer_gated_row(q[bi, h, i], kk, vv, i, b, sel, g)
+    res = {"idx": sel, "o": o, "lse": lse}
+    if dout is not None:
+        dg = gate_grad_rows_outer(q[bi, h, lo:hi], kk, vv, range(lo, hi), b, sel,
+                                  dout[bi, h, lo:hi])
         res["dg"] = np.array([dg[m] for m in sel])
     return res
 

@@ -199,3 +199,17 @@ def test_decode_step_ex_rejects_bad_arguments(bsa_lib):
     assert f(*bad) == 1
     assert bsa_lib.bsa_round_summaries_bf16(None, FAKE, 16, None) == 1
     assert bsa_lib.bsa_round_summaries_bf16(FAKE, FAKE, -1, None) == 1
+
+
+def test_outer_gate_arguments(bsa_lib):
+    f = bsa_lib.bsa_sparse_attn_fwd
+    base = [FAKE, FAKE, FAKE, 1, 2, 8, 2, 1, 1024, 128, 64, None, 64, FAKE, None, 4, 2, 0, FAKE,
+            16, FAKE, None, FAKE, 1 << 20, None]
+    assert f(*base) == 4                    # decode form: the outer gate is a prefill gate
+    bad = list(base); bad[18] = None        # a gate needs scores
+    assert f(*bad) == 1
+    bad = list(base); bad[16] = 3           # unknown gate mode
+    assert f(*bad) == 1
+    g = bsa_lib.bsa_gate_grad_outer
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 8, 2, 1024, 128, 64, 64, FAKE, None, 4, 0,
+             None, 16, FAKE, None) == 1     # scores missing

@@ -469,3 +469,72 @@ def test_prefill_gated_full_size_sampled():
         if len(r["idx"]):
             err = np.max(np.abs(dg[bi, h, u, :len(r["idx"])] - r["dg"]))
             assert err <= 1e-2 * np.max(np.abs(r["dg"])), (bi, h, u, err)
+
+
+# -------------------------------------------------------------------------------------------
+# outer gate (the gate outside the softmax): forward and gradient, fp32 on the row kernels and
+# bf16 units on the tensor cores
+# -------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("norm", ["selected", "all"])
+def test_prefill_outer_gate_fp32_per_query(norm):
+    case = inputs.tiny_decode_case(1000)
+    B, H, d, n, b, K = 1, 2, 64, 1024, 64, 4
+    q = inputs.draw_normal(1000, "q_prefill", (B, H, n, d), False)
+    s = inputs.draw_normal(1000, "s_prefill", (B, H, n, n // b), False)
+    do = inputs.draw_normal(1000, "do_prefill", (B, H, n, d), False)
+    k, v = case.k, case.v
+    s_gpu = up(s, False)
+    qg, kg, vg = up(q, False), up(k, False), up(v, False)
+    idx, cnt = bsa.topk_blocks(s_gpu, K, units=n, q_block=1, b=b)
+    o, lse = bsa.sparse_attn_fwd(qg, kg, vg, idx, b, count=cnt, q_block=1, gate="outer",
+                                 norm=norm, scores=s_gpu)
+    dg = bsa.gate_grad(qg, kg, vg, o, lse, up(do, False), idx, b, s_gpu, q_block=1, count=cnt,
+                       norm=norm, outer=True).cpu().numpy()
+    o, lse = o.cpu().numpy(), lse.cpu().numpy()
+    rng = np.random.default_rng(4)
+    rows = sorted(set([0, 63, 64, 65, 255, 1023]) | set(rng.integers(0, n, 30).tolist()))
+    for h in range(H):
+        for i in rows:
+            r = orc.prefill_unit_reference_outer(q, k, v, s, b, 1, K, 0, h, i, norm, do)
+            assert np.max(np.abs(o[0, h, i] - r["o"][0])) < 1e-4, (h, i)
+            assert abs(lse[0, h, i] - r["lse"][0]) < 1e-4, (h, i)
+            if len(r["idx"]):
+                err = np.max(np.abs(dg[0, h, i, :len(r["idx"])] - r["dg"]))
+                assert err <= 1e-4 * max(1e-3, np.max(np.abs(r["dg"]))), (h, i, err)
+
+
+def test_prefill_outer_gate_bf16_units():
+    """bf16 units of 64 queries on the tensor-core forward and gradient: forward and dg against
+    the oracle on sampled units."""
+    B, Hq, Hk, n, d, b, K = 1, 4, 2, 1024 + 37, 128, 64, 6
+    case = inputs.prefill_case(17, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, q_block=64)
+    s_gpu = up(case.scores, False)
+    q, k, v = up(case.q, True), up(case.k, True), up(case.v, True)
+    idx, cnt = bsa.topk_blocks(s_gpu, K, units=case.U, q_block=64, b=b)
+    o, lse = bsa.sparse_attn_fwd(q, k, v, idx, b, count=cnt, q_block=64, gate="outer",
+                                 norm="all", scores=s_gpu)
+    dg = bsa.gate_grad(q, k, v, o, lse, up(case.dout, True), idx, b, s_gpu, q_block=64,
+                       count=cnt, norm="all", outer=True).cpu().numpy()
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    for h in range(Hq):
+        for u in [0, 1, 5, 9, 16]:
+            r = orc.prefill_unit_reference_outer(case.q, case.k, case.v, case.scores, b, 64, K, 0,
+                                                 h, u, "all", case.dout)
+            lo = u * 64
+            assert np.max(np.abs(o[0, h, lo:lo + len(r["o"])] - r["o"])) < 2e-2, (h, u)
+            assert np.max(np.abs(lse[0, h, lo:lo + len(r["o"])] - r["lse"])) < 2e-2, (h, u)
+            if len(r["idx"]):
+                err = np.max(np.abs(dg[0, h, u, :len(r["idx"])] - r["dg"]))
+                assert err <= 1e-2 * np.max(np.abs(r["dg"])), (h, u, err)
+
+
+def test_outer_gate_decode_unsupported():
+    case = inputs.tiny_decode_case(1000)
+    q = up(case.q, False)
+    idx = torch.zeros(q.shape[0], q.shape[1], 2, dtype=torch.int32, device=DEV)
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.sparse_attn_fwd(q, up(case.k, False), up(case.v, False), idx, 64, gate="outer",
+                            scores=torch.zeros(q.shape[0], q.shape[1], 64, device=DEV))
+    assert e.value.code == 4

@@ -651,3 +651,52 @@ def test_shared_selection_reduces_to_per_head():
     a4 = orc.decode_reference_shared(q4, k, v, seq, b, K)
     for (bi, h), row in a4.items():
         assert row["idx"] == r[(bi, h // 4)]["idx"]
+
+
+# ------------------------------------------------------------------------------------------
+# Outer gate (R20)
+# ------------------------------------------------------------------------------------------
+
+
+def _outer_loss(qs, k, v, positions, b, selected, g, douts):
+    return sum(float(np.dot(np.asarray(do), orc.outer_gated_row(q, k, v, int(i), b, selected,
+                                                                   g)[0]))
+               for q, i, do in zip(qs, positions, douts))
+
+
+def test_outer_gate_unit_gates_give_plain_attention():
+    rng = np.random.default_rng(95)
+    n, d, b = 300, 16, 32
+    q, k, v = rng.standard_normal(d), rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    sel = [1, 4, 6]
+    o, lse = orc.outer_gated_row(q, k, v, 250, b, sel, {m: 1.0 for m in sel})
+    ro, rl = orc.sparse_attention_row(q, k, v, 250, b, sel)
+    assert np.allclose(o, ro, rtol=0, atol=1e-13) and abs(lse - rl) < 1e-13
+    # scaling one block's gate by c adds (c - 1) times that block's weighted values, lse unchanged
+    o2, lse2 = orc.outer_gated_row(q, k, v, 250, b, sel, {1: 1.0, 4: 3.0, 6: 1.0})
+    assert abs(lse2 - rl) < 1e-13
+    toks, owner = orc.token_set(250, b, sel, n)
+    _, _, p = orc.attend(q, k, v, toks, np.zeros(len(toks)))
+    part = sum(p[t] * v[toks[t]] for t, m in enumerate(owner) if m == 4)
+    assert np.allclose(o2 - ro, 2.0 * part, rtol=0, atol=1e-12)
+
+
+def test_outer_gate_gradient_matches_finite_differences():
+    """The loss is linear in each outer gate, so a central difference recovers dg_m exactly
+    (up to rounding); a planted sign error or a dropped block fails."""
+    rng = np.random.default_rng(96)
+    n, d, b = 256, 16, 32
+    k, v = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    positions = [192, 200, 223]
+    qs = rng.standard_normal((3, d))
+    douts = rng.standard_normal((3, d))
+    sel = [0, 2, 5]
+    g = {0: 0.2, 2: 0.5, 5: 0.3}
+    dg = orc.gate_grad_rows_outer(qs, k, v, positions, b, sel, douts)
+    for m in sel:
+        h = 1e-3
+        up = dict(g); up[m] += h
+        dn = dict(g); dn[m] -= h
+        fd = (_outer_loss(qs, k, v, positions, b, sel, up, douts)
+              - _outer_loss(qs, k, v, positions, b, sel, dn, douts)) / (2 * h)
+        assert abs(fd - dg[m]) < 1e-9 * max(1.0, abs(fd)), (m, fd, dg[m])
