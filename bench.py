@@ -69,6 +69,24 @@ def measured_traffic(workload: str, kernel: str):
         return None
     return rec["bytes"]
 
+def job_timing(total_ms: float, e2e_ms: float, world: int, device) -> tuple[float, float]:
+    """The job's device times: the maximum over ranks (one all-reduce, taken by every rank in the
+    same order; a single rank returns its own)."""
+    if world <= 1:
+        return total_ms, e2e_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms, e2e_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t[0]), float(t[1])
+
+
+def job_throughput(tokens_per_rank_step: int, world: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank decodes its own batch (weak scaling), so the tokens of all
+    ranks count over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -635,15 +653,10 @@ def run_gpu(args):
     clocks = sampler.summary()
     st_word = int(status.max().item())
 
-    mx_total = total_ms
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mx_total, e2e_total = float(t[0]), float(t[1])
+    mx_total, e2e_total = job_timing(total_ms, e2e_total, world, dev)
     ms_per_step = mx_total / args.steps
-    tokens = B * world * args.steps
-    value = tokens / (mx_total / 1e3)
-    e2e_value = tokens / (e2e_total / 1e3)
+    value = job_throughput(B, world, args.steps, mx_total)
+    e2e_value = job_throughput(B, world, args.steps, e2e_total)
 
     peaks = load_peaks()
     avg_ms = total_ms / args.steps  # one fused kernel per step
