@@ -629,11 +629,14 @@ def run_gpu(args):
                           "union_blocks": v_union, "needle_recall": v_hits / max(1, tot),
                           "index_agreement_vs_per_head_fp32": agree}
 
-    # end to end through the public API: pinned host q in, the bsa_decode_step call (binding ->
-    # C-ABI, no graph), o out, every step
+    # end to end through the public API: pinned host q in, the decode step (a prepared binding
+    # call, bsa.DecodeStep -> bsa_decode_step_ex, no graph), o out, every step
     q_host = [torch.from_numpy(np.ascontiguousarray(L["q"].float().cpu().numpy()))
               .to(torch.bfloat16).pin_memory() for L in layers]
     o_host = torch.empty(B, Hq, d, dtype=torch.bfloat16).pin_memory()
+    plans = [bsa.DecodeStep(L["q"], L["k"], L["v"], L["mean_k"], b, K, append=True,
+                            max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
+                            idx=L["idx"], count=L["count"], status=status) for L in layers]
     e2e_ms = []
     with torch.cuda.stream(stream):
         for i in range(args.warmup + args.steps):
@@ -642,7 +645,7 @@ def run_gpu(args):
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             L["q"].copy_(q_host[i % R], non_blocking=True)
-            fused(L)
+            plans[i % R](stream)
             o_host.copy_(L["o"], non_blocking=True)
             e1.record(stream)
             if i >= args.warmup:
@@ -688,8 +691,9 @@ def run_gpu(args):
         "needle_recall": hits / max(1, tot), "status_word": st_word,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * Hq * d * 2,
                 "d2h_bytes_per_step": B * Hq * d * 2,
-                "what": "per step: pinned-host q -> device, bsa_decode_step through the binding "
-                        "and the C ABI (no graph), o -> pinned host; CUDA events on the stream"},
+                "what": "per step: pinned-host q -> device, the decode step through a prepared "
+                        "binding call (bsa.DecodeStep) and the C ABI (bsa_decode_step_ex, no "
+                        "graph), o -> pinned host; CUDA events on the stream"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],

@@ -443,6 +443,49 @@ def decode_step_ex(q, k, v, mean_k, b, K, flags, seq_lens=None, append=True, max
     return o, lse, idx, count
 
 
+class DecodeStep:
+    """A prepared bsa_decode_step_ex call for fixed buffers (a serving loop's decode step).
+
+    The argument list (pointers, sizes, flags) is marshalled once here; each call passes it and
+    the stream to the C ABI, so a step costs the host one foreign call instead of re-checking and
+    re-wrapping every tensor.  The tensors given (and the outputs allocated here) are kept alive
+    by this object and must keep their storage: write new queries into ``q`` in place.
+    ``outputs`` is (o, lse, idx, count).
+    """
+
+    def __init__(self, q, k, v, mean_k, b, K, flags=0, seq_lens=None, append=True,
+                 max_norm=None, centre=None, lambda_h=None, sigma_h=None, prefix_block=0,
+                 o=None, lse=None, idx=None, count=None, status=None):
+        _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count)
+        B, Hk, n, d = k.shape
+        Hq = q.shape[1]
+        if o is None:
+            o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+        if lse is None:
+            lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+        if idx is None:
+            idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+        if count is None:
+            count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+        sl = _i32(seq_lens)
+        self._keep = (q, k, v, mean_k, sl, max_norm, centre, lambda_h, sigma_h, status)
+        self.outputs = (o, lse, idx, count)
+        self._fn = lib().bsa_decode_step_ex
+        self._args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b, _ptr(sl),
+                      _ptr(mean_k), _ptr(max_norm), _ptr(centre), 1 if append else 0,
+                      _ptr(lambda_h), _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse),
+                      _ptr(idx), _ptr(count), _ptr(status), int(flags))
+        self._device = q.device
+
+    def __call__(self, stream=None):
+        """Run the step on ``stream`` (a torch.cuda.Stream; default: the current stream)."""
+        st = stream if stream is not None else torch.cuda.current_stream(self._device)
+        code = self._fn(*self._args, ctypes.c_void_p(st.cuda_stream))
+        if code != 0:
+            raise BsaError(code, "bsa_decode_step_ex")
+        return self.outputs
+
+
 def round_summaries_bf16(mean_k, out=None):
     """bf16 copy of float32 mean keys (round to nearest even), for DECODE_BF16_SUMMARIES."""
     _cuda(mean_k, out)

@@ -270,3 +270,22 @@ def test_fused_shared_bf16_full_size():
         ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, h // 4, :L],
                                           case.v[bi, h // 4, :L], L - 1, 64, gsel)
         assert np.max(np.abs(o[bi, h].float().cpu().numpy() - ro)) < 2e-2, (bi, h)
+
+
+def test_prepared_decode_step_matches_the_binding_call():
+    """bsa.DecodeStep (arguments marshalled once) runs the same step as decode_step_fused."""
+    case = inputs.decode_case(87, B=2, Hq=8, Hk=2, d=128, n=2000, b=64, K=6, needles=3,
+                              seq_lens=[2000, 1100])
+    q, k, v, sl = upload(case)
+    mk1, mx1, ce1 = bsa.build_block_summaries(k, 64, sl)
+    mk2, mx2, ce2 = mk1.clone(), mx1.clone(), ce1.clone()
+    o1, lse1, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mk1, 64, 6, seq_lens=sl, append=True,
+                                                 max_norm=mx1, centre=ce1)
+    plan = bsa.DecodeStep(q, k, v, mk2, 64, 6, seq_lens=sl, append=True, max_norm=mx2,
+                          centre=ce2)
+    o2, lse2, idx2, cnt2 = plan()
+    o3, _, _, _ = plan(torch.cuda.current_stream())  # a second call reuses the same buffers
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2) and torch.equal(cnt1, cnt2)
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2) and o3 is o2
+    assert torch.equal(mk1, mk2) and torch.equal(mx1, mx2) and torch.equal(ce1, ce2)
