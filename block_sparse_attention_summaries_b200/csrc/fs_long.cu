@@ -467,72 +467,69 @@ __global__ void __launch_bounds__(LongSmem<D, CELL>::kThreads, LongSmem<D, CELL>
 }
 
 // ---- 5. merge a query's partials and mix into the short-branch output -----------------------
-// Sixteen lanes per query (two queries per warp, d / 16 elements per lane); every load of the
-// query (its slots' positions and (max, sum), all K partial rows, the short-branch row) is issued
-// up front, so each warp waits for memory once.  Slots that were not attended have no record:
-// their loads are in bounds but unused (selected away, never multiplied, so whatever the buffer
-// holds cannot leak into the result).
+// A thread per (query, 8 output elements): it loads the query's slot positions and (max, sum)
+// itself (the 16 / 8 threads of a query read the same words, served once per warp), all K partial
+// chunks and the short-branch chunk up front, and merges without any exchange between threads.
+// Slots that were not attended have no record: their loads are in bounds but unused (selected
+// away, never multiplied, so whatever the buffer holds cannot leak into the result).
 template <int D>
 __global__ void __launch_bounds__(256)
     fs_long_combine_kernel(const int* __restrict__ slotpos, const float2* __restrict__ part_ml,
                            const __nv_bfloat16* __restrict__ part_o,
                            const float* __restrict__ alpha, int H, int n, int K, long long rows,
                            __nv_bfloat16* __restrict__ o) {
-  constexpr int E = D / 16;  // elements per lane: 4 (8-byte loads) or 8 (16-byte loads)
-  using V = typename std::conditional<E == 4, uint2, uint4>::type;
-  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
-  const int lane = threadIdx.x & 31, sub = lane & 15, seg = lane & 16;
-  const bool live = row < rows;
-  const long long r0 = (live ? row : 0) * K;
-  const int sp = live && sub < K ? slotpos[r0 + sub] : -1;
-  const float2 ml = live && sub < K ? part_ml[r0 + sub] : make_float2(-INFINITY, 0.f);
-  V part[kMaxKL];
-#pragma unroll
-  for (int k = 0; k < kMaxKL; ++k)
-    if (live && k < K)
-      part[k] = *reinterpret_cast<const V*>(part_o + (size_t)(r0 + k) * D + sub * E);
-  __nv_bfloat16* dst = o + (size_t)(live ? row : 0) * D + sub * E;
-  V sh{};
-  if (live) sh = *reinterpret_cast<const V*>(dst);
-  const bool valid = sp >= 0;
-  float M = valid ? ml.x : -INFINITY;
-#pragma unroll
-  for (int off = 4; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  M = __shfl_sync(0xffffffffu, M, seg);  // sub-lanes 0 .. 7 hold the slots
-  const float w = valid ? ml.y * exp2f(ml.x - M) : 0.f;  // the slot's share of the softmax mass
-  float Lsum = w;
-#pragma unroll
-  for (int off = 4; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
-  Lsum = __shfl_sync(0xffffffffu, Lsum, seg);
-  float acc[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  constexpr int TPR = D / 8;  // threads per query
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gid / TPR;
+  const int c8 = (int)(gid % TPR) * 8;
+  if (row >= rows) return;
+  const long long r0 = row * K;
+  int sp[kMaxKL];
+  float2 ml[kMaxKL];
+  uint4 part[kMaxKL];
 #pragma unroll
   for (int k = 0; k < kMaxKL; ++k) {
-    if (k >= K) break;
-    const float wk = __shfl_sync(0xffffffffu, w, seg + k);
-    const bool vk = __shfl_sync(0xffffffffu, valid ? 1 : 0, seg + k) != 0;
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&part[k]);
-#pragma unroll
-    for (int e = 0; e < E / 2; ++e) {
-      const float2 f = __bfloat1622float2(h[e]);
-      acc[2 * e] += vk ? wk * f.x : 0.f;
-      acc[2 * e + 1] += vk ? wk * f.y : 0.f;
+    if (k < K) {
+      sp[k] = slotpos[r0 + k];
+      ml[k] = part_ml[r0 + k];
+      part[k] = *reinterpret_cast<const uint4*>(part_o + (size_t)(r0 + k) * D + c8);
     }
   }
-  if (!live || M == -INFINITY) return;  // no cell attended: o keeps the short branch
+  __nv_bfloat16* dst = o + (size_t)row * D + c8;
+  const uint4 sh = *reinterpret_cast<const uint4*>(dst);
+  float M = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kMaxKL; ++k)
+    if (k < K && sp[k] >= 0) M = fmaxf(M, ml[k].x);
+  if (M == -INFINITY) return;  // no cell attended: o keeps the short branch
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float Lsum = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxKL; ++k) {
+    if (k < K && sp[k] >= 0) {
+      const float w = ml[k].y * exp2f(ml[k].x - M);  // the slot's share of the softmax mass
+      Lsum += w;
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&part[k]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+      }
+    }
+  }
   const float a = alpha[(row / n) % H];
   const float inv = 1.f / Lsum;
-  V out;
   const __nv_bfloat162* hs = reinterpret_cast<const __nv_bfloat162*>(&sh);
+  uint4 out;
   __nv_bfloat162* ho = reinterpret_cast<__nv_bfloat162*>(&out);
 #pragma unroll
-  for (int e = 0; e < E / 2; ++e) {
+  for (int e = 0; e < 4; ++e) {
     const float2 f = __bfloat1622float2(hs[e]);
     ho[e] = __floats2bfloat162_rn((1.f - a) * f.x + a * (acc[2 * e] * inv),
                                   (1.f - a) * f.y + a * (acc[2 * e + 1] * inv));
   }
-  *reinterpret_cast<V*>(dst) = out;
+  *reinterpret_cast<uint4*>(dst) = out;
 }
 
 // ---- host side ------------------------------------------------------------------------------
@@ -660,7 +657,7 @@ bsa_status long_cells(const void* q, const void* k, const void* v, int B, int H,
          : cell == 32 ? run_dc(fs_long_tile_kernel<128, 32>, Tag<LongSmem<128, 32>>{})
                       : run_dc(fs_long_tile_kernel<128, 64>, Tag<LongSmem<128, 64>>{});
   if (rc != BSA_OK) return rc;
-  const unsigned cblocks = (unsigned)((rows * 16 + 255) / 256);
+  const unsigned cblocks = (unsigned)((rows * (d / 8) + 255) / 256);
   if (d == 64)
     fs_long_combine_kernel<64><<<cblocks, 256, 0, st>>>(w.slotpos, w.part_ml, w.part_o, alpha, H,
                                                          n, K, rows,
