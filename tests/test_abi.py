@@ -213,3 +213,16 @@ def test_outer_gate_arguments(bsa_lib):
     g = bsa_lib.bsa_gate_grad_outer
     assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 8, 2, 1024, 128, 64, 64, FAKE, None, 4, 0,
              None, 16, FAKE, None) == 1     # scores missing
+
+
+def test_freesolo_workspace_size_query(bsa_lib):
+    f = bsa_lib.bsa_freesolo_workspace_bytes
+    rows = 1 * 16 * 65536
+    base = f(1, 1, 16, 65536, 64, 32, 4)             # bf16, cell-major long branch
+    assert base >= 256 + 2 * rows * 64 * 2 + rows * 4 * (2 * 64 + 8)
+    assert f(1, 1, 16, 65536, 64, 32, 8) > base      # more slots, more partial rows
+    assert f(1, 1, 16, 65536, 64, 4, 4) > 0          # other cells: per-unit block unions
+    assert f(0, 1, 16, 65536, 64, 32, 4) == 256 + rows * 64 * 4   # fp32: rotated keys only
+    assert f(1, 0, 16, 65536, 64, 32, 4) == 0
+    assert f(1, 1, 16, 65536, 64, 32, 0) == 0
+    assert f(1, 1, 16, 65536, 64, 0, 4) == 0
