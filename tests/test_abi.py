@@ -226,3 +226,11 @@ def test_freesolo_workspace_size_query(bsa_lib):
     assert f(1, 0, 16, 65536, 64, 32, 4) == 0
     assert f(1, 1, 16, 65536, 64, 32, 0) == 0
     assert f(1, 1, 16, 65536, 64, 0, 4) == 0
+
+
+def test_recorded_traffic_matches_the_kernel_source():
+    """The bench reports a kernel's ncu DRAM traffic only while the device code it was captured
+    from is unchanged; after a kernel edit the capture must be taken again and re-keyed."""
+    import bench
+    for (workload, kernel), rec in bench.MEASURED_TRAFFIC.items():
+        assert bench.measured_traffic(workload, kernel) == rec["bytes"], (workload, kernel)
