@@ -8,8 +8,15 @@ refresh the summary of the current block, score every history block, Top-K, spar
 "layer" instances of the KV cache and summaries in turn, so the data a step touches is never in
 the 126 MB L2; the steps are timed with CUDA events on the launching stream.
 
+The same line carries the other rows of the hot path, each with a roofline block: the long
+decode at 512K (same fused step, plus its score / Top-K / attention breakdown through the
+separate calls), the summaries build (GB/s), the SAS gated prefill forward and gate gradient, and
+the FreeSolo prefill (TFLOP/s on the gathered FLOPs).  ``cpu_baseline`` is the fp64 oracle run on
+every host core (a process pool forked before the first GPU call), next to its one-thread figure.
+
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead (a bounded sample of
-batch rows per step) and prints the same JSON line with "impl": "reference".
+the decode step per timed step, on every host core) and prints the same JSON line with
+"impl": "reference".
 """
 from __future__ import annotations
 
@@ -41,8 +48,8 @@ WORKLOADS = {
 
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture of the kernel
-# built from the source whose hash is given (the capture command is in the profile summary
-# decode_fused_kernel__sas_gqa_decode_32k.md).  Reported only while the source is unchanged.
+# built from the source whose hash is given (the capture command is recorded with the decode
+# profile summary under profiles/).  Reported only while the source is unchanged.
 # The hash covers the device code of the source: the file up to its first host function
 # (`device_end`), so a change of the host-side launcher alone keeps the figure.
 MEASURED_TRAFFIC = {
@@ -179,13 +186,89 @@ def oracle_decode_sample(case, rows_b, summaries):
 
 def oracle_summaries(case, rows_b):
     from oracle import bsa_oracle as orc
-    G = case.Hq // case.Hk
     out = {}
     for bi in rows_b:
         for kh in range(case.Hk):
             out[(bi, kh)] = orc.block_summaries(case.k[bi, kh, :case.seq_lens[bi]], case.b)
-    del G
     return out
+
+
+# The oracle pool: worker processes forked from the parent BEFORE its first CUDA call (a process
+# forked after CUDA initialisation can hang), reading the case copy-on-write.  One task is one
+# (batch row, kv head) group: its G query heads scored, selected and attended by the oracle.
+_POOL_CASE = None
+
+
+def _oracle_group(task):
+    from threadpoolctl import threadpool_limits
+
+    from oracle import bsa_oracle as orc
+    bi, kh = task
+    case, summ = _POOL_CASE
+    G = case.Hq // case.Hk
+    with threadpool_limits(limits=1):
+        orc.decode_reference(case.q, case.k, case.v, case.seq_lens, case.b, case.K,
+                             rows=[(bi, h) for h in range(kh * G, (kh + 1) * G)],
+                             summaries={(bi, kh): summ[(bi, kh)]})
+    return bi, kh
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class OraclePool:
+    """Whole decode steps of the oracle (every batch row, every head) spread over ``cores``
+    forked worker processes, one single-threaded task per (batch row, kv head) group."""
+
+    def __init__(self, case, summ, cores):
+        import multiprocessing as mp
+        global _POOL_CASE
+        _POOL_CASE = (case, summ)
+        self.case, self.cores = case, cores
+        self.tasks = [(bi, kh) for bi in range(case.B) for kh in range(case.Hk)]
+        self.pool = mp.get_context("fork").Pool(cores)
+        self.pool.map(_oracle_group, self.tasks[:cores], chunksize=1)  # workers up and warm
+
+    def step(self) -> float:
+        """One decode step of the whole batch; returns seconds."""
+        t = time.perf_counter()
+        self.pool.map(_oracle_group, self.tasks, chunksize=1)
+        return time.perf_counter() - t
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baselines(case, seconds: float):
+    """The oracle as it stands on the host: on every core (whole decode steps, as many as fit in
+    about ``seconds``) and on one thread (batch rows, about ``seconds`` / 2).  Must run before the
+    process makes its first CUDA call (the pool forks)."""
+    summ = oracle_summaries(case, range(case.B))
+    cores = host_cores()
+    pool = OraclePool(case, summ, cores)
+    total, steps = 0.0, 0
+    while total < seconds or steps < 1:
+        total += pool.step()
+        steps += 1
+    pool.close()
+    multi = {"value": steps * case.B / total, "unit": "tokens/s", "cores": cores,
+             "kind": "oracle",
+             "sample": f"{steps} whole decode steps ({steps * case.B} tokens: every batch row, "
+                       f"all {case.Hq} heads) of the same workload, one forked single-threaded "
+                       "worker per core, one task per (batch row, kv head) group, summaries "
+                       "precomputed"}
+    tsec, done = 0.0, 0
+    while tsec < seconds / 2 and done < 64:
+        tsec += oracle_decode_sample(case, [done % case.B], summ)
+        done += 1
+    single = {"value": done / tsec, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+              "sample": f"{done} decode tokens (batch rows, all {case.Hq} heads), one thread"}
+    return multi, single
 
 
 def make_case(wl):
@@ -197,19 +280,20 @@ def make_case(wl):
 
 
 def run_reference(args):
-    """fp64 CPU oracle timed on the host: each step decodes one batch row (all heads)."""
+    """fp64 CPU oracle timed on the host cores: each timed step is one whole decode step of the
+    workload (every batch row, all heads) spread over a forked process pool."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
     case = make_case(args.workload)
-    nb = case.B
-    summ = oracle_summaries(case, range(nb))
-    for i in range(args.warmup):
-        oracle_decode_sample(case, [i % nb], summ)
-    total = 0.0
-    for i in range(args.steps):
-        total += oracle_decode_sample(case, [i % nb], summ)
+    summ = oracle_summaries(case, range(case.B))
+    cores = host_cores()
+    pool = OraclePool(case, summ, cores)
+    for _ in range(args.warmup):
+        pool.step()
+    total = sum(pool.step() for _ in range(args.steps))
+    pool.close()
     ms = total / args.steps * 1e3
-    value = args.steps / total  # one token (all heads of one sequence) per step
+    value = args.steps * case.B / total
     w = WORKLOADS[args.workload]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -218,13 +302,26 @@ def run_reference(args):
         "data": "synthetic (seeded N(0,1), bf16-rounded, planted needle blocks)",
         "config": {"workload": args.workload, **{k: w[k] for k in ("B", "Hq", "Hk", "d", "n",
                                                                    "b", "K")}},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": "one batch row (all 32 query heads) per step, summaries "
-                                   "precomputed as on the GPU"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step one whole decode step ({case.B} tokens, all "
+                                   f"{case.Hq} heads) on {cores} forked single-threaded workers, "
+                                   "summaries precomputed as on the GPU"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def roofline(bound, kernel, achieved, peak, unit, traffic=None, algorithmic=None,
+             peak_source=""):
+    """The roofline block of one row: achieved against the measured peak (frac), and the
+    ncu-recorded DRAM traffic of one launch when a capture of the current kernel exists."""
+    out = {"bound": bound, "kernel": kernel, "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": achieved / peak if peak else None, "traffic": traffic}
+    if algorithmic is not None:
+        out["algorithmic"] = algorithmic
+    out["peak_source"] = peak_source
+    return out
 
 
 def time_cuda(fn, reps, stream):
@@ -289,24 +386,31 @@ def run_prefill(dev, peaks, reps=5):
     t_ofwd = statistics.fmean(time_cuda(ofwd, max(2, reps // 2), stream))
     t_ograd = statistics.fmean(time_cuda(ograd, max(2, reps // 2), stream))
     peak = peaks["bf16_tflops"]
+    src = peaks["source"] + " bf16 (burst)"
     out["sas_gated_prefill_16k"] = {
         "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
                    "q_block": 64, "K": pc.K, "gate": "log-softmax over the selected blocks"},
         "forward": {"kernel": "prefill_tc_kernel (tcgen05)", "ms": t_fwd,
                     "gathered_gflop": fwd_flops / 1e9, "tflops": fwd_flops / t_fwd / 1e9,
-                    "roofline": {"bound": "tensor", "achieved": fwd_flops / t_fwd / 1e9,
-                                 "peak": peak, "unit": "TFLOP/s",
-                                 "frac": fwd_flops / t_fwd / 1e9 / peak,
-                                 "peak_source": peaks["source"] + " bf16 (burst)"}},
+                    "roofline": roofline("tensor", "prefill_tc_kernel", fwd_flops / t_fwd / 1e9,
+                                         peak, "TFLOP/s", peak_source=src)},
         "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
                       "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
-                      "frac_of_bf16_peak": grad_flops / t_grad / 1e9 / peak},
+                      "roofline": roofline("tensor", "gate_grad_tc_kernel",
+                                           grad_flops / t_grad / 1e9, peak, "TFLOP/s",
+                                           peak_source=src)},
         "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
                           "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
-                          "frac_of_hbm": sgrad_bytes / t_sgrad / 1e6 / peaks["hbm_gbs"]},
+                          "roofline": roofline("hbm", "selector_grad_kernel",
+                                               sgrad_bytes / t_sgrad / 1e6, peaks["hbm_gbs"],
+                                               "GB/s", algorithmic=sgrad_bytes,
+                                               peak_source=peaks["source"] + " (burst copy)")},
         "outer_gate": {"kernels": "prefill_tc_kernel, gate_grad_tc_kernel (tcgen05)",
                        "forward_ms": t_ofwd, "forward_tflops": fwd_flops / t_ofwd / 1e9,
-                       "grad_ms": t_ograd, "grad_tflops": grad_flops / t_ograd / 1e9},
+                       "grad_ms": t_ograd, "grad_tflops": grad_flops / t_ograd / 1e9,
+                       "roofline": roofline("tensor", "prefill_tc_kernel (outer gate)",
+                                            fwd_flops / t_ofwd / 1e9, peak, "TFLOP/s",
+                                            peak_source=src)},
     }
     del q, k, v, do, o, s, idx, cnt, lse, dg, o2, lse2, dg2
     torch.cuda.empty_cache()
@@ -339,10 +443,16 @@ def run_prefill(dev, peaks, reps=5):
         "config": {"B": fc.B, "H": fc.H, "d": fc.d, "n": fc.n, "cell": fc.cell,
                    "q_block": fc.q_block, "K": fc.K, "window": fc.window},
         "select": {"kernel": "split_hi_lo + freesolo_select_tc_kernel (tcgen05)", "ms": t_sel,
-                   "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9},
-        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode + block unions + prefill_tc_kernel long-branch mode (tcgen05)", "ms": t_att,
+                   "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9,
+                   "roofline": roofline("tensor", "freesolo_select_tc_kernel",
+                                        score_flops / t_sel / 1e9, peak, "TFLOP/s",
+                                        peak_source=src)},
+        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode + cell-major long "
+                                "branch (fs_long_* kernels, tcgen05 tiles) + combine", "ms": t_att,
                       "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,
-                      "frac_of_bf16_peak": att_flops / t_att / 1e9 / peak},
+                      "roofline": roofline("tensor", "freesolo attention (all launches)",
+                                           att_flops / t_att / 1e9, peak, "TFLOP/s",
+                                           peak_source=src)},
         "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),
     }
     del q, k, v, o, ws, sws, idx, cnt
@@ -405,37 +515,14 @@ def run_prefill(dev, peaks, reps=5):
     return out
 
 
-def run_gpu(args):
+def build_layers(dev, case, w, R):
+    """R "layers": the seeded case and R-1 copies with the kv heads (and their query heads)
+    rotated, so that each step reads memory the previous steps did not leave in L2."""
     import torch
-    import torch.distributed as dist
 
     import block_sparse_attention_summaries_b200 as bsa
-
-    if args.prefill_only:
-        torch.cuda.set_device(0)
-        bsa.lib()
-        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), load_peaks())}),
-              flush=True)
-        return
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev)
-    bsa.lib()
-
-    w = WORKLOADS[args.workload]
-    case = make_case(args.workload)
-    B, Hq, Hk, d, n, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K"))
+    B, Hq, Hk, d, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "b", "K"))
     G = Hq // Hk
-    C = (n + b - 1) // b
-    R = args.layers
-
-    # R "layers": the seeded case and R-1 copies with the kv heads (and their query heads)
-    # rotated, so each step reads cold memory (R x ~52 MB touched per cycle >> 126 MB of L2).
     q0 = torch.from_numpy(case.q).to(dev, torch.bfloat16)
     k0 = torch.from_numpy(case.k).to(dev, torch.bfloat16)
     v0 = torch.from_numpy(case.v).to(dev, torch.bfloat16)
@@ -450,14 +537,21 @@ def run_gpu(args):
                            lse=torch.empty(B, Hq, device=dev, dtype=torch.float32),
                            idx=torch.empty(B, Hq, K, device=dev, dtype=torch.int32),
                            count=torch.empty(B, Hq, device=dev, dtype=torch.int32)))
-    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    return layers
+
+
+def capture_fused(dev, layers, w, status, stream):
+    """One CUDA graph per layer holding the fused decode step (one kernel launch)."""
+    import torch
+
+    import block_sparse_attention_summaries_b200 as bsa
+    b, K = w["b"], w["K"]
 
     def fused(L):
         bsa.decode_step_fused(L["q"], L["k"], L["v"], L["mean_k"], b, K, append=True,
                               max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
                               idx=L["idx"], count=L["count"], status=status)
 
-    stream = torch.cuda.Stream(dev)
     graphs = []
     with torch.cuda.stream(stream):
         for L in layers:
@@ -469,11 +563,35 @@ def run_gpu(args):
                 fused(L)
             graphs.append(g)
     torch.cuda.synchronize(dev)
-    launches_per_step = 1
+    return graphs
 
-    # algorithmic bytes of one step: summaries scored + union of selected K/V blocks + q/o/idx
-    L0 = layers[0]
-    idx_h = L0["idx"].cpu().numpy()
+
+def time_graph_cycle(dev, graphs, steps, warmup, stream):
+    """Milliseconds of ``steps`` replays (graph i % R in turn) between two events on the
+    stream (an event recorded between two replays would cost the step about 2 us: it ends the
+    overlap of one launch's tail with the next one's start)."""
+    import torch
+    R = len(graphs)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            graphs[i % R].replay()
+        torch.cuda.synchronize(dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for i in range(steps):
+            graphs[i % R].replay()
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+    return ev[0].elapsed_time(ev[1])
+
+
+def decode_accounting(case, w, idx_h):
+    """Algorithmic bytes of one decode step and the needle recall of its selection: summaries
+    scored (every history block of every kv head, fp32) + the union over each GQA group of the
+    selected K/V blocks (each crosses HBM once) + the current block; q, o, the indices and the
+    appended summary as I/O."""
+    B, Hq, Hk, d, n, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K"))
+    G = Hq // Hk
     cur = (n - 1) // b
     union_blocks = per_head_blocks = 0
     for bi in range(B):
@@ -484,40 +602,26 @@ def run_gpu(args):
     cur_tokens = n - cur * b
     kv_bytes = (union_blocks - B * Hk) * b * d * 2 * 2 + B * Hk * cur_tokens * d * 2 * 2
     summary_bytes = B * Hk * cur * d * 4
-    step_bytes = kv_bytes + summary_bytes  # the benchmark spec's count: selected K/V + summaries
     io_bytes = B * Hq * d * 2 * 2 + B * Hq * (K * 4 + 8) + B * Hk * (d + 2) * 4
     hits = tot = 0
     for (bi, kh), blocks in case.needles.items():
         sel = set(int(x) for x in idx_h[bi, kh * G:(kh + 1) * G].ravel() if x >= 0)
         hits += len(sel & set(int(c) for c in blocks))
         tot += len(blocks)
+    return {"union_blocks": union_blocks, "per_head_blocks": per_head_blocks,
+            "kv_bytes": kv_bytes, "summary_bytes": summary_bytes, "io_bytes": io_bytes,
+            "needle_recall": hits / max(1, tot), "cur_tokens": cur_tokens}
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % R].replay()
-        torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        sampler.mark("t0")
-        # events bracket the K steps only: an event recorded between two replays costs the step
-        # about 2 us (it ends the overlap of one launch's tail with the next one's start)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        ev[0].record(stream)
-        for i in range(args.steps):
-            graphs[i % R].replay()
-        ev[1].record(stream)
-        torch.cuda.synchronize(dev)
-        sampler.mark("t1")
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-    total_ms = ev[0].elapsed_time(ev[1])
 
-    # the same step through the separate calls (score, Top-K, attention), for the breakdown
+def separate_calls(dev, layers, w, warmup, nsep, stream):
+    """The same step through the separate C-ABI calls (summary append + scores, Top-K, split-K
+    attention), each captured in its own graph: the per-stage breakdown in microseconds."""
+    import torch
+
+    import block_sparse_attention_summaries_b200 as bsa
+    B, Hq, Hk, d, n, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K"))
+    C = (n + b - 1) // b
+    R = len(layers)
     sep = []
     with torch.cuda.stream(stream):
         scores = torch.empty(B, Hq, C, device=dev, dtype=torch.float32)
@@ -544,8 +648,7 @@ def run_gpu(args):
                     fn()
                 gs.append(g)
             stage_graphs.append(gs)
-        nsep = max(50, min(args.steps, 400))
-        for i in range(args.warmup):
+        for i in range(warmup):
             for g in stage_graphs[i % R]:
                 g.replay()
         torch.cuda.synchronize(dev)
@@ -561,14 +664,187 @@ def run_gpu(args):
             e[3].record(stream)
             sep.append(e)
         torch.cuda.synchronize(dev)
-    sep_sel = statistics.fmean(e[0].elapsed_time(e[1]) for e in sep) * 1e3
-    sep_topk = statistics.fmean(e[1].elapsed_time(e[2]) for e in sep) * 1e3
-    sep_attn = statistics.fmean(e[2].elapsed_time(e[3]) for e in sep) * 1e3
-    sep_step = statistics.fmean(e[0].elapsed_time(e[3]) for e in sep) * 1e3
+    out = {"append+score": statistics.fmean(e[0].elapsed_time(e[1]) for e in sep) * 1e3,
+           "topk": statistics.fmean(e[1].elapsed_time(e[2]) for e in sep) * 1e3,
+           "attention": statistics.fmean(e[2].elapsed_time(e[3]) for e in sep) * 1e3,
+           "step": statistics.fmean(e[0].elapsed_time(e[3]) for e in sep) * 1e3}
+    out["selection_share"] = (out["append+score"] + out["topk"]) / max(out["step"], 1e-9)
+    del stage_graphs  # graphs before the buffers they replay into
+    return out
+
+
+def run_long_decode(dev, peaks, args, stream):
+    """The long-context decode row: 512K context, batch 1, K = 31 (the context of the SAS
+    review's headline decode figure, "Decoding efficiency", Fig. 7a/7c): the fused step timed
+    as the headline is, its roofline, the separate-call breakdown and the needle recall."""
+    import torch
+    wl = "long_decode_512k"
+    w = WORKLOADS[wl]
+    case = make_case(wl)
+    R = max(2, min(args.layers, 4))  # 4 x (33.5 MB summaries + union K/V) per cycle > 126 MB L2
+    layers = build_layers(dev, case, w, R)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    graphs = capture_fused(dev, layers, w, status, stream)
+    steps = max(50, min(args.steps, 400))
+    ms = time_graph_cycle(dev, graphs, steps, args.warmup, stream) / steps
+    acc = decode_accounting(case, w, layers[0]["idx"].cpu().numpy())
+    sep = separate_calls(dev, layers, w, args.warmup, max(20, min(args.steps, 100)), stream)
+    algo = acc["kv_bytes"] + acc["summary_bytes"] + acc["io_bytes"]
+    gbs = algo / (ms / 1e3) / 1e9
+    out = {"config": {"workload": wl, **{x: w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K")},
+                      "l2": f"{R} rotated layer instances"},
+           "us_per_step": ms * 1e3, "tokens_per_s": w["B"] / (ms / 1e3),
+           "algorithmic_bytes": algo, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+           "union_blocks": acc["union_blocks"], "needle_recall": acc["needle_recall"],
+           "status_word": int(status.max().item()),
+           "separate_calls_us": sep,
+           "roofline": roofline("hbm", "decode_fused_kernel", gbs, peaks["hbm_gbs"], "GB/s",
+                                traffic=measured_traffic(wl, "decode_fused_kernel"),
+                                algorithmic=algo,
+                                peak_source=peaks["source"] + " (burst copy)")}
+    del graphs
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_summaries_build(dev, peaks, layers, w, stream):
+    """The summaries build over the whole cache of each layer (prefill-time state): one HBM read
+    of K and the write of mean key, max norm and centre per block, as GB/s of those bytes."""
+    import torch
+
+    import block_sparse_attention_summaries_b200 as bsa
+    B, Hk, d, n, b = (w[x] for x in ("B", "Hk", "d", "n", "b"))
+    C = (n + b - 1) // b
+    L0 = layers[0]
+    mk, mx, ce = (torch.empty_like(L0[x]) for x in ("mean_k", "max_norm", "centre"))
+    R = len(layers)
+    fns = [lambda L=L: bsa.build_block_summaries(L["k"], b, None, 0, -1, mk, mx, ce)
+           for L in layers]
+    ts = []
+    with torch.cuda.stream(stream):
+        for f in fns:
+            f()
+        torch.cuda.synchronize(dev)
+        for i in range(3 * R):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fns[i % R]()
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize(dev)
+    ms = statistics.fmean(a.elapsed_time(z) for a, z in ts)
+    nbytes = B * Hk * n * d * 2 + B * Hk * C * (d + 2) * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": "summaries_kernel", "ms": ms, "bytes": nbytes, "gbs": gbs,
+            "roofline": roofline("hbm", "summaries_kernel", gbs, peaks["hbm_gbs"], "GB/s",
+                                 algorithmic=nbytes,
+                                 peak_source=peaks["source"] + " (burst copy)")}
+
+
+def flat_rows(rows):
+    """Scalar summary of the secondary rows (time, throughput, roofline fraction per row)."""
+    out = {}
+    sas = rows.get("sas_gated_prefill_16k")
+    if sas:
+        for key, name in (("forward", "sas_fwd"), ("gate_grad", "sas_gate_grad")):
+            out[f"{name}_ms"] = sas[key]["ms"]
+            out[f"{name}_tflops"] = sas[key]["tflops"]
+            out[f"{name}_frac"] = sas[key]["roofline"]["frac"]
+        out["sas_outer_fwd_frac"] = sas["outer_gate"]["roofline"]["frac"]
+    fs = rows.get("freesolo_prefill_64k")
+    if fs:
+        for key, name in (("select", "freesolo_select"), ("attention", "freesolo_attn")):
+            out[f"{name}_ms"] = fs[key]["ms"]
+            out[f"{name}_tflops"] = fs[key]["tflops"]
+            out[f"{name}_frac"] = fs[key]["roofline"]["frac"]
+    ld = rows.get("long_decode_512k")
+    if ld:
+        out["long_decode_512k_us"] = ld["us_per_step"]
+        out["long_decode_512k_tokens_per_s"] = ld["tokens_per_s"]
+        out["long_decode_512k_frac"] = ld["roofline"]["frac"]
+        out["long_decode_512k_selection_share"] = ld["separate_calls_us"]["selection_share"]
+    sb = rows.get("summaries_build_32k")
+    if sb:
+        out["summaries_build_gbs"] = sb["gbs"]
+        out["summaries_build_frac"] = sb["roofline"]["frac"]
+    return out
+
+
+def run_gpu(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    case = make_case(args.workload)
+    cpu_multi = cpu_single = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.prefill_only:
+        # the oracle pool forks: before this process makes its first CUDA call
+        cpu_multi, cpu_single = cpu_baselines(case, args.cpu_seconds)
+
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_summaries_b200 as bsa
+
+    if args.prefill_only:
+        torch.cuda.set_device(0)
+        bsa.lib()
+        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), load_peaks())}),
+              flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev)
+    bsa.lib()
+    peaks = load_peaks()
+
+    B, Hq, Hk, d, n, b, K = (w[x] for x in ("B", "Hq", "Hk", "d", "n", "b", "K"))
+    R = args.layers
+    layers = build_layers(dev, case, w, R)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    graphs = capture_fused(dev, layers, w, status, stream)
+    launches_per_step = 1
+    idx_h = layers[0]["idx"].cpu().numpy()
+    acc = decode_accounting(case, w, idx_h)
+    step_bytes = acc["kv_bytes"] + acc["summary_bytes"]  # selected K/V + summaries
+    io_bytes = acc["io_bytes"]
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        sampler.mark("t0")
+        # events bracket the K steps only: an event recorded between two replays costs the step
+        # about 2 us (it ends the overlap of one launch's tail with the next one's start)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ev[0].record(stream)
+        for i in range(args.steps):
+            graphs[i % R].replay()
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+        sampler.mark("t1")
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+    total_ms = ev[0].elapsed_time(ev[1])
+
+    sep = separate_calls(dev, layers, w, args.warmup, max(50, min(args.steps, 400)), stream)
 
     # GQA-shared selection and bf16 summaries (bsa_decode_step_ex flags): time per step on the same
     # rotated layers, algorithmic bytes, and how far the selection moves from the per-head fp32 one
     variants = {}
+    G = Hq // Hk
+    cur = (n - 1) // b
     ref_sets = [set(int(x) for x in row if x >= 0) for row in idx_h.reshape(-1, K)]
     for name, flags in (("bf16_summaries", bsa.DECODE_BF16_SUMMARIES),
                         ("per_head_fp32_control", 0),
@@ -597,27 +873,19 @@ def run_gpu(args):
                 with torch.cuda.graph(g, stream=stream):
                     vstep()
                 vgraphs.append(g)
-            nv = max(50, min(args.steps, 400))
-            for i in range(args.warmup):
-                vgraphs[i % R].replay()
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for i in range(nv):
-                vgraphs[i % R].replay()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-        v_us = e0.elapsed_time(e1) / nv * 1e3
+        nv = max(50, min(args.steps, 400))
+        v_us = time_graph_cycle(dev, vgraphs, nv, args.warmup, stream) / nv * 1e3
         del vgraphs  # graphs first, then the buffers they replay into
         del vbufs
-        v_union = v_hits = 0
+        v_union = v_hits = tot = 0
         for bi in range(B):
             for kh in range(Hk):
                 sel = set(int(x) for x in vidx[bi, kh * G:(kh + 1) * G].ravel() if x >= 0)
                 v_union += len(sel) + 1
                 blocks = case.needles.get((bi, kh), [])
                 v_hits += len(sel & set(int(c) for c in blocks))
-        v_kv = (v_union - B * Hk) * b * d * 2 * 2 + B * Hk * cur_tokens * d * 2 * 2
+                tot += len(blocks)
+        v_kv = (v_union - B * Hk) * b * d * 2 * 2 + B * Hk * acc["cur_tokens"] * d * 2 * 2
         v_sum = B * Hk * cur * d * (2 if bf16_sum else 4)
         v_bytes = v_kv + v_sum + io_bytes
         agree = statistics.fmean(
@@ -625,7 +893,7 @@ def run_gpu(args):
             for ref, row in zip(ref_sets, vidx.reshape(-1, K)))
         variants[name] = {"us_per_step": v_us, "tokens_per_s": B / (v_us / 1e6),
                           "algorithmic_bytes": v_bytes, "gbs": v_bytes / (v_us / 1e6) / 1e9,
-                          "frac_of_hbm": v_bytes / (v_us / 1e6) / 1e9 / load_peaks()["hbm_gbs"],
+                          "frac_of_hbm": v_bytes / (v_us / 1e6) / 1e9 / peaks["hbm_gbs"],
                           "union_blocks": v_union, "needle_recall": v_hits / max(1, tot),
                           "index_agreement_vs_per_head_fp32": agree}
 
@@ -661,7 +929,6 @@ def run_gpu(args):
     value = job_throughput(B, world, args.steps, mx_total)
     e2e_value = job_throughput(B, world, args.steps, e2e_total)
 
-    peaks = load_peaks()
     avg_ms = total_ms / args.steps  # one fused kernel per step
     achieved = (step_bytes + io_bytes) / (avg_ms / 1e3) / 1e9
     line = {
@@ -681,14 +948,14 @@ def run_gpu(args):
                      "traffic": measured_traffic(args.workload, "decode_fused_kernel"),
                      "algorithmic_bytes": step_bytes + io_bytes,
                      "peak_source": peaks["source"] + " (burst copy)"},
-        "hbm": {"north_star_bytes": step_bytes, "gbs": step_bytes / (avg_ms / 1e3) / 1e9,
+        "hbm": {"selected_kv_plus_summary_bytes": step_bytes,
+                "gbs": step_bytes / (avg_ms / 1e3) / 1e9,
                 "frac": step_bytes / (avg_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                 "what": "selected K/V (union per GQA group) + summaries, per step time"},
-        "separate_calls_us": {"append+score": sep_sel, "topk": sep_topk, "attention": sep_attn,
-                              "step": sep_step},
+        "separate_calls_us": sep,
         "variants": variants,
-        "union_blocks": union_blocks, "per_head_blocks": per_head_blocks,
-        "needle_recall": hits / max(1, tot), "status_word": st_word,
+        "union_blocks": acc["union_blocks"], "per_head_blocks": acc["per_head_blocks"],
+        "needle_recall": acc["needle_recall"], "status_word": st_word,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * Hq * d * 2,
                 "d2h_bytes_per_step": B * Hq * d * 2,
                 "what": "per step: pinned-host q -> device, the decode step through a prepared "
@@ -698,23 +965,21 @@ def run_gpu(args):
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],
     }
+    rows = {}
+    rows["summaries_build_32k"] = run_summaries_build(dev, peaks, layers, w, stream)
+    del graphs, plans, layers
+    torch.cuda.empty_cache()
+    if not args.no_long and args.workload != "long_decode_512k":
+        rows["long_decode_512k"] = run_long_decode(dev, peaks, args, stream)
     if not args.no_prefill:
-        del layers
-        torch.cuda.empty_cache()
-        line["prefill"] = run_prefill(dev, peaks)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        summ = oracle_summaries(case, range(case.B))
-        tsec, done = 0.0, 0
-        while tsec < args.cpu_seconds and done < 64:
-            tsec += oracle_decode_sample(case, [done % case.B], summ)
-            done += 1
-        line["cpu_baseline"] = {"value": done / tsec, "unit": "tokens/s", "cores": 1,
-                                "kind": "oracle",
-                                "sample": f"{done} decode tokens (batch rows, all {Hq} heads) of "
-                                          "the same workload, summaries precomputed"}
+        rows.update(run_prefill(dev, peaks))
+    line["prefill"] = flat_rows(rows)
+    line["rows"] = rows
+    if cpu_multi is not None:
+        line["cpu_baseline"] = cpu_multi
+        line["cpu_baseline_one_thread"] = cpu_single
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graphs, stage_graphs
     if world > 1:
         dist.destroy_process_group()
 
@@ -726,10 +991,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="sas_gqa_decode_32k", choices=sorted(WORKLOADS))
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--layers", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the 512K long-decode row")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill rows (profiling the prefill kernels)")
     args = ap.parse_args()

@@ -42,6 +42,7 @@ SIGNATURES = [
     ("bsa_sparse_attn_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     ("bsa_sparse_attn_decode_noalloc", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P,
                                             _I, _I, _I, _P, _I, _P, _P, _P]),
+    ("bsa_noalloc_status", _I, [_P]),
     ("bsa_gate_grad_outer", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P,
                                  _I, _I, _P, _I, _P, _P]),
     ("bsa_gate_grad", _I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _I, _I,
@@ -266,6 +267,14 @@ def sparse_attn_decode_noalloc(q, k, v, idx, b, count=None, seq_lens=None, gate=
         _norm_code(norm), _ptr(scores), scores_ld, _ptr(o), _ptr(lse), _stream(q.device)),
         "bsa_sparse_attn_decode_noalloc")
     return o, lse
+
+
+def noalloc_status(device=None) -> int:
+    """Status of the last allocation-free decode call on ``device`` (0 ok, else
+    BSA_ERR_TIMEOUT); reads and clears the status word of the library's fixed array."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(device):  # the array of the current device is read
+        return int(lib().bsa_noalloc_status(_stream(torch.device(device))))
 
 
 def gate_grad(q, k, v, o, lse, dout, idx, b, scores, q_block=None, count=None, norm="selected",

@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
 
+  int i_stop = ne;  // the iteration at which a timed-out wait ended the loop (ne: none did)
   for (int i = 0; i < ne; ++i) {
     const int st = i & 1;
     const int ue = s + i * S;
@@ -241,7 +242,10 @@ __global__ void __launch_bounds__(kThreads)
     }
     if (!mbar_wait_bounded(&bar[st], (i >> 1) & 1)) s_abort = 1;
     __syncthreads();
-    if (s_abort) break;
+    if (s_abort) {
+      i_stop = i;
+      break;
+    }
     const T* kt = kbuf[st];
     const T* vt = vbuf[st];
 
@@ -324,32 +328,36 @@ __global__ void __launch_bounds__(kThreads)
     if (tid == 0 && i + 2 < ne) issue(i + 2);
   }
 
-  if (s_abort) {
-    // give copies still in flight a bounded chance to land before the CTA exits
+  const bool aborted = s_abort != 0;
+  if (aborted) {
+    // The copies still in flight are those of iterations i_stop and i_stop + 1 (if issued), with
+    // the parities of their own phases; give them a bounded chance to land before the CTA leaves
+    // its shared memory, then record the timeout.  The CTA still arrives on the counter below, so
+    // the counter ends the call at zero for the next one.
     if (tid == 0) {
-      for (int i = 0; i < min(ne, 2); ++i) (void)mbar_wait_bounded(&bar[i], 0, 1u << 16);
+      for (int j = i_stop; j < min(ne, i_stop + 2); ++j)
+        (void)mbar_wait_bounded(&bar[j & 1], (j >> 1) & 1, 1u << 16);
       report_timeout(p.status, 1);
     }
-    return;
-  }
-
-  // ---- 4. partial (m, l, o) of this split -------------------------------------------------
-  float* red = reinterpret_cast<float*>(smem);  // reuse the K stage: [TP][G][D]
+  } else {
+    // ---- 4. partial (m, l, o) of this split -----------------------------------------------
+    float* red = reinterpret_cast<float*>(smem);  // reuse the K stage: [TP][G][D]
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    red[((size_t)tp * G + g) * D + 2 * cg] = acc[g][0];
-    red[((size_t)tp * G + g) * D + 2 * cg + 1] = acc[g][1];
-  }
-  __syncthreads();
-  for (int e = tid; e < G * D; e += kThreads) {
-    const int g = e / D, dcol = e % D;
-    float sum = 0.f;
-    for (int u = 0; u < TP; ++u) sum += red[((size_t)u * G + g) * D + dcol];
-    float* pp = p.part + (((size_t)bi * Hq + h0 + g) * S + s) * (D + 2);
-    pp[dcol] = sum;
-    if (dcol == 0) {
-      pp[D] = s_m[g];
-      pp[D + 1] = s_l[g];
+    for (int g = 0; g < G; ++g) {
+      red[((size_t)tp * G + g) * D + 2 * cg] = acc[g][0];
+      red[((size_t)tp * G + g) * D + 2 * cg + 1] = acc[g][1];
+    }
+    __syncthreads();
+    for (int e = tid; e < G * D; e += kThreads) {
+      const int g = e / D, dcol = e % D;
+      float sum = 0.f;
+      for (int u = 0; u < TP; ++u) sum += red[((size_t)u * G + g) * D + dcol];
+      float* pp = p.part + (((size_t)bi * Hq + h0 + g) * S + s) * (D + 2);
+      pp[dcol] = sum;
+      if (dcol == 0) {
+        pp[D] = s_m[g];
+        pp[D + 1] = s_l[g];
+      }
     }
   }
 
@@ -363,6 +371,13 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // A split that timed out wrote the status word before it arrived: its partial is missing, so
+  // the merge is skipped (the output is not written; the caller reads BSA_ERR_TIMEOUT) and the
+  // counter is reset for the next call.
+  if (p.status && *reinterpret_cast<volatile int*>(p.status) != 0) {
+    if (tid == 0) p.counters[bi * p.Hk + kh] = 0;
+    return;
+  }
   float* wgt = reinterpret_cast<float*>(smem);  // [G][S] merge weights, in the stage area
   for (int g = warp; g < G; g += kWarps) {
     const float* pb = p.part + ((size_t)bi * Hq + h0 + g) * S * (D + 2);
@@ -557,4 +572,12 @@ extern "C" bsa_status bsa_sparse_attn_decode_noalloc(
   }
   return decode_attn(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, idx, count, K, gate, norm,
                      scores, scores_ld, o, lse, ws, kNoAllocScratchBytes, st);
+}
+
+extern "C" bsa_status bsa_noalloc_status(void* stream) {
+  using namespace bsa;
+  void* ws = nullptr;
+  const bsa_status rc = noalloc_scratch(&ws);
+  if (rc != BSA_OK) return rc;
+  return bsa_workspace_status(ws, stream);  // the status word sits at the array's start
 }

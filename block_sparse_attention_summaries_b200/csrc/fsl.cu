@@ -1,6 +1,6 @@
 // FS-L: pre-query pruning of the FreeSolo cells and selection over the kept cells (decode).
 //
-// [FreeSolo] "How it works", FS-L variant: before any query arrives each head keeps its W most
+// [FreeSolo] "How it differs", FS-L variant: before any query arrives each head keeps its W most
 // recent cells and the P cells of largest maximum key norm; a query then scores only the kept
 // cells with the full method's cell score
 //     r_c = q . kbar_c / sqrt(d) + lambda_h a_c erf((i - p_c) / (2 sigma_h))

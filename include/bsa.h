@@ -7,7 +7,8 @@
  *                Context Ranking": "Background" (Eq. 1-3), "The new approach" (Eq. 4, Eq. 9),
  *                "Why the four design choices matter" (Eq. 5, log g = s - LSE(s)),
  *                "How it works: a worked example", "Decoding efficiency" (Fig. 7).
- *   [FreeSolo]   summary page "FreeSolo가 학습 길이의 64배까지 제로샷 검색을 유지한다": "How it works".
+ *   [FreeSolo]   summary page "FreeSolo가 학습 길이의 64배까지 제로샷 검색을 유지한다": "How it works"
+ *                (cells, summaries, cell score, two branches), "How it differs" (FS-L, FS-B).
  *   [Monodratic] article "Monodratic、学習ルーティングによりスパース因果アテンションの選択性を高められると
  *                主張": guaranteed local block + exact causal softmax over the selected tokens.
  *
@@ -218,8 +219,11 @@ bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v, bsa_d
  *             log-sum-exp of the ungated logits.
  *   o         [B, Hq, nq, d] out (dtype dt);  lse  optional [B, Hq, nq] float32 out.
  *   workspace device scratch of bsa_sparse_attn_workspace_bytes() bytes, zero-filled before its
- *             first use; each successful call leaves it reusable.  Calls sharing one workspace
- *             must not run concurrently.
+ *             first use; each call leaves it reusable (its arrival counters back at zero, also
+ *             when a bounded wait ran out).  A wait that ran out writes the status word and the
+ *             call then leaves o and lse unwritten; until bsa_workspace_status() reads and clears
+ *             that word, later decode calls on the workspace skip their final merge as well.
+ *             Calls sharing one workspace must not run concurrently.
  */
 bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
                                int Hq, int Hk, int nq, int n, int d, int b,
@@ -278,7 +282,7 @@ bsa_status bsa_selector_grad(const float* scores, int scores_ld, const int* n_ca
                              bsa_gate_norm norm, int rows, float* ds, int ds_ld, void* stream);
 
 /*
- * bsa_fsl_prune -- FS-L pre-query pruning ([FreeSolo] "How it works", FS-L variant): before any
+ * bsa_fsl_prune -- FS-L pre-query pruning ([FreeSolo] "How it differs", FS-L): before any
  * query arrives, each (batch, head) row keeps its W most recent candidate cells and the P cells
  * of largest maximum key norm among the older ones (lower index on ties, NaN last).
  *   max_norm  [rows, C] float32 (from bsa_build_block_summaries with b = cell).
@@ -381,8 +385,9 @@ size_t bsa_freesolo_workspace_bytes(bsa_dtype dt, int B, int H, int n, int d, in
  *  - Every call shares the one array, which keeps the previous call's contents; each call zeroes
  *    the parts that must start at zero.  Calls that overlap on the GPU (other streams, other
  *    threads, concurrent graph launches) race on the array and give wrong results.
- *  - A bounded wait that runs out is not reported by this call (the status word is cleared at
- *    the start of the next one).
+ *  - A bounded wait that runs out writes the array's status word; o and lse are then left
+ *    unwritten.  bsa_noalloc_status() reads and clears that word (the next call on the device
+ *    also clears it when it starts).
  */
 bsa_status bsa_sparse_attn_decode_noalloc(const void* q, const void* k, const void* v,
                                           bsa_dtype dt, int B, int Hq, int Hk, int n, int d,
@@ -390,6 +395,12 @@ bsa_status bsa_sparse_attn_decode_noalloc(const void* q, const void* k, const vo
                                           const int* count, int K, bsa_gate_mode gate,
                                           bsa_gate_norm norm, const float* scores, int scores_ld,
                                           void* o, float* lse, void* stream);
+
+/* Status of the last bsa_sparse_attn_decode_noalloc call on the current device: reads and clears
+ * the status word of the library's fixed array (synchronises the stream; no counterpart in the
+ * pages).  Returns BSA_OK, BSA_ERR_TIMEOUT (a bounded wait of that call ran out; its o and lse
+ * were not written) or BSA_ERR_CUDA. */
+bsa_status bsa_noalloc_status(void* stream);
 
 /* Read and clear the status word a bounded device wait writes into a workspace
  * (synchronises the stream).  Returns BSA_OK or BSA_ERR_TIMEOUT (or BSA_ERR_CUDA). */

@@ -15,13 +15,16 @@ Sources (cited by page title and the section / equation on it):
   (Fig. 7).
 * [FreeSolo] the summary page "FreeSolo가 학습 길이의 64배까지 제로샷 검색을 유지한다" --
   section "How it works" (cells, the three summaries, the query-block prefix, the erf-biased cell
-  score, top-K cells, the RoPE sliding-window branch, the NoPE long branch, the per-head mix).
+  score, top-K cells, the RoPE sliding-window branch, the NoPE long branch, the per-head mix)
+  and section "How it differs" (the FS-L variant: W recent cells plus the P largest key norms,
+  pruned before the query arrives, a fixed-size state; the FS-B variant: two forests per head
+  searched by a beam with node upper bounds, log-sum-exp re-rank over token keys).
 * [Monodratic] the article "Monodratic、学習ルーティングによりスパース因果アテンションの選択性を高め
   られると主張" -- section on turning sparse attention into a retrieval decision (guaranteed local
   block, exact causal softmax over the selected tokens, no future block reachable, sparse-vs-dense
   mask parity).
 
-Readings where the pages are silent or garbled (each listed with its reason in the design doc):
+Readings where the pages are silent or garbled (the numbering is that of the design notes):
 
 * R1 gate normaliser: log g_m = s_m - LSE over either the selected history blocks
   ("selected") or every history block ("all"); the worked example of [SAS] uses all blocks.
@@ -171,7 +174,7 @@ def topk_blocks(s, n_cand: int, K: int) -> list[int]:
 def fsl_candidates(max_norm, n_cells: int, W: int, P: int) -> list[int]:
     """FS-L pre-query pruning: the cells a head keeps before any query arrives.
 
-    [FreeSolo] "How it works", the FS-L variant: each head keeps its W most recent cells and the
+    [FreeSolo] "How it differs" (FS-L): each head keeps its W most recent cells and the
     P cells of largest maximum key norm, and queries pick their top K inside that set.  R18: the
     P cells are taken among the cells older than the W recent ones (the two parts are disjoint),
     larger norm first, lower index on ties, NaN last; fewer cells than W + P are all kept.
@@ -185,8 +188,9 @@ def fsl_candidates(max_norm, n_cells: int, W: int, P: int) -> list[int]:
 def fsl_select(q, i, mean_k, max_norm, centre, lam, sigma, cand, K) -> list[int]:
     """Top-K of the FreeSolo cell score over the pruned candidates only (ascending cells).
 
-    [FreeSolo] "How it works": the FS-L query scores the kept cells with the same r_ic as the
-    full method and reads its K best.  R18 tie rule: larger score, then lower cell index.
+    [FreeSolo] "How it differs" (FS-L) with the cell score of "How it works": the FS-L query
+    scores the kept cells with the same r_ic as the full method and reads its K best.  R18 tie
+    rule: larger score, then lower cell index.
     """
     cand = [int(c) for c in cand]
     if not cand:

@@ -1,4 +1,4 @@
-"""GPU parity of FS-L pre-query pruning and selection ([FreeSolo] "How it works", FS-L variant)
+"""GPU parity of FS-L pre-query pruning and selection ([FreeSolo] "How it differs", FS-L)
 against the fp64 oracle: pruning bit-exact; selection bit-exact where the K-th and (K+1)-th
 kept scores differ by more than 1e-4 relative, else one of the oracle's valid sets."""
 import numpy as np
@@ -56,15 +56,24 @@ def test_fsl_select_matches_oracle(lam):
         sig_t = torch.full((H,), 4096.0, device=DEV)
     idx, cnt = bsa.fsl_select(q, torch.from_numpy(pos).to(DEV), mean_k, mx, ce, lam_t, sig_t,
                               cand, ccnt, K)
-    cand, idx, cnt = cand.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy()
-    mx_h = mx.cpu().numpy()
+    cand, ccnt, idx, cnt = (x.cpu().numpy() for x in (cand, ccnt, idx, cnt))
     for bi in range(B):
         for h in range(H):
             summ = orc.block_summaries(fc.k[bi, h].astype(np.float64), cell)
             mk, a, c = summ
             nc = int(n_cells[bi, h])
-            kept = orc.fsl_candidates(mx_h[bi, h].astype(np.float64), nc, W, P)
-            assert list(cand[bi, h, :len(kept)]) == kept
+            # the kept set from the oracle's own key norms (fp64 from K, rounded to fp32, the
+            # precision the kernel decides in): the W newest cells plus a valid P-set of the older
+            # ones -- exact unless the P-th and (P+1)-th norms lie within 1e-4 relative
+            recent = list(range(max(0, nc - W), nc))
+            older = nc - len(recent)
+            p_sets = orc.valid_selections(orc.round_f32(a), older, P)
+            assert p_sets is not None
+            kept_sets = [sorted(list(ps) + recent) for ps in p_sets]
+            assert orc.fsl_candidates(orc.round_f32(a), nc, W, P) in kept_sets
+            kept = [int(x) for x in cand[bi, h, :int(ccnt[bi, h])]]
+            assert kept in kept_sets, (bi, h)
+            assert np.all(cand[bi, h, int(ccnt[bi, h]):] == -1)
             qv = q_np[bi, h].astype(np.float64)
             i = int(pos[bi])
             r = orc.round_f32(orc.freesolo_scores(qv, i, mk, a, c, lam or 0.0, 4096.0, nc))

@@ -436,6 +436,27 @@ def test_rope_properties():
     assert np.allclose(orc.rope(x, 0), x, atol=0)
 
 
+def test_rope_hand_values():
+    """R8 written out by hand for d = 4 at position 100 (base 10000, rotate-half pairing): the
+    pair (0, 2) turns by 100 * 10000^0 = 100 rad and the pair (1, 3) by 100 * 10000^(-2/4) = 1 rad.
+    cos 100 = 0.8623188722876839, sin 100 = -0.5063656411097588 (100 - 15 * 2 pi = 5.7522 rad),
+    cos 1 = 0.5403023058681398, sin 1 = 0.8414709848078965.  An interleaved pairing ((0, 1),
+    (2, 3)) or another frequency exponent (for example 10000^(-t/d)) gives other numbers."""
+    got = orc.rope(np.array([1.0, 2.0, 3.0, 4.0]), 100)
+    want = [1 * 0.8623188722876839 - 3 * -0.5063656411097588,   # 2.3814157956169604
+            2 * 0.5403023058681398 - 4 * 0.8414709848078965,    # -2.2852793274953065
+            3 * 0.8623188722876839 + 1 * -0.5063656411097588,   # 2.0805909757532928
+            4 * 0.5403023058681398 + 2 * 0.8414709848078965]    # 3.844151193088352
+    assert np.allclose(got, want, rtol=0, atol=1e-13)
+    assert np.allclose(got, [2.3814157956169604, -2.2852793274953065, 2.0805909757532928,
+                             3.844151193088352], rtol=0, atol=1e-13)
+    # the same rotation as complex multiplication: (x_t + i x_{t+d/2}) * exp(i pos theta^(-2t/d))
+    d, pos = 8, 37
+    x = rnd(33, d)
+    z = (x[:d // 2] + 1j * x[d // 2:]) * np.exp(1j * pos * 10000.0 ** (-np.arange(d // 2) / (d / 2)))
+    assert np.allclose(orc.rope(x, pos), np.concatenate([z.real, z.imag]), atol=1e-13)
+
+
 def test_freesolo_infinite_window_short_branch_is_dense_rope_attention():
     n, d, cell, qb = 96, 8, 8, 32
     q, k, v = rnd(30, n, d), rnd(31, n, d), rnd(32, n, d)
