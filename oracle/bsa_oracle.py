@@ -47,6 +47,12 @@ Readings where the pages are silent or garbled (the numbering is that of the des
 * R20 outer gate (f1 variant): the gate multiplies the value contributions of its block outside
   the softmax, o = sum_j g_m(j) p_j v_j with p the ungated softmax; the current block has gate 1;
   g = softmax of the scores over the normaliser set, as for the inner gate.
+* R21 FS-B (the pages name the forests' contents, the beam width and the re-rank but not the tree
+  shape): per head one forest over every candidate cell and one over the ceil(n/2) cells of
+  largest key norm; a forest is a row of perfect binary trees over consecutive cells in position
+  order (one per set bit of the cell count); a node keeps the mean of its leaves' mean keys, the
+  largest distance of a leaf mean key from it (radius), the largest leaf norm and the smallest
+  leaf centre; the beam ranks nodes by the Cauchy-Schwarz bound built from those four values.
 * R19 GQA-shared selection (a variant; the pages leave per-head versus shared selection open):
   the group's score of a block is the mean of its query heads' scores, its top-K is attended by
   every head of the group; bf16 summaries are the float32 mean keys rounded to the nearest
@@ -198,6 +204,65 @@ def fsl_select(q, i, mean_k, max_norm, centre, lam, sigma, cand, K) -> list[int]
     r = freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, max(cand) + 1)
     order = sorted(cand, key=lambda c: _rank_key(float(round_f32(r[c])), c))
     return sorted(order[:min(K, len(cand))])
+
+
+def _outranks(a, x: int, y: int) -> bool:
+    """Cell x ranks above cell y by maximum key norm (larger first, lower index on ties, NaN last)."""
+    return _rank_key(float(a[x]), x) < _rank_key(float(a[y]), y)
+
+
+def fsl_state_new(W: int, P: int) -> dict:
+    """An empty FS-L state: no candidate cell yet ([FreeSolo] "How it differs", FS-L: the state a
+    head keeps has a fixed size, W recent cells plus P cells chosen by key norm)."""
+    return {"W": W, "P": P, "n_cells": 0, "older": []}
+
+
+def fsl_state_advance(state: dict, max_norm, n_cells: int) -> dict:
+    """Grow the candidate prefix of an FS-L state to ``n_cells`` cells, one cell at a time.
+
+    [FreeSolo] "How it differs" (FS-L): the pruning happens before the query arrives and the state
+    stays W + P cells.  R18 as an update rule: the W newest candidate cells are kept outright; when
+    a cell drops out of them it joins the older cells, of which the state keeps the P best by
+    maximum key norm (larger first, lower index on ties, NaN last).  The joining cell has the
+    highest index of all older cells, so it enters only if it strictly outranks the lowest-ranked
+    kept older cell (which it then replaces), or if fewer than P are kept.  Each step looks at
+    the P kept cells only, never at the whole prefix.
+    """
+    W, P = state["W"], state["P"]
+    older = list(state["older"])
+    for m in range(state["n_cells"] + 1, n_cells + 1):  # the prefix grows to m cells
+        c = m - 1 - W  # the cell leaving the W newest
+        if c < 0 or P == 0:
+            continue
+        if len(older) < P:
+            older.append(c)
+            continue
+        worst = older[0]
+        for x in older[1:]:
+            if _outranks(max_norm, worst, x):
+                worst = x
+        if _outranks(max_norm, c, worst):
+            older.remove(worst)
+            older.append(c)
+    return {"W": W, "P": P, "n_cells": max(n_cells, state["n_cells"]), "older": older}
+
+
+def fsl_state_cells(state: dict) -> list[int]:
+    """The cells an FS-L state keeps: its older cells and the W newest, ascending."""
+    n, W = state["n_cells"], state["W"]
+    return sorted(state["older"]) + list(range(max(0, n - W), n))
+
+
+def fsl_decode_row(q, k, v, i, summaries, cand, cell, K, window, lam, sigma, alpha, theta):
+    """FS-L decode output of the query at position i of one head: the two branches of the full
+    method ([FreeSolo] "How it works": RoPE window, NoPE long branch, per-head mix) with the long
+    branch's cells chosen among the state's kept cells ``cand`` only ([FreeSolo] "How it
+    differs", FS-L: the query takes its top K inside the pruned set)."""
+    mean_k, max_norm, centre = summaries
+    sel = fsl_select(q, i, mean_k, max_norm, centre, lam, sigma, cand, K)
+    o, _ = freesolo_row(q, k, v, i, summaries, cell, 128, K, window, lam, sigma, alpha, theta,
+                        selection=sel)
+    return o, sel
 
 
 def round_f32(x):
@@ -625,13 +690,155 @@ def freesolo_row(q, k, v, i, summaries, cell, q_block, K, window, lam, sigma, al
     w /= w.sum()
     o_short = w @ np.asarray(v[lo:i + 1], dtype=np.float64)
     nc = freesolo_num_candidates(i, cell, q_block)
-    if nc == 0:
+    if nc == 0 or (selection is not None and len(selection) == 0):
         return o_short, []
     r = round_f32(freesolo_scores(q, i, mean_k, max_norm, centre, lam, sigma, nc))
     sel = topk_blocks(r, nc, K) if selection is None else list(selection)
     toks = np.concatenate([np.arange(*block_range(c, k.shape[0], cell)) for c in sel])
     o_long, _, _ = attend(q, k, v, toks, np.zeros(len(toks)))
     return (1.0 - alpha) * o_short + alpha * o_long, sel
+
+
+# ----------------------------------------------------------------------------------------------
+# FS-B: forests of cell summaries searched by a beam (FreeSolo "How it differs")
+# ----------------------------------------------------------------------------------------------
+
+
+def fsb_high_cells(max_norm, n_cells: int) -> list[int]:
+    """The cells of the second FS-B forest: those of norm at or above the median of the prefix.
+
+    [FreeSolo] "How it differs" (FS-B): one forest holds the whole prefix, the other only the
+    high-norm cells at or above the median.  R21: "at or above the median" is read as the
+    ceil(n / 2) cells of largest maximum key norm (larger first, lower index on ties, NaN last) --
+    the same set as norm >= median whenever no two norms tie at the middle, and always exactly
+    half (rounded up).  Returns ascending cell indices.
+    """
+    return topk_blocks(max_norm, n_cells, (n_cells + 1) // 2)
+
+
+def fsb_forest(cells, mean_k, max_norm, centre) -> list[dict]:
+    """FS-B forest over ``cells`` (ascending): its nodes, each with the page's four summaries.
+
+    [FreeSolo] "How it differs" (FS-B): every node stores a mean key, a radius, a maximum norm and
+    a minimum position.  R21: the trees are perfect binary trees over consecutive cells in position
+    order, one per set bit of the cell count, largest first (m = 13 cells give trees over the
+    first 8, the next 4 and the last one); a node over leaves L has mean key mu = mean of their
+    mean keys, radius rho = max over L of ||kbar_c - mu||_2, maximum norm = max over L of a_c and
+    minimum position = min over L of p_c.  Returns every node as a dict with its leaves' range
+    [lo, hi) in ``cells``, its height (leaves 0), whether it is a root, and the indices of its
+    children in the returned list.
+    """
+    cells = [int(c) for c in cells]
+    m = len(cells)
+    nodes = []
+
+    def build(lo, hi, height, root):
+        leaves = cells[lo:hi]
+        mu = np.mean([mean_k[c] for c in leaves], axis=0)
+        rho = max(math.sqrt(float(np.dot(mean_k[c] - mu, mean_k[c] - mu))) for c in leaves)
+        if height == 0:
+            rho = 0.0
+        node = {"lo": lo, "hi": hi, "height": height, "root": root, "first": leaves[0],
+                "mu": mu, "rho": rho, "amax": max(float(max_norm[c]) for c in leaves),
+                "pmin": min(float(centre[c]) for c in leaves), "children": []}
+        at = len(nodes)
+        nodes.append(node)
+        if height > 0:
+            mid = (lo + hi) // 2
+            node["children"] = [build(lo, mid, height - 1, False),
+                                build(mid, hi, height - 1, False)]
+        return at
+
+    lo = 0
+    for h in range(max(m, 1).bit_length() - 1, -1, -1):
+        if m & (1 << h):
+            build(lo, lo + (1 << h), h, True)
+            lo += 1 << h
+    return nodes
+
+
+def fsb_bound(node, q, i: int, lam: float, sigma: float) -> float:
+    """Node score U_v: an upper bound of the cell score r_ic of every leaf below the node.
+
+    [FreeSolo] "How it differs" (FS-B): U_v bounds the scores of the cells below v and justifies
+    pruning.  R21: from the four summaries, q . kbar_c <= q . mu + ||q|| rho (Cauchy-Schwarz) and,
+    with lambda >= 0 and the leaves in the query's past, a_c erf((i - p_c) / (2 sigma)) <=
+    a_max erf((i - p_min) / (2 sigma)) (erf increasing, a_c <= a_max, p_c >= p_min):
+        U_v = (q . mu + ||q|| rho) / sqrt(d) + lambda a_max erf((i - p_min) / (2 sigma)),
+    which equals r_ic at a leaf (rho = 0).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    dot = float(np.dot(q, node["mu"])) + math.sqrt(float(np.dot(q, q))) * node["rho"]
+    return dot / math.sqrt(d) + lam * node["amax"] * float(_erf((i - node["pmin"]) / (2.0 * sigma)))
+
+
+def fsb_beam(nodes, q, i: int, lam: float, sigma: float, width: int):
+    """Beam search down one forest: the cells the beam reaches, and the smallest relative gap at
+    any beam cut (how close the search came to a tie).
+
+    [FreeSolo] "How it differs" (FS-B): a beam of W_b nodes per level descends the forest, ranked by
+    U_v.  R21: level h holds the children of the previous level's beam and the roots of height h;
+    the ``width`` best of them by U_v (rounded to float32, the decision precision; larger first,
+    lower first cell on ties, NaN last) form the beam of level h; the beam of the leaf level is the
+    set of candidate cells.
+    """
+    if not nodes:
+        return [], math.inf
+    top = max(n["height"] for n in nodes)
+    beam = []
+    gap = math.inf
+    for h in range(top, -1, -1):
+        pool = [c for b in beam for c in nodes[b]["children"]]
+        pool += [j for j, n in enumerate(nodes) if n["root"] and n["height"] == h]
+        scored = [(float(round_f32(fsb_bound(nodes[j], q, i, lam, sigma))), j) for j in pool]
+        scored.sort(key=lambda x: _rank_key(x[0], nodes[x[1]]["first"]))
+        if len(scored) > width:
+            a, b = scored[width - 1][0], scored[width][0]
+            if not (math.isnan(a) or math.isnan(b)):
+                gap = min(gap, (a - b) / max(abs(a), abs(b), 1e-30))
+        beam = [j for _, j in scored[:width]]
+    return sorted(nodes[j]["first"] for j in beam), gap
+
+
+def fsb_rerank_scores(q, k, cells, cell: int) -> np.ndarray:
+    """Re-rank score of each candidate cell: log-sum-exp over the cell's tokens of the raw
+    (unrotated) logits q . k_j / sqrt(d) ([FreeSolo] "How it differs", FS-B: the reached cells are
+    re-ranked by logsumexp with their token keys)."""
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    out = []
+    for c in cells:
+        lo, hi = block_range(int(c), k.shape[0], cell)
+        z = np.asarray(k[lo:hi], dtype=np.float64) @ q / math.sqrt(d)
+        out.append(logsumexp(z))
+    return np.array(out)
+
+
+def fsb_select(q, i: int, k, summaries, cell: int, q_block: int, K: int, lam: float,
+               sigma: float, width: int):
+    """FS-B selection of the query at position i: both forests over its candidate cells, a beam of
+    ``width`` per level in each, the union of the cells reached, re-ranked by log-sum-exp over
+    their tokens, top K (larger first, lower index on ties, NaN last; R11: the re-rank score is
+    rounded to float32 before the decision).  Returns (selected cells ascending, candidate cells,
+    smallest relative gap at a beam cut or at the final top-K cut)."""
+    mean_k, max_norm, centre = summaries
+    nc = freesolo_num_candidates(i, cell, q_block)
+    if nc == 0:
+        return [], [], math.inf
+    cand = set()
+    gap = math.inf
+    for cells in (list(range(nc)), fsb_high_cells(max_norm, nc)):
+        reached, g = fsb_beam(fsb_forest(cells, mean_k, max_norm, centre), q, i, lam, sigma, width)
+        cand |= set(reached)
+        gap = min(gap, g)
+    cand = sorted(cand)
+    r = round_f32(fsb_rerank_scores(q, k, cand, cell))
+    order = sorted(range(len(cand)), key=lambda j: _rank_key(float(r[j]), cand[j]))
+    if len(cand) > K:
+        a, b = float(r[order[K - 1]]), float(r[order[K]])
+        gap = min(gap, (a - b) / max(abs(a), abs(b), 1e-30))
+    return sorted(cand[j] for j in order[:K]), cand, gap
 
 
 # ----------------------------------------------------------------------------------------------

@@ -599,6 +599,59 @@ def test_fsl_select_with_every_cell_kept_is_the_full_selection():
     assert set(got) <= set(cand) and len(got) == 4
 
 
+def test_fsl_state_update_equals_the_pruning_recomputed_from_scratch():
+    """The O(W + P) state update (one cell at a time, the cell leaving the W newest competing with
+    the lowest-ranked kept older cell) keeps exactly the set the pruning rule picks from the whole
+    prefix, after every growth step; ties and NaN norms included."""
+    rng = np.random.default_rng(42)
+    for trial in range(120):
+        total = int(rng.integers(1, 120))
+        W, P = int(rng.integers(0, 9)), int(rng.integers(0, 12))
+        a = np.round(rng.standard_normal(total) * 2) / 2  # many ties
+        if trial % 5 == 0:
+            a[rng.integers(0, total, 3)] = np.nan
+        st = orc.fsl_state_new(W, P)
+        n = 0
+        while n < total:
+            n = min(total, n + int(rng.integers(0, 6)))
+            st = orc.fsl_state_advance(st, a, n)
+            assert orc.fsl_state_cells(st) == orc.fsl_candidates(a, n, W, P), (trial, n)
+            assert len(st["older"]) <= P
+    # the state never looks past its P cells: a norm changed after a cell was dropped does not
+    # bring it back (the update reads only the joining cell and the kept ones)
+    a = np.array([5.0, 1.0, 4.0, 0.5, 0.2, 0.1])
+    st = orc.fsl_state_advance(orc.fsl_state_new(1, 2), a, 6)
+    assert orc.fsl_state_cells(st) == [0, 2, 5]
+
+
+def test_fsl_decode_row_keeping_every_cell_is_the_full_method():
+    """With W + P covering every candidate cell the FS-L decode output equals the full method's
+    two-branch output; with a pruned state its long branch reads only kept cells."""
+    rng = np.random.default_rng(43)
+    n, d, cell = 1536, 16, 32
+    q, k, v = rng.standard_normal((n, d)), rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    summ = orc.block_summaries(k, cell)
+    for i in [200, 700, 1535]:
+        nc = orc.freesolo_num_candidates(i, cell, 128)
+        st = orc.fsl_state_advance(orc.fsl_state_new(8, nc), summ[1], nc)
+        cand = orc.fsl_state_cells(st)
+        o1, sel1 = orc.fsl_decode_row(q[i], k, v, i, summ, cand, cell, 4, 256, 0.5, 300.0, 0.3,
+                                      10000.0)
+        o2, sel2 = orc.freesolo_row(q[i], k, v, i, summ, cell, 128, 4, 256, 0.5, 300.0, 0.3,
+                                    10000.0)
+        assert sel1 == sel2
+        assert np.allclose(o1, o2, atol=1e-12)
+    i = 1535
+    nc = orc.freesolo_num_candidates(i, cell, 128)
+    st = orc.fsl_state_advance(orc.fsl_state_new(2, 3), summ[1], nc)
+    cand = orc.fsl_state_cells(st)
+    o, sel = orc.fsl_decode_row(q[i], k, v, i, summ, cand, cell, 4, 256, 0.5, 300.0, 0.3, 10000.0)
+    assert set(sel) <= set(cand) and len(sel) == 4
+    o_ref, _ = orc.freesolo_row(q[i], k, v, i, summ, cell, 128, 4, 256, 0.5, 300.0, 0.3, 10000.0,
+                                selection=sel)
+    assert np.allclose(o, o_ref, atol=1e-12)
+
+
 # ------------------------------------------------------------------------------------------
 # bf16 summaries and GQA-shared selection (R19)
 # ------------------------------------------------------------------------------------------
@@ -721,3 +774,102 @@ def test_outer_gate_gradient_matches_finite_differences():
         fd = (_outer_loss(qs, k, v, positions, b, sel, up, douts)
               - _outer_loss(qs, k, v, positions, b, sel, dn, douts)) / (2 * h)
         assert abs(fd - dg[m]) < 1e-9 * max(1.0, abs(fd)), (m, fd, dg[m])
+
+
+# ------------------------------------------------------------------------------------------
+# FS-B forests and beam search (R21)
+# ------------------------------------------------------------------------------------------
+
+
+def test_fsb_forest_structure_and_node_summaries():
+    """Trees per set bit of the cell count, largest first; a node's mean key is the mean of the
+    raw keys below it (cells are full), its radius the largest leaf distance (brute force), its
+    maximum norm and minimum position those of its leaves."""
+    rng = np.random.default_rng(50)
+    n, d, cell = 64 * 23, 8, 64
+    k = rng.standard_normal((n, d))
+    mean_k, max_norm, centre = orc.block_summaries(k, cell)
+    for m in [1, 2, 3, 7, 8, 13, 23]:
+        cells = list(range(m))
+        nodes = orc.fsb_forest(cells, mean_k, max_norm, centre)
+        roots = [(x["lo"], x["hi"]) for x in nodes if x["root"]]
+        sizes = [1 << h for h in range(m.bit_length() - 1, -1, -1) if m & (1 << h)]
+        assert [hi - lo for lo, hi in roots] == sizes
+        assert roots[0][0] == 0 and all(a[1] == b[0] for a, b in zip(roots, roots[1:]))
+        assert len(nodes) == sum(2 * s - 1 for s in sizes)
+        for x in nodes:
+            lo, hi = x["lo"], x["hi"]
+            assert hi - lo == 1 << x["height"]
+            toks = k[lo * cell:hi * cell]
+            assert np.allclose(x["mu"], toks.mean(0), atol=1e-12)
+            dist = np.linalg.norm(mean_k[lo:hi] - x["mu"], axis=1)
+            assert abs(x["rho"] - (dist.max() if hi - lo > 1 else 0.0)) < 1e-12
+            assert x["amax"] == max_norm[lo:hi].max() and x["pmin"] == centre[lo]
+            if x["children"]:
+                a, b = (nodes[j] for j in x["children"])
+                assert (a["lo"], a["hi"], b["lo"], b["hi"]) == (lo, (lo + hi) // 2, (lo + hi) // 2, hi)
+
+
+def test_fsb_node_bound_dominates_every_leaf_score():
+    """U_v >= r_ic for every cell below v (equality at the leaves), for random queries, both
+    forests, lambda > 0."""
+    rng = np.random.default_rng(51)
+    n, d, cell = 32 * 100, 16, 32
+    k = rng.standard_normal((n, d)) * rng.uniform(0.5, 2.0, (n, 1))
+    mean_k, max_norm, centre = orc.block_summaries(k, cell)
+    for trial in range(6):
+        q = rng.standard_normal(d) * 2
+        i = int(rng.integers(100 * 32 - 200, 100 * 32))
+        lam, sig = float(rng.uniform(0.1, 2.0)), float(rng.uniform(50, 3000))
+        nc = orc.freesolo_num_candidates(i, cell, 128)
+        r = orc.freesolo_scores(q, i, mean_k, max_norm, centre, lam, sig, nc)
+        for cells in (list(range(nc)), orc.fsb_high_cells(max_norm, nc)):
+            nodes = orc.fsb_forest(cells, mean_k, max_norm, centre)
+            for x in nodes:
+                below = cells[x["lo"]:x["hi"]]
+                u = orc.fsb_bound(x, q, i, lam, sig)
+                assert u >= max(r[c] for c in below) - 1e-12
+                if x["height"] == 0:
+                    assert abs(u - r[below[0]]) < 1e-12
+
+
+def test_fsb_high_cells_are_those_at_or_above_the_median():
+    rng = np.random.default_rng(52)
+    for nc in [1, 2, 9, 10, 101, 400]:
+        a = rng.standard_normal(500)
+        got = orc.fsb_high_cells(a, nc)
+        assert got == sorted(c for c in range(nc) if a[c] >= np.median(a[:nc]))
+        assert len(got) == (nc + 1) // 2
+
+
+def test_fsb_rerank_is_the_cells_log_sum_exp():
+    rng = np.random.default_rng(53)
+    n, d, cell = 32 * 20, 16, 32
+    k, q = rng.standard_normal((n, d)), rng.standard_normal(d)
+    cells = [0, 3, 19]
+    got = orc.fsb_rerank_scores(q, k, cells, cell)
+    for j, c in enumerate(cells):
+        z = torch.as_tensor(k[c * cell:(c + 1) * cell]) @ torch.as_tensor(q) / math.sqrt(d)
+        assert abs(got[j] - float(torch.logsumexp(z, 0))) < 1e-12
+
+
+def test_fsb_beam_as_wide_as_the_forest_is_the_exhaustive_rerank():
+    """A beam at least as wide as the cell count keeps every cell at every level, so the
+    selection is the top K of the log-sum-exp re-rank over every candidate cell (full sort)."""
+    rng = np.random.default_rng(54)
+    n, d, cell = 32 * 64, 16, 32
+    k = rng.standard_normal((n, d))
+    summ = orc.block_summaries(k, cell)
+    for i in [600, 1300, 2047]:
+        q = rng.standard_normal(d)
+        nc = orc.freesolo_num_candidates(i, cell, 128)
+        sel, cand, _ = orc.fsb_select(q, i, k, summ, cell, 128, 4, 0.5, 300.0, width=nc)
+        assert cand == list(range(nc))
+        lse = [float(torch.logsumexp(torch.as_tensor(k[c * cell:(c + 1) * cell]) @
+                                     torch.as_tensor(q) / math.sqrt(d), 0)) for c in range(nc)]
+        want = sorted(sorted(range(nc), key=lambda c: (-lse[c], c))[:4])
+        assert sel == want
+    # a narrow beam reaches at most 2 x width cells and selects among them
+    q = rng.standard_normal(d)
+    sel, cand, _ = orc.fsb_select(q, 2047, k, summ, cell, 128, 4, 0.5, 300.0, width=2)
+    assert len(cand) <= 4 and set(sel) <= set(cand)
