@@ -52,12 +52,7 @@ WORKLOADS = {
 # profile summary under profiles/).  Reported only while the source is unchanged.
 # The hash covers the device code of the source: the file up to its first host function
 # (`device_end`), so a change of the host-side launcher alone keeps the figure.
-MEASURED_TRAFFIC = {
-    ("sas_gqa_decode_32k", "decode_fused_kernel"): {
-        "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "655f3f3d4f809aee",
-        "bytes": 52_592_384 + 344_320},
-}
+MEASURED_TRAFFIC = {}
 
 
 def device_source_hash(path: str, device_end: str) -> str:

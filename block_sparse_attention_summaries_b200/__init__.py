@@ -51,6 +51,13 @@ SIGNATURES = [
     ("bsa_fsl_prune", _I, [_P, _I, _I, _P, _I, _I, _P, _P, _P]),
     ("bsa_fsl_select", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _P,
                             _P, _P]),
+    ("bsa_fsl_state_update", _I, [_P, _I, _I, _P, _I, _I, _P, _P, _P, _P, _P, _P]),
+    ("bsa_fsl_decode", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P,
+                            _P, _I, _I, _I, ctypes.c_float, _P, _P, _P, _P, _P]),
+    ("bsa_fsb_forest_bytes", _Z, [_I, _I, _I, _I]),
+    ("bsa_fsb_build", _I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _Z, _P]),
+    ("bsa_fsb_select", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _Z, _P, _P, _I, _I, _P, _P, _P,
+                            _P]),
     ("bsa_freesolo_select", _I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _P,
                                  _P, _Z, _P]),
     ("bsa_freesolo_select_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
@@ -328,6 +335,90 @@ def fsl_prune(max_norm, n_cells, W, P):
     _check(lib().bsa_fsl_prune(_ptr(max_norm), rows, C, _ptr(_i32(n_cells)), W, P, _ptr(cand),
                                _ptr(cnt), _stream(max_norm.device)), "bsa_fsl_prune")
     return cand, cnt
+
+
+class FslState:
+    """FS-L fixed-size state of ``rows`` (batch x head) rows: the P kept older cells per row, their
+    count and the candidate cells covered (device tensors, zero = empty), plus the kept-cell list
+    the last update wrote (bsa_fsl_state_update)."""
+
+    def __init__(self, rows, W, P, device):
+        self.W, self.P = W, P
+        self.older = torch.full((rows, P), -1, dtype=torch.int32, device=device)
+        self.older_count = torch.zeros(rows, dtype=torch.int32, device=device)
+        self.state_cells = torch.zeros(rows, dtype=torch.int32, device=device)
+        self.cand = torch.full((rows, W + P), -1, dtype=torch.int32, device=device)
+        self.cand_count = torch.zeros(rows, dtype=torch.int32, device=device)
+
+    def update(self, max_norm, n_cells):
+        """Grow every row's candidate prefix to n_cells [rows] (int32): returns (cand, count)."""
+        _cuda(max_norm, n_cells)
+        rows = self.older.shape[0]
+        C = max_norm.shape[-1]
+        _check(lib().bsa_fsl_state_update(_ptr(max_norm), rows, C, _ptr(_i32(n_cells)), self.W,
+                                          self.P, _ptr(self.older), _ptr(self.older_count),
+                                          _ptr(self.state_cells), _ptr(self.cand),
+                                          _ptr(self.cand_count), _stream(max_norm.device)),
+               "bsa_fsl_state_update")
+        return self.cand, self.cand_count
+
+
+def fsl_decode(q, k, v, pos, cell, mean_k, max_norm, centre, lambda_h, sigma_h, alpha_h, cand,
+               cand_count, K, window=512, rope_theta=10000.0, o=None, idx=None, count=None,
+               status=None):
+    """FS-L decode output (bsa_fsl_decode): q [B, H, d], k/v [B, H, n, d], pos [B] int32.
+    Returns (o, idx, count)."""
+    _cuda(q, k, v, pos, mean_k, max_norm, centre, lambda_h, sigma_h, alpha_h, cand, cand_count,
+          o, idx, count, status)
+    B, H, n, d = k.shape
+    if o is None:
+        o = torch.empty(B, H, d, device=q.device, dtype=q.dtype)
+    if idx is None:
+        idx = torch.empty(B, H, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, H, device=q.device, dtype=torch.int32)
+    _check(lib().bsa_fsl_decode(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, H, n, d,
+                                _ptr(_i32(pos)), cell, _ptr(mean_k), _ptr(max_norm),
+                                _ptr(centre), _ptr(lambda_h), _ptr(sigma_h), _ptr(alpha_h),
+                                _ptr(_i32(cand)), _ptr(_i32(cand_count)), cand.shape[-1], K,
+                                window, float(rope_theta), _ptr(o), _ptr(idx), _ptr(count),
+                                _ptr(status), _stream(q.device)), "bsa_fsl_decode")
+    return o, idx, count
+
+
+def fsb_build(mean_k, max_norm, centre, n_cells, forest=None):
+    """Both FS-B forests of every (batch, head) row for its prefix of n_cells [B * H] cells
+    (bsa_fsb_build); returns the forest buffer."""
+    _cuda(mean_k, max_norm, centre, n_cells, forest)
+    B, H, C, d = mean_k.shape
+    nbytes = int(lib().bsa_fsb_forest_bytes(B, H, C, d))
+    if nbytes == 0:
+        raise BsaError(4, "bsa_fsb_forest_bytes")
+    if forest is None:
+        forest = torch.empty(nbytes, dtype=torch.uint8, device=mean_k.device)
+    _check(lib().bsa_fsb_build(_ptr(mean_k), _ptr(max_norm), _ptr(centre), B, H, C, d,
+                               _ptr(_i32(n_cells)), _ptr(forest), forest.numel(),
+                               _stream(mean_k.device)), "bsa_fsb_build")
+    return forest
+
+
+def fsb_select(q, k, pos, cell, forest, lambda_h, sigma_h, width, K, idx=None, count=None,
+               lse=None):
+    """FS-B selection of one query per (batch, head) (bsa_fsb_select): q [B, H, d], k [B, H, n, d];
+    returns (idx [B, H, K], count [B, H], lse [B, H, K])."""
+    _cuda(q, k, pos, forest, lambda_h, sigma_h, idx, count, lse)
+    B, H, n, d = k.shape
+    if idx is None:
+        idx = torch.empty(B, H, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, H, device=q.device, dtype=torch.int32)
+    if lse is None:
+        lse = torch.empty(B, H, K, device=q.device, dtype=torch.float32)
+    _check(lib().bsa_fsb_select(_ptr(q), _ptr(k), _dtype_code(q), B, H, n, d, _ptr(_i32(pos)),
+                                cell, _ptr(forest), forest.numel(), _ptr(lambda_h),
+                                _ptr(sigma_h), width, K, _ptr(idx), _ptr(count), _ptr(lse),
+                                _stream(q.device)), "bsa_fsb_select")
+    return idx, count, lse
 
 
 def fsl_select(q, pos, mean_k, max_norm, centre, lambda_h, sigma_h, cand, cand_count, K):

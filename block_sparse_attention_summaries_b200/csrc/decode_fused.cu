@@ -9,23 +9,31 @@
 // B200 design.  The step is HBM-bound (summaries + selected K/V) and short (~10 us), so launch
 // boundaries, global round trips and serial latency chains cost as much as the bytes.  The CL
 // CTAs of a cluster (CL <= 16) cooperate through distributed shared memory (DSMEM):
-//   1. CTA r scores its slice of the history blocks: the mean-key rows stream through a
-//      two-stage shared-memory ring filled by bulk copies (TMA engine); the G query heads of the
-//      group share every row (one 31-shuffle transpose-reduce per 32/G rows).  Per head, a warp
-//      selects the slice's local Top-K (bisection on order-preserving keys with warp reductions)
-//      and PUSHES the candidates into every peer's merge buffer with DSMEM stores.
-//   2. cluster barrier; each CTA selects the global Top-K per head from its own merge buffer
-//      (same exact order everywhere: larger score, then lower index) and builds the sorted union
-//      of the G heads' selections (a bitmap over the history blocks, compacted by one warp), plus
-//      the current block, with a head mask per entry.
-//   3. CTA r attends union entries r, r+CL, ...  bf16: each K/V block arrives as 128-byte swizzled
-//      64x64 TMA tiles; two groups of four warps take alternate entries; a warp owns 16 tokens of
-//      a block and computes S = Q K^T and O += P V with warp-level MMAs (the G heads padded to 16
-//      rows), keeping its own online-softmax state, so the per-block work is ~30 MMAs per warp
-//      instead of ~1,200 scalar FMAs/shuffles.  fp32: the same split with scalar FMAs.  The CTA
-//      holding the current block also rewrites that block's summary from shared memory.
-//   4. Each CTA merges its warps, then pushes to CTA r' the partial (m, l, o) of the output columns
+//   1. CTA r scores its slice of the history blocks.  Its mean-key rows stream through a ring of
+//      shared-memory stages filled by bulk copies (TMA engine), every stage issued at the start
+//      (refilled as they drain when the slice is larger than the ring); the G query heads of the
+//      group share every row (one 31-shuffle transpose-reduce per 32/G rows).
+//   2. Selection.  When the history fits one warp select (<= 512 blocks) every CTA pushes its
+//      slice's order keys into every peer's copy of the whole row (DSMEM vector stores), and after
+//      one cluster barrier each CTA selects every head's Top-K from the whole row itself.  Longer
+//      histories select a local Top-K per slice and merge the CL x K candidates the same way.
+//      The warp select takes the K-th largest of 64 group maxima as a threshold (at least K keys
+//      lie at or above it), compacts the keys at or above it in index order and ranks them
+//      exactly; a radix select with 4-bit digits is the fallback when too many keys pass.
+//   3. Each CTA builds the sorted union of the G heads' selections (a bitmap over the history
+//      blocks, compacted by one warp) plus the current block, with a head mask per entry.
+//   4. bf16, 64-token blocks: the union's tokens are cut into 16-token slices and every CTA of
+//      the cluster takes an equal contiguous range of them; slices arrive as 128-byte swizzled
+//      16-row TMA boxes, four slices per stage, through a ring of stages; one group of four warps
+//      takes a stage, each warp one slice, and computes S = Q K^T and O += P V with warp-level
+//      MMAs (the G heads padded to 16 rows) with its own online-softmax state, so the per-slice
+//      work is ~30 MMAs per warp instead of ~1,200 scalar FMAs/shuffles.  Other block sizes and
+//      fp32: CTA r attends union entries r, r+CL, ... with scalar FMAs, the CTA holding the
+//      current block rewriting that block's summary from shared memory.
+//   5. Each CTA merges its warps, then pushes to CTA r' the partial (m, l, o) of the output columns
 //      CTA r' owns; cluster barrier; each CTA finishes its columns and writes o (and lse).
+// On the 64-token bf16 path the summary of the block being filled is rewritten by the last CTA of
+// the cluster from global memory at the start, while its first summary stages are in flight.
 // Variants (flags of bsa_decode_step_ex): shared selection -- the group's score of a block is the
 // mean of its G heads' scores, ranked once and attended by every head (one selection per kv
 // head instead of G); bf16 summaries -- the mean keys are read (and appended) in bf16, halving the
@@ -50,6 +58,11 @@ constexpr int kMaxKf = 32;        // Top-K bound of the fused path
 constexpr int kMaxUnion = 8 * kMaxKf + 1;
 constexpr int kMaxWords = 512;    // history bitmap words: C <= 16384
 constexpr int kSub = 64;          // summary rows per ring stage
+constexpr int kSelItems = 16;     // keys per lane of one warp select: N <= 512
+constexpr int kSelMax = 32 * kSelItems;
+constexpr int kCandMax = 64;      // candidates the threshold pass may leave for exact ranking
+constexpr int kMaxStages = 8;     // ring stages (summaries or K/V)
+constexpr int kSlice = 16;        // tokens per warp slice (64-token bf16 path)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.f;   // lazy rescale threshold (log2 units)
@@ -72,8 +85,14 @@ struct FusedParams {
   int* idx;
   int* count;
   int* status;
-  int chunk;  // history blocks scored per CTA (multiple of kSub)
+  int chunk;   // history blocks scored per CTA (multiple of kSub)
   int shared;  // one selection per kv head from the mean of its heads' scores
+  int gather;  // whole-row selection (history <= kSelMax blocks) instead of local + merge
+  int row_ld;  // stride of the whole-row key copies (gather) in keys
+  int ns;      // summary ring stages
+  int nkv;     // K/V ring stages
+  // dynamic shared-memory layout (byte offsets from the 1024-aligned base)
+  int off_keys, off_sel, off_recv, off_zp, off_bar;
 };
 
 // ---- cluster helpers ---------------------------------------------------------------------
@@ -88,6 +107,12 @@ __device__ __forceinline__ uint32_t cluster_size() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
@@ -100,6 +125,11 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
 __device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -111,17 +141,9 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Top-K of N order keys (shared memory, index order) by one warp: an exact radix select with
-// 4-bit digits.  The keys sit in registers (lane l holds positions l + 32 j).  Each pass counts
-// the next digit of the keys that share the prefix found so far: every lane keeps sixteen 4-bit
-// counters in one 64-bit word (at most 8 keys between two flushes into 16-bit fields), the eight
-// 32-bit words of 16-bit bins are summed over the warp, and the pass keeps the digit at which the
-// count of keys at or above the threshold reaches K.  It stops as soon as that count is exactly K
-// ({key >= T} is then the answer); otherwise after the last digit T is the K-th largest key and
-// the lowest-indexed keys equal to T fill the remaining places.
-// Writes the selected positions ascending to `out`; returns min(K, N).  Up to 64 keys an exact
-// rank count (below) is cheaper than the radix passes.
-constexpr int kSelItems = 16;  // N <= 32 * kSelItems
+// ---- warp Top-K selection -------------------------------------------------------------------
+// All selections rank order keys (larger first) and break ties toward the lower position; the
+// positions of the winners are written ascending.
 
 // count of digit d in the reduced words: parity p = d & 1 picks words 4p.., the byte k = d >> 1
 // of the nibble-split word sits in b[k & 1] as 16-bit field k >> 1 (see flush_nibbles)
@@ -141,8 +163,8 @@ __device__ __forceinline__ void flush_nibbles(uint64_t a, uint32_t (&r)[8]) {
   }
 }
 
-// Small N (<= 32 R): rank every key by counting the keys above it (ties: the lower position
-// ranks higher) and keep ranks below K -- N broadcast loads per lane, no passes.
+// Exact rank select over N <= 32 R keys: rank every key by counting the keys above it (ties: the
+// lower position ranks higher) and keep ranks below kk -- N broadcast loads per lane.
 template <int R>
 __device__ __forceinline__ int warp_select_rank(const uint32_t* keys, int N, int kk, int lane,
                                                 int* out) {
@@ -153,6 +175,7 @@ __device__ __forceinline__ int warp_select_rank(const uint32_t* keys, int N, int
     mk[q] = lane + 32 * q < N ? keys[lane + 32 * q] : 0u;
     rk[q] = 0;
   }
+#pragma unroll 4
   for (int j = 0; j < N; ++j) {
     const uint32_t kj = keys[j];
 #pragma unroll
@@ -171,15 +194,15 @@ __device__ __forceinline__ int warp_select_rank(const uint32_t* keys, int N, int
   return taken;
 }
 
-__device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out) {
-  const int kk = min(K, N);
-  if (kk <= 0) return 0;
-  if (kk == N) {
-    for (int i = lane; i < N; i += 32) out[i] = i;
-    __syncwarp();
-    return N;
-  }
-  if (N <= 64) return warp_select_rank<2>(keys, N, kk, lane, out);
+// Exact radix select with 4-bit digits (lane l holds positions l + 32 j in registers).
+// Each pass counts the next digit of the keys that share the prefix found so far: every lane keeps
+// sixteen 4-bit counters in one 64-bit word (at most 8 keys between two flushes into 16-bit
+// fields), the eight 32-bit words of 16-bit bins are summed over the warp, and the pass keeps the
+// digit at which the count of keys at or above the threshold reaches K.  It stops as soon as that
+// count is exactly K ({key >= T} is then the answer); otherwise after the last digit T is the K-th
+// largest key and the lowest-indexed keys equal to T fill the remaining places.
+__device__ __noinline__ int warp_select_radix(const uint32_t* keys, int N, int kk, int lane,
+                                              int* out) {
   const int nv = (N - lane + 31) >> 5;  // keys of this lane: positions lane + 32 j, j < nv
   uint32_t kr[kSelItems];
 #pragma unroll
@@ -250,6 +273,98 @@ __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int 
   return taken;
 }
 
+// Top-min(K, N) of N <= kSelMax order keys (shared memory, index order) by one warp; writes the
+// winners' positions ascending to `out`, returns their number.  `ck` / `cp` are the warp's
+// scratch for kCandMax candidate keys / positions.
+//
+// Threshold pass: lane l holds positions l + 32 j; the even-j and odd-j keys of every lane form 64
+// groups.  T0 = the kk-th largest group maximum: the kk groups whose maxima reach T0 hold kk
+// distinct keys >= T0, so every key of the Top-kk is >= T0.  The keys >= T0 are compacted in
+// position order (usually a few more than kk) and ranked exactly; if more than kCandMax pass, the
+// radix select runs on all N keys instead.
+__device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out,
+                                        uint32_t* ck, int* cp) {
+  const int kk = min(K, N);
+  if (kk <= 0) return 0;
+  if (kk == N) {
+    for (int i = lane; i < N; i += 32) out[i] = i;
+    __syncwarp();
+    return N;
+  }
+  if (N <= kCandMax) return warp_select_rank<kCandMax / 32>(keys, N, kk, lane, out);
+  const int nv = (N - lane + 31) >> 5;  // keys of this lane: positions lane + 32 j, j < nv
+  uint32_t kr[kSelItems];
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) kr[j] = j < nv ? keys[lane + 32 * j] : 0u;
+  uint32_t g0 = 0u, g1 = 0u;  // group maxima (even j, odd j)
+#pragma unroll
+  for (int j = 0; j < kSelItems; j += 2) {
+    g0 = max(g0, kr[j]);
+    g1 = max(g1, kr[j + 1]);
+  }
+  // rank of each group maximum among the 64 (ties: lower group id ranks higher); the one of rank
+  // kk - 1 is T0
+  int r0 = 0, r1 = 0;
+#pragma unroll 8
+  for (int src = 0; src < 32; ++src) {
+    const uint32_t a0 = __shfl_sync(0xffffffffu, g0, src);
+    const uint32_t a1 = __shfl_sync(0xffffffffu, g1, src);
+    // group ids: 2 * lane (even) and 2 * lane + 1 (odd)
+    r0 += (a0 > g0 || (a0 == g0 && src < lane)) + (a1 > g0 || (a1 == g0 && src < lane));
+    r1 += (a0 > g1 || (a0 == g1 && src <= lane)) + (a1 > g1 || (a1 == g1 && src < lane));
+  }
+  const unsigned h0 = __ballot_sync(0xffffffffu, r0 == kk - 1);
+  const unsigned h1 = __ballot_sync(0xffffffffu, r1 == kk - 1);
+  const uint32_t T0 = h0 ? __shfl_sync(0xffffffffu, g0, __ffs(h0) - 1)
+                         : __shfl_sync(0xffffffffu, g1, __ffs(h1) - 1);
+  int cnt = 0;
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) cnt += (j < nv && kr[j] >= T0) ? 1 : 0;
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (cnt > kCandMax) return warp_select_radix(keys, N, kk, lane, out);
+  // compact the candidates in position order (position 32 j + lane grows with (j, lane))
+  const unsigned lt = (1u << lane) - 1u;
+  int base = 0;
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) {
+    if (32 * j >= N) break;  // warp-uniform
+    const bool c = j < nv && kr[j] >= T0;
+    const unsigned bal = __ballot_sync(0xffffffffu, c);
+    if (c) {
+      ck[base + __popc(bal & lt)] = kr[j];
+      cp[base + __popc(bal & lt)] = 32 * j + lane;
+    }
+    base += __popc(bal);
+  }
+  __syncwarp();
+  // rank the candidates; the winners keep the candidates' (ascending) position order
+  uint32_t mk[2];
+  int rk[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    mk[q] = lane + 32 * q < cnt ? ck[lane + 32 * q] : 0u;
+    rk[q] = 0;
+  }
+#pragma unroll 4
+  for (int j = 0; j < cnt; ++j) {
+    const uint32_t kj = ck[j];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) rk[q] += (kj > mk[q] || (kj == mk[q] && j < lane + 32 * q)) ? 1 : 0;
+  }
+  int taken = 0;
+  int mypos[2] = {lane < cnt ? cp[lane] : 0, lane + 32 < cnt ? cp[lane + 32] : 0};
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const bool take = lane + 32 * q < cnt && rk[q] < kk;
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) out[taken + __popc(tb & lt)] = mypos[q];
+    taken += __popc(tb);
+  }
+  __syncwarp();
+  return taken;
+}
+
 // ---- warp MMA (legacy mma.sync, bf16 in, fp32 accumulate) ---------------------------------
 __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -270,28 +385,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Shared-memory layout (dynamic part).  MMA: the bf16 warp-MMA path over 64-token blocks.
-template <typename T, int D, int G, bool MMA>
+// Byte sizes of the pieces of the dynamic shared memory (host and device agree through them).
+template <typename T, typename TS, int D, int G, bool MMA>
 struct FusedSmem {
-  // region A: summary ring (2 x kSub x D fp32) / K,V stages (2 x {K,V} tile) / warp partials
-  __host__ __device__ static size_t tile(int b) {
+  // one K/V stage: four 16-token slices (MMA) or one whole block (scalar path), K then V
+  __host__ __device__ static size_t kv_tile(int b) {
     return align_up((size_t)(MMA ? 64 : b) * D * sizeof(T), 1024);
   }
-  __host__ __device__ static size_t region_a(int b) {
-    size_t x = (size_t)2 * kSub * D * sizeof(float);
-    x = max_sz(x, 4 * tile(b));
-    x = max_sz(x, (size_t)kWarps * G * (D + 2) * 4 + 4096);  // warp partials
-    return align_up(x, 1024);
+  __host__ __device__ static size_t kv_stage(int b) { return 2 * kv_tile(b); }
+  __host__ __device__ static size_t sum_stage() { return (size_t)kSub * D * sizeof(TS); }
+  __host__ __device__ static size_t partials() {
+    return align_up((size_t)kWarps * G * (D + 2) * 4, 1024);
   }
-  __host__ __device__ static size_t scores(int chunk) { return align_up((size_t)G * chunk * 4, 16); }
-  __host__ __device__ static size_t merge(int CL, int K) { return align_up((size_t)G * CL * K * 8, 16); }
+  __host__ __device__ static size_t keys(int chunk) { return align_up((size_t)G * chunk * 4, 16); }
+  __host__ __device__ static size_t sel(int gather, int row_ld, int CL, int K) {
+    return gather ? align_up((size_t)G * row_ld * 4, 16) : align_up((size_t)G * CL * K * 8, 16);
+  }
   __host__ __device__ static size_t recv(int CL) {
     return align_up((size_t)CL * G * (D / CL + 2) * 4, 16);
   }
-  __host__ __device__ static size_t zp(int b) { return 2 * align_up((size_t)b * G * 4, 16); }
-  __host__ __device__ static size_t bytes(int b, int chunk, int CL, int K) {
-    return region_a(b) + scores(chunk) + merge(CL, K) + recv(CL) + zp(b) + 256 + 1024;
-  }
+  __host__ __device__ static size_t zp(int b) { return MMA ? 0 : 2 * align_up((size_t)b * G * 4, 16); }
 };
 
 template <typename T, typename TS, int D, int G, bool MMA>
@@ -306,16 +419,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ int s_pick[G][kMaxKf];
+  __shared__ int s_pick[kWarps][kMaxKf];
   __shared__ int s_sel[G][kMaxKf];
   __shared__ int s_nsel[G];
   __shared__ uint32_t s_bits[kMaxWords];
   __shared__ int s_ublk[kMaxUnion];
   __shared__ unsigned s_umask[kMaxUnion];
+  __shared__ uint32_t s_scratch[kWarps * 2 * kCandMax];  // select candidates / append partials
+  __shared__ int s_kv_last[kMaxStages];  // the last K/V stage issued into each slot (-1: none)
   __shared__ int s_U;
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
+  static_assert(kWarps * 2 * kCandMax >= kWarps * 128, "append partials fit the scratch");
 
   const int b = p.b, K = p.K, Hq = p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -328,25 +444,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int cur = pos / b;
   int nc = p.prefix_block > 0 ? ((pos / p.prefix_block) * p.prefix_block) / b : cur;
   nc = max(0, min(nc, cur));
+  const int NS = p.ns, NKV = p.nkv;
 
-  using SM = FusedSmem<T, D, G, MMA>;
-  TS* ring = reinterpret_cast<TS*>(smem);  // fits: region A holds 2 x kSub fp32 rows
+  using SM = FusedSmem<T, TS, D, G, MMA>;
+  TS* ring = reinterpret_cast<TS*>(smem);  // region A: summary ring, then K/V ring, then partials
   TS* mean_k = static_cast<TS*>(p.mean_k);
   const int Gs = p.shared ? 1 : G;  // selections made per group
-  unsigned char* after_a = smem + SM::region_a(b);
-  uint32_t* s_keys = reinterpret_cast<uint32_t*>(after_a);                  // [G][chunk]
-  unsigned char* merge = after_a + SM::scores(p.chunk);                        // [G][CL*K] x 2
-  uint32_t* m_key = reinterpret_cast<uint32_t*>(merge);
-  int* m_idx = reinterpret_cast<int*>(merge) + G * CL * K;
-  float* recv = reinterpret_cast<float*>(merge + SM::merge(CL, K));          // [CL][G][cols+2]
-  float* zs = reinterpret_cast<float*>(merge + SM::merge(CL, K) + SM::recv(CL));
+  uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);  // [G][chunk]
+  uint32_t* sel_buf = reinterpret_cast<uint32_t*>(smem + p.off_sel);  // whole rows / merge
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);           // [CL][G][cols+2]
+  float* zs = reinterpret_cast<float*>(smem + p.off_zp);
   float* ps = zs + align_up((size_t)b * G, 4);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(merge + SM::merge(CL, K) + SM::recv(CL) + SM::zp(b));
-  // bar[0], bar[1]: summary ring; bar[2], bar[3]: K/V stages
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+  // bar[0 .. NS): summary stages; bar[NS .. NS + NKV): K/V stages
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
+    for (int i = 0; i < kMaxStages; ++i) s_kv_last[i] = -1;
     s_abort = 0;
     s_U = 0;
   }
@@ -355,17 +470,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     s_l[tid] = 0.f;
   }
   __syncthreads();
+  // every CTA of the cluster has started before any peer writes into its shared memory
+  cluster_arrive_relaxed();
 
   // ---- 1. score my slice of the history blocks --------------------------------------------
-  float qv[G][EPL];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float tmp[EPL];
-    load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + g) * D + lane * EPL,
-                     tmp);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
-  }
   const int c_lo = min(nc, rank * p.chunk);
   const int c_hi = min(nc, c_lo + p.chunk);
   const int rows = c_hi - c_lo;
@@ -375,22 +483,74 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const int r0 = c_lo + j * kSub;
     const int nr = min(kSub, c_hi - r0);
     const uint32_t bytes = (uint32_t)(nr * D * sizeof(TS));
-    mbar_arrive_expect_tx(&bar[j & 1], bytes);
-    bulk_g2s(ring + (size_t)(j & 1) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j & 1]);
+    mbar_arrive_expect_tx(&bar[j % NS], bytes);
+    bulk_g2s(ring + (size_t)(j % NS) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j % NS]);
   };
+  int sub_issued = 0;  // (thread 0) summary stages issued so far
   if (tid == 0)
-    for (int j = 0; j < min(nsub, 2); ++j) issue_sub(j);
+    for (; sub_issued < min(nsub, NS); ++sub_issued) issue_sub(sub_issued);
+  float qv[G][EPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float tmp[EPL];
+    load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + g) * D + lane * EPL,
+                     tmp);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
+  }
+  if constexpr (kMma) {
+    // the block being filled: its summary is rewritten from its keys (global memory) by the last
+    // CTA while the first summary stages are in flight
+    if (p.append && rank == CL - 1) {
+      const int tok = pos - cur * b + 1;
+      const T* kb = static_cast<const T*>(p.k) + ((size_t)(bi * p.Hk + kh) * p.n + (size_t)cur * b) * D;
+      float cs[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cs[e] = 0.f;
+      float nmax = 0.f;
+      for (int t = warp; t < tok; t += kWarps) {
+        float x[EPL];
+        load_vec<T, EPL>(kb + (size_t)t * D + lane * EPL, x);
+        float sq = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          cs[e] += x[e];
+          sq = fmaf(x[e], x[e], sq);
+        }
+        nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
+      }
+      float* part = reinterpret_cast<float*>(s_scratch);  // [kWarps][D]
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) part[warp * D + lane * EPL + e] = cs[e];
+      if (lane == 0) s_red[warp] = nmax;
+      __syncthreads();
+      const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+      for (int col = tid; col < D; col += kThreads) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += part[w * D + col];
+        mean_k[row * D + col] = Elem<TS>::from_f(sum / (float)tok);
+      }
+      if (tid == 0) {
+        float nm = 0.f;
+        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
+        if (p.max_norm) p.max_norm[row] = nm;
+        if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
+      }
+      __syncthreads();
+    }
+  }
   const float scale = rsqrtf((float)D);
   const int my_r = lane / G, my_g = lane % G;
   const float lam_h = p.lam ? p.lam[h0 + my_g] : 0.f;
   const float inv2sig = p.lam ? 0.5f / p.sig[h0 + my_g] : 0.f;
   for (int j = 0; j < nsub; ++j) {
-    if (!s_abort && !mbar_wait_bounded(&bar[j & 1], (j >> 1) & 1)) s_abort = 1;
+    if (!s_abort && !mbar_wait_bounded(&bar[j % NS], (j / NS) & 1)) s_abort = 1;
     __syncthreads();
     if (!s_abort) {
       const int r0 = j * kSub;
       const int nr = min(kSub, rows - r0);
-      const TS* base = ring + (size_t)(j & 1) * kSub * D;
+      const TS* base = ring + (size_t)(j % NS) * kSub * D;
       for (int t0 = warp * R; t0 < nr; t0 += kWarps * R) {
         float a[32];
 #pragma unroll
@@ -425,53 +585,94 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         if (t < nr && my_g < Gs) s_keys[my_g * p.chunk + r0 + t] = order_key(s);
       }
     }
-    __syncthreads();
-    if (tid == 0 && j + 2 < nsub && !s_abort) issue_sub(j + 2);
-  }
-  // local Top-K per head (per group when shared), pushed into every CTA's merge buffer at slot
-  // rank*K
-  for (int g = warp; g < Gs; g += kWarps) {
-    const uint32_t* keys = s_keys + g * p.chunk;
-    const int cnt = warp_select(keys, rows, K, lane, s_pick[g]);
-    for (int e = lane; e < CL * K; e += 32) {
-      const int r = e / K, j = e % K;
-      const uint32_t key = j < cnt ? keys[s_pick[g][j]] : 0u;
-      const int gi = j < cnt ? c_lo + s_pick[g][j] : -1;  // -1: empty slot
-      const int slot = g * CL * K + rank * K + j;
-      st_dsmem_u32(dsmem_addr(&m_key[slot], r), key);
-      st_dsmem_u32(dsmem_addr(&m_idx[slot], r), (uint32_t)gi);
+    if (j + NS < nsub) {  // the stage is drained: refill it
+      __syncthreads();
+      if (tid == 0 && !s_abort) issue_sub(sub_issued++);
     }
-  }
-  cluster_sync();
-
-  // ---- 2. global Top-K per head, then the union -------------------------------------------
-  const int nwords = (nc + 31) / 32;
-  for (int w = tid; w < nwords; w += kThreads) s_bits[w] = 0u;
-  for (int g = warp; g < Gs; g += kWarps) {
-    // empty slots carry key 0 and index -1: compact the valid ones first (index order kept)
-    uint32_t* mk_g = m_key + g * CL * K;
-    int* mi_g = m_idx + g * CL * K;
-    int nvalid = 0;
-    for (int e0 = 0; e0 < CL * K; e0 += 32) {
-      const int e = e0 + lane;
-      const bool ok = e < CL * K && mi_g[e] >= 0;
-      const uint32_t kk2 = ok ? mk_g[e] : 0u;
-      const int ii = ok ? mi_g[e] : 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, ok);
-      __syncwarp();
-      if (ok) {
-        const int at = nvalid + __popc(bal & ((1u << lane) - 1u));
-        mk_g[at] = kk2;
-        mi_g[at] = ii;
-      }
-      nvalid += __popc(bal);
-      __syncwarp();
-    }
-    const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[g]);
-    for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[g][j]];
-    if (lane == 0) s_nsel[g] = cnt;
   }
   __syncthreads();
+  if (s_abort && tid == 0) {
+    // summary copies still in flight: the last stage issued into each slot, on its own parity
+    for (int j = max(0, sub_issued - NS); j < sub_issued; ++j)
+      (void)mbar_wait_bounded(&bar[j % NS], (j / NS) & 1, 1u << 12);
+    report_timeout(p.status, 1);
+  }
+
+  // ---- 2. Top-K per head (per group when shared) -----------------------------------------
+  uint32_t* ck = s_scratch + warp * 2 * kCandMax;
+  int* cp = reinterpret_cast<int*>(ck + kCandMax);
+  cluster_wait();  // every peer has started: DSMEM stores may begin
+  if (p.gather) {
+    // push my slice of every selecting head's keys into every CTA's whole-row copy
+    const int nvec = rows >> 2, tail = rows & 3;
+    const int per_g = CL * (nvec + tail);
+    for (int e = tid; e < Gs * per_g; e += kThreads) {
+      const int g = e / per_g, rem = e % per_g;
+      const int r = rem / (nvec + tail), v = rem % (nvec + tail);
+      const uint32_t* src = s_keys + g * p.chunk;
+      uint32_t* dst = sel_buf + (size_t)g * p.row_ld + c_lo;
+      if (v < nvec) {
+        const uint4 x = *reinterpret_cast<const uint4*>(src + 4 * v);
+        st_dsmem_v4(dsmem_addr(dst + 4 * v, r), x);
+      } else {
+        const int t = 4 * nvec + (v - nvec);
+        st_dsmem_u32(dsmem_addr(dst + t, r), src[t]);
+      }
+    }
+    cluster_sync();
+    for (int g = warp; g < Gs; g += kWarps) {
+      const int cnt = warp_select(sel_buf + (size_t)g * p.row_ld, nc, K, lane, s_pick[warp], ck, cp);
+      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = s_pick[warp][j];
+      if (lane == 0) s_nsel[g] = cnt;
+    }
+  } else {
+    // local Top-K per head, pushed into every CTA's merge buffer at slot rank * K
+    uint32_t* m_key = sel_buf;
+    int* m_idx = reinterpret_cast<int*>(sel_buf) + G * CL * K;
+    for (int g = warp; g < Gs; g += kWarps) {
+      const uint32_t* keys = s_keys + g * p.chunk;
+      const int cnt = warp_select(keys, rows, K, lane, s_pick[warp], ck, cp);
+      for (int e = lane; e < CL * K; e += 32) {
+        const int r = e / K, j = e % K;
+        const uint32_t key = j < cnt ? keys[s_pick[warp][j]] : 0u;
+        const int gi = j < cnt ? c_lo + s_pick[warp][j] : -1;  // -1: empty slot
+        const int slot = g * CL * K + rank * K + j;
+        st_dsmem_u32(dsmem_addr(&m_key[slot], r), key);
+        st_dsmem_u32(dsmem_addr(&m_idx[slot], r), (uint32_t)gi);
+      }
+    }
+    cluster_sync();
+    for (int g = warp; g < Gs; g += kWarps) {
+      // empty slots carry key 0 and index -1: compact the valid ones first (index order kept:
+      // slot order is rank order and each rank's slots are ascending)
+      uint32_t* mk_g = m_key + g * CL * K;
+      int* mi_g = m_idx + g * CL * K;
+      int nvalid = 0;
+      for (int e0 = 0; e0 < CL * K; e0 += 32) {
+        const int e = e0 + lane;
+        const bool ok = e < CL * K && mi_g[e] >= 0;
+        const uint32_t kk2 = ok ? mk_g[e] : 0u;
+        const int ii = ok ? mi_g[e] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, ok);
+        __syncwarp();
+        if (ok) {
+          const int at = nvalid + __popc(bal & ((1u << lane) - 1u));
+          mk_g[at] = kk2;
+          mi_g[at] = ii;
+        }
+        nvalid += __popc(bal);
+        __syncwarp();
+      }
+      const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[warp], ck, cp);
+      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[warp][j]];
+      if (lane == 0) s_nsel[g] = cnt;
+    }
+  }
+  __syncthreads();
+
+  // ---- 3. the union of the selections, plus the current block ------------------------------
+  const int nwords = (nc + 31) / 32;
+  for (int w = tid; w < nwords; w += kThreads) s_bits[w] = 0u;
   if (rank == 0) {  // optional outputs: the selection of every head
     for (int e = tid; e < G * K; e += kThreads) {
       const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
@@ -480,6 +681,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       if (p.count && j == 0) p.count[row] = s_nsel[gs];
     }
   }
+  for (int e = tid; e < kMaxUnion; e += kThreads) s_umask[e] = 0u;
+  __syncthreads();
   for (int e = tid; e < Gs * K; e += kThreads) {
     const int g = e / K, j = e % K;
     if (j < s_nsel[g]) {
@@ -487,7 +690,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       atomicOr(&s_bits[x >> 5], 1u << (x & 31));
     }
   }
-  for (int e = tid; e < kMaxUnion; e += kThreads) s_umask[e] = 0u;
   __syncthreads();
   if (warp == 0) {  // compact the bitmap into the sorted union (one word per lane up to 32)
     const int per = (nwords + 31) / 32;
@@ -530,33 +732,55 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   }
   __syncthreads();
 
-  // ---- 3. attend my union entries -----------------------------------------------------------
-  const int ne = rank < U ? (U - rank + CL - 1) / CL : 0;
-  auto entry_tokens = [&](int m) { return m == cur ? pos - cur * b + 1 : b; };
-  float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 3: [warp][G][D+2]
+  // ---- 4. attend my share of the union ------------------------------------------------------
+  float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 4: [warp][G][D+2]
 
   if constexpr (kMma) {
-    // two groups of four warps take alternate entries; stage st = entry & 1 holds K then V
+    // 16-token slices: history entries have 4, the current block ceil(tok / 16); CTA r takes
+    // slices [r S / CL, (r + 1) S / CL); a stage holds four consecutive slices (K then V tiles,
+    // 64 rows x 128 bytes per 64-column half, 128-byte swizzle), stage i is taken by group i & 1
+    const int tok_cur = pos - cur * b + 1;
+    const int s_hist = 4 * (U - 1);
+    const int S_tot = s_hist + (tok_cur + kSlice - 1) / kSlice;
+    const int s_begin = (int)(((long long)rank * S_tot) / CL);
+    const int s_end = (int)(((long long)(rank + 1) * S_tot) / CL);
+    const int n_my = s_end - s_begin;
+    const int nst = (n_my + 3) / 4;
     const int grp = warp >> 2, wg = warp & 3;
-    const size_t tl = SM::tile(b);
+    const size_t tl = SM::kv_tile(b);
     auto ktile = [&](int st) { return smem + (size_t)st * 2 * tl; };
     auto vtile = [&](int st) { return smem + (size_t)st * 2 * tl + tl; };
-    uint64_t* kvbar = bar + 2;
+    uint64_t* kvbar = bar + NS;
     const int row0 = (bi * p.Hk + kh) * p.n;
+    // Each group owns NKV / 2 slots and refills them itself: stage i (group i & 1, its (i >> 1)-th)
+    // uses slot (i & 1) + 2 ((i >> 1) % nper) in phase (i >> 1) / nper, and the group issues
+    // stage i + NKV into the same slot once it has finished stage i.  A group therefore never waits
+    // on a phase of a slot that has not been issued yet, however far it runs ahead of the other.
+    const int nper = NKV / 2;
+    auto slot_of = [&](int i) { return (i & 1) + 2 * ((i >> 1) % nper); };
+    auto parity_of = [&](int i) { return (uint32_t)(((i >> 1) / nper) & 1); };
+    // slice -> (block, first token of the slice within the block)
+    auto slice_blk = [&](int s) { return s < s_hist ? s_ublk[s >> 2] : cur; };
+    auto slice_tok0 = [&](int s) { return s < s_hist ? (s & 3) * kSlice : (s - s_hist) * kSlice; };
     auto issue_kv = [&](int i) {
-      const int m = s_ublk[rank + i * CL];
-      const int st = i & 1;
-      mbar_arrive_expect_tx(&kvbar[st], 2 * 64 * D * 2);
+      const int st = slot_of(i);
+      s_kv_last[st] = i;
+      const int first = s_begin + 4 * i;
+      const int nsl = min(4, s_end - first);
+      mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
+      for (int w = 0; w < nsl; ++w) {
+        const int s = first + w;
+        const int y = row0 + slice_blk(s) * b + slice_tok0(s);
 #pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        tc::tma_load_2d(ktile(st) + hf * 8192, &tmk, hf * 64, row0 + m * b, &kvbar[st]);
-        tc::tma_load_2d(vtile(st) + hf * 8192, &tmv, hf * 64, row0 + m * b, &kvbar[st]);
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tc::tma_load_2d(ktile(st) + hf * 8192 + w * kSlice * 128, &tmk, hf * 64, y, &kvbar[st]);
+          tc::tma_load_2d(vtile(st) + hf * 8192 + w * kSlice * 128, &tmv, hf * 64, y, &kvbar[st]);
+        }
       }
     };
     if (tid == 0 && !s_abort) {
       fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
-      if (ne > 0) issue_kv(0);
-      if (ne > 1) issue_kv(1);
+      for (int i = 0; i < min(nst, NKV); ++i) issue_kv(i);
     }
     // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
     const int grow = lane >> 2, tig = lane & 3;
@@ -582,13 +806,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
     float m_run = -INFINITY, l_part = 0.f;
-    for (int i = grp; i < ne; i += 2) {
-      const int st = i & 1;
-      const int m = s_ublk[rank + i * CL];
-      const unsigned hm = s_umask[rank + i * CL];
-      const int tok = entry_tokens(m);
+    const int n_run = s_abort ? 0 : nst;  // nothing was issued after an earlier timeout
+    for (int i = grp; i < n_run; i += 2) {
+      const int st = slot_of(i);
       // group-uniform decision: the OR over the group's four warps of "my wait ran out"
-      const int bad = mbar_wait_bounded(&kvbar[st], (i >> 1) & 1) ? 0 : 1;
+      const int bad = mbar_wait_bounded(&kvbar[st], parity_of(i)) ? 0 : 1;
       int any_bad;
       asm volatile(
           "{\n\t.reg .pred pin, pout;\n\t"
@@ -602,124 +824,97 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         s_abort = 1;
         break;
       }
-      const unsigned char* kt = ktile(st);
-      const unsigned char* vt = vtile(st);
-      const int t0 = wg * 16;  // this warp's 16 tokens
-      // S = Q K^T over two 8-token tiles
-      float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      const int s = s_begin + 4 * i + wg;  // this warp's slice
+      if (s < s_end) {
+        const int m = slice_blk(s);
+        const unsigned hm = s < s_hist ? s_umask[s >> 2] : (1u << G) - 1u;
+        const int tv = m == cur ? min(kSlice, tok_cur - slice_tok0(s)) : kSlice;  // valid tokens
+        const unsigned char* kt = ktile(st);
+        const unsigned char* vt = vtile(st);
+        const int t0 = wg * kSlice;  // this warp's 16 rows of the stage tile
+        // S = Q K^T over two 8-token tiles
+        float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
+        for (int nt = 0; nt < 2; ++nt) {
+          const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int hf = ks >> 2, ch = (ks & 3) * 2;
-          const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
-          const uint32_t b0 =
-              *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
-          const uint32_t b1 =
-              *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
-          mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
-        }
-      }
-      // masks, per-row online softmax (row = head grow; the quad shares the row)
-      const bool head_on = grow < G && ((hm >> grow) & 1u);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = t0 + 8 * nt + 2 * tig + e;
-          if (!head_on || t >= tok) sfr[nt][e] = -INFINITY;
-          mx = fmaxf(mx, sfr[nt][e]);
-        }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
-      if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
-        corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
-        m_run = mx;
-        l_part *= corr;
-      }
-      // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
-      const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
-      const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
-      if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-          oacc[c][0] *= corr_a;
-          oacc[c][1] *= corr_b;
-          oacc[c][2] *= corr_a;
-          oacc[c][3] *= corr_b;
-        }
-      }
-      float pv[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float z = sfr[nt][e];
-          pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
-          l_part += pv[nt][e];
-        }
-      // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
-      const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
-      const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
-      // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
-#pragma unroll
-      for (int mt = 0; mt < D / 16; ++mt) {
-        const int mi = lane >> 3, rr = lane & 7;
-        const int tokr = t0 + (mi >> 1) * 8 + rr;
-        const int chunk = 2 * mt + (mi & 1);  // 16-byte chunk along d (0..D/8-1)
-        const int hf = chunk >> 3, cin = chunk & 7;
-        const uint32_t addr =
-            smem_u32(vt + hf * 8192 + tokr * 128 + ((cin ^ (tokr & 7)) << 4));
-        uint32_t v0, v1, v2, v3;
-        ldsm_x4_trans(addr, v0, v1, v2, v3);
-        mma_16816(oacc[mt], v0, v1, v2, v3, pb0, pb1);
-      }
-      // the block being filled: rewrite its summary from the swizzled K tile
-      if (p.append && m == cur) {  // taken by the whole group that holds the current block
-        const int gt = tid & 127;
-        const int col = gt;  // one column per thread (D <= 128)
-        if (col < D) {
-          float sum = 0.f;
-          const int hf = col >> 6, cin = (col & 63) >> 3, e8 = col & 7;
-          for (int t = 0; t < tok; ++t)
-            sum += Elem<T>::to_f(*reinterpret_cast<const T*>(
-                kt + hf * 8192 + t * 128 + ((cin ^ (t & 7)) << 4) + e8 * 2));
-          mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = Elem<TS>::from_f(sum / (float)tok);
-        }
-        // max key norm: thread t < tok takes token t
-        float nrm = 0.f;
-        if (gt < tok) {
-          float sq = 0.f;
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            const int hf = c8 >> 3, cin = c8 & 7;
-            float xx[8];
-            load_vec<T, 8>(reinterpret_cast<const T*>(kt + hf * 8192 + gt * 128 +
-                                                      ((cin ^ (gt & 7)) << 4)),
-                           xx);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sq = fmaf(xx[e], xx[e], sq);
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const int hf = ks >> 2, ch = (ks & 3) * 2;
+            const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
+            const uint32_t b0 =
+                *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
+            const uint32_t b1 =
+                *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
+            mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
           }
-          nrm = sqrtf(sq);
         }
-        nrm = warp_max(nrm);
-        if (lane == 0) s_red[4 * grp + wg] = nrm;
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));
-        if (gt == 0) {
-          const float* rr = s_red + 4 * grp;
-          float nm = fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3]));
-          const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
-          if (p.max_norm) p.max_norm[row] = nm;
-          if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
+        // masks, per-row online softmax (row = head grow; the quad shares the row)
+        const bool head_on = grow < G && ((hm >> grow) & 1u);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = 8 * nt + 2 * tig + e;
+            if (!head_on || t >= tv) sfr[nt][e] = -INFINITY;
+            mx = fmaxf(mx, sfr[nt][e]);
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
+        if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
+          corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
+          m_run = mx;
+          l_part *= corr;
+        }
+        // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
+        const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
+        const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
+        if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            oacc[c][0] *= corr_a;
+            oacc[c][1] *= corr_b;
+            oacc[c][2] *= corr_a;
+            oacc[c][3] *= corr_b;
+          }
+        }
+        float pv[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float z = sfr[nt][e];
+            pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
+            l_part += pv[nt][e];
+          }
+        // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
+        const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
+        const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+        // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int mi = lane >> 3, rr = lane & 7;
+          const int tokr = t0 + (mi >> 1) * 8 + rr;
+          const int chunk = 2 * mt + (mi & 1);  // 16-byte chunk along d (0..D/8-1)
+          const int hf = chunk >> 3, cin = chunk & 7;
+          const uint32_t addr =
+              smem_u32(vt + hf * 8192 + tokr * 128 + ((cin ^ (tokr & 7)) << 4));
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(addr, v0, v1, v2, v3);
+          mma_16816(oacc[mt], v0, v1, v2, v3, pb0, pb1);
         }
       }
       asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
-      if (wg == 0 && lane == 0 && i + 2 < ne) issue_kv(i + 2);
+      if (wg == 0 && lane == 0 && i + NKV < nst) issue_kv(i + NKV);
     }
+    __syncthreads();
     if (s_abort && tid == 0) {
-      for (int i = 0; i < 2; ++i) (void)mbar_wait_bounded(&kvbar[i], 0, 1u << 12);
+      // copies still in flight: the last stage issued into each slot; waiting on its own phase
+      // parity returns at once if it already landed
+      for (int st = 0; st < NKV; ++st)
+        if (s_kv_last[st] >= 0)
+          (void)mbar_wait_bounded(&kvbar[st], parity_of(s_kv_last[st]), 1u << 12);
       report_timeout(p.status, 2);
     }
     __syncthreads();
@@ -745,11 +940,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     }
     __syncthreads();
   } else {
-    // fp32: scalar FMAs; warps split each block's tokens, one CTA-wide softmax per block
-    const size_t tl = SM::tile(b);
+    // fp32 / other block sizes: scalar FMAs; CTA r takes union entries r, r + CL, ...; warps split
+    // each block's tokens, one CTA-wide softmax per block
+    const int ne = rank < U ? (U - rank + CL - 1) / CL : 0;
+    auto entry_tokens = [&](int m) { return m == cur ? pos - cur * b + 1 : b; };
+    const size_t tl = SM::kv_tile(b);
     T* kbuf[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem + 2 * tl)};
     T* vbuf[2] = {reinterpret_cast<T*>(smem + tl), reinterpret_cast<T*>(smem + 3 * tl)};
-    uint64_t* kvbar = bar + 2;
+    uint64_t* kvbar = bar + NS;
     const T* kbase = static_cast<const T*>(p.k) + (size_t)(bi * p.Hk + kh) * p.n * D;
     const T* vbase = static_cast<const T*>(p.v) + (size_t)(bi * p.Hk + kh) * p.n * D;
     auto issue_kv = [&](int i) {
@@ -776,14 +974,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     float acc[G][2];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
-    for (int i = 0; i < ne; ++i) {
+    int i_stop = ne;
+    const int n_run = s_abort ? 0 : ne;  // nothing was issued after an earlier timeout
+    for (int i = 0; i < n_run; ++i) {
       const int st = i & 1;
       const int m = s_ublk[rank + i * CL];
       const unsigned hm = s_umask[rank + i * CL];
       const int tok = entry_tokens(m);
       if (!s_abort && !mbar_wait_bounded(&kvbar[st], (i >> 1) & 1)) s_abort = 1;
       __syncthreads();
-      if (s_abort) break;
+      if (s_abort) {
+        i_stop = i;
+        break;
+      }
       const T* kt = kbuf[st];
       const T* vt = vbuf[st];
       for (int t0 = warp * R; t0 < tok; t0 += kWarps * R) {
@@ -873,8 +1076,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       __syncthreads();
       if (tid == 0 && i + 2 < ne) issue_kv(i + 2);
     }
-    if (s_abort && tid == 0) {
-      for (int i = 0; i < 2; ++i) (void)mbar_wait_bounded(&kvbar[i], 0, 1u << 12);
+    if (s_abort && tid == 0 && n_run > 0) {
+      // copies in flight: stages i_stop and i_stop + 1 (if issued), each on its own parity
+      for (int j = i_stop; j < min(ne, i_stop + 2); ++j)
+        (void)mbar_wait_bounded(&kvbar[j & 1], (j >> 1) & 1, 1u << 12);
       report_timeout(p.status, 2);
     }
     __syncthreads();
@@ -896,7 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     __syncthreads();
   }
 
-  // ---- 4. merge the warps, push column slices to their owners, finish -----------------------
+  // ---- 5. merge the warps, push column slices to their owners, finish -----------------------
   const int cols = D / CL;
   // per head: combined max over warps, then weights
   for (int g = warp; g < G; g += kWarps) {
@@ -977,12 +1182,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// K or V as [rows, D] bf16 with 64-column x 16-row boxes, 128-byte swizzle
 bool kv_map(CUtensorMap* m, const void* base, long long rows, int D) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, (cuuint32_t)kSlice};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1001,9 +1207,14 @@ LaunchCache& launch_cache() {
   return c;
 }
 
+// Shared memory one SM gives its resident CTAs (228 KB less 1 KB reserved per CTA) and the static
+// shared memory of the fused kernel (G <= 8), both with margin.
+constexpr size_t kSmemPerSM = 227 * 1024;
+constexpr size_t kStaticSmemBound = 12 * 1024;
+
 template <typename T, typename TS, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
-  using SM = FusedSmem<T, D, G, MMA>;
+  using SM = FusedSmem<T, TS, D, G, MMA>;
   CUtensorMap tmk{}, tmv{};
   if (MMA) {
     const long long rows = (long long)p.B * p.Hk * p.n;
@@ -1012,20 +1223,56 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
   auto kern = decode_fused_kernel<T, TS, D, G, MMA>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
   for (;;) {
     const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
-    if (chunk > 32 * kSelItems) {  // the local select holds at most 512 keys per head
+    if (chunk > kSelMax) {  // the local select holds at most kSelMax keys per head
       if (CL < kMaxCL) { CL <<= 1; continue; }
       return BSA_ERR_UNSUPPORTED;
     }
     p.chunk = chunk;
-    const size_t smem = SM::bytes(p.b, chunk, CL, p.K) + 1024;  // + alignment slack
-    if (smem > 220 * 1024) return BSA_ERR_UNSUPPORTED;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
-      (void)cudaGetLastError();
-      return BSA_ERR_CUDA;
+    // whole-row selection when every history fits one warp select
+    p.gather = p.C <= kSelMax ? 1 : 0;
+    p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
+    // the fixed pieces, then region A as large as the CTAs resident per SM allow
+    size_t off = 0;
+    const size_t fixed = SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K) + SM::recv(CL) +
+                         SM::zp(p.b) + 256;
+    const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage();
+    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), SM::partials());
+    // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
+    // (two K/V stages) does not fit that way
+    int per_sm = groups * CL > kSMs ? 2 : 1;
+    size_t ra = 0;
+    for (;; per_sm = 1) {
+      const size_t budget = kSmemPerSM / per_sm - kStaticSmemBound - 1024 /* alignment slack */;
+      ra = budget > fixed ? (budget - fixed) / 1024 * 1024 : 0;
+      if (ra >= need_min || per_sm == 1) break;
     }
+    if (ra < need_min) return BSA_ERR_UNSUPPORTED;
+    ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus),
+                             SM::partials()));
+    p.ns = (int)std::min<size_t>(kMaxStages, ra / sus);
+    // the MMA path's groups own half of the K/V slots each: an even count
+    p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) / 2 * 2 : 2;
+    off = align_up(ra, 1024);
+    p.off_keys = (int)off;
+    off += SM::keys(chunk);
+    p.off_sel = (int)off;
+    off += SM::sel(p.gather, p.row_ld, CL, p.K);
+    p.off_recv = (int)off;
+    off += SM::recv(CL);
+    p.off_zp = (int)off;
+    off += SM::zp(p.b);
+    off = align_up(off, 16);
+    p.off_bar = (int)off;
+    off += 256;
+    const size_t smem = off + 1024;  // + alignment slack of the dynamic base
+    if (smem > 227 * 1024) return BSA_ERR_UNSUPPORTED;
     LaunchCache& lc = launch_cache();
     {
       std::lock_guard<std::mutex> lock(lc.mu);

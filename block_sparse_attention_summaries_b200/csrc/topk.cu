@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(THREADS)
   // the older ones; their indices are all larger, so the row stays ascending
   const int newest = min(keep_newest, nc);
   nc -= newest;
-  const int kk = min(K, nc);
+  // K < 0: the upper half of the candidates, ceil(nc / 2) (FS-B's high-norm cells)
+  const int kk = K < 0 ? (nc + 1) / 2 : min(K, nc);
   int* out = idx + (size_t)row * out_ld;
   if (count && tid == 0) count[row] = kk + newest;
   for (int j = kk + tid; j < out_ld; j += THREADS) out[j] = j - kk < newest ? nc + (j - kk) : -1;

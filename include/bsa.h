@@ -311,6 +311,98 @@ bsa_status bsa_fsl_select(const void* q, bsa_dtype dt, int B, int H, int d, cons
                           void* stream);
 
 /*
+ * bsa_fsl_state_update -- the FS-L state as a fixed-size structure updated in O(P) per new cell
+ * ([FreeSolo] "How it differs", FS-L: the prefix is pruned before the query arrives, cost O(N),
+ * state of fixed size).  Per row (batch x head) the state is
+ *     older       [rows, P] int32: the kept older cells, ascending, -1 padded (in/out),
+ *     older_count [rows] int32: how many of them are valid (in/out),
+ *     state_cells [rows] int32: the candidate cells the state covers (in/out);
+ * a new row starts with older_count = state_cells = 0.  The call grows each row's candidate
+ * prefix from state_cells to n_cells[row] (never shrinks it), one cell at a time: the cell leaving
+ * the W newest joins the older cells and replaces the lowest-ranked kept one if its maximum key
+ * norm ranks higher (larger first, lower index on ties, NaN last), or joins outright while fewer
+ * than P are kept.  The result equals bsa_fsl_prune's set for the same n_cells.
+ *   max_norm  [rows, C] float32 (bsa_build_block_summaries with b = cell).
+ *   n_cells   [rows] int32: candidate cells of the row's current query (cells wholly before its
+ *             query block: floor(i / 128) * 128 / cell at query position i).
+ *   cand      [rows, W + P] int32 out: the kept cells ascending (older ones, then the W newest),
+ *             -1 padded; cand_count [rows] optional out.   Limits: P <= 128, W + P <= 128.
+ */
+bsa_status bsa_fsl_state_update(const float* max_norm, int rows, int C, const int* n_cells, int W,
+                                int P, int* older, int* older_count, int* state_cells, int* cand,
+                                int* cand_count, void* stream);
+
+/*
+ * bsa_fsl_decode -- FS-L decode output of one query per (batch, head) ([FreeSolo] "How it works"
+ * two-branch output, with the long branch's top K taken among the FS-L state's kept cells,
+ * "How it differs"):
+ *     o = (1 - alpha_h) o_short + alpha_h o_long      (o_short alone when no cell is kept)
+ * o_short: softmax of RoPE(q_i) . RoPE(k_j) / sqrt(d) over j in [i - window + 1, i] (base
+ * rope_theta, rotate-half pairing, absolute positions) against v_j; o_long: softmax of the raw
+ * q_i . k_j / sqrt(d) over the tokens of the K best kept cells by the FreeSolo cell score (as
+ * bsa_fsl_select: ties to the lower cell, NaN last).
+ *   q [B, H, d], k / v [B, H, n, d] (MHA), pos [B] int32 device: the query position i of each
+ *   batch row (its own key at i is in the cache).
+ *   mean_k / max_norm / centre: cell summaries [B, H, C, *], C = ceil(n / cell); lambda_h,
+ *   sigma_h [H] or NULL (plain dot score); alpha_h [H].
+ *   cand, cand_count, cand_ld: the kept cells (bsa_fsl_state_update or bsa_fsl_prune).
+ *   o [B, H, d] out; idx [B, H, K] optional out (selected cells ascending, -1 padded); count
+ *   [B, H] optional out; status optional device int, set nonzero if a bounded wait ran out.
+ *   Limits: K <= 8, window <= 1024, cell <= 128, cand_ld <= 128.  Needs no workspace: four CTAs
+ *   per row form a cluster and merge through distributed shared memory.
+ */
+bsa_status bsa_fsl_decode(const void* q, const void* k, const void* v, bsa_dtype dt, int B, int H,
+                          int n, int d, const int* pos, int cell, const float* mean_k,
+                          const float* max_norm, const float* centre, const float* lambda_h,
+                          const float* sigma_h, const float* alpha_h, const int* cand,
+                          const int* cand_count, int cand_ld, int K, int window,
+                          float rope_theta, void* o, int* idx, int* count, int* status,
+                          void* stream);
+
+/*
+ * FS-B ([FreeSolo] "How it differs", FS-B): per (batch, head) two forests of cell summaries --
+ * one over every candidate cell, one over the cells of norm at or above the median -- searched by
+ * a beam of W_b nodes per level with the node score U_v as an upper bound of the cell scores
+ * below v; the cells reached are re-ranked by log-sum-exp over their token keys and the top K
+ * are read.  The page gives the node contents (mean key, radius, maximum norm, minimum position)
+ * and the search, not the tree shape; this library reads it as follows.  A forest over m cells in
+ * position order is the row of perfect binary trees given by the set bits of m (largest first);
+ * the "median" forest holds the ceil(m / 2) cells of largest maximum key norm (lower index on
+ * ties, NaN last), in position order; a node keeps the mean of its leaves' mean keys, the
+ * largest distance of a leaf mean key from it, the largest leaf norm and the smallest leaf
+ * centre; U_v = (q . mu_v + ||q|| rho_v) / sqrt(d) + lambda_h a_max erf((i - p_min) / (2 sigma_h)).
+ * Level h of the beam holds the W_b best (U as float32, larger first, lower first cell on ties)
+ * of the previous beam's children and the root of height h, if any.
+ *
+ * bsa_fsb_forest_bytes -- bytes of the forest buffer for B x H rows over C cells of head dim d
+ * (0 for unsupported sizes: C > 16384, d not in {64, 128}).
+ *
+ * bsa_fsb_build -- build both forests of every row for its candidate prefix of n_cells[row]
+ * cells (cells wholly before the query block: floor(i / 128) * 128 / cell).
+ *   mean_k [B, H, C, d], max_norm / centre [B, H, C] float32 (bsa_build_block_summaries, b = cell).
+ *   n_cells [B * H] int32 device.   forest: device buffer of bsa_fsb_forest_bytes() bytes, 16-byte
+ *   aligned (written; the caller owns it).
+ *
+ * bsa_fsb_select -- the FS-B selection of one query per (batch, head) over forests built for its
+ * candidate prefix.
+ *   q [B, H, d], k [B, H, n, d] (the token keys of the re-rank, unrotated), pos [B] int32 device:
+ *   query position i (for the erf bias); cell, n: C = ceil(n / cell) must equal the build's C.
+ *   lambda_h, sigma_h [H] or NULL (plain dot score in U).   width: W_b (1..16).   K: 1..8.
+ *   idx [B, H, K] int32 out (selected cells ascending, -1 padded); count [B, H] optional out;
+ *   lse [B, H, K] optional out: the re-rank score of each selected cell.
+ * The selected cells feed bsa_fsl_decode as its kept set (cand = idx, cand_count = count, the
+ * same K) for the two-branch decode output.
+ */
+size_t bsa_fsb_forest_bytes(int B, int H, int C, int d);
+bsa_status bsa_fsb_build(const float* mean_k, const float* max_norm, const float* centre, int B,
+                         int H, int C, int d, const int* n_cells, void* forest,
+                         size_t forest_bytes, void* stream);
+bsa_status bsa_fsb_select(const void* q, const void* k, bsa_dtype dt, int B, int H, int n, int d,
+                          const int* pos, int cell, const void* forest, size_t forest_bytes,
+                          const float* lambda_h, const float* sigma_h, int width, int K, int* idx,
+                          int* count, float* lse, void* stream);
+
+/*
  * bsa_freesolo_select -- per-query cell selection of the FreeSolo long branch (prefill),
  * [FreeSolo] "How it works": for the query at position i of head h the candidates are the cells
  * c lying wholly before the start of its query block, (c + 1) * cell <= floor(i / q_block) *

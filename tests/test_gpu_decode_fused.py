@@ -119,9 +119,12 @@ def test_fused_full_size(wl):
     torch.cuda.synchronize()
     assert torch.equal(idx1, idx2)
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
-    rng = np.random.default_rng(7)
-    rows = sorted({(int(bi), int(h)) for bi, h in zip(rng.integers(0, w["B"], 6),
-                                                        rng.integers(0, 32, 6))} | {(0, 0)})
+    if w["B"] == 1:  # long context: every head of the sequence
+        rows = [(0, h) for h in range(32)]
+    else:
+        rng = np.random.default_rng(7)
+        rows = sorted({(int(bi), int(h)) for bi, h in zip(rng.integers(0, w["B"], 16),
+                                                            rng.integers(0, 32, 16))} | {(0, 0)})
     oracle_check(case, idx1.cpu().numpy(), o1.float().cpu().numpy(), lse1.cpu().numpy(), rows,
                  2e-2)
     # needle recall: every head of a group sees its planted blocks first
@@ -132,6 +135,56 @@ def test_fused_full_size(wl):
         hits += len(sel & set(int(c) for c in blocks))
         tot += len(blocks)
     assert hits / tot > 0.9
+
+
+@pytest.mark.parametrize("n,B", [(40000, 2), (64 * 513 + 10, 1)])
+def test_fused_long_history_local_and_merged_selection(n, B):
+    """More than 512 history blocks: each CTA selects its slice's Top-K and the cluster merges the
+    candidates (some CTAs of the cluster hold no block at all); every row against the separate
+    calls and sampled rows against the oracle."""
+    case = inputs.decode_case(64 + B, B=B, Hq=8, Hk=2, d=128, n=n, b=64, K=13, needles=9,
+                              seq_lens=[n, n - 3000][:B])
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, 64, sl)
+    o1, lse1, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, 64, 13, seq_lens=sl,
+                                                 append=False)
+    o2, lse2, idx2 = bsa.decode_step(q, k, v, mean_k, 64, 13, seq_lens=sl, append=False)
+    torch.cuda.synchronize()
+    assert torch.equal(idx1, idx2)
+    assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+    rows = [(bi, h) for bi in range(B) for h in (0, 3, 5, 7)]
+    oracle_check(case, idx1.cpu().numpy(), o1.float().cpu().numpy(), lse1.cpu().numpy(), rows,
+                 2e-2)
+
+
+@pytest.mark.parametrize("C", [300, 1000])
+def test_fused_all_scores_tied_take_the_lowest_blocks(C):
+    """Every history block scores exactly 0 (all keys zero): the Top-K is the K lowest block
+    indices for every head, on the whole-row path (300 blocks) and on the local + merge path
+    (1000 blocks); the threshold pass leaves every key as a candidate, so the radix select runs."""
+    B, Hk, G, d, b, K = 2, 2, 4, 64, 64, 11
+    n = C * b
+    k = torch.zeros(B, Hk, n, d, device=DEV, dtype=torch.bfloat16)
+    g = torch.Generator(device=DEV).manual_seed(5)
+    v = torch.randn(B, Hk, n, d, device=DEV, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Hk * G, d, device=DEV, generator=g).to(torch.bfloat16)
+    mean_k, _, _ = bsa.build_block_summaries(k, b)
+    o1, _, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, b, K, append=False)
+    o2, _, idx2 = bsa.decode_step(q, k, v, mean_k, b, K, append=False)
+    torch.cuda.synchronize()
+    want = torch.arange(K, device=DEV, dtype=torch.int32).expand(B, Hk * G, K)
+    assert torch.equal(idx1, want) and torch.equal(idx2, want)
+    assert torch.equal(cnt1, torch.full_like(cnt1, K))
+    # zero keys: every attended token has logit 0, so o is the mean of the attended values
+    vf = v.float()
+    cur = (n - 1) // b
+    for bi in range(B):
+        for kh in range(Hk):
+            toks = torch.cat([vf[bi, kh, :K * b], vf[bi, kh, cur * b:n]])
+            ref = toks.mean(0)
+            for h in range(kh * G, (kh + 1) * G):
+                assert (o1[bi, h].float() - ref).abs().max().item() < 2e-2
+    assert (o1.float() - o2.float()).abs().max().item() < 1e-2
 
 
 # ---- variants: GQA-shared selection and bf16 summaries (bsa_decode_step_ex) ------------------
