@@ -453,38 +453,49 @@ def run_prefill(dev, peaks, reps=5):
     del q, k, v, o, ws, sws, idx, cnt
     torch.cuda.empty_cache()
 
-    # FS-L decode selection at 256K: the pruned state (W + P cells) against full O(C) scoring
-    H, d, n, cell, K, W, P = 16, 64, 262144, 32, 4, 8, 64
+    # FS-L / FS-B decode at 256K, batch 1 ([FreeSolo] "How it differs": FS-L keeps W + P cells
+    # per head in a fixed-size state, FS-B searches two forests): the kept-cell selection against
+    # full O(C) scoring, the FS-L state update per query block, the decode call (window + long
+    # branch + mix) and the FS-B build and search.  Each call of a timed graph decodes its own
+    # position (positions 600 tokens apart, so no call finds another's window in L2).
+    H, d, n, cell, K, W, P, window, width = 16, 64, 262144, 32, 4, 8, 64, 512, 16
     g = torch.Generator(device=dev).manual_seed(4200)
     kf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
+    vf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
     qf = torch.randn(1, H, d, device=dev, generator=g).to(torch.bfloat16)
     mk, mx, ce = bsa.build_block_summaries(kf, cell)
-    del kf
     C = mk.shape[2]
-    posv = n - 1
-    pos = torch.full((1,), posv, dtype=torch.int32, device=dev)
     lam = torch.full((H,), 0.5, device=dev)
     sig = torch.full((H,), 4096.0, device=dev)
-    n_cells = torch.full((1, H), (posv // 128) * 128 // cell, dtype=torch.int32, device=dev)
-    cand, ccnt = bsa.fsl_prune(mx, n_cells, W, P)
+    alpha = torch.rand(H, device=dev, generator=g)
+    iters = 20
+    positions = [n - 1 - 600 * r for r in range(iters)]
+    pos_t = [torch.full((1,), p_, dtype=torch.int32, device=dev) for p_ in positions]
+    ncell_t = [torch.full((H,), (p_ // 128) * 128 // cell, dtype=torch.int32, device=dev)
+               for p_ in positions]
+    states = []
+    for r in range(iters):  # a state per position, grown from empty
+        st = bsa.FslState(H, W, P, dev)
+        st.update(mx.view(H, C), ncell_t[r])
+        states.append(st)
     seq = torch.full((1,), n, dtype=torch.int32, device=dev)
     sc = torch.empty(1, H, C, device=dev)
     ncnd = torch.empty(H, device=dev, dtype=torch.int32)
-    full = lambda: bsa.topk_blocks(bsa.score_blocks(qf, mk, n, cell, seq_lens=seq, max_norm=mx,
-                                                    centre=ce, lambda_h=lam, sigma_h=sig,
-                                                    prefix_block=128, scores=sc, n_cand=ncnd)[0],
-                                   K, n_cand=ncnd)
-    fsl = lambda: bsa.fsl_select(qf, pos, mk, mx, ce, lam, sig, cand, ccnt, K)
-    prune = lambda: bsa.fsl_prune(mx, n_cells, W, P)
-    def graph_ms(fn, iters=20):
-        """Device time per call: `iters` calls captured in one CUDA graph (these calls are a
-        few microseconds each, far below the cost of launching them one by one from Python)."""
+    o_f = torch.empty(1, H, d, device=dev, dtype=torch.bfloat16)
+    idx_f = torch.empty(1, H, K, device=dev, dtype=torch.int32)
+    cnt_f = torch.empty(1, H, device=dev, dtype=torch.int32)
+    stat_f = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def graph_ms(fns):
+        """Device time per call: the calls captured in one CUDA graph (these calls are a few
+        microseconds each, far below the cost of launching them one by one from Python)."""
         with torch.cuda.stream(stream):
-            fn()
+            for fn in fns:
+                fn()
         torch.cuda.synchronize(dev)
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            for _ in range(iters):
+            for fn in fns:
                 fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
@@ -494,19 +505,88 @@ def run_prefill(dev, peaks, reps=5):
                 gr.replay()
             e1.record(stream)
         e1.synchronize()
-        return e0.elapsed_time(e1) / (reps * iters)
+        del gr
+        return e0.elapsed_time(e1) / (reps * len(fns))
 
+    seqs = [p_ + 1 for p_ in pos_t]
+    full = [lambda r=r: bsa.topk_blocks(bsa.score_blocks(
+        qf, mk, n, cell, seq_lens=seqs[r], max_norm=mx, centre=ce, lambda_h=lam, sigma_h=sig,
+        prefix_block=128, scores=sc, n_cand=ncnd)[0], K, n_cand=ncnd) for r in range(iters)]
+    fsl_sel = [lambda r=r: bsa.fsl_select(qf, pos_t[r], mk, mx, ce, lam, sig,
+                                          states[r].cand.view(1, H, -1),
+                                          states[r].cand_count.view(1, H), K)
+               for r in range(iters)]
+    fsl_dec = [lambda r=r: bsa.fsl_decode(qf, kf, vf, pos_t[r], cell, mk, mx, ce, lam, sig, alpha,
+                                          states[r].cand.view(1, H, -1),
+                                          states[r].cand_count.view(1, H), K, window=window,
+                                          o=o_f, idx=idx_f, count=cnt_f, status=stat_f)
+               for r in range(iters)]
     t_full = graph_ms(full)
-    t_fsl = graph_ms(fsl)
-    t_prune = graph_ms(prune)
+    t_fsl_sel = graph_ms(fsl_sel)
+    t_fsl_dec = graph_ms(fsl_dec)
+    # the state update at a query-block boundary: 4 new cells per head (the state is reset to
+    # its previous prefix inside the graph, three small copies)
+    saved = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
+    prev = [c - 4 for c in ncell_t]
+    for st, p_ in zip(states, prev):  # states one query block earlier
+        st.older.fill_(-1)
+        st.older_count.zero_()
+        st.state_cells.zero_()
+        st.update(mx.view(H, C), p_)
+    base = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
+
+    def upd(r):
+        st = states[r]
+        st.older.copy_(base[r][0])
+        st.older_count.copy_(base[r][1])
+        st.state_cells.copy_(base[r][2])
+        st.update(mx.view(H, C), ncell_t[r])
+    t_reset = graph_ms([lambda r=r: (states[r].older.copy_(base[r][0]),
+                                     states[r].older_count.copy_(base[r][1]),
+                                     states[r].state_cells.copy_(base[r][2]))
+                        for r in range(iters)])
+    t_upd = graph_ms([lambda r=r: upd(r) for r in range(iters)]) - t_reset
+    for st, sv in zip(states, saved):
+        assert torch.equal(st.older_count, sv[1]) and torch.equal(st.older, sv[0])
+    # FS-B: forests built for the query block's prefix, then beam search + re-rank + decode
+    forests = [bsa.fsb_build(mk, mx, ce, ncell_t[r]) for r in range(iters)]
+    fidx = torch.empty(1, H, K, device=dev, dtype=torch.int32)
+    fcnt = torch.empty(1, H, device=dev, dtype=torch.int32)
+    flse = torch.empty(1, H, K, device=dev)
+    t_fsb_build = graph_ms([lambda r=r: bsa.fsb_build(mk, mx, ce, ncell_t[r], forest=forests[r])
+                            for r in range(4)])
+    t_fsb_sel = graph_ms([lambda r=r: bsa.fsb_select(qf, kf, pos_t[r], cell, forests[r], lam,
+                                                     sig, width, K, idx=fidx, count=fcnt,
+                                                     lse=flse)
+                          for r in range(iters)])
+    del forests
+    # algorithmic bytes of one FS-L decode call: the window's K and V, the K selected cells' K
+    # and V, the kept cells' summaries, q and o
+    win = min(window, positions[0] + 1)
+    dec_bytes = H * (win * d * 2 * 2 + K * cell * d * 2 * 2 + (W + P) * (d + 2) * 4 + 2 * d * 2)
+    gbs = dec_bytes / (t_fsl_dec / 1e3) / 1e9
     out["fsl_decode_256k"] = {
         "config": {"B": 1, "H": H, "d": d, "n": n, "cell": cell, "K": K, "W": W, "P": P,
-                   "cells": C},
-        "full_select_ms": t_full, "fsl_select_ms": t_fsl, "fsl_prune_ms": t_prune,
+                   "window": window, "cells": C, "fsb_beam": width},
+        "full_select_ms": t_full, "fsl_select_ms": t_fsl_sel,
+        "fsl_state_update_ms": t_upd, "fsl_decode_ms": t_fsl_dec,
+        "fsl_step_ms": t_fsl_dec + t_upd / 128.0,
+        "fsl_tokens_per_s": 1.0 / ((t_fsl_dec + t_upd / 128.0) / 1e3),
+        "fsb_build_ms": t_fsb_build, "fsb_select_ms": t_fsb_sel,
+        "fsb_step_ms": t_fsb_sel + t_fsl_dec + t_fsb_build / 128.0,
+        "decode_bytes": dec_bytes,
+        "roofline": roofline("hbm", "fsl_decode_kernel", gbs, peaks["hbm_gbs"], "GB/s",
+                             algorithmic=dec_bytes,
+                             peak_source=peaks["source"] + " (burst copy)"),
         "kernels": "full: score_decode_kernel + topk_kernel over every cell; FS-L: "
-                   "fsl_select_kernel over W + P kept cells (prune: topk_kernel over key norms, "
-                   "once per new cell)",
+                   "fsl_select_kernel over the W + P kept cells; fsl_state_update_kernel (4 new "
+                   "cells per 128-token query block, amortised over its 128 steps); "
+                   "fsl_decode_kernel (4-CTA cluster per head); FS-B: topk_kernel (upper half) + "
+                   "fsb_build_levels/radius_kernel per query block (amortised over 128 steps), "
+                   "fsb_search_kernel per step",
     }
+    del kf, vf
+    torch.cuda.empty_cache()
     return out
 
 
@@ -759,6 +839,12 @@ def flat_rows(rows):
         out["long_decode_512k_tokens_per_s"] = ld["tokens_per_s"]
         out["long_decode_512k_frac"] = ld["roofline"]["frac"]
         out["long_decode_512k_selection_share"] = ld["separate_calls_us"]["selection_share"]
+    fl = rows.get("fsl_decode_256k")
+    if fl:
+        out["fsl_decode_256k_us"] = fl["fsl_decode_ms"] * 1e3
+        out["fsl_decode_256k_frac"] = fl["roofline"]["frac"]
+        out["fsl_state_update_us"] = fl["fsl_state_update_ms"] * 1e3
+        out["fsb_select_256k_us"] = fl["fsb_select_ms"] * 1e3
     sb = rows.get("summaries_build_32k")
     if sb:
         out["summaries_build_gbs"] = sb["gbs"]

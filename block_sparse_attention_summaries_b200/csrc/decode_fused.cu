@@ -33,7 +33,7 @@
 //   5. Each CTA merges its warps, then pushes to CTA r' the partial (m, l, o) of the output columns
 //      CTA r' owns; cluster barrier; each CTA finishes its columns and writes o (and lse).
 // On the 64-token bf16 path the summary of the block being filled is rewritten by the last CTA of
-// the cluster from global memory at the start, while its first summary stages are in flight.
+// the cluster from global memory, while its first K/V stages are in flight.
 // Variants (flags of bsa_decode_step_ex): shared selection -- the group's score of a block is the
 // mean of its G heads' scores, ranked once and attended by every head (one selection per kv
 // head instead of G); bf16 summaries -- the mean keys are read (and appended) in bf16, halving the
@@ -92,7 +92,7 @@ struct FusedParams {
   int ns;      // summary ring stages
   int nkv;     // K/V ring stages
   // dynamic shared-memory layout (byte offsets from the 1024-aligned base)
-  int off_keys, off_sel, off_recv, off_zp, off_bar;
+  int off_keys, off_sel, off_hbits, off_recv, off_zp, off_bar;
 };
 
 // ---- cluster helpers ---------------------------------------------------------------------
@@ -282,8 +282,8 @@ __device__ __noinline__ int warp_select_radix(const uint32_t* keys, int N, int k
 // distinct keys >= T0, so every key of the Top-kk is >= T0.  The keys >= T0 are compacted in
 // position order (usually a few more than kk) and ranked exactly; if more than kCandMax pass, the
 // radix select runs on all N keys instead.
-__device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out,
-                                        uint32_t* ck, int* cp) {
+__device__ __forceinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out,
+                                           uint32_t* ck, int* cp) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
   if (kk == N) {
@@ -401,6 +401,7 @@ struct FusedSmem {
   __host__ __device__ static size_t sel(int gather, int row_ld, int CL, int K) {
     return gather ? align_up((size_t)G * row_ld * 4, 16) : align_up((size_t)G * CL * K * 8, 16);
   }
+  __host__ __device__ static size_t hbits(int C) { return align_up((size_t)G * ((C + 31) / 32) * 4, 16); }
   __host__ __device__ static size_t recv(int CL) {
     return align_up((size_t)CL * G * (D / CL + 2) * 4, 16);
   }
@@ -452,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int Gs = p.shared ? 1 : G;  // selections made per group
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);  // [G][chunk]
   uint32_t* sel_buf = reinterpret_cast<uint32_t*>(smem + p.off_sel);  // whole rows / merge
+  uint32_t* hbits = reinterpret_cast<uint32_t*>(smem + p.off_hbits);  // [Gs][nwords] selections
   float* recv = reinterpret_cast<float*>(smem + p.off_recv);           // [CL][G][cols+2]
   float* zs = reinterpret_cast<float*>(smem + p.off_zp);
   float* ps = zs + align_up((size_t)b * G, 4);
@@ -497,48 +499,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
                      tmp);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
-  }
-  if constexpr (kMma) {
-    // the block being filled: its summary is rewritten from its keys (global memory) by the last
-    // CTA while the first summary stages are in flight
-    if (p.append && rank == CL - 1) {
-      const int tok = pos - cur * b + 1;
-      const T* kb = static_cast<const T*>(p.k) + ((size_t)(bi * p.Hk + kh) * p.n + (size_t)cur * b) * D;
-      float cs[EPL];
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) cs[e] = 0.f;
-      float nmax = 0.f;
-      for (int t = warp; t < tok; t += kWarps) {
-        float x[EPL];
-        load_vec<T, EPL>(kb + (size_t)t * D + lane * EPL, x);
-        float sq = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-          cs[e] += x[e];
-          sq = fmaf(x[e], x[e], sq);
-        }
-        nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
-      }
-      float* part = reinterpret_cast<float*>(s_scratch);  // [kWarps][D]
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) part[warp * D + lane * EPL + e] = cs[e];
-      if (lane == 0) s_red[warp] = nmax;
-      __syncthreads();
-      const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
-      for (int col = tid; col < D; col += kThreads) {
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) sum += part[w * D + col];
-        mean_k[row * D + col] = Elem<TS>::from_f(sum / (float)tok);
-      }
-      if (tid == 0) {
-        float nm = 0.f;
-        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
-        if (p.max_norm) p.max_norm[row] = nm;
-        if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
-      }
-      __syncthreads();
-    }
   }
   const float scale = rsqrtf((float)D);
   const int my_r = lane / G, my_g = lane % G;
@@ -671,8 +631,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __syncthreads();
 
   // ---- 3. the union of the selections, plus the current block ------------------------------
+  // every selection as a bitmap over the history blocks; one warp compacts the OR of the bitmaps
+  // into the sorted union and takes each entry's head mask from the same words
   const int nwords = (nc + 31) / 32;
-  for (int w = tid; w < nwords; w += kThreads) s_bits[w] = 0u;
+  for (int g = warp; g < Gs; g += kWarps) {
+    uint32_t* hb = hbits + g * nwords;
+    for (int w = lane; w < nwords; w += 32) hb[w] = 0u;
+    __syncwarp();
+    for (int j = lane; j < s_nsel[g]; j += 32) {
+      const int x = s_sel[g][j];
+      atomicOr(&hb[x >> 5], 1u << (x & 31));
+    }
+  }
   if (rank == 0) {  // optional outputs: the selection of every head
     for (int e = tid; e < G * K; e += kThreads) {
       const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
@@ -681,20 +651,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       if (p.count && j == 0) p.count[row] = s_nsel[gs];
     }
   }
-  for (int e = tid; e < kMaxUnion; e += kThreads) s_umask[e] = 0u;
   __syncthreads();
-  for (int e = tid; e < Gs * K; e += kThreads) {
-    const int g = e / K, j = e % K;
-    if (j < s_nsel[g]) {
-      const int x = s_sel[g][j];
-      atomicOr(&s_bits[x >> 5], 1u << (x & 31));
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {  // compact the bitmap into the sorted union (one word per lane up to 32)
+  if (warp == 0) {  // a contiguous run of words per lane, prefix sums of their union counts
     const int per = (nwords + 31) / 32;
+    const int w0 = min(nwords, lane * per), w1 = min(nwords, w0 + per);
     int mine = 0;
-    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) mine += __popc(s_bits[w]);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t u = 0u;
+      for (int g = 0; g < Gs; ++g) u |= hbits[g * nwords + w];
+      mine += __popc(u);
+    }
     int incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -702,12 +668,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       if (lane >= o) incl += y;
     }
     int at = incl - mine;
-    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) {
-      uint32_t bits = s_bits[w];
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        s_ublk[at++] = w * 32 + bit;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t hw[G];
+      uint32_t u = 0u;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        hw[g] = g < Gs ? hbits[g * nwords + w] : 0u;
+        u |= hw[g];
+      }
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        unsigned m = 0u;
+#pragma unroll
+        for (int g = 0; g < G; ++g) m |= ((hw[g] >> bit) & 1u) << g;
+        s_ublk[at] = w * 32 + bit;
+        s_umask[at] = p.shared ? (1u << G) - 1u : m;
+        ++at;
       }
     }
     if (lane == 31) {
@@ -718,19 +695,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   }
   __syncthreads();
   const int U = s_U;
-  for (int e = tid; e < Gs * K; e += kThreads) {  // head masks by binary search in the union
-    const int g = e / K, j = e % K;
-    if (j < s_nsel[g]) {
-      const int x = s_sel[g][j];
-      int lo = 0, hi = U - 2;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (s_ublk[mid] < x) lo = mid + 1; else hi = mid;
-      }
-      atomicOr(&s_umask[lo], p.shared ? (1u << G) - 1u : 1u << g);
-    }
-  }
-  __syncthreads();
 
   // ---- 4. attend my share of the union ------------------------------------------------------
   float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 4: [warp][G][D+2]
@@ -781,6 +745,57 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     if (tid == 0 && !s_abort) {
       fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
       for (int i = 0; i < min(nst, NKV); ++i) issue_kv(i);
+    }
+    if (p.append && rank == CL - 1) {
+      // the block being filled: its summary rewritten from its keys in global memory by the last
+      // CTA while its first K/V stages are in flight; every row is requested at once (a warp
+      // takes rows warp, warp + 8, ...: at most 8 of a 64-token block)
+      const T* kb =
+          static_cast<const T*>(p.k) + ((size_t)(bi * p.Hk + kh) * p.n + (size_t)cur * b) * D;
+      float x[8][EPL];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = warp + kWarps * u;
+        if (t < tok_cur) {
+          load_vec<T, EPL>(kb + (size_t)t * D + lane * EPL, x[u]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) x[u][e] = 0.f;
+        }
+      }
+      float cs[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cs[e] = 0.f;
+      float nmax = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float sq = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          cs[e] += x[u][e];
+          sq = fmaf(x[u][e], x[u][e], sq);
+        }
+        nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));  // rows past the block add 0
+      }
+      float* part = reinterpret_cast<float*>(s_scratch);  // [kWarps][D]
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) part[warp * D + lane * EPL + e] = cs[e];
+      if (lane == 0) s_red[warp] = nmax;
+      __syncthreads();
+      const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+      for (int col = tid; col < D; col += kThreads) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += part[w * D + col];
+        mean_k[row * D + col] = Elem<TS>::from_f(sum / (float)tok_cur);
+      }
+      if (tid == 0) {
+        float nm = 0.f;
+        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
+        if (p.max_norm) p.max_norm[row] = nm;
+        if (p.centre)
+          p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok_cur - 1);
+      }
     }
     // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
     const int grow = lane >> 2, tig = lane & 3;
@@ -1240,8 +1255,8 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
     // the fixed pieces, then region A as large as the CTAs resident per SM allow
     size_t off = 0;
-    const size_t fixed = SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K) + SM::recv(CL) +
-                         SM::zp(p.b) + 256;
+    const size_t fixed = SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K) +
+                         SM::hbits(p.C) + SM::recv(CL) + SM::zp(p.b) + 256;
     const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage();
     const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), SM::partials());
     // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
@@ -1264,6 +1279,8 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     off += SM::keys(chunk);
     p.off_sel = (int)off;
     off += SM::sel(p.gather, p.row_ld, CL, p.K);
+    p.off_hbits = (int)off;
+    off += SM::hbits(p.C);
     p.off_recv = (int)off;
     off += SM::recv(CL);
     p.off_zp = (int)off;

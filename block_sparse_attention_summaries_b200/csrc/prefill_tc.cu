@@ -983,18 +983,6 @@ bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void*
 
 // Sliding-window causal attention (window keys j in [i - window + 1, i]) of already rotated q/k
 // on the tensor cores: the short branch of the FreeSolo prefill, written to o.
-bsa_status window_attn_tc(const void* q, const void* k, const void* v, int B, int H, int Hk,
-                          int n, int d, int window, void* o, int* status, cudaStream_t st) {
-  TcParams p{};
-  p.B = B; p.Hq = H; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = 0;
-  p.o = o; p.lse = nullptr; p.status = status; p.mode = 1; p.window = window;
-  if (ceil_div(window - 1, kTiles) > kMaxKtc) return BSA_ERR_UNSUPPORTED;
-  bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
-  if (rc != BSA_OK) return rc;
-  BSA_LAUNCH_CHECK();
-  return BSA_OK;
-}
-
 // Long branch of the FreeSolo prefill on the tensor cores (mode 2), mixing into o.
 // Workspace: union counts [B * H * U] then lists [B * H * U][ucap], ucap = min(64 * 8, blocks).
 static int long_ucap(int n) { return min(64 * 8, ceil_div(n, kTiles)); }
