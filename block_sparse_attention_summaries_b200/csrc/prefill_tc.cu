@@ -1029,11 +1029,20 @@ bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq
   return G % 2 == 0;  // units are paired by head within one kv group
 }
 
+bsa_status sas_fwd_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hk, int n,
+                      int d, const int* idx, const int* count, int K, int gate, int norm,
+                      const float* scores, int scores_ld, void* o, float* lse, int* status,
+                      cudaStream_t st);
+
 bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hk, int n,
                       int d, int b, const int* idx, const int* count, int K, int gate, int norm,
                       const float* scores, int scores_ld, void* o, float* lse, int* status,
                       cudaStream_t st) {
   (void)b;
+  // up to 32 selected blocks: two unit pairs per CTA in ping-pong
+  const bsa_status pp = sas_fwd_tc(q, k, v, B, Hq, Hk, n, d, idx, count, K, gate, norm, scores,
+                                   scores_ld, o, lse, status, st);
+  if (pp != BSA_ERR_UNSUPPORTED) return pp;
   TcParams p{};
   p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = K;
   p.idx = idx; p.count = count; p.gate = gate; p.norm = norm;
