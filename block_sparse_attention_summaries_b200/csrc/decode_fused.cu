@@ -91,11 +91,8 @@ struct FusedParams {
   int row_ld;  // stride of the whole-row key copies (gather) in keys
   int ns;      // summary ring stages
   int nkv;     // K/V ring stages
-  int ng;      // groups per cluster (1, or 2 pipelined)
-  // dynamic shared-memory layout (byte offsets from the 1024-aligned base; per-group pieces at
-  // off + k * bytes)
-  int off_sum, off_kv, off_keys, off_sel, off_hbits, off_recv, off_zp, off_bar;
-  int keys_bytes, sel_bytes, recv_bytes;
+  // dynamic shared-memory layout (byte offsets from the 1024-aligned base)
+  int off_keys, off_sel, off_hbits, off_recv, off_zp, off_bar;
 };
 
 // ---- cluster helpers ---------------------------------------------------------------------
@@ -411,11 +408,6 @@ struct FusedSmem {
   __host__ __device__ static size_t zp(int b) { return MMA ? 0 : 2 * align_up((size_t)b * G * 4, 16); }
 };
 
-// One (batch, kv head) group of a cluster: its position, history and the CTA's slice of it.
-struct GroupCtx {
-  int valid, bi, kh, h0, pos, cur, nc, c_lo, rows, nsub;
-};
-
 template <typename T, typename TS, int D, int G, bool MMA>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -431,11 +423,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ int s_pick[kWarps][kMaxKf];
   __shared__ int s_sel[G][kMaxKf];
   __shared__ int s_nsel[G];
-  __shared__ int s_ublk[2][kMaxUnion];
-  __shared__ unsigned s_umask[2][kMaxUnion];
+  __shared__ uint32_t s_bits[kMaxWords];
+  __shared__ int s_ublk[kMaxUnion];
+  __shared__ unsigned s_umask[kMaxUnion];
   __shared__ uint32_t s_scratch[kWarps * 2 * kCandMax];  // select candidates / append partials
   __shared__ int s_kv_last[kMaxStages];  // the last K/V stage issued into each slot (-1: none)
-  __shared__ int s_U[2];
+  __shared__ int s_U;
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
@@ -445,820 +438,739 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = (int)cluster_rank();
   const int CL = (int)cluster_size();
-  const int NS = p.ns, NKV = p.nkv, NG = p.ng;
-  auto group_ctx = [&](int k) {
-    GroupCtx c{};
-    const int gi = (int)blockIdx.y * NG + k;
-    c.valid = k < NG && gi < p.B * p.Hk;
-    c.bi = c.valid ? gi / p.Hk : 0;
-    c.kh = c.valid ? gi % p.Hk : 0;
-    c.h0 = c.kh * G;
-    const int L = p.seq_lens ? min(p.seq_lens[c.bi], p.n) : p.n;
-    c.pos = L - 1;
-    c.cur = c.pos / b;
-    int nc = p.prefix_block > 0 ? ((c.pos / p.prefix_block) * p.prefix_block) / b : c.cur;
-    c.nc = c.valid ? max(0, min(nc, c.cur)) : 0;
-    c.c_lo = min(c.nc, rank * p.chunk);
-    c.rows = min(c.nc, c.c_lo + p.chunk) - c.c_lo;
-    c.nsub = (c.rows + kSub - 1) / kSub;
-    return c;
-  };
-  const GroupCtx g0 = group_ctx(0), g1 = group_ctx(1);
-  auto gctx = [&](int k) -> const GroupCtx& { return k == 0 ? g0 : g1; };
+  const int kh = blockIdx.y, bi = blockIdx.z;
+  const int h0 = kh * G;
+  const int L = p.seq_lens ? min(p.seq_lens[bi], p.n) : p.n;
+  const int pos = L - 1;
+  const int cur = pos / b;
+  int nc = p.prefix_block > 0 ? ((pos / p.prefix_block) * p.prefix_block) / b : cur;
+  nc = max(0, min(nc, cur));
+  const int NS = p.ns, NKV = p.nkv;
 
   using SM = FusedSmem<T, TS, D, G, MMA>;
-  TS* ring = reinterpret_cast<TS*>(smem + p.off_sum);  // summary ring, later the warp partials
-  unsigned char* kvbase = smem + p.off_kv;             // K/V stages (aliases the ring when NG = 1)
+  TS* ring = reinterpret_cast<TS*>(smem);  // region A: summary ring, then K/V ring, then partials
   TS* mean_k = static_cast<TS*>(p.mean_k);
   const int Gs = p.shared ? 1 : G;  // selections made per group
-  // group k's own scores; one buffer serves both groups (group 1 is scored after group 0's
-  // selection has read them, and no peer writes it)
-  auto s_keys = [&](int) { return reinterpret_cast<uint32_t*>(smem + p.off_keys); };
-  auto sel_buf = [&](int k) { return reinterpret_cast<uint32_t*>(smem + p.off_sel + k * p.sel_bytes); };
-  auto recv = [&](int k) { return reinterpret_cast<float*>(smem + p.off_recv + k * p.recv_bytes); };
+  uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);  // [G][chunk]
+  uint32_t* sel_buf = reinterpret_cast<uint32_t*>(smem + p.off_sel);  // whole rows / merge
   uint32_t* hbits = reinterpret_cast<uint32_t*>(smem + p.off_hbits);  // [Gs][nwords] selections
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);           // [CL][G][cols+2]
   float* zs = reinterpret_cast<float*>(smem + p.off_zp);
   float* ps = zs + align_up((size_t)b * G, 4);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   // bar[0 .. NS): summary stages; bar[NS .. NS + NKV): K/V stages
-  uint64_t* kvbar = bar + NS;
 
   if (tid == 0) {
     for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     for (int i = 0; i < kMaxStages; ++i) s_kv_last[i] = -1;
     s_abort = 0;
-    s_U[0] = s_U[1] = 0;
+    s_U = 0;
+  }
+  if (tid < G) {
+    s_m[tid] = -INFINITY;
+    s_l[tid] = 0.f;
   }
   __syncthreads();
   // every CTA of the cluster has started before any peer writes into its shared memory
   cluster_arrive_relaxed();
 
-  // ---- summary ring: the stages of group 0's slice, then group 1's, issued as slots free ---
-  const int nsub_tot = g0.nsub + g1.nsub;
-  auto issue_sub = [&](int J) {  // J-th stage of the whole sequence
-    const int k = J < g0.nsub ? 0 : 1;
-    const GroupCtx& c = gctx(k);
-    const int j = J - (k ? g0.nsub : 0);
-    const int r0 = c.c_lo + j * kSub;
-    const int nr = min(kSub, c.c_lo + c.rows - r0);
+  // ---- 1. score my slice of the history blocks --------------------------------------------
+  const int c_lo = min(nc, rank * p.chunk);
+  const int c_hi = min(nc, c_lo + p.chunk);
+  const int rows = c_hi - c_lo;
+  const int nsub = (rows + kSub - 1) / kSub;
+  const TS* mk = mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
+  auto issue_sub = [&](int j) {
+    const int r0 = c_lo + j * kSub;
+    const int nr = min(kSub, c_hi - r0);
     const uint32_t bytes = (uint32_t)(nr * D * sizeof(TS));
-    const TS* src = mean_k + ((size_t)(c.bi * p.Hk + c.kh) * p.C + r0) * D;
-    mbar_arrive_expect_tx(&bar[J % NS], bytes);
-    bulk_g2s(ring + (size_t)(J % NS) * kSub * D, src, bytes, &bar[J % NS]);
+    mbar_arrive_expect_tx(&bar[j % NS], bytes);
+    bulk_g2s(ring + (size_t)(j % NS) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j % NS]);
   };
   int sub_issued = 0;  // (thread 0) summary stages issued so far
   if (tid == 0)
-    for (; sub_issued < min(nsub_tot, NS); ++sub_issued) issue_sub(sub_issued);
-
-  // ---- 1. score group k's slice of the history blocks --------------------------------------
-  auto score_group = [&](int k) {
-    const GroupCtx& c = gctx(k);
-    const int base = k ? g0.nsub : 0;
-    float qv[G][EPL];
+    for (; sub_issued < min(nsub, NS); ++sub_issued) issue_sub(sub_issued);
+  float qv[G][EPL];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float tmp[EPL];
-      load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)c.bi * Hq + c.h0 + g) * D + lane * EPL,
-                       tmp);
+  for (int g = 0; g < G; ++g) {
+    float tmp[EPL];
+    load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + g) * D + lane * EPL,
+                     tmp);
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
-    }
-    const float scale = rsqrtf((float)D);
-    const int my_r = lane / G, my_g = lane % G;
-    const float lam_h = p.lam ? p.lam[c.h0 + my_g] : 0.f;
-    const float inv2sig = p.lam ? 0.5f / p.sig[c.h0 + my_g] : 0.f;
-    uint32_t* keys = s_keys(k);
-    for (int j = 0; j < c.nsub; ++j) {
-      const int J = base + j;
-      if (!s_abort && !mbar_wait_bounded(&bar[J % NS], (J / NS) & 1)) s_abort = 1;
-      __syncthreads();
-      if (!s_abort) {
-        const int r0 = j * kSub;
-        const int nr = min(kSub, c.rows - r0);
-        const TS* sb = ring + (size_t)(J % NS) * kSub * D;
-        for (int t0 = warp * R; t0 < nr; t0 += kWarps * R) {
-          float a[32];
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            float x[EPL];
-            if (t0 + r < nr) {
-              load_vec<TS, EPL>(sb + (size_t)(t0 + r) * D + lane * EPL, x);
-            } else {
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) x[e] = 0.f;
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              float s = 0.f;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) s = fmaf(qv[g][e], x[e], s);
-              a[r * G + g] = s;
-            }
-          }
-          warp_transpose_reduce32(a, lane);
-          const int t = t0 + my_r;
-          float s = a[0] * scale;
-          if (p.lam && t < nr) {
-            const size_t row = (size_t)(c.bi * p.Hk + c.kh) * p.C + c.c_lo + r0 + t;
-            s += lam_h * p.max_norm[row] * erff(((float)c.pos - p.centre[row]) * inv2sig);
-          }
-          if (p.shared) {  // mean over the G lanes of this row (lane = my_r * G + my_g)
-#pragma unroll
-            for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            s *= 1.f / (float)G;
-          }
-          if (t < nr && my_g < Gs) keys[my_g * p.chunk + r0 + t] = order_key(s);
-        }
-      }
-      if (J + NS < nsub_tot) {  // the stage is drained: refill it with the next of the sequence
-        __syncthreads();
-        if (tid == 0 && !s_abort) issue_sub(sub_issued++);
-      }
-    }
+    for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
+  }
+  const float scale = rsqrtf((float)D);
+  const int my_r = lane / G, my_g = lane % G;
+  const float lam_h = p.lam ? p.lam[h0 + my_g] : 0.f;
+  const float inv2sig = p.lam ? 0.5f / p.sig[h0 + my_g] : 0.f;
+  for (int j = 0; j < nsub; ++j) {
+    if (!s_abort && !mbar_wait_bounded(&bar[j % NS], (j / NS) & 1)) s_abort = 1;
     __syncthreads();
-  };
-
-  // ---- 2. Top-K per head of group k and the union of the selections ----------------------
-  uint32_t* ck = s_scratch + warp * 2 * kCandMax;
-  int* cp = reinterpret_cast<int*>(ck + kCandMax);
-  auto select_group = [&](int k) {
-    const GroupCtx& c = gctx(k);
-    const int rows = c.rows;
-    uint32_t* keys_k = s_keys(k);
-    uint32_t* sb = sel_buf(k);
-    if (p.gather) {
-      // push my slice of every selecting head's keys into every CTA's whole-row copy
-      const int nvec = rows >> 2, tail = rows & 3;
-      const int per_g = CL * (nvec + tail);
-      for (int e = tid; e < Gs * per_g; e += kThreads) {
-        const int g = e / per_g, rem = e % per_g;
-        const int r = rem / (nvec + tail), v = rem % (nvec + tail);
-        const uint32_t* src = keys_k + g * p.chunk;
-        uint32_t* dst = sb + (size_t)g * p.row_ld + c.c_lo;
-        if (v < nvec) {
-          const uint4 x = *reinterpret_cast<const uint4*>(src + 4 * v);
-          st_dsmem_v4(dsmem_addr(dst + 4 * v, r), x);
-        } else {
-          const int t = 4 * nvec + (v - nvec);
-          st_dsmem_u32(dsmem_addr(dst + t, r), src[t]);
-        }
-      }
-      cluster_sync();
-      for (int g = warp; g < Gs; g += kWarps) {
-        const int cnt = warp_select(sb + (size_t)g * p.row_ld, c.nc, K, lane, s_pick[warp], ck, cp);
-        for (int j = lane; j < cnt; j += 32) s_sel[g][j] = s_pick[warp][j];
-        if (lane == 0) s_nsel[g] = cnt;
-      }
-    } else {
-      // local Top-K per head, pushed into every CTA's merge buffer at slot rank * K
-      uint32_t* m_key = sb;
-      int* m_idx = reinterpret_cast<int*>(sb) + G * CL * K;
-      for (int g = warp; g < Gs; g += kWarps) {
-        const uint32_t* kk = keys_k + g * p.chunk;
-        const int cnt = warp_select(kk, rows, K, lane, s_pick[warp], ck, cp);
-        for (int e = lane; e < CL * K; e += 32) {
-          const int r = e / K, j = e % K;
-          const uint32_t key = j < cnt ? kk[s_pick[warp][j]] : 0u;
-          const int gi = j < cnt ? c.c_lo + s_pick[warp][j] : -1;  // -1: empty slot
-          const int slot = g * CL * K + rank * K + j;
-          st_dsmem_u32(dsmem_addr(&m_key[slot], r), key);
-          st_dsmem_u32(dsmem_addr(&m_idx[slot], r), (uint32_t)gi);
-        }
-      }
-      cluster_sync();
-      for (int g = warp; g < Gs; g += kWarps) {
-        // empty slots carry key 0 and index -1: compact the valid ones first (index order kept:
-        // slot order is rank order and each rank's slots are ascending)
-        uint32_t* mk_g = m_key + g * CL * K;
-        int* mi_g = m_idx + g * CL * K;
-        int nvalid = 0;
-        for (int e0 = 0; e0 < CL * K; e0 += 32) {
-          const int e = e0 + lane;
-          const bool ok = e < CL * K && mi_g[e] >= 0;
-          const uint32_t kk2 = ok ? mk_g[e] : 0u;
-          const int ii = ok ? mi_g[e] : 0;
-          const unsigned bal = __ballot_sync(0xffffffffu, ok);
-          __syncwarp();
-          if (ok) {
-            const int at = nvalid + __popc(bal & ((1u << lane) - 1u));
-            mk_g[at] = kk2;
-            mi_g[at] = ii;
-          }
-          nvalid += __popc(bal);
-          __syncwarp();
-        }
-        const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[warp], ck, cp);
-        for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[warp][j]];
-        if (lane == 0) s_nsel[g] = cnt;
-      }
-    }
-    __syncthreads();
-
-    // every selection as a bitmap over the history blocks; one warp compacts the OR of the
-    // bitmaps into the sorted union and takes each entry's head mask from the same words
-    const int nwords = (c.nc + 31) / 32;
-    for (int g = warp; g < Gs; g += kWarps) {
-      uint32_t* hb = hbits + g * nwords;
-      for (int w = lane; w < nwords; w += 32) hb[w] = 0u;
-      __syncwarp();
-      for (int j = lane; j < s_nsel[g]; j += 32) {
-        const int x = s_sel[g][j];
-        atomicOr(&hb[x >> 5], 1u << (x & 31));
-      }
-    }
-    if (rank == 0 && c.valid) {  // optional outputs: the selection of every head
-      for (int e = tid; e < G * K; e += kThreads) {
-        const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
-        const size_t row = (size_t)c.bi * Hq + c.h0 + g;
-        if (p.idx) p.idx[row * K + j] = j < s_nsel[gs] ? s_sel[gs][j] : -1;
-        if (p.count && j == 0) p.count[row] = s_nsel[gs];
-      }
-    }
-    __syncthreads();
-    if (warp == 0) {  // a contiguous run of words per lane, prefix sums of their union counts
-      const int per = (nwords + 31) / 32;
-      const int w0 = min(nwords, lane * per), w1 = min(nwords, w0 + per);
-      int mine = 0;
-      for (int w = w0; w < w1; ++w) {
-        uint32_t u = 0u;
-        for (int g = 0; g < Gs; ++g) u |= hbits[g * nwords + w];
-        mine += __popc(u);
-      }
-      int incl = mine;
+    if (!s_abort) {
+      const int r0 = j * kSub;
+      const int nr = min(kSub, rows - r0);
+      const TS* base = ring + (size_t)(j % NS) * kSub * D;
+      for (int t0 = warp * R; t0 < nr; t0 += kWarps * R) {
+        float a[32];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int at = incl - mine;
-      for (int w = w0; w < w1; ++w) {
-        uint32_t hw[G];
-        uint32_t u = 0u;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          hw[g] = g < Gs ? hbits[g * nwords + w] : 0u;
-          u |= hw[g];
-        }
-        while (u) {
-          const int bit = __ffs(u) - 1;
-          u &= u - 1;
-          unsigned m = 0u;
-#pragma unroll
-          for (int g = 0; g < G; ++g) m |= ((hw[g] >> bit) & 1u) << g;
-          s_ublk[k][at] = w * 32 + bit;
-          s_umask[k][at] = p.shared ? (1u << G) - 1u : m;
-          ++at;
-        }
-      }
-      if (lane == 31) {
-        // the current block, always kept, follows every history block (no block for a group
-        // the cluster does not have)
-        s_ublk[k][incl] = c.cur;
-        s_umask[k][incl] = (1u << G) - 1u;
-        s_U[k] = c.valid ? incl + 1 : 0;
-      }
-    }
-    __syncthreads();
-  };
-
-  // ---- 3. attention: stages of both groups in one sequence ---------------------------------
-  // MMA path: 16-token slices (history entries 4, the current block ceil(tok / 16)); CTA r takes
-  // slices [r S / CL, (r + 1) S / CL) of its group; a stage holds four consecutive slices (K then
-  // V tiles, 64 rows x 128 bytes per 64-column half, 128-byte swizzle); stage I of the sequence is
-  // taken by warp group I & 1, which owns NKV / 2 slots and refills them itself
-  const int nper = NKV / 2;
-  auto slot_of = [&](int I) { return (I & 1) + 2 * ((I >> 1) % nper); };
-  auto parity_of = [&](int I) { return (uint32_t)(((I >> 1) / nper) & 1); };
-  const size_t tl = SM::kv_tile(b);
-  auto ktile = [&](int st) { return kvbase + (size_t)st * 2 * tl; };
-  auto vtile = [&](int st) { return kvbase + (size_t)st * 2 * tl + tl; };
-  struct SliceRange { int s_hist, tok_cur, s_begin, s_end, nst; };
-  auto slice_range = [&](int k) {
-    SliceRange sr;
-    const GroupCtx& c = gctx(k);
-    const int U = s_U[k];
-    sr.tok_cur = c.pos - c.cur * b + 1;
-    sr.s_hist = U > 0 ? 4 * (U - 1) : 0;
-    const int S_tot = U > 0 ? sr.s_hist + (sr.tok_cur + kSlice - 1) / kSlice : 0;
-    sr.s_begin = (int)(((long long)rank * S_tot) / CL);
-    sr.s_end = (int)(((long long)(rank + 1) * S_tot) / CL);
-    sr.nst = (sr.s_end - sr.s_begin + 3) / 4;
-    return sr;
-  };
-  SliceRange sr0{}, sr1{};  // filled once each union is known
-  auto issue_kv = [&](int I) {  // stage I of the sequence (group 0's stages, then group 1's)
-    const int k = I < sr0.nst ? 0 : 1;
-    const SliceRange& sr = k ? sr1 : sr0;
-    const GroupCtx& c = gctx(k);
-    const int i = I - (k ? sr0.nst : 0);
-    const int st = slot_of(I);
-    s_kv_last[st] = I;
-    const int first = sr.s_begin + 4 * i;
-    const int nsl = min(4, sr.s_end - first);
-    const int row0 = (c.bi * p.Hk + c.kh) * p.n;
-    mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
-    for (int w = 0; w < nsl; ++w) {
-      const int s = first + w;
-      const int blk = s < sr.s_hist ? s_ublk[k][s >> 2] : c.cur;
-      const int tok0 = s < sr.s_hist ? (s & 3) * kSlice : (s - sr.s_hist) * kSlice;
-      const int y = row0 + blk * b + tok0;
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        tc::tma_load_2d(ktile(st) + hf * 8192 + w * kSlice * 128, &tmk, hf * 64, y, &kvbar[st]);
-        tc::tma_load_2d(vtile(st) + hf * 8192 + w * kSlice * 128, &tmv, hf * 64, y, &kvbar[st]);
-      }
-    }
-  };
-  int kv_next = 0;  // (thread 0) first stage of the sequence not issued among the initial NKV
-
-  float* wpart = reinterpret_cast<float*>(smem + p.off_sum);  // [warp][G][D+2] after scoring
-
-  auto attend_group = [&](int k) {
-    const GroupCtx& c = gctx(k);
-    if constexpr (kMma) {
-      const SliceRange& sr = k ? sr1 : sr0;
-      const int I0 = k ? sr0.nst : 0;
-      const int I_end = I0 + sr.nst;
-      const int I_tot = sr0.nst + sr1.nst;
-      const int grp = warp >> 2, wg = warp & 3;
-      if (p.append && rank == CL - 1 && c.valid) {
-        // the block being filled: its summary rewritten from its keys in global memory by the
-        // last CTA while the group's K/V stages are in flight; every row is requested at once (a
-        // warp takes rows warp, warp + 8, ...: at most 8 of a 64-token block)
-        const T* kb = static_cast<const T*>(p.k) +
-                      ((size_t)(c.bi * p.Hk + c.kh) * p.n + (size_t)c.cur * b) * D;
-        float x[8][EPL];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = warp + kWarps * u;
-          if (t < sr.tok_cur) {
-            load_vec<T, EPL>(kb + (size_t)t * D + lane * EPL, x[u]);
+        for (int r = 0; r < R; ++r) {
+          float x[EPL];
+          if (t0 + r < nr) {
+            load_vec<TS, EPL>(base + (size_t)(t0 + r) * D + lane * EPL, x);
           } else {
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) x[u][e] = 0.f;
+            for (int e = 0; e < EPL; ++e) x[e] = 0.f;
           }
-        }
-        float cs[EPL];
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) cs[e] = 0.f;
-        float nmax = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          float sq = 0.f;
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) {
-            cs[e] += x[u][e];
-            sq = fmaf(x[u][e], x[u][e], sq);
-          }
-          nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));  // rows past the block add 0
-        }
-        float* part = reinterpret_cast<float*>(s_scratch);  // [kWarps][D]
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) part[warp * D + lane * EPL + e] = cs[e];
-        if (lane == 0) s_red[warp] = nmax;
-        __syncthreads();
-        const size_t row = (size_t)(c.bi * p.Hk + c.kh) * p.C + c.cur;
-        for (int col = tid; col < D; col += kThreads) {
-          float sum = 0.f;
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) sum += part[w * D + col];
-          mean_k[row * D + col] = Elem<TS>::from_f(sum / (float)sr.tok_cur);
-        }
-        if (tid == 0) {
-          float nm = 0.f;
-          for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
-          if (p.max_norm) p.max_norm[row] = nm;
-          if (p.centre)
-            p.centre[row] = 0.5f * (float)(c.cur * b) + 0.5f * (float)(c.cur * b + sr.tok_cur - 1);
-        }
-        __syncthreads();
-      }
-      // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
-      const int grow = lane >> 2, tig = lane & 3;
-      uint32_t qa0[D / 16], qa1[D / 16];
-      {
-        const float qs = rsqrtf((float)D) * kLog2e;
-        const T* qrow = static_cast<const T*>(p.q) + ((size_t)c.bi * Hq + c.h0 + min(grow, G - 1)) * D;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-          if (grow < G) {
-            x0 = Elem<T>::to_f(qrow[16 * ks + 2 * tig]) * qs;
-            x1 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 1]) * qs;
-            x2 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 8]) * qs;
-            x3 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 9]) * qs;
-          }
-          qa0[ks] = pack_bf16(x0, x1);
-          qa1[ks] = pack_bf16(x2, x3);
-        }
-      }
-      // O^T accumulators: m-tile mt covers d rows 16 mt .. 16 mt + 15, columns are heads
-      float oacc[D / 16][4];
-#pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) oacc[cc][0] = oacc[cc][1] = oacc[cc][2] = oacc[cc][3] = 0.f;
-      float m_run = -INFINITY, l_part = 0.f;
-      const int n_run = s_abort ? 0 : I_end;  // nothing was issued after an earlier timeout
-      for (int I = I0 + (((I0 & 1) != grp) ? 1 : 0); I < n_run; I += 2) {
-        const int st = slot_of(I);
-        const int i = I - I0;
-        // group-uniform decision: the OR over the group's four warps of "my wait ran out"
-        const int bad = mbar_wait_bounded(&kvbar[st], parity_of(I)) ? 0 : 1;
-        int any_bad;
-        asm volatile(
-            "{\n\t.reg .pred pin, pout;\n\t"
-            "setp.ne.s32 pin, %1, 0;\n\t"
-            "barrier.red.or.pred pout, %2, 128, pin;\n\t"
-            "selp.s32 %0, 1, 0, pout;\n\t}"
-            : "=r"(any_bad)
-            : "r"(bad), "r"(1 + grp)
-            : "memory");
-        if (any_bad) {
-          s_abort = 1;
-          break;
-        }
-        const int s = sr.s_begin + 4 * i + wg;  // this warp's slice
-        if (s < sr.s_end) {
-          const int m = s < sr.s_hist ? s_ublk[k][s >> 2] : c.cur;
-          const unsigned hm = s < sr.s_hist ? s_umask[k][s >> 2] : (1u << G) - 1u;
-          const int tok0 = s < sr.s_hist ? (s & 3) * kSlice : (s - sr.s_hist) * kSlice;
-          const int tv = m == c.cur ? min(kSlice, sr.tok_cur - tok0) : kSlice;  // valid tokens
-          const unsigned char* kt = ktile(st);
-          const unsigned char* vt = vtile(st);
-          const int t0 = wg * kSlice;  // this warp's 16 rows of the stage tile
-          // S = Q K^T over two 8-token tiles
-          float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const int hf = ks >> 2, ch = (ks & 3) * 2;
-              const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
-              const uint32_t b0 =
-                  *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
-              const uint32_t b1 =
-                  *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
-              mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
-            }
-          }
-          // masks, per-row online softmax (row = head grow; the quad shares the row)
-          const bool head_on = grow < G && ((hm >> grow) & 1u);
-          float mx = -INFINITY;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int t = 8 * nt + 2 * tig + e;
-              if (!head_on || t >= tv) sfr[nt][e] = -INFINITY;
-              mx = fmaxf(mx, sfr[nt][e]);
-            }
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
-          if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
-            corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
-            m_run = mx;
-            l_part *= corr;
-          }
-          // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
-          const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
-          const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
-          if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
-#pragma unroll
-            for (int cc = 0; cc < D / 16; ++cc) {
-              oacc[cc][0] *= corr_a;
-              oacc[cc][1] *= corr_b;
-              oacc[cc][2] *= corr_a;
-              oacc[cc][3] *= corr_b;
-            }
-          }
-          float pv[2][2];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float z = sfr[nt][e];
-              pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
-              l_part += pv[nt][e];
-            }
-          // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
-          const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
-          const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
-          // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
-#pragma unroll
-          for (int mt = 0; mt < D / 16; ++mt) {
-            const int mi = lane >> 3, rr = lane & 7;
-            const int tokr = t0 + (mi >> 1) * 8 + rr;
-            const int chunk = 2 * mt + (mi & 1);  // 16-byte chunk along d (0..D/8-1)
-            const int hf = chunk >> 3, cin = chunk & 7;
-            const uint32_t addr =
-                smem_u32(vt + hf * 8192 + tokr * 128 + ((cin ^ (tokr & 7)) << 4));
-            uint32_t v0, v1, v2, v3;
-            ldsm_x4_trans(addr, v0, v1, v2, v3);
-            mma_16816(oacc[mt], v0, v1, v2, v3, pb0, pb1);
-          }
-        }
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
-        if (wg == 0 && lane == 0 && I + NKV < I_tot) issue_kv(I + NKV);
-      }
-      __syncthreads();
-      if (s_abort && tid == 0) {
-        // copies still in flight: the last stage issued into each slot; waiting on its own phase
-        // parity returns at once if it already landed
-        for (int st = 0; st < NKV; ++st)
-          if (s_kv_last[st] >= 0)
-            (void)mbar_wait_bounded(&kvbar[st], parity_of(s_kv_last[st]), 1u << 12);
-        report_timeout(p.status, 2);
-      }
-      __syncthreads();
-      // warp partials (rows < G): m, l and o
-      l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-      l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-      if (grow < G && tig == 0) {
-        float* wp = wpart + ((size_t)warp * G + grow) * (D + 2);
-        wp[D] = m_run;
-        wp[D + 1] = l_part;
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {  // O^T element (d, head 2 tig + e)
-        const int hh = 2 * tig + e;
-        if (hh < G) {
-          float* wp = wpart + ((size_t)warp * G + hh) * (D + 2);
-#pragma unroll
-          for (int mt = 0; mt < D / 16; ++mt) {
-            wp[16 * mt + grow] = oacc[mt][e];
-            wp[16 * mt + grow + 8] = oacc[mt][2 + e];
-          }
-        }
-      }
-      __syncthreads();
-    } else {
-      // fp32 / other block sizes (one group per cluster): scalar FMAs; CTA r takes union entries
-      // r, r + CL, ...; warps split each block's tokens, one CTA-wide softmax per block
-      const int U = s_U[k];
-      const int ne = rank < U ? (U - rank + CL - 1) / CL : 0;
-      auto entry_tokens = [&](int m) { return m == c.cur ? c.pos - c.cur * b + 1 : b; };
-      T* kbuf[2] = {reinterpret_cast<T*>(kvbase), reinterpret_cast<T*>(kvbase + 2 * tl)};
-      T* vbuf[2] = {reinterpret_cast<T*>(kvbase + tl), reinterpret_cast<T*>(kvbase + 3 * tl)};
-      const T* kbase = static_cast<const T*>(p.k) + (size_t)(c.bi * p.Hk + c.kh) * p.n * D;
-      const T* vbase = static_cast<const T*>(p.v) + (size_t)(c.bi * p.Hk + c.kh) * p.n * D;
-      auto issue_blk = [&](int i) {
-        const int m = s_ublk[k][rank + i * CL];
-        const uint32_t bytes = (uint32_t)(entry_tokens(m) * D * sizeof(T));
-        const int st = i & 1;
-        mbar_arrive_expect_tx(&kvbar[st], 2 * bytes);
-        bulk_g2s(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st]);
-        bulk_g2s(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st]);
-      };
-      if (tid < G) {
-        s_m[tid] = -INFINITY;
-        s_l[tid] = 0.f;
-      }
-      if (tid == 0 && !s_abort) {
-        fence_proxy_async();
-        if (ne > 0) issue_blk(0);
-        if (ne > 1) issue_blk(1);
-      }
-      __syncthreads();
-      constexpr int CG = D / 2;
-      constexpr int TP = kThreads / CG;
-      float qa[G][EPL];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float tmp[EPL];
-        load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)c.bi * Hq + c.h0 + g) * D + lane * EPL,
-                         tmp);
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) qa[g][e] = tmp[e] * rsqrtf((float)D) * kLog2e;
-      }
-      const int cg = tid % CG, tp = tid / CG;
-      float acc[G][2];
-#pragma unroll
-      for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
-      int i_stop = ne;
-      const int n_run = s_abort ? 0 : ne;  // nothing was issued after an earlier timeout
-      for (int i = 0; i < n_run; ++i) {
-        const int st = i & 1;
-        const int m = s_ublk[k][rank + i * CL];
-        const unsigned hm = s_umask[k][rank + i * CL];
-        const int tok = entry_tokens(m);
-        if (!s_abort && !mbar_wait_bounded(&kvbar[st], (i >> 1) & 1)) s_abort = 1;
-        __syncthreads();
-        if (s_abort) {
-          i_stop = i;
-          break;
-        }
-        const T* kt = kbuf[st];
-        const T* vt = vbuf[st];
-        for (int t0 = warp * R; t0 < tok; t0 += kWarps * R) {
-          float a[32];
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            float x[EPL];
-            if (t0 + r < tok) {
-              load_vec<T, EPL>(kt + (size_t)(t0 + r) * D + lane * EPL, x);
-            } else {
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) x[e] = 0.f;
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-              float sacc = 0.f;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) sacc = fmaf(qa[g][e], x[e], sacc);
-              a[r * G + g] = sacc;
-            }
-          }
-          warp_transpose_reduce32(a, lane);
-          const int t = t0 + lane / G, g = lane % G;
-          if (t < tok) zs[t * G + g] = ((hm >> g) & 1u) ? a[0] : -INFINITY;
-        }
-        if (p.append && m == c.cur) {
-          for (int col = tid; col < D; col += kThreads) {
-            float sum = 0.f;
-            for (int t = 0; t < tok; ++t) sum += Elem<T>::to_f(kt[(size_t)t * D + col]);
-            mean_k[((size_t)(c.bi * p.Hk + c.kh) * p.C + c.cur) * D + col] =
-                Elem<TS>::from_f(sum / (float)tok);
-          }
-          float nmax = 0.f;
-          for (int t = warp; t < tok; t += kWarps) {
-            float x[EPL];
-            load_vec<T, EPL>(kt + (size_t)t * D + lane * EPL, x);
-            float sq = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) sq = fmaf(x[e], x[e], sq);
-            nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
-          }
-          if (lane == 0) s_red[warp] = nmax;
-        }
-        __syncthreads();
-        if (p.append && m == c.cur && tid == 0) {
-          float nm = 0.f;
-          for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
-          const size_t row = (size_t)(c.bi * p.Hk + c.kh) * p.C + c.cur;
-          if (p.max_norm) p.max_norm[row] = nm;
-          if (p.centre) p.centre[row] = 0.5f * (float)(c.cur * b) + 0.5f * (float)(c.cur * b + tok - 1);
-        }
-        for (int g = warp; g < G; g += kWarps) {
-          float mx = -INFINITY;
-          for (int t = lane; t < tok; t += 32) mx = fmaxf(mx, zs[t * G + g]);
-          mx = warp_max(mx);
-          const float m_old = s_m[g];
-          const float m_new = fmaxf(m_old, mx);
-          float sum = 0.f;
-          for (int t = lane; t < tok; t += 32) {
-            const float pvv = (m_new == -INFINITY) ? 0.f : exp2f(zs[t * G + g] - m_new);
-            ps[t * G + g] = pvv;
-            sum += pvv;
-          }
-          sum = warp_sum(sum);
-          if (lane == 0) {
-            const float corr = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
-            s_corr[g] = corr;
-            s_l[g] = s_l[g] * corr + sum;
-            s_m[g] = m_new;
-          }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          acc[g][0] *= s_corr[g];
-          acc[g][1] *= s_corr[g];
-        }
-        for (int t = tp; t < tok; t += TP) {
-          float vv[2];
-          load_vec<T, 2>(vt + (size_t)t * D + 2 * cg, vv);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float pw = ps[t * G + g];
-            acc[g][0] = fmaf(pw, vv[0], acc[g][0]);
-            acc[g][1] = fmaf(pw, vv[1], acc[g][1]);
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) s = fmaf(qv[g][e], x[e], s);
+            a[r * G + g] = s;
           }
         }
-        __syncthreads();
-        if (tid == 0 && i + 2 < ne) issue_blk(i + 2);
-      }
-      if (s_abort && tid == 0 && n_run > 0) {
-        // copies in flight: stages i_stop and i_stop + 1 (if issued), each on its own parity
-        for (int j = i_stop; j < min(ne, i_stop + 2); ++j)
-          (void)mbar_wait_bounded(&kvbar[j & 1], (j >> 1) & 1, 1u << 12);
-        report_timeout(p.status, 2);
-      }
-      __syncthreads();
-      // token partitions tp -> "warp partial" slots 0..TP-1 with the shared (m, l)
-      for (int e = tid; e < kWarps * G * (D + 2); e += kThreads) wpart[e] = 0.f;
-      __syncthreads();
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float* wp = wpart + ((size_t)tp * G + g) * (D + 2);
-        wp[2 * cg] = acc[g][0];
-        wp[2 * cg + 1] = acc[g][1];
-        if (cg == 0) {
-          wp[D] = s_m[g];
-          wp[D + 1] = tp == 0 ? s_l[g] : 0.f;
+        warp_transpose_reduce32(a, lane);
+        const int t = t0 + my_r;
+        float s = a[0] * scale;
+        if (p.lam && t < nr) {
+          const size_t row = (size_t)(bi * p.Hk + kh) * p.C + c_lo + r0 + t;
+          s += lam_h * p.max_norm[row] * erff(((float)pos - p.centre[row]) * inv2sig);
         }
-      }
-      for (int w = TP + tid; w < kWarps; w += kThreads)  // unused slots: empty
-        for (int g = 0; g < G; ++g) wpart[((size_t)w * G + g) * (D + 2) + D] = -INFINITY;
-      __syncthreads();
-    }
-  };
-
-  // ---- 4. merge the warps, push column slices to their owners, finish ---------------------
-  const int cols = D / CL;
-  auto merge_group = [&](int k) {
-    const GroupCtx& c = gctx(k);
-    float* rv = recv(k);
-    // per head: combined max over warps, then weights
-    for (int g = warp; g < G; g += kWarps) {
-      float M = -INFINITY;
-      if (lane < kWarps) M = wpart[((size_t)lane * G + g) * (D + 2) + D];
-      M = warp_max(M);
-      float lsum = 0.f;
-      if (lane < kWarps) {
-        const float mw = wpart[((size_t)lane * G + g) * (D + 2) + D];
-        const float w = mw == -INFINITY ? 0.f : exp2f(mw - M);
-        lsum = w * wpart[((size_t)lane * G + g) * (D + 2) + D + 1];
-      }
-      lsum = warp_sum(lsum);
-      if (lane == 0) {
-        s_m[g] = M;
-        s_l[g] = lsum;
-      }
-    }
-    __syncthreads();
-    for (int e = tid; e < G * D; e += kThreads) {
-      const int g = e / D, col = e % D;
-      const float M = s_m[g];
-      float osum = 0.f;
+        if (p.shared) {  // mean over the G lanes of this row (lane = my_r * G + my_g)
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = wpart[((size_t)w * G + g) * (D + 2) + D];
-        if (mw != -INFINITY) osum = fmaf(exp2f(mw - M), wpart[((size_t)w * G + g) * (D + 2) + col], osum);
+          for (int o = 1; o < G; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          s *= 1.f / (float)G;
+        }
+        if (t < nr && my_g < Gs) s_keys[my_g * p.chunk + r0 + t] = order_key(s);
       }
-      // push to the owner of this column: recv[rank][g][col % cols], plus (m, l)
-      const int owner = col / cols;
-      float* slot = rv + ((size_t)rank * G + g) * (cols + 2);
-      st_dsmem_f32(dsmem_addr(&slot[col % cols], owner), osum);
-      if (col % cols == 0) {
-        st_dsmem_f32(dsmem_addr(&slot[cols], owner), M);
-        st_dsmem_f32(dsmem_addr(&slot[cols + 1], owner), s_l[g]);
+    }
+    if (j + NS < nsub) {  // the stage is drained: refill it
+      __syncthreads();
+      if (tid == 0 && !s_abort) issue_sub(sub_issued++);
+    }
+  }
+  __syncthreads();
+  if (s_abort && tid == 0) {
+    // summary copies still in flight: the last stage issued into each slot, on its own parity
+    for (int j = max(0, sub_issued - NS); j < sub_issued; ++j)
+      (void)mbar_wait_bounded(&bar[j % NS], (j / NS) & 1, 1u << 12);
+    report_timeout(p.status, 1);
+  }
+
+  // ---- 2. Top-K per head (per group when shared) -----------------------------------------
+  uint32_t* ck = s_scratch + warp * 2 * kCandMax;
+  int* cp = reinterpret_cast<int*>(ck + kCandMax);
+  cluster_wait();  // every peer has started: DSMEM stores may begin
+  if (p.gather) {
+    // push my slice of every selecting head's keys into every CTA's whole-row copy
+    const int nvec = rows >> 2, tail = rows & 3;
+    const int per_g = CL * (nvec + tail);
+    for (int e = tid; e < Gs * per_g; e += kThreads) {
+      const int g = e / per_g, rem = e % per_g;
+      const int r = rem / (nvec + tail), v = rem % (nvec + tail);
+      const uint32_t* src = s_keys + g * p.chunk;
+      uint32_t* dst = sel_buf + (size_t)g * p.row_ld + c_lo;
+      if (v < nvec) {
+        const uint4 x = *reinterpret_cast<const uint4*>(src + 4 * v);
+        st_dsmem_v4(dsmem_addr(dst + 4 * v, r), x);
+      } else {
+        const int t = 4 * nvec + (v - nvec);
+        st_dsmem_u32(dsmem_addr(dst + t, r), src[t]);
       }
     }
     cluster_sync();
-    if (c.valid) {
-      for (int e = tid; e < G * cols; e += kThreads) {
-        const int g = e / cols, cc = e % cols, col = rank * cols + cc;
-        float M = -INFINITY;
-        for (int r = 0; r < CL; ++r) M = fmaxf(M, rv[((size_t)r * G + g) * (cols + 2) + cols]);
-        float lsum = 0.f, osum = 0.f;
-        for (int r = 0; r < CL; ++r) {
-          const float* slot = rv + ((size_t)r * G + g) * (cols + 2);
-          const float mr = slot[cols];
-          if (mr == -INFINITY) continue;
-          const float w = exp2f(mr - M);
-          lsum = fmaf(w, slot[cols + 1], lsum);
-          osum = fmaf(w, slot[cc], osum);
-        }
-        const size_t row = (size_t)c.bi * Hq + c.h0 + g;
-        static_cast<T*>(p.o)[row * D + col] = Elem<T>::from_f(osum / lsum);
-        if (col == 0 && p.lse) p.lse[row] = (M + log2f(lsum)) * kLn2;
+    for (int g = warp; g < Gs; g += kWarps) {
+      const int cnt = warp_select(sel_buf + (size_t)g * p.row_ld, nc, K, lane, s_pick[warp], ck, cp);
+      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = s_pick[warp][j];
+      if (lane == 0) s_nsel[g] = cnt;
+    }
+  } else {
+    // local Top-K per head, pushed into every CTA's merge buffer at slot rank * K
+    uint32_t* m_key = sel_buf;
+    int* m_idx = reinterpret_cast<int*>(sel_buf) + G * CL * K;
+    for (int g = warp; g < Gs; g += kWarps) {
+      const uint32_t* keys = s_keys + g * p.chunk;
+      const int cnt = warp_select(keys, rows, K, lane, s_pick[warp], ck, cp);
+      for (int e = lane; e < CL * K; e += 32) {
+        const int r = e / K, j = e % K;
+        const uint32_t key = j < cnt ? keys[s_pick[warp][j]] : 0u;
+        const int gi = j < cnt ? c_lo + s_pick[warp][j] : -1;  // -1: empty slot
+        const int slot = g * CL * K + rank * K + j;
+        st_dsmem_u32(dsmem_addr(&m_key[slot], r), key);
+        st_dsmem_u32(dsmem_addr(&m_idx[slot], r), (uint32_t)gi);
       }
     }
-    __syncthreads();  // the partials and the peers' pushes may be overwritten by the next group
-  };
+    cluster_sync();
+    for (int g = warp; g < Gs; g += kWarps) {
+      // empty slots carry key 0 and index -1: compact the valid ones first (index order kept:
+      // slot order is rank order and each rank's slots are ascending)
+      uint32_t* mk_g = m_key + g * CL * K;
+      int* mi_g = m_idx + g * CL * K;
+      int nvalid = 0;
+      for (int e0 = 0; e0 < CL * K; e0 += 32) {
+        const int e = e0 + lane;
+        const bool ok = e < CL * K && mi_g[e] >= 0;
+        const uint32_t kk2 = ok ? mk_g[e] : 0u;
+        const int ii = ok ? mi_g[e] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, ok);
+        __syncwarp();
+        if (ok) {
+          const int at = nvalid + __popc(bal & ((1u << lane) - 1u));
+          mk_g[at] = kk2;
+          mi_g[at] = ii;
+        }
+        nvalid += __popc(bal);
+        __syncwarp();
+      }
+      const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[warp], ck, cp);
+      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[warp][j]];
+      if (lane == 0) s_nsel[g] = cnt;
+    }
+  }
+  __syncthreads();
 
-  // ---- the schedule -------------------------------------------------------------------------
-  // One group: score, select, attend, merge.  Two groups: group 1's summaries stream in while
-  // group 0 selects, group 0's K/V streams while group 1 scores and selects, group 1's K/V while
-  // group 0 merges -- the selection and merge phases of one group overlap the other's bytes.
-  score_group(0);
-  cluster_wait();  // every peer has started: DSMEM stores may begin
-  select_group(0);
-  sr0 = slice_range(0);
-  if (kMma && tid == 0 && !s_abort) {
-    fence_proxy_async();  // generic accesses of the summary phase precede the async K/V writes
-    for (; kv_next < min(NKV, sr0.nst); ++kv_next) issue_kv(kv_next);
+  // ---- 3. the union of the selections, plus the current block ------------------------------
+  // every selection as a bitmap over the history blocks; one warp compacts the OR of the bitmaps
+  // into the sorted union and takes each entry's head mask from the same words
+  const int nwords = (nc + 31) / 32;
+  for (int g = warp; g < Gs; g += kWarps) {
+    uint32_t* hb = hbits + g * nwords;
+    for (int w = lane; w < nwords; w += 32) hb[w] = 0u;
+    __syncwarp();
+    for (int j = lane; j < s_nsel[g]; j += 32) {
+      const int x = s_sel[g][j];
+      atomicOr(&hb[x >> 5], 1u << (x & 31));
+    }
   }
-  if (NG > 1) {
-    score_group(1);
-    select_group(1);
-    sr1 = slice_range(1);
-    if (kMma && tid == 0 && !s_abort)
-      for (; kv_next < min(NKV, sr0.nst + sr1.nst); ++kv_next) issue_kv(kv_next);
+  if (rank == 0) {  // optional outputs: the selection of every head
+    for (int e = tid; e < G * K; e += kThreads) {
+      const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
+      const size_t row = (size_t)bi * Hq + h0 + g;
+      if (p.idx) p.idx[row * K + j] = j < s_nsel[gs] ? s_sel[gs][j] : -1;
+      if (p.count && j == 0) p.count[row] = s_nsel[gs];
+    }
   }
-  if (s_abort && tid == 0) {
-    // summary copies still in flight: the last stage issued into each slot, on its own parity
-    for (int J = max(0, sub_issued - NS); J < sub_issued; ++J)
-      (void)mbar_wait_bounded(&bar[J % NS], (J / NS) & 1, 1u << 12);
-    report_timeout(p.status, 1);
+  __syncthreads();
+  if (warp == 0) {  // a contiguous run of words per lane, prefix sums of their union counts
+    const int per = (nwords + 31) / 32;
+    const int w0 = min(nwords, lane * per), w1 = min(nwords, w0 + per);
+    int mine = 0;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t u = 0u;
+      for (int g = 0; g < Gs; ++g) u |= hbits[g * nwords + w];
+      mine += __popc(u);
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int at = incl - mine;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t hw[G];
+      uint32_t u = 0u;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        hw[g] = g < Gs ? hbits[g * nwords + w] : 0u;
+        u |= hw[g];
+      }
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        unsigned m = 0u;
+#pragma unroll
+        for (int g = 0; g < G; ++g) m |= ((hw[g] >> bit) & 1u) << g;
+        s_ublk[at] = w * 32 + bit;
+        s_umask[at] = p.shared ? (1u << G) - 1u : m;
+        ++at;
+      }
+    }
+    if (lane == 31) {
+      s_ublk[incl] = cur;  // the current block, always kept, follows every history block
+      s_umask[incl] = (1u << G) - 1u;
+      s_U = incl + 1;
+    }
   }
-  attend_group(0);
-  merge_group(0);
-  if (NG > 1) {
-    attend_group(1);
-    merge_group(1);
+  __syncthreads();
+  const int U = s_U;
+
+  // ---- 4. attend my share of the union ------------------------------------------------------
+  float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 4: [warp][G][D+2]
+
+  if constexpr (kMma) {
+    // 16-token slices: history entries have 4, the current block ceil(tok / 16); CTA r takes
+    // slices [r S / CL, (r + 1) S / CL); a stage holds four consecutive slices (K then V tiles,
+    // 64 rows x 128 bytes per 64-column half, 128-byte swizzle), stage i is taken by group i & 1
+    const int tok_cur = pos - cur * b + 1;
+    const int s_hist = 4 * (U - 1);
+    const int S_tot = s_hist + (tok_cur + kSlice - 1) / kSlice;
+    const int s_begin = (int)(((long long)rank * S_tot) / CL);
+    const int s_end = (int)(((long long)(rank + 1) * S_tot) / CL);
+    const int n_my = s_end - s_begin;
+    const int nst = (n_my + 3) / 4;
+    const int grp = warp >> 2, wg = warp & 3;
+    const size_t tl = SM::kv_tile(b);
+    auto ktile = [&](int st) { return smem + (size_t)st * 2 * tl; };
+    auto vtile = [&](int st) { return smem + (size_t)st * 2 * tl + tl; };
+    uint64_t* kvbar = bar + NS;
+    const int row0 = (bi * p.Hk + kh) * p.n;
+    // Each group owns NKV / 2 slots and refills them itself: stage i (group i & 1, its (i >> 1)-th)
+    // uses slot (i & 1) + 2 ((i >> 1) % nper) in phase (i >> 1) / nper, and the group issues
+    // stage i + NKV into the same slot once it has finished stage i.  A group therefore never waits
+    // on a phase of a slot that has not been issued yet, however far it runs ahead of the other.
+    const int nper = NKV / 2;
+    auto slot_of = [&](int i) { return (i & 1) + 2 * ((i >> 1) % nper); };
+    auto parity_of = [&](int i) { return (uint32_t)(((i >> 1) / nper) & 1); };
+    // slice -> (block, first token of the slice within the block)
+    auto slice_blk = [&](int s) { return s < s_hist ? s_ublk[s >> 2] : cur; };
+    auto slice_tok0 = [&](int s) { return s < s_hist ? (s & 3) * kSlice : (s - s_hist) * kSlice; };
+    auto issue_kv = [&](int i) {
+      const int st = slot_of(i);
+      s_kv_last[st] = i;
+      const int first = s_begin + 4 * i;
+      const int nsl = min(4, s_end - first);
+      mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
+      for (int w = 0; w < nsl; ++w) {
+        const int s = first + w;
+        const int y = row0 + slice_blk(s) * b + slice_tok0(s);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tc::tma_load_2d(ktile(st) + hf * 8192 + w * kSlice * 128, &tmk, hf * 64, y, &kvbar[st]);
+          tc::tma_load_2d(vtile(st) + hf * 8192 + w * kSlice * 128, &tmv, hf * 64, y, &kvbar[st]);
+        }
+      }
+    };
+    if (tid == 0 && !s_abort) {
+      fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
+      for (int i = 0; i < min(nst, NKV); ++i) issue_kv(i);
+    }
+    if (p.append && rank == CL - 1) {
+      // the block being filled: its summary rewritten from its keys in global memory by the last
+      // CTA while its first K/V stages are in flight; every row is requested at once (a warp
+      // takes rows warp, warp + 8, ...: at most 8 of a 64-token block)
+      const T* kb =
+          static_cast<const T*>(p.k) + ((size_t)(bi * p.Hk + kh) * p.n + (size_t)cur * b) * D;
+      float x[8][EPL];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = warp + kWarps * u;
+        if (t < tok_cur) {
+          load_vec<T, EPL>(kb + (size_t)t * D + lane * EPL, x[u]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) x[u][e] = 0.f;
+        }
+      }
+      float cs[EPL];
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) cs[e] = 0.f;
+      float nmax = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        float sq = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          cs[e] += x[u][e];
+          sq = fmaf(x[u][e], x[u][e], sq);
+        }
+        nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));  // rows past the block add 0
+      }
+      float* part = reinterpret_cast<float*>(s_scratch);  // [kWarps][D]
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) part[warp * D + lane * EPL + e] = cs[e];
+      if (lane == 0) s_red[warp] = nmax;
+      __syncthreads();
+      const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+      for (int col = tid; col < D; col += kThreads) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) sum += part[w * D + col];
+        mean_k[row * D + col] = Elem<TS>::from_f(sum / (float)tok_cur);
+      }
+      if (tid == 0) {
+        float nm = 0.f;
+        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
+        if (p.max_norm) p.max_norm[row] = nm;
+        if (p.centre)
+          p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok_cur - 1);
+      }
+    }
+    // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
+    const int grow = lane >> 2, tig = lane & 3;
+    uint32_t qa0[D / 16], qa1[D / 16];
+    {
+      const float qs = scale * kLog2e;
+      const T* qrow = static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + min(grow, G - 1)) * D;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+        if (grow < G) {
+          x0 = Elem<T>::to_f(qrow[16 * ks + 2 * tig]) * qs;
+          x1 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 1]) * qs;
+          x2 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 8]) * qs;
+          x3 = Elem<T>::to_f(qrow[16 * ks + 2 * tig + 9]) * qs;
+        }
+        qa0[ks] = pack_bf16(x0, x1);
+        qa1[ks] = pack_bf16(x2, x3);
+      }
+    }
+    // O^T accumulators: m-tile mt covers d rows 16 mt .. 16 mt + 15, columns are heads
+    float oacc[D / 16][4];
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
+    float m_run = -INFINITY, l_part = 0.f;
+    const int n_run = s_abort ? 0 : nst;  // nothing was issued after an earlier timeout
+    for (int i = grp; i < n_run; i += 2) {
+      const int st = slot_of(i);
+      // group-uniform decision: the OR over the group's four warps of "my wait ran out"
+      const int bad = mbar_wait_bounded(&kvbar[st], parity_of(i)) ? 0 : 1;
+      int any_bad;
+      asm volatile(
+          "{\n\t.reg .pred pin, pout;\n\t"
+          "setp.ne.s32 pin, %1, 0;\n\t"
+          "barrier.red.or.pred pout, %2, 128, pin;\n\t"
+          "selp.s32 %0, 1, 0, pout;\n\t}"
+          : "=r"(any_bad)
+          : "r"(bad), "r"(1 + grp)
+          : "memory");
+      if (any_bad) {
+        s_abort = 1;
+        break;
+      }
+      const int s = s_begin + 4 * i + wg;  // this warp's slice
+      if (s < s_end) {
+        const int m = slice_blk(s);
+        const unsigned hm = s < s_hist ? s_umask[s >> 2] : (1u << G) - 1u;
+        const int tv = m == cur ? min(kSlice, tok_cur - slice_tok0(s)) : kSlice;  // valid tokens
+        const unsigned char* kt = ktile(st);
+        const unsigned char* vt = vtile(st);
+        const int t0 = wg * kSlice;  // this warp's 16 rows of the stage tile
+        // S = Q K^T over two 8-token tiles
+        float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const int hf = ks >> 2, ch = (ks & 3) * 2;
+            const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
+            const uint32_t b0 =
+                *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
+            const uint32_t b1 =
+                *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
+            mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+          }
+        }
+        // masks, per-row online softmax (row = head grow; the quad shares the row)
+        const bool head_on = grow < G && ((hm >> grow) & 1u);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int t = 8 * nt + 2 * tig + e;
+            if (!head_on || t >= tv) sfr[nt][e] = -INFINITY;
+            mx = fmaxf(mx, sfr[nt][e]);
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
+        if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
+          corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
+          m_run = mx;
+          l_part *= corr;
+        }
+        // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
+        const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
+        const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
+        if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            oacc[c][0] *= corr_a;
+            oacc[c][1] *= corr_b;
+            oacc[c][2] *= corr_a;
+            oacc[c][3] *= corr_b;
+          }
+        }
+        float pv[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float z = sfr[nt][e];
+            pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
+            l_part += pv[nt][e];
+          }
+        // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
+        const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
+        const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+        // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int mi = lane >> 3, rr = lane & 7;
+          const int tokr = t0 + (mi >> 1) * 8 + rr;
+          const int chunk = 2 * mt + (mi & 1);  // 16-byte chunk along d (0..D/8-1)
+          const int hf = chunk >> 3, cin = chunk & 7;
+          const uint32_t addr =
+              smem_u32(vt + hf * 8192 + tokr * 128 + ((cin ^ (tokr & 7)) << 4));
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(addr, v0, v1, v2, v3);
+          mma_16816(oacc[mt], v0, v1, v2, v3, pb0, pb1);
+        }
+      }
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
+      if (wg == 0 && lane == 0 && i + NKV < nst) issue_kv(i + NKV);
+    }
+    __syncthreads();
+    if (s_abort && tid == 0) {
+      // copies still in flight: the last stage issued into each slot; waiting on its own phase
+      // parity returns at once if it already landed
+      for (int st = 0; st < NKV; ++st)
+        if (s_kv_last[st] >= 0)
+          (void)mbar_wait_bounded(&kvbar[st], parity_of(s_kv_last[st]), 1u << 12);
+      report_timeout(p.status, 2);
+    }
+    __syncthreads();
+    // warp partials (rows < G): m, l and o
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+    if (grow < G && tig == 0) {
+      float* wp = wpart + ((size_t)warp * G + grow) * (D + 2);
+      wp[D] = m_run;
+      wp[D + 1] = l_part;
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {  // O^T element (d, head 2 tig + e)
+      const int hh = 2 * tig + e;
+      if (hh < G) {
+        float* wp = wpart + ((size_t)warp * G + hh) * (D + 2);
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          wp[16 * mt + grow] = oacc[mt][e];
+          wp[16 * mt + grow + 8] = oacc[mt][2 + e];
+        }
+      }
+    }
+    __syncthreads();
+  } else {
+    // fp32 / other block sizes: scalar FMAs; CTA r takes union entries r, r + CL, ...; warps split
+    // each block's tokens, one CTA-wide softmax per block
+    const int ne = rank < U ? (U - rank + CL - 1) / CL : 0;
+    auto entry_tokens = [&](int m) { return m == cur ? pos - cur * b + 1 : b; };
+    const size_t tl = SM::kv_tile(b);
+    T* kbuf[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem + 2 * tl)};
+    T* vbuf[2] = {reinterpret_cast<T*>(smem + tl), reinterpret_cast<T*>(smem + 3 * tl)};
+    uint64_t* kvbar = bar + NS;
+    const T* kbase = static_cast<const T*>(p.k) + (size_t)(bi * p.Hk + kh) * p.n * D;
+    const T* vbase = static_cast<const T*>(p.v) + (size_t)(bi * p.Hk + kh) * p.n * D;
+    auto issue_kv = [&](int i) {
+      const int m = s_ublk[rank + i * CL];
+      const uint32_t bytes = (uint32_t)(entry_tokens(m) * D * sizeof(T));
+      const int st = i & 1;
+      mbar_arrive_expect_tx(&kvbar[st], 2 * bytes);
+      bulk_g2s(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st]);
+      bulk_g2s(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st]);
+    };
+    if (tid == 0 && !s_abort) {
+      fence_proxy_async();
+      if (ne > 0) issue_kv(0);
+      if (ne > 1) issue_kv(1);
+    }
+    constexpr int CG = D / 2;
+    constexpr int TP = kThreads / CG;
+    float qa[G][EPL];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) qa[g][e] = qv[g][e] * scale * kLog2e;
+    const int cg = tid % CG, tp = tid / CG;
+    float acc[G][2];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = 0.f;
+    int i_stop = ne;
+    const int n_run = s_abort ? 0 : ne;  // nothing was issued after an earlier timeout
+    for (int i = 0; i < n_run; ++i) {
+      const int st = i & 1;
+      const int m = s_ublk[rank + i * CL];
+      const unsigned hm = s_umask[rank + i * CL];
+      const int tok = entry_tokens(m);
+      if (!s_abort && !mbar_wait_bounded(&kvbar[st], (i >> 1) & 1)) s_abort = 1;
+      __syncthreads();
+      if (s_abort) {
+        i_stop = i;
+        break;
+      }
+      const T* kt = kbuf[st];
+      const T* vt = vbuf[st];
+      for (int t0 = warp * R; t0 < tok; t0 += kWarps * R) {
+        float a[32];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float x[EPL];
+          if (t0 + r < tok) {
+            load_vec<T, EPL>(kt + (size_t)(t0 + r) * D + lane * EPL, x);
+          } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) x[e] = 0.f;
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float sacc = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) sacc = fmaf(qa[g][e], x[e], sacc);
+            a[r * G + g] = sacc;
+          }
+        }
+        warp_transpose_reduce32(a, lane);
+        const int t = t0 + lane / G, g = lane % G;
+        if (t < tok) zs[t * G + g] = ((hm >> g) & 1u) ? a[0] : -INFINITY;
+      }
+      if (p.append && m == cur) {
+        for (int col = tid; col < D; col += kThreads) {
+          float sum = 0.f;
+          for (int t = 0; t < tok; ++t) sum += Elem<T>::to_f(kt[(size_t)t * D + col]);
+          mean_k[((size_t)(bi * p.Hk + kh) * p.C + cur) * D + col] = Elem<TS>::from_f(sum / (float)tok);
+        }
+        float nmax = 0.f;
+        for (int t = warp; t < tok; t += kWarps) {
+          float x[EPL];
+          load_vec<T, EPL>(kt + (size_t)t * D + lane * EPL, x);
+          float sq = 0.f;
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) sq = fmaf(x[e], x[e], sq);
+          nmax = fmaxf(nmax, sqrtf(warp_sum(sq)));
+        }
+        if (lane == 0) s_red[warp] = nmax;
+      }
+      __syncthreads();
+      if (p.append && m == cur && tid == 0) {
+        float nm = 0.f;
+        for (int w = 0; w < kWarps; ++w) nm = fmaxf(nm, s_red[w]);
+        const size_t row = (size_t)(bi * p.Hk + kh) * p.C + cur;
+        if (p.max_norm) p.max_norm[row] = nm;
+        if (p.centre) p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok - 1);
+      }
+      for (int g = warp; g < G; g += kWarps) {
+        float mx = -INFINITY;
+        for (int t = lane; t < tok; t += 32) mx = fmaxf(mx, zs[t * G + g]);
+        mx = warp_max(mx);
+        const float m_old = s_m[g];
+        const float m_new = fmaxf(m_old, mx);
+        float sum = 0.f;
+        for (int t = lane; t < tok; t += 32) {
+          const float pvv = (m_new == -INFINITY) ? 0.f : exp2f(zs[t * G + g] - m_new);
+          ps[t * G + g] = pvv;
+          sum += pvv;
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) {
+          const float corr = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
+          s_corr[g] = corr;
+          s_l[g] = s_l[g] * corr + sum;
+          s_m[g] = m_new;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        acc[g][0] *= s_corr[g];
+        acc[g][1] *= s_corr[g];
+      }
+      for (int t = tp; t < tok; t += TP) {
+        float vv[2];
+        load_vec<T, 2>(vt + (size_t)t * D + 2 * cg, vv);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pw = ps[t * G + g];
+          acc[g][0] = fmaf(pw, vv[0], acc[g][0]);
+          acc[g][1] = fmaf(pw, vv[1], acc[g][1]);
+        }
+      }
+      __syncthreads();
+      if (tid == 0 && i + 2 < ne) issue_kv(i + 2);
+    }
+    if (s_abort && tid == 0 && n_run > 0) {
+      // copies in flight: stages i_stop and i_stop + 1 (if issued), each on its own parity
+      for (int j = i_stop; j < min(ne, i_stop + 2); ++j)
+        (void)mbar_wait_bounded(&kvbar[j & 1], (j >> 1) & 1, 1u << 12);
+      report_timeout(p.status, 2);
+    }
+    __syncthreads();
+    // token partitions tp -> "warp partial" slots 0..TP-1 with the shared (m, l)
+    for (int e = tid; e < kWarps * G * (D + 2); e += kThreads) wpart[e] = 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float* wp = wpart + ((size_t)tp * G + g) * (D + 2);
+      wp[2 * cg] = acc[g][0];
+      wp[2 * cg + 1] = acc[g][1];
+      if (cg == 0) {
+        wp[D] = s_m[g];
+        wp[D + 1] = tp == 0 ? s_l[g] : 0.f;
+      }
+    }
+    for (int w = TP + tid; w < kWarps; w += kThreads)  // unused slots: empty
+      for (int g = 0; g < G; ++g) wpart[((size_t)w * G + g) * (D + 2) + D] = -INFINITY;
+    __syncthreads();
+  }
+
+  // ---- 5. merge the warps, push column slices to their owners, finish -----------------------
+  const int cols = D / CL;
+  // per head: combined max over warps, then weights
+  for (int g = warp; g < G; g += kWarps) {
+    float M = -INFINITY;
+    if (lane < kWarps) M = wpart[((size_t)lane * G + g) * (D + 2) + D];
+    M = warp_max(M);
+    float lsum = 0.f;
+    if (lane < kWarps) {
+      const float mw = wpart[((size_t)lane * G + g) * (D + 2) + D];
+      const float w = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      lsum = w * wpart[((size_t)lane * G + g) * (D + 2) + D + 1];
+    }
+    lsum = warp_sum(lsum);
+    if (lane == 0) {
+      s_m[g] = M;
+      s_l[g] = lsum;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += kThreads) {
+    const int g = e / D, col = e % D;
+    const float M = s_m[g];
+    float osum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wpart[((size_t)w * G + g) * (D + 2) + D];
+      if (mw != -INFINITY) osum = fmaf(exp2f(mw - M), wpart[((size_t)w * G + g) * (D + 2) + col], osum);
+    }
+    // push to the owner of this column: recv[rank][g][col % cols], plus (m, l)
+    const int owner = col / cols;
+    float* slot = recv + ((size_t)rank * G + g) * (cols + 2);
+    st_dsmem_f32(dsmem_addr(&slot[col % cols], owner), osum);
+    if (col % cols == 0) {
+      st_dsmem_f32(dsmem_addr(&slot[cols], owner), M);
+      st_dsmem_f32(dsmem_addr(&slot[cols + 1], owner), s_l[g]);
+    }
+  }
+  cluster_sync();
+  for (int e = tid; e < G * cols; e += kThreads) {
+    const int g = e / cols, cc = e % cols, col = rank * cols + cc;
+    float M = -INFINITY;
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, recv[((size_t)r * G + g) * (cols + 2) + cols]);
+    float lsum = 0.f, osum = 0.f;
+    for (int r = 0; r < CL; ++r) {
+      const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
+      const float mr = slot[cols];
+      if (mr == -INFINITY) continue;
+      const float w = exp2f(mr - M);
+      lsum = fmaf(w, slot[cols + 1], lsum);
+      osum = fmaf(w, slot[cc], osum);
+    }
+    const size_t row = (size_t)bi * Hq + h0 + g;
+    static_cast<T*>(p.o)[row * D + col] = Elem<T>::from_f(osum / lsum);
+    if (col == 0 && p.lse) p.lse[row] = (M + log2f(lsum)) * kLn2;
   }
 }
 
@@ -1313,124 +1225,71 @@ LaunchCache& launch_cache() {
 // Shared memory one SM gives its resident CTAs (228 KB less 1 KB reserved per CTA) and the static
 // shared memory of the fused kernel (G <= 8), both with margin.
 constexpr size_t kSmemPerSM = 227 * 1024;
-constexpr size_t kStaticSmemBound = 11 * 1024;
-
-// Shared-memory layout of one launch shape (groups per cluster ng, cluster size CL): returns the
-// dynamic bytes, or 0 when the shape does not fit per_sm CTAs on one SM.
-template <typename T, typename TS, int D, int G, bool MMA>
-size_t fused_layout(FusedParams& p, int ng, int CL, int per_sm) {
-  using SM = FusedSmem<T, TS, D, G, MMA>;
-  const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
-  if (chunk > kSelMax) return 0;  // the local select holds at most kSelMax keys per head
-  p.chunk = chunk;
-  p.ng = ng;
-  // whole-row selection when every history fits one warp select
-  p.gather = p.C <= kSelMax ? 1 : 0;
-  p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
-  p.keys_bytes = (int)SM::keys(chunk);
-  p.sel_bytes = (int)SM::sel(p.gather, p.row_ld, CL, p.K);
-  p.recv_bytes = (int)SM::recv(CL);
-  const size_t fixed = p.keys_bytes + (size_t)ng * (p.sel_bytes + p.recv_bytes) +
-                       SM::hbits(p.C) + SM::zp(p.b) + 256;
-  const size_t budget = kSmemPerSM / per_sm - kStaticSmemBound - 1024 /* alignment slack */;
-  if (budget <= fixed) return 0;
-  const size_t avail = (budget - fixed) / 1024 * 1024;
-  const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage(), part = SM::partials();
-  const int subs = ng * ceil_div(chunk, kSub);  // summary stages a CTA streams
-  size_t sum_bytes, kv_bytes;
-  if (ng == 1) {
-    // one region: the summary ring, then the K/V stages, then the warp partials
-    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), part);
-    if (avail < need_min) return 0;
-    const size_t ra = std::min(avail, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus), part));
-    p.ns = (int)std::min<size_t>(kMaxStages, ra / sus);
-    // the MMA path's groups own half of the K/V slots each: an even count
-    p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) / 2 * 2 : 2;
-    sum_bytes = align_up(ra, 1024);
-    kv_bytes = 0;
-  } else {
-    // two groups in flight: the summary ring (later the partials) and the K/V ring apart; two
-    // summary stages already stream group 1's slice during group 0's selection, so the K/V ring
-    // takes four stages (two per warp group) when they fit
-    if (!MMA) return 0;
-    const size_t sum2 = align_up(max_sz(2 * sus, part), 1024);
-    p.nkv = avail >= sum2 + 4 * kvs ? 4 : 2;
-    kv_bytes = p.nkv * kvs;
-    if (avail < kv_bytes + sum2) return 0;
-    const int ns = (int)std::min<size_t>(std::min(kMaxStages, subs), (avail - kv_bytes) / sus);
-    if (ns < 2) return 0;
-    p.ns = ns;
-    sum_bytes = align_up(max_sz((size_t)ns * sus, part), 1024);
-  }
-  size_t off = 0;
-  p.off_sum = 0;
-  off += sum_bytes;
-  p.off_kv = ng == 1 ? 0 : (int)off;
-  off += kv_bytes;
-  off = align_up(off, 1024);
-  p.off_keys = (int)off;
-  off += p.keys_bytes;
-  p.off_sel = (int)off;
-  off += (size_t)ng * p.sel_bytes;
-  p.off_hbits = (int)off;
-  off += SM::hbits(p.C);
-  p.off_recv = (int)off;
-  off += (size_t)ng * p.recv_bytes;
-  p.off_zp = (int)off;
-  off += SM::zp(p.b);
-  off = align_up(off, 16);
-  p.off_bar = (int)off;
-  off += 256;
-  const size_t smem = off + 1024;  // + alignment slack of the dynamic base
-  return smem <= 227 * 1024 ? smem : 0;
-}
+constexpr size_t kStaticSmemBound = 12 * 1024;
 
 template <typename T, typename TS, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
+  using SM = FusedSmem<T, TS, D, G, MMA>;
   CUtensorMap tmk{}, tmv{};
   if (MMA) {
     const long long rows = (long long)p.B * p.Hk * p.n;
     if (!kv_map(&tmk, p.k, rows, D) || !kv_map(&tmv, p.v, rows, D)) return BSA_ERR_CUDA;
   }
   const int groups = p.B * p.Hk;
+  int CL = pick_cluster(groups);
   auto kern = decode_fused_kernel<T, TS, D, G, MMA>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
-  // Launch shape.  One group per cluster while every cluster fits at two CTAs per SM with one
-  // CTA per SM being too few; when one group per cluster would need two CTAs per SM, two groups
-  // per cluster at one CTA per SM instead (the MMA path), so that one group's selection and merge
-  // run while the other's bytes stream.
-  int CL = pick_cluster(groups), ng = 1;
-  size_t smem = 0;
-  if (MMA && groups * CL > kSMs) {
-    const int clusters = ceil_div(groups, 2);
-    int cl2 = 2;
-    while (cl2 * 2 <= kMaxCL && clusters * cl2 * 2 <= kSMs) cl2 <<= 1;
-    if (clusters * cl2 <= kSMs && clusters <= 65535) {
-      FusedParams q2 = p;
-      const size_t sm2 = fused_layout<T, TS, D, G, MMA>(q2, 2, cl2, 1);
-      if (sm2) {
-        p = q2;
-        CL = cl2;
-        ng = 2;
-        smem = sm2;
-      }
-    }
-  }
   for (;;) {
-    if (ng == 1) {
-      const int per_sm = groups * CL > kSMs ? 2 : 1;
-      smem = fused_layout<T, TS, D, G, MMA>(p, 1, CL, per_sm);
-      if (!smem && per_sm == 2) smem = fused_layout<T, TS, D, G, MMA>(p, 1, CL, 1);
-      if (!smem) {
-        if (CL < kMaxCL && p.C > CL * kSelMax) { CL <<= 1; continue; }
-        return BSA_ERR_UNSUPPORTED;
-      }
-      if (groups > 65535) return BSA_ERR_UNSUPPORTED;
+    const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
+    if (chunk > kSelMax) {  // the local select holds at most kSelMax keys per head
+      if (CL < kMaxCL) { CL <<= 1; continue; }
+      return BSA_ERR_UNSUPPORTED;
     }
+    p.chunk = chunk;
+    // whole-row selection when every history fits one warp select
+    p.gather = p.C <= kSelMax ? 1 : 0;
+    p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
+    // the fixed pieces, then region A as large as the CTAs resident per SM allow
+    size_t off = 0;
+    const size_t fixed = SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K) +
+                         SM::hbits(p.C) + SM::recv(CL) + SM::zp(p.b) + 256;
+    const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage();
+    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), SM::partials());
+    // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
+    // (two K/V stages) does not fit that way
+    int per_sm = groups * CL > kSMs ? 2 : 1;
+    size_t ra = 0;
+    for (;; per_sm = 1) {
+      const size_t budget = kSmemPerSM / per_sm - kStaticSmemBound - 1024 /* alignment slack */;
+      ra = budget > fixed ? (budget - fixed) / 1024 * 1024 : 0;
+      if (ra >= need_min || per_sm == 1) break;
+    }
+    if (ra < need_min) return BSA_ERR_UNSUPPORTED;
+    ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus),
+                             SM::partials()));
+    p.ns = (int)std::min<size_t>(kMaxStages, ra / sus);
+    // the MMA path's groups own half of the K/V slots each: an even count
+    p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) / 2 * 2 : 2;
+    off = align_up(ra, 1024);
+    p.off_keys = (int)off;
+    off += SM::keys(chunk);
+    p.off_sel = (int)off;
+    off += SM::sel(p.gather, p.row_ld, CL, p.K);
+    p.off_hbits = (int)off;
+    off += SM::hbits(p.C);
+    p.off_recv = (int)off;
+    off += SM::recv(CL);
+    p.off_zp = (int)off;
+    off += SM::zp(p.b);
+    off = align_up(off, 16);
+    p.off_bar = (int)off;
+    off += 256;
+    const size_t smem = off + 1024;  // + alignment slack of the dynamic base
+    if (smem > 227 * 1024) return BSA_ERR_UNSUPPORTED;
     LaunchCache& lc = launch_cache();
     {
       std::lock_guard<std::mutex> lock(lc.mu);
@@ -1448,7 +1307,7 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
       }
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(CL, ceil_div(groups, ng), 1);
+    cfg.gridDim = dim3(CL, p.Hk, p.B);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -1475,11 +1334,6 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
       }
     }
     if (nclusters <= 0) {
-      if (ng == 2) {  // fall back to one group per cluster
-        ng = 1;
-        CL = pick_cluster(groups);
-        continue;
-      }
       if (CL <= 2) return BSA_ERR_UNSUPPORTED;
       CL >>= 1;
       continue;

@@ -1039,7 +1039,7 @@ bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq
                       const float* scores, int scores_ld, void* o, float* lse, int* status,
                       cudaStream_t st) {
   (void)b;
-  // up to 32 selected blocks: two unit pairs per CTA in ping-pong
+  // the step-split kernel (two softmax warpgroups) covers every shape this path accepts
   const bsa_status pp = sas_fwd_tc(q, k, v, B, Hq, Hk, n, d, idx, count, K, gate, norm, scores,
                                    scores_ld, o, lse, status, st);
   if (pp != BSA_ERR_UNSUPPORTED) return pp;
