@@ -616,7 +616,9 @@ def build_layers(dev, case, w, R):
 
 
 def capture_fused(dev, layers, w, status, stream):
-    """One CUDA graph per layer holding the fused decode step (one kernel launch)."""
+    """CUDA graphs of the fused decode step (one kernel launch per step): one graph per layer,
+    and one graph of a whole decode iteration (every layer's step in order, as a model replays
+    one graph per generated token). Returns (per-layer graphs, iteration graph)."""
     import torch
 
     import block_sparse_attention_summaries_b200 as bsa
@@ -627,34 +629,52 @@ def capture_fused(dev, layers, w, status, stream):
                               max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
                               idx=L["idx"], count=L["count"], status=status)
 
+    return capture_steps(dev, layers, fused, stream)
+
+
+def capture_steps(dev, layers, step, stream):
+    """``step(L)`` captured once per layer and once as a whole iteration over the layers."""
+    import torch
     graphs = []
     with torch.cuda.stream(stream):
         for L in layers:
-            fused(L)
+            step(L)
         torch.cuda.synchronize(dev)
         for L in layers:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                fused(L)
+                step(L)
             graphs.append(g)
+        cycle = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cycle, stream=stream):
+            for L in layers:
+                step(L)
     torch.cuda.synchronize(dev)
-    return graphs
+    return graphs, cycle
+
+
+def replay_steps(graphs, steps):
+    """``steps`` decode steps: whole iterations over the layers, then single layers for the
+    remainder (graphs as returned by capture_steps)."""
+    per_layer, cycle = graphs
+    R = len(per_layer)
+    for _ in range(steps // R):
+        cycle.replay()
+    for i in range(steps % R):
+        per_layer[i].replay()
 
 
 def time_graph_cycle(dev, graphs, steps, warmup, stream):
-    """Milliseconds of ``steps`` replays (graph i % R in turn) between two events on the
-    stream (an event recorded between two replays would cost the step about 2 us: it ends the
+    """Milliseconds of ``steps`` decode steps (layer i % R in turn) between two events on the
+    stream (an event recorded between two steps would cost the step about 2 us: it ends the
     overlap of one launch's tail with the next one's start)."""
     import torch
-    R = len(graphs)
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            graphs[i % R].replay()
+        replay_steps(graphs, warmup)
         torch.cuda.synchronize(dev)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record(stream)
-        for i in range(steps):
-            graphs[i % R].replay()
+        replay_steps(graphs, steps)
         ev[1].record(stream)
         torch.cuda.synchronize(dev)
     return ev[0].elapsed_time(ev[1])
@@ -898,19 +918,17 @@ def run_gpu(args):
     sampler.start()
     time.sleep(0.3)
     with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % R].replay()
+        replay_steps(graphs, args.warmup)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         sampler.mark("t0")
-        # events bracket the K steps only: an event recorded between two replays costs the step
+        # events bracket the K steps only: an event recorded between two steps costs the step
         # about 2 us (it ends the overlap of one launch's tail with the next one's start)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         ev[0].record(stream)
-        for i in range(args.steps):
-            graphs[i % R].replay()
+        replay_steps(graphs, args.steps)
         ev[1].record(stream)
         torch.cuda.synchronize(dev)
         sampler.mark("t1")
@@ -935,25 +953,19 @@ def run_gpu(args):
         # every buffer a captured graph uses stays referenced as long as the graphs live:
         # entering a capture empties the allocator's cache, so a buffer kept alive only by a
         # replaced closure would go back to the driver and its graph would replay into freed memory
-        vgraphs, vbufs, vidx = [], [], None
+        vbufs = []
         with torch.cuda.stream(stream):
-            for r, L in enumerate(layers):
+            for L in layers:
                 mk = bsa.round_summaries_bf16(L["mean_k"]) if bf16_sum else L["mean_k"].clone()
-                ix = torch.empty(B, Hq, K, device=dev, dtype=torch.int32)
-                vbufs.append((mk, ix))
+                vbufs.append(dict(L, mean_k=mk, idx=torch.empty(B, Hq, K, device=dev,
+                                                               dtype=torch.int32)))
 
-                def vstep(L=L, mk=mk, ix=ix):
-                    bsa.decode_step_ex(L["q"], L["k"], L["v"], mk, b, K, flags, append=True,
-                                       max_norm=L["max_norm"], centre=L["centre"], o=L["o"],
-                                       lse=L["lse"], idx=ix, count=L["count"], status=status)
-                vstep()
-                torch.cuda.synchronize(dev)
-                if r == 0:
-                    vidx = ix.cpu().numpy()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    vstep()
-                vgraphs.append(g)
+        def vstep(L, flags=flags):
+            bsa.decode_step_ex(L["q"], L["k"], L["v"], L["mean_k"], b, K, flags, append=True,
+                               max_norm=L["max_norm"], centre=L["centre"], o=L["o"],
+                               lse=L["lse"], idx=L["idx"], count=L["count"], status=status)
+        vgraphs = capture_steps(dev, vbufs, vstep, stream)
+        vidx = vbufs[0]["idx"].cpu().numpy()
         nv = max(50, min(args.steps, 400))
         v_us = time_graph_cycle(dev, vgraphs, nv, args.warmup, stream) / nv * 1e3
         del vgraphs  # graphs first, then the buffers they replay into
@@ -1022,7 +1034,8 @@ def run_gpu(args):
                    "parallelism": f"replicas{world}",
                    "l2": f"inputs larger than L2: {R} rotated layer instances of the KV cache and "
                          "summaries (one step per instance in turn)",
-                   "graphs": "one CUDA graph (one fused kernel) per step"},
+                   "graphs": "one CUDA graph per decode iteration over the layers (one fused "
+                             "kernel per layer step, programmatic dependent launch)"},
         "roofline": {"bound": "hbm", "kernel": "decode_fused_kernel",
                      "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"],

@@ -228,6 +228,23 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
       : "memory");
 }
 
+// An L2 policy under which the lines a copy brings in are the first to be evicted: for data
+// streamed once per launch (the K/V cache, block summaries), so that it does not push out what
+// every launch reuses (the kernel's code, its small inputs).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void bulk_g2s_stream(void* smem_dst, const void* gmem_src,
+                                                uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 // Status word at the start of a workspace: set once by the first failing CTA.
 __device__ __forceinline__ void report_timeout(int* status, int where) {
   if (status) atomicCAS(status, 0, where);

@@ -61,6 +61,7 @@ constexpr int kSub = 64;          // summary rows per ring stage
 constexpr int kSelItems = 16;     // keys per lane of one warp select: N <= 512
 constexpr int kSelMax = 32 * kSelItems;
 constexpr int kCandMax = 64;      // candidates the threshold pass may leave for exact ranking
+constexpr int kScratchPerWarp = 2 * kCandMax + 4;  // candidate keys (+ 4 padding), positions
 constexpr int kMaxStages = 8;     // ring stages (summaries or K/V)
 constexpr int kSlice = 16;        // tokens per warp slice (64-token bf16 path)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -275,14 +276,16 @@ __device__ __noinline__ int warp_select_radix(const uint32_t* keys, int N, int k
 
 // Top-min(K, N) of N <= kSelMax order keys (shared memory, index order) by one warp; writes the
 // winners' positions ascending to `out`, returns their number.  `ck` / `cp` are the warp's
-// scratch for kCandMax candidate keys / positions.
+// scratch for kCandMax candidate keys / positions (ck 16-byte aligned, kCandMax + 4 entries).
 //
 // Threshold pass: lane l holds positions l + 32 j; the even-j and odd-j keys of every lane form 64
-// groups.  T0 = the kk-th largest group maximum: the kk groups whose maxima reach T0 hold kk
-// distinct keys >= T0, so every key of the Top-kk is >= T0.  The keys >= T0 are compacted in
-// position order (usually a few more than kk) and ranked exactly; if more than kCandMax pass, the
-// radix select runs on all N keys instead.
-__device__ __forceinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out,
+// groups.  T0 = the kk-th largest group maximum (a bitonic sort of the 64 maxima across the warp,
+// fifteen shuffle stages): the kk groups whose maxima reach T0 hold kk distinct keys >= T0, so
+// every key of the Top-kk is >= T0.  The keys >= T0 are compacted in position order (usually a few
+// more than kk) and ranked exactly; if more than kCandMax pass, the radix select runs on all N
+// keys instead.  Every step is a short dependency chain: the sixteen compaction ballots are
+// independent of one another and the ranking reads the candidates four at a time.
+__device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int lane, int* out,
                                            uint32_t* ck, int* cp) {
   const int kk = min(K, N);
   if (kk <= 0) return 0;
@@ -296,48 +299,60 @@ __device__ __forceinline__ int warp_select(const uint32_t* keys, int N, int K, i
   uint32_t kr[kSelItems];
 #pragma unroll
   for (int j = 0; j < kSelItems; ++j) kr[j] = j < nv ? keys[lane + 32 * j] : 0u;
-  uint32_t g0 = 0u, g1 = 0u;  // group maxima (even j, odd j)
+  // group maxima: element e = 2 lane + h of the 64 (h = 0: even j, h = 1: odd j)
+  uint32_t v0 = 0u, v1 = 0u;
 #pragma unroll
   for (int j = 0; j < kSelItems; j += 2) {
-    g0 = max(g0, kr[j]);
-    g1 = max(g1, kr[j + 1]);
+    v0 = max(v0, kr[j]);
+    v1 = max(v1, kr[j + 1]);
   }
-  // rank of each group maximum among the 64 (ties: lower group id ranks higher); the one of rank
-  // kk - 1 is T0
-  int r0 = 0, r1 = 0;
-#pragma unroll 8
-  for (int src = 0; src < 32; ++src) {
-    const uint32_t a0 = __shfl_sync(0xffffffffu, g0, src);
-    const uint32_t a1 = __shfl_sync(0xffffffffu, g1, src);
-    // group ids: 2 * lane (even) and 2 * lane + 1 (odd)
-    r0 += (a0 > g0 || (a0 == g0 && src < lane)) + (a1 > g0 || (a1 == g0 && src < lane));
-    r1 += (a0 > g1 || (a0 == g1 && src <= lane)) + (a1 > g1 || (a1 == g1 && src < lane));
-  }
-  const unsigned h0 = __ballot_sync(0xffffffffu, r0 == kk - 1);
-  const unsigned h1 = __ballot_sync(0xffffffffu, r1 == kk - 1);
-  const uint32_t T0 = h0 ? __shfl_sync(0xffffffffu, g0, __ffs(h0) - 1)
-                         : __shfl_sync(0xffffffffu, g1, __ffs(h1) - 1);
-  int cnt = 0;
+  // bitonic sort of the 64 maxima, descending: in a block of size k the lower element of a
+  // compared pair keeps the larger value when the block runs downward ((e & k) == 0)
 #pragma unroll
-  for (int j = 0; j < kSelItems; ++j) cnt += (j < nv && kr[j] >= T0) ? 1 : 0;
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  for (int k = 2; k <= 64; k <<= 1) {
+    const bool down = ((2 * lane) & k) == 0;
+#pragma unroll
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      if (jj == 1) {  // the pair sits in one lane
+        const uint32_t hi = max(v0, v1), lo = min(v0, v1);
+        v0 = down ? hi : lo;
+        v1 = down ? lo : hi;
+      } else {
+        const int lm = jj >> 1;  // partner lane distance
+        const uint32_t w0 = __shfl_xor_sync(0xffffffffu, v0, lm);
+        const uint32_t w1 = __shfl_xor_sync(0xffffffffu, v1, lm);
+        const bool keep_max = ((lane & lm) == 0) == down;
+        v0 = keep_max ? max(v0, w0) : min(v0, w0);
+        v1 = keep_max ? max(v1, w1) : min(v1, w1);
+      }
+    }
+  }
+  const uint32_t T0 = __shfl_sync(0xffffffffu, ((kk - 1) & 1) ? v1 : v0, (kk - 1) >> 1);
+  uint32_t cm = 0u;  // my candidates: bit j for position 32 j + lane
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) cm |= (j < nv && kr[j] >= T0) ? (1u << j) : 0u;
+  const int cnt = __reduce_add_sync(0xffffffffu, __popc(cm));
   if (cnt > kCandMax) return warp_select_radix(keys, N, kk, lane, out);
-  // compact the candidates in position order (position 32 j + lane grows with (j, lane))
+  // compact in position order: the candidates at j take places P_j + (rank among lanes), P_j the
+  // candidates at smaller j
   const unsigned lt = (1u << lane) - 1u;
+  unsigned bal[kSelItems];
+#pragma unroll
+  for (int j = 0; j < kSelItems; ++j) bal[j] = __ballot_sync(0xffffffffu, (cm >> j) & 1u);
   int base = 0;
 #pragma unroll
   for (int j = 0; j < kSelItems; ++j) {
-    if (32 * j >= N) break;  // warp-uniform
-    const bool c = j < nv && kr[j] >= T0;
-    const unsigned bal = __ballot_sync(0xffffffffu, c);
-    if (c) {
-      ck[base + __popc(bal & lt)] = kr[j];
-      cp[base + __popc(bal & lt)] = 32 * j + lane;
+    if ((cm >> j) & 1u) {
+      const int at = base + __popc(bal[j] & lt);
+      ck[at] = kr[j];
+      cp[at] = 32 * j + lane;
     }
-    base += __popc(bal);
+    base += __popc(bal[j]);
   }
+  if (lane < 4) ck[cnt + lane] = 0u;  // padding of the last group of four (never taken)
   __syncwarp();
-  // rank the candidates; the winners keep the candidates' (ascending) position order
+  // rank the candidates (ties: the lower position ranks higher); the winners keep the
+  // candidates' ascending position order
   uint32_t mk[2];
   int rk[2];
 #pragma unroll
@@ -345,14 +360,22 @@ __device__ __forceinline__ int warp_select(const uint32_t* keys, int N, int K, i
     mk[q] = lane + 32 * q < cnt ? ck[lane + 32 * q] : 0u;
     rk[q] = 0;
   }
+  const uint4* ck4 = reinterpret_cast<const uint4*>(ck);
+  const int n4 = (cnt + 3) >> 2;
 #pragma unroll 4
-  for (int j = 0; j < cnt; ++j) {
-    const uint32_t kj = ck[j];
+  for (int c = 0; c < n4; ++c) {
+    const uint4 g4 = ck4[c];
+    const uint32_t kv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-    for (int q = 0; q < 2; ++q) rk[q] += (kj > mk[q] || (kj == mk[q] && j < lane + 32 * q)) ? 1 : 0;
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * c + e;
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        rk[q] += (kv[e] > mk[q] || (kv[e] == mk[q] && j < lane + 32 * q)) ? 1 : 0;
+    }
   }
   int taken = 0;
-  int mypos[2] = {lane < cnt ? cp[lane] : 0, lane + 32 < cnt ? cp[lane + 32] : 0};
+  const int mypos[2] = {lane < cnt ? cp[lane] : 0, lane + 32 < cnt ? cp[lane + 32] : 0};
   __syncwarp();
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
@@ -426,14 +449,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ uint32_t s_bits[kMaxWords];
   __shared__ int s_ublk[kMaxUnion];
   __shared__ unsigned s_umask[kMaxUnion];
-  __shared__ uint32_t s_scratch[kWarps * 2 * kCandMax];  // select candidates / append partials
+  // select candidates (per warp: kCandMax + 4 keys, kCandMax positions) / append partials
+  __shared__ __align__(16) uint32_t s_scratch[kWarps * kScratchPerWarp];
   __shared__ int s_kv_last[kMaxStages];  // the last K/V stage issued into each slot (-1: none)
   __shared__ int s_U;
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
-  static_assert(kWarps * 2 * kCandMax >= kWarps * 128, "append partials fit the scratch");
+  static_assert(kWarps * kScratchPerWarp >= kWarps * 128, "append partials fit the scratch");
 
+  // Programmatic dependent launch: every input may come from the work queued before this kernel
+  // on the stream, so nothing is read before that work has completed and its writes are visible;
+  // a launch queued after this one may be scheduled at once and wait the same way.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = p.b, K = p.K, Hq = p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = (int)cluster_rank();
@@ -481,12 +510,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int rows = c_hi - c_lo;
   const int nsub = (rows + kSub - 1) / kSub;
   const TS* mk = mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
+  // summaries and K/V are read once per step: their L2 lines go first, so that the kernel's code
+  // (fetched again by every launch) stays in L2 (the policy is made where it is used: one
+  // instruction, no register held across the kernel)
   auto issue_sub = [&](int j) {
     const int r0 = c_lo + j * kSub;
     const int nr = min(kSub, c_hi - r0);
     const uint32_t bytes = (uint32_t)(nr * D * sizeof(TS));
     mbar_arrive_expect_tx(&bar[j % NS], bytes);
-    bulk_g2s(ring + (size_t)(j % NS) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j % NS]);
+    bulk_g2s_stream(ring + (size_t)(j % NS) * kSub * D, mk + (size_t)r0 * D, bytes, &bar[j % NS],
+                    l2_evict_first());
   };
   int sub_issued = 0;  // (thread 0) summary stages issued so far
   if (tid == 0)
@@ -559,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   }
 
   // ---- 2. Top-K per head (per group when shared) -----------------------------------------
-  uint32_t* ck = s_scratch + warp * 2 * kCandMax;
-  int* cp = reinterpret_cast<int*>(ck + kCandMax);
+  uint32_t* ck = s_scratch + warp * kScratchPerWarp;
+  int* cp = reinterpret_cast<int*>(ck + kCandMax + 4);
   cluster_wait();  // every peer has started: DSMEM stores may begin
   if (p.gather) {
     // push my slice of every selecting head's keys into every CTA's whole-row copy
@@ -732,13 +765,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       const int first = s_begin + 4 * i;
       const int nsl = min(4, s_end - first);
       mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
+      const uint64_t pol = l2_evict_first();
       for (int w = 0; w < nsl; ++w) {
         const int s = first + w;
         const int y = row0 + slice_blk(s) * b + slice_tok0(s);
 #pragma unroll
         for (int hf = 0; hf < D / 64; ++hf) {
-          tc::tma_load_2d(ktile(st) + hf * 8192 + w * kSlice * 128, &tmk, hf * 64, y, &kvbar[st]);
-          tc::tma_load_2d(vtile(st) + hf * 8192 + w * kSlice * 128, &tmv, hf * 64, y, &kvbar[st]);
+          tc::tma_load_2d_hint(ktile(st) + hf * 8192 + w * kSlice * 128, &tmk, hf * 64, y,
+                               &kvbar[st], pol);
+          tc::tma_load_2d_hint(vtile(st) + hf * 8192 + w * kSlice * 128, &tmv, hf * 64, y,
+                               &kvbar[st], pol);
         }
       }
     };
@@ -970,8 +1006,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       const uint32_t bytes = (uint32_t)(entry_tokens(m) * D * sizeof(T));
       const int st = i & 1;
       mbar_arrive_expect_tx(&kvbar[st], 2 * bytes);
-      bulk_g2s(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st]);
-      bulk_g2s(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st]);
+      const uint64_t pol = l2_evict_first();
+      bulk_g2s_stream(kbuf[st], kbase + (size_t)m * b * D, bytes, &kvbar[st], pol);
+      bulk_g2s_stream(vbuf[st], vbase + (size_t)m * b * D, bytes, &kvbar[st], pol);
     };
     if (tid == 0 && !s_abort) {
       fence_proxy_async();
@@ -1243,6 +1280,7 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
+  int min_per_sm = 1;
   for (;;) {
     const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
     if (chunk > kSelMax) {  // the local select holds at most kSelMax keys per head
@@ -1261,7 +1299,7 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), SM::partials());
     // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
     // (two K/V stages) does not fit that way
-    int per_sm = groups * CL > kSMs ? 2 : 1;
+    int per_sm = std::max(min_per_sm, groups * CL > kSMs ? 2 : 1);
     size_t ra = 0;
     for (;; per_sm = 1) {
       const size_t budget = kSmemPerSM / per_sm - kStaticSmemBound - 1024 /* alignment slack */;
@@ -1311,13 +1349,17 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // the kernel may be scheduled while the previous launch on the stream drains (it waits for
+    // that launch's completion before reading anything)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     int nclusters = 0;
     {
       std::lock_guard<std::mutex> lock(lc.mu);
@@ -1336,6 +1378,12 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     if (nclusters <= 0) {
       if (CL <= 2) return BSA_ERR_UNSUPPORTED;
       CL >>= 1;
+      continue;
+    }
+    if (nclusters < groups && per_sm == 1 && min_per_sm == 1) {
+      // not every cluster is resident at one CTA per SM (large clusters are placed one per GPC):
+      // two CTAs per SM with smaller rings keep the whole grid in one wave
+      min_per_sm = 2;
       continue;
     }
     if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) {
