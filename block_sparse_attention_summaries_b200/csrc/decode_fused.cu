@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   // select candidates (per warp: kCandMax + 4 keys, kCandMax positions) / append partials
   __shared__ __align__(16) uint32_t s_scratch[kWarps * kScratchPerWarp];
   __shared__ int s_kv_last[kMaxStages];  // the last K/V stage issued into each slot (-1: none)
+  __shared__ int s_gst[kMaxStages];      // global K/V stage held by each slot (-1: none left)
+  __shared__ unsigned s_next;            // (rank 0) dynamic K/V stages handed out so far
   __shared__ int s_U;
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
@@ -493,6 +495,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     for (int i = 0; i < kMaxStages; ++i) s_kv_last[i] = -1;
+    s_next = 0;
     s_abort = 0;
     s_U = 0;
   }
@@ -733,17 +736,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   float* wpart = reinterpret_cast<float*>(smem);  // reused after phase 4: [warp][G][D+2]
 
   if constexpr (kMma) {
-    // 16-token slices: history entries have 4, the current block ceil(tok / 16); CTA r takes
-    // slices [r S / CL, (r + 1) S / CL); a stage holds four consecutive slices (K then V tiles,
-    // 64 rows x 128 bytes per 64-column half, 128-byte swizzle), stage i is taken by group i & 1
+    // 16-token slices: history entries have 4, the current block ceil(tok / 16); a global stage
+    // holds four consecutive slices (K then V tiles, 64 rows x 128 bytes per 64-column half,
+    // 128-byte swizzle).  CTA r first takes global stages r, r + CL, ... into its NKV slots; every
+    // later stage is handed out by a counter in rank 0's shared memory when a slot frees, so CTAs
+    // whose copies land early take more of the union (HBM serves the CTAs of a cluster unevenly:
+    // with static shares the slowest CTA took twice the median).  Local stage i (the i-th stage a
+    // CTA takes) is processed by warp group i & 1.
     const int tok_cur = pos - cur * b + 1;
     const int s_hist = 4 * (U - 1);
     const int S_tot = s_hist + (tok_cur + kSlice - 1) / kSlice;
-    const int s_begin = (int)(((long long)rank * S_tot) / CL);
-    const int s_end = (int)(((long long)(rank + 1) * S_tot) / CL);
-    const int n_my = s_end - s_begin;
-    const int nst = (n_my + 3) / 4;
+    const int G_st = (S_tot + 3) / 4;
     const int grp = warp >> 2, wg = warp & 3;
+    const uint32_t next_addr = dsmem_addr(&s_next, 0);
     const size_t tl = SM::kv_tile(b);
     auto ktile = [&](int st) { return smem + (size_t)st * 2 * tl; };
     auto vtile = [&](int st) { return smem + (size_t)st * 2 * tl + tl; };
@@ -759,11 +764,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     // slice -> (block, first token of the slice within the block)
     auto slice_blk = [&](int s) { return s < s_hist ? s_ublk[s >> 2] : cur; };
     auto slice_tok0 = [&](int s) { return s < s_hist ? (s & 3) * kSlice : (s - s_hist) * kSlice; };
-    auto issue_kv = [&](int i) {
+    // local stage i holds global stage g (g < 0: none left; the slot's phase then completes with no
+    // data, and the group that reaches it stops)
+    auto issue_kv = [&](int i, int g) {
       const int st = slot_of(i);
+      s_gst[st] = g;
+      if (g < 0) {
+        mbar_arrive(&kvbar[st]);
+        return;
+      }
       s_kv_last[st] = i;
-      const int first = s_begin + 4 * i;
-      const int nsl = min(4, s_end - first);
+      const int first = 4 * g;
+      const int nsl = min(4, S_tot - first);
       mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
       const uint64_t pol = l2_evict_first();
       for (int w = 0; w < nsl; ++w) {
@@ -780,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     };
     if (tid == 0 && !s_abort) {
       fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
-      for (int i = 0; i < min(nst, NKV); ++i) issue_kv(i);
+      for (int i = 0; i < NKV; ++i) issue_kv(i, rank + CL * i < G_st ? rank + CL * i : -1);
     }
     if (p.append && rank == CL - 1) {
       // the block being filled: its summary rewritten from its keys in global memory by the last
@@ -857,8 +869,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
     float m_run = -INFINITY, l_part = 0.f;
-    const int n_run = s_abort ? 0 : nst;  // nothing was issued after an earlier timeout
-    for (int i = grp; i < n_run; i += 2) {
+    // the group leader asks for the global stage of its next refill one stage ahead, so that the
+    // remote atomic's round trip overlaps a stage's work
+    const bool leader = wg == 0 && lane == 0;
+    int g_ahead = -1;
+    auto grab = [&]() {
+      uint32_t v;
+      asm volatile("atom.shared::cluster.add.u32 %0, [%1], 1;" : "=r"(v) : "r"(next_addr) : "memory");
+      const int g = CL * NKV + (int)v;
+      return g < G_st ? g : -1;
+    };
+    if (leader && !s_abort) g_ahead = grab();
+    for (int i = grp; !s_abort; i += 2) {
       const int st = slot_of(i);
       // group-uniform decision: the OR over the group's four warps of "my wait ran out"
       const int bad = mbar_wait_bounded(&kvbar[st], parity_of(i)) ? 0 : 1;
@@ -875,8 +897,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         s_abort = 1;
         break;
       }
-      const int s = s_begin + 4 * i + wg;  // this warp's slice
-      if (s < s_end) {
+      const int gst = s_gst[st];
+      if (gst < 0) break;  // no stage left for this group (uniform over the group)
+      const int s = 4 * gst + wg;  // this warp's slice
+      if (s < S_tot) {
         const int m = slice_blk(s);
         const unsigned hm = s < s_hist ? s_umask[s >> 2] : (1u << G) - 1u;
         const int tv = m == cur ? min(kSlice, tok_cur - slice_tok0(s)) : kSlice;  // valid tokens
@@ -957,7 +981,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         }
       }
       asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
-      if (wg == 0 && lane == 0 && i + NKV < nst) issue_kv(i + NKV);
+      if (leader) {
+        issue_kv(i + NKV, g_ahead);
+        if (g_ahead >= 0) g_ahead = grab();
+      }
     }
     __syncthreads();
     if (s_abort && tid == 0) {
