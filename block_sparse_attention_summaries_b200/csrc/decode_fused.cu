@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ unsigned s_umask[kMaxUnion];
   // select candidates (per warp: kCandMax + 4 keys, kCandMax positions) / append partials
   __shared__ __align__(16) uint32_t s_scratch[kWarps * kScratchPerWarp];
-  __shared__ int s_kv_last[kMaxStages];  // the last K/V stage issued into each slot (-1: none)
+  __shared__ int s_kv_par[kMaxStages];   // phase parity of the last copy into each slot (-1: none)
   __shared__ int s_gst[kMaxStages];      // global K/V stage held by each slot (-1: none left)
   __shared__ unsigned s_next;            // (rank 0) dynamic K/V stages handed out so far
   __shared__ int s_U;
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   if (tid == 0) {
     for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
-    for (int i = 0; i < kMaxStages; ++i) s_kv_last[i] = -1;
+    for (int i = 0; i < kMaxStages; ++i) s_kv_par[i] = -1;
     s_next = 0;
     s_abort = 0;
     s_U = 0;
@@ -754,26 +754,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     auto vtile = [&](int st) { return smem + (size_t)st * 2 * tl + tl; };
     uint64_t* kvbar = bar + NS;
     const int row0 = (bi * p.Hk + kh) * p.n;
-    // Each group owns NKV / 2 slots and refills them itself: stage i (group i & 1, its (i >> 1)-th)
-    // uses slot (i & 1) + 2 ((i >> 1) % nper) in phase (i >> 1) / nper, and the group issues
-    // stage i + NKV into the same slot once it has finished stage i.  A group therefore never waits
-    // on a phase of a slot that has not been issued yet, however far it runs ahead of the other.
-    const int nper = NKV / 2;
-    auto slot_of = [&](int i) { return (i & 1) + 2 * ((i >> 1) % nper); };
-    auto parity_of = [&](int i) { return (uint32_t)(((i >> 1) / nper) & 1); };
+    // Group 0 owns slots [0, n0), group 1 slots [n0, NKV) (n0 = ceil(NKV / 2)); a group's k-th
+    // local stage uses its slot k % n in phase k / n, and the group refills that slot itself once
+    // it has finished the stage.  A group therefore never waits on a phase of a slot that has not
+    // been issued yet, however far it runs ahead of the other.
+    const int n0 = (NKV + 1) >> 1;
+    const int nmine = grp == 0 ? n0 : NKV - n0, sbase = grp == 0 ? 0 : n0;
     // slice -> (block, first token of the slice within the block)
     auto slice_blk = [&](int s) { return s < s_hist ? s_ublk[s >> 2] : cur; };
     auto slice_tok0 = [&](int s) { return s < s_hist ? (s & 3) * kSlice : (s - s_hist) * kSlice; };
-    // local stage i holds global stage g (g < 0: none left; the slot's phase then completes with no
-    // data, and the group that reaches it stops)
-    auto issue_kv = [&](int i, int g) {
-      const int st = slot_of(i);
+    // slot st's next phase (parity par) holds global stage g (g < 0: none left; the phase then
+    // completes with no data, and the group that reaches it stops)
+    auto issue_kv = [&](int st, uint32_t par, int g) {
       s_gst[st] = g;
       if (g < 0) {
         mbar_arrive(&kvbar[st]);
         return;
       }
-      s_kv_last[st] = i;
+      s_kv_par[st] = (int)par;
       const int first = 4 * g;
       const int nsl = min(4, S_tot - first);
       mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
@@ -792,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     };
     if (tid == 0 && !s_abort) {
       fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
-      for (int i = 0; i < NKV; ++i) issue_kv(i, rank + CL * i < G_st ? rank + CL * i : -1);
+      for (int st = 0; st < NKV; ++st) issue_kv(st, 0u, rank + CL * st < G_st ? rank + CL * st : -1);
     }
     if (p.append && rank == CL - 1) {
       // the block being filled: its summary rewritten from its keys in global memory by the last
@@ -880,10 +878,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       return g < G_st ? g : -1;
     };
     if (leader && !s_abort) g_ahead = grab();
-    for (int i = grp; !s_abort; i += 2) {
-      const int st = slot_of(i);
+    for (int k = 0; !s_abort; ++k) {
+      const int st = sbase + k % nmine;
+      const uint32_t par = (uint32_t)((k / nmine) & 1);
       // group-uniform decision: the OR over the group's four warps of "my wait ran out"
-      const int bad = mbar_wait_bounded(&kvbar[st], parity_of(i)) ? 0 : 1;
+      const int bad = mbar_wait_bounded(&kvbar[st], par) ? 0 : 1;
       int any_bad;
       asm volatile(
           "{\n\t.reg .pred pin, pout;\n\t"
@@ -982,7 +981,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       }
       asm volatile("bar.sync %0, 128;" ::"r"(1 + grp));  // stage free
       if (leader) {
-        issue_kv(i + NKV, g_ahead);
+        issue_kv(st, par ^ 1u, g_ahead);
         if (g_ahead >= 0) g_ahead = grab();
       }
     }
@@ -991,8 +990,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       // copies still in flight: the last stage issued into each slot; waiting on its own phase
       // parity returns at once if it already landed
       for (int st = 0; st < NKV; ++st)
-        if (s_kv_last[st] >= 0)
-          (void)mbar_wait_bounded(&kvbar[st], parity_of(s_kv_last[st]), 1u << 12);
+        if (s_kv_par[st] >= 0) (void)mbar_wait_bounded(&kvbar[st], (uint32_t)s_kv_par[st], 1u << 12);
       report_timeout(p.status, 2);
     }
     __syncthreads();
@@ -1318,12 +1316,15 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     // whole-row selection when every history fits one warp select
     p.gather = p.C <= kSelMax ? 1 : 0;
     p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
-    // the fixed pieces, then region A as large as the CTAs resident per SM allow
+    // Region A as large as the CTAs resident per SM allow, then the fixed pieces.  Region A holds
+    // the summary ring with the keys and the whole-row / merge buffer above it (phases 1-2), then
+    // the K/V ring over all of it (phase 4, once the keys are dead), then the warp partials.
     size_t off = 0;
-    const size_t fixed = SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K) +
-                         SM::hbits(p.C) + SM::recv(CL) + SM::zp(p.b) + 256;
+    const size_t fixed = SM::hbits(p.C) + SM::recv(CL) + SM::zp(p.b) + 256;
+    const size_t tail =
+        align_up(SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K), (size_t)1024);
     const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage();
-    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus), SM::partials());
+    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus + tail), SM::partials());
     // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
     // (two K/V stages) does not fit that way
     int per_sm = std::max(min_per_sm, groups * CL > kSMs ? 2 : 1);
@@ -1334,16 +1335,13 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
       if (ra >= need_min || per_sm == 1) break;
     }
     if (ra < need_min) return BSA_ERR_UNSUPPORTED;
-    ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus),
+    ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus + tail),
                              SM::partials()));
-    p.ns = (int)std::min<size_t>(kMaxStages, ra / sus);
-    // the MMA path's groups own half of the K/V slots each: an even count
-    p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) / 2 * 2 : 2;
+    p.ns = (int)std::min<size_t>(kMaxStages, (ra - tail) / sus);
+    p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) : 2;
+    p.off_keys = (int)(ra - tail);
+    p.off_sel = p.off_keys + (int)SM::keys(chunk);
     off = align_up(ra, 1024);
-    p.off_keys = (int)off;
-    off += SM::keys(chunk);
-    p.off_sel = (int)off;
-    off += SM::sel(p.gather, p.row_ld, CL, p.K);
     p.off_hbits = (int)off;
     off += SM::hbits(p.C);
     p.off_recv = (int)off;
