@@ -339,7 +339,7 @@ def time_cuda(fn, reps, stream):
     return [ev[i].elapsed_time(ev[i + 1]) for i in range(reps)]
 
 
-def run_prefill(dev, peaks, reps=5):
+def run_prefill(dev, peaks, reps=5, rows=("sas", "freesolo", "fsl")):
     """Prefill rows: SAS gated training prefill (forward on tcgen05 + gate gradient) and FreeSolo
     two-branch prefill, each as TFLOP/s on the gathered FLOPs (4 d per attended query-key pair)."""
     import torch
@@ -349,249 +349,251 @@ def run_prefill(dev, peaks, reps=5):
 
     out = {}
     stream = torch.cuda.Stream(dev)
-    pc = inputs.prefill_case(5000)
     bf = lambda x: torch.from_numpy(x).to(dev, torch.bfloat16)
-    q, k, v, do = bf(pc.q), bf(pc.k), bf(pc.v), bf(pc.dout)
-    s = torch.from_numpy(pc.scores).to(dev)
-    idx, cnt = bsa.topk_blocks(s, pc.K, units=pc.U, q_block=64, b=64)
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
-    dg = torch.empty(pc.B, pc.Hq, pc.U, pc.K, device=dev, dtype=torch.float32)
-    cnt_h = cnt.cpu().numpy().astype(np.int64)  # [B, Hq, U]
-    d = pc.d
-    per_unit = cnt_h * 64 * 64 + 64 * 65 // 2  # attended pairs per unit (history + causal diag)
-    fwd_flops = float(4 * d * per_unit.sum())
-    grad_flops = float(4 * d * (cnt_h * 64 * 64).sum())
-    fwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate=True,
-                                      norm="selected", scores=s, o=o, lse=lse)
-    grad = lambda: bsa.gate_grad(q, k, v, o, lse, do, idx, 64, s, q_block=64, count=cnt,
-                                 norm="selected", dg=dg)
-    t_fwd = statistics.fmean(time_cuda(fwd, reps, stream))
-    t_grad = statistics.fmean(time_cuda(grad, max(2, reps // 2), stream))
-    n_cand = torch.arange(pc.U, dtype=torch.int32, device=dev).expand(pc.B, pc.Hq, pc.U).contiguous()
-    ds = torch.empty_like(s)
-    sgrad = lambda: bsa.selector_grad(s, n_cand, idx, cnt, dg, bsa.NORM_SELECTED, ds=ds)
-    t_sgrad = statistics.fmean(time_cuda(sgrad, reps, stream))
-    # selected normaliser: ds written over every candidate slot; idx, dg and the selected scores
-    # read per slot; count and n_cand per unit
-    sgrad_bytes = float(s.numel() * 4 + idx.numel() * 4 * 3 + cnt.numel() * 4 * 2)
-    # the outer-gate variant (gate outside the softmax) on the CUDA-core row kernels
-    o2 = torch.empty_like(q)
-    lse2 = torch.empty_like(lse)
-    dg2 = torch.empty_like(dg)
-    ofwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate="outer",
-                                       norm="selected", scores=s, o=o2, lse=lse2)
-    ograd = lambda: bsa.gate_grad(q, k, v, o2, lse2, do, idx, 64, s, q_block=64, count=cnt,
-                                  norm="selected", dg=dg2, outer=True)
-    t_ofwd = statistics.fmean(time_cuda(ofwd, max(2, reps // 2), stream))
-    t_ograd = statistics.fmean(time_cuda(ograd, max(2, reps // 2), stream))
     peak = peaks["bf16_tflops"]
     src = peaks["source"] + " bf16 (burst)"
-    out["sas_gated_prefill_16k"] = {
-        "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
-                   "q_block": 64, "K": pc.K, "gate": "log-softmax over the selected blocks"},
-        "forward": {"kernel": "prefill_tc_kernel (tcgen05)", "ms": t_fwd,
-                    "gathered_gflop": fwd_flops / 1e9, "tflops": fwd_flops / t_fwd / 1e9,
-                    "roofline": roofline("tensor", "prefill_tc_kernel", fwd_flops / t_fwd / 1e9,
-                                         peak, "TFLOP/s", peak_source=src)},
-        "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
-                      "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
-                      "roofline": roofline("tensor", "gate_grad_tc_kernel",
-                                           grad_flops / t_grad / 1e9, peak, "TFLOP/s",
-                                           peak_source=src)},
-        "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
-                          "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
-                          "roofline": roofline("hbm", "selector_grad_kernel",
-                                               sgrad_bytes / t_sgrad / 1e6, peaks["hbm_gbs"],
-                                               "GB/s", algorithmic=sgrad_bytes,
-                                               peak_source=peaks["source"] + " (burst copy)")},
-        "outer_gate": {"kernels": "prefill_tc_kernel, gate_grad_tc_kernel (tcgen05)",
-                       "forward_ms": t_ofwd, "forward_tflops": fwd_flops / t_ofwd / 1e9,
-                       "grad_ms": t_ograd, "grad_tflops": grad_flops / t_ograd / 1e9,
-                       "roofline": roofline("tensor", "prefill_tc_kernel (outer gate)",
-                                            fwd_flops / t_ofwd / 1e9, peak, "TFLOP/s",
+    if "sas" in rows:
+        pc = inputs.prefill_case(5000)
+        q, k, v, do = bf(pc.q), bf(pc.k), bf(pc.v), bf(pc.dout)
+        s = torch.from_numpy(pc.scores).to(dev)
+        idx, cnt = bsa.topk_blocks(s, pc.K, units=pc.U, q_block=64, b=64)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
+        dg = torch.empty(pc.B, pc.Hq, pc.U, pc.K, device=dev, dtype=torch.float32)
+        cnt_h = cnt.cpu().numpy().astype(np.int64)  # [B, Hq, U]
+        d = pc.d
+        per_unit = cnt_h * 64 * 64 + 64 * 65 // 2  # attended pairs per unit (history + causal diag)
+        fwd_flops = float(4 * d * per_unit.sum())
+        grad_flops = float(4 * d * (cnt_h * 64 * 64).sum())
+        fwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate=True,
+                                          norm="selected", scores=s, o=o, lse=lse)
+        grad = lambda: bsa.gate_grad(q, k, v, o, lse, do, idx, 64, s, q_block=64, count=cnt,
+                                     norm="selected", dg=dg)
+        t_fwd = statistics.fmean(time_cuda(fwd, reps, stream))
+        t_grad = statistics.fmean(time_cuda(grad, max(2, reps // 2), stream))
+        n_cand = torch.arange(pc.U, dtype=torch.int32, device=dev).expand(pc.B, pc.Hq, pc.U).contiguous()
+        ds = torch.empty_like(s)
+        sgrad = lambda: bsa.selector_grad(s, n_cand, idx, cnt, dg, bsa.NORM_SELECTED, ds=ds)
+        t_sgrad = statistics.fmean(time_cuda(sgrad, reps, stream))
+        # selected normaliser: ds written over every candidate slot; idx, dg and the selected scores
+        # read per slot; count and n_cand per unit
+        sgrad_bytes = float(s.numel() * 4 + idx.numel() * 4 * 3 + cnt.numel() * 4 * 2)
+        # the outer-gate variant (gate outside the softmax) on the CUDA-core row kernels
+        o2 = torch.empty_like(q)
+        lse2 = torch.empty_like(lse)
+        dg2 = torch.empty_like(dg)
+        ofwd = lambda: bsa.sparse_attn_fwd(q, k, v, idx, 64, count=cnt, q_block=64, gate="outer",
+                                           norm="selected", scores=s, o=o2, lse=lse2)
+        ograd = lambda: bsa.gate_grad(q, k, v, o2, lse2, do, idx, 64, s, q_block=64, count=cnt,
+                                      norm="selected", dg=dg2, outer=True)
+        t_ofwd = statistics.fmean(time_cuda(ofwd, max(2, reps // 2), stream))
+        t_ograd = statistics.fmean(time_cuda(ograd, max(2, reps // 2), stream))
+        out["sas_gated_prefill_16k"] = {
+            "config": {"B": pc.B, "Hq": pc.Hq, "Hk": pc.Hk, "d": d, "n": pc.n, "b": 64,
+                       "q_block": 64, "K": pc.K, "gate": "log-softmax over the selected blocks"},
+            "forward": {"kernel": "sas_fwd_tc_kernel (tcgen05, two softmax warpgroups)", "ms": t_fwd,
+                        "gathered_gflop": fwd_flops / 1e9, "tflops": fwd_flops / t_fwd / 1e9,
+                        "roofline": roofline("tensor", "sas_fwd_tc_kernel", fwd_flops / t_fwd / 1e9,
+                                             peak, "TFLOP/s", peak_source=src)},
+            "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
+                          "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
+                          "roofline": roofline("tensor", "gate_grad_tc_kernel",
+                                               grad_flops / t_grad / 1e9, peak, "TFLOP/s",
+                                               peak_source=src)},
+            "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
+                              "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
+                              "roofline": roofline("hbm", "selector_grad_kernel",
+                                                   sgrad_bytes / t_sgrad / 1e6, peaks["hbm_gbs"],
+                                                   "GB/s", algorithmic=sgrad_bytes,
+                                                   peak_source=peaks["source"] + " (burst copy)")},
+            "outer_gate": {"kernels": "sas_fwd_tc_kernel, gate_grad_tc_kernel (tcgen05)",
+                           "forward_ms": t_ofwd, "forward_tflops": fwd_flops / t_ofwd / 1e9,
+                           "grad_ms": t_ograd, "grad_tflops": grad_flops / t_ograd / 1e9,
+                           "roofline": roofline("tensor", "sas_fwd_tc_kernel (outer gate)",
+                                                fwd_flops / t_ofwd / 1e9, peak, "TFLOP/s",
+                                                peak_source=src)},
+        }
+        del q, k, v, do, o, s, idx, cnt, lse, dg, o2, lse2, dg2
+        torch.cuda.empty_cache()
+    if "freesolo" in rows:
+        fc = inputs.freesolo_case(4000)
+        q, k, v = bf(fc.q), bf(fc.k), bf(fc.v)
+        lam, sig, alpha = (torch.from_numpy(x).to(dev) for x in (fc.lam, fc.sigma, fc.alpha))
+        mk, mx, ce = bsa.build_block_summaries(k, fc.cell)
+        idx, cnt = bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K)
+        o = torch.empty_like(q)
+        ws = torch.zeros(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
+                                                                      fc.d, fc.cell, fc.K)),
+                         dtype=torch.uint8, device=dev)
+        sws = torch.zeros(max(1, int(bsa.lib().bsa_freesolo_select_workspace_bytes(
+            bsa.BSA_BF16, fc.B, fc.H, fc.n, fc.d, fc.cell, fc.q_block, fc.K))), dtype=torch.uint8,
+            device=dev)
+        sel = lambda: bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K,
+                                          idx=idx, count=cnt, ws=sws)
+        att = lambda: bsa.freesolo_attn(q, k, v, alpha, idx, cnt, fc.cell, fc.window, fc.rope_theta,
+                                        o=o, ws=ws)
+        t_sel = statistics.fmean(time_cuda(sel, 2, stream))
+        t_att = statistics.fmean(time_cuda(att, 2, stream))
+        cnt_h = cnt.cpu().numpy().astype(np.int64)
+        pos = np.arange(fc.n)
+        win = np.minimum(pos + 1, fc.window).sum() * fc.B * fc.H
+        att_flops = float(4 * fc.d * (win + (cnt_h * fc.cell).sum()))
+        ncand = ((pos // fc.q_block) * fc.q_block) // fc.cell
+        score_flops = float(2 * fc.d * ncand.sum() * fc.B * fc.H)
+        out["freesolo_prefill_64k"] = {
+            "config": {"B": fc.B, "H": fc.H, "d": fc.d, "n": fc.n, "cell": fc.cell,
+                       "q_block": fc.q_block, "K": fc.K, "window": fc.window},
+            "select": {"kernel": "split_hi_lo + freesolo_select_tc_kernel (tcgen05)", "ms": t_sel,
+                       "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9,
+                       "roofline": roofline("tensor", "freesolo_select_tc_kernel",
+                                            score_flops / t_sel / 1e9, peak, "TFLOP/s",
                                             peak_source=src)},
-    }
-    del q, k, v, do, o, s, idx, cnt, lse, dg, o2, lse2, dg2
-    torch.cuda.empty_cache()
+            "attention": {"kernel": "rope (q, k) + window_tc_kernel (persistent 128-query tiles) + "
+                                    "cell-major long branch (fs_long_* kernels, tcgen05 tiles) + "
+                                    "combine", "ms": t_att,
+                          "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,
+                          "roofline": roofline("tensor", "freesolo attention (all launches)",
+                                               att_flops / t_att / 1e9, peak, "TFLOP/s",
+                                               peak_source=src)},
+            "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),
+        }
+        del q, k, v, o, ws, sws, idx, cnt
+        torch.cuda.empty_cache()
+    if "fsl" in rows:
+        # FS-L / FS-B decode at 256K, batch 1 ([FreeSolo] "How it differs": FS-L keeps W + P cells
+        # per head in a fixed-size state, FS-B searches two forests): the kept-cell selection against
+        # full O(C) scoring, the FS-L state update per query block, the decode call (window + long
+        # branch + mix) and the FS-B build and search.  Each call of a timed graph decodes its own
+        # position (positions 600 tokens apart, so no call finds another's window in L2).
+        H, d, n, cell, K, W, P, window, width = 16, 64, 262144, 32, 4, 8, 64, 512, 16
+        g = torch.Generator(device=dev).manual_seed(4200)
+        kf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
+        vf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
+        qf = torch.randn(1, H, d, device=dev, generator=g).to(torch.bfloat16)
+        mk, mx, ce = bsa.build_block_summaries(kf, cell)
+        C = mk.shape[2]
+        lam = torch.full((H,), 0.5, device=dev)
+        sig = torch.full((H,), 4096.0, device=dev)
+        alpha = torch.rand(H, device=dev, generator=g)
+        iters = 20
+        positions = [n - 1 - 600 * r for r in range(iters)]
+        pos_t = [torch.full((1,), p_, dtype=torch.int32, device=dev) for p_ in positions]
+        ncell_t = [torch.full((H,), (p_ // 128) * 128 // cell, dtype=torch.int32, device=dev)
+                   for p_ in positions]
+        states = []
+        for r in range(iters):  # a state per position, grown from empty
+            st = bsa.FslState(H, W, P, dev)
+            st.update(mx.view(H, C), ncell_t[r])
+            states.append(st)
+        seq = torch.full((1,), n, dtype=torch.int32, device=dev)
+        sc = torch.empty(1, H, C, device=dev)
+        ncnd = torch.empty(H, device=dev, dtype=torch.int32)
+        o_f = torch.empty(1, H, d, device=dev, dtype=torch.bfloat16)
+        idx_f = torch.empty(1, H, K, device=dev, dtype=torch.int32)
+        cnt_f = torch.empty(1, H, device=dev, dtype=torch.int32)
+        stat_f = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    fc = inputs.freesolo_case(4000)
-    q, k, v = bf(fc.q), bf(fc.k), bf(fc.v)
-    lam, sig, alpha = (torch.from_numpy(x).to(dev) for x in (fc.lam, fc.sigma, fc.alpha))
-    mk, mx, ce = bsa.build_block_summaries(k, fc.cell)
-    idx, cnt = bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K)
-    o = torch.empty_like(q)
-    ws = torch.zeros(int(bsa.lib().bsa_freesolo_workspace_bytes(bsa.BSA_BF16, fc.B, fc.H, fc.n,
-                                                                  fc.d, fc.cell, fc.K)),
-                     dtype=torch.uint8, device=dev)
-    sws = torch.zeros(max(1, int(bsa.lib().bsa_freesolo_select_workspace_bytes(
-        bsa.BSA_BF16, fc.B, fc.H, fc.n, fc.d, fc.cell, fc.q_block, fc.K))), dtype=torch.uint8,
-        device=dev)
-    sel = lambda: bsa.freesolo_select(q, mk, mx, ce, lam, sig, fc.cell, fc.q_block, fc.K,
-                                      idx=idx, count=cnt, ws=sws)
-    att = lambda: bsa.freesolo_attn(q, k, v, alpha, idx, cnt, fc.cell, fc.window, fc.rope_theta,
-                                    o=o, ws=ws)
-    t_sel = statistics.fmean(time_cuda(sel, 2, stream))
-    t_att = statistics.fmean(time_cuda(att, 2, stream))
-    cnt_h = cnt.cpu().numpy().astype(np.int64)
-    pos = np.arange(fc.n)
-    win = np.minimum(pos + 1, fc.window).sum() * fc.B * fc.H
-    att_flops = float(4 * fc.d * (win + (cnt_h * fc.cell).sum()))
-    ncand = ((pos // fc.q_block) * fc.q_block) // fc.cell
-    score_flops = float(2 * fc.d * ncand.sum() * fc.B * fc.H)
-    out["freesolo_prefill_64k"] = {
-        "config": {"B": fc.B, "H": fc.H, "d": fc.d, "n": fc.n, "cell": fc.cell,
-                   "q_block": fc.q_block, "K": fc.K, "window": fc.window},
-        "select": {"kernel": "split_hi_lo + freesolo_select_tc_kernel (tcgen05)", "ms": t_sel,
-                   "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9,
-                   "roofline": roofline("tensor", "freesolo_select_tc_kernel",
-                                        score_flops / t_sel / 1e9, peak, "TFLOP/s",
-                                        peak_source=src)},
-        "attention": {"kernel": "rope (q, k) + prefill_tc_kernel window mode + cell-major long "
-                                "branch (fs_long_* kernels, tcgen05 tiles) + combine", "ms": t_att,
-                      "gathered_gflop": att_flops / 1e9, "tflops": att_flops / t_att / 1e9,
-                      "roofline": roofline("tensor", "freesolo attention (all launches)",
-                                           att_flops / t_att / 1e9, peak, "TFLOP/s",
-                                           peak_source=src)},
-        "tokens_per_s": fc.n * fc.B / ((t_sel + t_att) / 1e3),
-    }
-    del q, k, v, o, ws, sws, idx, cnt
-    torch.cuda.empty_cache()
-
-    # FS-L / FS-B decode at 256K, batch 1 ([FreeSolo] "How it differs": FS-L keeps W + P cells
-    # per head in a fixed-size state, FS-B searches two forests): the kept-cell selection against
-    # full O(C) scoring, the FS-L state update per query block, the decode call (window + long
-    # branch + mix) and the FS-B build and search.  Each call of a timed graph decodes its own
-    # position (positions 600 tokens apart, so no call finds another's window in L2).
-    H, d, n, cell, K, W, P, window, width = 16, 64, 262144, 32, 4, 8, 64, 512, 16
-    g = torch.Generator(device=dev).manual_seed(4200)
-    kf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
-    vf = torch.randn(1, H, n, d, device=dev, generator=g).to(torch.bfloat16)
-    qf = torch.randn(1, H, d, device=dev, generator=g).to(torch.bfloat16)
-    mk, mx, ce = bsa.build_block_summaries(kf, cell)
-    C = mk.shape[2]
-    lam = torch.full((H,), 0.5, device=dev)
-    sig = torch.full((H,), 4096.0, device=dev)
-    alpha = torch.rand(H, device=dev, generator=g)
-    iters = 20
-    positions = [n - 1 - 600 * r for r in range(iters)]
-    pos_t = [torch.full((1,), p_, dtype=torch.int32, device=dev) for p_ in positions]
-    ncell_t = [torch.full((H,), (p_ // 128) * 128 // cell, dtype=torch.int32, device=dev)
-               for p_ in positions]
-    states = []
-    for r in range(iters):  # a state per position, grown from empty
-        st = bsa.FslState(H, W, P, dev)
-        st.update(mx.view(H, C), ncell_t[r])
-        states.append(st)
-    seq = torch.full((1,), n, dtype=torch.int32, device=dev)
-    sc = torch.empty(1, H, C, device=dev)
-    ncnd = torch.empty(H, device=dev, dtype=torch.int32)
-    o_f = torch.empty(1, H, d, device=dev, dtype=torch.bfloat16)
-    idx_f = torch.empty(1, H, K, device=dev, dtype=torch.int32)
-    cnt_f = torch.empty(1, H, device=dev, dtype=torch.int32)
-    stat_f = torch.zeros(1, dtype=torch.int32, device=dev)
-
-    def graph_ms(fns):
-        """Device time per call: the calls captured in one CUDA graph (these calls are a few
-        microseconds each, far below the cost of launching them one by one from Python)."""
-        with torch.cuda.stream(stream):
-            for fn in fns:
-                fn()
-        torch.cuda.synchronize(dev)
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            for fn in fns:
-                fn()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            gr.replay()
-            e0.record(stream)
-            for _ in range(reps):
+        def graph_ms(fns):
+            """Device time per call: the calls captured in one CUDA graph (these calls are a few
+            microseconds each, far below the cost of launching them one by one from Python)."""
+            with torch.cuda.stream(stream):
+                for fn in fns:
+                    fn()
+            torch.cuda.synchronize(dev)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for fn in fns:
+                    fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
                 gr.replay()
-            e1.record(stream)
-        e1.synchronize()
-        del gr
-        return e0.elapsed_time(e1) / (reps * len(fns))
+                e0.record(stream)
+                for _ in range(reps):
+                    gr.replay()
+                e1.record(stream)
+            e1.synchronize()
+            del gr
+            return e0.elapsed_time(e1) / (reps * len(fns))
 
-    seqs = [p_ + 1 for p_ in pos_t]
-    full = [lambda r=r: bsa.topk_blocks(bsa.score_blocks(
-        qf, mk, n, cell, seq_lens=seqs[r], max_norm=mx, centre=ce, lambda_h=lam, sigma_h=sig,
-        prefix_block=128, scores=sc, n_cand=ncnd)[0], K, n_cand=ncnd) for r in range(iters)]
-    fsl_sel = [lambda r=r: bsa.fsl_select(qf, pos_t[r], mk, mx, ce, lam, sig,
-                                          states[r].cand.view(1, H, -1),
-                                          states[r].cand_count.view(1, H), K)
-               for r in range(iters)]
-    fsl_dec = [lambda r=r: bsa.fsl_decode(qf, kf, vf, pos_t[r], cell, mk, mx, ce, lam, sig, alpha,
-                                          states[r].cand.view(1, H, -1),
-                                          states[r].cand_count.view(1, H), K, window=window,
-                                          o=o_f, idx=idx_f, count=cnt_f, status=stat_f)
-               for r in range(iters)]
-    t_full = graph_ms(full)
-    t_fsl_sel = graph_ms(fsl_sel)
-    t_fsl_dec = graph_ms(fsl_dec)
-    # the state update at a query-block boundary: 4 new cells per head (the state is reset to
-    # its previous prefix inside the graph, three small copies)
-    saved = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
-    prev = [c - 4 for c in ncell_t]
-    for st, p_ in zip(states, prev):  # states one query block earlier
-        st.older.fill_(-1)
-        st.older_count.zero_()
-        st.state_cells.zero_()
-        st.update(mx.view(H, C), p_)
-    base = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
+        seqs = [p_ + 1 for p_ in pos_t]
+        full = [lambda r=r: bsa.topk_blocks(bsa.score_blocks(
+            qf, mk, n, cell, seq_lens=seqs[r], max_norm=mx, centre=ce, lambda_h=lam, sigma_h=sig,
+            prefix_block=128, scores=sc, n_cand=ncnd)[0], K, n_cand=ncnd) for r in range(iters)]
+        fsl_sel = [lambda r=r: bsa.fsl_select(qf, pos_t[r], mk, mx, ce, lam, sig,
+                                              states[r].cand.view(1, H, -1),
+                                              states[r].cand_count.view(1, H), K)
+                   for r in range(iters)]
+        fsl_dec = [lambda r=r: bsa.fsl_decode(qf, kf, vf, pos_t[r], cell, mk, mx, ce, lam, sig, alpha,
+                                              states[r].cand.view(1, H, -1),
+                                              states[r].cand_count.view(1, H), K, window=window,
+                                              o=o_f, idx=idx_f, count=cnt_f, status=stat_f)
+                   for r in range(iters)]
+        t_full = graph_ms(full)
+        t_fsl_sel = graph_ms(fsl_sel)
+        t_fsl_dec = graph_ms(fsl_dec)
+        # the state update at a query-block boundary: 4 new cells per head (the state is reset to
+        # its previous prefix inside the graph, three small copies)
+        saved = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
+        prev = [c - 4 for c in ncell_t]
+        for st, p_ in zip(states, prev):  # states one query block earlier
+            st.older.fill_(-1)
+            st.older_count.zero_()
+            st.state_cells.zero_()
+            st.update(mx.view(H, C), p_)
+        base = [(st.older.clone(), st.older_count.clone(), st.state_cells.clone()) for st in states]
 
-    def upd(r):
-        st = states[r]
-        st.older.copy_(base[r][0])
-        st.older_count.copy_(base[r][1])
-        st.state_cells.copy_(base[r][2])
-        st.update(mx.view(H, C), ncell_t[r])
-    t_reset = graph_ms([lambda r=r: (states[r].older.copy_(base[r][0]),
-                                     states[r].older_count.copy_(base[r][1]),
-                                     states[r].state_cells.copy_(base[r][2]))
-                        for r in range(iters)])
-    t_upd = graph_ms([lambda r=r: upd(r) for r in range(iters)]) - t_reset
-    for st, sv in zip(states, saved):
-        assert torch.equal(st.older_count, sv[1]) and torch.equal(st.older, sv[0])
-    # FS-B: forests built for the query block's prefix, then beam search + re-rank + decode
-    forests = [bsa.fsb_build(mk, mx, ce, ncell_t[r]) for r in range(iters)]
-    fidx = torch.empty(1, H, K, device=dev, dtype=torch.int32)
-    fcnt = torch.empty(1, H, device=dev, dtype=torch.int32)
-    flse = torch.empty(1, H, K, device=dev)
-    t_fsb_build = graph_ms([lambda r=r: bsa.fsb_build(mk, mx, ce, ncell_t[r], forest=forests[r])
-                            for r in range(4)])
-    t_fsb_sel = graph_ms([lambda r=r: bsa.fsb_select(qf, kf, pos_t[r], cell, forests[r], lam,
-                                                     sig, width, K, idx=fidx, count=fcnt,
-                                                     lse=flse)
-                          for r in range(iters)])
-    del forests
-    # algorithmic bytes of one FS-L decode call: the window's K and V, the K selected cells' K
-    # and V, the kept cells' summaries, q and o
-    win = min(window, positions[0] + 1)
-    dec_bytes = H * (win * d * 2 * 2 + K * cell * d * 2 * 2 + (W + P) * (d + 2) * 4 + 2 * d * 2)
-    gbs = dec_bytes / (t_fsl_dec / 1e3) / 1e9
-    out["fsl_decode_256k"] = {
-        "config": {"B": 1, "H": H, "d": d, "n": n, "cell": cell, "K": K, "W": W, "P": P,
-                   "window": window, "cells": C, "fsb_beam": width},
-        "full_select_ms": t_full, "fsl_select_ms": t_fsl_sel,
-        "fsl_state_update_ms": t_upd, "fsl_decode_ms": t_fsl_dec,
-        "fsl_step_ms": t_fsl_dec + t_upd / 128.0,
-        "fsl_tokens_per_s": 1.0 / ((t_fsl_dec + t_upd / 128.0) / 1e3),
-        "fsb_build_ms": t_fsb_build, "fsb_select_ms": t_fsb_sel,
-        "fsb_step_ms": t_fsb_sel + t_fsl_dec + t_fsb_build / 128.0,
-        "decode_bytes": dec_bytes,
-        "roofline": roofline("hbm", "fsl_decode_kernel", gbs, peaks["hbm_gbs"], "GB/s",
-                             algorithmic=dec_bytes,
-                             peak_source=peaks["source"] + " (burst copy)"),
-        "kernels": "full: score_decode_kernel + topk_kernel over every cell; FS-L: "
-                   "fsl_select_kernel over the W + P kept cells; fsl_state_update_kernel (4 new "
-                   "cells per 128-token query block, amortised over its 128 steps); "
-                   "fsl_decode_kernel (4-CTA cluster per head); FS-B: topk_kernel (upper half) + "
-                   "fsb_build_levels/radius_kernel per query block (amortised over 128 steps), "
-                   "fsb_search_kernel per step",
-    }
-    del kf, vf
-    torch.cuda.empty_cache()
+        def upd(r):
+            st = states[r]
+            st.older.copy_(base[r][0])
+            st.older_count.copy_(base[r][1])
+            st.state_cells.copy_(base[r][2])
+            st.update(mx.view(H, C), ncell_t[r])
+        t_reset = graph_ms([lambda r=r: (states[r].older.copy_(base[r][0]),
+                                         states[r].older_count.copy_(base[r][1]),
+                                         states[r].state_cells.copy_(base[r][2]))
+                            for r in range(iters)])
+        t_upd = graph_ms([lambda r=r: upd(r) for r in range(iters)]) - t_reset
+        for st, sv in zip(states, saved):
+            assert torch.equal(st.older_count, sv[1]) and torch.equal(st.older, sv[0])
+        # FS-B: forests built for the query block's prefix, then beam search + re-rank + decode
+        forests = [bsa.fsb_build(mk, mx, ce, ncell_t[r]) for r in range(iters)]
+        fidx = torch.empty(1, H, K, device=dev, dtype=torch.int32)
+        fcnt = torch.empty(1, H, device=dev, dtype=torch.int32)
+        flse = torch.empty(1, H, K, device=dev)
+        t_fsb_build = graph_ms([lambda r=r: bsa.fsb_build(mk, mx, ce, ncell_t[r], forest=forests[r])
+                                for r in range(4)])
+        t_fsb_sel = graph_ms([lambda r=r: bsa.fsb_select(qf, kf, pos_t[r], cell, forests[r], lam,
+                                                         sig, width, K, idx=fidx, count=fcnt,
+                                                         lse=flse)
+                              for r in range(iters)])
+        del forests
+        # algorithmic bytes of one FS-L decode call: the window's K and V, the K selected cells' K
+        # and V, the kept cells' summaries, q and o
+        win = min(window, positions[0] + 1)
+        dec_bytes = H * (win * d * 2 * 2 + K * cell * d * 2 * 2 + (W + P) * (d + 2) * 4 + 2 * d * 2)
+        gbs = dec_bytes / (t_fsl_dec / 1e3) / 1e9
+        out["fsl_decode_256k"] = {
+            "config": {"B": 1, "H": H, "d": d, "n": n, "cell": cell, "K": K, "W": W, "P": P,
+                       "window": window, "cells": C, "fsb_beam": width},
+            "full_select_ms": t_full, "fsl_select_ms": t_fsl_sel,
+            "fsl_state_update_ms": t_upd, "fsl_decode_ms": t_fsl_dec,
+            "fsl_step_ms": t_fsl_dec + t_upd / 128.0,
+            "fsl_tokens_per_s": 1.0 / ((t_fsl_dec + t_upd / 128.0) / 1e3),
+            "fsb_build_ms": t_fsb_build, "fsb_select_ms": t_fsb_sel,
+            "fsb_step_ms": t_fsb_sel + t_fsl_dec + t_fsb_build / 128.0,
+            "decode_bytes": dec_bytes,
+            "roofline": roofline("hbm", "fsl_decode_kernel", gbs, peaks["hbm_gbs"], "GB/s",
+                                 algorithmic=dec_bytes,
+                                 peak_source=peaks["source"] + " (burst copy)"),
+            "kernels": "full: score_decode_kernel + topk_kernel over every cell; FS-L: "
+                       "fsl_select_kernel over the W + P kept cells; fsl_state_update_kernel (4 new "
+                       "cells per 128-token query block, amortised over its 128 steps); "
+                       "fsl_decode_kernel (4-CTA cluster per head); FS-B: topk_kernel (upper half) + "
+                       "fsb_build_levels/radius_kernel per query block (amortised over 128 steps), "
+                       "fsb_search_kernel per step",
+        }
+        del kf, vf
+        torch.cuda.empty_cache()
     return out
 
 
@@ -896,8 +898,9 @@ def run_gpu(args):
     if args.prefill_only:
         torch.cuda.set_device(0)
         bsa.lib()
-        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), load_peaks())}),
-              flush=True)
+        rows = tuple(x for x in args.prefill_rows.split(",") if x)
+        print(json.dumps({"prefill": run_prefill(torch.device("cuda", 0), load_peaks(),
+                                                 rows=rows)}), flush=True)
         return
 
     torch.cuda.set_device(local)
@@ -1097,6 +1100,8 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the 512K long-decode row")
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill rows (profiling the prefill kernels)")
+    ap.add_argument("--prefill-rows", default="sas,freesolo,fsl",
+                    help="with --prefill-only: which rows (sas, freesolo, fsl)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

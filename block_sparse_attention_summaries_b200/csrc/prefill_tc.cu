@@ -1,28 +1,29 @@
-// Sparse prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// FreeSolo long branch over unit block unions, and the SAS gate gradient, on the 5th-generation
+// tensor cores (tcgen05 + TMEM + TMA).
 //
-// [SAS] review: "Background" Eq. 2 (exact softmax over the selected set only), "The new approach"
-// Eq. 4 / Eq. 9 (current block always kept with gate 1; in training mode log g_m added to the
-// logits of selected history block m), "Kernel implementation" paragraph of "How it works" (the
-// gate is fused into a FlashAttention-style tiled qK^T loop: K/V tiles stream in, the log-gate is
-// added to the logits, unselected blocks never enter, the current block is unbiased, an online
-// softmax keeps the attention matrix out of memory).
+// [FreeSolo] "How it works": the NoPE long branch attends each query to the tokens of its top-K
+// cells, and the two branches mix through alpha_h.  For cells other than 16, 32 or 64 tokens this
+// runs per 64-query unit over the sorted union of the 64-key blocks that hold the unit's rows'
+// cells, with a per-row mask keeping only the row's own cells (the cell-major kernel of fs_long.cu
+// takes cells of 16, 32 and 64).
 //
-// One CTA takes two query units (64 queries each) -- heads h and h+1 of the same kv group at the
-// same unit u -- and runs them in lockstep over their block lists (selected history blocks, then
-// the diagonal current block).  Each unit is an M = 64 tile; the two tiles' accumulators occupy
-// complementary halves of the TMEM lanes (rows of unit 0 in lanes 0-15 of every 32-lane
-// sub-partition, unit 1 in lanes 16-31), so the four softmax warps own one row per thread.
+// One CTA takes two units (units 2up and 2up+1 of head h) and runs them in lockstep over their
+// union lists.  Each unit is an M = 64 tile; the two tiles' accumulators occupy complementary
+// halves of the TMEM lanes (rows of unit 0 in lanes 0-15 of every 32-lane sub-partition, unit 1 in
+// lanes 16-31), so the four softmax warps own one row per thread.
 //
-//   warp 4  (1 thread): TMA producer: Q tiles once, then per step the K and V blocks of both units
-//                       (128-byte swizzled 64x64 boxes) into a 2-stage ring.
+//   warp 4  (1 thread): TMA producer: Q tiles once, then per step the K blocks of both units
+//                       (128-byte swizzled 64x64 boxes) into their ring.
 //   warp 5  (1 thread): MMA issuer: S_j = Q K_j^T into a double-buffered TMEM score tile, issued one
 //                       step ahead; O += P_j V_j once the softmax has written P_j.
-//   warps 0-3 (128):    softmax: tcgen05.ld of the score row, gate bias / causal mask, online max
-//                       with lazy rescaling (O in TMEM is rescaled only when the row max grows by
-//                       more than 2^8), P written to shared memory in the MMA's swizzled layout;
-//                       epilogue O / l and lse.
+//   warp 6  (1 thread): V producer.
+//   warps 0-3 (128):    softmax: tcgen05.ld of the score row, the row's cell mask, online max with
+//                       lazy rescaling (O in TMEM is rescaled only when the row max grows by more
+//                       than 2^8), P written to shared memory in the MMA's swizzled layout;
+//                       epilogue: o = (1 - alpha) o_short + alpha o_long.
 // Every mbarrier wait is bounded; on timeout the CTA records it, skips the rest of its work and
-// still reaches its final barrier and TMEM release.
+// still reaches its final barrier and TMEM release.  The SAS forward has its own kernel
+// (sas_fwd_tc.cu).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -37,24 +38,14 @@ constexpr int kMaxKtc = 64;        // selected history blocks per unit
 constexpr int kThreadsTc = 192;    // gate gradient: 4 reduction warps + producer + MMA
 constexpr int kThreadsFwd = 224;   // forward: 4 softmax warps + K producer + MMA + V producer
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.f;    // lazy rescale threshold (log2 units)
 
 struct TcParams {
-  int B, Hq, Hk, n, U, K;
-  const int* idx;
-  const int* count;
-  int gate, norm;
-  const float* scores;
-  int scores_ld;
+  int B, Hq, Hk, n, U;
   void* o;
-  float* lse;
   int* status;
-  int mode;    // 0: heads 2hp, 2hp+1 at unit u (selected blocks); 1: units 2up, 2up+1 of head h
-               // over a sliding window; 2: units 2up, 2up+1 of head h over their selected cells
-  int window;  // mode 1: keys j >= i - window + 1 of a sliding window (blocks of the window)
-  // mode 2 (FreeSolo long branch): each unit walks the sorted union of the 64-key blocks that
-  // hold its rows' selected cells; a row sees only the keys of its own cells
+  // each unit walks the sorted union of the 64-key blocks that hold its rows' selected cells; a
+  // row sees only the keys of its own cells
   const int* ulist;    // [B * Hq * U][ucap] union blocks of each unit
   const int* ucnt;     // [B * Hq * U]
   int ucap;
@@ -83,10 +74,9 @@ struct TcSmem {
   static constexpr int kTotal = kP + 4 * kPBytes;  // mbarriers live in static shared memory
 };
 
-// MODE (p.mode) is a template argument so that each mode compiles without the others' code.
-template <int D, int MODE>
+template <int D>
 __global__ void __launch_bounds__(kThreadsFwd, 1)
-    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq,
+    long_union_tc_kernel(const __grid_constant__ CUtensorMap tmq,
                       const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const TcParams p) {
   using L = TcSmem<D>;
@@ -107,81 +97,23 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   uint64_t* fin = bars + 29;
 
   __shared__ uint32_t s_tmem;
-  __shared__ int s_blk[2][kMaxKtc + 1];
-  __shared__ float s_bias[2][kMaxKtc + 1];
   __shared__ int s_cnt[2];
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bi = blockIdx.z;
-  constexpr bool win = MODE == 1;
-  constexpr bool fsl = MODE == 2;
-  constexpr bool unit_pairs = MODE != 0;
-  // the two work items: (head, unit) pairs sharing one kv head
-  const int hq[2] = {unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y,
-                     unit_pairs ? (int)blockIdx.y : 2 * (int)blockIdx.y + 1};
-  const int uu[2] = {unit_pairs ? 2 * (int)blockIdx.x : (int)blockIdx.x,
-                     unit_pairs ? 2 * (int)blockIdx.x + 1 : (int)blockIdx.x};
+  // the two work items: units 2up, 2up+1 of head h
+  const int hq[2] = {(int)blockIdx.y, (int)blockIdx.y};
+  const int uu[2] = {2 * (int)blockIdx.x, 2 * (int)blockIdx.x + 1};
   const bool item_ok[2] = {uu[0] < p.U, uu[1] < p.U};
   const int G = p.Hq / p.Hk;
-  const int kh = hq[0] / G;  // both items read the same kv head
-  const int wblocks = win ? (p.window - 1 + kTiles - 1) / kTiles : 0;
+  const int kh = hq[0] / G;
 
-  // ---- prologue: block lists and gate biases of both items (warps 0 and 1) -----------------
-  if (warp < 2 && fsl) {  // union lists come from global memory
-    if (lane == 0) {
-      const int it = warp;
-      const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
-      s_cnt[it] = item_ok[it] ? min(p.ucnt[urow], p.ucap) : 0;
-    }
-  } else if (warp < 2 && win) {  // sliding window: blocks u - wblocks .. u - 1 before the diagonal one
+  // ---- prologue: the sizes of both items' union lists (warps 0 and 1) ---------------------
+  if (warp < 2 && lane == 0) {
     const int it = warp;
-    const int u = uu[it];
-    const int first = item_ok[it] ? max(0, u - wblocks) : 0;
-    const int cnt = item_ok[it] ? u - first : 0;
-    for (int j = lane; j < cnt && j < kMaxKtc; j += 32) {
-      s_blk[it][j] = first + j;
-      s_bias[it][j] = 0.f;
-    }
-    if (lane == 0) s_cnt[it] = min(cnt, kMaxKtc);
-  } else if (warp < 2) {
-    const int it = warp;
-    const int u = uu[it];
-    const int nc = u;  // history blocks before unit u (q_block == b)
-    const size_t row = ((size_t)bi * p.Hq + hq[it]) * p.U + u;
-    const int cnt_in = p.count ? min(p.count[row], p.K) : p.K;
-    int base = 0;
-    for (int j0 = 0; j0 < cnt_in; j0 += 32) {
-      const int j = j0 + lane;
-      const int m = j < cnt_in ? p.idx[row * p.K + j] : -1;
-      const bool ok = j < cnt_in && m >= 0 && m < nc;
-      const unsigned bal = __ballot_sync(0xffffffffu, ok);
-      if (ok && base + __popc(bal & ((1u << lane) - 1u)) < kMaxKtc)
-        s_blk[it][base + __popc(bal & ((1u << lane) - 1u))] = m;
-      base += __popc(bal);
-    }
-    base = min(base, kMaxKtc);
-    float lnorm = 0.f;
-    if (p.gate != BSA_GATE_NONE) {  // log2 g_m of the softmax gate, inside or outside the softmax
-      const float* srow = p.scores + row * p.scores_ld;
-      __syncwarp();
-      float mx = -INFINITY, acc = 0.f;
-      if (p.norm == BSA_NORM_ALL_HISTORY) {
-        for (int c = lane; c < nc; c += 32) mx = fmaxf(mx, srow[c]);
-        mx = warp_max(mx);
-        for (int c = lane; c < nc; c += 32) acc += exp2f((srow[c] - mx) * kLog2e);
-      } else {
-        for (int j = lane; j < base; j += 32) mx = fmaxf(mx, srow[s_blk[it][j]]);
-        mx = warp_max(mx);
-        for (int j = lane; j < base; j += 32) acc += exp2f((srow[s_blk[it][j]] - mx) * kLog2e);
-      }
-      acc = warp_sum(acc);
-      lnorm = mx == -INFINITY ? 0.f : mx + logf(acc);
-      for (int j = lane; j < base; j += 32) s_bias[it][j] = (srow[s_blk[it][j]] - lnorm) * kLog2e;
-    } else {
-      for (int j = lane; j < base; j += 32) s_bias[it][j] = 0.f;
-    }
-    if (lane == 0) s_cnt[it] = base;
+    const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
+    s_cnt[it] = item_ok[it] ? min(p.ucnt[urow], p.ucap) : 0;
   }
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -215,16 +147,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // modes 0 and 1 end on the diagonal block; the long branch has none
-  const int steps = max(s_cnt[0], s_cnt[1]) + (fsl ? 0 : 1);
+  const int steps = max(s_cnt[0], s_cnt[1]);
   const uint32_t tmem = s_tmem;
-  // step j of unit it: history block, filler (fully masked) or the current block (last step)
+  // step j of unit it: a block of its union, or a filler (fully masked) past the list's end
   auto step_block = [&](int it, int j) {
-    if (fsl) {
-      const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
-      return j < s_cnt[it] ? p.ulist[urow * p.ucap + j] : 0;
-    }
-    return j < s_cnt[it] ? s_blk[it][j] : (item_ok[it] ? uu[it] : uu[0]);
+    const size_t urow = ((size_t)bi * p.Hq + hq[it]) * p.U + uu[it];
+    return j < s_cnt[it] ? p.ulist[urow * p.ucap + j] : 0;
   };
 
   auto kslot = [&](int slot) { return smem + L::kK + slot * 2 * L::kTileBytes; };
@@ -335,16 +263,15 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     const int it = lane >> 4;                  // item of this thread's row
     const int r = 16 * warp + (lane & 15);     // row within the unit
     const int i = uu[it] * kTiles + r;         // query position
-    const int wlo = win ? i - p.window + 1 : INT_MIN;  // lowest key of the window
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
     const float qk_scale = rsqrtf((float)D) * kLog2e;
-    // long branch: this row's cells that lie wholly at or before it (never a future key)
+    // this row's cells that lie wholly at or before it (never a future key)
     constexpr int kSelMax = 8;
     int my_cells[kSelMax];
     int nmine = 0;
 #pragma unroll
     for (int k = 0; k < kSelMax; ++k) my_cells[k] = -1;
-    if (fsl && item_ok[it] && i < p.n) {
+    if (item_ok[it] && i < p.n) {
       const size_t qrow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
       const int cnt = p.sel_cnt ? min(p.sel_cnt[qrow], p.ksel) : p.ksel;
 #pragma unroll
@@ -379,22 +306,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (j >> 1) & 1));
       if (!ok) break;
       tc::fence_after_sync();
-      // bias or mask of this step's block for my unit
-      const bool is_cur = !fsl && (j == steps - 1);
-      const bool filler = !is_cur && j >= s_cnt[it];
-      const float lg = (!is_cur && !filler && !fsl) ? s_bias[it][j] : 0.f;  // log2 g_m
-      // inner gate: a logit bias; outer gate: P scaled by g_m for P V (the row sum stays ungated)
-      const bool outer = p.gate == BSA_GATE_OUTER;
-      const float bias = outer ? 0.f : lg;
-      const float vs = outer ? tc::ex2_approx(lg) : 1.f;
-      const int kpos0 = blk * kTiles;  // position of this block's first key
-      // keys of this block the row may see: all of a history block; none of a filler; c <= r on
-      // the diagonal; c >= wlo - kpos0 inside a sliding window; the keys of the row's own cells
-      // in the long branch
+      // keys of this block the row may see: the keys of the row's own cells (none for a filler)
+      const bool filler = j >= s_cnt[it];
+      const float bias = 0.f;
       uint64_t keep = filler ? 0ull : ~0ull;
-      if (is_cur) keep &= r >= 63 ? ~0ull : ((2ull << r) - 1ull);
-      if (wlo - kpos0 > 0) keep &= wlo - kpos0 >= 64 ? 0ull : (~0ull << (wlo - kpos0));
-      if (fsl && !filler) {
+      if (!filler) {
         uint64_t mine = 0ull;
 #pragma unroll
         for (int k = 0; k < kSelMax; ++k) mine |= cell_blk[k] == blk ? cell_keys[k] : 0ull;
@@ -422,7 +338,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       mbar_arrive(&s_free[st]);
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (warp_live) {
-        if (fsl && p.cell >= 8) {
+        if (p.cell >= 8) {
           // cell masks are whole 8-key chunks: per chunk a (scale, bias) of (0, -inf) masks it
           // with the same one FMA per key as the unmasked path (scores are finite); every lane
           // takes this path, so a warp whose rows see different cells does not diverge
@@ -463,13 +379,13 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
-      if (warp_live) {  // outer gate: P V takes g_m p (vs = g_m), the row sum p; inner: vs = 1
+      if (warp_live) {
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float p0 = tc::ex2_approx(x[c] - m_use);
           const float p1 = tc::ex2_approx(x[c + 1] - m_use);
           sum4[(c >> 1) & 3] += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0 * vs, p1 * vs);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
         }
       } else {
@@ -522,10 +438,10 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
     if (ok && steps > 0) {
       tc::fence_after_sync();
       // the long branch mixes into the short branch already in o, for rows that saw a cell
-      const bool live = i < p.n && item_ok[it] && (!fsl || nmine > 0);
+      const bool live = i < p.n && item_ok[it] && nmine > 0;
       const size_t orow = ((size_t)bi * p.Hq + hq[it]) * p.n + i;
-      const float a_mix = fsl ? p.alpha[hq[it]] : 1.f;
-      const float inv = (fsl ? a_mix : 1.f) / l_run;
+      const float a_mix = p.alpha[hq[it]];
+      const float inv = a_mix / l_run;
       __nv_bfloat16* op = static_cast<__nv_bfloat16*>(p.o) + orow * D;
       for (int c0 = 0; c0 < D; c0 += 32) {
         float ov[32];
@@ -533,16 +449,11 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
         tc::tmem_wait_ld();
         if (live) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            if (fsl) {  // o = (1 - alpha) o_short + alpha o_long
-              float sh[8];
-              load_vec<__nv_bfloat16, 8>(op + c0 + c, sh);
+          for (int c = 0; c < 32; c += 8) {  // o = (1 - alpha) o_short + alpha o_long
+            float sh[8];
+            load_vec<__nv_bfloat16, 8>(op + c0 + c, sh);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) ov[c + e] = fmaf(ov[c + e], inv, (1.f - a_mix) * sh[e]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) ov[c + e] *= inv;
-            }
+            for (int e = 0; e < 8; ++e) ov[c + e] = fmaf(ov[c + e], inv, (1.f - a_mix) * sh[e]);
             uint4 w4;
             __nv_bfloat162 h;
             h = __floats2bfloat162_rn(ov[c], ov[c + 1]);
@@ -557,7 +468,6 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
           }
         }
       }
-      if (live && p.lse) p.lse[orow] = (m_run + log2f(l_run)) * kLn2;
     } else if (steps > 0) {
       ok = false;
     }
@@ -579,7 +489,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
 //     dg_m = sum_{i in B_m} (ptilde_i / g_m) do^T (v_i - o),
 // summed over the unit's queries, in the stable form
 //     dg_m = sum_q sum_{j in B_m} exp(z_qj - lse_q) (do_q . v_j - do_q . o_q),   z = q . k / sqrt(d).
-// Same CTA shape as the forward: heads h and h+1 at unit u, rows in the lane order of the M = 64
+// One CTA per pair of units (heads h and h+1 at unit u), rows in the lane order of the M = 64
 // accumulators.  Per selected history block j the MMA thread computes Z_j = [Q_0; Q_1] [K_0; K_1]^T
 // and DV_j = [dO_0; dO_1] [V_0; V_1]^T as M = 128, N = 128 chains (the cross products are never
 // read) into a double-buffered TMEM pair; each reduction-warp thread reduces its row, and the 64
@@ -930,14 +840,13 @@ bsa_status launch_tc(const void* q, const void* k, const void* v, const TcParams
       !make_map(&tmv, v, (long long)p.B * p.Hk * p.n, D))
     return BSA_ERR_CUDA;
   const int smem = TcSmem<D>::kTotal + 1024;  // + alignment slack
-  auto kern = p.mode == 0 ? prefill_tc_kernel<D, 0>
-                          : (p.mode == 1 ? prefill_tc_kernel<D, 1> : prefill_tc_kernel<D, 2>);
+  auto kern = long_union_tc_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess) {
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
-  dim3 grid = p.mode != 0 ? dim3((p.U + 1) / 2, p.Hq, p.B) : dim3(p.U, p.Hq / 2, p.B);
+  const dim3 grid((p.U + 1) / 2, p.Hq, p.B);
   kern<<<grid, kThreadsFwd, smem, st>>>(tmq, tmk, tmv, p);
   return BSA_OK;
 }
@@ -981,9 +890,8 @@ bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void*
   return BSA_OK;
 }
 
-// Sliding-window causal attention (window keys j in [i - window + 1, i]) of already rotated q/k
-// on the tensor cores: the short branch of the FreeSolo prefill, written to o.
-// Long branch of the FreeSolo prefill on the tensor cores (mode 2), mixing into o.
+// Long branch of the FreeSolo prefill on the tensor cores over each unit's block union, mixing
+// into o.
 // Workspace: union counts [B * H * U] then lists [B * H * U][ucap], ucap = min(64 * 8, blocks).
 static int long_ucap(int n) { return min(64 * 8, ceil_div(n, kTiles)); }
 
@@ -1012,8 +920,8 @@ bsa_status long_attn_tc(const void* q, const void* k, const void* v, int B, int 
       sel, sel_cnt, H, n, U, ksel, cell, ucap, ucnt, ulist);
   BSA_LAUNCH_CHECK();
   TcParams p{};
-  p.B = B; p.Hq = H; p.Hk = H; p.n = n; p.U = U; p.K = 0;
-  p.o = o; p.lse = nullptr; p.status = status; p.mode = 2; p.window = 0;
+  p.B = B; p.Hq = H; p.Hk = H; p.n = n; p.U = U;
+  p.o = o; p.status = status;
   p.ulist = ulist; p.ucnt = ucnt; p.ucap = ucap;
   p.sel = sel; p.sel_cnt = sel_cnt; p.ksel = ksel; p.cell = cell; p.alpha = alpha;
   bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
@@ -1039,18 +947,10 @@ bsa_status prefill_tc(const void* q, const void* k, const void* v, int B, int Hq
                       const float* scores, int scores_ld, void* o, float* lse, int* status,
                       cudaStream_t st) {
   (void)b;
-  // the step-split kernel (two softmax warpgroups) covers every shape this path accepts
-  const bsa_status pp = sas_fwd_tc(q, k, v, B, Hq, Hk, n, d, idx, count, K, gate, norm, scores,
-                                   scores_ld, o, lse, status, st);
-  if (pp != BSA_ERR_UNSUPPORTED) return pp;
-  TcParams p{};
-  p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.U = ceil_div(n, kTiles); p.K = K;
-  p.idx = idx; p.count = count; p.gate = gate; p.norm = norm;
-  p.scores = scores; p.scores_ld = scores_ld; p.o = o; p.lse = lse; p.status = status;
-  bsa_status rc = d == 64 ? launch_tc<64>(q, k, v, p, st) : launch_tc<128>(q, k, v, p, st);
-  if (rc != BSA_OK) return rc;
-  BSA_LAUNCH_CHECK();
-  return BSA_OK;
+  // the forward runs on the step-split kernel of sas_fwd_tc.cu, which takes every shape that
+  // prefill_tc_supported admits
+  return sas_fwd_tc(q, k, v, B, Hq, Hk, n, d, idx, count, K, gate, norm, scores, scores_ld, o, lse,
+                    status, st);
 }
 
 }  // namespace bsa
