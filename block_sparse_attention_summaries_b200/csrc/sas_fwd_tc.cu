@@ -41,6 +41,13 @@ constexpr float kSLog2e = 1.4426950408889634f;
 constexpr float kSLn2 = 0.6931471805599453f;
 constexpr float kSRescale = 8.f;
 
+// max(a, b, c) in one instruction (the three-input form of sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 struct SasParams {
   int B, Hq, Hk, n, U, K;
   const int* idx;
@@ -316,24 +323,29 @@ __global__ void __launch_bounds__(kSasThreads, 1)
       // inner gate: a logit bias; outer gate: P scaled by g_m for P V (the row sum stays ungated)
       const float bias = outer ? 0.f : lg;
       const float vs = outer ? tc::ex2_approx(lg) : 1.f;
-      // keys the row sees: all of a history block, none of a filler, c <= r on the diagonal
+      // keys the row sees: all of a history block, none of a filler, c <= r on the diagonal (the
+      // masked form runs for the whole warp when any of its rows needs it)
       uint64_t keep = filler ? 0ull : ~0ull;
       if (is_cur) keep &= r >= 63 ? ~0ull : ((2ull << r) - 1ull);
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (keep == ~0ull) {
+      if (__any_sync(0xffffffffu, keep != ~0ull)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = fmaf(x[c], qk_scale, bias);
-          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = ((keep >> c) & 1ull) ? fmaf(x[c], qk_scale, bias) : -INFINITY;
-          mx4[c & 3] = fmaxf(mx4[c & 3], x[c]);
-        }
+        for (int c = 0; c < 64; ++c) x[c] = ((keep >> c) & 1ull) ? x[c] : -INFINITY;
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      // row maximum of the raw scores (three-input maxima); the scale is positive and the bias
+      // the same for the whole block, so the logit maximum is max * scale + bias and each key
+      // needs one FMA before its exp2
+      float mx4[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = max3f(x[q4], x[4 + q4], x[8 + q4]);  // 0-11
+#pragma unroll
+      for (int c = 12; c + 8 <= 64; c += 8) {  // 12-59
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = max3f(mx4[q4], x[c + q4], x[c + 4 + q4]);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = fmaxf(mx4[q4], x[60 + q4]);  // 60-63
+      const float mraw = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+      const float mx = mraw == -INFINITY ? -INFINITY : fmaf(mraw, qk_scale, bias);
       const float m_new = fmaxf(m_run, mx);
       // the first finite max needs no O scaling (the row's O and l are still 0); later ones
       // rescale O only when the max grows by more than 2^8
@@ -341,13 +353,14 @@ __global__ void __launch_bounds__(kSasThreads, 1)
       float corr = 1.f;
       if (rescale) corr = tc::ex2_approx(m_run - m_new);
       if (rescale || m_run == -INFINITY) m_run = m_new;
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;  // masked keys give 2^-inf = 0
+      // masked keys give 2^-inf = 0; a row with nothing seen yet subtracts 0
+      const float off = bias - (m_run == -INFINITY ? 0.f : m_run);
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float p0 = tc::ex2_approx(x[c] - m_use);
-        const float p1 = tc::ex2_approx(x[c + 1] - m_use);
+        const float p0 = tc::ex2_approx(fmaf(x[c], qk_scale, off));
+        const float p1 = tc::ex2_approx(fmaf(x[c + 1], qk_scale, off));
         sum4[(c >> 1) & 3] += p0 + p1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0 * vs, p1 * vs);
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);

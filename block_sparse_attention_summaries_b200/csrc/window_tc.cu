@@ -35,6 +35,13 @@ constexpr int kWThreads = 224;  // 4 softmax warps + Q/K producer + MMA + V prod
 constexpr float kWLog2e = 1.4426950408889634f;
 constexpr float kWRescale = 8.f;  // lazy O rescale threshold (log2 units)
 
+// max(a, b, c) in one instruction (the three-input form of sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 template <int D>
 struct WinSmem {
   static constexpr int kQBytes = kWT * D * 2;    // [half][128 rows x 128 B]
@@ -282,35 +289,39 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
       tc::reg_fence(x);
       tc::fence_before_sync();
       mbar_arrive(&s_free[st]);
-      // keys of block b the row sees: j in [i - window + 1, i]
+      // keys of block b the row sees: j in [i - window + 1, i]; the masked form runs for the
+      // whole warp when any of its rows needs it (most blocks of a tile need none)
       const int lo = i - w.window + 1 - kWB * b, hi = i - kWB * b;  // column bounds
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (lo <= 0 && hi >= kWB - 1) {
+      if (!__all_sync(0xffffffffu, lo <= 0 && hi >= kWB - 1)) {
 #pragma unroll
-        for (int col = 0; col < kWB; ++col) {
-          x[col] *= qk_scale;
-          mx4[col & 3] = fmaxf(mx4[col & 3], x[col]);
-        }
-      } else {
-#pragma unroll
-        for (int col = 0; col < kWB; ++col) {
-          x[col] = (col >= lo && col <= hi) ? x[col] * qk_scale : -INFINITY;
-          mx4[col & 3] = fmaxf(mx4[col & 3], x[col]);
-        }
+        for (int col = 0; col < kWB; ++col) x[col] = (col >= lo && col <= hi) ? x[col] : -INFINITY;
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      // row maximum of the raw scores (three-input maxima), then in log2 units: the scale is
+      // positive, so the maximum commutes with it and each key needs one FMA before its exp2
+      static_assert(kWB == 64, "the maximum below covers 64 columns");
+      float mx4[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = max3f(x[q4], x[4 + q4], x[8 + q4]);  // 0-11
+#pragma unroll
+      for (int col = 12; col + 8 <= kWB; col += 8) {  // 12-59
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = max3f(mx4[q4], x[col + q4], x[col + 4 + q4]);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) mx4[q4] = fmaxf(mx4[q4], x[60 + q4]);  // 60-63
+      const float mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * qk_scale;
       const float m_new = fmaxf(m_run, mx);
       const bool rescale = m_run != -INFINITY && m_new > m_run + kWRescale;
       float corr = 1.f;
       if (rescale) corr = tc::ex2_approx(m_run - m_new);
       if (rescale || m_run == -INFINITY) m_run = m_new;
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const float neg_m = m_run == -INFINITY ? 0.f : -m_run;  // masked keys give 2^-inf = 0
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
 #pragma unroll
       for (int col = 0; col < kWB; col += 2) {
-        const float p0 = tc::ex2_approx(x[col] - m_use);
-        const float p1 = tc::ex2_approx(x[col + 1] - m_use);
+        const float p0 = tc::ex2_approx(fmaf(x[col], qk_scale, neg_m));
+        const float p1 = tc::ex2_approx(fmaf(x[col + 1], qk_scale, neg_m));
         sum4[(col >> 1) & 3] += p0 + p1;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[col / 2] = *reinterpret_cast<const uint32_t*>(&h2);
