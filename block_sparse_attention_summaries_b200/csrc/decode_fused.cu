@@ -397,6 +397,12 @@ __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, ui
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                               uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -434,6 +440,7 @@ struct FusedSmem {
 template <typename T, typename TS, int D, int G, bool MMA>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+    const __grid_constant__ CUtensorMap tmk64, const __grid_constant__ CUtensorMap tmv64,
     const FusedParams p) {
   constexpr bool kMma = MMA;
   static_assert(!MMA || std::is_same<T, __nv_bfloat16>::value, "warp MMAs take bf16");
@@ -776,6 +783,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       const int nsl = min(4, S_tot - first);
       mbar_arrive_expect_tx(&kvbar[st], (uint32_t)(nsl * 2 * kSlice * D * 2));
       const uint64_t pol = l2_evict_first();
+      if (first < s_hist) {  // a whole history block (four aligned slices): 64-row boxes
+        const int y = row0 + s_ublk[g] * b;
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          tc::tma_load_2d_hint(ktile(st) + hf * 8192, &tmk64, hf * 64, y, &kvbar[st], pol);
+          tc::tma_load_2d_hint(vtile(st) + hf * 8192, &tmv64, hf * 64, y, &kvbar[st], pol);
+        }
+        return;
+      }
       for (int w = 0; w < nsl; ++w) {
         const int s = first + w;
         const int y = row0 + slice_blk(s) * b + slice_tok0(s);
@@ -843,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
           p.centre[row] = 0.5f * (float)(cur * b) + 0.5f * (float)(cur * b + tok_cur - 1);
       }
     }
-    // A fragments of Q (rows = heads, zero beyond G), pre-scaled into log2 units
+    // B fragments of Q^T (k = d, n = heads, zero beyond G), pre-scaled into log2 units
     const int grow = lane >> 2, tig = lane & 3;
     uint32_t qa0[D / 16], qa1[D / 16];
     {
@@ -866,7 +882,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     float oacc[D / 16][4];
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) oacc[c][0] = oacc[c][1] = oacc[c][2] = oacc[c][3] = 0.f;
-    float m_run = -INFINITY, l_part = 0.f;
+    // online softmax of heads 2 tig and 2 tig + 1 (the accumulator columns this lane holds)
+    float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
     // the group leader asks for the global stage of its next refill one stage ahead, so that the
     // remote atomic's round trip overlaps a stage's work
     const bool leader = wg == 0 && lane == 0;
@@ -906,65 +923,63 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         const unsigned char* kt = ktile(st);
         const unsigned char* vt = vtile(st);
         const int t0 = wg * kSlice;  // this warp's 16 rows of the stage tile
-        // S = Q K^T over two 8-token tiles
-        float sfr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          const int tokr = t0 + 8 * nt + grow;  // B fragment row (token)
+        // S^T = K Q^T (m = the slice's 16 tokens, n = heads): one m16n8k16 per 16-wide d step,
+        // its A fragments (K rows) from one ldmatrix.x4 (matrices: tokens 0-7 / 8-15 x d chunks
+        // 2 (ks & 3) and 2 (ks & 3) + 1)
+        float sfr[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          const int mi = lane >> 3, rr = lane & 7;
+          const int tokr = t0 + ((mi & 1) << 3) + rr;  // the token row this lane addresses
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            const int hf = ks >> 2, ch = (ks & 3) * 2;
-            const unsigned char* rowp = kt + hf * 8192 + tokr * 128;
-            const uint32_t b0 =
-                *reinterpret_cast<const uint32_t*>(rowp + ((ch ^ (tokr & 7)) << 4) + 4 * tig);
-            const uint32_t b1 =
-                *reinterpret_cast<const uint32_t*>(rowp + (((ch + 1) ^ (tokr & 7)) << 4) + 4 * tig);
-            mma_16816(sfr[nt], qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+            const int chunk = (ks & 3) * 2 + (mi >> 1);
+            const uint32_t addr =
+                smem_u32(kt + (ks >> 2) * 8192 + tokr * 128 + ((chunk ^ (tokr & 7)) << 4));
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+            mma_16816(sfr, a0, a1, a2, a3, qa0[ks], qa1[ks]);
           }
         }
-        // masks, per-row online softmax (row = head grow; the quad shares the row)
-        const bool head_on = grow < G && ((hm >> grow) & 1u);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int t = 8 * nt + 2 * tig + e;
-            if (!head_on || t >= tv) sfr[nt][e] = -INFINITY;
-            mx = fmaxf(mx, sfr[nt][e]);
-          }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        float corr = 1.f;  // rescale of head `grow` (lazy: only when its max grows by > 2^8)
-        if (mx > m_run + kRescale || (m_run == -INFINITY && mx != -INFINITY)) {
-          corr = m_run == -INFINITY ? 0.f : exp2f(m_run - mx);
-          m_run = mx;
-          l_part *= corr;
-        }
-        // O^T columns are heads: this lane holds heads 2 tig and 2 tig + 1
-        const float corr_a = __shfl_sync(0xffffffffu, corr, 8 * tig);
-        const float corr_b = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
-        if (__any_sync(0xffffffffu, corr_a != 1.f || corr_b != 1.f)) {
-#pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            oacc[c][0] *= corr_a;
-            oacc[c][1] *= corr_b;
-            oacc[c][2] *= corr_a;
-            oacc[c][3] *= corr_b;
-          }
-        }
+        // masks and the online softmax per head; this lane holds tokens grow and grow + 8 of
+        // heads 2 tig + e (sfr[e], sfr[2 + e]); the slice's other tokens of the same heads are in
+        // the lanes of the same tig
         float pv[2][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float z = sfr[nt][e];
-            pv[nt][e] = z == -INFINITY ? 0.f : exp2f(z - m_run);
-            l_part += pv[nt][e];
+        for (int e = 0; e < 2; ++e) {
+          const int h = 2 * tig + e;
+          const bool head_on = h < G && ((hm >> h) & 1u);
+          if (!head_on || grow >= tv) sfr[e] = -INFINITY;
+          if (!head_on || grow + 8 >= tv) sfr[2 + e] = -INFINITY;
+          float mx = fmaxf(sfr[e], sfr[2 + e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          // lazy rescale: only when the head's max grows by more than 2^8
+          float corr = 1.f;
+          if (mx > m_run[e] + kRescale || (m_run[e] == -INFINITY && mx != -INFINITY)) {
+            corr = m_run[e] == -INFINITY ? 0.f : exp2f(m_run[e] - mx);
+            m_run[e] = mx;
+            l_part[e] *= corr;
           }
-        // P^T as the B operand (k = tokens, n = heads): exactly the S accumulator pairs
-        const uint32_t pb0 = pack_bf16(pv[0][0], pv[0][1]);
-        const uint32_t pb1 = pack_bf16(pv[1][0], pv[1][1]);
+          if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+              oacc[c][e] *= corr;
+              oacc[c][2 + e] *= corr;
+            }
+          }
+          pv[0][e] = sfr[e] == -INFINITY ? 0.f : exp2f(sfr[e] - m_run[e]);
+          pv[1][e] = sfr[2 + e] == -INFINITY ? 0.f : exp2f(sfr[2 + e] - m_run[e]);
+          l_part[e] += pv[0][e] + pv[1][e];
+        }
+        // P^T as the B operand (k = tokens, n = heads): the 8 x 8 blocks (tokens 0-7 and 8-15 x
+        // heads) this lane holds by token rows, transposed in registers
+        uint32_t pb0, pb1;
+        {
+          const uint32_t x0 = pack_bf16(pv[0][0], pv[0][1]), x1 = pack_bf16(pv[1][0], pv[1][1]);
+          asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb0) : "r"(x0));
+          asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(pb1) : "r"(x1));
+        }
         // O^T += V^T P^T: A fragments of V^T by transposed 8x8 loads of the swizzled V tile
 #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt) {
@@ -994,13 +1009,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       report_timeout(p.status, 2);
     }
     __syncthreads();
-    // warp partials (rows < G): m, l and o
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-    if (grow < G && tig == 0) {
-      float* wp = wpart + ((size_t)warp * G + grow) * (D + 2);
-      wp[D] = m_run;
-      wp[D + 1] = l_part;
+    // warp partials (heads < G): m, l and o
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 4);
+      l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 8);
+      l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 16);
+      const int h = 2 * tig + e;
+      if (grow == 0 && h < G) {
+        float* wp = wpart + ((size_t)warp * G + h) * (D + 2);
+        wp[D] = m_run[e];
+        wp[D + 1] = l_part[e];
+      }
     }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {  // O^T element (d, head 2 tig + e)
@@ -1259,13 +1279,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// K or V as [rows, D] bf16 with 64-column x 16-row boxes, 128-byte swizzle
-bool kv_map(CUtensorMap* m, const void* base, long long rows, int D) {
+// K or V as [rows, D] bf16 with 64-column x box_rows boxes (16: one slice; 64: a whole block),
+// 128-byte swizzle
+bool kv_map(CUtensorMap* m, const void* base, long long rows, int D, int box_rows = kSlice) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kSlice};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1292,10 +1313,12 @@ constexpr size_t kStaticSmemBound = 12 * 1024;
 template <typename T, typename TS, int D, int G, bool MMA>
 bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   using SM = FusedSmem<T, TS, D, G, MMA>;
-  CUtensorMap tmk{}, tmv{};
+  CUtensorMap tmk{}, tmv{}, tmk64{}, tmv64{};
   if (MMA) {
     const long long rows = (long long)p.B * p.Hk * p.n;
-    if (!kv_map(&tmk, p.k, rows, D) || !kv_map(&tmv, p.v, rows, D)) return BSA_ERR_CUDA;
+    if (!kv_map(&tmk, p.k, rows, D) || !kv_map(&tmv, p.v, rows, D) ||
+        !kv_map(&tmk64, p.k, rows, D, 64) || !kv_map(&tmv64, p.v, rows, D, 64))
+      return BSA_ERR_CUDA;
   }
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
@@ -1411,7 +1434,7 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
       min_per_sm = 2;
       continue;
     }
-    if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, tmk64, tmv64, p) != cudaSuccess) {
       (void)cudaGetLastError();
       return BSA_ERR_CUDA;
     }
