@@ -52,12 +52,7 @@ WORKLOADS = {
 # profile summary under profiles/).  Reported only while the source is unchanged.
 # The hash covers the device code of the source: the file up to its first host function
 # (`device_end`), so a change of the host-side launcher alone keeps the figure.
-MEASURED_TRAFFIC = {
-    ("sas_gqa_decode_32k", "decode_fused_kernel"): {
-        "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "d20e35e11a12f316",
-        "bytes": 52_598_784 + 298_496},
-}
+MEASURED_TRAFFIC = {}
 
 
 def device_source_hash(path: str, device_end: str) -> str:
@@ -622,16 +617,22 @@ def build_layers(dev, case, w, R):
     return layers
 
 
-def capture_fused(dev, layers, w, status, stream):
-    """CUDA graphs of the fused decode step (one kernel launch per step): one graph per layer,
-    and one graph of a whole decode iteration (every layer's step in order, as a model replays
-    one graph per generated token). Returns (per-layer graphs, iteration graph)."""
+def capture_fused(dev, layers, w, status, stream, ws=None):
+    """CUDA graphs of the fused decode step (one kernel launch per step; with a workspace ``ws``,
+    long histories take the two-launch path of bsa_decode_step_ws): one graph per layer, and one
+    graph of a whole decode iteration (every layer's step in order, as a model replays one graph
+    per generated token). Returns (per-layer graphs, iteration graph)."""
     import torch
 
     import block_sparse_attention_summaries_b200 as bsa
     b, K = w["b"], w["K"]
 
     def fused(L):
+        if ws is not None:
+            bsa.decode_step_ws(L["q"], L["k"], L["v"], L["mean_k"], b, K, ws=ws, append=True,
+                               max_norm=L["max_norm"], centre=L["centre"], o=L["o"],
+                               lse=L["lse"], idx=L["idx"], count=L["count"], status=status)
+            return
         bsa.decode_step_fused(L["q"], L["k"], L["v"], L["mean_k"], b, K, append=True,
                               max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
                               idx=L["idx"], count=L["count"], status=status)
@@ -786,7 +787,11 @@ def run_long_decode(dev, peaks, args, stream):
     R = max(2, min(args.layers, 4))  # 4 x (33.5 MB summaries + union K/V) per cycle > 126 MB L2
     layers = build_layers(dev, case, w, R)
     status = torch.zeros(4, dtype=torch.int32, device=dev)
-    graphs = capture_fused(dev, layers, w, status, stream)
+    import block_sparse_attention_summaries_b200 as bsa
+    ws_bytes = bsa.decode_step_workspace_bytes(w["B"], w["Hq"], w["Hk"], w["n"], w["d"], w["b"],
+                                               w["K"])
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    graphs = capture_fused(dev, layers, w, status, stream, ws=ws)
     steps = max(50, min(args.steps, 400))
     ms = time_graph_cycle(dev, graphs, steps, args.warmup, stream) / steps
     acc = decode_accounting(case, w, layers[0]["idx"].cpu().numpy())
@@ -799,6 +804,7 @@ def run_long_decode(dev, peaks, args, stream):
            "algorithmic_bytes": algo, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
            "union_blocks": acc["union_blocks"], "needle_recall": acc["needle_recall"],
            "status_word": int(status.max().item()),
+           "launches_per_step": 2 if ws_bytes > 0 else 1, "workspace_bytes": ws_bytes,
            "separate_calls_us": sep,
            "roofline": roofline("hbm", "decode_fused_kernel", gbs, peaks["hbm_gbs"], "GB/s",
                                 traffic=measured_traffic(wl, "decode_fused_kernel"),

@@ -36,6 +36,9 @@ SIGNATURES = [
                              _I, _I, _P, _P, _P, _P, _P, _P]),
     ("bsa_decode_step_ex", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P,
                                 _P, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
+    ("bsa_decode_step_ws", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P,
+                                _P, _I, _I, _P, _P, _P, _P, _P, _I, _P, _Z, _P]),
+    ("bsa_decode_step_workspace_bytes", _Z, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     ("bsa_round_summaries_bf16", _I, [_P, _P, ctypes.c_longlong, _P]),
     ("bsa_sparse_attn_fwd", _I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P, _I,
                                  _I, _I, _P, _I, _P, _P, _P, _Z, _P]),
@@ -540,6 +543,41 @@ def decode_step_ex(q, k, v, mean_k, b, K, flags, seq_lens=None, append=True, max
                                     _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse), _ptr(idx),
                                     _ptr(count), _ptr(status), int(flags), _stream(q.device)),
            "bsa_decode_step_ex")
+    return o, lse, idx, count
+
+
+def decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, flags=0, dtype=None) -> int:
+    """Workspace bytes of bsa_decode_step_ws for this shape (0: the step is one launch)."""
+    dt = 1 if dtype in (None, torch.bfloat16) else 0
+    return int(lib().bsa_decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, int(flags), dt))
+
+
+def decode_step_ws(q, k, v, mean_k, b, K, flags=0, ws=None, seq_lens=None, append=True,
+                   max_norm=None, centre=None, lambda_h=None, sigma_h=None, prefix_block=0,
+                   o=None, lse=None, idx=None, count=None, status=None):
+    """bsa_decode_step_ws: the fused decode step; long histories on the 64-token bf16 path run as
+    two launches through the workspace ``ws`` (a uint8 device tensor; allocated here when None).
+    Returns (o, lse, idx, count)."""
+    _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count, ws)
+    B, Hk, n, d = k.shape
+    Hq = q.shape[1]
+    if o is None:
+        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+    if lse is None:
+        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+    if idx is None:
+        idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+    if count is None:
+        count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+    if ws is None:
+        need = decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, flags, q.dtype)
+        ws = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _check(lib().bsa_decode_step_ws(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b,
+                                    _ptr(_i32(seq_lens)), _ptr(mean_k), _ptr(max_norm),
+                                    _ptr(centre), 1 if append else 0, _ptr(lambda_h),
+                                    _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse), _ptr(idx),
+                                    _ptr(count), _ptr(status), int(flags), _ptr(ws), ws.numel(),
+                                    _stream(q.device)), "bsa_decode_step_ws")
     return o, lse, idx, count
 
 

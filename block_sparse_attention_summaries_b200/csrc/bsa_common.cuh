@@ -174,6 +174,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory advanced to its first 1024-byte boundary.  The advance is taken as an
+// offset on the array itself, so every pointer derived from the result stays visibly in the
+// shared state space and its accesses compile to shared-memory instructions; rounding the address
+// through an integer would hide that and turn them into generic accesses, which queue in the same
+// pipeline as global-memory requests.
+__device__ __forceinline__ unsigned char* smem_align1024(unsigned char* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }

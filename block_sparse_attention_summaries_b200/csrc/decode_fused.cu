@@ -92,6 +92,13 @@ struct FusedParams {
   int row_ld;  // stride of the whole-row key copies (gather) in keys
   int ns;      // summary ring stages
   int nkv;     // K/V ring stages
+  // Long histories in two launches: mode 1 scores one chunk of the history per CTA (no cluster)
+  // and writes every selecting head's chunk Top-K to `cand`; mode 2 merges those lists and runs
+  // phases 3-5.  Mode 0 is the whole step in one launch.
+  int mode;
+  int nchunk;      // chunks per group (modes 1 and 2)
+  int cand_ld;     // words per (chunk, head) record: K keys, K positions (rank order), count
+  uint32_t* cand;  // [B * Hk][nchunk][Gs][cand_ld]
   // dynamic shared-memory layout (byte offsets from the 1024-aligned base)
   int off_keys, off_sel, off_hbits, off_recv, off_zp, off_bar;
 };
@@ -388,6 +395,31 @@ __device__ __noinline__ int warp_select(const uint32_t* keys, int N, int K, int 
   return taken;
 }
 
+// Bitonic sort of one value per lane across the warp: descending (largest at lane 0) or ascending.
+template <typename V, bool kDescending>
+__device__ __forceinline__ V warp_sort(V v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const V o = __shfl_xor_sync(0xffffffffu, v, j);
+      // the block of size k runs in the final direction when (lane & k) == 0; the lower lane of
+      // a pair keeps the value that comes first in its block's direction
+      const bool first = (((lane & k) == 0) == ((lane & j) == 0));
+      v = (first == kDescending) ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  }
+  return v;
+}
+
+// The largest 64-bit value over the warp (two 32-bit reductions: the high words, then the low
+// words of the lanes holding the largest high word).
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+  const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32));
+  const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32) == hi ? (uint32_t)v : 0u);
+  return ((unsigned long long)hi << 32) | lo;
+}
+
 // ---- warp MMA (legacy mma.sync, bf16 in, fp32 accumulate) ---------------------------------
 __device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -430,30 +462,32 @@ struct FusedSmem {
   __host__ __device__ static size_t sel(int gather, int row_ld, int CL, int K) {
     return gather ? align_up((size_t)G * row_ld * 4, 16) : align_up((size_t)G * CL * K * 8, 16);
   }
-  __host__ __device__ static size_t hbits(int C) { return align_up((size_t)G * ((C + 31) / 32) * 4, 16); }
+  // per-head selection bitmaps, the union bitmap and the union's prefix counts per word
+  __host__ __device__ static size_t hbits(int C) { return align_up((size_t)(G + 2) * ((C + 31) / 32) * 4, 16); }
   __host__ __device__ static size_t recv(int CL) {
     return align_up((size_t)CL * G * (D / CL + 2) * 4, 16);
   }
   __host__ __device__ static size_t zp(int b) { return MMA ? 0 : 2 * align_up((size_t)b * G * 4, 16); }
 };
 
-template <typename T, typename TS, int D, int G, bool MMA>
+// kMode: 0 the whole step; 1 and 2 the two launches of a long history (FusedParams::mode), each
+// its own instantiation so that the one-launch step's code is unchanged by them.
+template <typename T, typename TS, int D, int G, bool MMA, int kMode = 0>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const __grid_constant__ CUtensorMap tmk64, const __grid_constant__ CUtensorMap tmv64,
     const FusedParams p) {
   constexpr bool kMma = MMA;
   static_assert(!MMA || std::is_same<T, __nv_bfloat16>::value, "warp MMAs take bf16");
+  static_assert(kMode == 0 || MMA, "the two-launch path is the 64-token bf16 path");
   constexpr int EPL = D / 32;
   constexpr int R = 32 / G;
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   __shared__ int s_pick[kWarps][kMaxKf];
   __shared__ int s_sel[G][kMaxKf];
   __shared__ int s_nsel[G];
-  __shared__ uint32_t s_bits[kMaxWords];
   __shared__ int s_ublk[kMaxUnion];
   __shared__ unsigned s_umask[kMaxUnion];
   // select candidates (per warp: kCandMax + 4 keys, kCandMax positions) / append partials
@@ -467,6 +501,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ float s_m[G], s_l[G], s_corr[G];
   static_assert(kWarps * kScratchPerWarp >= kWarps * 128, "append partials fit the scratch");
 
+  // The K/V tensor maps are kernel parameters: their descriptors are fetched while the launch
+  // waits, not at the first copy after the selection.
+  if (kMma && threadIdx.x == 0) {
+    tc::prefetch_tmap(&tmk);
+    tc::prefetch_tmap(&tmv);
+    tc::prefetch_tmap(&tmk64);
+    tc::prefetch_tmap(&tmv64);
+  }
   // Programmatic dependent launch: every input may come from the work queued before this kernel
   // on the stream, so nothing is read before that work has completed and its writes are visible;
   // a launch queued after this one may be scheduled at once and wait the same way.
@@ -474,8 +516,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = p.b, K = p.K, Hq = p.Hq;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int rank = (int)cluster_rank();
-  const int CL = (int)cluster_size();
+  // mode 1 runs without clusters: the CTA's chunk is its x index
+  const int rank = kMode == 1 ? (int)blockIdx.x : (int)cluster_rank();
+  const int CL = kMode == 1 ? (int)gridDim.x : (int)cluster_size();
   const int kh = blockIdx.y, bi = blockIdx.z;
   const int h0 = kh * G;
   const int L = p.seq_lens ? min(p.seq_lens[bi], p.n) : p.n;
@@ -488,7 +531,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   using SM = FusedSmem<T, TS, D, G, MMA>;
   TS* ring = reinterpret_cast<TS*>(smem);  // region A: summary ring, then K/V ring, then partials
   TS* mean_k = static_cast<TS*>(p.mean_k);
-  const int Gs = p.shared ? 1 : G;  // selections made per group
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);  // [G][chunk]
   uint32_t* sel_buf = reinterpret_cast<uint32_t*>(smem + p.off_sel);  // whole rows / merge
   uint32_t* hbits = reinterpret_cast<uint32_t*>(smem + p.off_hbits);  // [Gs][nwords] selections
@@ -501,6 +543,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   if (tid == 0) {
     for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
+    if (kMode == 2) {  // the group's chunk lists (one contiguous block) into region A, first
+      const size_t words = (size_t)p.nchunk * (p.shared ? 1 : G) * p.cand_ld;
+      mbar_arrive_expect_tx(&bar[0], (uint32_t)(words * 4));
+      bulk_g2s(ring, p.cand + (size_t)(bi * p.Hk + kh) * words, (uint32_t)(words * 4), &bar[0]);
+    }
     for (int i = 0; i < kMaxStages; ++i) s_kv_par[i] = -1;
     s_next = 0;
     s_abort = 0;
@@ -510,15 +557,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     s_m[tid] = -INFINITY;
     s_l[tid] = 0.f;
   }
+  const int Gs = p.shared ? 1 : G;  // selections made per group
+  const int nwords = (nc + 31) / 32;
+  uint32_t* s_ubits = hbits + Gs * nwords;  // union of the selections over the history blocks
+  int* s_upre = reinterpret_cast<int*>(s_ubits + nwords);  // union entries before each word
+  if (kMode != 1)
+    for (int e = tid; e < (Gs + 1) * nwords; e += kThreads) hbits[e] = 0u;
   __syncthreads();
   // every CTA of the cluster has started before any peer writes into its shared memory
-  cluster_arrive_relaxed();
+  if (kMode != 1) cluster_arrive_relaxed();
 
   // ---- 1. score my slice of the history blocks --------------------------------------------
   const int c_lo = min(nc, rank * p.chunk);
   const int c_hi = min(nc, c_lo + p.chunk);
   const int rows = c_hi - c_lo;
-  const int nsub = (rows + kSub - 1) / kSub;
+  const int nsub = kMode == 2 ? 0 : (rows + kSub - 1) / kSub;  // mode 2 scores nothing
   const TS* mk = mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
   // summaries and K/V are read once per step: their L2 lines go first, so that the kernel's code
   // (fetched again by every launch) stays in L2 (the policy is made where it is used: one
@@ -534,6 +587,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   int sub_issued = 0;  // (thread 0) summary stages issued so far
   if (tid == 0)
     for (; sub_issued < min(nsub, NS); ++sub_issued) issue_sub(sub_issued);
+  const int cand_group = Gs * p.cand_ld;  // mode 2: words per chunk of the lists
   float qv[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -604,8 +658,84 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   // ---- 2. Top-K per head (per group when shared) -----------------------------------------
   uint32_t* ck = s_scratch + warp * kScratchPerWarp;
   int* cp = reinterpret_cast<int*>(ck + kCandMax + 4);
-  cluster_wait();  // every peer has started: DSMEM stores may begin
-  if (p.gather) {
+  if (kMode != 1) cluster_wait();  // every peer has started: DSMEM stores may begin
+  if constexpr (kMode == 1) {
+    // this chunk's Top-K of every selecting head in rank order (key descending, ties to the lower
+    // block: the pair sorts as key, then the complement of the block index), with its count
+    for (int g = warp; g < Gs; g += kWarps) {
+      const uint32_t* keys = s_keys + g * p.chunk;
+      const int cnt = s_abort ? 0 : warp_select(keys, rows, K, lane, s_pick[warp], ck, cp);
+      unsigned long long e = 0ull;  // empty places sort last
+      if (lane < cnt)
+        e = ((unsigned long long)keys[s_pick[warp][lane]] << 32) |
+            (unsigned long long)(~(uint32_t)(c_lo + s_pick[warp][lane]));
+      e = warp_sort<unsigned long long, true>(e, lane);
+      uint32_t* rec = p.cand + (((size_t)(bi * p.Hk + kh) * p.nchunk + rank) * Gs + g) * p.cand_ld;
+      if (lane < cnt) {
+        rec[lane] = (uint32_t)(e >> 32);
+        rec[K + lane] = ~(uint32_t)e;
+      }
+      if (lane == 0) rec[2 * K] = (uint32_t)cnt;
+    }
+    return;
+  }
+  if constexpr (kMode == 2) {
+    // Merge of the chunk lists.  Each list is in rank order; an entry is its key, then the
+    // complement of its block index (never 0; 0 marks "none").  Lane c follows chunk c's list
+    // with its head and the entry after it.  Every entry below a head is at most the largest of
+    // those next entries X, so all heads above X are larger than everything left outside the
+    // heads: a round takes them all at once (while they fit in K; otherwise one round takes the
+    // largest head alone) and advances their lists.  The K taken are the K largest of the whole
+    // history, since each of them is in its chunk's list.
+    if (!s_abort && !mbar_wait_bounded(&bar[0], 0)) s_abort = 1;
+    __syncthreads();
+    const uint32_t* blk = reinterpret_cast<const uint32_t*>(ring);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int g = warp; g < Gs && !s_abort; g += kWarps) {
+      const uint32_t* rec = blk + (size_t)min(lane, p.nchunk - 1) * cand_group + g * p.cand_ld;
+      const int n_c = lane < p.nchunk ? (int)rec[2 * K] : 0;
+      auto entry = [&](int j) -> unsigned long long {
+        return j < n_c ? ((unsigned long long)rec[j] << 32) | (unsigned long long)(~rec[K + j])
+                       : 0ull;
+      };
+      int ptr = 0;
+      unsigned long long hc = entry(0), nx = entry(1);
+      int* out = s_pick[warp];
+      int taken = 0;
+      while (taken < K) {
+        if (__ballot_sync(0xffffffffu, hc != 0ull) == 0u) break;
+        const unsigned long long X = warp_max_u64(nx);
+        bool take = hc != 0ull && hc > X;
+        unsigned tb = __ballot_sync(0xffffffffu, take);
+        if (taken + __popc(tb) > K) {  // too many at once: the largest head alone
+          const unsigned long long m = warp_max_u64(hc);
+          take = hc != 0ull && hc == m;
+          tb = __ballot_sync(0xffffffffu, take);
+        }
+        if (take) {
+          out[taken + __popc(tb & lt)] = (int)~(uint32_t)hc;
+          ++ptr;
+          hc = nx;
+          nx = entry(ptr + 1);
+        }
+        taken += __popc(tb);
+      }
+      __syncwarp();
+      int mine = lane < taken ? out[lane] : 0x7fffffff;
+      mine = warp_sort<int, false>(mine, lane);  // ascending block order
+      if (lane < taken) {
+        s_sel[g][lane] = mine;
+        atomicOr(&hbits[g * nwords + (mine >> 5)], 1u << (mine & 31));
+        atomicOr(&s_ubits[mine >> 5], 1u << (mine & 31));
+      }
+      if (lane == 0) s_nsel[g] = taken;
+    }
+    if (s_abort && tid == 0) {
+      (void)mbar_wait_bounded(&bar[0], 0, 1u << 12);  // the copy may still be in flight
+      report_timeout(p.status, 1);
+    }
+    if (s_abort && tid < Gs) s_nsel[tid] = 0;
+  } else if (p.gather) {
     // push my slice of every selecting head's keys into every CTA's whole-row copy
     const int nvec = rows >> 2, tail = rows & 3;
     const int per_g = CL * (nvec + tail);
@@ -625,7 +755,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     cluster_sync();
     for (int g = warp; g < Gs; g += kWarps) {
       const int cnt = warp_select(sel_buf + (size_t)g * p.row_ld, nc, K, lane, s_pick[warp], ck, cp);
-      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = s_pick[warp][j];
+      for (int j = lane; j < cnt; j += 32) {
+        const int x = s_pick[warp][j];
+        s_sel[g][j] = x;
+        atomicOr(&hbits[g * nwords + (x >> 5)], 1u << (x & 31));
+        atomicOr(&s_ubits[x >> 5], 1u << (x & 31));
+      }
       if (lane == 0) s_nsel[g] = cnt;
     }
   } else {
@@ -667,25 +802,22 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         __syncwarp();
       }
       const int cnt = warp_select(mk_g, nvalid, K, lane, s_pick[warp], ck, cp);
-      for (int j = lane; j < cnt; j += 32) s_sel[g][j] = mi_g[s_pick[warp][j]];
+      for (int j = lane; j < cnt; j += 32) {
+        const int x = mi_g[s_pick[warp][j]];
+        s_sel[g][j] = x;
+        atomicOr(&hbits[g * nwords + (x >> 5)], 1u << (x & 31));
+        atomicOr(&s_ubits[x >> 5], 1u << (x & 31));
+      }
       if (lane == 0) s_nsel[g] = cnt;
     }
   }
   __syncthreads();
 
   // ---- 3. the union of the selections, plus the current block ------------------------------
-  // every selection as a bitmap over the history blocks; one warp compacts the OR of the bitmaps
-  // into the sorted union and takes each entry's head mask from the same words
-  const int nwords = (nc + 31) / 32;
-  for (int g = warp; g < Gs; g += kWarps) {
-    uint32_t* hb = hbits + g * nwords;
-    for (int w = lane; w < nwords; w += 32) hb[w] = 0u;
-    __syncwarp();
-    for (int j = lane; j < s_nsel[g]; j += 32) {
-      const int x = s_sel[g][j];
-      atomicOr(&hb[x >> 5], 1u << (x & 31));
-    }
-  }
+  // Every selection has set its bits in its head's bitmap and in the union bitmap.  The union in
+  // block order comes from exclusive prefix counts of the union words: each selected entry finds
+  // its place on its own, and the lowest head holding a block writes that block's entry with the
+  // mask of every head holding it.  The current block, always kept, follows every history block.
   if (rank == 0) {  // optional outputs: the selection of every head
     for (int e = tid; e < G * K; e += kThreads) {
       const int g = e / K, j = e % K, gs = p.shared ? 0 : g;
@@ -694,47 +826,44 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       if (p.count && j == 0) p.count[row] = s_nsel[gs];
     }
   }
-  __syncthreads();
-  if (warp == 0) {  // a contiguous run of words per lane, prefix sums of their union counts
+  if (warp == kWarps - 1) {  // a contiguous run of words per lane
     const int per = (nwords + 31) / 32;
     const int w0 = min(nwords, lane * per), w1 = min(nwords, w0 + per);
     int mine = 0;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t u = 0u;
-      for (int g = 0; g < Gs; ++g) u |= hbits[g * nwords + w];
-      mine += __popc(u);
-    }
+    for (int w = w0; w < w1; ++w) mine += __popc(s_ubits[w]);
     int incl = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    int at = incl - mine;
+    int run = incl - mine;
     for (int w = w0; w < w1; ++w) {
-      uint32_t hw[G];
-      uint32_t u = 0u;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        hw[g] = g < Gs ? hbits[g * nwords + w] : 0u;
-        u |= hw[g];
-      }
-      while (u) {
-        const int bit = __ffs(u) - 1;
-        u &= u - 1;
-        unsigned m = 0u;
-#pragma unroll
-        for (int g = 0; g < G; ++g) m |= ((hw[g] >> bit) & 1u) << g;
-        s_ublk[at] = w * 32 + bit;
+      s_upre[w] = run;
+      run += __popc(s_ubits[w]);
+    }
+    if (lane == 31) s_U = incl;  // history entries
+  }
+  __syncthreads();
+  for (int e = tid; e < Gs * K; e += kThreads) {
+    const int g = e / K, j = e % K;
+    if (j < s_nsel[g]) {
+      const int x = s_sel[g][j], w = x >> 5;
+      const uint32_t bit = 1u << (x & 31);
+      unsigned m = 0u;
+      for (int h = Gs - 1; h >= 0; --h) m = (m << 1) | ((hbits[h * nwords + w] & bit) ? 1u : 0u);
+      if ((m & ((1u << g) - 1u)) == 0u) {  // no lower head holds the block
+        const int at = s_upre[w] + __popc(s_ubits[w] & (bit - 1u));
+        s_ublk[at] = x;
         s_umask[at] = p.shared ? (1u << G) - 1u : m;
-        ++at;
       }
     }
-    if (lane == 31) {
-      s_ublk[incl] = cur;  // the current block, always kept, follows every history block
-      s_umask[incl] = (1u << G) - 1u;
-      s_U = incl + 1;
-    }
+  }
+  if (tid == 0) {
+    const int uh = s_U;
+    s_ublk[uh] = cur;
+    s_umask[uh] = (1u << G) - 1u;
+    s_U = uh + 1;
   }
   __syncthreads();
   const int U = s_U;
@@ -804,9 +933,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
         }
       }
     };
-    if (tid == 0 && !s_abort) {
+    if (lane == 0 && warp < NKV && !s_abort) {  // slot st filled by warp st
       fence_proxy_async();  // generic accesses of phase 1 precede the async writes into region A
-      for (int st = 0; st < NKV; ++st) issue_kv(st, 0u, rank + CL * st < G_st ? rank + CL * st : -1);
+      issue_kv(warp, 0u, rank + CL * warp < G_st ? rank + CL * warp : -1);
     }
     if (p.append && rank == CL - 1) {
       // the block being filled: its summary rewritten from its keys in global memory by the last
@@ -1299,6 +1428,7 @@ struct LaunchCache {
   std::mutex mu;
   std::map<std::tuple<int, const void*, size_t, int>, int> clusters;  // -> max active clusters
   std::map<std::pair<int, const void*>, size_t> smem_set;              // -> attribute set to
+  std::map<const void*, size_t> static_smem;                           // -> static shared bytes
 };
 LaunchCache& launch_cache() {
   static LaunchCache c;
@@ -1322,32 +1452,40 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   }
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
-  auto kern = decode_fused_kernel<T, TS, D, G, MMA>;
+  auto kern = decode_fused_kernel<T, TS, D, G, MMA, 0>;
+  if constexpr (MMA)
+    if (p.mode == 2) kern = decode_fused_kernel<T, TS, D, G, MMA, 2>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
     return BSA_ERR_CUDA;
   }
   int min_per_sm = 1;
+  const int Gs = p.shared ? 1 : G;
   for (;;) {
     const int chunk = std::max(kSub, ceil_div(ceil_div(std::max(p.C, 1), CL), kSub) * kSub);
-    if (chunk > kSelMax) {  // the local select holds at most kSelMax keys per head
+    if (chunk > kSelMax && p.mode == 0) {  // the local select holds at most kSelMax keys per head
       if (CL < kMaxCL) { CL <<= 1; continue; }
       return BSA_ERR_UNSUPPORTED;
     }
     p.chunk = chunk;
     // whole-row selection when every history fits one warp select
-    p.gather = p.C <= kSelMax ? 1 : 0;
+    p.gather = p.C <= kSelMax && p.mode == 0 ? 1 : 0;
     p.row_ld = (int)align_up((size_t)std::max(p.C, 1), 4);
     // Region A as large as the CTAs resident per SM allow, then the fixed pieces.  Region A holds
     // the summary ring with the keys and the whole-row / merge buffer above it (phases 1-2), then
     // the K/V ring over all of it (phase 4, once the keys are dead), then the warp partials.
     size_t off = 0;
     const size_t fixed = SM::hbits(p.C) + SM::recv(CL) + SM::zp(p.b) + 256;
-    const size_t tail =
+    size_t tail =
         align_up(SM::keys(chunk) + SM::sel(p.gather, p.row_ld, CL, p.K), (size_t)1024);
     const size_t kvs = SM::kv_stage(p.b), sus = SM::sum_stage();
-    const size_t need_min = max_sz(max_sz(2 * kvs, 2 * sus + tail), SM::partials());
+    // mode 2: region A starts with the group's chunk lists; no summary ring
+    const size_t cand_bytes = align_up((size_t)p.nchunk * Gs * p.cand_ld * 4, (size_t)1024);
+    const size_t head2 = cand_bytes;
+    if (p.mode == 2) tail = 0;
+    const size_t need_min = p.mode == 2 ? max_sz(max_sz(2 * kvs, head2), SM::partials())
+                                        : max_sz(max_sz(2 * kvs, 2 * sus + tail), SM::partials());
     // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
     // (two K/V stages) does not fit that way
     int per_sm = std::max(min_per_sm, groups * CL > kSMs ? 2 : 1);
@@ -1359,11 +1497,11 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     }
     if (ra < need_min) return BSA_ERR_UNSUPPORTED;
     ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus + tail),
-                             SM::partials()));
-    p.ns = (int)std::min<size_t>(kMaxStages, (ra - tail) / sus);
+                             max_sz(SM::partials(), p.mode == 2 ? head2 : 0)));
+    p.ns = p.mode == 2 ? 1 : (int)std::min<size_t>(kMaxStages, (ra - tail) / sus);
     p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) : 2;
-    p.off_keys = (int)(ra - tail);
-    p.off_sel = p.off_keys + (int)SM::keys(chunk);
+    p.off_keys = p.mode == 2 ? 0 : (int)(ra - tail);
+    p.off_sel = p.mode == 2 ? (int)cand_bytes : p.off_keys + (int)SM::keys(chunk);
     off = align_up(ra, 1024);
     p.off_hbits = (int)off;
     off += SM::hbits(p.C);
@@ -1442,13 +1580,140 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   }
 }
 
+// The two-launch plan of a long history (more than kSelMax blocks) on the 64-token bf16 path:
+// about two CTAs per SM over the groups (each chunk at most kSelMax blocks), and the group's chunk
+// lists small enough for the merge launch's shared memory.  nchunk = 0: the plan does not apply.
+struct SplitPlan {
+  int nchunk = 0, chunk = 0, cand_ld = 0;
+  size_t bytes = 0;  // workspace
+};
+SplitPlan split_plan(int B, int Hk, int G, int C, int K, bool shared, bool mma) {
+  SplitPlan s;
+  if (!mma || C <= kSelMax) return s;
+  const int groups = B * Hk, Gs = shared ? 1 : G;
+  int nchunk = std::max(ceil_div(C, kSelMax), std::min(32, ceil_div(2 * kSMs, groups)));
+  const int chunk = std::max(kSub, ceil_div(ceil_div(C, nchunk), kSub) * kSub);
+  nchunk = ceil_div(C, chunk);
+  const int cand_ld = (int)align_up((size_t)(2 * K + 2), (size_t)4);
+  if (nchunk > 32 || (size_t)nchunk * Gs * cand_ld * 4 > 64 * 1024) return s;
+  s.nchunk = nchunk;
+  s.chunk = chunk;
+  s.cand_ld = cand_ld;
+  s.bytes = (size_t)groups * nchunk * Gs * cand_ld * 4;
+  return s;
+}
+
+size_t static_smem_bytes(const void* kern) {
+  LaunchCache& lc = launch_cache();
+  std::lock_guard<std::mutex> lock(lc.mu);
+  auto it = lc.static_smem.find(kern);
+  if (it != lc.static_smem.end()) return it->second;
+  cudaFuncAttributes fa{};
+  size_t v = kStaticSmemBound;
+  if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess)
+    v = fa.sharedSizeBytes;
+  else
+    (void)cudaGetLastError();
+  lc.static_smem[kern] = v;
+  return v;
+}
+
+// Launch 1 of the long-history plan (mode 1): CTA (c, kh, b) scores chunk c of group (b, kh) and
+// writes every selecting head's chunk Top-K to the workspace; no cluster, two CTAs per SM with a
+// summary ring as deep as that leaves room for.  Launch 2 is launch_fused in mode 2.
+template <typename T, typename TS, int D, int G, bool MMA>
+bsa_status launch_chunk_topk(const FusedParams& p, cudaStream_t st) {
+  using SM = FusedSmem<T, TS, D, G, MMA>;
+  auto kern = decode_fused_kernel<T, TS, D, G, MMA, 1>;
+  FusedParams p1 = p;
+  p1.mode = 1;
+  p1.gather = 0;
+  p1.row_ld = 4;
+  const size_t sus = SM::sum_stage();
+  const size_t keys = align_up(SM::keys(p.chunk), (size_t)1024);
+  // two CTAs per SM: 228 KB less 1 KB reserved per CTA, the static part, alignment slack
+  const size_t budget = 228 * 1024 / 2 - 1024 - static_smem_bytes(reinterpret_cast<const void*>(kern)) - 1024;
+  const size_t small = SM::recv(1) + SM::zp(p.b) + 256 + 64;
+  if (budget < keys + small + sus) return BSA_ERR_UNSUPPORTED;
+  const int need_st = ceil_div(p.chunk, kSub);
+  p1.ns = (int)std::min<size_t>(std::min(kMaxStages, need_st), (budget - keys - small) / sus);
+  p1.nkv = 1;
+  size_t off = (size_t)p1.ns * sus;
+  p1.off_keys = (int)off;
+  p1.off_sel = (int)off;
+  off += keys;
+  p1.off_hbits = (int)off;  // no bitmaps in mode 1
+  p1.off_recv = (int)off;
+  off += SM::recv(1);
+  p1.off_zp = (int)off;
+  off += SM::zp(p.b);
+  off = align_up(off, 16);
+  p1.off_bar = (int)off;
+  off += 256;
+  const size_t smem = off + 1024;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  LaunchCache& lc = launch_cache();
+  {
+    std::lock_guard<std::mutex> lock(lc.mu);
+    size_t& set_to = lc.smem_set[{dev, reinterpret_cast<const void*>(kern)}];
+    if (set_to < smem) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess) {
+        (void)cudaGetLastError();
+        return BSA_ERR_CUDA;
+      }
+      set_to = smem;
+    }
+  }
+  CUtensorMap tm{};  // mode 1 copies no K/V: the maps are never used
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.nchunk, p.Hk, p.B);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tm, tm, tm, tm, p1) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
+template <typename T, typename TS, int D, int G, bool MMA>
+bsa_status launch_step(FusedParams& p, const SplitPlan& plan, uint32_t* ws, cudaStream_t st) {
+  if constexpr (MMA) {
+    if (plan.nchunk > 0 && ws) {
+      p.nchunk = plan.nchunk;
+      p.chunk = plan.chunk;
+      p.cand_ld = plan.cand_ld;
+      p.cand = ws;
+      const bsa_status rc = launch_chunk_topk<T, TS, D, G, MMA>(p, st);
+      if (rc != BSA_OK) return rc;
+      p.mode = 2;
+    }
+  }
+  return launch_fused<T, TS, D, G, MMA>(p, st);
+}
+
 template <typename T, typename TS, int D, bool MMA>
-bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st) {
+bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st, uint32_t* ws = nullptr,
+                          size_t ws_bytes = 0) {
+  SplitPlan plan = split_plan(p.B, p.Hk, G, p.C, p.K, p.shared != 0, MMA);
+  if (plan.nchunk > 0 && ws && ws_bytes < plan.bytes) return BSA_ERR_WORKSPACE;
+  if (!ws) plan = SplitPlan{};
   switch (G) {
-    case 1: return launch_fused<T, TS, D, 1, MMA>(p, st);
-    case 2: return launch_fused<T, TS, D, 2, MMA>(p, st);
-    case 4: return launch_fused<T, TS, D, 4, MMA>(p, st);
-    case 8: return launch_fused<T, TS, D, 8, MMA>(p, st);
+    case 1: return launch_step<T, TS, D, 1, MMA>(p, plan, ws, st);
+    case 2: return launch_step<T, TS, D, 2, MMA>(p, plan, ws, st);
+    case 4: return launch_step<T, TS, D, 4, MMA>(p, plan, ws, st);
+    case 8: return launch_step<T, TS, D, 8, MMA>(p, plan, ws, st);
     default: return BSA_ERR_UNSUPPORTED;
   }
 }
@@ -1456,14 +1721,15 @@ bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st) {
 }  // namespace
 }  // namespace bsa
 
-extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v,
-                                         bsa_dtype dt, int B, int Hq, int Hk, int n, int d, int b,
-                                         const int* seq_lens, void* mean_k, float* max_norm,
-                                         float* centre, int append, const float* lambda_h,
-                                         const float* sigma_h, int prefix_block, int K, void* o,
-                                         float* lse, int* idx, int* count, int* status,
-                                         int flags, void* stream) {
-  using namespace bsa;
+namespace bsa {
+namespace {
+
+bsa_status decode_step_impl(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                            int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                            void* mean_k, float* max_norm, float* centre, int append,
+                            const float* lambda_h, const float* sigma_h, int prefix_block, int K,
+                            void* o, float* lse, int* idx, int* count, int* status, int flags,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   BSA_REQUIRE(dtype_ok(dt), BSA_ERR_DTYPE);
   BSA_REQUIRE(q && k && v && mean_k && o, BSA_ERR_ARG);
   BSA_REQUIRE(B > 0 && Hq > 0 && Hk > 0 && n > 0 && d > 0 && b > 0 && K > 0 && prefix_block >= 0,
@@ -1493,13 +1759,15 @@ extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const voi
   p.shared = (flags & BSA_DECODE_SHARED_SELECTION) != 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   using bf = __nv_bfloat16;
+  BSA_REQUIRE(!workspace || aligned16(workspace), BSA_ERR_ARG);
+  uint32_t* ws = workspace_bytes > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
   bsa_status rc;
   if (dt == BSA_BF16 && b == 64 && bf16_sum)
-    rc = d == 64 ? dispatch_fused<bf, bf, 64, true>(Hq / Hk, p, st)
-                 : dispatch_fused<bf, bf, 128, true>(Hq / Hk, p, st);
+    rc = d == 64 ? dispatch_fused<bf, bf, 64, true>(Hq / Hk, p, st, ws, workspace_bytes)
+                 : dispatch_fused<bf, bf, 128, true>(Hq / Hk, p, st, ws, workspace_bytes);
   else if (dt == BSA_BF16 && b == 64)  // 64-token blocks: warp MMAs over swizzled TMA tiles
-    rc = d == 64 ? dispatch_fused<bf, float, 64, true>(Hq / Hk, p, st)
-                 : dispatch_fused<bf, float, 128, true>(Hq / Hk, p, st);
+    rc = d == 64 ? dispatch_fused<bf, float, 64, true>(Hq / Hk, p, st, ws, workspace_bytes)
+                 : dispatch_fused<bf, float, 128, true>(Hq / Hk, p, st, ws, workspace_bytes);
   else if (dt == BSA_BF16)
     rc = d == 64 ? dispatch_fused<bf, float, 64, false>(Hq / Hk, p, st)
                  : dispatch_fused<bf, float, 128, false>(Hq / Hk, p, st);
@@ -1509,6 +1777,44 @@ extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const voi
   if (rc != BSA_OK) return rc;
   BSA_LAUNCH_CHECK();
   return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v,
+                                         bsa_dtype dt, int B, int Hq, int Hk, int n, int d, int b,
+                                         const int* seq_lens, void* mean_k, float* max_norm,
+                                         float* centre, int append, const float* lambda_h,
+                                         const float* sigma_h, int prefix_block, int K, void* o,
+                                         float* lse, int* idx, int* count, int* status,
+                                         int flags, void* stream) {
+  return bsa::decode_step_impl(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, mean_k, max_norm,
+                               centre, append, lambda_h, sigma_h, prefix_block, K, o, lse, idx,
+                               count, status, flags, nullptr, 0, stream);
+}
+
+extern "C" size_t bsa_decode_step_workspace_bytes(int B, int Hq, int Hk, int n, int d, int b,
+                                                  int K, int flags, int dt) {
+  using namespace bsa;
+  if (B <= 0 || Hq <= 0 || Hk <= 0 || n <= 0 || d <= 0 || b <= 0 || K <= 0 || Hq % Hk != 0)
+    return 0;
+  const bool mma = dt == BSA_BF16 && b == 64 && (d == 64 || d == 128);
+  return split_plan(B, Hk, Hq / Hk, ceil_div(n, b), K,
+                    (flags & BSA_DECODE_SHARED_SELECTION) != 0, mma).bytes;
+}
+
+extern "C" bsa_status bsa_decode_step_ws(const void* q, const void* k, const void* v,
+                                         bsa_dtype dt, int B, int Hq, int Hk, int n, int d, int b,
+                                         const int* seq_lens, void* mean_k, float* max_norm,
+                                         float* centre, int append, const float* lambda_h,
+                                         const float* sigma_h, int prefix_block, int K, void* o,
+                                         float* lse, int* idx, int* count, int* status,
+                                         int flags, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  return bsa::decode_step_impl(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, mean_k, max_norm,
+                               centre, append, lambda_h, sigma_h, prefix_block, K, o, lse, idx,
+                               count, status, flags, workspace, workspace_bytes, stream);
 }
 
 extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtype dt,

@@ -201,8 +201,7 @@ __global__ void __launch_bounds__(FsTcSmem<D>::kThreads, 1)
   constexpr int kNC = L::kNC;
   constexpr int kEpiWarps = L::kEpiWarps;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]

@@ -219,8 +219,7 @@ __global__ void __launch_bounds__(LongSmem<D, CELL>::kThreads, LongSmem<D, CELL>
   using L = LongSmem<D, CELL>;
   constexpr int NS = L::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[2 * 3 + 9];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;

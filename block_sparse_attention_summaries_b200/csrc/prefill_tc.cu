@@ -82,8 +82,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 1)
   using L = TcSmem<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 1024-byte alignment of the swizzled tiles
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[30];
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [kKSlots <= 6]
@@ -529,8 +528,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                         const __grid_constant__ CUtensorMap tmv, const GgParams p) {
   using L = GgSmem<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]

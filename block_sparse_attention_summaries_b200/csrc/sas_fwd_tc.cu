@@ -81,8 +81,7 @@ __global__ void __launch_bounds__(kSasThreads, 1)
   using L = SasSmem<D>;
   constexpr int KS = L::kKSlots, VS = L::kVSlots;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[30];
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [KS <= 6]

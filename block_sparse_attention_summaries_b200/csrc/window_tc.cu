@@ -97,8 +97,7 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
                      const __grid_constant__ CUtensorMap tmv, const WinParams w) {
   using L = WinSmem<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* smem = smem_align1024(smem_raw);
   __shared__ __align__(8) uint64_t bars[24];
   uint64_t* q_full = bars + 0;    // [2]
   uint64_t* q_empty = bars + 2;   // [2]

@@ -196,6 +196,33 @@ bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v, bsa_d
                               void* stream);
 
 /*
+ * bsa_decode_step_ws -- bsa_decode_step_ex with a workspace that lets long histories use the
+ * whole GPU ([SAS] "Decoding efficiency": at long contexts the block scoring and Top-K dominate
+ * the step).  On the 64-token bf16 path with more than 512 history blocks the step runs as two
+ * launches: the first scores the history in chunks (about two CTAs per SM) and writes each chunk's
+ * Top-K of every selecting head to the workspace; the second merges those lists -- only entries at
+ * or above the largest threshold of a full chunk can be among the K largest -- and then forms the
+ * union and attends exactly as bsa_decode_step_ex.  Selection, o, lse, idx and count are those of
+ * bsa_decode_step_ex (same scores, same order, ties to the lower block).
+ *   workspace        device memory, 16-byte aligned, owned by the caller; no initialisation is
+ *                    needed and it may be reused once the stream has passed the call.  NULL or
+ *                    workspace_bytes = 0: bsa_decode_step_ex (one launch).
+ *   workspace_bytes  its size; BSA_ERR_WORKSPACE if nonzero and below
+ *                    bsa_decode_step_workspace_bytes().
+ */
+bsa_status bsa_decode_step_ws(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                              int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                              void* mean_k, float* max_norm, float* centre, int append,
+                              const float* lambda_h, const float* sigma_h, int prefix_block, int K,
+                              void* o, float* lse, int* idx, int* count, int* status, int flags,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes bsa_decode_step_ws uses for this shape (dt is a bsa_dtype value); 0 when the
+ * step runs as one launch (short histories, other dtypes or block sizes, invalid sizes). */
+size_t bsa_decode_step_workspace_bytes(int B, int Hq, int Hk, int n, int d, int b, int K,
+                                       int flags, int dt);
+
+/*
  * bsa_sparse_attn_fwd -- exact causal softmax over the gathered tokens
  * ([SAS] Eq. 2 and "How it works" step 6; [Monodratic]), optionally with the log-gate of
  * [SAS] Eq. 9.

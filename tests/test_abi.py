@@ -215,6 +215,29 @@ def test_outer_gate_arguments(bsa_lib):
              None, 16, FAKE, None) == 1     # scores missing
 
 
+def test_decode_step_workspace(bsa_lib):
+    """The workspace of bsa_decode_step_ws: none for whole-row histories (<= 512 blocks), other
+    dtypes or block sizes; for long histories one record of K keys, K positions, count and
+    threshold (padded to 4 words) per chunk and head; a short workspace is refused before any
+    launch, and the call without one takes bsa_decode_step_ex's checks."""
+    q = bsa_lib.bsa_decode_step_workspace_bytes
+    assert q(8, 32, 8, 32768, 128, 64, 15, 0, 1) == 0            # 512 blocks: one launch
+    need = q(1, 32, 8, 524288, 128, 64, 31, 0, 1)                # 8192 blocks, 8 groups
+    assert need == 8 * 32 * 4 * 64 * 4                           # 32 chunks of 256 blocks
+    assert q(1, 32, 8, 524288, 128, 64, 31, 1, 1) == need // 4   # shared selection: one list
+    assert q(1, 32, 8, 524288, 128, 64, 31, 0, 0) == 0           # fp32 K/V: one launch
+    assert q(1, 32, 8, 524288, 128, 32, 31, 0, 1) == 0           # 32-token blocks: one launch
+    assert q(0, 32, 8, 524288, 128, 64, 31, 0, 1) == 0
+    f = bsa_lib.bsa_decode_step_ws
+    base = [FAKE, FAKE, FAKE, 1, 1, 32, 8, 524288, 128, 64, None, FAKE, None, None, 0, None,
+            None, 0, 31, FAKE, None, None, None, None, 0, FAKE, need - 16, None]
+    assert f(*base) == 7                                         # BSA_ERR_WORKSPACE
+    bad = list(base); bad[25] = ctypes.c_void_p(0x1004)          # misaligned workspace
+    assert f(*bad) == 1
+    bad = list(base); bad[24] = 4                                # unknown flag bit
+    assert f(*bad) == 1
+
+
 def test_freesolo_workspace_size_query(bsa_lib):
     f = bsa_lib.bsa_freesolo_workspace_bytes
     rows = 1 * 16 * 65536

@@ -114,11 +114,19 @@ def test_fused_full_size(wl):
                               needles=w["needles"], needle_layout=w["needle_layout"])
     q, k, v, sl = upload(case)
     mean_k, _, _ = bsa.build_block_summaries(k, 64)
-    o1, lse1, idx1, _ = bsa.decode_step_fused(q, k, v, mean_k, 64, w["K"], append=False)
+    o1, lse1, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, 64, w["K"], append=False)
     o2, lse2, idx2 = bsa.decode_step(q, k, v, mean_k, 64, w["K"], append=False)
+    # with a workspace: two launches at 512K (chunk Top-K over the whole GPU, then the merge),
+    # one launch at 32K; the same selection either way
+    need = bsa.decode_step_workspace_bytes(w["B"], 32, 8, w["n"], 128, 64, w["K"])
+    assert (need > 0) == (w["n"] // 64 > 512)
+    o3, lse3, idx3, cnt3 = bsa.decode_step_ws(q, k, v, mean_k, 64, w["K"], append=False)
     torch.cuda.synchronize()
     assert torch.equal(idx1, idx2)
+    assert torch.equal(idx3, idx1) and torch.equal(cnt3, cnt1)
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+    assert (o3.float() - o1.float()).abs().max().item() < 1e-2
+    assert (lse3 - lse1).abs().max().item() < 1e-3
     if w["B"] == 1:  # long context: every head of the sequence
         rows = [(0, h) for h in range(32)]
     else:
@@ -149,9 +157,13 @@ def test_fused_long_history_local_and_merged_selection(n, B):
     o1, lse1, idx1, cnt1 = bsa.decode_step_fused(q, k, v, mean_k, 64, 13, seq_lens=sl,
                                                  append=False)
     o2, lse2, idx2 = bsa.decode_step(q, k, v, mean_k, 64, 13, seq_lens=sl, append=False)
+    o3, lse3, idx3, cnt3 = bsa.decode_step_ws(q, k, v, mean_k, 64, 13, seq_lens=sl,
+                                              append=False)  # chunk Top-K + merge launches
     torch.cuda.synchronize()
     assert torch.equal(idx1, idx2)
+    assert torch.equal(idx3, idx1) and torch.equal(cnt3, cnt1)
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+    assert (o3.float() - o1.float()).abs().max().item() < 1e-2
     rows = [(bi, h) for bi in range(B) for h in (0, 3, 5, 7)]
     oracle_check(case, idx1.cpu().numpy(), o1.float().cpu().numpy(), lse1.cpu().numpy(), rows,
                  2e-2)
@@ -185,6 +197,41 @@ def test_fused_all_scores_tied_take_the_lowest_blocks(C):
             for h in range(kh * G, (kh + 1) * G):
                 assert (o1[bi, h].float() - ref).abs().max().item() < 2e-2
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+
+
+@pytest.mark.parametrize("C,K", [(1000, 11), (4096, 32)])
+def test_workspace_path_all_scores_tied_take_the_lowest_blocks(C, K):
+    """The two-launch path with every score tied: each chunk keeps its K lowest blocks, every
+    chunk threshold equals the common key, so every kept entry survives the bound; at 4096 blocks
+    (32 chunks x 32 entries) the survivors overflow one merge buffer and the running Top-K keeps
+    the lowest blocks.  The result is the K lowest block indices, as on the one-launch path."""
+    B, Hk, G, d, b = 1, 2, 4, 64, 64
+    n = C * b + 17
+    k = torch.zeros(B, Hk, n, d, device=DEV, dtype=torch.bfloat16)
+    g = torch.Generator(device=DEV).manual_seed(6)
+    v = torch.randn(B, Hk, n, d, device=DEV, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, Hk * G, d, device=DEV, generator=g).to(torch.bfloat16)
+    mean_k, _, _ = bsa.build_block_summaries(k, b)
+    assert bsa.decode_step_workspace_bytes(B, Hk * G, Hk, n, d, b, K) > 0
+    o1, lse1, idx1, cnt1 = bsa.decode_step_ws(q, k, v, mean_k, b, K, append=False)
+    o2, lse2, idx2, cnt2 = bsa.decode_step_fused(q, k, v, mean_k, b, K, append=False)
+    torch.cuda.synchronize()
+    want = torch.arange(K, device=DEV, dtype=torch.int32).expand(B, Hk * G, K)
+    assert torch.equal(idx1, want) and torch.equal(idx2, want)
+    assert torch.equal(cnt1, torch.full_like(cnt1, K))
+    assert (o1.float() - o2.float()).abs().max().item() < 1e-2
+
+
+def test_workspace_too_small_is_refused():
+    n, b, K = 600 * 64, 64, 8
+    need = bsa.decode_step_workspace_bytes(1, 8, 2, n, 128, b, K)
+    assert need > 0
+    q = torch.randn(1, 8, 128, device=DEV).to(torch.bfloat16)
+    k = torch.randn(1, 2, n, 128, device=DEV).to(torch.bfloat16)
+    mean_k, _, _ = bsa.build_block_summaries(k, b)
+    ws = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(bsa.BsaError):
+        bsa.decode_step_ws(q, k, k, mean_k, b, K, ws=ws, append=False)
 
 
 # ---- variants: GQA-shared selection and bf16 summaries (bsa_decode_step_ex) ------------------
