@@ -52,7 +52,17 @@ WORKLOADS = {
 # profile summary under profiles/).  Reported only while the source is unchanged.
 # The hash covers the device code of the source: the file up to its first host function
 # (`device_end`), so a change of the host-side launcher alone keeps the figure.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    ("sas_gqa_decode_32k", "decode_fused_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
+        "device_end": "int pick_cluster(", "sha256_16": "34d6ff7c98961cf4",
+        "bytes": 52_599_808 + 212_992},
+    # two launches per step (chunk Top-K, then merge + attention): their sum
+    ("long_decode_512k", "decode_fused_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
+        "device_end": "int pick_cluster(", "sha256_16": "34d6ff7c98961cf4",
+        "bytes": 33_624_064 + 16_130_304},
+}
 
 
 def device_source_hash(path: str, device_end: str) -> str:
@@ -921,8 +931,11 @@ def run_gpu(args):
     layers = build_layers(dev, case, w, R)
     status = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream(dev)
-    graphs = capture_fused(dev, layers, w, status, stream)
-    launches_per_step = 1
+    # long histories take the two-launch path (bsa_decode_step_ws) through a workspace
+    ws_bytes = bsa.decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes > 0 else None
+    graphs = capture_fused(dev, layers, w, status, stream, ws=ws)
+    launches_per_step = 2 if ws is not None else 1
     idx_h = layers[0]["idx"].cpu().numpy()
     acc = decode_accounting(case, w, idx_h)
     step_bytes = acc["kv_bytes"] + acc["summary_bytes"]  # selected K/V + summaries
@@ -1005,13 +1018,15 @@ def run_gpu(args):
                           "index_agreement_vs_per_head_fp32": agree}
 
     # end to end through the public API: pinned host q in, the decode step (a prepared binding
-    # call, bsa.DecodeStep -> bsa_decode_step_ex, no graph), o out, every step
+    # call, bsa.DecodeStep -> bsa_decode_step_ex, or _ws for long histories, no graph), o out,
+    # every step
     q_host = [torch.from_numpy(np.ascontiguousarray(L["q"].float().cpu().numpy()))
               .to(torch.bfloat16).pin_memory() for L in layers]
     o_host = torch.empty(B, Hq, d, dtype=torch.bfloat16).pin_memory()
     plans = [bsa.DecodeStep(L["q"], L["k"], L["v"], L["mean_k"], b, K, append=True,
                             max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
-                            idx=L["idx"], count=L["count"], status=status) for L in layers]
+                            idx=L["idx"], count=L["count"], status=status, ws=ws)
+             for L in layers]
     e2e_ms = []
     with torch.cuda.stream(stream):
         for i in range(args.warmup + args.steps):
@@ -1067,8 +1082,9 @@ def run_gpu(args):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * Hq * d * 2,
                 "d2h_bytes_per_step": B * Hq * d * 2,
                 "what": "per step: pinned-host q -> device, the decode step through a prepared "
-                        "binding call (bsa.DecodeStep) and the C ABI (bsa_decode_step_ex, no "
-                        "graph), o -> pinned host; CUDA events on the stream"},
+                        "binding call (bsa.DecodeStep) and the C ABI (bsa_decode_step_ex; "
+                        "bsa_decode_step_ws past 512 history blocks; no graph), o -> pinned "
+                        "host; CUDA events on the stream"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],

@@ -588,13 +588,16 @@ class DecodeStep:
     the stream to the C ABI, so a step costs the host one foreign call instead of re-checking and
     re-wrapping every tensor.  The tensors given (and the outputs allocated here) are kept alive
     by this object and must keep their storage: write new queries into ``q`` in place.
-    ``outputs`` is (o, lse, idx, count).
+    ``outputs`` is (o, lse, idx, count).  With a workspace ``ws`` (a uint8 device tensor of at
+    least decode_step_workspace_bytes) the call is bsa_decode_step_ws: long histories take the
+    two-launch path.
     """
 
     def __init__(self, q, k, v, mean_k, b, K, flags=0, seq_lens=None, append=True,
                  max_norm=None, centre=None, lambda_h=None, sigma_h=None, prefix_block=0,
-                 o=None, lse=None, idx=None, count=None, status=None):
-        _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count)
+                 o=None, lse=None, idx=None, count=None, status=None, ws=None):
+        _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count,
+              ws)
         B, Hk, n, d = k.shape
         Hq = q.shape[1]
         if o is None:
@@ -606,13 +609,16 @@ class DecodeStep:
         if count is None:
             count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
         sl = _i32(seq_lens)
-        self._keep = (q, k, v, mean_k, sl, max_norm, centre, lambda_h, sigma_h, status)
+        self._keep = (q, k, v, mean_k, sl, max_norm, centre, lambda_h, sigma_h, status, ws)
         self.outputs = (o, lse, idx, count)
-        self._fn = lib().bsa_decode_step_ex
+        self._fn = lib().bsa_decode_step_ex if ws is None else lib().bsa_decode_step_ws
+        self._name = "bsa_decode_step_ex" if ws is None else "bsa_decode_step_ws"
         self._args = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b, _ptr(sl),
                       _ptr(mean_k), _ptr(max_norm), _ptr(centre), 1 if append else 0,
                       _ptr(lambda_h), _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse),
                       _ptr(idx), _ptr(count), _ptr(status), int(flags))
+        if ws is not None:
+            self._args = self._args + (_ptr(ws), ws.numel())
         self._device = q.device
 
     def __call__(self, stream=None):
@@ -620,7 +626,7 @@ class DecodeStep:
         st = stream if stream is not None else torch.cuda.current_stream(self._device)
         code = self._fn(*self._args, ctypes.c_void_p(st.cuda_stream))
         if code != 0:
-            raise BsaError(code, "bsa_decode_step_ex")
+            raise BsaError(code, self._name)
         return self.outputs
 
 
