@@ -96,6 +96,10 @@ struct FusedParams {
   // and writes every selecting head's chunk Top-K to `cand`; mode 2 merges those lists and runs
   // phases 3-5.  Mode 0 is the whole step in one launch.
   int mode;
+  // Mode 3 is the attention of a given selection (the decode form of bsa_sparse_attn_fwd):
+  // phases 3-5 over sel_idx [B, Hq, K] (entries outside the history ignored), sel_count [B, Hq].
+  const int* sel_idx;
+  const int* sel_count;
   int nchunk;      // chunks per group (modes 1 and 2)
   int cand_ld;     // words per (chunk, head) record: K keys, K positions (rank order), count
   uint32_t* cand;  // [B * Hk][nchunk][Gs][cand_ld]
@@ -470,8 +474,9 @@ struct FusedSmem {
   __host__ __device__ static size_t zp(int b) { return MMA ? 0 : 2 * align_up((size_t)b * G * 4, 16); }
 };
 
-// kMode: 0 the whole step; 1 and 2 the two launches of a long history (FusedParams::mode), each
-// its own instantiation so that the one-launch step's code is unchanged by them.
+// kMode: 0 the whole step; 1 and 2 the two launches of a long history; 3 the attention of a given
+// selection (FusedParams::mode), each its own instantiation so that the one-launch step's code is
+// unchanged by them.
 template <typename T, typename TS, int D, int G, bool MMA, int kMode = 0>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -479,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const FusedParams p) {
   constexpr bool kMma = MMA;
   static_assert(!MMA || std::is_same<T, __nv_bfloat16>::value, "warp MMAs take bf16");
-  static_assert(kMode == 0 || MMA, "the two-launch path is the 64-token bf16 path");
+  static_assert(kMode == 0 || MMA, "modes 1-3 are the 64-token bf16 path");
   constexpr int EPL = D / 32;
   constexpr int R = 32 / G;
 
@@ -571,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   const int c_lo = min(nc, rank * p.chunk);
   const int c_hi = min(nc, c_lo + p.chunk);
   const int rows = c_hi - c_lo;
-  const int nsub = kMode == 2 ? 0 : (rows + kSub - 1) / kSub;  // mode 2 scores nothing
+  const int nsub = kMode >= 2 ? 0 : (rows + kSub - 1) / kSub;  // modes 2 and 3 score nothing
   const TS* mk = mean_k + ((size_t)(bi * p.Hk + kh) * p.C) * D;
   // summaries and K/V are read once per step: their L2 lines go first, so that the kernel's code
   // (fetched again by every launch) stays in L2 (the policy is made where it is used: one
@@ -679,7 +684,29 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     }
     return;
   }
-  if constexpr (kMode == 2) {
+  if constexpr (kMode == 3) {
+    // the given selection of every head: entries outside the history are ignored, repeats
+    // collapse in the bitmaps
+    const unsigned lt = (1u << lane) - 1u;
+    for (int g = warp; g < G; g += kWarps) {
+      const size_t row = (size_t)bi * Hq + h0 + g;
+      const int cnt = p.sel_count ? min(p.sel_count[row], K) : K;
+      int taken = 0;
+      for (int j0 = 0; j0 < cnt; j0 += 32) {
+        const int j = j0 + lane;
+        const int m = j < cnt ? p.sel_idx[row * K + j] : -1;
+        const bool good = j < cnt && m >= 0 && m < nc;
+        const unsigned bal = __ballot_sync(0xffffffffu, good);
+        if (good) {
+          s_sel[g][taken + __popc(bal & lt)] = m;
+          atomicOr(&hbits[g * nwords + (m >> 5)], 1u << (m & 31));
+          atomicOr(&s_ubits[m >> 5], 1u << (m & 31));
+        }
+        taken += __popc(bal);
+      }
+      if (lane == 0) s_nsel[g] = taken;
+    }
+  } else if constexpr (kMode == 2) {
     // Merge of the chunk lists.  Each list is in rank order; an entry is its key, then the
     // complement of its block index (never 0; 0 marks "none").  Lane c follows chunk c's list
     // with its head and the entry after it.  Every entry below a head is at most the largest of
@@ -1453,8 +1480,10 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   const int groups = p.B * p.Hk;
   int CL = pick_cluster(groups);
   auto kern = decode_fused_kernel<T, TS, D, G, MMA, 0>;
-  if constexpr (MMA)
+  if constexpr (MMA) {
     if (p.mode == 2) kern = decode_fused_kernel<T, TS, D, G, MMA, 2>;
+    if (p.mode == 3) kern = decode_fused_kernel<T, TS, D, G, MMA, 3>;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -1483,8 +1512,8 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     // mode 2: region A starts with the group's chunk lists; no summary ring
     const size_t cand_bytes = align_up((size_t)p.nchunk * Gs * p.cand_ld * 4, (size_t)1024);
     const size_t head2 = cand_bytes;
-    if (p.mode == 2) tail = 0;
-    const size_t need_min = p.mode == 2 ? max_sz(max_sz(2 * kvs, head2), SM::partials())
+    if (p.mode >= 2) tail = 0;
+    const size_t need_min = p.mode >= 2 ? max_sz(max_sz(2 * kvs, head2), SM::partials())
                                         : max_sz(max_sz(2 * kvs, 2 * sus + tail), SM::partials());
     // two CTAs per SM when the grid needs them to be resident at once, unless region A's minimum
     // (two K/V stages) does not fit that way
@@ -1498,10 +1527,10 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
     if (ra < need_min) return BSA_ERR_UNSUPPORTED;
     ra = std::min(ra, max_sz(max_sz((size_t)kMaxStages * kvs, (size_t)kMaxStages * sus + tail),
                              max_sz(SM::partials(), p.mode == 2 ? head2 : 0)));
-    p.ns = p.mode == 2 ? 1 : (int)std::min<size_t>(kMaxStages, (ra - tail) / sus);
+    p.ns = p.mode >= 2 ? 1 : (int)std::min<size_t>(kMaxStages, (ra - tail) / sus);
     p.nkv = MMA ? (int)std::min<size_t>(kMaxStages, ra / kvs) : 2;
-    p.off_keys = p.mode == 2 ? 0 : (int)(ra - tail);
-    p.off_sel = p.mode == 2 ? (int)cand_bytes : p.off_keys + (int)SM::keys(chunk);
+    p.off_keys = p.mode >= 2 ? 0 : (int)(ra - tail);
+    p.off_sel = p.mode >= 2 ? (int)cand_bytes : p.off_keys + (int)SM::keys(chunk);
     off = align_up(ra, 1024);
     p.off_hbits = (int)off;
     off += SM::hbits(p.C);
@@ -1780,6 +1809,38 @@ bsa_status decode_step_impl(const void* q, const void* k, const void* v, bsa_dty
 }
 
 }  // namespace
+
+// Decode attention of a given selection on the cluster step (mode 3): bf16 K/V in 64-token blocks,
+// no gate.  BSA_ERR_UNSUPPORTED for every other request (the caller then takes the split-K kernel).
+bsa_status decode_attn_given(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                             int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                             const int* idx, const int* count, int K, int gate, void* o,
+                             float* lse, int* status, cudaStream_t st) {
+  if (dt != BSA_BF16 || b != 64 || gate != BSA_GATE_NONE || (d != 64 && d != 128) ||
+      K > kMaxKf || Hq % Hk != 0 || !group_ok(Hq, Hk) || B > 65535 || Hk > 65535)
+    return BSA_ERR_UNSUPPORTED;
+  const int C = ceil_div(n, b);
+  if (C > kMaxWords * 32) return BSA_ERR_UNSUPPORTED;
+  FusedParams p{};
+  p.q = q; p.k = k; p.v = v;
+  p.B = B; p.Hq = Hq; p.Hk = Hk; p.n = n; p.b = b; p.C = C; p.K = K;
+  p.seq_lens = seq_lens;
+  p.o = o; p.lse = lse; p.status = status;
+  p.sel_idx = idx; p.sel_count = count;
+  p.mode = 3;
+  using bf = __nv_bfloat16;
+  const int G = Hq / Hk;
+  bsa_status rc;
+  switch (G) {
+    case 1: rc = d == 64 ? launch_fused<bf, float, 64, 1, true>(p, st) : launch_fused<bf, float, 128, 1, true>(p, st); break;
+    case 2: rc = d == 64 ? launch_fused<bf, float, 64, 2, true>(p, st) : launch_fused<bf, float, 128, 2, true>(p, st); break;
+    case 4: rc = d == 64 ? launch_fused<bf, float, 64, 4, true>(p, st) : launch_fused<bf, float, 128, 4, true>(p, st); break;
+    case 8: rc = d == 64 ? launch_fused<bf, float, 64, 8, true>(p, st) : launch_fused<bf, float, 128, 8, true>(p, st); break;
+    default: rc = BSA_ERR_UNSUPPORTED;
+  }
+  return rc;
+}
+
 }  // namespace bsa
 
 extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v,

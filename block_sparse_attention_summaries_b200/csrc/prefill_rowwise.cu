@@ -26,6 +26,10 @@ bsa_status decode_attn(const void* q, const void* k, const void* v, bsa_dtype dt
                        const int* count, int K, int gate, int norm, const float* scores,
                        int scores_ld, void* o, float* lse, void* ws, size_t ws_bytes,
                        cudaStream_t st);
+bsa_status decode_attn_given(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
+                             int Hq, int Hk, int n, int d, int b, const int* seq_lens,
+                             const int* idx, const int* count, int K, int gate, void* o,
+                             float* lse, int* status, cudaStream_t st);
 bool prefill_tc_supported(bsa_dtype dt, int d, int b, int q_block, int K, int Hq, int Hk);
 bsa_status gate_grad_tc(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, int B, int Hq, int Hk, int n, int d,
@@ -337,6 +341,19 @@ extern "C" bsa_status bsa_sparse_attn_fwd(const void* q, const void* k, const vo
   if (nq == 1) {
     BSA_REQUIRE(gate != BSA_GATE_OUTER, BSA_ERR_UNSUPPORTED);  // a training-mode (prefill) gate
     BSA_REQUIRE(b <= 128, BSA_ERR_UNSUPPORTED);
+    // bf16 in 64-token blocks without a gate: the cluster step of bsa_decode_step on the given
+    // selection (warp MMAs over TMA tiles); its status word is the workspace's
+    const int G = Hq / Hk;
+    const int S = decode_splits(B, Hk, G, K);
+    BSA_REQUIRE(workspace && workspace_bytes >= decode_workspace_bytes(B, Hq, Hk, d, K, S),
+                BSA_ERR_WORKSPACE);
+    rc = decode_attn_given(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, idx, count, K, gate, o, lse,
+                           static_cast<int*>(workspace), st);
+    if (rc == BSA_OK) {
+      BSA_LAUNCH_CHECK();
+      return BSA_OK;
+    }
+    if (rc != BSA_ERR_UNSUPPORTED) return rc;
     return decode_attn(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, idx, count, K, gate, norm,
                        scores, scores_ld, o, lse, workspace, workspace_bytes, st);
   }

@@ -248,6 +248,45 @@ def test_decode_chain_ragged_bf16(G, K, b):
             assert eo < 2e-2 and el < 2e-2, (bi, h, eo, el)
 
 
+def test_decode_given_selection_cluster_path_matches_split_k():
+    """bf16 K/V in 64-token blocks without a gate: bsa_sparse_attn_fwd (decode) runs the cluster
+    step on the given selection.  Lists with repeats, negative and out-of-history entries and
+    short counts: against the split-K kernel (the allocation-free entry) and the oracle over each
+    row's distinct valid blocks."""
+    B, Hq, Hk, n, d, b, K = 2, 8, 2, 4000, 128, 64, 9
+    seq = [4000, 1234]
+    case = inputs.decode_case(77, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, needles=2,
+                              seq_lens=seq)
+    q, k, v = up(case.q, True), up(case.k, True), up(case.v, True)
+    sl = up_i32(case.seq_lens)
+    rng = np.random.default_rng(5)
+    idx = rng.integers(-2, 70, size=(B, Hq, K)).astype(np.int32)
+    idx[0, 0, 1] = idx[0, 0, 0]
+    idx[1, 3, :] = 5
+    cnt = rng.integers(0, K + 1, size=(B, Hq)).astype(np.int32)
+    cnt[0, 0] = K
+    o1, lse1 = bsa.sparse_attn_fwd(q, k, v, up_i32(idx), b, count=up_i32(cnt), seq_lens=sl)
+    o2, lse2 = bsa.sparse_attn_decode_noalloc(q, k, v, up_i32(idx), b, count=up_i32(cnt),
+                                              seq_lens=sl)
+    torch.cuda.synchronize()
+    assert bsa.noalloc_status() == 0
+    # the cluster step rounds the scaled query to bf16 for its MMAs: the bf16 output bar
+    assert (o1.float() - o2.float()).abs().max().item() < 2e-2
+    assert (lse1 - lse2).abs().max().item() < 1e-2
+    o1, lse1 = o1.float().cpu().numpy(), lse1.cpu().numpy()
+    G = Hq // Hk
+    for bi in range(B):
+        L = seq[bi]
+        cur = (L - 1) // b
+        for h in range(Hq):
+            kh = h // G
+            sel = sorted({int(m) for m in idx[bi, h, :cnt[bi, h]] if 0 <= m < cur})
+            ro, rl = orc.sparse_attention_row(case.q[bi, h], case.k[bi, kh, :L],
+                                              case.v[bi, kh, :L], L - 1, b, sel)
+            assert np.max(np.abs(o1[bi, h] - ro)) < 2e-2, (bi, h)
+            assert abs(lse1[bi, h] - rl) < 2e-2, (bi, h)
+
+
 def test_decode_gated_bf16_all_history():
     B, Hq, Hk, n, d, b, K = 2, 8, 2, 2048, 128, 64, 6
     case = inputs.decode_case(16, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, needles=0,
