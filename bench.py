@@ -55,13 +55,13 @@ WORKLOADS = {
 MEASURED_TRAFFIC = {
     ("sas_gqa_decode_32k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "34d6ff7c98961cf4",
-        "bytes": 52_599_808 + 212_992},
+        "device_end": "int pick_cluster(", "sha256_16": "56f3917e0cf88e54",
+        "bytes": 52_599_808 + 278_528},
     # two launches per step (chunk Top-K, then merge + attention): their sum
     ("long_decode_512k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "34d6ff7c98961cf4",
-        "bytes": 33_624_064 + 16_130_304},
+        "device_end": "int pick_cluster(", "sha256_16": "56f3917e0cf88e54",
+        "bytes": 33_624_320 + 5_888 + 16_130_048},
 }
 
 
