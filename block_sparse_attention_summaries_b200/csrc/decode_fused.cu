@@ -504,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ int s_abort;
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
+  __shared__ float s_wt[G][kWarps];  // merge weights of the warp partials
   static_assert(kWarps * kScratchPerWarp >= kWarps * 128, "append partials fit the scratch");
 
   // The K/V tensor maps are kernel parameters: their descriptors are fetched while the launch
@@ -1157,14 +1158,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
       }
     }
     __syncthreads();
-    if (s_abort && tid == 0) {
-      // copies still in flight: the last stage issued into each slot; waiting on its own phase
-      // parity returns at once if it already landed
-      for (int st = 0; st < NKV; ++st)
-        if (s_kv_par[st] >= 0) (void)mbar_wait_bounded(&kvbar[st], (uint32_t)s_kv_par[st], 1u << 12);
-      report_timeout(p.status, 2);
+    // a group stops at the first slot whose phase holds no stage, after every slot ahead of it in
+    // its ring: no copy is left in flight unless a wait ran out (s_abort is uniform here)
+    if (s_abort) {
+      if (tid == 0) {
+        // copies still in flight: the last stage issued into each slot; waiting on its own phase
+        // parity returns at once if it already landed
+        for (int st = 0; st < NKV; ++st)
+          if (s_kv_par[st] >= 0)
+            (void)mbar_wait_bounded(&kvbar[st], (uint32_t)s_kv_par[st], 1u << 12);
+        report_timeout(p.status, 2);
+      }
+      __syncthreads();
     }
-    __syncthreads();
     // warp partials (heads < G): m, l and o
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -1356,17 +1362,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
 
   // ---- 5. merge the warps, push column slices to their owners, finish -----------------------
   const int cols = D / CL;
-  // per head: combined max over warps, then weights
+  // per head: combined max over warps, each warp's weight, the weighted sum of the l's
   for (int g = warp; g < G; g += kWarps) {
-    float M = -INFINITY;
-    if (lane < kWarps) M = wpart[((size_t)lane * G + g) * (D + 2) + D];
-    M = warp_max(M);
-    float lsum = 0.f;
-    if (lane < kWarps) {
-      const float mw = wpart[((size_t)lane * G + g) * (D + 2) + D];
-      const float w = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      lsum = w * wpart[((size_t)lane * G + g) * (D + 2) + D + 1];
-    }
+    const float mw = lane < kWarps ? wpart[((size_t)lane * G + g) * (D + 2) + D] : -INFINITY;
+    const float M = warp_max(mw);
+    const float w = mw == -INFINITY ? 0.f : exp2f(mw - M);
+    if (lane < kWarps) s_wt[g][lane] = w;
+    float lsum = lane < kWarps ? w * wpart[((size_t)lane * G + g) * (D + 2) + D + 1] : 0.f;
     lsum = warp_sum(lsum);
     if (lane == 0) {
       s_m[g] = M;
@@ -1379,10 +1381,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const float M = s_m[g];
     float osum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = wpart[((size_t)w * G + g) * (D + 2) + D];
-      if (mw != -INFINITY) osum = fmaf(exp2f(mw - M), wpart[((size_t)w * G + g) * (D + 2) + col], osum);
-    }
+    for (int w = 0; w < kWarps; ++w)
+      osum = fmaf(s_wt[g][w], wpart[((size_t)w * G + g) * (D + 2) + col], osum);
     // push to the owner of this column: recv[rank][g][col % cols], plus (m, l)
     const int owner = col / cols;
     float* slot = recv + ((size_t)rank * G + g) * (cols + 2);
