@@ -55,13 +55,13 @@ WORKLOADS = {
 MEASURED_TRAFFIC = {
     ("sas_gqa_decode_32k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "42981fd643edd9d3",
-        "bytes": 52_598_272 + 296_704},
+        "device_end": "int pick_cluster(", "sha256_16": "b5120e81ff9f32e1",
+        "bytes": 52_599_040 + 269_824},
     # two launches per step (chunk Top-K, then merge + attention): their sum
     ("long_decode_512k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "42981fd643edd9d3",
-        "bytes": 33_624_320 + 16_130_048},
+        "device_end": "int pick_cluster(", "sha256_16": "b5120e81ff9f32e1",
+        "bytes": 33_624_320 + 16_130_304},
 }
 
 
@@ -1017,16 +1017,21 @@ def run_gpu(args):
                           "union_blocks": v_union, "needle_recall": v_hits / max(1, tot),
                           "index_agreement_vs_per_head_fp32": agree}
 
-    # end to end through the public API: pinned host q in, the decode step (a prepared binding
-    # call, bsa.DecodeStep -> bsa_decode_step_ex, or _ws for long histories, no graph), o out,
-    # every step
+    # end to end through the public API with host buffers: a prepared binding call per step
+    # (bsa.DecodeStep -> bsa_decode_step_ws with DECODE_HOST_IO, no graph) whose q is page-locked
+    # host memory that the step moves to the device itself and whose o it writes back to
+    # page-locked host memory
     q_host = [torch.from_numpy(np.ascontiguousarray(L["q"].float().cpu().numpy()))
               .to(torch.bfloat16).pin_memory() for L in layers]
     o_host = torch.empty(B, Hq, d, dtype=torch.bfloat16).pin_memory()
-    plans = [bsa.DecodeStep(L["q"], L["k"], L["v"], L["mean_k"], b, K, append=True,
-                            max_norm=L["max_norm"], centre=L["centre"], o=L["o"], lse=L["lse"],
-                            idx=L["idx"], count=L["count"], status=status, ws=ws)
-             for L in layers]
+    ws_io = torch.empty(bsa.decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K,
+                                                        bsa.DECODE_HOST_IO),
+                        dtype=torch.uint8, device=dev)
+    plans = [bsa.DecodeStep(q_host[r], L["k"], L["v"], L["mean_k"], b, K,
+                            flags=bsa.DECODE_HOST_IO, append=True, max_norm=L["max_norm"],
+                            centre=L["centre"], o=o_host, lse=L["lse"], idx=L["idx"],
+                            count=L["count"], status=status, ws=ws_io)
+             for r, L in enumerate(layers)]
     # two events bracket the timed steps, as for the device-only figure (an event between two
     # steps would add its own cost to every step)
     with torch.cuda.stream(stream):
@@ -1035,10 +1040,7 @@ def run_gpu(args):
                 torch.cuda.synchronize(dev)
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            L = layers[i % R]
-            L["q"].copy_(q_host[i % R], non_blocking=True)
             plans[i % R](stream)
-            o_host.copy_(L["o"], non_blocking=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -1082,10 +1084,11 @@ def run_gpu(args):
         "needle_recall": acc["needle_recall"], "status_word": st_word,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * Hq * d * 2,
                 "d2h_bytes_per_step": B * Hq * d * 2,
-                "what": "per step: pinned-host q -> device, the decode step through a prepared "
-                        "binding call (bsa.DecodeStep) and the C ABI (bsa_decode_step_ex; "
-                        "bsa_decode_step_ws past 512 history blocks; no graph), o -> pinned "
-                        "host; CUDA events on the stream"},
+                "what": "per step one prepared binding call (bsa.DecodeStep) into the C ABI "
+                        "(bsa_decode_step_ws, DECODE_HOST_IO; no graph): q read from pinned "
+                        "host memory into the device by the step's staging kernel, the fused "
+                        "step, o written by it to pinned host memory; two CUDA events bracket "
+                        "the timed steps"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": {k2: clocks[k2] for k2 in ("sm_mhz", "sm_max_mhz", "reasons")},
         "clock_samples": clocks["samples"],

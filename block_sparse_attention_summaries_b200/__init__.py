@@ -127,6 +127,16 @@ def _cuda(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _host_io(*ts):
+    """q / o of a host-I/O decode step: contiguous page-locked host tensors."""
+    for t in ts:
+        if t is not None:
+            if t.is_cuda or not t.is_pinned():
+                raise ValueError("host-I/O tensors must be page-locked host memory")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
 def _i32(t):
     if t is None:
         return None
@@ -519,6 +529,7 @@ def decode_step_fused(q, k, v, mean_k, b, K, seq_lens=None, append=True, max_nor
 
 DECODE_SHARED_SELECTION = 1
 DECODE_BF16_SUMMARIES = 2
+DECODE_HOST_IO = 4
 
 
 def decode_step_ex(q, k, v, mean_k, b, K, flags, seq_lens=None, append=True, max_norm=None,
@@ -557,27 +568,36 @@ def decode_step_ws(q, k, v, mean_k, b, K, flags=0, ws=None, seq_lens=None, appen
                    o=None, lse=None, idx=None, count=None, status=None):
     """bsa_decode_step_ws: the fused decode step; long histories on the 64-token bf16 path run as
     two launches through the workspace ``ws`` (a uint8 device tensor; allocated here when None).
-    Returns (o, lse, idx, count)."""
-    _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count, ws)
+    With DECODE_HOST_IO in ``flags``, q and o are page-locked host tensors (o allocated pinned
+    here when None).  Returns (o, lse, idx, count)."""
+    host_io = bool(flags & DECODE_HOST_IO)
+    if host_io:
+        _host_io(q, o)
+        _cuda(k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, lse, idx, count, ws)
+    else:
+        _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count,
+              ws)
     B, Hk, n, d = k.shape
     Hq = q.shape[1]
+    dev = k.device
     if o is None:
-        o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+        o = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if host_io
+             else torch.empty(q.shape, device=dev, dtype=q.dtype))
     if lse is None:
-        lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+        lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
     if idx is None:
-        idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+        idx = torch.empty(B, Hq, K, device=dev, dtype=torch.int32)
     if count is None:
-        count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+        count = torch.empty(B, Hq, device=dev, dtype=torch.int32)
     if ws is None:
         need = decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, flags, q.dtype)
-        ws = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+        ws = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
     _check(lib().bsa_decode_step_ws(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), B, Hq, Hk, n, d, b,
                                     _ptr(_i32(seq_lens)), _ptr(mean_k), _ptr(max_norm),
                                     _ptr(centre), 1 if append else 0, _ptr(lambda_h),
                                     _ptr(sigma_h), prefix_block, K, _ptr(o), _ptr(lse), _ptr(idx),
                                     _ptr(count), _ptr(status), int(flags), _ptr(ws), ws.numel(),
-                                    _stream(q.device)), "bsa_decode_step_ws")
+                                    _stream(dev)), "bsa_decode_step_ws")
     return o, lse, idx, count
 
 
@@ -590,24 +610,35 @@ class DecodeStep:
     by this object and must keep their storage: write new queries into ``q`` in place.
     ``outputs`` is (o, lse, idx, count).  With a workspace ``ws`` (a uint8 device tensor of at
     least decode_step_workspace_bytes) the call is bsa_decode_step_ws: long histories take the
-    two-launch path.
+    two-launch path, and with DECODE_HOST_IO in ``flags`` q and o are page-locked host tensors
+    (the step reads q from and writes o to host memory itself).
     """
 
     def __init__(self, q, k, v, mean_k, b, K, flags=0, seq_lens=None, append=True,
                  max_norm=None, centre=None, lambda_h=None, sigma_h=None, prefix_block=0,
                  o=None, lse=None, idx=None, count=None, status=None, ws=None):
-        _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx, count,
-              ws)
+        host_io = bool(flags & DECODE_HOST_IO)
+        if host_io:
+            if ws is None:
+                raise ValueError("DECODE_HOST_IO needs a workspace")
+            _host_io(q, o)
+            _cuda(k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, lse, idx, count,
+                  ws)
+        else:
+            _cuda(q, k, v, mean_k, seq_lens, max_norm, centre, lambda_h, sigma_h, o, lse, idx,
+                  count, ws)
         B, Hk, n, d = k.shape
         Hq = q.shape[1]
+        dev = k.device
         if o is None:
-            o = torch.empty(q.shape, device=q.device, dtype=q.dtype)
+            o = (torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if host_io
+                 else torch.empty(q.shape, device=dev, dtype=q.dtype))
         if lse is None:
-            lse = torch.empty(q.shape[:-1], device=q.device, dtype=torch.float32)
+            lse = torch.empty(q.shape[:-1], device=dev, dtype=torch.float32)
         if idx is None:
-            idx = torch.empty(B, Hq, K, device=q.device, dtype=torch.int32)
+            idx = torch.empty(B, Hq, K, device=dev, dtype=torch.int32)
         if count is None:
-            count = torch.empty(B, Hq, device=q.device, dtype=torch.int32)
+            count = torch.empty(B, Hq, device=dev, dtype=torch.int32)
         sl = _i32(seq_lens)
         self._keep = (q, k, v, mean_k, sl, max_norm, centre, lambda_h, sigma_h, status, ws)
         self.outputs = (o, lse, idx, count)
@@ -619,7 +650,7 @@ class DecodeStep:
                       _ptr(idx), _ptr(count), _ptr(status), int(flags))
         if ws is not None:
             self._args = self._args + (_ptr(ws), ws.numel())
-        self._device = q.device
+        self._device = dev
 
     def __call__(self, stream=None):
         """Run the step on ``stream`` (a torch.cuda.Stream; default: the current stream)."""

@@ -92,6 +92,7 @@ struct FusedParams {
   int row_ld;  // stride of the whole-row key copies (gather) in keys
   int ns;      // summary ring stages
   int nkv;     // K/V ring stages
+  int host_io;  // q and o through their device mappings of page-locked host memory (modes 0, 2)
   // Long histories in two launches: mode 1 scores one chunk of the history per CTA (no cluster)
   // and writes every selecting head's chunk Top-K to `cand`; mode 2 merges those lists and runs
   // phases 3-5.  Mode 0 is the whole step in one launch.
@@ -142,6 +143,28 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t addr, uint4 v) {
                "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
+// Arrive, with release at cluster scope, on the mbarrier at a shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+               : "memory");
+}
+// Bounded wait with acquire at cluster scope (for a phase completed by another CTA's arrive).
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_t parity,
+                                                          uint32_t limit = (1u << 20)) {
+  for (uint32_t it = 0; it < limit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+
 __device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -477,7 +500,10 @@ struct FusedSmem {
 // kMode: 0 the whole step; 1 and 2 the two launches of a long history; 3 the attention of a given
 // selection (FusedParams::mode), each its own instantiation so that the one-launch step's code is
 // unchanged by them.
-template <typename T, typename TS, int D, int G, bool MMA, int kMode = 0>
+// kHostIO: q and o through their device mappings of page-locked host memory (its own
+// instantiation too: the staging of q and the packed stores of o leave the device-buffer code
+// unchanged).
+template <typename T, typename TS, int D, int G, bool MMA, int kMode = 0, bool kHostIO = false>
 __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
     const __grid_constant__ CUtensorMap tmk64, const __grid_constant__ CUtensorMap tmv64,
@@ -485,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   constexpr bool kMma = MMA;
   static_assert(!MMA || std::is_same<T, __nv_bfloat16>::value, "warp MMAs take bf16");
   static_assert(kMode == 0 || MMA, "modes 1-3 are the 64-token bf16 path");
+  static_assert(!kHostIO || (MMA && (kMode == 0 || kMode == 2)), "host I/O: cluster steps");
   constexpr int EPL = D / 32;
   constexpr int R = 32 / G;
 
@@ -505,6 +532,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
   __shared__ float s_wt[G][kWarps];  // merge weights of the warp partials
+  // With q in page-locked host memory, the group's G query rows are read once by rank 0 of the
+  // cluster and pushed to every CTA (one read of q per group).  bf16 path, cluster modes.
+  constexpr bool kStageQ = kHostIO;
+  __shared__ __align__(16) T s_q[kStageQ ? G * D : 8];
+  __shared__ __align__(8) uint64_t s_qbar;
   static_assert(kWarps * kScratchPerWarp >= kWarps * 128, "append partials fit the scratch");
 
   // The K/V tensor maps are kernel parameters: their descriptors are fetched while the launch
@@ -548,6 +580,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
 
   if (tid == 0) {
     for (int i = 0; i < NS + NKV; ++i) mbar_init(&bar[i], 1);
+    if constexpr (kStageQ) mbar_init(&s_qbar, 1);
     fence_mbar_init();
     if (kMode == 2) {  // the group's chunk lists (one contiguous block) into region A, first
       const size_t words = (size_t)p.nchunk * (p.shared ? 1 : G) * p.cand_ld;
@@ -594,12 +627,30 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   if (tid == 0)
     for (; sub_issued < min(nsub, NS); ++sub_issued) issue_sub(sub_issued);
   const int cand_group = Gs * p.cand_ld;  // mode 2: words per chunk of the lists
+  const T* qsrc = static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0) * D;  // the G rows
+  constexpr bool stage_q = kStageQ;
+  if constexpr (stage_q) {
+    // rank 0 reads the G rows once and pushes them to every CTA, then arrives on each CTA's q
+    // barrier (its threads wait for the cluster here; the other CTAs' threads in phase 2)
+    constexpr int kQ16 = G * D * (int)sizeof(T) / 16;
+    static_assert(kQ16 <= kThreads, "one 16-byte piece of q per thread");
+    if (rank == 0) {
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (tid < kQ16) x = reinterpret_cast<const uint4*>(qsrc)[tid];
+      cluster_wait();  // every peer has started: DSMEM stores may begin
+      if (tid < kQ16)
+        for (int r = 0; r < CL; ++r) st_dsmem_v4(dsmem_addr(reinterpret_cast<uint4*>(s_q) + tid, r), x);
+      __syncthreads();
+      if (tid < CL) mbar_arrive_remote(dsmem_addr(&s_qbar, tid));
+    }
+    if (!mbar_wait_cluster_bounded(&s_qbar, 0)) s_abort = 1;  // reported with phase 1's timeouts
+    qsrc = s_q;
+  }
   float qv[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     float tmp[EPL];
-    load_vec<T, EPL>(static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + g) * D + lane * EPL,
-                     tmp);
+    load_vec<T, EPL>(qsrc + (size_t)g * D + lane * EPL, tmp);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) qv[g][e] = tmp[e];
   }
@@ -664,7 +715,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   // ---- 2. Top-K per head (per group when shared) -----------------------------------------
   uint32_t* ck = s_scratch + warp * kScratchPerWarp;
   int* cp = reinterpret_cast<int*>(ck + kCandMax + 4);
-  if (kMode != 1) cluster_wait();  // every peer has started: DSMEM stores may begin
+  // every peer has started: DSMEM stores may begin (rank 0 of a q-staging launch waited already)
+  if (kMode != 1 && !(stage_q && rank == 0)) cluster_wait();
   if constexpr (kMode == 1) {
     // this chunk's Top-K of every selecting head in rank order (key descending, ties to the lower
     // block: the pair sorts as key, then the complement of the block index), with its count
@@ -1021,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     uint32_t qa0[D / 16], qa1[D / 16];
     {
       const float qs = scale * kLog2e;
-      const T* qrow = static_cast<const T*>(p.q) + ((size_t)bi * Hq + h0 + min(grow, G - 1)) * D;
+      const T* qrow = qsrc + (size_t)min(grow, G - 1) * D;
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
         float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
@@ -1393,21 +1445,45 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     }
   }
   cluster_sync();
-  for (int e = tid; e < G * cols; e += kThreads) {
-    const int g = e / cols, cc = e % cols, col = rank * cols + cc;
+  // each thread finishes V consecutive columns of one head and writes them with one 8- or 16-byte
+  // store when o lives in page-locked host memory (cols = D / CL is a power of two >= 4), one
+  // column per thread otherwise
+  const int V = kHostIO ? (cols >= 8 ? 8 : 4) : 1, per_g = cols / V;
+  for (int e = tid; e < G * per_g; e += kThreads) {
+    const int g = e / per_g, cc = (e % per_g) * V, col = rank * cols + cc;
     float M = -INFINITY;
     for (int r = 0; r < CL; ++r) M = fmaxf(M, recv[((size_t)r * G + g) * (cols + 2) + cols]);
-    float lsum = 0.f, osum = 0.f;
+    float lsum = 0.f, osum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < CL; ++r) {
       const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
       const float mr = slot[cols];
       if (mr == -INFINITY) continue;
       const float w = exp2f(mr - M);
       lsum = fmaf(w, slot[cols + 1], lsum);
-      osum = fmaf(w, slot[cc], osum);
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        if (v < V) osum[v] = fmaf(w, slot[cc + v], osum[v]);
     }
     const size_t row = (size_t)bi * Hq + h0 + g;
-    static_cast<T*>(p.o)[row * D + col] = Elem<T>::from_f(osum / lsum);
+    const float inv = 1.f / lsum;
+    T* dst = static_cast<T*>(p.o) + row * D + col;
+    if (V == 1) {
+      *dst = Elem<T>::from_f(osum[0] / lsum);
+    } else if constexpr (sizeof(T) == 2) {
+      const uint32_t w0 = pack_bf16(osum[0] * inv, osum[1] * inv);
+      const uint32_t w1 = pack_bf16(osum[2] * inv, osum[3] * inv);
+      if (V == 8)
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w0, w1, pack_bf16(osum[4] * inv, osum[5] * inv),
+                                                    pack_bf16(osum[6] * inv, osum[7] * inv));
+      else
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w0, w1);
+    } else {
+      *reinterpret_cast<float4*>(dst) =
+          make_float4(osum[0] * inv, osum[1] * inv, osum[2] * inv, osum[3] * inv);
+      if (V == 8)
+        *reinterpret_cast<float4*>(dst + 4) =
+            make_float4(osum[4] * inv, osum[5] * inv, osum[6] * inv, osum[7] * inv);
+    }
     if (col == 0 && p.lse) p.lse[row] = (M + log2f(lsum)) * kLn2;
   }
 }
@@ -1483,6 +1559,8 @@ bsa_status launch_fused(FusedParams& p, cudaStream_t st) {
   if constexpr (MMA) {
     if (p.mode == 2) kern = decode_fused_kernel<T, TS, D, G, MMA, 2>;
     if (p.mode == 3) kern = decode_fused_kernel<T, TS, D, G, MMA, 3>;
+    if (p.host_io && p.mode == 0) kern = decode_fused_kernel<T, TS, D, G, MMA, 0, true>;
+    if (p.host_io && p.mode == 2) kern = decode_fused_kernel<T, TS, D, G, MMA, 2, true>;
   }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -1753,18 +1831,37 @@ bsa_status dispatch_fused(int G, FusedParams& p, cudaStream_t st, uint32_t* ws =
 namespace bsa {
 namespace {
 
+// q of a host-I/O step into the workspace: the host reads are issued at once (the launch may be
+// scheduled while the previous step still runs), the stores into the staging buffer only after
+// the work queued before it -- the previous step, which reads that buffer -- has completed.
+__global__ void __launch_bounds__(128) stage_q_kernel(const uint4* __restrict__ src,
+                                                      uint4* __restrict__ dst, int n16) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  uint4 x = make_uint4(0u, 0u, 0u, 0u);
+  if (i < n16) x = src[i];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (i < n16) dst[i] = x;
+}
+
+constexpr int kHostIo = 4;  // BSA_DECODE_HOST_IO
+
+size_t q_stage_offset(size_t plan_bytes) { return align_up(plan_bytes, (size_t)256); }
+
 bsa_status decode_step_impl(const void* q, const void* k, const void* v, bsa_dtype dt, int B,
                             int Hq, int Hk, int n, int d, int b, const int* seq_lens,
                             void* mean_k, float* max_norm, float* centre, int append,
                             const float* lambda_h, const float* sigma_h, int prefix_block, int K,
                             void* o, float* lse, int* idx, int* count, int* status, int flags,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+                            void* workspace, size_t workspace_bytes, bool allow_host_io,
+                            void* stream) {
   BSA_REQUIRE(dtype_ok(dt), BSA_ERR_DTYPE);
   BSA_REQUIRE(q && k && v && mean_k && o, BSA_ERR_ARG);
   BSA_REQUIRE(B > 0 && Hq > 0 && Hk > 0 && n > 0 && d > 0 && b > 0 && K > 0 && prefix_block >= 0,
               BSA_ERR_ARG);
-  BSA_REQUIRE((flags & ~(BSA_DECODE_SHARED_SELECTION | BSA_DECODE_BF16_SUMMARIES)) == 0,
-              BSA_ERR_ARG);
+  const int known = BSA_DECODE_SHARED_SELECTION | BSA_DECODE_BF16_SUMMARIES |
+                    (allow_host_io ? kHostIo : 0);
+  BSA_REQUIRE((flags & ~known) == 0, BSA_ERR_ARG);
   BSA_REQUIRE((lambda_h == nullptr) == (sigma_h == nullptr), BSA_ERR_ARG);
   BSA_REQUIRE(!lambda_h || (max_norm && centre), BSA_ERR_ARG);
   BSA_REQUIRE(Hq % Hk == 0, BSA_ERR_SHAPE);
@@ -1790,6 +1887,46 @@ bsa_status decode_step_impl(const void* q, const void* k, const void* v, bsa_dty
   using bf = __nv_bfloat16;
   BSA_REQUIRE(!workspace || aligned16(workspace), BSA_ERR_ARG);
   uint32_t* ws = workspace_bytes > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
+  if (flags & kHostIo) {
+    // q and o in page-locked host memory: o written by the step straight to its device mapping;
+    // q read through its device mapping by rank 0 of each cluster, once per group, on the
+    // one-launch bf16 path, and otherwise staged into the workspace (after the chunk lists) by a
+    // copy kernel first
+    const bool mma = dt == BSA_BF16 && b == 64;
+    const SplitPlan sp = split_plan(B, Hk, Hq / Hk, C, K, p.shared != 0, mma);
+    const size_t qoff = q_stage_offset(sp.bytes);
+    const size_t qbytes = (size_t)B * Hq * d * (dt == BSA_BF16 ? 2 : 4);
+    BSA_REQUIRE(ws && workspace_bytes >= qoff + qbytes, BSA_ERR_WORKSPACE);
+    void* qd = nullptr;
+    void* od = nullptr;
+    if (cudaHostGetDevicePointer(&qd, const_cast<void*>(q), 0) != cudaSuccess ||
+        cudaHostGetDevicePointer(&od, o, 0) != cudaSuccess || !aligned16(qd) || !aligned16(od)) {
+      (void)cudaGetLastError();
+      return BSA_ERR_ARG;
+    }
+    p.o = od;
+    p.q = qd;
+    p.host_io = 1;
+    if (!(mma && sp.nchunk == 0)) {
+      unsigned char* stage = reinterpret_cast<unsigned char*>(ws) + qoff;
+      const int n16 = (int)(qbytes / 16);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)ceil_div(n16, 128), 1, 1);
+      cfg.blockDim = dim3(128, 1, 1);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, stage_q_kernel, static_cast<const uint4*>(qd),
+                             reinterpret_cast<uint4*>(stage), n16) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BSA_ERR_CUDA;
+      }
+      p.q = stage;
+    }
+  }
   bsa_status rc;
   if (dt == BSA_BF16 && b == 64 && bf16_sum)
     rc = d == 64 ? dispatch_fused<bf, bf, 64, true>(Hq / Hk, p, st, ws, workspace_bytes)
@@ -1852,7 +1989,7 @@ extern "C" bsa_status bsa_decode_step_ex(const void* q, const void* k, const voi
                                          int flags, void* stream) {
   return bsa::decode_step_impl(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, mean_k, max_norm,
                                centre, append, lambda_h, sigma_h, prefix_block, K, o, lse, idx,
-                               count, status, flags, nullptr, 0, stream);
+                               count, status, flags, nullptr, 0, false, stream);
 }
 
 extern "C" size_t bsa_decode_step_workspace_bytes(int B, int Hq, int Hk, int n, int d, int b,
@@ -1861,8 +1998,10 @@ extern "C" size_t bsa_decode_step_workspace_bytes(int B, int Hq, int Hk, int n, 
   if (B <= 0 || Hq <= 0 || Hk <= 0 || n <= 0 || d <= 0 || b <= 0 || K <= 0 || Hq % Hk != 0)
     return 0;
   const bool mma = dt == BSA_BF16 && b == 64 && (d == 64 || d == 128);
-  return split_plan(B, Hk, Hq / Hk, ceil_div(n, b), K,
-                    (flags & BSA_DECODE_SHARED_SELECTION) != 0, mma).bytes;
+  const size_t plan = split_plan(B, Hk, Hq / Hk, ceil_div(n, b), K,
+                                 (flags & BSA_DECODE_SHARED_SELECTION) != 0, mma).bytes;
+  if (!(flags & kHostIo)) return plan;
+  return q_stage_offset(plan) + (size_t)B * Hq * d * (dt == BSA_BF16 ? 2 : 4);
 }
 
 extern "C" bsa_status bsa_decode_step_ws(const void* q, const void* k, const void* v,
@@ -1875,7 +2014,7 @@ extern "C" bsa_status bsa_decode_step_ws(const void* q, const void* k, const voi
                                          void* stream) {
   return bsa::decode_step_impl(q, k, v, dt, B, Hq, Hk, n, d, b, seq_lens, mean_k, max_norm,
                                centre, append, lambda_h, sigma_h, prefix_block, K, o, lse, idx,
-                               count, status, flags, workspace, workspace_bytes, stream);
+                               count, status, flags, workspace, workspace_bytes, true, stream);
 }
 
 extern "C" bsa_status bsa_decode_step(const void* q, const void* k, const void* v, bsa_dtype dt,

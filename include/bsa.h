@@ -75,7 +75,14 @@ typedef enum {
   BSA_DECODE_SHARED_SELECTION = 1,
   /* mean_k is bf16 [B, Hk, C, d] (see bsa_round_summaries_bf16): half the summary bytes; the dot
    * products still accumulate in fp32.  Needs dt = BSA_BF16 and b = 64. */
-  BSA_DECODE_BF16_SUMMARIES = 2
+  BSA_DECODE_BF16_SUMMARIES = 2,
+  /* bsa_decode_step_ws only: q and o are page-locked host buffers (cudaHostAlloc, or a pinned
+   * torch tensor) instead of device memory.  The step moves q into its workspace with one small
+   * kernel -- whose host reads may start before the work queued ahead of it on the stream has
+   * finished, so that work must not write q -- and its last phase writes o straight to host
+   * memory; o is complete once the stream has passed the call.  BSA_ERR_ARG if q or o is not
+   * page-locked host memory mapped for the device. */
+  BSA_DECODE_HOST_IO = 4
 } bsa_decode_flags;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -206,7 +213,8 @@ bsa_status bsa_decode_step_ex(const void* q, const void* k, const void* v, bsa_d
  * bsa_decode_step_ex (same scores, same order, ties to the lower block).
  *   workspace        device memory, 16-byte aligned, owned by the caller; no initialisation is
  *                    needed and it may be reused once the stream has passed the call.  NULL or
- *                    workspace_bytes = 0: bsa_decode_step_ex (one launch).
+ *                    workspace_bytes = 0: bsa_decode_step_ex (one launch).  With
+ *                    BSA_DECODE_HOST_IO it also holds the device copy of q.
  *   workspace_bytes  its size; BSA_ERR_WORKSPACE if nonzero and below
  *                    bsa_decode_step_workspace_bytes().
  */
@@ -217,8 +225,9 @@ bsa_status bsa_decode_step_ws(const void* q, const void* k, const void* v, bsa_d
                               void* o, float* lse, int* idx, int* count, int* status, int flags,
                               void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace bytes bsa_decode_step_ws uses for this shape (dt is a bsa_dtype value); 0 when the
- * step runs as one launch (short histories, other dtypes or block sizes, invalid sizes). */
+/* Workspace bytes bsa_decode_step_ws uses for this shape (dt is a bsa_dtype value): the chunk
+ * lists of a long history (none when the step runs as one launch: short histories, other dtypes
+ * or block sizes), plus the device copy of q with BSA_DECODE_HOST_IO; 0 for invalid sizes. */
 size_t bsa_decode_step_workspace_bytes(int B, int Hq, int Hk, int n, int d, int b, int K,
                                        int flags, int dt);
 

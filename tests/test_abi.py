@@ -234,8 +234,16 @@ def test_decode_step_workspace(bsa_lib):
     assert f(*base) == 7                                         # BSA_ERR_WORKSPACE
     bad = list(base); bad[25] = ctypes.c_void_p(0x1004)          # misaligned workspace
     assert f(*bad) == 1
-    bad = list(base); bad[24] = 4                                # unknown flag bit
+    bad = list(base); bad[24] = 8                                # unknown flag bit
     assert f(*bad) == 1
+    # host I/O: the workspace also holds the device copy of q, after the chunk lists
+    assert q(8, 32, 8, 32768, 128, 64, 15, 4, 1) == 8 * 32 * 128 * 2
+    assert q(1, 32, 8, 524288, 128, 64, 31, 4, 1) == need + 32 * 128 * 2
+    assert q(1, 32, 8, 524288, 128, 32, 31, 4, 0) == 32 * 128 * 4   # fp32 q, one launch
+    short = list(base); short[24] = 4; short[26] = need            # no room for q
+    assert f(*short) == 7
+    ex = list(base[:25]) + [None]; ex[24] = 4                      # _ex takes no host I/O
+    assert bsa_lib.bsa_decode_step_ex(*ex) == 1
 
 
 def test_freesolo_workspace_size_query(bsa_lib):

@@ -222,6 +222,36 @@ def test_workspace_path_all_scores_tied_take_the_lowest_blocks(C, K):
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
 
 
+@pytest.mark.parametrize("n,B,K", [(2048 + 17, 2, 7), (600 * 64 + 5, 1, 13)])
+def test_host_io_step_matches_device_buffers(n, B, K):
+    """DECODE_HOST_IO: q and o in page-locked host memory, the step staging q itself and writing o
+    to host memory (one launch at 32 history blocks, two past 512), against the same step on
+    device buffers; two calls in a row check that the staging buffer is reused safely."""
+    Hq, Hk, d, b = 8, 2, 128, 64
+    case = inputs.decode_case(90 + B, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, needles=3)
+    q, k, v, sl = upload(case)
+    mean_k, _, _ = bsa.build_block_summaries(k, b)
+    flags = bsa.DECODE_HOST_IO
+    ws = torch.empty(bsa.decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, flags),
+                     dtype=torch.uint8, device=DEV)
+    q2 = (q * 0.5).contiguous()
+    outs = []
+    for qq in (q, q2):
+        q_host = qq.cpu().pin_memory()
+        o_host = torch.full((B, Hq, d), float("nan"), dtype=torch.bfloat16).pin_memory()
+        o1, lse1, idx1, cnt1 = bsa.decode_step_ws(q_host, k, v, mean_k, b, K, flags=flags, ws=ws,
+                                                  o=o_host, append=False)
+        outs.append((o1, lse1.clone(), idx1.clone()))
+    torch.cuda.synchronize()
+    for qq, (o1, lse1, idx1) in zip((q, q2), outs):
+        o2, lse2, idx2, _ = bsa.decode_step_ws(qq, k, v, mean_k, b, K, append=False)
+        torch.cuda.synchronize()
+        assert not o1.is_cuda and torch.isfinite(o1.float()).all()
+        assert torch.equal(idx1, idx2)
+        assert (o1.float() - o2.float().cpu()).abs().max().item() < 1e-2
+        assert (lse1 - lse2).abs().max().item() < 1e-3
+
+
 def test_workspace_too_small_is_refused():
     n, b, K = 600 * 64, 64, 8
     need = bsa.decode_step_workspace_bytes(1, 8, 2, n, 128, b, K)
