@@ -77,11 +77,12 @@ typedef enum {
    * products still accumulate in fp32.  Needs dt = BSA_BF16 and b = 64. */
   BSA_DECODE_BF16_SUMMARIES = 2,
   /* bsa_decode_step_ws only: q and o are page-locked host buffers (cudaHostAlloc, or a pinned
-   * torch tensor) instead of device memory.  The step moves q into its workspace with one small
-   * kernel -- whose host reads may start before the work queued ahead of it on the stream has
-   * finished, so that work must not write q -- and its last phase writes o straight to host
-   * memory; o is complete once the stream has passed the call.  BSA_ERR_ARG if q or o is not
-   * page-locked host memory mapped for the device. */
+   * torch tensor) instead of device memory.  The step reads q itself (once per kv-head group, or
+   * through a small staging kernel whose host reads may start before the work queued ahead of it
+   * on the stream has finished, so that work must not write q) and its last phase writes o
+   * straight to host memory.  As with an asynchronous copy from page-locked memory, the host must
+   * leave q unchanged, and must not read o, until the stream has passed the call.  BSA_ERR_ARG if
+   * q or o is not page-locked host memory mapped for the device. */
   BSA_DECODE_HOST_IO = 4
 } bsa_decode_flags;
 
