@@ -222,16 +222,21 @@ def test_workspace_path_all_scores_tied_take_the_lowest_blocks(C, K):
     assert (o1.float() - o2.float()).abs().max().item() < 1e-2
 
 
-@pytest.mark.parametrize("n,B,K", [(2048 + 17, 2, 7), (600 * 64 + 5, 1, 13)])
-def test_host_io_step_matches_device_buffers(n, B, K):
+@pytest.mark.parametrize("n,B,K,extra", [(2048 + 17, 2, 7, 0), (600 * 64 + 5, 1, 13, 0),
+                                         (2048 + 17, 2, 7, 1), (600 * 64 + 5, 1, 13, 2)])
+def test_host_io_step_matches_device_buffers(n, B, K, extra):
     """DECODE_HOST_IO: q and o in page-locked host memory, the step staging q itself and writing o
-    to host memory (one launch at 32 history blocks, two past 512), against the same step on
-    device buffers; two calls in a row check that the staging buffer is reused safely."""
+    to host memory (one launch at 32 history blocks, two past 512; alone, with the shared
+    selection and with bf16 summaries), against the same step on device buffers; two calls in a
+    row check that the staging is reused safely."""
     Hq, Hk, d, b = 8, 2, 128, 64
     case = inputs.decode_case(90 + B, B=B, Hq=Hq, Hk=Hk, d=d, n=n, b=b, K=K, needles=3)
     q, k, v, sl = upload(case)
     mean_k, _, _ = bsa.build_block_summaries(k, b)
-    flags = bsa.DECODE_HOST_IO
+    xf = {0: 0, 1: bsa.DECODE_SHARED_SELECTION, 2: bsa.DECODE_BF16_SUMMARIES}[extra]
+    if xf & bsa.DECODE_BF16_SUMMARIES:
+        mean_k = bsa.round_summaries_bf16(mean_k)
+    flags = bsa.DECODE_HOST_IO | xf
     ws = torch.empty(bsa.decode_step_workspace_bytes(B, Hq, Hk, n, d, b, K, flags),
                      dtype=torch.uint8, device=DEV)
     q2 = (q * 0.5).contiguous()
@@ -244,7 +249,7 @@ def test_host_io_step_matches_device_buffers(n, B, K):
         outs.append((o1, lse1.clone(), idx1.clone()))
     torch.cuda.synchronize()
     for qq, (o1, lse1, idx1) in zip((q, q2), outs):
-        o2, lse2, idx2, _ = bsa.decode_step_ws(qq, k, v, mean_k, b, K, append=False)
+        o2, lse2, idx2, _ = bsa.decode_step_ws(qq, k, v, mean_k, b, K, flags=xf, append=False)
         torch.cuda.synchronize()
         assert not o1.is_cuda and torch.isfinite(o1.float()).all()
         assert torch.equal(idx1, idx2)
