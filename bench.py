@@ -55,13 +55,13 @@ WORKLOADS = {
 MEASURED_TRAFFIC = {
     ("sas_gqa_decode_32k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "b5120e81ff9f32e1",
-        "bytes": 52_599_040 + 269_824},
+        "device_end": "int pick_cluster(", "sha256_16": "1c58f395bf756be1",
+        "bytes": 52_596_736 + 270_848},
     # two launches per step (chunk Top-K, then merge + attention): their sum
     ("long_decode_512k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "b5120e81ff9f32e1",
-        "bytes": 33_624_320 + 16_130_304},
+        "device_end": "int pick_cluster(", "sha256_16": "1c58f395bf756be1",
+        "bytes": 33_624_320 + 16_127_232},
 }
 
 

@@ -532,6 +532,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   __shared__ float s_red[kWarps];
   __shared__ float s_m[G], s_l[G], s_corr[G];
   __shared__ float s_wt[G][kWarps];  // merge weights of the warp partials
+  __shared__ float s_fw[G][kMaxCL];  // merge weights of the CTAs' partials (owner side)
+  __shared__ float s_fm[G], s_fl[G];
   // With q in page-locked host memory, the group's G query rows are read once by rank 0 of the
   // cluster and pushed to every CTA (one read of q per group).  bf16 path, cluster modes.
   constexpr bool kStageQ = kHostIO;
@@ -1445,21 +1447,41 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     }
   }
   cluster_sync();
+  // per head: the largest max over the CL partials, each partial's weight and the weighted sum of
+  // the l's, once (lanes of CL-wide groups; CL divides 32), so that a column costs CL FMAs
+  for (int t0 = 0; t0 < G * CL; t0 += kThreads) {
+    const int t = t0 + tid;
+    if (t0 + (tid & ~31) < G * CL) {  // warps holding any (head, partial) pair
+      const bool in = t < G * CL;
+      const int g = in ? t / CL : 0, r = in ? t % CL : 0;
+      const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
+      const float mr = in ? slot[cols] : -INFINITY;
+      float M = mr;
+      for (int o = 1; o < CL; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float w = mr == -INFINITY ? 0.f : exp2f(mr - M);
+      float l = in ? w * slot[cols + 1] : 0.f;
+      for (int o = 1; o < CL; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (in) {
+        s_fw[g][r] = w;
+        if (r == 0) {
+          s_fm[g] = M;
+          s_fl[g] = l;
+        }
+      }
+    }
+  }
+  __syncthreads();
   // each thread finishes V consecutive columns of one head and writes them with one 8- or 16-byte
   // store when o lives in page-locked host memory (cols = D / CL is a power of two >= 4), one
   // column per thread otherwise
   const int V = kHostIO ? (cols >= 8 ? 8 : 4) : 1, per_g = cols / V;
   for (int e = tid; e < G * per_g; e += kThreads) {
     const int g = e / per_g, cc = (e % per_g) * V, col = rank * cols + cc;
-    float M = -INFINITY;
-    for (int r = 0; r < CL; ++r) M = fmaxf(M, recv[((size_t)r * G + g) * (cols + 2) + cols]);
-    float lsum = 0.f, osum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const float M = s_fm[g], lsum = s_fl[g];
+    float osum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < CL; ++r) {
       const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
-      const float mr = slot[cols];
-      if (mr == -INFINITY) continue;
-      const float w = exp2f(mr - M);
-      lsum = fmaf(w, slot[cols + 1], lsum);
+      const float w = s_fw[g][r];
 #pragma unroll
       for (int v = 0; v < 8; ++v)
         if (v < V) osum[v] = fmaf(w, slot[cc + v], osum[v]);
