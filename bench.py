@@ -55,13 +55,13 @@ WORKLOADS = {
 MEASURED_TRAFFIC = {
     ("sas_gqa_decode_32k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "1c58f395bf756be1",
-        "bytes": 52_596_736 + 270_848},
+        "device_end": "int pick_cluster(", "sha256_16": "18c12307660d9922",
+        "bytes": 52_596_992 + 447_488},
     # two launches per step (chunk Top-K, then merge + attention): their sum
     ("long_decode_512k", "decode_fused_kernel"): {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
-        "device_end": "int pick_cluster(", "sha256_16": "1c58f395bf756be1",
-        "bytes": 33_624_320 + 16_127_232},
+        "device_end": "int pick_cluster(", "sha256_16": "18c12307660d9922",
+        "bytes": 33_624_064 + 16_127_232},
 }
 
 

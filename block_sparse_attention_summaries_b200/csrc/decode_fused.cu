@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
   uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + p.off_keys);  // [G][chunk]
   uint32_t* sel_buf = reinterpret_cast<uint32_t*>(smem + p.off_sel);  // whole rows / merge
   uint32_t* hbits = reinterpret_cast<uint32_t*>(smem + p.off_hbits);  // [Gs][nwords] selections
-  float* recv = reinterpret_cast<float*>(smem + p.off_recv);           // [CL][G][cols+2]
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);  // [CL][G][cols], then [CL][G][2]
   float* zs = reinterpret_cast<float*>(smem + p.off_zp);
   float* ps = zs + align_up((size_t)b * G, 4);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + p.off_bar);
@@ -1430,20 +1430,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     }
   }
   __syncthreads();
-  for (int e = tid; e < G * D; e += kThreads) {
-    const int g = e / D, col = e % D;
-    const float M = s_m[g];
-    float osum = 0.f;
+  // four consecutive columns per thread, pushed to their owner with one 16-byte store:
+  // recv[rank][g][col % cols]; (m, l) of the head to recv_ml[rank][g]
+  static_assert((D / kMaxCL) % 4 == 0, "every owner's column slice holds whole 16-byte pieces");
+  float* recv_ml = recv + (size_t)CL * G * cols;
+  for (int e = tid; e < G * D / 4; e += kThreads) {
+    const int g = e / (D / 4), col = (e % (D / 4)) * 4;
+    float o4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w)
-      osum = fmaf(s_wt[g][w], wpart[((size_t)w * G + g) * (D + 2) + col], osum);
-    // push to the owner of this column: recv[rank][g][col % cols], plus (m, l)
-    const int owner = col / cols;
-    float* slot = recv + ((size_t)rank * G + g) * (cols + 2);
-    st_dsmem_f32(dsmem_addr(&slot[col % cols], owner), osum);
-    if (col % cols == 0) {
-      st_dsmem_f32(dsmem_addr(&slot[cols], owner), M);
-      st_dsmem_f32(dsmem_addr(&slot[cols + 1], owner), s_l[g]);
+    for (int w = 0; w < kWarps; ++w) {
+      const float sw = s_wt[g][w];
+      const float* wp = wpart + ((size_t)w * G + g) * (D + 2) + col;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o4[i] = fmaf(sw, wp[i], o4[i]);
+    }
+    const int owner = col / cols, cc = col % cols;
+    st_dsmem_v4(dsmem_addr(recv + ((size_t)rank * G + g) * cols + cc, owner),
+                make_uint4(__float_as_uint(o4[0]), __float_as_uint(o4[1]),
+                           __float_as_uint(o4[2]), __float_as_uint(o4[3])));
+    if (cc == 0) {
+      st_dsmem_f32(dsmem_addr(&recv_ml[((size_t)rank * G + g) * 2], owner), s_m[g]);
+      st_dsmem_f32(dsmem_addr(&recv_ml[((size_t)rank * G + g) * 2 + 1], owner), s_l[g]);
     }
   }
   cluster_sync();
@@ -1454,12 +1461,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     if (t0 + (tid & ~31) < G * CL) {  // warps holding any (head, partial) pair
       const bool in = t < G * CL;
       const int g = in ? t / CL : 0, r = in ? t % CL : 0;
-      const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
-      const float mr = in ? slot[cols] : -INFINITY;
+      const float* ml = recv_ml + ((size_t)r * G + g) * 2;
+      const float mr = in ? ml[0] : -INFINITY;
       float M = mr;
       for (int o = 1; o < CL; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       const float w = mr == -INFINITY ? 0.f : exp2f(mr - M);
-      float l = in ? w * slot[cols + 1] : 0.f;
+      float l = in ? w * ml[1] : 0.f;
       for (int o = 1; o < CL; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
       if (in) {
         s_fw[g][r] = w;
@@ -1480,7 +1487,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_fused_kernel(
     const float M = s_fm[g], lsum = s_fl[g];
     float osum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int r = 0; r < CL; ++r) {
-      const float* slot = recv + ((size_t)r * G + g) * (cols + 2);
+      const float* slot = recv + ((size_t)r * G + g) * cols;
       const float w = s_fw[g][r];
 #pragma unroll
       for (int v = 0; v < 8; ++v)
