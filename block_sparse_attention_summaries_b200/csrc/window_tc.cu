@@ -13,8 +13,8 @@
 // The grid is persistent (two CTAs per SM at d = 64: 256 TMEM columns and ~105 KB of shared
 // memory each), every CTA walking tiles blockIdx.x, blockIdx.x + gridDim.x, ...; its producers
 // run ahead across tile boundaries (two Q buffers, rings of K and V blocks), the MMA thread issues
-// S one step ahead of the softmax (two S buffers in TMEM), and the next tile's first P V waits only
-// until the epilogue has read the previous tile's O.
+// S two steps ahead of the softmax (three S buffers in TMEM), and the next tile's first P V waits
+// only until the epilogue has read the previous tile's O.
 //   warps 0-3: softmax (row = 32 warp + lane), epilogue O / l -> o (bf16)
 //   warp 4:    Q and K producer (TMA, 128-byte swizzle)      warp 6: V producer
 //   warp 5:    MMA issuer (one thread)
@@ -55,7 +55,10 @@ struct WinSmem {
   static constexpr int kP = kV + kVSlots * kBlkBytes;  // two P buffers
   static constexpr int kTotal = kP + 2 * kPBytes;
   static constexpr int kPerSM = D == 64 ? 2 : 1;
-  static constexpr uint32_t kTmemCols = 256;     // S: 2 x 64 columns, O: D columns at 128
+  static constexpr int kSBufs = 3;                          // S buffers in TMEM, 64 columns each
+  static constexpr uint32_t kOCol = kSBufs * kWB;           // O: D columns after them
+  static constexpr uint32_t kTmemCols = kOCol + D <= 256 ? 256 : 512;
+  static_assert(kPerSM * kTmemCols <= 512, "the CTAs of an SM share its 512 TMEM columns");
 };
 
 struct WinParams {
@@ -98,19 +101,19 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
   using L = WinSmem<D>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = smem_align1024(smem_raw);
-  __shared__ __align__(8) uint64_t bars[24];
+  __shared__ __align__(8) uint64_t bars[26];
   uint64_t* q_full = bars + 0;    // [2]
   uint64_t* q_empty = bars + 2;   // [2]
   uint64_t* k_full = bars + 4;    // [3]
   uint64_t* k_empty = bars + 7;   // [3]
   uint64_t* v_full = bars + 10;   // [2]
   uint64_t* v_empty = bars + 12;  // [2]
-  uint64_t* s_full = bars + 14;   // [2]
-  uint64_t* s_free = bars + 16;   // [2]
-  uint64_t* p_full = bars + 18;   // [2]
-  uint64_t* o_done = bars + 20;   // [2] P_g V_g done (per P buffer)
-  uint64_t* o_free = bars + 22;   // the epilogue has read O
-  uint64_t* fin = bars + 23;
+  uint64_t* s_full = bars + 14;   // [3]
+  uint64_t* s_free = bars + 17;   // [3]
+  uint64_t* p_full = bars + 20;   // [2]
+  uint64_t* o_done = bars + 22;   // [2] P_g V_g done (per P buffer)
+  uint64_t* o_free = bars + 24;   // the epilogue has read O
+  uint64_t* fin = bars + 25;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -121,14 +124,16 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
       mbar_init(&q_empty[i], 1);
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&o_done[i], 1);
     }
     for (int i = 0; i < L::kKSlots; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < L::kSBufs; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
     }
     mbar_init(o_free, 128);
     mbar_init(fin, 1);
@@ -198,9 +203,9 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
     if (lane == 0) {
       constexpr uint32_t idS = tc::idesc_bf16(kWT, kWB, false, false);
       constexpr uint32_t idO = tc::idesc_bf16(kWT, D, false, true);
-      // S_g = Q K_g^T into S buffer g & 1
+      // S_g = Q K_g^T into S buffer g % 3
       auto issue_s = [&](int g, int qb) {
-        const uint32_t d_s = tmem + (uint32_t)((g & 1) * kWB);
+        const uint32_t d_s = tmem + (uint32_t)((g % L::kSBufs) * kWB);
         const unsigned char* kb = kblk(g % L::kKSlots);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -209,11 +214,11 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
           const uint64_t b = tc::smem_desc_sw128(kb + hf * (kWB * 128) + off, 16, 1024);
           tc::mma_f16_ss(d_s, a, b, idS, kk > 0);
         }
-        tc::mma_commit(&s_full[g & 1]);
+        tc::mma_commit(&s_full[g % L::kSBufs]);
         tc::mma_commit(&k_empty[g % L::kKSlots]);
       };
       bool ok = true;
-      // the S cursor runs one step ahead of the P V cursor
+      // the S cursor runs two steps ahead of the P V cursor
       WinCursor cs, cp;
       cs.start(w);
       cp.start(w);
@@ -222,7 +227,9 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
         const int qb = ts & 1;
         if (cs.s == 0 && !mbar_wait_bounded(&q_full[qb], (ts >> 1) & 1)) return false;
         if (!mbar_wait_bounded(&k_full[gs % L::kKSlots], (gs / L::kKSlots) & 1)) return false;
-        if (gs >= 2 && !mbar_wait_bounded(&s_free[gs & 1], ((gs >> 1) - 1) & 1)) return false;
+        if (gs >= L::kSBufs &&
+            !mbar_wait_bounded(&s_free[gs % L::kSBufs], ((gs / L::kSBufs) - 1) & 1))
+          return false;
         tc::fence_after_sync();
         issue_s(gs, qb);
         const bool tile_end = cs.s + 1 == cs.nst;
@@ -232,7 +239,7 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
         if (tile_end) ++ts;
         return true;
       };
-      if (cs.valid(w)) ok = s_step();
+      for (int a = 0; a < L::kSBufs - 1 && ok && cs.valid(w); ++a) ok = s_step();
       int g = 0, tp = 0;  // P V cursor
       while (ok && cp.valid(w)) {
         if (cs.valid(w)) {
@@ -245,7 +252,7 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
         if (ok && cp.s == 0 && tp > 0) ok = mbar_wait_bounded(o_free, (tp - 1) & 1);
         if (!ok) break;
         tc::fence_after_sync();
-        const uint32_t d_o = tmem + 128u;
+        const uint32_t d_o = tmem + L::kOCol;
         const unsigned char* vt = vblk(g % L::kVSlots);
 #pragma unroll
         for (int kk = 0; kk < kWB / 16; ++kk) {  // 64 keys in steps of 16
@@ -277,17 +284,18 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
     while (ok && c.valid(w)) {
       const int i = kWT * c.p + r;  // query position
       const int b = c.first + c.s;  // key block
-      const int st = g & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[st], (g >> 1) & 1));
+      const int st = g & 1;              // P buffer
+      const int sb = g % L::kSBufs;      // S buffer
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&s_full[sb], (g / L::kSBufs) & 1));
       if (!ok) break;
       tc::fence_after_sync();
       float x[64];
-      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * kWB), x);
-      tc::tmem_ld32(tmem + lane_base + (uint32_t)(st * kWB + 32), x + 32);
+      tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kWB), x);
+      tc::tmem_ld32(tmem + lane_base + (uint32_t)(sb * kWB + 32), x + 32);
       tc::tmem_wait_ld();
       tc::reg_fence(x);
       tc::fence_before_sync();
-      mbar_arrive(&s_free[st]);
+      mbar_arrive(&s_free[sb]);
       // keys of block b the row sees: j in [i - window + 1, i]; the masked form runs for the
       // whole warp when any of its rows needs it (most blocks of a tile need none)
       const int lo = i - w.window + 1 - kWB * b, hi = i - kWB * b;  // column bounds
@@ -341,11 +349,11 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           float ov[32];
-          tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+          tc::tmem_ld32(tmem + lane_base + L::kOCol + (uint32_t)c0, ov);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] *= corr;
-          tc::tmem_st32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+          tc::tmem_st32(tmem + lane_base + L::kOCol + (uint32_t)c0, ov);
         }
         tc::tmem_wait_st();
       }
@@ -371,7 +379,7 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           float ov[32];
-          tc::tmem_ld32(tmem + lane_base + 128u + (uint32_t)c0, ov);
+          tc::tmem_ld32(tmem + lane_base + L::kOCol + (uint32_t)c0, ov);
           tc::tmem_wait_ld();
           if (live) {
 #pragma unroll
