@@ -354,17 +354,27 @@ __global__ void __launch_bounds__(kSasThreads, 1)
       if (rescale || m_run == -INFINITY) m_run = m_new;
       // masked keys give 2^-inf = 0; a row with nothing seen yet subtracts 0
       const float off = bias - (m_run == -INFINITY ? 0.f : m_run);
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // two keys per packed FMA (exponent argument), packed multiply (gate) and packed add (four
+      // pairs of partial row sums)
+      const uint64_t sc2 = tc::pack_f2(qk_scale, qk_scale), off2 = tc::pack_f2(off, off);
+      const uint64_t vs2 = tc::pack_f2(vs, vs);
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float p0 = tc::ex2_approx(fmaf(x[c], qk_scale, off));
-        const float p1 = tc::ex2_approx(fmaf(x[c + 1], qk_scale, off));
-        sum4[(c >> 1) & 3] += p0 + p1;
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0 * vs, p1 * vs);
+        float a0, a1;
+        tc::unpack_f2(tc::fma_f2(tc::pack_f2(x[c], x[c + 1]), sc2, off2), a0, a1);
+        const uint64_t p2 = tc::pack_f2(tc::ex2_approx(a0), tc::ex2_approx(a1));
+        sum2[(c >> 1) & 3] = tc::add_f2(sum2[(c >> 1) & 3], p2);
+        float g0, g1;
+        tc::unpack_f2(tc::mul_f2(p2, vs2), g0, g1);
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(g0, g1);
         pk[c / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      l_run = l_run * corr + (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      float sl[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tc::unpack_f2(sum2[e], sl[2 * e], sl[2 * e + 1]);
+      l_run = l_run * corr + (((sl[0] + sl[1]) + (sl[2] + sl[3])) + ((sl[4] + sl[5]) + (sl[6] + sl[7])));
       // this warpgroup's previous P V (step j - 2) has completed before its accumulator is
       // rescaled and its P buffer rewritten
       if (k > 0) {

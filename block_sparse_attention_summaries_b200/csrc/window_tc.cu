@@ -323,17 +323,25 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
       if (rescale) corr = tc::ex2_approx(m_run - m_new);
       if (rescale || m_run == -INFINITY) m_run = m_new;
       const float neg_m = m_run == -INFINITY ? 0.f : -m_run;  // masked keys give 2^-inf = 0
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      // two keys per packed FMA (exponent argument) and per packed add (four pairs of partial
+      // row sums)
+      const uint64_t sc2 = tc::pack_f2(qk_scale, qk_scale), nm2 = tc::pack_f2(neg_m, neg_m);
+      uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[32];
 #pragma unroll
       for (int col = 0; col < kWB; col += 2) {
-        const float p0 = tc::ex2_approx(fmaf(x[col], qk_scale, neg_m));
-        const float p1 = tc::ex2_approx(fmaf(x[col + 1], qk_scale, neg_m));
-        sum4[(col >> 1) & 3] += p0 + p1;
+        float a0, a1;
+        tc::unpack_f2(tc::fma_f2(tc::pack_f2(x[col], x[col + 1]), sc2, nm2), a0, a1);
+        const float p0 = tc::ex2_approx(a0);
+        const float p1 = tc::ex2_approx(a1);
+        sum2[(col >> 1) & 3] = tc::add_f2(sum2[(col >> 1) & 3], tc::pack_f2(p0, p1));
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[col / 2] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      l_run = l_run * corr + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      float sl[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tc::unpack_f2(sum2[e], sl[2 * e], sl[2 * e + 1]);
+      l_run = l_run * corr + (((sl[0] + sl[1]) + (sl[2] + sl[3])) + ((sl[4] + sl[5]) + (sl[6] + sl[7])));
       // O may be rescaled only after P_{g-1} V_{g-1} (same tile) completed; P buffer st may be
       // rewritten once P_{g-2} V_{g-2} completed (implied by the former)
       const bool any_rescale = c.s > 0 && __any_sync(0xffffffffu, rescale);
