@@ -694,7 +694,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         // this row's 64 columns of Z and DV: unit it's block (the loads are warp-wide, so each
         // lane keeps its own unit's half); 32 columns at a time
         const bool use = live && j < s_cnt[it];
-        float t4[4] = {0.f, 0.f, 0.f, 0.f};
+        // two columns per packed FMA (exponent argument), packed add (dv - D_i) and packed FMA
+        // (two pairs of partial sums)
+        const uint64_t zs2 = tc::pack_f2(zs, zs), nl2 = tc::pack_f2(-lse2, -lse2);
+        const uint64_t nd2 = tc::pack_f2(-Di, -Di);
+        uint64_t t2[2] = {0ull, 0ull};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float za[32], zb[32], da[32], db[32];
@@ -710,15 +714,21 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tc::reg_fence(db);
           if (use) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const float z = it ? zb[c] : za[c];
-              const float dv = it ? db[c] : da[c];
-              t4[c & 3] = fmaf(tc::ex2_approx(fmaf(z, zs, -lse2)), dv - Di, t4[c & 3]);
+            for (int c = 0; c < 32; c += 2) {
+              const uint64_t z2 = tc::pack_f2(it ? zb[c] : za[c], it ? zb[c + 1] : za[c + 1]);
+              const uint64_t d2 = tc::pack_f2(it ? db[c] : da[c], it ? db[c + 1] : da[c + 1]);
+              float a0, a1;
+              tc::unpack_f2(tc::fma_f2(z2, zs2, nl2), a0, a1);
+              const uint64_t e2 = tc::pack_f2(tc::ex2_approx(a0), tc::ex2_approx(a1));
+              t2[(c >> 1) & 1] = tc::fma_f2(e2, tc::add_f2(d2, nd2), t2[(c >> 1) & 1]);
             }
           }
         }
         tc::fence_before_sync();
         mbar_arrive(&s_free[st]);
+        float t4[4];
+        tc::unpack_f2(t2[0], t4[0], t4[1]);
+        tc::unpack_f2(t2[1], t4[2], t4[3]);
         float t = (t4[0] + t4[1]) + (t4[2] + t4[3]);
         // sum over the 16 rows of this unit held by this warp, then across warps
 #pragma unroll
