@@ -300,8 +300,14 @@ __global__ void __launch_bounds__(kWThreads, WinSmem<D>::kPerSM)
       // whole warp when any of its rows needs it (most blocks of a tile need none)
       const int lo = i - w.window + 1 - kWB * b, hi = i - kWB * b;  // column bounds
       if (!__all_sync(0xffffffffu, lo <= 0 && hi >= kWB - 1)) {
+        // the kept columns [max(lo, 0), min(hi, 63)] as two 32-bit masks: one bit test per column
+        const int ca = max(lo, 0), cz = min(hi, kWB - 1);
+        uint64_t keep = 0ull;
+        if (ca <= cz) keep = (cz >= 63 ? ~0ull : ((2ull << cz) - 1ull)) & ~((1ull << ca) - 1ull);
+        const uint32_t k0 = (uint32_t)keep, k1 = (uint32_t)(keep >> 32);
 #pragma unroll
-        for (int col = 0; col < kWB; ++col) x[col] = (col >= lo && col <= hi) ? x[col] : -INFINITY;
+        for (int col = 0; col < kWB; ++col)
+          x[col] = ((col < 32 ? k0 : k1) & (1u << (col & 31))) ? x[col] : -INFINITY;
       }
       // row maximum of the raw scores (three-input maxima), then in log2 units: the scale is
       // positive, so the maximum commutes with it and each key needs one FMA before its exp2
