@@ -81,6 +81,18 @@ def test_freesolo_small(window, sigma, d, q_block, K):
     check_rows(case, idx, cnt, o, rows)
 
 
+@pytest.mark.parametrize("window,d", [(1, 64), (63, 64), (65, 64), (2000, 64), (1, 128),
+                                      (65, 128)])
+def test_freesolo_window_edges_every_row(window, d):
+    """Every row of a ragged case (400 queries: three 128-query tiles and a tail of 16) at the
+    window branch's mask edges: the query alone (w = 1), one key less and one more than a 64-key
+    block (63, 65), and a window longer than the sequence (no window mask at all)."""
+    case = inputs.freesolo_case(49, B=1, H=2, d=d, n=400, cell=32, q_block=128, K=4,
+                                window=window, sigma=500.0)
+    idx, cnt, o = run_gpu(case)
+    check_rows(case, idx, cnt, o, [(0, h, i) for h in range(2) for i in range(case.n)])
+
+
 @pytest.mark.parametrize("cell", [4, 64])
 def test_freesolo_cell_sizes(cell):
     """Cells of 4 keys (per-key masks in the tensor-core long branch) and of 64 (a cell fills a
