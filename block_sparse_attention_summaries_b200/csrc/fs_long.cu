@@ -111,6 +111,47 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The same positions with the atomics aggregated over a block of 256 queries of one (batch,
+// head) (n a multiple of 256): each pair first takes a place among the block's pairs of its cell
+// (shared-memory counters, one per cell of the head), then every cell the block touched reserves
+// that many places in the cell's list with one global atomic.
+__global__ void __launch_bounds__(256)
+    fs_long_count_block_kernel(const int* __restrict__ idx, const int* __restrict__ count, int n,
+                               int K, int cell, int C, int* __restrict__ ccount,
+                               int* __restrict__ slotpos) {
+  extern __shared__ int s_cnt[];  // [C] pairs of each cell in this block, then their base
+  const long long row = (long long)blockIdx.x * 256 + threadIdx.x;  // rows = B H n, n % 256 == 0
+  const int i = (int)(row % n);
+  const long long bh = ((long long)blockIdx.x * 256) / n;  // one (batch, head) per block
+  for (int c = threadIdx.x; c < C; c += 256) s_cnt[c] = 0;
+  __syncthreads();
+  const int cnt = count ? min(max(count[row], 0), K) : K;
+  int cells[kMaxKL], local[kMaxKL];
+#pragma unroll
+  for (int k = 0; k < kMaxKL; ++k) {
+    cells[k] = -1;
+    local[k] = 0;
+    if (k >= K) continue;
+    const int c = k < cnt ? idx[row * K + k] : -1;
+    bool ok = c >= 0 && c < C && (long long)(c + 1) * cell <= (long long)i + 1;
+#pragma unroll
+    for (int e = 0; e < k; ++e) ok = ok && cells[e] != c;
+    if (ok) {
+      cells[k] = c;
+      local[k] = atomicAdd(&s_cnt[c], 1);
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < C; c += 256) {
+    const int m = s_cnt[c];
+    s_cnt[c] = m > 0 ? atomicAdd(&ccount[bh * C + c], m) : 0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kMaxKL; ++k)
+    if (k < K) slotpos[row * K + k] = cells[k] >= 0 ? s_cnt[cells[k]] + local[k] : -1;
+}
+
 // ---- 2. cell offsets and the tile list ----------------------------------------------------
 __global__ void __launch_bounds__(256)
     fs_long_offsets_kernel(const int* __restrict__ ccount, long long cells,
@@ -615,9 +656,14 @@ bsa_status long_cells(const void* q, const void* k, const void* v, int B, int H,
   if (cudaMemsetAsync(w.ccount, 0, (size_t)cells * 4, st) != cudaSuccess ||
       cudaMemsetAsync(w.ntiles, 0, 16, st) != cudaSuccess)
     return BSA_ERR_CUDA;
-  fs_long_count_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(idx, count, H, n, K, cell,
-                                                                        C, rows, w.ccount,
-                                                                        w.slotpos);
+  if (n % 256 == 0 && C <= 12288) {  // a block is 256 queries of one head; C counters fit 48 KB
+    fs_long_count_block_kernel<<<(unsigned)(rows / 256), 256, (size_t)C * 4, st>>>(
+        idx, count, n, K, cell, C, w.ccount, w.slotpos);
+  } else {
+    fs_long_count_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(idx, count, H, n, K, cell,
+                                                                          C, rows, w.ccount,
+                                                                          w.slotpos);
+  }
   BSA_LAUNCH_CHECK();
   fs_long_offsets_kernel<<<(unsigned)((cells + 255) / 256), 256, 0, st>>>(
       w.ccount, cells, w.cell_off, w.tiles, w.tile_cap, w.ntiles);

@@ -93,6 +93,17 @@ def test_freesolo_window_edges_every_row(window, d):
     check_rows(case, idx, cnt, o, [(0, h, i) for h in range(2) for i in range(case.n)])
 
 
+@pytest.mark.parametrize("cell,q_block", [(32, 128), (16, 64)])
+def test_freesolo_block_count_every_row(cell, q_block):
+    """n a multiple of 256, so the long branch places its pairs with the block-aggregated counts
+    (shared-memory counters per cell, one global reservation per cell and block): every row of
+    two heads."""
+    case = inputs.freesolo_case(50, B=1, H=2, d=64, n=1024, cell=cell, q_block=q_block, K=4,
+                                window=300, sigma=800.0)
+    idx, cnt, o = run_gpu(case)
+    check_rows(case, idx, cnt, o, [(0, h, i) for h in range(2) for i in range(case.n)])
+
+
 @pytest.mark.parametrize("cell", [4, 64])
 def test_freesolo_cell_sizes(cell):
     """Cells of 4 keys (per-key masks in the tensor-core long branch) and of 64 (a cell fills a
