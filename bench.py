@@ -62,6 +62,15 @@ MEASURED_TRAFFIC = {
         "source": "block_sparse_attention_summaries_b200/csrc/decode_fused.cu",
         "device_end": "int pick_cluster(", "sha256_16": "18c12307660d9922",
         "bytes": 33_624_064 + 16_127_232},
+    # one launch each, full captures of the gated prefill forward and the gate gradient
+    ("sas_gated_prefill_16k", "sas_fwd_tc_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/sas_fwd_tc.cu",
+        "device_end": "bsa_status launch_sas(", "sha256_16": "6cb98727de799ac2",
+        "bytes": 412_782_336 + 240_278_016},
+    ("sas_gated_prefill_16k", "gate_grad_tc_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/prefill_tc.cu",
+        "device_end": "bsa_status launch_tc(", "sha256_16": "09671dc7350d5094",
+        "bytes": 940_605_952 + 4_610_304},
 }
 
 
@@ -399,12 +408,16 @@ def run_prefill(dev, peaks, reps=5, rows=("sas", "freesolo", "fsl")):
             "forward": {"kernel": "sas_fwd_tc_kernel (tcgen05, two softmax warpgroups)", "ms": t_fwd,
                         "gathered_gflop": fwd_flops / 1e9, "tflops": fwd_flops / t_fwd / 1e9,
                         "roofline": roofline("tensor", "sas_fwd_tc_kernel", fwd_flops / t_fwd / 1e9,
-                                             peak, "TFLOP/s", peak_source=src)},
+                                             peak, "TFLOP/s", peak_source=src,
+                                             traffic=measured_traffic("sas_gated_prefill_16k",
+                                                                      "sas_fwd_tc_kernel"))},
             "gate_grad": {"kernel": "gate_grad_tc_kernel (tcgen05)", "ms": t_grad,
                           "gathered_gflop": grad_flops / 1e9, "tflops": grad_flops / t_grad / 1e9,
                           "roofline": roofline("tensor", "gate_grad_tc_kernel",
                                                grad_flops / t_grad / 1e9, peak, "TFLOP/s",
-                                               peak_source=src)},
+                                               peak_source=src,
+                                               traffic=measured_traffic("sas_gated_prefill_16k",
+                                                                        "gate_grad_tc_kernel"))},
             "selector_grad": {"kernel": "selector_grad_kernel", "ms": t_sgrad,
                               "bytes": sgrad_bytes, "gbs": sgrad_bytes / t_sgrad / 1e6,
                               "roofline": roofline("hbm", "selector_grad_kernel",
