@@ -71,6 +71,10 @@ MEASURED_TRAFFIC = {
         "source": "block_sparse_attention_summaries_b200/csrc/prefill_tc.cu",
         "device_end": "bsa_status launch_tc(", "sha256_16": "09671dc7350d5094",
         "bytes": 940_605_952 + 4_610_304},
+    ("freesolo_prefill_64k", "freesolo_select_tc_kernel"): {
+        "source": "block_sparse_attention_summaries_b200/csrc/freesolo_tc.cu",
+        "device_end": "size_t freesolo_select_tc_workspace(", "sha256_16": "79ef22b094ee8af3",
+        "bytes": 142_674_432 + 14_409_472},
 }
 
 
@@ -465,7 +469,9 @@ def run_prefill(dev, peaks, reps=5, rows=("sas", "freesolo", "fsl")):
                        "score_gflop": score_flops / 1e9, "tflops": score_flops / t_sel / 1e9,
                        "roofline": roofline("tensor", "freesolo_select_tc_kernel",
                                             score_flops / t_sel / 1e9, peak, "TFLOP/s",
-                                            peak_source=src)},
+                                            peak_source=src,
+                                            traffic=measured_traffic("freesolo_prefill_64k",
+                                                                     "freesolo_select_tc_kernel"))},
             "attention": {"kernel": "rope (q, k) + window_tc_kernel (persistent 128-query tiles) + "
                                     "cell-major long branch (fs_long_* kernels, tcgen05 tiles) + "
                                     "combine", "ms": t_att,
