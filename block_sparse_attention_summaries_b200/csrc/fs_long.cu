@@ -6,8 +6,10 @@
 //
 // Every query picks only K cells of `cell` tokens, but queries that pick the same cell share its
 // keys.  So the work is regrouped by cell instead of by query:
-//   1. fs_long_count_kernel: each valid (query, slot) pair takes a position in its cell's list
-//      (warp-aggregated atomics: neighbouring queries tend to pick the same cells);
+//   1. fs_long_count_block_kernel (n a multiple of 256) or fs_long_count_kernel: each valid
+//      (query, slot) pair takes a position in its cell's list (shared-memory counters per
+//      block of 256 queries and one global atomic per cell and block, or warp-aggregated
+//      atomics: neighbouring queries tend to pick the same cells);
 //   2. fs_long_offsets_kernel: each cell reserves a contiguous range of the pair list and one
 //      tile per 128 of its pairs (a warp scan, then one atomic per warp on the two totals: the
 //      order of the cells in the lists does not matter);
