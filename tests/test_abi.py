@@ -265,3 +265,20 @@ def test_recorded_traffic_matches_the_kernel_source():
     import bench
     for (workload, kernel), rec in bench.MEASURED_TRAFFIC.items():
         assert bench.measured_traffic(workload, kernel) == rec["bytes"], (workload, kernel)
+
+
+def test_recorded_traffic_is_dropped_when_the_device_code_changes(tmp_path, monkeypatch):
+    """A record whose source no longer hashes to the captured value reports no traffic (null in
+    the bench line), and only the text before the host-code marker counts."""
+    import bench
+    src = tmp_path / "kernel.cu"
+    src.write_text("__global__ void k() {}\nint host_marker() { return 1; }\n")
+    h = bench.device_source_hash(str(src), "int host_marker(")
+    rec = {"source": str(src), "device_end": "int host_marker(", "sha256_16": h, "bytes": 123}
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, ("w", "k"), rec)
+    assert bench.measured_traffic("w", "k") == 123
+    src.write_text("__global__ void k() {}\nint host_marker() { return 2; }\n")  # host edit
+    assert bench.measured_traffic("w", "k") == 123
+    src.write_text("__global__ void k() { int x = 0; }\nint host_marker() { return 2; }\n")
+    assert bench.measured_traffic("w", "k") is None
+    assert bench.measured_traffic("w", "other") is None
